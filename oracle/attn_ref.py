@@ -1,0 +1,136 @@
+"""Float64 CPU oracle for bf16 causal multi-head self-attention, forward and backward.
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may
+import this module. It shares no code with the CUDA path and never calls it.
+
+What it computes. The pages call the attention as ``flash_attn_func(q, k, v, causal=True, window_size=...)`` on
+[B, T, H, D] tensors (apidog "Train your own ChatGPT", section 5 "Flash Attention integration", and section 1
+"GPT model" for the [B, T, n_head, head_dim] view); the model trains through it, so a backward exists. The pages
+print neither the formula nor the backward, so this file writes out the textbook definition of scaled
+dot-product attention under a causal mask, the one the pages' SDPA fallback computes (same section 5):
+
+  per (b, h), with s the softmax scale and i, j query/key positions,
+    S[i, j]  = s * sum_d Q[i, d] K[j, d]     for j <= i,   -inf for j > i   (top-left aligned, T_q = T_k)
+    m_i      = max_j S[i, j],   l_i = sum_j exp(S[i, j] - m_i)
+    P[i, j]  = exp(S[i, j] - m_i) / l_i
+    O        = P V
+    LSE_i    = m_i + ln l_i                     (natural log of the scaled, masked logits)
+  and, for an upstream gradient dO of a loss L = sum(dO * O):
+    dV       = P^T dO
+    dP       = dO V^T
+    Delta_i  = sum_d dO[i, d] O[i, d]          (= sum_j P[i, j] dP[i, j])
+    dS       = P * (dP - Delta)                 (zero where masked, because P is)
+    dQ       = s dS K,      dK = s dS^T Q
+
+Everything is dense over the full T x T matrix of each (b, h) and masked afterwards: no blocking, no online
+softmax, no reordering. A blockwise online-softmax kernel reaches the same values in exact arithmetic.
+
+Readings where the pages are silent: scale = 1/sqrt(D) passed explicitly; mask aligned top-left; LSE in
+natural log over the scaled logits; inputs are bf16 values upcast exactly to float64 with no intermediate
+rounding here (the GPU rounds P and dS to bf16 before its matrix products; the parity tolerances absorb that).
+
+Pins (tests/test_oracle.py): softmax rows sum to one; causality under perturbation of later positions; T = 1;
+Q = 0 closed form (prefix mean, LSE = ln(t + 1)); equal keys; shift invariance of the keys; agreement with
+torch's float64 ``scaled_dot_product_attention`` and its autograd; central finite differences; the Delta
+identity; a hand-derived worked example under tests/golden/.
+"""
+from __future__ import annotations
+
+from typing import Tuple
+
+import numpy as np
+
+
+def _as_f64(x) -> np.ndarray:
+    """Upcast an array-like (numpy, or a CPU torch tensor of any float dtype) to float64 numpy, exactly."""
+    if hasattr(x, "detach"):
+        import torch  # local: the oracle itself is numpy; torch only as an input container
+        x = x.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def causal_mask(T: int) -> np.ndarray:
+    """Boolean [T, T] matrix, True where key j may be seen by query i (j <= i)."""
+    return np.tril(np.ones((T, T), dtype=bool))
+
+
+def head_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
+    """Forward of one (b, h) slice: q, k, v are [T, D] float64. Returns (O [T, D], LSE [T], P [T, T])."""
+    T = q.shape[0]
+    S = scale * (q @ k.T)
+    S = np.where(causal_mask(T), S, -np.inf)
+    m = S.max(axis=1, keepdims=True)           # finite: the diagonal is always visible
+    E = np.exp(S - m)                          # exp(-inf) = 0 on masked entries
+    l = E.sum(axis=1, keepdims=True)
+    P = E / l
+    O = P @ v
+    lse = (m + np.log(l))[:, 0]
+    return O, lse, P
+
+
+def head_backward(q, k, v, do, scale: float, o=None):
+    """Backward of one (b, h) slice from the definition. Returns (dQ, dK, dV, Delta).
+
+    ``o`` is the forward output used for Delta; by default the exact float64 output of ``head_forward``.
+    """
+    O, _, P = head_forward(q, k, v, scale)
+    if o is None:
+        o = O
+    dV = P.T @ do
+    dP = do @ v.T
+    delta = (do * o).sum(axis=1)
+    dS = P * (dP - delta[:, None])
+    dQ = scale * (dS @ k)
+    dK = scale * (dS.T @ q)
+    return dQ, dK, dV, delta
+
+
+def attention_forward(q, k, v, scale: float) -> Tuple[np.ndarray, np.ndarray]:
+    """Full forward over [B, T, H, D] inputs. Returns O [B, T, H, D] and LSE [B, H, T], both float64."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, T, H, D = q.shape
+    O = np.empty((B, T, H, D))
+    LSE = np.empty((B, H, T))
+    for b in range(B):
+        for h in range(H):
+            o_bh, lse_bh, _ = head_forward(q[b, :, h], k[b, :, h], v[b, :, h], scale)
+            O[b, :, h] = o_bh
+            LSE[b, h] = lse_bh
+    return O, LSE
+
+
+def attention_backward(q, k, v, do, scale: float, o=None):
+    """Full backward over [B, T, H, D] inputs. Returns dQ, dK, dV [B, T, H, D] and Delta [B, H, T]."""
+    q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
+    o = None if o is None else _as_f64(o)
+    B, T, H, D = q.shape
+    dQ, dK, dV = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    delta = np.empty((B, H, T))
+    for b in range(B):
+        for h in range(H):
+            o_bh = None if o is None else o[b, :, h]
+            gq, gk, gv, dl = head_backward(q[b, :, h], k[b, :, h], v[b, :, h], do[b, :, h], scale, o_bh)
+            dQ[b, :, h], dK[b, :, h], dV[b, :, h] = gq, gk, gv
+            delta[b, h] = dl
+    return dQ, dK, dV, delta
+
+
+def slice_forward_backward(q, k, v, do, b: int, h: int, scale: float):
+    """Forward and backward of the single (b, h) slice of [B, T, H, D] inputs (slices are independent).
+
+    Returns a dict of float64 arrays: o [T, D], lse [T], dq, dk, dv [T, D], delta [T].
+    """
+    qs, ks, vs = _as_f64(q[b, :, h]), _as_f64(k[b, :, h]), _as_f64(v[b, :, h])
+    o, lse, _ = head_forward(qs, ks, vs, scale)
+    out = {"o": o, "lse": lse}
+    if do is not None:
+        dos = _as_f64(do[b, :, h])
+        dq, dk, dv, delta = head_backward(qs, ks, vs, dos, scale)
+        out.update(dq=dq, dk=dk, dv=dv, delta=delta)
+    return out
+
+
+def causal_flops(B: int, H: int, T: int, D: int) -> Tuple[float, float]:
+    """FLOP convention of the measurement: forward 2*B*H*T^2*D, backward 2.5x that."""
+    f = 2.0 * B * H * T * T * D
+    return f, 2.5 * f

@@ -1,0 +1,282 @@
+"""Pins for the float64 oracle, each tied to something other than the oracle itself.
+
+The pages define the operation only as ``flash_attn_func(q, k, v, causal=True)`` (apidog "Train your own
+ChatGPT", section 5), with a PyTorch SDPA fallback on other hardware (same section). So the oracle is pinned
+by: a hand-derived worked example (tests/golden), closed forms (T = 1, Q = 0, equal keys), invariants
+(softmax rows, causality, key shift), torch's own float64 SDPA and autograd (the fallback the pages name), and
+central finite differences. The last test plants mistakes in a copy of the oracle and checks that these pins
+catch each one.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attn_ref
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_example_T3.txt")
+
+
+def load_golden(path=GOLDEN):
+    cases, cur = {}, None
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            if key == "case":
+                cur = cases.setdefault(vals[0], {})
+            else:
+                cur[key] = np.array([float(x) for x in vals])
+    return cases
+
+
+def rand_qkvdo(T, D, seed, B=1, H=1):
+    rng = np.random.default_rng(seed)
+    return [rng.standard_normal((B, T, H, D)) for _ in range(4)]
+
+
+# ---------------------------------------------------------------------------------------------------------
+# Pin checks, parameterised by the implementation so that the mutation test can reuse them.
+# An implementation is a pair (fwd(q,k,v,s) -> (O, lse, P), bwd(q,k,v,do,s) -> (dq, dk, dv, delta)) per head.
+
+ORACLE = (attn_ref.head_forward, lambda q, k, v, do, s: attn_ref.head_backward(q, k, v, do, s))
+
+
+def check_golden(impl):
+    fwd, bwd = impl
+    for name, c in load_golden().items():
+        T = len(c["lse"])
+        D = len(c["q"]) // T
+        q, k, v, do = (c[n].reshape(T, D) for n in ("q", "k", "v", "do"))
+        s = float(c["scale"][0])
+        O, lse, _ = fwd(q, k, v, s)
+        dq, dk, dv, delta = bwd(q, k, v, do, s)
+        np.testing.assert_allclose(O, c["o"].reshape(T, D), rtol=0, atol=1e-14, err_msg=f"{name}: O")
+        np.testing.assert_allclose(lse, c["lse"], rtol=0, atol=1e-14, err_msg=f"{name}: lse")
+        np.testing.assert_allclose(delta, c["delta"], rtol=0, atol=1e-14, err_msg=f"{name}: delta")
+        np.testing.assert_allclose(dv, c["dv"].reshape(T, D), rtol=0, atol=1e-14, err_msg=f"{name}: dv")
+        np.testing.assert_allclose(dq, c["dq"].reshape(T, D), rtol=0, atol=1e-14, err_msg=f"{name}: dq")
+        np.testing.assert_allclose(dk, c["dk"].reshape(T, D), rtol=0, atol=1e-14, err_msg=f"{name}: dk")
+
+
+def check_softmax_rows(impl, T=37, D=16, seed=0):
+    fwd, _ = impl
+    q, k, v, _ = (x[0, :, 0] for x in rand_qkvdo(T, D, seed))
+    _, _, P = fwd(q, k, v, 1 / math.sqrt(D))
+    assert np.all(P >= 0)
+    assert np.all(P[np.triu_indices(T, 1)] == 0), "weight on a future key"
+    np.testing.assert_allclose(P.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+
+
+def check_causality(impl, T=29, D=8, seed=1):
+    fwd, _ = impl
+    q, k, v, _ = (x[0, :, 0] for x in rand_qkvdo(T, D, seed))
+    s = 1 / math.sqrt(D)
+    O, lse, _ = fwd(q, k, v, s)
+    rng = np.random.default_rng(seed + 100)
+    for t in (0, 5, T - 2):
+        q2, k2, v2 = q.copy(), k.copy(), v.copy()
+        for a in (q2, k2, v2):
+            a[t + 1:] += 10 * rng.standard_normal(a[t + 1:].shape)
+        O2, lse2, _ = fwd(q2, k2, v2, s)
+        np.testing.assert_array_equal(O2[:t + 1], O[:t + 1])
+        np.testing.assert_array_equal(lse2[:t + 1], lse[:t + 1])
+
+
+def check_T1(impl, D=8, seed=2):
+    fwd, bwd = impl
+    q, k, v, do = (x[0, :, 0] for x in rand_qkvdo(1, D, seed))
+    s = 0.37
+    O, lse, _ = fwd(q, k, v, s)
+    np.testing.assert_allclose(O, v, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(lse, [s * float(q[0] @ k[0])], rtol=1e-15, atol=1e-15)
+    dq, dk, dv, _ = bwd(q, k, v, do, s)
+    np.testing.assert_allclose(dv, do, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(dq, 0, atol=1e-15)
+    np.testing.assert_allclose(dk, 0, atol=1e-15)
+
+
+def check_zero_query(impl, T=23, D=8, seed=3):
+    fwd, _ = impl
+    _, k, v, _ = (x[0, :, 0] for x in rand_qkvdo(T, D, seed))
+    q = np.zeros((T, D))
+    O, lse, _ = fwd(q, k, v, 0.5)
+    prefix_mean = np.cumsum(v, axis=0) / np.arange(1, T + 1)[:, None]
+    np.testing.assert_allclose(O, prefix_mean, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(lse, np.log(np.arange(1, T + 1)), rtol=1e-14, atol=1e-14)
+
+
+def check_equal_keys(impl, T=19, D=8, seed=4):
+    fwd, _ = impl
+    q, k, v, _ = (x[0, :, 0] for x in rand_qkvdo(T, D, seed))
+    k = np.repeat(k[:1], T, axis=0)
+    O, _, _ = fwd(q, k, v, 0.3)
+    prefix_mean = np.cumsum(v, axis=0) / np.arange(1, T + 1)[:, None]
+    np.testing.assert_allclose(O, prefix_mean, rtol=1e-13, atol=1e-14)
+
+
+def check_key_shift(impl, T=31, D=8, seed=5):
+    """Adding one vector b to every key shifts logit row i by s q_i . b: P, O unchanged, LSE shifted."""
+    fwd, bwd = impl
+    q, k, v, do = (x[0, :, 0] for x in rand_qkvdo(T, D, seed))
+    b = np.random.default_rng(seed).standard_normal(D)
+    s = 1 / math.sqrt(D)
+    O, lse, _ = fwd(q, k, v, s)
+    O2, lse2, _ = fwd(q, k + b, v, s)
+    np.testing.assert_allclose(O2, O, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse2, lse + s * (q @ b), rtol=1e-12, atol=1e-12)
+    dq, dk, dv, _ = bwd(q, k, v, do, s)
+    dq2, dk2, dv2, _ = bwd(q, k + b, v, do, s)
+    np.testing.assert_allclose(dv2, dv, rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(dk2, dk, rtol=1e-11, atol=1e-11)
+    # dQ picks up s * sum_j dS_ij b = 0, since each row of dS sums to zero.
+    np.testing.assert_allclose(dq2, dq, rtol=1e-11, atol=1e-11)
+
+
+def check_torch_sdpa(impl, T=45, D=16, seed=6):
+    """Agreement with torch's float64 CPU scaled_dot_product_attention and its autograd."""
+    fwd, bwd = impl
+    q, k, v, do = (x[0, :, 0] for x in rand_qkvdo(T, D, seed))
+    s = 1 / math.sqrt(D)
+    tq, tk, tv = (torch.tensor(x[None, None], dtype=torch.float64, requires_grad=True) for x in (q, k, v))
+    to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True, scale=s)
+    (to * torch.tensor(do[None, None])).sum().backward()
+    O, _, _ = fwd(q, k, v, s)
+    dq, dk, dv, _ = bwd(q, k, v, do, s)
+    np.testing.assert_allclose(O, to[0, 0].detach().numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dq, tq.grad[0, 0].numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dk, tk.grad[0, 0].numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dv, tv.grad[0, 0].numpy(), rtol=1e-11, atol=1e-12)
+
+
+def check_finite_differences(impl, T=6, D=5, seed=7, h=1e-6):
+    """Central differences of f = sum(dO * O) against the analytic gradient."""
+    fwd, bwd = impl
+    q, k, v, do = (x[0, :, 0] for x in rand_qkvdo(T, D, seed))
+    s = 0.45
+
+    def f(q_, k_, v_):
+        return float((do * fwd(q_, k_, v_, s)[0]).sum())
+
+    dq, dk, dv, _ = bwd(q, k, v, do, s)
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        num = np.zeros_like(grad)
+        for idx in np.ndindex(grad.shape):
+            args_p = [q.copy(), k.copy(), v.copy()]
+            args_m = [q.copy(), k.copy(), v.copy()]
+            args_p[which][idx] += h
+            args_m[which][idx] -= h
+            num[idx] = (f(*args_p) - f(*args_m)) / (2 * h)
+        rel = np.linalg.norm(num - grad) / max(np.linalg.norm(grad), 1e-30)
+        assert rel < 1e-6, f"finite differences, input {which}: relative error {rel:.3e}"
+
+
+def check_delta_identity(impl, T=33, D=8, seed=8):
+    fwd, bwd = impl
+    q, k, v, do = (x[0, :, 0] for x in rand_qkvdo(T, D, seed))
+    s = 1 / math.sqrt(D)
+    _, _, P = fwd(q, k, v, s)
+    _, _, _, delta = bwd(q, k, v, do, s)
+    dP = do @ v.T
+    np.testing.assert_allclose(delta, (P * dP).sum(axis=1), rtol=1e-12, atol=1e-12)
+
+
+ALL_PINS = [check_golden, check_softmax_rows, check_causality, check_T1, check_zero_query, check_equal_keys,
+            check_key_shift, check_torch_sdpa, check_finite_differences, check_delta_identity]
+
+
+@pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
+def test_oracle_pin(pin):
+    pin(ORACLE)
+
+
+# ---------------------------------------------------------------------------------------------------------
+# The full-tensor entry points agree with the per-head ones and with torch on a batched [B, T, H, D] case.
+
+def test_full_tensor_entry_points_match_torch():
+    B, T, H, D = 2, 40, 3, 16
+    q, k, v, do = rand_qkvdo(T, D, 11, B=B, H=H)
+    s = 1 / math.sqrt(D)
+    O, LSE = attn_ref.attention_forward(q, k, v, s)
+    dQ, dK, dV, delta = attn_ref.attention_backward(q, k, v, do, s)
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64).transpose(1, 2).requires_grad_() for x in (q, k, v))
+    to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True, scale=s)
+    (to * torch.tensor(do).transpose(1, 2)).sum().backward()
+    np.testing.assert_allclose(O, to.transpose(1, 2).detach().numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dQ, tq.grad.transpose(1, 2).numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dK, tk.grad.transpose(1, 2).numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dV, tv.grad.transpose(1, 2).numpy(), rtol=1e-11, atol=1e-12)
+    # LSE against torch.logsumexp of the masked, scaled logits.
+    S = s * torch.einsum("bhid,bhjd->bhij", tq.detach(), tk.detach())
+    S = S.masked_fill(~torch.ones(T, T, dtype=torch.bool).tril(), float("-inf"))
+    np.testing.assert_allclose(LSE, torch.logsumexp(S, dim=-1).numpy(), rtol=1e-13, atol=1e-13)
+    # Slices are independent: the slice entry point returns the same numbers.
+    sl = attn_ref.slice_forward_backward(q, k, v, do, 1, 2, s)
+    np.testing.assert_allclose(sl["o"], O[1, :, 2], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(sl["dk"], dK[1, :, 2], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(sl["delta"], delta[1, 2], rtol=0, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------------------------------------
+# Mutation test: plant plausible mistakes in a copy of the oracle and require that some pin fails.
+
+def _mutant(kind):
+    def fwd(q, k, v, s):
+        T = q.shape[0]
+        S = s * (q @ (k if kind == "no_transpose_qk" else k).T)
+        off = -1 if kind == "mask_excludes_diagonal" else 0
+        mask = np.tril(np.ones((T, T), dtype=bool), k=off)
+        if kind == "mask_excludes_diagonal":
+            mask[0, 0] = True
+        if kind == "no_mask":
+            mask[:] = True
+        S = np.where(mask, S, -np.inf)
+        m = S.max(axis=1, keepdims=True)
+        E = np.exp(S - m)
+        l = E.sum(axis=1, keepdims=True)
+        P = E / l
+        O = (P.T if kind == "transposed_pv" else P) @ v
+        lse = (m + (np.log2(l) if kind == "lse_log2" else np.log(l)))[:, 0]
+        return O, lse, P
+
+    def bwd(q, k, v, do, s):
+        O, _, P = fwd(q, k, v, s)
+        dV = (P @ do) if kind == "dv_not_transposed" else P.T @ do
+        dP = do @ v.T
+        delta = (do * O).sum(axis=1)
+        dS = P * (dP + delta[:, None]) if kind == "delta_sign" else P * (dP - delta[:, None])
+        if kind == "dropped_delta":
+            dS = P * dP
+        dQ = (1.0 if kind == "dq_no_scale" else s) * (dS @ k)
+        dK = (1.0 if kind == "dk_no_scale" else s) * (dS.T @ q)
+        if kind == "dk_uses_k":
+            dK = s * (dS.T @ k)
+        return dQ, dK, dV, delta
+
+    return fwd, bwd
+
+
+MUTANTS = ["mask_excludes_diagonal", "no_mask", "transposed_pv", "lse_log2", "dv_not_transposed", "delta_sign",
+           "dropped_delta", "dq_no_scale", "dk_no_scale", "dk_uses_k"]
+
+
+def test_mutant_control_passes():
+    """The mutant factory without a mutation reproduces the oracle, so a failure below is the planted bug."""
+    for pin in ALL_PINS:
+        pin(_mutant("none"))
+
+
+@pytest.mark.parametrize("kind", MUTANTS)
+def test_pins_catch_planted_mistake(kind):
+    impl = _mutant(kind)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(impl)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the planted mistake {kind!r}"

@@ -1,0 +1,126 @@
+"""Seeded synthetic inputs for causal self-attention, shared by the oracle side and the CUDA side.
+
+This module holds no attention arithmetic: it only names the workloads and draws their inputs. Both the
+float64 oracle (``oracle/``) and the CUDA path (``causal_self_attention_bf16_b200``) receive the same bf16
+tensors from here, so that a parity comparison sees identical bytes.
+
+Shapes follow nanochat's single depth dial: the model width is 64 * depth and every head has 128 dims, so
+depth d gives H = d / 2 heads (apidog "Train your own ChatGPT", section "Philosophy: one dial"; aisight.pl
+nanochat review, "Model and scaling assumptions": d20 = 1280 channels, 10 heads of 128). Rows are full
+2048-token packed sequences (apidog, section 4 "Data loading", best-fit packing to 2048), and the device batch
+is 32, halved to 16 for d24/d26 (ja.news.hada.io summary, "Bigger models"; apidog leaderboard run 6 flags).
+
+Layout of every tensor: [B, T, H, D] contiguous, the layout the pages' model reshapes into before calling
+``flash_attn_func`` (apidog, section 1 "GPT model", the value-embedding ``view(B, T, n_kv_head, head_dim)``).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, Optional
+
+import torch
+
+HEAD_DIM = 128
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One synthetic attention workload: shape, value recipe and seed."""
+
+    name: str
+    B: int
+    H: int
+    T: int
+    D: int = HEAD_DIM
+    seed: int = 0
+    qk_prescale: float = 1.0     # multiply the fp32 draws of q and k by this before the bf16 cast
+    key_bias: bool = False       # add one shared N(0,1) vector of length D to every key row
+    recipe: str = ""
+
+    @property
+    def scale(self) -> float:
+        """Softmax scale 1/sqrt(D) (the usual choice; the pages do not print it)."""
+        return 1.0 / math.sqrt(self.D)
+
+    @property
+    def fwd_flops(self) -> float:
+        """Causal forward FLOPs by the convention 2*B*H*T^2*D (half of the dense 4*B*H*T^2*D)."""
+        return 2.0 * self.B * self.H * self.T * self.T * self.D
+
+    @property
+    def bwd_flops(self) -> float:
+        """Backward FLOPs counted as 2.5x the forward."""
+        return 2.5 * self.fwd_flops
+
+    def with_shape(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+WORKLOADS: Dict[str, Workload] = {
+    "tiny": Workload("tiny", B=1, H=2, T=128,
+                     recipe="q,k,v,dO ~ N(0,1) fp32 from seed 0, cast to bf16"),
+    "d12": Workload("d12", B=32, H=6, T=2048, qk_prescale=0.5,
+                    recipe="q,k,v,dO ~ N(0,1); q,k multiplied by 0.5 before the bf16 cast"),
+    "d20": Workload("d20", B=32, H=10, T=2048,
+                    recipe="q,k,v,dO ~ N(0,1) fp32 from seed 0, cast to bf16"),
+    "d24": Workload("d24", B=16, H=12, T=2048, key_bias=True,
+                    recipe="q,k,v,dO ~ N(0,1); one shared bias b ~ N(0,1)^D added to every key row"),
+    "d26": Workload("d26", B=16, H=13, T=2048,
+                    recipe="q,k,v,dO ~ N(0,1) fp32 from seed 0, cast to bf16"),
+}
+# d26 sequence-length sweep at a fixed B*T = 32768 tokens per device.
+for _T in (512, 1024, 2048, 4096):
+    WORKLOADS[f"d26_T{_T}"] = Workload(f"d26_T{_T}", B=32768 // _T, H=13, T=_T,
+                                       recipe="d26 heads, B*T = 32768 tokens, q,k,v,dO ~ N(0,1)")
+
+HEADLINE = "d20"
+
+
+def make_inputs(w: Workload, device: Optional[torch.device] = None, need_grad_input: bool = True):
+    """Draw (q, k, v, dO) for a workload as bf16 [B, T, H, D] tensors.
+
+    One CPU ``torch.Generator`` seeded with ``w.seed`` draws fp32 standard normals in the order q, k, v, dO and
+    then (d24 only) the key bias. Pre-scaling and the bias are applied in fp32, then each tensor is rounded to
+    bf16 (round to nearest even). The same bytes go to the GPU and, upcast exactly, to the oracle.
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    shape = (w.B, w.T, w.H, w.D)
+    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(shape, generator=g, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    do = torch.randn(shape, generator=g, dtype=torch.float32) if need_grad_input else None
+    if w.qk_prescale != 1.0:
+        q.mul_(w.qk_prescale)
+        k.mul_(w.qk_prescale)
+    if w.key_bias:
+        bias = torch.randn((w.D,), generator=g, dtype=torch.float32)
+        k.add_(bias)
+    out = [t.to(torch.bfloat16) if t is not None else None for t in (q, k, v, do)]
+    if device is not None:
+        out = [t.to(device) if t is not None else None for t in out]
+    return tuple(out)
+
+
+def key_bias_vector(w: Workload) -> torch.Tensor:
+    """The shared key bias of a ``key_bias`` workload (fp32, length D), redrawn from the same stream."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    n = w.B * w.T * w.H * w.D
+    for _ in range(4):
+        torch.randn((n,), generator=g, dtype=torch.float32)
+    return torch.randn((w.D,), generator=g, dtype=torch.float32)
+
+
+def sample_slices(w: Workload, k: int = 4, seed: int = 1234):
+    """Seeded sample of (b, h) slices, always including (0, 0) and (B-1, H-1)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    picks = [(0, 0), (w.B - 1, w.H - 1)]
+    while len(picks) < min(k, w.B * w.H):
+        b = int(torch.randint(0, w.B, (1,), generator=g))
+        h = int(torch.randint(0, w.H, (1,), generator=g))
+        if (b, h) not in picks:
+            picks.append((b, h))
+    return picks
