@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Benchmark of the bf16 causal self-attention hot path (forward + backward) on B200.
+
+One step = one forward (attn_fwd) and one backward (attn_bwd's three stages: preprocess, dK/dV with dQ
+accumulation, dQ conversion) over one batch of the workload, inputs resident in HBM. The metric is causal
+TFLOP/s with the convention fwd = 2*B*H*T^2*D and bwd = 2.5 x fwd, and its fraction of the measured dense
+bf16 tensor peak. Launch:
+
+  python bench.py [--gpus 1] [--steps K] [--warmup W] [--workload d20] [--impl ours|reference]
+  torchrun --nproc-per-node N bench.py --gpus N ...      (replicas: every rank runs its own batch)
+
+Rank 0 prints one JSON line. ``--impl reference`` times the float64 CPU oracle (the only reference this
+path has) on a bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, Workload  # noqa: E402
+
+METRIC = "causal attention fwd+bwd TFLOP/s (bf16, d20 shape) and % of B200 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+KERNEL_SOURCES = ["attn_api.cu", "attn_fwd.cuh", "attn_bwd.cuh", "attn_common.cuh", "sm100.cuh"]
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="d20", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------------------------------------------ helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS)
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "causal_self_attention_bf16_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = d.get(kernel, {}).get(workload)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def flops(w: Workload):
+    f = 2.0 * w.B * w.H * w.T * w.T * w.D
+    return f, 2.5 * f
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max over ranks (identity at world size 1). Works with nccl (device tensor) and gloo (CPU tensor)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(per_rank_units: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return per_rank_units * world / max_seconds
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled in the background during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.count(",") >= 8]
+        self.file.close()
+        os.unlink(self.file.name)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+                power.append(float(r[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------------ CPU oracle
+
+def oracle_sample(w: Workload, seconds: float, min_slices: int = 2, max_slices: int = 256):
+    """Time the float64 oracle (fwd + bwd) on seeded (b, h) slices of the workload's shape on the host cores.
+
+    Slices are independent problems of identical cost, so TFLOP/s over a sample equals TFLOP/s over the
+    whole batch. Returns (TFLOP/s, cores, description, seconds).
+    """
+    import numpy as np  # noqa: F401
+    from threadpoolctl import threadpool_limits
+
+    from oracle import attn_ref
+    from workloads import make_inputs
+
+    cores = len(os.sched_getaffinity(0))
+    with threadpool_limits(limits=cores):
+        probe = make_inputs(w.with_shape(B=1, H=1, seed=w.seed + 1000))
+        t0 = time.perf_counter()
+        attn_ref.slice_forward_backward(*probe, 0, 0, w.scale)
+        t1 = time.perf_counter() - t0
+        k = int(max(min_slices, min(max_slices, round(seconds / max(t1, 1e-6)))))
+        q, kk, v, do = make_inputs(w.with_shape(B=1, H=k, seed=w.seed + 1001))
+        t0 = time.perf_counter()
+        for h in range(k):
+            attn_ref.slice_forward_backward(q, kk, v, do, 0, h, w.scale)
+        dt = time.perf_counter() - t0
+    f_slice = 3.5 * 2.0 * w.T * w.T * w.D
+    tflops = k * f_slice / dt / 1e12
+    desc = (f"{k} (b,h) slices of {w.name} (T={w.T}, D={w.D}), fwd+bwd float64 numpy, "
+            f"{dt:.1f} s; equal-cost independent slices, so the rate holds for the full batch of {w.B * w.H}")
+    return tflops, cores, desc, dt
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0  # the reference arm runs on rank 0 only
+    w = WORKLOADS[args.workload]
+    from threadpoolctl import threadpool_limits
+
+    from oracle import attn_ref
+    from workloads import make_inputs
+
+    cores = len(os.sched_getaffinity(0))
+    slices = 2  # per step: a bounded sample of the workload
+    q, k, v, do = make_inputs(w.with_shape(B=1, H=slices, seed=w.seed + 2000))
+    times = []
+    with threadpool_limits(limits=cores):
+        for it in range(args.warmup + args.steps):
+            t0 = time.perf_counter()
+            for h in range(slices):
+                attn_ref.slice_forward_backward(q, k, v, do, 0, h, w.scale)
+            if it >= args.warmup:
+                times.append(time.perf_counter() - t0)
+    step = sum(times) / len(times)
+    f_step = slices * 3.5 * 2.0 * w.T * w.T * w.D
+    value = f_step / step / 1e12
+    sample = f"{slices} (b,h) slices of {w.name} per step, float64 numpy oracle fwd+bwd"
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w: Workload):
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D, "causal": True,
+            "scale": "1/sqrt(D)", "recipe": w.recipe,
+            "flop_convention": "fwd 2*B*H*T^2*D, bwd 2.5x fwd",
+            "l2": "no flush: q,k,v,dO together exceed the 126 MB L2" if 4 * w.B * w.T * w.H * w.D * 2 > 126e6
+            else "inputs smaller than L2"}
+
+
+# ------------------------------------------------------------------------------------------------ GPU arm
+
+def make_device_inputs(w: Workload, device):
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed)
+    shape = (w.B, w.T, w.H, w.D)
+    q = torch.randn(shape, generator=g, device=device)
+    k = torch.randn(shape, generator=g, device=device)
+    v = torch.randn(shape, generator=g, device=device)
+    do = torch.randn(shape, generator=g, device=device)
+    if w.qk_prescale != 1.0:
+        q.mul_(w.qk_prescale)
+        k.mul_(w.qk_prescale)
+    if w.key_bias:
+        k.add_(torch.randn((w.D,), generator=g, device=device))
+    return [t.to(torch.bfloat16) for t in (q, k, v, do)]
+
+
+def run_ours(args):
+    import torch
+
+    import causal_self_attention_bf16_b200 as attn
+
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    w = WORKLOADS[args.workload]
+    lib = attn.load_library()
+    B, H, T, D = w.B, w.H, w.T, w.D
+    scale = w.scale
+    q, k, v, do = make_device_inputs(w, device)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws_bytes = attn.attn_bwd_workspace_bytes(B, H, T, D)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    sh = stream.cuda_stream
+    bwd_args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws_bytes, B, H, T, D, scale, sh)
+
+    def check(st, name):
+        if st != 0:
+            raise RuntimeError(f"{name}: {attn._STATUS.get(st, st)} {lib.attn_last_cuda_error().decode()}")
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        check(lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, T, D,
+                           scale, sh), "attn_fwd")
+        if ev is not None:
+            ev[1].record(stream)
+        check(lib.attn_bwd_preprocess(*bwd_args), "attn_bwd_preprocess")
+        if ev is not None:
+            ev[2].record(stream)
+        check(lib.attn_bwd_dkdv(*bwd_args), "attn_bwd_dkdv")
+        if ev is not None:
+            ev[3].record(stream)
+        check(lib.attn_bwd_dq_convert(*bwd_args), "attn_bwd_dq_convert")
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(device)
+    if attn.get_device_error() != 0:
+        raise RuntimeError("a kernel gave up on a bounded wait during warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    sampler = ClockSampler(gpu_id)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    sampler.start()
+    time.sleep(0.1)  # let the sampler start before the timed region
+    start.record(stream)
+    for i in range(args.steps):
+        step(events[i])
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = start.elapsed_time(end)
+    err = attn.get_device_error()
+    if err != 0:
+        raise RuntimeError(f"a kernel gave up on a bounded wait (error word {err:#x}); no number is reported")
+    names = ["attn_fwd_kernel", "attn_bwd_prep_kernel", "attn_bwd_dkdv_kernel", "attn_bwd_dq_kernel"]
+    per = {n: [] for n in names}
+    for ev in events:
+        for j, n in enumerate(names):
+            per[n].append(ev[j].elapsed_time(ev[j + 1]))
+    avg = {n: sum(v_) / len(v_) for n, v_ in per.items()}
+    max_total_ms = reduce_max(total_ms, world, device)
+    ms_step = max_total_ms / args.steps
+    f_fwd, f_bwd = flops(w)
+    value = aggregate((f_fwd + f_bwd) * args.steps, world, max_total_ms / 1e3) / 1e12
+
+    peaks = load_peaks()
+    peak_tf = float(peaks["bf16_tflops"])
+    peak_tf_sus = float(peaks.get("bf16_tflops_sustained", peak_tf))
+    hbm = float(peaks["hbm_gbs"])
+    n = B * T * H * D
+    kernels = {
+        "attn_fwd_kernel": {"bound": "tensor", "unit": "TFLOP/s", "work": f_fwd, "per": 1e12,
+                            "alg_bytes": 4 * n * 2 + B * H * T * 4},
+        "attn_bwd_prep_kernel": {"bound": "hbm", "unit": "GB/s", "work": 2 * n * 2 + B * H * T * 4 * 3 +
+                                 B * H * ((T + 127) // 128 * 128) * 128 * 4, "per": 1e9},
+        "attn_bwd_dkdv_kernel": {"bound": "tensor", "unit": "TFLOP/s", "work": f_bwd, "per": 1e12,
+                                 "alg_bytes": 7 * n * 2 + B * H * T * 8},
+        "attn_bwd_dq_kernel": {"bound": "hbm", "unit": "GB/s", "work": n * 4 + n * 2, "per": 1e9},
+    }
+    breakdown = {}
+    for name, kinfo in kernels.items():
+        t = avg[name] / 1e3
+        ach = kinfo["work"] / t / kinfo["per"]
+        pk = peak_tf if kinfo["bound"] == "tensor" else hbm
+        breakdown[name] = {"avg_ms": avg[name], "share": avg[name] / sum(avg.values()), "achieved": ach,
+                           "unit": kinfo["unit"], "frac": ach / pk}
+    dom = max(avg, key=avg.get)
+    kd = kernels[dom]
+    ach = breakdown[dom]["achieved"]
+    pk = peak_tf if kd["bound"] == "tensor" else hbm
+    roofline = {"kernel": dom, "bound": kd["bound"], "achieved": ach, "peak": pk, "unit": kd["unit"],
+                "frac": ach / pk, "traffic": recorded_traffic(dom, w.name),
+                "peak_source": f"{peaks['source']} ({'bf16_tflops burst' if kd['bound'] == 'tensor' else 'hbm_gbs'})"}
+    if kd["bound"] == "tensor":
+        roofline["frac_of_sustained_peak"] = ach / peak_tf_sus
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "ours",
+        "config": dict(workload_config(w), parallelism=f"replicas x{world} (no collective on the data path)"),
+        "pct_of_peak": 100.0 * (value / world) / peak_tf,
+        "fwd_tflops": f_fwd / (avg["attn_fwd_kernel"] / 1e3) / 1e12,
+        "bwd_tflops": f_bwd / (sum(avg.values()) - avg["attn_fwd_kernel"]) * 1e3 / 1e12,
+        "roofline": roofline, "kernels": breakdown, "gpu_launches": 4 * args.steps, "clocks": clocks,
+        "kernel_source_hash": kernel_source_hash(),
+    }
+
+    # End to end through the public Python API with host buffers: H2D of q, k, v, dO from pinned memory,
+    # forward, backward, D2H of o, lse, dq, dk, dv, every step.
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+        ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=torch.bfloat16).pin_memory() for _ in range(4))
+        hlse = torch.empty((B, H, T), dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            do.copy_(hdo, non_blocking=True)
+            attn.attn_fwd(q, k, v, scale, o=o, lse=lse)
+            attn.attn_bwd(q, k, v, o, lse, do, scale, dq=dq, dk=dk, dv=dv, workspace=ws)
+            ho.copy_(o, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+            hdq.copy_(dq, non_blocking=True)
+            hdk.copy_(dk, non_blocking=True)
+            hdv.copy_(dv, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize(device)
+        e_steps = 5
+        if world > 1:
+            torch.distributed.barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        s1.record(stream)
+        torch.cuda.synchronize(device)
+        e_ms = reduce_max(s0.elapsed_time(s1), world, device)
+        line["e2e"] = {"value": aggregate((f_fwd + f_bwd) * e_steps, world, e_ms / 1e3) / 1e12, "unit": UNIT,
+                       "h2d_bytes_per_step": 4 * n * 2, "d2h_bytes_per_step": 4 * n * 2 + B * H * T * 4,
+                       "ms_per_step": e_ms / e_steps}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, cores, desc, _ = oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

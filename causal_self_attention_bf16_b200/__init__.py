@@ -1,0 +1,209 @@
+"""Thin Python binding of libattn.so: bf16 causal multi-head self-attention, forward and backward, on B200.
+
+Every step of the computation runs in the library's sm_100a kernels. This module only marshals arguments:
+it checks dtypes/shapes, allocates outputs with torch (device memory is plumbing), and passes raw device
+pointers and the current CUDA stream through the C ABI declared in include/attn.h. There is no CPU path: if
+the library is missing or the device is not an sm_100 GPU, the calls raise.
+
+The operation is nanochat's ``flash_attn_func(q, k, v, causal=True)`` on [B, T, H, D] tensors (apidog "Train
+your own ChatGPT", section 5 "Flash Attention integration"), with the textbook definition written out in
+include/attn.h.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libattn.so")
+
+ATTN_OK = 0
+_STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_MISALIGNED",
+           4: "ATTN_ERR_CUDA", 5: "ATTN_ERR_TIMEOUT", 6: "ATTN_ERR_WORKSPACE"}
+
+# Exported symbols of the C ABI (include/attn.h), with their ctypes signatures.
+_VP, _I, _F, _SZ, _U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint64
+SIGNATURES = {
+    "attn_abi_version": ([], _I),
+    "attn_status_string": ([_I], ctypes.c_char_p),
+    "attn_last_cuda_error": ([], ctypes.c_char_p),
+    "attn_fwd": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _VP], _I),
+    "attn_bwd_workspace_bytes": ([_I, _I, _I, _I], _SZ),
+    "attn_bwd": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _F, _VP], _I),
+    "attn_bwd_preprocess": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _F, _VP], _I),
+    "attn_bwd_dkdv": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _F, _VP], _I),
+    "attn_bwd_dq_convert": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _F, _VP], _I),
+    "attn_get_device_error": ([ctypes.POINTER(ctypes.c_uint32)], _I),
+    "attn_clear_device_error": ([], _I),
+    "attn_set_wait_limit_ns": ([_U64], _I),
+    "attn_selftest_wait_timeout": ([_U64, _VP], _I),
+}
+
+
+class AttnError(RuntimeError):
+    """A non-OK status returned by libattn.so."""
+
+    def __init__(self, fn: str, status: int, detail: str = ""):
+        self.status = status
+        msg = f"{fn} returned {_STATUS.get(status, status)}"
+        if detail:
+            msg += f" ({detail})"
+        super().__init__(msg)
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libattn.so (once) and attach the C signatures. Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m causal_self_attention_bf16_b200.build` "
+                          "(or __graft_entry__.build()); there is no fallback implementation")
+    lib = ctypes.CDLL(path)
+    for name, (argtypes, restype) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.argtypes = argtypes
+        fn.restype = restype
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, status: int):
+    if status != ATTN_OK:
+        detail = ""
+        if status == 4:
+            detail = load_library().attn_last_cuda_error().decode(errors="replace")
+        raise AttnError(fn, status, detail)
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream], device: torch.device) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return s.cuda_stream
+
+
+def _check_qkv(name: str, t: torch.Tensor, shape=None):
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be bfloat16, got {t.dtype}")
+    if t.dim() != 4 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous [B, T, H, D] tensor")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,
+             o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+             stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Causal attention forward. q, k, v: bf16 [B, T, H, D] on one CUDA device. Returns (o, lse [B, H, T])."""
+    lib = load_library()
+    _check_qkv("q", q)
+    B, T, H, D = q.shape
+    _check_qkv("k", k, q.shape)
+    _check_qkv("v", v, q.shape)
+    if o is None:
+        o = torch.empty_like(q)
+    _check_qkv("o", o, q.shape)
+    if lse is None:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, T) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, T] tensor")
+    scale = default_scale(D) if scale is None else float(scale)
+    st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, T, D, scale,
+                      _stream_handle(stream, q.device))
+    _check("attn_fwd", st)
+    return o, lse
+
+
+def attn_bwd_workspace_bytes(B: int, H: int, T: int, D: int) -> int:
+    return int(load_library().attn_bwd_workspace_bytes(B, H, T, D))
+
+
+def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+             dO: torch.Tensor, scale: Optional[float] = None, dq: Optional[torch.Tensor] = None,
+             dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
+             workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+    """Causal attention backward. Returns (dq, dk, dv), bf16 [B, T, H, D]."""
+    lib = load_library()
+    _check_qkv("q", q)
+    B, T, H, D = q.shape
+    for name, t in (("k", k), ("v", v), ("o", o), ("dO", dO)):
+        _check_qkv(name, t, q.shape)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, T) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 [B, H, T] tensor")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _check_qkv(name, t, q.shape)
+    need = attn_bwd_workspace_bytes(B, H, T, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    scale = default_scale(D) if scale is None else float(scale)
+    st = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dO.data_ptr(),
+                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                      workspace.numel() * workspace.element_size(), B, H, T, D, scale,
+                      _stream_handle(stream, q.device))
+    _check("attn_bwd", st)
+    return dq, dk, dv
+
+
+def get_device_error() -> int:
+    """The library's device-side error word (0 = no kernel gave up on a bounded wait). Synchronises."""
+    word = ctypes.c_uint32(0)
+    st = load_library().attn_get_device_error(ctypes.byref(word))
+    if st not in (0, 5):
+        _check("attn_get_device_error", st)
+    return int(word.value)
+
+
+def clear_device_error():
+    _check("attn_clear_device_error", load_library().attn_clear_device_error())
+
+
+def set_wait_limit_ns(limit_ns: int):
+    _check("attn_set_wait_limit_ns", load_library().attn_set_wait_limit_ns(int(limit_ns)))
+
+
+def selftest_wait_timeout(limit_ns: int, stream: Optional[torch.cuda.Stream] = None):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _check("attn_selftest_wait_timeout",
+           load_library().attn_selftest_wait_timeout(int(limit_ns), _stream_handle(stream, dev)))
+
+
+class CausalAttentionFunction(torch.autograd.Function):
+    """autograd wrapper: forward saves (q, k, v, o, lse); backward calls attn_bwd."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, scale):
+        o, lse = attn_fwd(q, k, v, scale)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.scale = scale
+        return o
+
+    @staticmethod
+    def backward(ctx, dO):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = attn_bwd(q, k, v, o, lse, dO.contiguous(), ctx.scale)
+        return dq, dk, dv, None
+
+
+def causal_attention(q, k, v, scale: Optional[float] = None):
+    """Differentiable causal attention on bf16 [B, T, H, D] tensors (the flash_attn_func(causal=True) call)."""
+    return CausalAttentionFunction.apply(q, k, v, default_scale(q.shape[-1]) if scale is None else scale)
+
+
+__all__ = ["attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "causal_attention", "CausalAttentionFunction",
+           "get_device_error", "clear_device_error", "set_wait_limit_ns", "selftest_wait_timeout", "AttnError",
+           "load_library", "LIB_PATH", "SIGNATURES"]

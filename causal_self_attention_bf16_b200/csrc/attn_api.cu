@@ -1,0 +1,348 @@
+// Host side of libattn.so: argument validation, TMA tensor-map encoding and kernel launches behind the
+// C ABI declared in include/attn.h. No allocation, no synchronisation on the attention path.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "attn.h"
+#include "attn_bwd.cuh"
+#include "attn_fwd.cuh"
+
+namespace {
+
+thread_local char g_cuda_error[256] = "";
+uint64_t g_wait_limit_ns = 1000ull * 1000 * 1000;  // 1 s
+
+attn_status cuda_fail(cudaError_t e, const char* what) {
+  std::snprintf(g_cuda_error, sizeof(g_cuda_error), "%s: %s", what, cudaGetErrorString(e));
+  return ATTN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------------------------- tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn(cudaError_t* err) {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  static cudaError_t e0 = cudaSuccess;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    e0 = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e0 == cudaSuccess && q == cudaDriverEntryPointSuccess) fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  *err = e0;
+  return fn;
+}
+
+// A [B, T, H, 128] bf16 tensor seen by TMA as dims {D, H, T, B} (strides increase outward), with a box of
+// 64 head-dim columns (128 bytes, the 128-byte swizzle span) x one head x `rows` time steps.
+attn_status make_map(CUtensorMap* m, const void* ptr, int B, int H, int T, int rows) {
+  cudaError_t e;
+  EncodeTiledFn fn = encode_fn(&e);
+  if (!fn) return cuda_fail(e == cudaSuccess ? cudaErrorNotSupported : e, "cuTensorMapEncodeTiled lookup");
+  const cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {256, static_cast<cuuint64_t>(H) * 256, static_cast<cuuint64_t>(T) * H * 256};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(rows), 1};
+  const cuuint32_t elem[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, elem,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_cuda_error, sizeof(g_cuda_error), "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+// ---------------------------------------------------------------------------------------------- checks
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;
+};
+Range span(const void* p, size_t bytes) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  return {a, a + bytes};
+}
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+attn_status check_sizes(int B, int H, int T, int D, float scale) {
+  if (B < 1 || H < 1 || T < 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (D != 128) return ATTN_ERR_UNSUPPORTED;
+  // Kernel indexing: CTA counts and (b*H + h) fit in 31 bits; element offsets use 64-bit arithmetic.
+  const long long bh = static_cast<long long>(B) * H;
+  const long long qtiles = (static_cast<long long>(T) + 127) / 128;
+  if (bh * qtiles * 2 > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (T > (1 << 30)) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+// Set the dynamic shared-memory opt-in of both big kernels once per device.
+attn_status prepare_device(int* dev_out) {
+  static std::mutex mu;
+  static bool done[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  // Make the device's primary context current on this thread (a thread that has only queued work through
+  // another runtime, such as an autograd worker, may have none); the tensor-map encoder needs one.
+  if ((e = cudaSetDevice(dev)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  *dev_out = dev;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < 64 && done[dev]) return ATTN_OK;
+  int major = 0, minor = 0;
+  if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+    return cuda_fail(e, "cudaDeviceGetAttribute");
+  if (major != 10 || minor != 0) {
+    std::snprintf(g_cuda_error, sizeof(g_cuda_error), "device %d is sm_%d%d; this library is built for sm_100a",
+                  dev, major, minor);
+    return ATTN_ERR_CUDA;
+  }
+  if ((e = cudaFuncSetAttribute(attn::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                attn::kFwdSmemAlloc)) != cudaSuccess)
+    return cuda_fail(e, "cudaFuncSetAttribute(attn_fwd_kernel)");
+  if ((e = cudaFuncSetAttribute(attn::attn_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                attn::kBwdSmemAlloc)) != cudaSuccess)
+    return cuda_fail(e, "cudaFuncSetAttribute(attn_bwd_dkdv_kernel)");
+  if (dev >= 0 && dev < 64) done[dev] = true;
+  return ATTN_OK;
+}
+
+struct WorkspaceLayout {
+  size_t lse2, delta, acc, total;
+};
+WorkspaceLayout workspace_layout(int B, int H, int T) {
+  const size_t rows = static_cast<size_t>(B) * H * attn::padded_T(T);
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  WorkspaceLayout w;
+  w.lse2 = 0;
+  w.delta = up(rows * 4);
+  w.acc = w.delta + up(rows * 4);
+  w.total = w.acc + up(rows * 128 * 4);
+  return w;
+}
+
+int grid_for(size_t work_items, int per_block) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const size_t blocks = (work_items + per_block - 1) / per_block;
+  const size_t cap = static_cast<size_t>(sms) * 8;
+  return static_cast<int>(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
+}
+
+// Self-test kernel for the bounded-wait path (see attn_selftest_wait_timeout).
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    abort_flag = 0;
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) sm100::mbar_wait(&bar, 0, &abort_flag, limit_ns, &attn::g_device_error, 0x7f);
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_abi_version(void) { return 1; }
+
+const char* attn_status_string(attn_status s) {
+  switch (s) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_MISALIGNED: return "ATTN_ERR_MISALIGNED";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE";
+  }
+  return "ATTN_ERR_UNKNOWN";
+}
+
+const char* attn_last_cuda_error(void) { return g_cuda_error; }
+
+attn_status attn_set_wait_limit_ns(uint64_t limit_ns) {
+  if (limit_ns < 1000) return ATTN_ERR_INVALID_ARG;
+  g_wait_limit_ns = limit_ns;
+  return ATTN_OK;
+}
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T, int D,
+                     float scale, void* stream) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  attn_status st = check_sizes(B, H, T, D, scale);
+  if (st != ATTN_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return ATTN_ERR_MISALIGNED;
+  const size_t nbytes = static_cast<size_t>(B) * T * H * D * 2;
+  const size_t lbytes = static_cast<size_t>(B) * H * T * 4;
+  const Range rq = span(q, nbytes), rk = span(k, nbytes), rv = span(v, nbytes), ro = span(o, nbytes),
+              rl = span(lse, lbytes);
+  for (Range in : {rq, rk, rv})
+    if (overlap(ro, in) || overlap(rl, in)) return ATTN_ERR_INVALID_ARG;
+  if (overlap(ro, rl)) return ATTN_ERR_INVALID_ARG;
+
+  int dev = 0;
+  if ((st = prepare_device(&dev)) != ATTN_OK) return st;
+  CUtensorMap mq, mk, mv, mo;
+  if ((st = make_map(&mq, q, B, H, T, attn::kTile)) != ATTN_OK) return st;
+  if ((st = make_map(&mk, k, B, H, T, attn::kTile)) != ATTN_OK) return st;
+  if ((st = make_map(&mv, v, B, H, T, attn::kTile)) != ATTN_OK) return st;
+  if ((st = make_map(&mo, o, B, H, T, attn::kTile)) != ATTN_OK) return st;
+
+  attn::FwdParams p;
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.T = T;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_wait_limit_ns;
+  const unsigned n_qt = static_cast<unsigned>((T + attn::kTile - 1) / attn::kTile);
+  const dim3 grid(n_qt * static_cast<unsigned>(B * H));
+  attn::attn_fwd_kernel<<<grid, attn::kFwdThreads, attn::kFwdSmemAlloc, static_cast<cudaStream_t>(stream)>>>(
+      mq, mk, mv, mo, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
+  return ATTN_OK;
+}
+
+size_t attn_bwd_workspace_bytes(int B, int H, int T, int D) {
+  if (check_sizes(B, H, T, D, 1.0f) != ATTN_OK) return 0;
+  return workspace_layout(B, H, T).total;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Validates the backward arguments and launches the stages selected by `stages` (bit 0: preprocess,
+// bit 1: dK/dV with dQ accumulation, bit 2: dQ conversion) in that order on `stream`.
+attn_status bwd_launch(unsigned stages, const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B,
+                       int H, int T, int D, float scale, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+  attn_status st = check_sizes(B, H, T, D, scale);
+  if (st != ATTN_OK) return st;
+  const WorkspaceLayout wl = workspace_layout(B, H, T);
+  if (!workspace || workspace_bytes < wl.total) return ATTN_ERR_WORKSPACE;
+  for (const void* ptr : {q, k, v, o, dO, static_cast<const void*>(lse), static_cast<const void*>(dq),
+                          static_cast<const void*>(dk), static_cast<const void*>(dv)})
+    if (!aligned16(ptr)) return ATTN_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_MISALIGNED;
+  const size_t nbytes = static_cast<size_t>(B) * T * H * D * 2;
+  const size_t lbytes = static_cast<size_t>(B) * H * T * 4;
+  const Range ins[6] = {span(q, nbytes), span(k, nbytes), span(v, nbytes), span(o, nbytes), span(dO, nbytes),
+                        span(lse, lbytes)};
+  const Range outs[4] = {span(dq, nbytes), span(dk, nbytes), span(dv, nbytes), span(workspace, wl.total)};
+  for (int i = 0; i < 4; ++i) {
+    for (int j = 0; j < 6; ++j)
+      if (overlap(outs[i], ins[j])) return ATTN_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 4; ++j)
+      if (overlap(outs[i], outs[j])) return ATTN_ERR_INVALID_ARG;
+  }
+
+  int dev = 0;
+  if ((st = prepare_device(&dev)) != ATTN_OK) return st;
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
+  if ((st = make_map(&mq, q, B, H, T, attn::kBwdQTile)) != ATTN_OK) return st;
+  if ((st = make_map(&mdo, dO, B, H, T, attn::kBwdQTile)) != ATTN_OK) return st;
+  if ((st = make_map(&mk, k, B, H, T, attn::kBwdKTile)) != ATTN_OK) return st;
+  if ((st = make_map(&mv, v, B, H, T, attn::kBwdKTile)) != ATTN_OK) return st;
+  if ((st = make_map(&mdk, dk, B, H, T, attn::kBwdKTile)) != ATTN_OK) return st;
+  if ((st = make_map(&mdv, dv, B, H, T, attn::kBwdKTile)) != ATTN_OK) return st;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  attn::BwdParams p;
+  p.o = static_cast<const __nv_bfloat16*>(o);
+  p.dO = static_cast<const __nv_bfloat16*>(dO);
+  p.lse = lse;
+  p.lse2 = reinterpret_cast<float*>(ws + wl.lse2);
+  p.delta = reinterpret_cast<float*>(ws + wl.delta);
+  p.dq_acc = reinterpret_cast<float*>(ws + wl.acc);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.B = B;
+  p.H = H;
+  p.T = T;
+  p.Tp = attn::padded_T(T);
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_wait_limit_ns;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  cudaError_t e;
+  if (stages & 1u) {
+    const size_t rows = static_cast<size_t>(B) * H * p.Tp;
+    attn::attn_bwd_prep_kernel<<<grid_for(rows * 16, 256), 256, 0, s>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_bwd_prep_kernel launch");
+  }
+  if (stages & 2u) {
+    const unsigned n_kt = static_cast<unsigned>((T + attn::kBwdKTile - 1) / attn::kBwdKTile);
+    attn::attn_bwd_dkdv_kernel<<<dim3(n_kt * static_cast<unsigned>(B * H)), attn::kBwdThreads,
+                                 attn::kBwdSmemAlloc, s>>>(mq, mk, mv, mdo, mdk, mdv, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_bwd_dkdv_kernel launch");
+  }
+  if (stages & 4u) {
+    const size_t items = static_cast<size_t>(B) * H * ((T + 3) / 4) * 32;
+    attn::attn_bwd_dq_kernel<<<grid_for(items, 256), 256, 0, s>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_bwd_dq_kernel launch");
+  }
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+#define ATTN_BWD_ARGS                                                                                          \
+  const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dO, void *dq,     \
+      void *dk, void *dv, void *workspace, size_t workspace_bytes, int B, int H, int T, int D, float scale,     \
+      void *stream
+#define ATTN_BWD_PASS q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, H, T, D, scale, stream
+
+attn_status attn_bwd(ATTN_BWD_ARGS) { return bwd_launch(7u, ATTN_BWD_PASS); }
+attn_status attn_bwd_preprocess(ATTN_BWD_ARGS) { return bwd_launch(1u, ATTN_BWD_PASS); }
+attn_status attn_bwd_dkdv(ATTN_BWD_ARGS) { return bwd_launch(2u, ATTN_BWD_PASS); }
+attn_status attn_bwd_dq_convert(ATTN_BWD_ARGS) { return bwd_launch(4u, ATTN_BWD_PASS); }
+
+attn_status attn_get_device_error(uint32_t* word) {
+  if (!word) return ATTN_ERR_INVALID_ARG;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  e = cudaMemcpyFromSymbol(word, attn::g_device_error, sizeof(uint32_t));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol(g_device_error)");
+  return *word ? ATTN_ERR_TIMEOUT : ATTN_OK;
+}
+
+attn_status attn_clear_device_error(void) {
+  const uint32_t zero = 0;
+  cudaError_t e = cudaMemcpyToSymbol(attn::g_device_error, &zero, sizeof(uint32_t));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol(g_device_error)");
+  e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  return ATTN_OK;
+}
+
+attn_status attn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > 10ull * 1000 * 1000 * 1000) return ATTN_ERR_INVALID_ARG;
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "wait_timeout_selftest_kernel launch");
+  return ATTN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,133 @@
+/*
+ * attn.h - C ABI of the B200 (sm_100a) bf16 causal multi-head self-attention library (libattn.so).
+ *
+ * What it computes. nanochat calls flash_attn_func(q, k, v, causal=True, window_size=...) on [B, T, H, D]
+ * tensors and trains through it (apidog "Train your own ChatGPT", section 5 "Flash Attention integration";
+ * the [B, T, n_head, head_dim] view is in section 1 "GPT model"). The pages print no formula, so this
+ * library implements the textbook definition, per batch b and head h, with s = `scale`:
+ *
+ *   forward   S = s * Q K^T with S[i][j] = -inf for j > i (top-left causal mask, T_q = T_k)
+ *             O = softmax_rows(S) V,   LSE[i] = ln sum_j exp(S[i][j])          (natural log)
+ *   backward  P = exp(S - LSE),  dV = P^T dO,  dP = dO V^T,  Delta = rowsum(dO * O),
+ *             dS = P * (dP - Delta),  dQ = s * dS K,  dK = s * dS^T Q
+ *
+ * Shapes come from nanochat's depth dial: width 64 * depth, 128 dims per head (aisight.pl nanochat review,
+ * "Model and scaling assumptions": d20 = 1280 channels, 10 heads of 128), so D = 128 is the only head size.
+ *
+ * Conventions for every entry point
+ *   - Tensors are device pointers. q, k, v, o, dO, dq, dk, dv: bf16, [B, T, H, D] contiguous (D fastest).
+ *     lse: fp32 [B, H, T] contiguous. Every pointer must be 16-byte aligned (TMA requirement).
+ *   - The caller owns and allocates every buffer, including the backward workspace. The library never
+ *     allocates, frees or synchronises; all work is enqueued asynchronously on `stream` (a cudaStream_t;
+ *     NULL = legacy default stream) on the current CUDA device.
+ *   - Outputs must not overlap inputs or each other.
+ *   - Argument errors are detected on the host before anything is launched and leave outputs untouched.
+ *   - There is no CPU fallback: on a machine without an sm_100 device the calls return ATTN_ERR_CUDA.
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, non-finite or non-positive scale, overlap */
+  ATTN_ERR_UNSUPPORTED = 2,  /* D != 128, or sizes beyond the kernels' index range */
+  ATTN_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned */
+  ATTN_ERR_CUDA = 4,         /* a CUDA runtime/driver call or a launch failed; see attn_last_cuda_error() */
+  ATTN_ERR_TIMEOUT = 5,      /* a kernel gave up on a bounded wait (reported by attn_get_device_error) */
+  ATTN_ERR_WORKSPACE = 6     /* backward workspace missing or smaller than attn_bwd_workspace_bytes() */
+} attn_status;
+
+/* Version of this ABI; bumped on any incompatible change of a signature or of a buffer layout. */
+int attn_abi_version(void);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char* attn_status_string(attn_status s);
+
+/* Text of the last CUDA error seen by this library on the calling thread ("" if none). */
+const char* attn_last_cuda_error(void);
+
+/*
+ * Forward: o = softmax(scale * q k^T + causal mask) v and lse = per-row natural log-sum-exp of the scaled,
+ * masked logits (the saved statistic the backward needs).
+ *   q, k, v  in : bf16 [B, T, H, D]
+ *   o       out : bf16 [B, T, H, D]
+ *   lse     out : fp32 [B, H, T]
+ *   B, H, T >= 1; D must be 128; scale finite and > 0 (usually 1/sqrt(D)).
+ * Launches one kernel. Returns ATTN_OK once the launch is enqueued.
+ */
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T,
+                     int D, float scale, void* stream);
+
+/*
+ * Size in bytes of the scratch buffer attn_bwd needs for these sizes (0 if the sizes are invalid):
+ * per (b, h) row, LSE * log2(e) and Delta (fp32, T rounded up to 128) and an fp32 dQ accumulator.
+ */
+size_t attn_bwd_workspace_bytes(int B, int H, int T, int D);
+
+/*
+ * Backward: dq, dk, dv of L = sum(dO * o), for o and lse returned by attn_fwd on the same q, k, v, scale.
+ *   q, k, v, o, dO    in : bf16 [B, T, H, D];   lse in : fp32 [B, H, T]
+ *   dq, dk, dv       out : bf16 [B, T, H, D]
+ *   workspace  scratch   : device buffer of at least attn_bwd_workspace_bytes(B, H, T, D) bytes,
+ *                          256-byte aligned; its contents on entry do not matter and are overwritten.
+ * Launches three kernels (Delta/LSE preprocessing with accumulator zeroing; dK/dV with dQ accumulation;
+ * dQ conversion). Calls that share one workspace must not overlap in time on the GPU.
+ */
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                     int B, int H, int T, int D, float scale, void* stream);
+
+/*
+ * The three stages of attn_bwd, callable one at a time with exactly attn_bwd's arguments (the same checks
+ * apply). Calling attn_bwd_preprocess, attn_bwd_dkdv, attn_bwd_dq_convert in this order on one stream is
+ * the same work as one attn_bwd call; profilers and benchmarks use them to time each kernel on its own.
+ *   attn_bwd_preprocess : Delta = rowsum(dO * o), LSE * log2(e) into the workspace; zero the dQ accumulator.
+ *   attn_bwd_dkdv       : dk, dv, and dQ partial sums added into the workspace accumulator.
+ *   attn_bwd_dq_convert : dq = bf16(scale * accumulator).
+ */
+attn_status attn_bwd_preprocess(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                const void* dO, void* dq, void* dk, void* dv, void* workspace,
+                                size_t workspace_bytes, int B, int H, int T, int D, float scale, void* stream);
+attn_status attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                          const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                          int B, int H, int T, int D, float scale, void* stream);
+attn_status attn_bwd_dq_convert(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                const void* dO, void* dq, void* dk, void* dv, void* workspace,
+                                size_t workspace_bytes, int B, int H, int T, int D, float scale, void* stream);
+
+/*
+ * Device-side error word shared by the kernels of this library on the current device: 0 if no kernel has
+ * given up on a bounded wait since the last clear; otherwise (site << 8) | 1. Synchronises the device.
+ * Returns ATTN_ERR_TIMEOUT if the word is non-zero, ATTN_OK if it is zero, ATTN_ERR_CUDA on a CUDA error.
+ */
+attn_status attn_get_device_error(uint32_t* word);
+
+/* Clear the device-side error word of the current device (synchronous). */
+attn_status attn_clear_device_error(void);
+
+/*
+ * Upper bound, in nanoseconds of GPU global time, on any single wait inside the kernels (default 1e9).
+ * A wait that runs out ends its kernel early with the error word set, instead of hanging the GPU.
+ * Values below 1000 are rejected with ATTN_ERR_INVALID_ARG.
+ */
+attn_status attn_set_wait_limit_ns(uint64_t limit_ns);
+
+/*
+ * Self-test of the bounded-wait path: launches one CTA that waits on a barrier nothing ever completes,
+ * with a limit of `limit_ns`; the kernel gives up, records its site (0x7f) in the error word and returns.
+ * Used by the failure-detection test; never part of the attention path.
+ */
+attn_status attn_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H_ */

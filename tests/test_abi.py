@@ -1,0 +1,136 @@
+"""The C-ABI library loads, exports every symbol include/attn.h declares, and validates arguments on the host.
+
+No test here needs a GPU: argument errors are detected before any CUDA call, and a well-formed call on a
+machine without an sm_100 device must fail loudly (ATTN_ERR_CUDA), never fall back to a CPU path.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import causal_self_attention_bf16_b200 as attn
+from causal_self_attention_bf16_b200 import build as attn_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    attn_build.build()
+    return attn.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_status_string"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert names, "no declarations parsed"
+    for n in names:
+        assert hasattr(lib, n), f"libattn.so does not export {n}"
+    assert set(names) == set(attn.SIGNATURES), "binding signature table and header disagree"
+
+
+def test_abi_version_and_status_strings(lib):
+    assert lib.attn_abi_version() == 1
+    for code, name in attn._STATUS.items():
+        assert lib.attn_status_string(code).decode() == name
+
+
+def test_workspace_size_formula(lib):
+    # lse2 + delta: B*H*Tp fp32 each (256-byte rounded), accumulator B*H*Tp*128 fp32.
+    for B, H, T in ((1, 1, 1), (2, 3, 100), (32, 10, 2048)):
+        Tp = (T + 127) // 128 * 128
+        rows = B * H * Tp
+        up = lambda x: (x + 255) // 256 * 256
+        assert lib.attn_bwd_workspace_bytes(B, H, T, 128) == 2 * up(rows * 4) + up(rows * 512)
+    assert lib.attn_bwd_workspace_bytes(1, 1, 1, 64) == 0
+    assert lib.attn_bwd_workspace_bytes(0, 1, 1, 128) == 0
+
+
+# Fake, aligned, non-overlapping device addresses: never dereferenced on the host, and every call below
+# fails its checks before anything reaches CUDA.
+def fake_ptrs(n, size):
+    base = 1 << 40
+    return [base + i * (size + (1 << 20)) for i in range(n)]
+
+
+def fwd_call(lib, q, k, v, o, lse, B=1, H=2, T=128, D=128, scale=0.088):
+    return lib.attn_fwd(q, k, v, o, lse, B, H, T, D, scale, None)
+
+
+def test_fwd_argument_errors(lib):
+    size = 1 * 128 * 2 * 128 * 2
+    q, k, v, o, lse = fake_ptrs(5, size)
+    assert fwd_call(lib, None, k, v, o, lse) == 1
+    assert fwd_call(lib, q, k, v, None, lse) == 1
+    assert fwd_call(lib, q, k, v, o, lse, B=0) == 1
+    assert fwd_call(lib, q, k, v, o, lse, T=-3) == 1
+    assert fwd_call(lib, q, k, v, o, lse, scale=0.0) == 1
+    assert fwd_call(lib, q, k, v, o, lse, scale=float("nan")) == 1
+    assert fwd_call(lib, q, k, v, o, lse, scale=float("inf")) == 1
+    assert fwd_call(lib, q, k, v, o, lse, D=64) == 2
+    assert fwd_call(lib, q + 8, k, v, o, lse) == 3
+    assert fwd_call(lib, q, k, v, o, lse + 4) == 3
+    assert fwd_call(lib, q, k, v, q + 256, lse) == 1          # o overlaps q
+    assert fwd_call(lib, q, k, v, o, o + 1024) == 1           # lse overlaps o
+
+
+def bwd_call(lib, ptrs, ws_bytes, B=1, H=2, T=128, D=128, scale=0.088, **over):
+    names = ["q", "k", "v", "o", "lse", "dO", "dq", "dk", "dv", "ws"]
+    args = dict(zip(names, ptrs))
+    args.update(over)
+    return lib.attn_bwd(*[args[n] for n in names], ws_bytes, B, H, T, D, scale, None)
+
+
+def test_bwd_argument_errors(lib):
+    size = 1 * 128 * 2 * 128 * 2
+    ws = lib.attn_bwd_workspace_bytes(1, 2, 128, 128)
+    ptrs = fake_ptrs(10, max(size, ws))
+    assert bwd_call(lib, ptrs, ws, dq=None) == 1
+    assert bwd_call(lib, ptrs, ws, D=96) == 2
+    assert bwd_call(lib, ptrs, ws - 1) == 6
+    assert bwd_call(lib, ptrs, ws, ws=None) == 6
+    assert bwd_call(lib, ptrs, ws, dk=ptrs[7] + 8) == 3
+    assert bwd_call(lib, ptrs, ws, ws=ptrs[9] + 16) == 3      # workspace must be 256-byte aligned
+    assert bwd_call(lib, ptrs, ws, dq=ptrs[0]) == 1           # dq aliases q
+    assert bwd_call(lib, ptrs, ws, dv=ptrs[6]) == 1           # dv aliases dq
+    assert bwd_call(lib, ptrs, ws, ws=ptrs[8]) == 1           # workspace aliases dv
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_no_cpu_fallback_without_gpu(lib):
+    """A well-formed call on a machine without an sm_100 GPU fails loudly instead of computing on the CPU."""
+    size = 1 * 128 * 2 * 128 * 2
+    q, k, v, o, lse = fake_ptrs(5, size)
+    assert fwd_call(lib, q, k, v, o, lse) == 4
+    assert lib.attn_last_cuda_error().decode() != ""
+    ws = lib.attn_bwd_workspace_bytes(1, 2, 128, 128)
+    assert bwd_call(lib, fake_ptrs(10, max(size, ws)), ws) == 4
+
+
+def test_binding_rejects_cpu_tensors(lib):
+    q = torch.zeros(1, 128, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        attn.attn_fwd(q, q, q)
+
+
+def test_binding_signatures_match_header_argument_counts():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    for name, (argtypes, _) in attn.SIGNATURES.items():
+        m = re.search(name + r"\s*\(([^)]*)\)", text)
+        assert m, name
+        params = [p for p in m.group(1).split(",") if p.strip() and p.strip() != "void"]
+        assert len(params) == len(argtypes), f"{name}: header has {len(params)} params, binding {len(argtypes)}"

@@ -1,0 +1,211 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle.
+
+Tolerances (stated for the rebuilt path; the pages give none):
+  O      : max|err| <= 1e-2 * max|ref| + 1e-3
+  dQ/dK/dV: ||gpu - ref||_F / ||ref||_F <= 2e-2
+  LSE    : max|err| <= 1e-3 * max(1, |ref|)
+The GPU rounds inputs to bf16 (the oracle sees the same bf16 values), rounds P and dS to bf16 before its
+matrix products and rounds outputs to bf16; these bounds leave room for that and nothing else.
+
+Small cases compare every element; the full-size workloads (exactly the shapes and the launch the benchmark
+times) compare seeded (b, h) slices, which are independent problems the oracle computes one by one.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import causal_self_attention_bf16_b200 as attn
+from oracle import attn_ref
+from workloads import WORKLOADS, Workload, make_inputs, sample_slices
+
+pytestmark = pytest.mark.gpu
+
+O_REL, O_ABS = 1e-2, 1e-3
+GRAD_FRO = 2e-2
+LSE_TOL = 1e-3
+
+
+def check_o(o_gpu, o_ref, what=""):
+    o_gpu = np.asarray(o_gpu, dtype=np.float64)
+    err = np.abs(o_gpu - o_ref).max()
+    bound = O_REL * np.abs(o_ref).max() + O_ABS
+    assert err <= bound, f"{what} O: max err {err:.3e} > {bound:.3e}"
+
+
+def check_lse(l_gpu, l_ref, what=""):
+    err = np.abs(np.asarray(l_gpu, dtype=np.float64) - l_ref)
+    assert np.all(err <= LSE_TOL * np.maximum(1.0, np.abs(l_ref))), f"{what} LSE: max err {err.max():.3e}"
+
+
+def check_grad(g_gpu, g_ref, name, what=""):
+    g_gpu = np.asarray(g_gpu, dtype=np.float64)
+    assert np.all(np.isfinite(g_gpu)), f"{what} {name}: non-finite values"
+    if np.linalg.norm(g_ref) < 1e-9:
+        # The exact gradient is zero (T = 1 gives dQ = dK = 0); a relative error is undefined, so bound the
+        # fp32 rounding of dP - Delta that is all the kernels can leave.
+        assert np.abs(g_gpu).max() < 1e-2, f"{what} {name}: expected 0, got max |g| {np.abs(g_gpu).max():.3e}"
+        return
+    rel = np.linalg.norm(g_gpu - g_ref) / np.linalg.norm(g_ref)
+    assert rel <= GRAD_FRO, f"{what} {name}: relative Frobenius error {rel:.3e} > {GRAD_FRO}"
+
+
+def to64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def run_gpu(q, k, v, do, scale):
+    dev = torch.device("cuda")
+    qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, do))
+    o, lse = attn.attn_fwd(qd, kd, vd, scale)
+    dq, dk, dv = attn.attn_bwd(qd, kd, vd, o, lse, dod, scale)
+    torch.cuda.synchronize()
+    assert attn.get_device_error() == 0
+    return o, lse, dq, dk, dv
+
+
+def full_compare(w: Workload):
+    q, k, v, do = make_inputs(w)
+    o, lse, dq, dk, dv = run_gpu(q, k, v, do, w.scale)
+    O_ref, LSE_ref = attn_ref.attention_forward(q, k, v, w.scale)
+    dQ_ref, dK_ref, dV_ref, _ = attn_ref.attention_backward(q, k, v, do, w.scale)
+    what = f"{w.name} B={w.B} H={w.H} T={w.T}"
+    check_o(to64(o), O_ref, what)
+    check_lse(to64(lse), LSE_ref, what)
+    check_grad(to64(dq), dQ_ref, "dQ", what)
+    check_grad(to64(dk), dK_ref, "dK", what)
+    check_grad(to64(dv), dV_ref, "dV", what)
+
+
+def test_tiny_full():
+    full_compare(WORKLOADS["tiny"])
+
+
+# Ragged and edge sizes: T = 1 (O = V), tails inside the first tile, exactly one/two tiles, tails of 1 and
+# 63 rows past a tile boundary, several heads and batches. Each spans the kernels' tiles and tails.
+EDGE_SHAPES = [(1, 1, 1), (1, 1, 7), (2, 3, 64), (1, 2, 100), (1, 1, 128), (1, 2, 129), (2, 1, 191),
+               (1, 1, 256), (1, 2, 383), (3, 2, 513)]
+
+
+@pytest.mark.parametrize("B,H,T", EDGE_SHAPES, ids=[f"B{b}H{h}T{t}" for b, h, t in EDGE_SHAPES])
+def test_edge_shapes_full(B, H, T):
+    full_compare(Workload(f"edge", B=B, H=H, T=T, seed=T))
+
+
+@pytest.mark.parametrize("prescale", [3.0, 6.0])
+def test_peaky_rows_exercise_rescaling(prescale):
+    """Q and K scaled up so softmax rows are peaky and the running max jumps by more than 2^8 within a row:
+    the forward's lazy O rescaling runs, for some rows of a warp and not others."""
+    full_compare(Workload(f"peaky{prescale}", B=1, H=2, T=640, seed=21, qk_prescale=prescale))
+
+
+def test_T1_closed_form():
+    w = Workload("T1", B=2, H=3, T=1, seed=5)
+    q, k, v, do = make_inputs(w)
+    o, lse, dq, dk, dv = run_gpu(q, k, v, do, w.scale)
+    assert torch.equal(o.cpu(), v), "T = 1 must give O = V exactly"
+    assert torch.equal(dv.cpu(), do), "T = 1 must give dV = dO exactly"
+    # dQ = dK = 0 in closed form; the kernels leave only fp32 rounding of dP - Delta (a few 1e-4)
+    assert float(dq.float().abs().max()) < 1e-2 and float(dk.float().abs().max()) < 1e-2
+
+
+FULL = ["d12", "d20", "d24", "d26", "d26_T512", "d26_T1024", "d26_T4096"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled_slices(name):
+    """The benchmark's shapes and launch; the oracle checks seeded (b, h) slices one by one."""
+    w = WORKLOADS[name]
+    q, k, v, do = make_inputs(w)
+    o, lse, dq, dk, dv = run_gpu(q, k, v, do, w.scale)
+    for (b, h) in sample_slices(w, k=3):
+        ref = attn_ref.slice_forward_backward(q, k, v, do, b, h, w.scale)
+        what = f"{name} slice (b={b}, h={h})"
+        check_o(to64(o[b, :, h]), ref["o"], what)
+        check_lse(to64(lse[b, h]), ref["lse"], what)
+        check_grad(to64(dq[b, :, h]), ref["dq"], "dQ", what)
+        check_grad(to64(dk[b, :, h]), ref["dk"], "dK", what)
+        check_grad(to64(dv[b, :, h]), ref["dv"], "dV", what)
+    # Properties that hold at any size: finite everywhere, rows of dK and dV past no query are zero-free...
+    for t in (o, dq, dk, dv):
+        assert bool(torch.isfinite(t.float()).all())
+
+
+def test_causality_on_gpu():
+    """Perturbing q/k/v after position t leaves O and LSE at positions <= t bit-identical."""
+    w = Workload("causal", B=2, H=2, T=300, seed=9)
+    q, k, v, _ = make_inputs(w, need_grad_input=False)
+    dev = torch.device("cuda")
+    o1, l1 = attn.attn_fwd(q.to(dev), k.to(dev), v.to(dev), w.scale)
+    t = 150
+    q2, k2, v2 = q.clone(), k.clone(), v.clone()
+    for x in (q2, k2, v2):
+        x[:, t + 1:] = torch.randn_like(x[:, t + 1:].float()).to(torch.bfloat16) * 3
+    o2, l2 = attn.attn_fwd(q2.to(dev), k2.to(dev), v2.to(dev), w.scale)
+    assert torch.equal(o1[:, :t + 1], o2[:, :t + 1])
+    assert torch.equal(l1[:, :, :t + 1], l2[:, :, :t + 1])
+
+
+def test_key_shift_invariance_d24_recipe():
+    """Adding one vector to every key leaves O unchanged and shifts LSE by scale * q . b (d24's input recipe)."""
+    w = Workload("shift", B=1, H=2, T=512, seed=3)
+    q, k, v, _ = make_inputs(w, need_grad_input=False)
+    bias = torch.randn(w.D, generator=torch.Generator().manual_seed(7))
+    k2 = (k.float() + bias).to(torch.bfloat16)
+    dev = torch.device("cuda")
+    o1, l1 = attn.attn_fwd(q.to(dev), k.to(dev), v.to(dev), w.scale)
+    o2, l2 = attn.attn_fwd(q.to(dev), k2.to(dev), v.to(dev), w.scale)
+    ref_o, ref_l = attn_ref.attention_forward(q, k2, v, w.scale)
+    check_o(to64(o2), ref_o, "shifted keys")
+    check_lse(to64(l2), ref_l, "shifted keys")
+    check_o(to64(o2), to64(o1), "shift invariance")
+
+
+def test_repeated_calls_are_deterministic_forward():
+    w = Workload("det", B=2, H=3, T=777, seed=4)
+    q, k, v, _ = make_inputs(w, need_grad_input=False)
+    dev = torch.device("cuda")
+    a = attn.attn_fwd(q.to(dev), k.to(dev), v.to(dev), w.scale)
+    b = attn.attn_fwd(q.to(dev), k.to(dev), v.to(dev), w.scale)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_autograd_wrapper_matches_oracle():
+    w = Workload("autograd", B=1, H=2, T=200, seed=12)
+    q, k, v, do = make_inputs(w)
+    dev = torch.device("cuda")
+    qd, kd, vd = (x.to(dev).requires_grad_() for x in (q, k, v))
+    out = attn.causal_attention(qd, kd, vd)
+    out.backward(do.to(dev))
+    dQ_ref, dK_ref, dV_ref, _ = attn_ref.attention_backward(q, k, v, do, w.scale)
+    check_grad(to64(qd.grad), dQ_ref, "dQ")
+    check_grad(to64(kd.grad), dK_ref, "dK")
+    check_grad(to64(vd.grad), dV_ref, "dV")
+
+
+def test_argument_errors_on_gpu():
+    dev = torch.device("cuda")
+    q = torch.zeros(1, 64, 1, 128, dtype=torch.bfloat16, device=dev)
+    lib = attn.load_library()
+    lse = torch.empty(1, 1, 64, device=dev)
+    o = torch.empty_like(q)
+    # misaligned output pointer
+    assert lib.attn_fwd(q.data_ptr(), q.data_ptr(), q.data_ptr(), o.data_ptr() + 2, lse.data_ptr(), 1, 1, 64, 128,
+                        0.1, None) == 3
+    ws = torch.empty(attn.attn_bwd_workspace_bytes(1, 1, 64, 128) - 256, dtype=torch.uint8, device=dev)
+    with pytest.raises(attn.AttnError):
+        attn.attn_bwd(q, q, q, q, lse, q, 0.1, workspace=ws)
+
+
+def test_bounded_wait_reports_timeout():
+    """A kernel that waits on a barrier nothing completes gives up after its limit and reports the site."""
+    attn.clear_device_error()
+    attn.selftest_wait_timeout(2_000_000)  # 2 ms
+    torch.cuda.synchronize()
+    word = attn.get_device_error()
+    assert word == (0x7F << 8) | 1
+    attn.clear_device_error()
+    assert attn.get_device_error() == 0
+    # the context is still usable afterwards
+    test_tiny_full()
