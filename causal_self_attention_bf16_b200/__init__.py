@@ -37,6 +37,7 @@ SIGNATURES = {
     "attn_bwd_preprocess": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _F, _VP], _I),
     "attn_bwd_dkdv": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _F, _VP], _I),
     "attn_bwd_dq_convert": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _F, _VP], _I),
+    "attn_bwd_noalloc": ([_VP] * 9 + [_I, _I, _I, _I, _F, _VP], _I),
     "attn_get_device_error": ([ctypes.POINTER(ctypes.c_uint32)], _I),
     "attn_clear_device_error": ([], _I),
     "attn_set_wait_limit_ns": ([_U64], _I),
@@ -156,6 +157,28 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
                       workspace.numel() * workspace.element_size(), B, H, T, D, scale,
                       _stream_handle(stream, q.device))
     _check("attn_bwd", st)
+    return dq, dk, dv
+
+
+def attn_bwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+                     dO: torch.Tensor, scale: Optional[float] = None, dq: Optional[torch.Tensor] = None,
+                     dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
+                     stream: Optional[torch.cuda.Stream] = None):
+    """Backward using the library's built-in scratch array instead of a caller workspace (for callers that
+    cannot allocate device memory; sizes up to B*H*roundup(T,128) <= 64512). Returns (dq, dk, dv)."""
+    lib = load_library()
+    _check_qkv("q", q)
+    B, T, H, D = q.shape
+    for name, t in (("k", k), ("v", v), ("o", o), ("dO", dO)):
+        _check_qkv(name, t, q.shape)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    scale = default_scale(D) if scale is None else float(scale)
+    st = lib.attn_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                              dO.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, T, D, scale,
+                              _stream_handle(stream, q.device))
+    _check("attn_bwd_noalloc", st)
     return dq, dk, dv
 
 

@@ -345,4 +345,63 @@ attn_status attn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
   return ATTN_OK;
 }
 
+// ---------------------------------------------------------------------------------------------- no-alloc bwd
+//
+// Backward for callers that cannot allocate device memory: code running inside a framework's custom-op or
+// plugin interface that hands over tensors but offers no allocator and no workspace, and code working under
+// a fixed memory plan that forbids allocation (and the device-wide synchronisation cudaMalloc/cudaFree can
+// bring) during a step. The scratch space attn_bwd takes from its caller lives instead in the file-scope
+// device array below, which every GPU that loads this library holds until the process exits.
+
+}  // extern "C"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 32ull << 20;  // 32 MiB: B * H * roundup(T, 128) <= 64512 rows
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch, looked up once per device with that device current. In host code the
+// array's name is only a host-side stand-in, never a device address, so kernels get this pointer instead.
+attn_status noalloc_scratch_ptr(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    if ((e = cudaSetDevice(dev)) != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_noalloc_scratch)) != cudaSuccess)
+      return cuda_fail(e, "cudaGetSymbolAddress(g_noalloc_scratch)");
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                             const void* dO, void* dq, void* dk, void* dv, int B, int H, int T, int D, float scale,
+                             void* stream) {
+  attn_status st = check_sizes(B, H, T, D, scale);
+  if (st != ATTN_OK) return st;
+  const size_t need = workspace_layout(B, H, T).total;
+  if (need > kNoAllocScratchBytes) {
+    std::snprintf(g_cuda_error, sizeof(g_cuda_error),
+                  "attn_bwd_noalloc: these sizes need %zu bytes of scratch, the built-in array holds %zu", need,
+                  kNoAllocScratchBytes);
+    return ATTN_ERR_WORKSPACE;
+  }
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch_ptr(&scratch)) != ATTN_OK) return st;
+  // Same three kernels as attn_bwd; the preprocess kernel rewrites every scratch byte the later kernels read
+  // (including zeroing the dQ accumulator), so whatever an earlier call left there does not matter.
+  return bwd_launch(7u, q, k, v, o, lse, dO, dq, dk, dv, scratch, kNoAllocScratchBytes, B, H, T, D, scale, stream);
+}
+
 }  // extern "C"

@@ -103,6 +103,24 @@ attn_status attn_bwd_dq_convert(const void* q, const void* k, const void* v, con
                                 size_t workspace_bytes, int B, int H, int T, int D, float scale, void* stream);
 
 /*
+ * Backward without caller-provided workspace, for callers that cannot allocate device memory (a custom-op or
+ * plugin interface that passes tensors but no allocator or workspace; a fixed memory plan that forbids
+ * cudaMalloc/cudaFree, and the synchronisation they can cause, during a step). The pages have no counterpart:
+ * this is an addition of this library. Arguments and results are those of attn_bwd minus the workspace.
+ *   - Scratch: a 32 MiB array inside the library (held by every GPU that loads it, until the process exits),
+ *     enough for B * H * roundup(T, 128) <= 64512; larger sizes return ATTN_ERR_WORKSPACE and launch nothing.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on each device looks the array's device address up (cudaGetSymbolAddress, with that
+ *     device current); make that first call before any stream capture.
+ *   - All calls share the one array, which keeps the last call's contents; each call rewrites everything it
+ *     reads from it (the dQ accumulator is zeroed first). Calls that overlap in time on the GPU (different
+ *     streams, or different host threads on one device) race on the array and give wrong results.
+ */
+attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                             const void* dO, void* dq, void* dk, void* dv, int B, int H, int T, int D,
+                             float scale, void* stream);
+
+/*
  * Device-side error word shared by the kernels of this library on the current device: 0 if no kernel has
  * given up on a bounded wait since the last clear; otherwise (site << 8) | 1. Synchronises the device.
  * Returns ATTN_ERR_TIMEOUT if the word is non-zero, ATTN_OK if it is zero, ATTN_ERR_CUDA on a CUDA error.
