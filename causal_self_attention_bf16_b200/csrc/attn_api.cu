@@ -337,6 +337,20 @@ attn_status attn_clear_device_error(void) {
   return ATTN_OK;
 }
 
+#ifdef ATTN_TRACE
+// Profiling builds only (-DATTN_TRACE): copy the pipeline trace of the last launch to host memory.
+int attn_trace_dump(void* dst, size_t bytes) {
+  if (bytes < attn::kTraceBytes) return -1;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(dst, attn::g_trace, attn::kTraceBytes);
+  if (e == cudaSuccess) {
+    static unsigned long long zeros[attn::kTraceBytes / 8];
+    e = cudaMemcpyToSymbol(attn::g_trace, zeros, attn::kTraceBytes);
+  }
+  return e == cudaSuccess ? 0 : -1;
+}
+#endif
+
 attn_status attn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
   if (limit_ns < 1000 || limit_ns > 10ull * 1000 * 1000 * 1000) return ATTN_ERR_INVALID_ARG;
   wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);

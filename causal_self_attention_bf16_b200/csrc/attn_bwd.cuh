@@ -13,16 +13,17 @@
 //        S^T = K Q^T, dP^T = V dO^T            (K-major operands in shared memory)
 //        dV += P^T dO, dK += dS^T Q             (P^T, dS^T from tensor memory; dO, Q MN-major)
 //        dQ^T = K^T dS^T                        (both operands MN-major in shared memory)
-//      One thread per key row turns S^T, dP^T into P^T, dS^T (exp2 against the stored LSE); a second warp
-//      group reads dQ^T out of tensor memory and adds it into the fp32 accumulator with 16-byte vector
-//      reductions laid out so that each warp instruction covers 512 contiguous bytes. dK, dV stay in tensor
-//      memory for the whole walk and leave through a TMA store.
+//      Two warp groups taking alternate query tiles (one thread per key row) turn S^T, dP^T into P^T, dS^T
+//      (exp2 against the stored LSE); a third warp group stages dQ^T in shared memory in the accumulator's
+//      layout and adds each 64-query tile (32 contiguous KB) into the fp32 accumulator with one bulk
+//      reduction (cp.reduce.async.bulk .add.f32) on the async engine. dK, dV stay in tensor memory for the
+//      whole walk and leave through a TMA store.
 //   3. attn_bwd_dq_kernel: dQ = bf16(scale * accumulator) back in [B, T, H, D].
 //
 // Tensor memory of the dK/dV kernel (512 columns): dV [0,128), dK [128,256), and two 128-column tile
 // buffers R0 = [256,384), R1 = [384,512). A buffer holds S^T in its first 64 columns and dP^T in the last
-// 64; after the softmax step its first 32 columns hold P^T and the next 32 dS^T (bf16 pairs), and the dQ^T
-// MMA writes its last 64 columns.
+// 64; after the softmax step, for each half h of the 64 queries, columns [32h, 32h+16) hold P^T and
+// [32h+16, 32h+32) hold dS^T (bf16 pairs) of those 32 queries, and the dQ^T MMA writes the last 64 columns.
 #pragma once
 #include "attn_common.cuh"
 #include "sm100.cuh"
@@ -32,17 +33,17 @@ namespace attn {
 constexpr int kBwdQTile = 64;       // queries per inner tile
 constexpr int kBwdKTile = 128;      // keys per CTA
 constexpr int kBwdStages = 3;       // Q/dO/LSE/Delta ring depth
-constexpr int kBwdThreads = 320;    // warp 0 TMA, warp 1 MMA, warps 2..5 softmax, warps 6..9 dQ
+constexpr int kBwdThreads = 448;    // warp 0 TMA, warp 1 MMA, warps 2..9 softmax, warps 10..13 dQ
 
 constexpr uint32_t kBwdSmemK = 0;                                 // 32 KB
 constexpr uint32_t kBwdSmemV = 32768;                             // 32 KB
 constexpr uint32_t kBwdSmemQ = 65536;                             // 3 x 16 KB (two 8 KB boxes each)
 constexpr uint32_t kBwdSmemDO = kBwdSmemQ + kBwdStages * 16384;   // 3 x 16 KB
 constexpr uint32_t kBwdSmemDS = kBwdSmemDO + kBwdStages * 16384;  // 2 x 16 KB: dS^T [128 keys][64 q]
-constexpr uint32_t kBwdSmemLse = kBwdSmemDS + 2 * 16384;          // 3 x 256 B
+constexpr uint32_t kBwdSmemDQ = kBwdSmemDS + 2 * 16384;           // 32 KB: dQ^T tile staged for the bulk reduce
+constexpr uint32_t kBwdSmemLse = kBwdSmemDQ + 32768;              // 3 x 256 B
 constexpr uint32_t kBwdSmemDelta = kBwdSmemLse + kBwdStages * 256;  // 3 x 256 B
-constexpr uint32_t kBwdSmemBytes = kBwdSmemDelta + kBwdStages * 256;
-constexpr uint32_t kBwdSmemAlloc = kBwdSmemBytes + 1024;
+constexpr uint32_t kBwdSmemBytes = kBwdSmemDelta + kBwdStages * 256;  // barriers follow (see BwdBarriers)
 
 constexpr uint32_t kTmemDV = 0, kTmemDK = 128, kTmemR = 256;
 
@@ -144,22 +145,23 @@ struct BwdBarriers {
   uint64_t p_full[2];    // P^T, dS^T written (TMEM + smem)
   uint64_t dq_full[2];   // dQ^T of buffer b ready (also: dV, dK MMAs of that tile done)
   uint64_t dq_empty[2];  // dQ^T read out: buffer b free
+  uint64_t b_done[2];    // dV, dK MMAs of the tile in buffer b done (buffer's P^T, dS^T consumed)
   uint64_t acc_done;     // all MMAs done (epilogue)
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
+// The kernel uses no static shared memory, so the dynamic block starts 1024-byte aligned and needs no slack
+// (the kernel checks this and refuses to run otherwise): tiles, then the barriers. 226 KB in all.
+constexpr uint32_t kBwdSmemAlloc = kBwdSmemBytes + sizeof(BwdBarriers);
+static_assert(kBwdSmemAlloc <= 232448, "dK/dV kernel exceeds the 227 KB shared-memory opt-in");
 
 enum : uint32_t {
-  kSiteBwdProdQEmpty = 0x41, kSiteBwdMmaKV = 0x51, kSiteBwdMmaQ = 0x52, kSiteBwdMmaDqEmpty = 0x53,
+  kSiteBwdLayout = 0x40, kSiteBwdProdQEmpty = 0x41, kSiteBwdMmaKV = 0x51, kSiteBwdMmaQ = 0x52, kSiteBwdMmaDqEmpty = 0x53,
   kSiteBwdMmaP = 0x54, kSiteBwdSmS = 0x61, kSiteBwdSmQ = 0x62, kSiteBwdSmEpi = 0x63, kSiteBwdDq = 0x71,
   kSiteBwdDrain = 0x72
 };
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
 
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -168,13 +170,21 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                      const BwdParams p) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ BwdBarriers bars;
+  // 1024-byte aligned base for the 128-byte-swizzle tiles. Offsetting the array itself (not a round trip
+  // through an integer) keeps the pointer in the shared address space, so accesses compile to LDS/STS.
+  uint8_t* smem = smem_raw;
+  if (smem_u32(smem_raw) & 1023u) {  // the layout below needs a 1024-byte aligned dynamic block
+    if (threadIdx.x == 0) atomicOr(&g_device_error, sm100::DEV_ERR_TIMEOUT | (kSiteBwdLayout << 8));
+    return;
+  }
+  BwdBarriers& bars = *reinterpret_cast<BwdBarriers*>(smem + kBwdSmemBytes);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int BH = p.B * p.H;
-  const int kt = static_cast<int>(blockIdx.x / BH);  // key tile; low tiles (most query tiles) first
-  const int bh = static_cast<int>(blockIdx.x % BH);
+  // Head-major order, heaviest key tile (the first, seen by every query tile) first within a head: the CTAs in
+  // flight cover only ~10 heads, so their Q, dO and the head's fp32 dQ accumulator stay in L2.
+  const int n_kt = (p.T + kBwdKTile - 1) / kBwdKTile;
+  const int bh = static_cast<int>(blockIdx.x / n_kt);
+  const int kt = static_cast<int>(blockIdx.x % n_kt);
   const int b = bh / p.H, h = bh % p.H;
   const int k0 = kt * kBwdKTile;
   const int n_q64 = (p.T + kBwdQTile - 1) / kBwdQTile;
@@ -193,6 +203,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       mbar_init(&bars.p_full[s], 128);
       mbar_init(&bars.dq_full[s], 1);
       mbar_init(&bars.dq_empty[s], 128);
+      mbar_init(&bars.b_done[s], 1);
     }
     mbar_init(&bars.acc_done, 1);
     mbar_init(&bars.drain, 1);
@@ -207,10 +218,14 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
+  if (threadIdx.x == 0) ATTN_TRACE_EVENT(0, 0);
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // The whole warp walks the loop (warp-uniform control flow, so addresses and coordinates stay in uniform
+    // registers); one lane, elected once, issues every copy.
+    const bool leader = elect_one();
+    if (leader) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
       mbar_arrive_expect_tx(&bars.kv_full, 4 * 16384);
@@ -218,13 +233,16 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         tma_load_4d(smem + kBwdSmemK + c * 16384, &tm_k, &bars.kv_full, c * 64, h, k0, b);
         tma_load_4d(smem + kBwdSmemV + c * 16384, &tm_v, &bars.kv_full, c * 64, h, k0, b);
       }
-      int last_issued[kBwdStages] = {-1, -1, -1};
-      for (int i = 0; i < n; ++i) {
-        const int s = i % kBwdStages;
-        if (i >= kBwdStages && !mbar_wait(&bars.q_empty[s], ((i - kBwdStages) / kBwdStages) & 1, abort,
-                                          p.timeout_ns, &g_device_error, kSiteBwdProdQEmpty))
-          break;
-        const int q0 = (i0 + i) * kBwdQTile;
+    }
+    int last_issued[kBwdStages];
+    for (int s = 0; s < kBwdStages; ++s) last_issued[s] = -1;
+    for (int i = 0; i < n; ++i) {
+      const int s = i % kBwdStages;
+      if (i >= kBwdStages && !mbar_wait_warp(&bars.q_empty[s], ((i - kBwdStages) / kBwdStages) & 1, abort,
+                                             p.timeout_ns, &g_device_error, kSiteBwdProdQEmpty))
+        break;
+      const int q0 = (i0 + i) * kBwdQTile;
+      if (leader) {
         mbar_arrive_expect_tx(&bars.q_full[s], 2 * 16384 + 2 * 256);
         for (int c = 0; c < 2; ++c) {
           tma_load_4d(smem + kBwdSmemQ + s * 16384 + c * 8192, &tm_q, &bars.q_full[s], c * 64, h, q0, b);
@@ -232,95 +250,123 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         bulk_load(smem + kBwdSmemLse + s * 256, p.lse2 + static_cast<size_t>(bh) * p.Tp + q0, 256, &bars.q_full[s]);
         bulk_load(smem + kBwdSmemDelta + s * 256, p.delta + static_cast<size_t>(bh) * p.Tp + q0, 256, &bars.q_full[s]);
-        last_issued[s] = i;
+        ATTN_TRACE_EVENT(1, i);
       }
-      if (*abort) {
-        volatile int no_abort = 0;
-        mbar_wait(&bars.kv_full, 0, &no_abort, p.timeout_ns, &g_device_error, kSiteBwdDrain);
-        for (int s = 0; s < kBwdStages; ++s)
-          if (last_issued[s] >= 0)
-            mbar_wait(&bars.q_full[s], (last_issued[s] / kBwdStages) & 1, &no_abort, p.timeout_ns, &g_device_error,
-                      kSiteBwdDrain);
-      }
+      last_issued[s] = i;
+    }
+    if (*abort) {
+      volatile int no_abort = 0;
+      mbar_wait(&bars.kv_full, 0, &no_abort, p.timeout_ns, &g_device_error, kSiteBwdDrain);
+      for (int s = 0; s < kBwdStages; ++s)
+        if (last_issued[s] >= 0)
+          mbar_wait(&bars.q_full[s], (last_issued[s] / kBwdStages) & 1, &no_abort, p.timeout_ns, &g_device_error,
+                    kSiteBwdDrain);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t id_s = idesc_bf16_f32(128, 64, false, false);   // K x Q^T, V x dO^T
-      const uint32_t id_acc = idesc_bf16_f32(128, 128, false, true); // P^T (TMEM) x dO, dS^T (TMEM) x Q
-      const uint32_t id_dq = idesc_bf16_f32(128, 64, true, true);    // K^T (MN-major) x dS^T (MN-major)
-      const uint32_t sk = smem_u32(smem + kBwdSmemK), sv = smem_u32(smem + kBwdSmemV);
-      bool ok = mbar_wait(&bars.kv_full, 0, abort, p.timeout_ns, &g_device_error, kSiteBwdMmaKV);
+    // The whole warp walks the schedule and computes the descriptors (warp-uniform, so they live in uniform
+    // registers); the lane elected once issues every tcgen05.mma and tcgen05.commit (a commit tracks the
+    // MMAs of the thread that issues it, so it must be the same lane throughout).
+    const bool leader = elect_one();
+    const uint32_t id_s = idesc_bf16_f32(128, 64, false, false);   // K x Q^T, V x dO^T
+    const uint32_t id_acc = idesc_bf16_f32(128, 128, false, true); // P^T (TMEM) x dO, dS^T (TMEM) x Q
+    const uint32_t id_dq = idesc_bf16_f32(128, 64, true, true);    // K^T (MN-major) x dS^T (MN-major)
+    // Shared-memory descriptors are built once per operand and advanced by adding the byte offset in
+    // 16-byte units to the start-address field (a K step is one 64-bit add; tiles stay below 256 KB).
+    const uint64_t dk_kmaj = sdesc_sw128(smem_u32(smem + kBwdSmemK), 16, 1024);      // K as K-major A
+    const uint64_t dv_kmaj = sdesc_sw128(smem_u32(smem + kBwdSmemV), 16, 1024);      // V as K-major A
+    const uint64_t dk_mnmaj = sdesc_sw128(smem_u32(smem + kBwdSmemK), 16384, 1024);  // K^T as MN-major A
+    bool ok = mbar_wait_warp(&bars.kv_full, 0, abort, p.timeout_ns, &g_device_error, kSiteBwdMmaKV);
+    tc_fence_after();
+    // A(i): S^T and dP^T of query tile i into buffer i%2, once its Q/dO tile has landed and the buffer is free
+    // (dQ^T of tile i-2 read out, and its dV/dK MMAs, which read P^T/dS^T from the buffer, complete).
+    auto issue_a = [&](int i) -> bool {
+      const int s = i % kBwdStages, rb = i & 1;
+      if (!mbar_wait_warp(&bars.q_full[s], (i / kBwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdMmaQ))
+        return false;
+      if (i >= 2 && (!mbar_wait_warp(&bars.dq_empty[rb], ((i - 2) >> 1) & 1, abort, p.timeout_ns, &g_device_error,
+                                     kSiteBwdMmaDqEmpty) ||
+                     !mbar_wait_warp(&bars.b_done[rb], ((i - 2) >> 1) & 1, abort, p.timeout_ns, &g_device_error,
+                                     kSiteBwdMmaDqEmpty)))
+        return false;
+      if (leader) ATTN_TRACE_EVENT(12, i);
       tc_fence_after();
-      // A(i): S^T and dP^T of query tile i into buffer i%2.
-      auto issue_a = [&](int i) -> bool {
-        const int s = i % kBwdStages, rb = i & 1;
-        if (!mbar_wait(&bars.q_full[s], (i / kBwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdMmaQ))
-          return false;
-        if (i >= 2 && !mbar_wait(&bars.dq_empty[rb], ((i - 2) >> 1) & 1, abort, p.timeout_ns, &g_device_error,
-                                 kSiteBwdMmaDqEmpty))
-          return false;
-        tc_fence_after();
-        const uint32_t sq = smem_u32(smem + kBwdSmemQ + s * 16384), sdo = smem_u32(smem + kBwdSmemDO + s * 16384);
-        const uint32_t r = tmem + kTmemR + rb * 128;
+      const uint64_t dq0 = sdesc_sw128(smem_u32(smem + kBwdSmemQ + s * 16384), 16, 1024);
+      const uint64_t ddo0 = sdesc_sw128(smem_u32(smem + kBwdSmemDO + s * 16384), 16, 1024);
+      const uint32_t r = tmem + kTmemR + rb * 128;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32;  // 128-row boxes
-          const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;   // 64-row boxes
-          mma_ss(r, sdesc_sw128(sk + ka, 16, 1024), sdesc_sw128(sq + kb, 16, 1024), id_s, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;
-          mma_ss(r + 64, sdesc_sw128(sv + ka, 16, 1024), sdesc_sw128(sdo + kb, 16, 1024), id_s, kk > 0);
-        }
-        mma_commit(&bars.s_full[rb]);
-        return true;
-      };
-      // B(i): dV += P^T dO, dK += dS^T Q, dQ^T = K^T dS^T.
-      auto issue_b = [&](int i) -> bool {
-        const int s = i % kBwdStages, rb = i & 1;
-        if (!mbar_wait(&bars.p_full[rb], (i >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdMmaP))
-          return false;
-        tc_fence_after();
-        const uint32_t sq = smem_u32(smem + kBwdSmemQ + s * 16384), sdo = smem_u32(smem + kBwdSmemDO + s * 16384);
-        const uint32_t sds = smem_u32(smem + kBwdSmemDS + rb * 16384);
-        const uint32_t r = tmem + kTmemR + rb * 128;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + kTmemDV, r + kk * 8, sdesc_sw128(sdo + kk * 2048, 8192, 1024), id_acc, (i > 0 || kk > 0));
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(tmem + kTmemDK, r + 32 + kk * 8, sdesc_sw128(sq + kk * 2048, 8192, 1024), id_acc, (i > 0 || kk > 0));
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(r + 64, sdesc_sw128(sk + kk * 2048, 16384, 1024), sdesc_sw128(sds + kk * 2048, 8192, 1024), id_dq,
-                 kk > 0);
-        mma_commit(&bars.dq_full[rb]);
-        mma_commit(&bars.q_empty[s]);
-        return true;
-      };
-      // Pairs: A(i), A(i+1), B(i), B(i+1): the dQ read-out of one tile overlaps the MMAs of the next.
-      for (int i = 0; ok && i < n; i += 2) {
-        ok = issue_a(i) && (i + 1 >= n || issue_a(i + 1));
-        ok = ok && issue_b(i) && (i + 1 >= n || issue_b(i + 1));
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t ka = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;  // 128-row boxes, in 16-byte units
+        const uint32_t kb = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;   // 64-row boxes
+        if (leader) mma_ss(r, dk_kmaj + ka, dq0 + kb, id_s, kk > 0);
       }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t ka = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+        const uint32_t kb = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+        if (leader) mma_ss(r + 64, dv_kmaj + ka, ddo0 + kb, id_s, kk > 0);
+      }
+      if (leader) {
+        mma_commit(&bars.s_full[rb]);
+        ATTN_TRACE_EVENT(2, i);
+      }
+      return true;
+    };
+    // B(i): dQ^T = K^T dS^T first (its own commit, so the read-out of dQ^T overlaps the rest), then
+    // dV += P^T dO and dK += dS^T Q (commit: the tile's buffer and its Q/dO ring slot are free).
+    auto issue_b = [&](int i) -> bool {
+      const int s = i % kBwdStages, rb = i & 1;
+      if (!mbar_wait_warp(&bars.p_full[rb], (i >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdMmaP))
+        return false;
+      tc_fence_after();
+      const uint64_t dq_mn = sdesc_sw128(smem_u32(smem + kBwdSmemQ + s * 16384), 8192, 1024);
+      const uint64_t ddo_mn = sdesc_sw128(smem_u32(smem + kBwdSmemDO + s * 16384), 8192, 1024);
+      const uint64_t dds_mn = sdesc_sw128(smem_u32(smem + kBwdSmemDS + rb * 16384), 8192, 1024);
+      const uint32_t r = tmem + kTmemR + rb * 128;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        if (leader) mma_ss(r + 64, dk_mnmaj + kk * 128, dds_mn + kk * 128, id_dq, kk > 0);
+      if (leader) mma_commit(&bars.dq_full[rb]);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        if (leader) mma_ts(tmem + kTmemDV, r + (kk >> 1) * 32 + (kk & 1) * 8, ddo_mn + kk * 128, id_acc, (i > 0 || kk > 0));
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        if (leader) mma_ts(tmem + kTmemDK, r + (kk >> 1) * 32 + 16 + (kk & 1) * 8, dq_mn + kk * 128, id_acc, (i > 0 || kk > 0));
+      if (leader) {
+        mma_commit(&bars.b_done[rb]);
+        mma_commit(&bars.q_empty[s]);
+        ATTN_TRACE_EVENT(3, i);
+      }
+      return true;
+    };
+    // Pairs: A(i), A(i+1), B(i), B(i+1). The two softmax groups work on tiles i and i+1 at the same time,
+    // and the dQ^T read-out of a pair overlaps the next pair's first MMAs.
+    for (int i = 0; ok && i < n; i += 2) {
+      ok = issue_a(i) && (i + 1 >= n || issue_a(i + 1));
+      ok = ok && issue_b(i) && (i + 1 >= n || issue_b(i + 1));
+    }
+    if (leader) {
       mma_commit(&bars.acc_done);
       mma_commit(&bars.drain);
-      volatile int no_abort = 0;
-      mbar_wait(&bars.drain, 0, &no_abort, p.timeout_ns, &g_device_error, kSiteBwdDrain);
     }
-  } else if (warp < 6) {
-    // ------------------------------------------------------------------ softmax: one thread per key row
+    volatile int no_abort = 0;
+    mbar_wait(&bars.drain, 0, &no_abort, p.timeout_ns, &g_device_error, kSiteBwdDrain);
+  } else if (warp < 10) {
+    // ------------------------------------------------------------------ softmax: one thread per (key row, half)
+    // Two warp groups alternate tiles (ping-pong): group g (warps 2..5 or 6..9) handles the query tiles with
+    // i % 2 == g, which are exactly the tiles of tensor-memory buffer g, so each group has two tiles of
+    // tensor-core work to hide its softmax behind. A thread handles one key row, in two halves of 32 query
+    // columns; each half's packed P^T and dS^T (16 + 16 columns) go over that half's own 32 columns of S^T.
+    const int g = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int krow = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int kg = k0 + krow;
     const float c = p.scale_log2;
     bool ok = true;
-    for (int i = 0; i < n; ++i) {
-      const int s = i % kBwdStages, rb = i & 1;
+    for (int i = g; i < n; i += 2) {
+      const int s = i % kBwdStages, rb = g;
       const int q0 = (i0 + i) * kBwdQTile;
       if (!mbar_wait_warp(&bars.q_full[s], (i / kBwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdSmQ) ||
           !mbar_wait_warp(&bars.s_full[rb], (i >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdSmS)) {
@@ -328,124 +374,133 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         break;
       }
       tc_fence_after();
-      const uint32_t r = tmem + lane_base + kTmemR + rb * 128;
-      const float* lse2 = reinterpret_cast<const float*>(smem + kBwdSmemLse + s * 256);
-      const float* dlt = reinterpret_cast<const float*>(smem + kBwdSmemDelta + s * 256);
-      float pr[64];
-      {
-        uint32_t a[32], bb[32];
-        tmem_ld32(r + 0, a);
-        tmem_ld32(r + 32, bb);
-        tmem_wait_ld();
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          pr[q] = ex2(fmaf(__uint_as_float(a[q]), c, -lse2[q]));
-          pr[32 + q] = ex2(fmaf(__uint_as_float(bb[q]), c, -lse2[32 + q]));
-        }
-      }
-      if (q0 < k0 + kBwdKTile) {  // query tile overlaps the key tile: queries before a key see nothing
-#pragma unroll
-        for (int q = 0; q < 64; ++q)
-          if (q0 + q < kg) pr[q] = 0.f;
-      }
+      if (threadIdx.x == 64 || threadIdx.x == 192) ATTN_TRACE_EVENT(4, i);
+      const bool diag = q0 < k0 + kBwdKTile;  // tile overlaps the key tile: queries before a key see nothing
       uint8_t* dsrow = smem + kBwdSmemDS + rb * 16384;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t dp[32];
-        tmem_ld32(r + 64 + hh * 32, dp);
+#pragma unroll 1
+      for (int hh = 0; hh < 2; ++hh) {  // one half at a time keeps the live registers to one half's worth
+        const uint32_t r = tmem + lane_base + kTmemR + rb * 128 + 32 * hh;
+        const float4* lse4 = reinterpret_cast<const float4*>(smem + kBwdSmemLse + s * 256) + 8 * hh;
+        const float4* dlt4 = reinterpret_cast<const float4*>(smem + kBwdSmemDelta + s * 256) + 8 * hh;
+        uint32_t sv[32], dp[32];
+        tmem_ld32(r, sv);        // S^T of queries [32hh, 32hh+32)
+        tmem_ld32(r + 64, dp);   // dP^T of the same queries
         tmem_wait_ld();
         uint32_t ppk[16], dpk[16];
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const int qa = hh * 32 + 2 * q, qb = qa + 1;
-          const float ds0 = pr[qa] * (__uint_as_float(dp[2 * q]) - dlt[qa]);
-          const float ds1 = pr[qb] * (__uint_as_float(dp[2 * q + 1]) - dlt[qb]);
-          ppk[q] = pack_bf16x2(pr[qa], pr[qb]);
-          dpk[q] = pack_bf16x2(ds0, ds1);
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 l4 = lse4[q4], d4 = dlt4[q4];
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pv[4], dsv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int q = q4 * 4 + e;
+            float pe = ex2(fmaf(__uint_as_float(sv[q]), c, -lv[e]));
+            if (diag && q0 + 32 * hh + q < kg) pe = 0.f;
+            pv[e] = pe;
+            dsv[e] = pe * (__uint_as_float(dp[q]) - dv4[e]);
+          }
+          ppk[q4 * 2] = pack_bf16x2(pv[0], pv[1]);
+          ppk[q4 * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+          dpk[q4 * 2] = pack_bf16x2(dsv[0], dsv[1]);
+          dpk[q4 * 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
         }
-        tmem_st16(r + hh * 16, ppk);
-        tmem_st16(r + 32 + hh * 16, dpk);
+        tmem_st16(r, ppk);        // P^T  of these 32 queries: columns [32hh, 32hh+16)
+        tmem_st16(r + 16, dpk);   // dS^T of these 32 queries: columns [32hh+16, 32hh+32)
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           uint4 v = make_uint4(dpk[ch * 4 + 0], dpk[ch * 4 + 1], dpk[ch * 4 + 2], dpk[ch * 4 + 3]);
-          *reinterpret_cast<uint4*>(dsrow + sw128_offset(krow, hh * 4 + ch)) = v;
+          *reinterpret_cast<uint4*>(dsrow + sw128_offset(krow, 4 * hh + ch)) = v;
         }
       }
       tmem_wait_st();
       fence_async_shared();
       tc_fence_before();
       mbar_arrive(&bars.p_full[rb]);
+      if (threadIdx.x == 64 || threadIdx.x == 192) ATTN_TRACE_EVENT(5, i);
     }
-    // Epilogue: dV and scale*dK from TMEM -> bf16 -> swizzled staging -> TMA store (rows past T are clipped).
-    // Every thread of the group reaches the named barrier, failed or not; the stores are skipped on abort.
+    // Epilogue: group 0 writes dV, group 1 writes scale*dK: TMEM -> bf16 -> swizzled staging -> TMA store
+    // (rows past T are clipped). Both groups reach the named barrier, failed or not; no store on abort.
     const bool epi_ok = __all_sync(0xffffffffu, ok) &&
                         mbar_wait_warp(&bars.acc_done, 0, abort, p.timeout_ns, &g_device_error, kSiteBwdSmEpi);
+    uint8_t* stage = smem + (g == 0 ? kBwdSmemQ : kBwdSmemDO);  // 32 KB each (first two ring slots)
     if (epi_ok) {
       tc_fence_after();
+      const float mul = g == 0 ? 1.0f : p.scale;
+      const uint32_t col = g == 0 ? kTmemDV : kTmemDK;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        uint8_t* stage = smem + (which == 0 ? kBwdSmemQ : kBwdSmemDO);  // 32 KB each (first two stages)
-        const float mul = which == 0 ? 1.0f : p.scale;
-        const uint32_t col = which == 0 ? kTmemDV : kTmemDK;
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_base + col + cc * 32, o);
+        tmem_wait_ld();
+        uint8_t* box = stage + (cc >> 1) * 16384;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_base + col + cc * 32, o);
-          tmem_wait_ld();
-          uint8_t* box = stage + (cc >> 1) * 16384;
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(o[ch * 8 + 0]) * mul, __uint_as_float(o[ch * 8 + 1]) * mul);
-            v.y = pack_bf16x2(__uint_as_float(o[ch * 8 + 2]) * mul, __uint_as_float(o[ch * 8 + 3]) * mul);
-            v.z = pack_bf16x2(__uint_as_float(o[ch * 8 + 4]) * mul, __uint_as_float(o[ch * 8 + 5]) * mul);
-            v.w = pack_bf16x2(__uint_as_float(o[ch * 8 + 6]) * mul, __uint_as_float(o[ch * 8 + 7]) * mul);
-            *reinterpret_cast<uint4*>(box + sw128_offset(krow, (cc & 1) * 4 + ch)) = v;
-          }
+        for (int ch = 0; ch < 4; ++ch) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(o[ch * 8 + 0]) * mul, __uint_as_float(o[ch * 8 + 1]) * mul);
+          v.y = pack_bf16x2(__uint_as_float(o[ch * 8 + 2]) * mul, __uint_as_float(o[ch * 8 + 3]) * mul);
+          v.z = pack_bf16x2(__uint_as_float(o[ch * 8 + 4]) * mul, __uint_as_float(o[ch * 8 + 5]) * mul);
+          v.w = pack_bf16x2(__uint_as_float(o[ch * 8 + 6]) * mul, __uint_as_float(o[ch * 8 + 7]) * mul);
+          *reinterpret_cast<uint4*>(box + sw128_offset(krow, (cc & 1) * 4 + ch)) = v;
         }
       }
     }
     fence_async_shared();
-    named_barrier(1, 128);
-    if (warp == 2 && lane == 0 && !*abort) {
-      for (int cc = 0; cc < 2; ++cc) {
-        tma_store_4d(&tm_dv, smem + kBwdSmemQ + cc * 16384, cc * 64, h, k0, b);
-        tma_store_4d(&tm_dk, smem + kBwdSmemDO + cc * 16384, cc * 64, h, k0, b);
-      }
+    named_barrier(1, 256);
+    if ((warp == 2 || warp == 6) && lane == 0 && !*abort) {
+      const CUtensorMap* tm = g == 0 ? &tm_dv : &tm_dk;
+      for (int cc = 0; cc < 2; ++cc) tma_store_4d(tm, stage + cc * 16384, cc * 64, h, k0, b);
       tma_store_commit();
       tma_store_wait_read_all();
     }
   } else {
     // ------------------------------------------------------------------ dQ^T read-out: one thread per d
+    // The tile's dQ^T (thread d holds 64 query columns) goes to a shared staging buffer in the accumulator's
+    // own [q/4][d][4] layout, where the 64-query tile is one contiguous 32 KB block; one thread then adds it
+    // into global memory with a single bulk reduction on the async engine.
     const int quarter = warp & 3;
     const int d = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const bool dq_leader = threadIdx.x == 320;
     float* acc_bh = p.dq_acc + static_cast<size_t>(bh) * p.Tp * 128;
+    float* stage = reinterpret_cast<float*>(smem + kBwdSmemDQ);
     for (int i = 0; i < n; ++i) {
       const int rb = i & 1;
       const int q0 = (i0 + i) * kBwdQTile;
       if (!mbar_wait_warp(&bars.dq_full[rb], (i >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdDq)) break;
       tc_fence_after();
-      uint32_t a[32], bb[32];
-      tmem_ld32(tmem + lane_base + kTmemR + rb * 128 + 64, a);
-      tmem_ld32(tmem + lane_base + kTmemR + rb * 128 + 96, bb);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&bars.dq_empty[rb]);
-      float* dst = acc_bh + static_cast<size_t>(q0 >> 2) * 512 + d * 4;
+      if (threadIdx.x == 320) ATTN_TRACE_EVENT(6, i);
+      if (dq_leader) tma_store_wait_read_all();  // previous tile's reduction has read the staging buffer
+      named_barrier(2, 128);
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4)
-        red_add_v4(dst + q4 * 512, __uint_as_float(a[4 * q4]), __uint_as_float(a[4 * q4 + 1]),
-                   __uint_as_float(a[4 * q4 + 2]), __uint_as_float(a[4 * q4 + 3]));
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t a[32];
+        tmem_ld32(tmem + lane_base + kTmemR + rb * 128 + 64 + 32 * hh, a);
+        tmem_wait_ld();
+        if (hh == 1) {
+          tc_fence_before();
+          mbar_arrive(&bars.dq_empty[rb]);
+        }
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4)
-        red_add_v4(dst + (8 + q4) * 512, __uint_as_float(bb[4 * q4]), __uint_as_float(bb[4 * q4 + 1]),
-                   __uint_as_float(bb[4 * q4 + 2]), __uint_as_float(bb[4 * q4 + 3]));
+        for (int q4 = 0; q4 < 8; ++q4)
+          *reinterpret_cast<float4*>(stage + ((8 * hh + q4) * 128 + d) * 4) =
+              make_float4(__uint_as_float(a[4 * q4]), __uint_as_float(a[4 * q4 + 1]), __uint_as_float(a[4 * q4 + 2]),
+                          __uint_as_float(a[4 * q4 + 3]));
+      }
+      fence_async_shared();
+      named_barrier(2, 128);
+      if (dq_leader) {
+        bulk_reduce_add_f32(acc_bh + static_cast<size_t>(q0 >> 2) * 512, stage, 32768);
+        tma_store_commit();
+      }
+      if (threadIdx.x == 320) ATTN_TRACE_EVENT(7, i);
     }
+    if (dq_leader) tma_store_wait_all();  // the reductions are complete before the CTA retires
   }
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) ATTN_TRACE_EVENT(0, 1);
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem, 512);

@@ -5,8 +5,9 @@
 // own ChatGPT", section 5 "Flash Attention integration"; layout from section 1 "GPT model") and name the
 // Hopper Flash-Attention-3 kernel as the implementation. This kernel is a new design for Blackwell:
 //
-//   * one CTA per (128-query tile, batch, head); heavy (late) query tiles are launched first;
-//   * warp 0 stages Q once and K/V tiles (two-deep rings) with TMA into 128-byte-swizzled shared memory;
+//   * one CTA per (128-query tile, batch, head), head-major so a head's K/V stay in L2 while its tiles run,
+//     heaviest (latest) query tile of each head first;
+//   * warp 0 stages Q once and K/V tiles (three-deep rings) with TMA into 128-byte-swizzled shared memory;
 //   * warp 1 issues tcgen05.mma: S = Q K^T (both operands K-major in shared memory) and O += P V (P from
 //     tensor memory, V MN-major in shared memory), accumulating in fp32 tensor memory;
 //   * warps 2..5 (one thread per query row) run the online softmax straight out of tensor memory: each
@@ -29,9 +30,10 @@ constexpr int kFwdThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 softmax
 
 // Shared-memory layout of the forward kernel (offsets from a 1024-byte aligned base).
 constexpr uint32_t kFwdSmemQ = 0;                       // 32 KB: Q tile, two 64-column boxes of 16 KB
-constexpr uint32_t kFwdSmemK = 32768;                   // 2 x 32 KB: K ring
-constexpr uint32_t kFwdSmemV = kFwdSmemK + 2 * 32768;   // 2 x 32 KB: V ring
-constexpr uint32_t kFwdSmemBytes = kFwdSmemV + 2 * 32768;  // 160 KB
+constexpr int kFwdStages = 3;                           // depth of the K and V rings
+constexpr uint32_t kFwdSmemK = 32768;                   // 3 x 32 KB: K ring
+constexpr uint32_t kFwdSmemV = kFwdSmemK + kFwdStages * 32768;   // 3 x 32 KB: V ring
+constexpr uint32_t kFwdSmemBytes = kFwdSmemV + kFwdStages * 32768;  // 224 KB
 constexpr uint32_t kFwdSmemAlloc = kFwdSmemBytes + 1024;   // + alignment slack
 
 constexpr uint32_t kTmemS = 0, kTmemO = 256, kTmemP = 384;
@@ -48,8 +50,8 @@ struct FwdParams {
 
 struct FwdBarriers {
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[2];
-  uint64_t v_full[2], v_empty[2];
+  uint64_t k_full[kFwdStages], k_empty[kFwdStages];
+  uint64_t v_full[kFwdStages], v_empty[kFwdStages];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t pv_done;
@@ -72,14 +74,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const FwdParams p) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base for the 128-byte-swizzle tiles. Offsetting the array itself (not a round trip
+  // through an integer) keeps the pointer in the shared address space, so accesses compile to LDS/STS.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   __shared__ FwdBarriers bars;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int BH = p.B * p.H;
   const int n_qt = (p.T + kTile - 1) / kTile;
-  const int qt = n_qt - 1 - static_cast<int>(blockIdx.x / BH);  // heavy tiles first
-  const int bh = static_cast<int>(blockIdx.x % BH);
+  // Head-major order, heaviest (latest) query tile first within a head: the CTAs in flight at any time
+  // cover only ~10 heads, so their K/V stay in L2 while every query tile of the head reads them.
+  const int bh = static_cast<int>(blockIdx.x / n_qt);
+  const int qt = n_qt - 1 - static_cast<int>(blockIdx.x % n_qt);
   const int b = bh / p.H, h = bh % p.H;
   const int q0 = qt * kTile;
   const int n_kv = qt + 1;  // causal: KV tiles 0..qt
@@ -87,11 +92,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kFwdStages; ++s) {
       mbar_init(&bars.k_full[s], 1);
       mbar_init(&bars.k_empty[s], 1);
       mbar_init(&bars.v_full[s], 1);
       mbar_init(&bars.v_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&bars.s_full[s], 1);
       mbar_init(&bars.p_full[s], 128);
     }
@@ -109,86 +116,113 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
+  if (threadIdx.x == 0) ATTN_TRACE_EVENT(0, 0);
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // The whole warp walks the loop (warp-uniform control flow, so addresses and coordinates stay in uniform
+    // registers); one lane, elected once, issues every copy.
+    const bool leader = elect_one();
+    if (leader) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int issued_k[2] = {-1, -1}, issued_v[2] = {-1, -1};
       mbar_arrive_expect_tx(&bars.q_full, 2 * 16384);
       for (int c = 0; c < 2; ++c) tma_load_4d(smem + kFwdSmemQ + c * 16384, &tm_q, &bars.q_full, c * 64, h, q0, b);
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j & 1;
-        if (j >= 2 && !mbar_wait(&bars.k_empty[s], ((j - 2) >> 1) & 1, abort, p.timeout_ns, &g_device_error,
-                                 kSiteFwdProdKEmpty))
-          break;
+    }
+    int issued_k[kFwdStages], issued_v[kFwdStages];
+    for (int s = 0; s < kFwdStages; ++s) issued_k[s] = issued_v[s] = -1;
+    for (int j = 0; j < n_kv; ++j) {
+      const int s = j % kFwdStages;
+      const uint32_t prev = ((j - kFwdStages) / kFwdStages) & 1;  // phase of this slot's previous use
+      if (j >= kFwdStages &&
+          !mbar_wait_warp(&bars.k_empty[s], prev, abort, p.timeout_ns, &g_device_error, kSiteFwdProdKEmpty))
+        break;
+      if (leader) {
         mbar_arrive_expect_tx(&bars.k_full[s], 2 * 16384);
         for (int c = 0; c < 2; ++c)
           tma_load_4d(smem + kFwdSmemK + s * 32768 + c * 16384, &tm_k, &bars.k_full[s], c * 64, h, j * kTile, b);
-        issued_k[s] = j;
-        if (j >= 2 && !mbar_wait(&bars.v_empty[s], ((j - 2) >> 1) & 1, abort, p.timeout_ns, &g_device_error,
-                                 kSiteFwdProdVEmpty))
-          break;
+        ATTN_TRACE_EVENT(1, j);
+      }
+      issued_k[s] = j;
+      if (j >= kFwdStages &&
+          !mbar_wait_warp(&bars.v_empty[s], prev, abort, p.timeout_ns, &g_device_error, kSiteFwdProdVEmpty))
+        break;
+      if (leader) {
         mbar_arrive_expect_tx(&bars.v_full[s], 2 * 16384);
         for (int c = 0; c < 2; ++c)
           tma_load_4d(smem + kFwdSmemV + s * 32768 + c * 16384, &tm_v, &bars.v_full[s], c * 64, h, j * kTile, b);
-        issued_v[s] = j;
       }
-      if (*abort) {
-        // Let every copy this thread started land before the CTA's shared memory is released.
-        volatile int no_abort = 0;
-        const uint64_t lim = p.timeout_ns;
-        mbar_wait(&bars.q_full, 0, &no_abort, lim, &g_device_error, kSiteFwdDrain);
-        for (int s = 0; s < 2; ++s) {
-          if (issued_k[s] >= 0) mbar_wait(&bars.k_full[s], (issued_k[s] >> 1) & 1, &no_abort, lim, &g_device_error, kSiteFwdDrain);
-          if (issued_v[s] >= 0) mbar_wait(&bars.v_full[s], (issued_v[s] >> 1) & 1, &no_abort, lim, &g_device_error, kSiteFwdDrain);
-        }
+      issued_v[s] = j;
+    }
+    if (*abort) {
+      // Let every copy this warp started land before the CTA's shared memory is released.
+      volatile int no_abort = 0;
+      const uint64_t lim = p.timeout_ns;
+      mbar_wait(&bars.q_full, 0, &no_abort, lim, &g_device_error, kSiteFwdDrain);
+      for (int s = 0; s < kFwdStages; ++s) {
+        if (issued_k[s] >= 0)
+          mbar_wait(&bars.k_full[s], (issued_k[s] / kFwdStages) & 1, &no_abort, lim, &g_device_error, kSiteFwdDrain);
+        if (issued_v[s] >= 0)
+          mbar_wait(&bars.v_full[s], (issued_v[s] / kFwdStages) & 1, &no_abort, lim, &g_device_error, kSiteFwdDrain);
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer (one thread)
-    if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
-      const uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);  // P (TMEM) x V (MN-major)
-      const uint32_t sq = smem_u32(smem + kFwdSmemQ);
-      bool ok = mbar_wait(&bars.q_full, 0, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaQ);
-      auto issue_pv = [&](int jp) -> bool {
-        const int pb = jp & 1;
-        if (!mbar_wait(&bars.p_full[pb], (jp >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaP)) return false;
-        if (!mbar_wait(&bars.v_full[pb], (jp >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaV)) return false;
-        tc_fence_after();
-        const uint32_t sv = smem_u32(smem + kFwdSmemV + pb * 32768);
+    // ------------------------------------------------------------------ MMA issuer
+    // The whole warp walks the schedule and computes the descriptors (warp-uniform, so they live in uniform
+    // registers); the lane elected once issues every tcgen05.mma and tcgen05.commit (a commit tracks the
+    // MMAs of the thread that issues it, so it must be the same lane throughout).
+    const bool leader = elect_one();
+    const uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
+    const uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);  // P (TMEM) x V (MN-major)
+    // Descriptors are built once per operand and advanced by adding byte offsets in 16-byte units to the
+    // start-address field (one 64-bit add per K step; the tiles stay below 256 KB).
+    const uint64_t dq = sdesc_sw128(smem_u32(smem + kFwdSmemQ), 16, 1024);  // Q, K-major
+    bool ok = mbar_wait_warp(&bars.q_full, 0, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaQ);
+    // PV(jp): O += P(jp) V(jp); P from TMEM buffer jp % 2, V from ring slot jp % kFwdStages.
+    auto issue_pv = [&](int jp) -> bool {
+      const int pb = jp & 1, vs = jp % kFwdStages;
+      if (!mbar_wait_warp(&bars.p_full[pb], (jp >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaP))
+        return false;
+      if (!mbar_wait_warp(&bars.v_full[vs], (jp / kFwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaV))
+        return false;
+      tc_fence_after();
+      const uint64_t dv = sdesc_sw128(smem_u32(smem + kFwdSmemV + vs * 32768), 16384, 1024);  // V, MN-major
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + kTmemO, tmem + kTmemP + pb * 64 + kk * 8, sdesc_sw128(sv + kk * 2048, 16384, 1024), idesc_pv,
-                 (jp > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < 8; ++kk)  // K step kk: 16 keys = 2048 bytes further (128 in 16-byte units)
+        if (leader) mma_ts(tmem + kTmemO, tmem + kTmemP + pb * 64 + kk * 8, dv + kk * 128, idesc_pv, (jp > 0 || kk > 0) ? 1u : 0u);
+      if (leader) {
         mma_commit(&bars.pv_done);
-        mma_commit(&bars.v_empty[pb]);
-        return true;
-      };
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int s = j & 1;
-        if (!mbar_wait(&bars.k_full[s], (j >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaK)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sk = smem_u32(smem + kFwdSmemK + s * 32768);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tmem + kTmemS + s * 128, sdesc_sw128(sq + koff, 16, 1024), sdesc_sw128(sk + koff, 16, 1024), idesc_s,
-                 kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&bars.s_full[s]);
-        mma_commit(&bars.k_empty[s]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        ATTN_TRACE_EVENT(3, jp);
+        mma_commit(&bars.v_empty[vs]);
       }
-      if (ok && issue_pv(n_kv - 1)) mma_commit(&bars.o_final);
-      // Drain: wait until every MMA this thread issued has completed before tensor memory is released.
-      mma_commit(&bars.drain);
-      volatile int no_abort = 0;
-      mbar_wait(&bars.drain, 0, &no_abort, p.timeout_ns, &g_device_error, kSiteFwdDrain);
+      return true;
+    };
+    for (int j = 0; ok && j < n_kv; ++j) {
+      const int ks = j % kFwdStages, sb = j & 1;
+      if (!mbar_wait_warp(&bars.k_full[ks], (j / kFwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaK)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint64_t dk = sdesc_sw128(smem_u32(smem + kFwdSmemK + ks * 32768), 16, 1024);  // K, K-major
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {  // K step kk: second 64-column box from kk = 4, 32 bytes per step within
+        const uint32_t koff = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+        if (leader) mma_ss(tmem + kTmemS + sb * 128, dq + koff, dk + koff, idesc_s, kk > 0 ? 1u : 0u);
+      }
+      if (leader) {
+        mma_commit(&bars.s_full[sb]);
+        ATTN_TRACE_EVENT(2, j);
+        mma_commit(&bars.k_empty[ks]);
+      }
+      if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
     }
+    if (ok && issue_pv(n_kv - 1) && leader) mma_commit(&bars.o_final);
+    // Drain: wait until every MMA the leader issued has completed before tensor memory is released.
+    if (leader) mma_commit(&bars.drain);
+    volatile int no_abort = 0;
+    mbar_wait(&bars.drain, 0, &no_abort, p.timeout_ns, &g_device_error, kSiteFwdDrain);
   } else {
     // ------------------------------------------------------------------ softmax / correction / epilogue
     const int quarter = warp & 3;           // TMEM lane quarter this warp may access
@@ -205,6 +239,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         break;
       }
       tc_fence_after();
+      if (threadIdx.x == 64) ATTN_TRACE_EVENT(4, j);
       float s[128];
       {
         uint32_t r0[32], r1[32], r2[32], r3[32];
@@ -213,6 +248,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_ld32(tmem + lane_base + kTmemS + sb * 128 + 64, r2);
         tmem_ld32(tmem + lane_base + kTmemS + sb * 128 + 96, r3);
         tmem_wait_ld();
+        if (threadIdx.x == 64) ATTN_TRACE_EVENT(8, j);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           s[i] = __uint_as_float(r0[i]);
@@ -226,10 +262,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int i = 0; i < 128; ++i)
           if (i > row) s[i] = -INFINITY;
       }
-      float mx = s[0];
+      // Row max as a tree over 16 independent partial maxima (a single 128-long dependent chain would leave
+      // ~500 cycles of latency exposed: there is one softmax warp per SM sub-partition).
+      float pm[16];
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
-      const float m_tile = mx * c;
+      for (int i = 0; i < 16; ++i) pm[i] = s[i];
+#pragma unroll
+      for (int i = 16; i < 128; ++i) pm[i & 15] = fmaxf(pm[i & 15], s[i]);
+#pragma unroll
+      for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) pm[i] = fmaxf(pm[i], pm[i + w]);
+      const float m_tile = pm[0] * c;
+      if (threadIdx.x == 64) ATTN_TRACE_EVENT(11, j);
       if (j == 0) {
         m = m_tile;
       } else if (const bool need = m_tile > m + kRescaleThreshold; __any_sync(0xffffffffu, need)) {
@@ -260,7 +305,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       // P = exp2(c*S - m), row sum, pack to bf16 pairs into the P buffer of this tile.
       const float neg_m = -m;
-      float lsum = 0.f;
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial row sums
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t pk[16];
@@ -268,21 +313,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int i = 0; i < 16; ++i) {
           const float p0 = ex2(fmaf(s[cc * 32 + 2 * i], c, neg_m));
           const float p1 = ex2(fmaf(s[cc * 32 + 2 * i + 1], c, neg_m));
-          lsum += p0 + p1;
+          ps[(2 * i) & 7] += p0;
+          ps[(2 * i + 1) & 7] += p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tmem + lane_base + kTmemP + sb * 64 + cc * 16, pk);
       }
-      l += lsum;
+      l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      if (threadIdx.x == 64) ATTN_TRACE_EVENT(9, j);
       tmem_wait_st();
+      if (threadIdx.x == 64) ATTN_TRACE_EVENT(10, j);
       tc_fence_before();
       mbar_arrive(&bars.p_full[sb]);
+      if (threadIdx.x == 64) ATTN_TRACE_EVENT(5, j);
     }
     // Epilogue: O / l -> bf16 -> swizzled staging (reusing the Q buffer) -> TMA store; LSE in natural log.
     // Every thread of the group reaches the named barrier, failed or not; the store is skipped on abort.
+    if (threadIdx.x == 64) ATTN_TRACE_EVENT(6, 0);
     const bool epi_ok =
         __all_sync(0xffffffffu, ok) && mbar_wait_warp(&bars.o_final, 0, abort, p.timeout_ns, &g_device_error, kSiteFwdEpi);
     if (epi_ok) {
+      if (threadIdx.x == 64) ATTN_TRACE_EVENT(7, 0);
       tc_fence_after();
       const float inv_l = 1.0f / l;
       uint8_t* stage = smem + kFwdSmemQ;
@@ -311,11 +362,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int cc = 0; cc < 2; ++cc) tma_store_4d(&tm_o, smem + kFwdSmemQ + cc * 16384, cc * 64, h, q0, b);
       tma_store_commit();
       tma_store_wait_read_all();
+      ATTN_TRACE_EVENT(6, 1);
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) ATTN_TRACE_EVENT(0, 1);
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem, 512);

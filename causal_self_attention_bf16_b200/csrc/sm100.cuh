@@ -79,6 +79,19 @@ ATTN_DEVICE_INLINE bool mbar_try_wait(uint32_t bar_addr, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test: has the phase with the given parity of `bar` completed? (Unlike try_wait, never suspends.)
+ATTN_DEVICE_INLINE bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity of `bar` has completed. Gives up when `*abort` becomes
 // non-zero (another role of the CTA failed) or after `limit_ns`; on a timeout it raises `*abort`, records
 // `site` in `err_word` and returns false.
@@ -155,6 +168,16 @@ ATTN_DEVICE_INLINE void bulk_load(void* dst, const void* src, uint32_t bytes, ui
           smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Untiled bulk reduction shared -> global: dst[i] += src[i] for `bytes / 4` fp32 values, done by the async
+// engine (not the load/store unit). Both addresses 16-byte aligned, bytes a multiple of 16; completes through
+// the issuing thread's bulk group (tma_store_commit / tma_store_wait_*).
+ATTN_DEVICE_INLINE void bulk_reduce_add_f32(float* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(dst)),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
 }
 
 // ---------------------------------------------------------------------------------------------------------
