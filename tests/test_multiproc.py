@@ -1,0 +1,69 @@
+"""Multi-process plumbing of bench.py on CPU (gloo, world size 2): the path does not shard across GPUs (every
+rank runs its own replica of the batch, no collective on the data path), so what runs across ranks is the
+timing reduction (max over ranks) and the whole-job aggregation (units of all ranks over the slowest time)."""
+import os
+import socket
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, times, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        r, w, local = bench.dist_env()
+        assert (r, w, local) == (rank, world, rank)
+        mx = bench.reduce_max(times[rank], world)
+        dist.barrier()
+        q.put((rank, mx))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_reduce_max_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    times = [1.25, 3.5]
+    mp.spawn(_worker, args=(2, port, times, q), nprocs=2, join=True)
+    got = dict(q.get(timeout=30) for _ in range(2))
+    assert got == {0: 3.5, 1: 3.5}
+
+
+def test_aggregate_is_whole_job_over_slowest_rank():
+    # 2 ranks, each 10 units, slowest 2 s: 10 units/s for the whole job
+    assert bench.aggregate(10.0, 2, 2.0) == pytest.approx(10.0)
+    assert bench.aggregate(5.0, 1, 0.5) == pytest.approx(10.0)
+
+
+def test_reference_arm_runs_on_rank0_only(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    args = bench.parse_args(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0"])
+    assert bench.run_reference(args) == 0
+    assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    args = bench.parse_args(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "1"])
+    assert bench.run_reference(args) == 0
+    import json
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["config"]["workload"] == "tiny"
