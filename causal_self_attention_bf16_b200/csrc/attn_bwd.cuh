@@ -14,10 +14,10 @@
 //        dV += P^T dO, dK += dS^T Q             (P^T, dS^T from tensor memory; dO, Q MN-major)
 //        dQ^T = K^T dS^T                        (both operands MN-major in shared memory)
 //      Two warp groups taking alternate query tiles (one thread per key row) turn S^T, dP^T into P^T, dS^T
-//      (exp2 against the stored LSE); a third warp group stages dQ^T in shared memory in the accumulator's
-//      layout and adds each 64-query tile (32 contiguous KB) into the fp32 accumulator with one bulk
-//      reduction (cp.reduce.async.bulk .add.f32) on the async engine. dK, dV stay in tensor memory for the
-//      whole walk and leave through a TMA store.
+//      (exp2 against the stored LSE), then read their tile's dQ^T out of tensor memory, stage it in shared
+//      memory in the accumulator's layout and add it into the fp32 accumulator with one bulk reduction
+//      (cp.reduce.async.bulk .add.f32, 32 contiguous KB) on the async engine. dK, dV stay in tensor memory
+//      for the whole walk and leave through a TMA store.
 //   3. attn_bwd_dq_kernel: dQ = bf16(scale * accumulator) back in [B, T, H, D].
 //
 // Tensor memory of the dK/dV kernel (512 columns): dV [0,128), dK [128,256), and two 128-column tile
@@ -33,14 +33,14 @@ namespace attn {
 constexpr int kBwdQTile = 64;       // queries per inner tile
 constexpr int kBwdKTile = 128;      // keys per CTA
 constexpr int kBwdStages = 3;       // Q/dO/LSE/Delta ring depth
-constexpr int kBwdThreads = 448;    // warp 0 TMA, warp 1 MMA, warps 2..9 softmax, warps 10..13 dQ
+constexpr int kBwdThreads = 320;    // warp 0 TMA, warp 1 MMA, warps 2..9 two softmax/dQ groups
 
 constexpr uint32_t kBwdSmemK = 0;                                 // 32 KB
 constexpr uint32_t kBwdSmemV = 32768;                             // 32 KB
 constexpr uint32_t kBwdSmemQ = 65536;                             // 3 x 16 KB (two 8 KB boxes each)
 constexpr uint32_t kBwdSmemDO = kBwdSmemQ + kBwdStages * 16384;   // 3 x 16 KB
 constexpr uint32_t kBwdSmemDS = kBwdSmemDO + kBwdStages * 16384;  // 2 x 16 KB: dS^T [128 keys][64 q]
-constexpr uint32_t kBwdSmemDQ = kBwdSmemDS + 2 * 16384;           // 32 KB: dQ^T tile staged for the bulk reduce
+constexpr uint32_t kBwdSmemDQ = kBwdSmemDS + 2 * 16384;           // 32 KB: a dQ^T tile staged for its bulk reduce
 constexpr uint32_t kBwdSmemLse = kBwdSmemDQ + 32768;              // 3 x 256 B
 constexpr uint32_t kBwdSmemDelta = kBwdSmemLse + kBwdStages * 256;  // 3 x 256 B
 constexpr uint32_t kBwdSmemBytes = kBwdSmemDelta + kBwdStages * 256;  // barriers follow (see BwdBarriers)
@@ -146,6 +146,7 @@ struct BwdBarriers {
   uint64_t dq_full[2];   // dQ^T of buffer b ready (also: dV, dK MMAs of that tile done)
   uint64_t dq_empty[2];  // dQ^T read out: buffer b free
   uint64_t b_done[2];    // dV, dK MMAs of the tile in buffer b done (buffer's P^T, dS^T consumed)
+  uint64_t stage_free;   // dQ staging buffer read by the previous tile's bulk reduction (one phase per tile)
   uint64_t acc_done;     // all MMAs done (epilogue)
   uint64_t drain;
   uint32_t tmem_base;
@@ -205,6 +206,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       mbar_init(&bars.dq_empty[s], 128);
       mbar_init(&bars.b_done[s], 1);
     }
+    mbar_init(&bars.stage_free, 1);
     mbar_init(&bars.acc_done, 1);
     mbar_init(&bars.drain, 1);
     bars.abort = 0;
@@ -364,6 +366,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const int kg = k0 + krow;
     const float c = p.scale_log2;
+    const bool group_leader = lane == 0 && quarter == 2;  // first warp of the group
+    float* acc_bh = p.dq_acc + static_cast<size_t>(bh) * p.Tp * 128;
+    float* dq_stage = reinterpret_cast<float*>(smem + kBwdSmemDQ);
     bool ok = true;
     for (int i = g; i < n; i += 2) {
       const int s = i % kBwdStages, rb = g;
@@ -386,6 +391,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         tmem_ld32(r, sv);        // S^T of queries [32hh, 32hh+32)
         tmem_ld32(r + 64, dp);   // dP^T of the same queries
         tmem_wait_ld();
+        if (threadIdx.x == 64) ATTN_TRACE_EVENT(8, i * 2 + hh);
         uint32_t ppk[16], dpk[16];
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {
@@ -405,6 +411,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           dpk[q4 * 2] = pack_bf16x2(dsv[0], dsv[1]);
           dpk[q4 * 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
         }
+        if (threadIdx.x == 64) ATTN_TRACE_EVENT(9, i * 2 + hh);
         tmem_st16(r, ppk);        // P^T  of these 32 queries: columns [32hh, 32hh+16)
         tmem_st16(r + 16, dpk);   // dS^T of these 32 queries: columns [32hh+16, 32hh+32)
 #pragma unroll
@@ -414,11 +421,50 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
       }
       tmem_wait_st();
+      if (threadIdx.x == 64) ATTN_TRACE_EVENT(10, i);
       fence_async_shared();
+      if (threadIdx.x == 64) ATTN_TRACE_EVENT(11, i);
       tc_fence_before();
       mbar_arrive(&bars.p_full[rb]);
       if (threadIdx.x == 64 || threadIdx.x == 192) ATTN_TRACE_EVENT(5, i);
+
+      // dQ^T of this tile (thread = d, 64 query columns) -> staging buffer in the accumulator's [q/4][d][4]
+      // layout, where the tile is one contiguous 32 KB block -> one bulk reduce-add on the async engine. The
+      // staging buffer passes between the two groups in tile order through stage_free.
+      if (!mbar_wait_warp(&bars.dq_full[rb], (i >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdDq)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (threadIdx.x == 64) ATTN_TRACE_EVENT(6, i);
+      uint32_t a[2][32];
+      tmem_ld32(tmem + lane_base + kTmemR + rb * 128 + 64, a[0]);
+      tmem_ld32(tmem + lane_base + kTmemR + rb * 128 + 96, a[1]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars.dq_empty[rb]);  // dQ^T is in registers: the tensor-memory buffer is free
+      if (i > 0 && !mbar_wait_warp(&bars.stage_free, (i - 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdDq)) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4)
+          *reinterpret_cast<float4*>(dq_stage + ((8 * hh + q4) * 128 + krow) * 4) =
+              make_float4(__uint_as_float(a[hh][4 * q4]), __uint_as_float(a[hh][4 * q4 + 1]),
+                          __uint_as_float(a[hh][4 * q4 + 2]), __uint_as_float(a[hh][4 * q4 + 3]));
+      fence_async_shared();
+      named_barrier(2 + g, 128);
+      if (group_leader) {
+        bulk_reduce_add_f32(acc_bh + static_cast<size_t>(((i0 + i) * kBwdQTile) >> 2) * 512, dq_stage, 32768);
+        tma_store_commit();
+        tma_store_wait_read_all();  // the staging buffer has been read: hand it to the next tile
+        mbar_arrive(&bars.stage_free);
+        ATTN_TRACE_EVENT(7, i);
+      }
     }
+    if (group_leader) tma_store_wait_all();  // this group's reductions are complete before the CTA retires
     // Epilogue: group 0 writes dV, group 1 writes scale*dK: TMEM -> bf16 -> swizzled staging -> TMA store
     // (rows past T are clipped). Both groups reach the named barrier, failed or not; no store on abort.
     const bool epi_ok = __all_sync(0xffffffffu, ok) &&
@@ -453,49 +499,6 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       tma_store_commit();
       tma_store_wait_read_all();
     }
-  } else {
-    // ------------------------------------------------------------------ dQ^T read-out: one thread per d
-    // The tile's dQ^T (thread d holds 64 query columns) goes to a shared staging buffer in the accumulator's
-    // own [q/4][d][4] layout, where the 64-query tile is one contiguous 32 KB block; one thread then adds it
-    // into global memory with a single bulk reduction on the async engine.
-    const int quarter = warp & 3;
-    const int d = quarter * 32 + lane;
-    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const bool dq_leader = threadIdx.x == 320;
-    float* acc_bh = p.dq_acc + static_cast<size_t>(bh) * p.Tp * 128;
-    float* stage = reinterpret_cast<float*>(smem + kBwdSmemDQ);
-    for (int i = 0; i < n; ++i) {
-      const int rb = i & 1;
-      const int q0 = (i0 + i) * kBwdQTile;
-      if (!mbar_wait_warp(&bars.dq_full[rb], (i >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdDq)) break;
-      tc_fence_after();
-      if (threadIdx.x == 320) ATTN_TRACE_EVENT(6, i);
-      if (dq_leader) tma_store_wait_read_all();  // previous tile's reduction has read the staging buffer
-      named_barrier(2, 128);
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t a[32];
-        tmem_ld32(tmem + lane_base + kTmemR + rb * 128 + 64 + 32 * hh, a);
-        tmem_wait_ld();
-        if (hh == 1) {
-          tc_fence_before();
-          mbar_arrive(&bars.dq_empty[rb]);
-        }
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-          *reinterpret_cast<float4*>(stage + ((8 * hh + q4) * 128 + d) * 4) =
-              make_float4(__uint_as_float(a[4 * q4]), __uint_as_float(a[4 * q4 + 1]), __uint_as_float(a[4 * q4 + 2]),
-                          __uint_as_float(a[4 * q4 + 3]));
-      }
-      fence_async_shared();
-      named_barrier(2, 128);
-      if (dq_leader) {
-        bulk_reduce_add_f32(acc_bh + static_cast<size_t>(q0 >> 2) * 512, stage, 32768);
-        tma_store_commit();
-      }
-      if (threadIdx.x == 320) ATTN_TRACE_EVENT(7, i);
-    }
-    if (dq_leader) tma_store_wait_all();  // the reductions are complete before the CTA retires
   }
 
   tc_fence_before();
