@@ -13,7 +13,7 @@ __device__ uint32_t g_device_error;
 // the first kTraceCtas CTAs of a launch record SM clock64 stamps of pipeline events into g_trace, read back
 // by attn_trace_dump.
 #ifdef ATTN_TRACE
-constexpr int kTraceCtas = 64, kTraceEvents = 14, kTraceSlots = 64;
+constexpr int kTraceCtas = 64, kTraceEvents = 16, kTraceSlots = 64;
 constexpr size_t kTraceBytes = sizeof(unsigned long long) * kTraceCtas * kTraceEvents * kTraceSlots;
 __device__ unsigned long long g_trace[kTraceCtas][kTraceEvents][kTraceSlots];
 #define ATTN_TRACE_EVENT(ev, slot)                                                              \

@@ -7,17 +7,23 @@
 //
 //   * one CTA per (128-query tile, batch, head), head-major so a head's K/V stay in L2 while its tiles run,
 //     heaviest (latest) query tile of each head first;
-//   * warp 0 stages Q once and K/V tiles (three-deep rings) with TMA into 128-byte-swizzled shared memory;
-//   * warp 1 issues tcgen05.mma: S = Q K^T (both operands K-major in shared memory) and O += P V (P from
-//     tensor memory, V MN-major in shared memory), accumulating in fp32 tensor memory;
-//   * warps 2..5 (one thread per query row) run the online softmax straight out of tensor memory: each
+//   * warp 0 stages Q once and K tiles, warp 10 V tiles (three-deep rings) with TMA into 128-byte-swizzled
+//     shared memory;
+//   * warp 1 issues tcgen05.mma with the A operand in tensor memory: S = Q K^T (Q copied into tensor memory
+//     once, K K-major in shared memory) and O += P V (V MN-major in shared memory), accumulating in fp32
+//     tensor memory. (With both operands in shared memory an M=128, N=128 MMA runs at ~60% of the tensor
+//     rate on B200: its operand reads from shared memory are the limit.)
+//   * warps 2..9, two groups of four, run the online softmax straight out of tensor memory, one thread per
+//     query row: group g takes KV tiles j = g, g+2, ..., and only the running row max passes between the
+//     groups (through shared memory), so one tile's exponentials overlap the next tile's load and max. A
 //     thread owns a whole row of S, so row max and row sum need no shuffles; masking happens only on the
 //     diagonal tile (tiles above it are skipped); O is rescaled lazily, only when the running max grows by
 //     more than 2^8; the epilogue normalises O, stages it in shared memory and writes it with a TMA store.
 //
-// Tensor memory (512 columns): S double buffer [0,256), O [256,384), P double buffer (bf16 pairs) [384,512).
-// Issue order of the MMA warp: S(0), S(1), PV(0), S(2), PV(1), ... so that a commit after S(j) also covers
-// PV(j-2); that is what frees S buffer j%2 and P buffer j%2 for reuse without further handshakes.
+// Tensor memory (512 columns): S double buffer [0,256) (buffer j%2 belongs to the group of tile j), O
+// [256,384), Q (bf16 pairs) [384,448), P (bf16 pairs) [448,512). The MMA warp issues S(j+2) as soon as S(j)
+// has been read out, ahead of PV(j): S(0), S(1), S(2), PV(0), S(3), PV(1), ...; the group of tile j stores
+// P(j) once PV(j-1) has landed, while the tensor core works on S(j+1).
 #pragma once
 #include "attn_common.cuh"
 #include "sm100.cuh"
@@ -26,20 +32,41 @@ namespace attn {
 
 constexpr int kTile = 128;        // query rows per CTA and keys per KV tile
 constexpr int kHeadDim = 128;     // D
-constexpr int kFwdThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 softmax
+constexpr int kFwdThreads = 352;  // warp 0 TMA (Q, K), warp 1 MMA, warps 2..9 two softmax groups, warp 10 TMA (V)
+constexpr int kFwdWarpV = 10;
 
 // Shared-memory layout of the forward kernel (offsets from a 1024-byte aligned base).
 constexpr uint32_t kFwdSmemQ = 0;                       // 32 KB: Q tile, two 64-column boxes of 16 KB
 constexpr int kFwdStages = 3;                           // depth of the K and V rings
 constexpr uint32_t kFwdSmemK = 32768;                   // 3 x 32 KB: K ring
 constexpr uint32_t kFwdSmemV = kFwdSmemK + kFwdStages * 32768;   // 3 x 32 KB: V ring
-constexpr uint32_t kFwdSmemBytes = kFwdSmemV + kFwdStages * 32768;  // 224 KB
-constexpr uint32_t kFwdSmemAlloc = kFwdSmemBytes + 1024;   // + alignment slack
+constexpr uint32_t kFwdSmemXchg = kFwdSmemV + kFwdStages * 32768;   // 2 KB: row-max / row-sum exchange
+constexpr uint32_t kFwdSmemBytes = kFwdSmemXchg + 2 * 2 * 128 * 4;     // barriers follow (see FwdBarriers)
 
-constexpr uint32_t kTmemS = 0, kTmemO = 256, kTmemP = 384;
+constexpr uint32_t kTmemS = 0, kTmemO = 256, kTmemQ = 384, kTmemP = 448;
 
 // Lazy rescaling threshold on the running max, in log2 units (values of P stay below 2^8).
 constexpr float kRescaleThreshold = 8.0f;
+
+// Pairs of columns, out of every 16, whose exp2 runs on the FMA pipe (exp2_poly) instead of MUFU.
+#ifndef ATTN_FWD_POLY_PAIRS
+#define ATTN_FWD_POLY_PAIRS 0
+#endif
+constexpr int kFwdPolyPairs = ATTN_FWD_POLY_PAIRS;
+
+// 2^x on the FMA pipe, for x <= 8 (softmax arguments). Cody-Waite style reduction: n = round(x) by the
+// 1.5 * 2^23 magic addition (t's low mantissa bits then hold n), f = x - n in [-1/2, 1/2]; 2^f by a cubic
+// fitted for least maximum relative error (7.5e-5; fit_exp2_poly.py prints the coefficients and the bound);
+// 2^n by adding n to the exponent field (n << 23 equals t's bits << 23 modulo 2^32 because the magic
+// constant's bits vanish under that shift). Below -126 the exponent field would underflow, so those
+// arguments (true values under 1.2e-38, masked keys at -inf among them) return exactly 0.
+__device__ __forceinline__ float exp2_poly(float x) {
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(0.0551716668f, f, 0.242611135f), f, 0.693260987f), f, 0.999928073f);
+  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  return x < -126.0f ? 0.0f : r;  // masked keys (-inf) give exactly 0
+}
 
 struct FwdParams {
   float* lse;        // [B, H, T] fp32
@@ -50,21 +77,28 @@ struct FwdParams {
 
 struct FwdBarriers {
   uint64_t q_full;
+  uint64_t q_tmem;      // Q copied from shared into tensor memory by the softmax warps
   uint64_t k_full[kFwdStages], k_empty[kFwdStages];
   uint64_t v_full[kFwdStages], v_empty[kFwdStages];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t pv_done;
-  uint64_t o_final;  // committed once after the last PV: the epilogue's wait (pv_done may be 2 phases behind)
+  uint64_t s_full[2];   // S(j) landed in buffer j%2
+  uint64_t s_free[2];   // S(j) read out of buffer j%2: S(j+2) may overwrite it
+  uint64_t p_full[2];   // P(j) stored in buffer j%2 (and O rescaled if needed): PV(j) may be issued
+  uint64_t xchg[2];     // running max after tile j published in slot j%2
+  uint64_t pv_done[2];  // PV(j) completed (barrier j%2): P is free, O holds tiles 0..j
+  uint64_t o_final;     // committed once after the last PV: the epilogue's wait
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
+// No static shared memory: the dynamic block starts 1024-byte aligned and needs no slack (the kernel checks
+// this and refuses to run otherwise): tiles, the exchange area, then the barriers. 226 KB in all.
+constexpr uint32_t kFwdSmemAlloc = kFwdSmemBytes + sizeof(FwdBarriers);
+static_assert(kFwdSmemAlloc <= 232448, "forward kernel exceeds the 227 KB shared-memory opt-in");
 
 // Error sites (recorded with a timeout in the device error word): 0x10 + barrier id, per role.
 enum : uint32_t {
-  kSiteFwdProdKEmpty = 0x11, kSiteFwdProdVEmpty = 0x12, kSiteFwdMmaQ = 0x21, kSiteFwdMmaK = 0x22,
-  kSiteFwdMmaP = 0x23, kSiteFwdMmaV = 0x24, kSiteFwdSmS = 0x31, kSiteFwdSmPV = 0x32, kSiteFwdEpi = 0x33,
+  kSiteFwdLayout = 0x10, kSiteFwdProdKEmpty = 0x11, kSiteFwdProdVEmpty = 0x12, kSiteFwdMmaQ = 0x21, kSiteFwdMmaK = 0x22,
+  kSiteFwdMmaP = 0x23, kSiteFwdMmaV = 0x24, kSiteFwdMmaS = 0x25, kSiteFwdSmS = 0x31, kSiteFwdSmPV = 0x32, kSiteFwdEpi = 0x33, kSiteFwdSmX = 0x35, kSiteFwdSmQ = 0x36,
   kSiteFwdDrain = 0x34
 };
 
@@ -76,8 +110,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base for the 128-byte-swizzle tiles. Offsetting the array itself (not a round trip
   // through an integer) keeps the pointer in the shared address space, so accesses compile to LDS/STS.
-  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  __shared__ FwdBarriers bars;
+  uint8_t* smem = smem_raw;
+  if (smem_u32(smem_raw) & 1023u) {  // the layout needs a 1024-byte aligned dynamic block
+    if (threadIdx.x == 0) atomicOr(&g_device_error, sm100::DEV_ERR_TIMEOUT | (kSiteFwdLayout << 8));
+    return;
+  }
+  FwdBarriers& bars = *reinterpret_cast<FwdBarriers*>(smem + kFwdSmemBytes);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_qt = (p.T + kTile - 1) / kTile;
@@ -92,6 +130,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
+    mbar_init(&bars.q_tmem, 256);
     for (int s = 0; s < kFwdStages; ++s) {
       mbar_init(&bars.k_full[s], 1);
       mbar_init(&bars.k_empty[s], 1);
@@ -100,9 +139,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars.s_full[s], 1);
+      mbar_init(&bars.s_free[s], 128);
       mbar_init(&bars.p_full[s], 128);
+      mbar_init(&bars.xchg[s], 128);
+      mbar_init(&bars.pv_done[s], 1);
     }
-    mbar_init(&bars.pv_done, 1);
     mbar_init(&bars.o_final, 1);
     mbar_init(&bars.drain, 1);
     bars.abort = 0;
@@ -118,54 +159,48 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const uint32_t tmem = bars.tmem_base;
   if (threadIdx.x == 0) ATTN_TRACE_EVENT(0, 0);
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    // The whole warp walks the loop (warp-uniform control flow, so addresses and coordinates stay in uniform
-    // registers); one lane, elected once, issues every copy.
+  if (warp == 0 || warp == kFwdWarpV) {
+    // ------------------------------------------------------------------ TMA producers
+    // Warp 0 stages Q and the K ring, warp 10 the V ring. One thread's TMA loads are served largely one
+    // after another on B200 (~38-53 B/clk per SM for 32 KB loads from one issuer, ~75 from two), and a KV
+    // tile needs 64 KB per ~1000 cycles of tensor work, hence two issuing warps. Each walks its loop
+    // warp-uniformly (addresses and coordinates stay in uniform registers); one elected lane issues.
+    const bool is_k = warp == 0;
     const bool leader = elect_one();
+    const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+    uint64_t* full = is_k ? bars.k_full : bars.v_full;
+    uint64_t* empty = is_k ? bars.k_empty : bars.v_empty;
+    uint8_t* ring = smem + (is_k ? kFwdSmemK : kFwdSmemV);
     if (leader) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(&bars.q_full, 2 * 16384);
-      for (int c = 0; c < 2; ++c) tma_load_4d(smem + kFwdSmemQ + c * 16384, &tm_q, &bars.q_full, c * 64, h, q0, b);
+      tma_prefetch_desc(tm);
+      if (is_k) {
+        tma_prefetch_desc(&tm_q);
+        mbar_arrive_expect_tx(&bars.q_full, 2 * 16384);
+        for (int c = 0; c < 2; ++c) tma_load_4d(smem + kFwdSmemQ + c * 16384, &tm_q, &bars.q_full, c * 64, h, q0, b);
+      }
     }
-    int issued_k[kFwdStages], issued_v[kFwdStages];
-    for (int s = 0; s < kFwdStages; ++s) issued_k[s] = issued_v[s] = -1;
+    int issued[kFwdStages];
+    for (int s = 0; s < kFwdStages; ++s) issued[s] = -1;
     for (int j = 0; j < n_kv; ++j) {
       const int s = j % kFwdStages;
-      const uint32_t prev = ((j - kFwdStages) / kFwdStages) & 1;  // phase of this slot's previous use
-      if (j >= kFwdStages &&
-          !mbar_wait_warp(&bars.k_empty[s], prev, abort, p.timeout_ns, &g_device_error, kSiteFwdProdKEmpty))
+      if (j >= kFwdStages && !mbar_wait_warp(&empty[s], ((j - kFwdStages) / kFwdStages) & 1, abort, p.timeout_ns,
+                                             &g_device_error, is_k ? kSiteFwdProdKEmpty : kSiteFwdProdVEmpty))
         break;
       if (leader) {
-        mbar_arrive_expect_tx(&bars.k_full[s], 2 * 16384);
-        for (int c = 0; c < 2; ++c)
-          tma_load_4d(smem + kFwdSmemK + s * 32768 + c * 16384, &tm_k, &bars.k_full[s], c * 64, h, j * kTile, b);
-        ATTN_TRACE_EVENT(1, j);
+        mbar_arrive_expect_tx(&full[s], 2 * 16384);
+        for (int c = 0; c < 2; ++c) tma_load_4d(ring + s * 32768 + c * 16384, tm, &full[s], c * 64, h, j * kTile, b);
+        if (is_k) ATTN_TRACE_EVENT(1, j);
       }
-      issued_k[s] = j;
-      if (j >= kFwdStages &&
-          !mbar_wait_warp(&bars.v_empty[s], prev, abort, p.timeout_ns, &g_device_error, kSiteFwdProdVEmpty))
-        break;
-      if (leader) {
-        mbar_arrive_expect_tx(&bars.v_full[s], 2 * 16384);
-        for (int c = 0; c < 2; ++c)
-          tma_load_4d(smem + kFwdSmemV + s * 32768 + c * 16384, &tm_v, &bars.v_full[s], c * 64, h, j * kTile, b);
-      }
-      issued_v[s] = j;
+      issued[s] = j;
     }
     if (*abort) {
       // Let every copy this warp started land before the CTA's shared memory is released.
       volatile int no_abort = 0;
       const uint64_t lim = p.timeout_ns;
-      mbar_wait(&bars.q_full, 0, &no_abort, lim, &g_device_error, kSiteFwdDrain);
-      for (int s = 0; s < kFwdStages; ++s) {
-        if (issued_k[s] >= 0)
-          mbar_wait(&bars.k_full[s], (issued_k[s] / kFwdStages) & 1, &no_abort, lim, &g_device_error, kSiteFwdDrain);
-        if (issued_v[s] >= 0)
-          mbar_wait(&bars.v_full[s], (issued_v[s] / kFwdStages) & 1, &no_abort, lim, &g_device_error, kSiteFwdDrain);
-      }
+      if (is_k) mbar_wait(&bars.q_full, 0, &no_abort, lim, &g_device_error, kSiteFwdDrain);
+      for (int s = 0; s < kFwdStages; ++s)
+        if (issued[s] >= 0)
+          mbar_wait(&full[s], (issued[s] / kFwdStages) & 1, &no_abort, lim, &g_device_error, kSiteFwdDrain);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -173,97 +208,133 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // registers); the lane elected once issues every tcgen05.mma and tcgen05.commit (a commit tracks the
     // MMAs of the thread that issues it, so it must be the same lane throughout).
     const bool leader = elect_one();
-    const uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);  // Q (K-major) x K (K-major)
+    const uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);  // Q (TMEM) x K (K-major)
     const uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);  // P (TMEM) x V (MN-major)
     // Descriptors are built once per operand and advanced by adding byte offsets in 16-byte units to the
     // start-address field (one 64-bit add per K step; the tiles stay below 256 KB).
-    const uint64_t dq = sdesc_sw128(smem_u32(smem + kFwdSmemQ), 16, 1024);  // Q, K-major
-    bool ok = mbar_wait_warp(&bars.q_full, 0, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaQ);
-    // PV(jp): O += P(jp) V(jp); P from TMEM buffer jp % 2, V from ring slot jp % kFwdStages.
+    bool ok = mbar_wait_warp(&bars.q_tmem, 0, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaQ);
+    // PV(jp): O += P(jp) V(jp); P from tensor memory, V from ring slot jp % kFwdStages.
     auto issue_pv = [&](int jp) -> bool {
       const int pb = jp & 1, vs = jp % kFwdStages;
       if (!mbar_wait_warp(&bars.p_full[pb], (jp >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaP))
         return false;
       if (!mbar_wait_warp(&bars.v_full[vs], (jp / kFwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaV))
         return false;
+      if (leader) ATTN_TRACE_EVENT(15, jp);
       tc_fence_after();
       const uint64_t dv = sdesc_sw128(smem_u32(smem + kFwdSmemV + vs * 32768), 16384, 1024);  // V, MN-major
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)  // K step kk: 16 keys = 2048 bytes further (128 in 16-byte units)
-        if (leader) mma_ts(tmem + kTmemO, tmem + kTmemP + pb * 64 + kk * 8, dv + kk * 128, idesc_pv, (jp > 0 || kk > 0) ? 1u : 0u);
+        if (leader) mma_ts(tmem + kTmemO, tmem + kTmemP + kk * 8, dv + kk * 128, idesc_pv, (jp > 0 || kk > 0) ? 1u : 0u);
       if (leader) {
-        mma_commit(&bars.pv_done);
+        mma_commit(&bars.pv_done[pb]);
         ATTN_TRACE_EVENT(3, jp);
         mma_commit(&bars.v_empty[vs]);
       }
       return true;
     };
-    for (int j = 0; ok && j < n_kv; ++j) {
+    // S(j) = Q K(j)^T into S buffer j%2, once S(j-2) has been read out of it.
+    auto issue_s = [&](int j) -> bool {
       const int ks = j % kFwdStages, sb = j & 1;
-      if (!mbar_wait_warp(&bars.k_full[ks], (j / kFwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaK)) {
-        ok = false;
-        break;
-      }
+      if (j >= 2 &&
+          !mbar_wait_warp(&bars.s_free[sb], ((j - 2) >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaS))
+        return false;
+      if (!mbar_wait_warp(&bars.k_full[ks], (j / kFwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaK))
+        return false;
+      if (leader) ATTN_TRACE_EVENT(14, j);
       tc_fence_after();
       const uint64_t dk = sdesc_sw128(smem_u32(smem + kFwdSmemK + ks * 32768), 16, 1024);  // K, K-major
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {  // K step kk: second 64-column box from kk = 4, 32 bytes per step within
+      for (int kk = 0; kk < 8; ++kk) {  // K step kk: 16 head-dim columns = 8 TMEM columns of Q; for K the
+        // second 64-column box from kk = 4, 32 bytes per step within a box
         const uint32_t koff = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-        if (leader) mma_ss(tmem + kTmemS + sb * 128, dq + koff, dk + koff, idesc_s, kk > 0 ? 1u : 0u);
+        if (leader) mma_ts(tmem + kTmemS + sb * 128, tmem + kTmemQ + kk * 8, dk + koff, idesc_s, kk > 0 ? 1u : 0u);
       }
       if (leader) {
         mma_commit(&bars.s_full[sb]);
         ATTN_TRACE_EVENT(2, j);
         mma_commit(&bars.k_empty[ks]);
       }
-      if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      return true;
+    };
+    // Issue order S(0), S(1), S(2), PV(0), S(3), PV(1), ..., PV(n-2), PV(n-1): S(j+2) goes ahead of PV(j), so
+    // the group that owns tile j finds S(j+2) ready when it finishes tile j.
+    for (int j = 0; ok && j < n_kv + 2; ++j) {
+      if (j < n_kv && !issue_s(j)) ok = false;
+      else if (j >= 2 && !issue_pv(j - 2)) ok = false;
     }
-    if (ok && issue_pv(n_kv - 1) && leader) mma_commit(&bars.o_final);
+    if (ok && leader) mma_commit(&bars.o_final);
     // Drain: wait until every MMA the leader issued has completed before tensor memory is released.
     if (leader) mma_commit(&bars.drain);
     volatile int no_abort = 0;
     mbar_wait(&bars.drain, 0, &no_abort, p.timeout_ns, &g_device_error, kSiteFwdDrain);
   } else {
     // ------------------------------------------------------------------ softmax / correction / epilogue
+    // Two warp groups take the KV tiles in turn: group g (warps 2..5 or 6..9) owns tiles j = g, g+2, ... and
+    // S buffer g. A thread holds one query row of its tile (128 keys) in registers. The online softmax is
+    // sequential only through the running max: the group publishes the max after its tile in shared memory
+    // and the other group, which has already loaded and reduced the next tile, takes it from there. So the
+    // exponentials of one tile overlap the load, max and exchange of the next, and two softmax warps per SM
+    // sub-partition keep the MUFU and FMA pipes busy.
+    const int g = (warp - 2) >> 2;
     const int quarter = warp & 3;           // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;    // query row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const float c = p.scale_log2;
-    float m = -INFINITY;  // running max of scale*log2(e)*S (possibly stale by < 2^8)
-    float l = 0.f;        // running row sum of exp2(...)
-    bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
+    float* xm = reinterpret_cast<float*>(smem + kFwdSmemXchg);  // [2 slots, by tile parity][128 rows]: running max
+    float* xl = xm + 2 * 128;                                    // [2 groups][128 rows]: partial sums, at the end
+    const bool tracer = (threadIdx.x & 127) == 64;               // one thread per group records trace events
+    float m = -INFINITY;  // running max (scale*log2(e) units, stale by < 2^8) after this group's last tile
+    float l = 0.f;        // this group's partial row sum of exp2(c*S - m)
+    // Q goes to tensor memory once, so S = Q K^T reads only K from shared memory (an MMA with both operands
+    // in shared memory runs well below the tensor rate at N = 128). Group g copies head-dim box g of its
+    // row: word w of the row (head dims 2w, 2w+1) becomes TMEM column w, the A-operand layout of the MMA.
+    bool ok = mbar_wait_warp(&bars.q_full, 0, abort, p.timeout_ns, &g_device_error, kSiteFwdSmQ);
+    if (ok) {
+      uint32_t qw[32];
+      const uint8_t* box = smem + kFwdSmemQ + g * 16384;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        const uint4 v = *reinterpret_cast<const uint4*>(box + sw128_offset(row, ch));
+        qw[ch * 4 + 0] = v.x;
+        qw[ch * 4 + 1] = v.y;
+        qw[ch * 4 + 2] = v.z;
+        qw[ch * 4 + 3] = v.w;
+      }
+      tmem_st32(tmem + lane_base + kTmemQ + 32 * g, qw);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars.q_tmem);
+    }
+    for (int j = g; ok && j < n_kv; j += 2) {
+      const int sb = g;  // = j % 2
       if (!mbar_wait_warp(&bars.s_full[sb], (j >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdSmS)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      if (threadIdx.x == 64) ATTN_TRACE_EVENT(4, j);
+      if (tracer) ATTN_TRACE_EVENT(4, j);
       float s[128];
       {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        tmem_ld32(tmem + lane_base + kTmemS + sb * 128 + 0, r0);
-        tmem_ld32(tmem + lane_base + kTmemS + sb * 128 + 32, r1);
-        tmem_ld32(tmem + lane_base + kTmemS + sb * 128 + 64, r2);
-        tmem_ld32(tmem + lane_base + kTmemS + sb * 128 + 96, r3);
-        tmem_wait_ld();
-        if (threadIdx.x == 64) ATTN_TRACE_EVENT(8, j);
+        uint32_t r[4][32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          s[i] = __uint_as_float(r0[i]);
-          s[32 + i] = __uint_as_float(r1[i]);
-          s[64 + i] = __uint_as_float(r2[i]);
-          s[96 + i] = __uint_as_float(r3[i]);
-        }
+        for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem + lane_base + kTmemS + sb * 128 + cc * 32, r[cc]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(r[cc][i]);
       }
+      tc_fence_before();
+      mbar_arrive(&bars.s_free[sb]);  // S(j+2) may now be written over this buffer
+      if (lane == 0 && j < 8) ATTN_TRACE_EVENT(12, j * 8 + warp - 2);
+      if (tracer) ATTN_TRACE_EVENT(8, j);
       if (j == qt) {  // diagonal tile: key column > query row is masked
 #pragma unroll
         for (int i = 0; i < 128; ++i)
           if (i > row) s[i] = -INFINITY;
       }
-      // Row max as a tree over 16 independent partial maxima (a single 128-long dependent chain would leave
-      // ~500 cycles of latency exposed: there is one softmax warp per SM sub-partition).
+      // Row max of the tile as a tree over 16 independent partial maxima.
       float pm[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) pm[i] = s[i];
@@ -274,23 +345,63 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int i = 0; i < w; ++i) pm[i] = fmaxf(pm[i], pm[i + w]);
       const float m_tile = pm[0] * c;
-      if (threadIdx.x == 64) ATTN_TRACE_EVENT(11, j);
-      if (j == 0) {
-        m = m_tile;
-      } else if (const bool need = m_tile > m + kRescaleThreshold; __any_sync(0xffffffffu, need)) {
-        // Some row of this warp saw its running max grow by more than 2^8. TMEM access is warp-collective,
-        // so the whole warp walks its rows of O, but only the rows that crossed the threshold change: the
-        // others keep their max and get alpha = 1 exactly, so every row's arithmetic is independent of its
-        // neighbours (outputs before a position do not depend on inputs after it, bit for bit).
-        // O may be touched only after PV(j-1) has landed: S(j) completing implies PV(j-2) completed, and
-        // PV(j) is not issued yet, so pv_done is within one phase of j-1 and the parity wait is unambiguous.
-        const float m_new = need ? m_tile : m;
-        const float alpha = need ? ex2(m - m_new) : 1.0f;
-        if (!mbar_wait_warp(&bars.pv_done, (j - 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdSmPV)) {
+      // Running max after tile j-1, from the other group. A slot is rewritten two tiles later only after its
+      // reader has published the tile in between, so one phase of xchg per tile suffices.
+      float m_prev = -INFINITY;
+      if (j > 0) {
+        if (!mbar_wait_warp(&bars.xchg[sb ^ 1], ((j - 1) >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdSmX)) {
+          ok = false;
+          break;
+        }
+        m_prev = xm[(sb ^ 1) * 128 + row];
+      }
+      // Lazy rescaling: the running max moves only when the tile's max exceeds it by more than 2^8 (always on
+      // tile 0). Each row decides for itself, so a row's arithmetic never depends on another row's inputs
+      // (outputs before a position do not depend on inputs after it, bit for bit).
+      const bool need = m_tile > m_prev + kRescaleThreshold;
+      const float m_j = need ? m_tile : m_prev;
+      xm[sb * 128 + row] = m_j;
+      mbar_arrive(&bars.xchg[sb]);
+      if (tracer) ATTN_TRACE_EVENT(11, j);
+      // P = exp2(c*S - m_j) for the 128 keys and the row sum, packed to bf16 pairs in registers. The last
+      // kFwdPolyPairs pairs of every 16 go through the FMA-pipe exp2 (exp2_poly), the rest through MUFU ex2.
+      const float neg_m = -m_j;
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial row sums
+      uint32_t pk[4][16];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float x0 = fmaf(s[cc * 32 + 2 * i], c, neg_m), x1 = fmaf(s[cc * 32 + 2 * i + 1], c, neg_m);
+          const bool poly = i >= 16 - kFwdPolyPairs;
+          const float p0 = poly ? exp2_poly(x0) : ex2(x0);
+          const float p1 = poly ? exp2_poly(x1) : ex2(x1);
+          ps[(2 * i) & 7] += p0;
+          ps[(2 * i + 1) & 7] += p1;
+          pk[cc][i] = pack_bf16x2(p0, p1);
+        }
+      }
+      const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      l = (m == m_j ? l : l * ex2(m - m_j)) + rs;  // this group's sum was relative to its previous max
+      m = m_j;
+      if (tracer) ATTN_TRACE_EVENT(9, j);
+      // The P buffer and O are free once PV(j-1) has landed. PV(j-3) landed before S(j) (issue order) and
+      // PV(j+1) waits for PV(j), which waits for this group, so pv_done[sb^1] is within one phase of j-1.
+      if (j > 0) {
+        if (!mbar_wait_warp(&bars.pv_done[sb ^ 1], ((j - 1) >> 1) & 1, abort, p.timeout_ns, &g_device_error,
+                            kSiteFwdSmPV)) {
           ok = false;
           break;
         }
         tc_fence_after();
+      }
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_st16(tmem + lane_base + kTmemP + cc * 16, pk[cc]);
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // Some row of this warp moved its max: O (tiles 0..j-1, relative to m_prev) is scaled by
+        // 2^(m_prev - m_j) before PV(j) is issued. TMEM access is warp-collective, so the whole warp walks its
+        // rows; rows that kept their max get alpha = 1 exactly.
+        const float alpha = need ? ex2(m_prev - m_j) : 1.0f;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t o[32];
@@ -300,49 +411,36 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           tmem_st32(tmem + lane_base + kTmemO + cc * 32, o);
         }
-        l *= alpha;
-        m = m_new;
       }
-      // P = exp2(c*S - m), row sum, pack to bf16 pairs into the P buffer of this tile.
-      const float neg_m = -m;
-      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial row sums
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(fmaf(s[cc * 32 + 2 * i], c, neg_m));
-          const float p1 = ex2(fmaf(s[cc * 32 + 2 * i + 1], c, neg_m));
-          ps[(2 * i) & 7] += p0;
-          ps[(2 * i + 1) & 7] += p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(tmem + lane_base + kTmemP + sb * 64 + cc * 16, pk);
-      }
-      l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      if (threadIdx.x == 64) ATTN_TRACE_EVENT(9, j);
       tmem_wait_st();
-      if (threadIdx.x == 64) ATTN_TRACE_EVENT(10, j);
+      if (tracer) ATTN_TRACE_EVENT(10, j);
       tc_fence_before();
       mbar_arrive(&bars.p_full[sb]);
-      if (threadIdx.x == 64) ATTN_TRACE_EVENT(5, j);
+      if (tracer) ATTN_TRACE_EVENT(5, j);
+      if (lane == 0 && j < 8) ATTN_TRACE_EVENT(13, j * 8 + warp - 2);
     }
     // Epilogue: O / l -> bf16 -> swizzled staging (reusing the Q buffer) -> TMA store; LSE in natural log.
-    // Every thread of the group reaches the named barrier, failed or not; the store is skipped on abort.
-    if (threadIdx.x == 64) ATTN_TRACE_EVENT(6, 0);
+    // The final running max is the one published for the last tile; each group brings its partial sum to it
+    // and the two are added. Every thread of both groups reaches the named barriers, failed or not; the
+    // store is skipped on abort.
+    if (tracer) ATTN_TRACE_EVENT(6, g);
+    named_barrier(1, 256);
+    const float m_f = xm[((n_kv - 1) & 1) * 128 + row];
+    xl[g * 128 + row] = m == m_f ? l : l * ex2(m - m_f);  // a group without tiles has l = 0, m = -inf
+    named_barrier(1, 256);
+    const float l_row = xl[row] + xl[128 + row];
     const bool epi_ok =
         __all_sync(0xffffffffu, ok) && mbar_wait_warp(&bars.o_final, 0, abort, p.timeout_ns, &g_device_error, kSiteFwdEpi);
     if (epi_ok) {
       if (threadIdx.x == 64) ATTN_TRACE_EVENT(7, 0);
       tc_fence_after();
-      const float inv_l = 1.0f / l;
-      uint8_t* stage = smem + kFwdSmemQ;
+      const float inv_l = 1.0f / l_row;
+      uint8_t* box = smem + kFwdSmemQ + g * 16384;  // this group's 64 head-dim columns = one 64-column box
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t o[32];
-        tmem_ld32(tmem + lane_base + kTmemO + cc * 32, o);
+        tmem_ld32(tmem + lane_base + kTmemO + 64 * g + cc * 32, o);
         tmem_wait_ld();
-        uint8_t* box = stage + (cc >> 1) * 16384;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
           uint4 v;
@@ -350,19 +448,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           v.y = pack_bf16x2(__uint_as_float(o[ch * 8 + 2]) * inv_l, __uint_as_float(o[ch * 8 + 3]) * inv_l);
           v.z = pack_bf16x2(__uint_as_float(o[ch * 8 + 4]) * inv_l, __uint_as_float(o[ch * 8 + 5]) * inv_l);
           v.w = pack_bf16x2(__uint_as_float(o[ch * 8 + 6]) * inv_l, __uint_as_float(o[ch * 8 + 7]) * inv_l);
-          *reinterpret_cast<uint4*>(box + sw128_offset(row, (cc & 1) * 4 + ch)) = v;
+          *reinterpret_cast<uint4*>(box + sw128_offset(row, cc * 4 + ch)) = v;
         }
       }
       const int t = q0 + row;
-      if (t < p.T) p.lse[static_cast<size_t>(bh) * p.T + t] = (m + __log2f(l)) * 0.69314718055994531f;
+      if (g == 0 && t < p.T) p.lse[static_cast<size_t>(bh) * p.T + t] = (m_f + __log2f(l_row)) * 0.69314718055994531f;
     }
     fence_async_shared();
-    named_barrier(1, 128);
+    named_barrier(1, 256);
     if (warp == 2 && lane == 0 && !*abort) {
       for (int cc = 0; cc < 2; ++cc) tma_store_4d(&tm_o, smem + kFwdSmemQ + cc * 16384, cc * 64, h, q0, b);
       tma_store_commit();
       tma_store_wait_read_all();
-      ATTN_TRACE_EVENT(6, 1);
+      ATTN_TRACE_EVENT(6, 2);
     }
   }
 
