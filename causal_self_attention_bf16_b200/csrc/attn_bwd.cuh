@@ -201,9 +201,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars.s_full[s], 1);
-      mbar_init(&bars.p_full[s], 128);
+      mbar_init(&bars.p_full[s], 4);    // counts the warps of one softmax group
       mbar_init(&bars.dq_full[s], 1);
-      mbar_init(&bars.dq_empty[s], 128);
+      mbar_init(&bars.dq_empty[s], 4);  // likewise
       mbar_init(&bars.b_done[s], 1);
     }
     mbar_init(&bars.stage_free, 1);
@@ -425,7 +425,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       fence_async_shared();
       if (threadIdx.x == 64) ATTN_TRACE_EVENT(11, i);
       tc_fence_before();
-      mbar_arrive(&bars.p_full[rb]);
+      mbar_arrive_warp(&bars.p_full[rb]);
       if (threadIdx.x == 64 || threadIdx.x == 192) ATTN_TRACE_EVENT(5, i);
 
       // dQ^T of this tile (thread = d, 64 query columns) -> staging buffer in the accumulator's [q/4][d][4]
@@ -442,7 +442,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       tmem_ld32(tmem + lane_base + kTmemR + rb * 128 + 96, a[1]);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&bars.dq_empty[rb]);  // dQ^T is in registers: the tensor-memory buffer is free
+      mbar_arrive_warp(&bars.dq_empty[rb]);  // dQ^T is in registers: the tensor-memory buffer is free
       if (i > 0 && !mbar_wait_warp(&bars.stage_free, (i - 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdDq)) {
         ok = false;
         break;

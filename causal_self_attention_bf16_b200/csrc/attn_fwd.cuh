@@ -130,7 +130,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
-    mbar_init(&bars.q_tmem, 256);
+    mbar_init(&bars.q_tmem, 8);  // counts warps (one arrival per softmax warp)
     for (int s = 0; s < kFwdStages; ++s) {
       mbar_init(&bars.k_full[s], 1);
       mbar_init(&bars.k_empty[s], 1);
@@ -139,9 +139,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars.s_full[s], 1);
-      mbar_init(&bars.s_free[s], 128);
-      mbar_init(&bars.p_full[s], 128);
-      mbar_init(&bars.xchg[s], 128);
+      mbar_init(&bars.s_free[s], 4);  // these three count the warps of one softmax group
+      mbar_init(&bars.p_full[s], 4);
+      mbar_init(&bars.xchg[s], 4);
       mbar_init(&bars.pv_done[s], 1);
     }
     mbar_init(&bars.o_final, 1);
@@ -304,7 +304,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tmem_st32(tmem + lane_base + kTmemQ + 32 * g, qw);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars.q_tmem);
+      mbar_arrive_warp(&bars.q_tmem);
     }
     for (int j = g; ok && j < n_kv; j += 2) {
       const int sb = g;  // = j % 2
@@ -326,7 +326,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(r[cc][i]);
       }
       tc_fence_before();
-      mbar_arrive(&bars.s_free[sb]);  // S(j+2) may now be written over this buffer
+      mbar_arrive_warp(&bars.s_free[sb]);  // S(j+2) may now be written over this buffer
       if (lane == 0 && j < 8) ATTN_TRACE_EVENT(12, j * 8 + warp - 2);
       if (tracer) ATTN_TRACE_EVENT(8, j);
       if (j == qt) {  // diagonal tile: key column > query row is masked
@@ -361,7 +361,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const bool need = m_tile > m_prev + kRescaleThreshold;
       const float m_j = need ? m_tile : m_prev;
       xm[sb * 128 + row] = m_j;
-      mbar_arrive(&bars.xchg[sb]);
+      mbar_arrive_warp(&bars.xchg[sb]);
       if (tracer) ATTN_TRACE_EVENT(11, j);
       // P = exp2(c*S - m_j) for the 128 keys and the row sum, packed to bf16 pairs in registers. The last
       // kFwdPolyPairs pairs of every 16 go through the FMA-pipe exp2 (exp2_poly), the rest through MUFU ex2.
@@ -415,7 +415,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tmem_wait_st();
       if (tracer) ATTN_TRACE_EVENT(10, j);
       tc_fence_before();
-      mbar_arrive(&bars.p_full[sb]);
+      mbar_arrive_warp(&bars.p_full[sb]);
       if (tracer) ATTN_TRACE_EVENT(5, j);
       if (lane == 0 && j < 8) ATTN_TRACE_EVENT(13, j * 8 + warp - 2);
     }

@@ -113,6 +113,15 @@ ATTN_DEVICE_INLINE bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* 
   }
 }
 
+// One arrival for the whole warp: the lanes synchronise, which orders their earlier writes (and, after a
+// tcgen05.fence::before_thread_sync, their tensor-memory accesses) before lane 0's release-arrive, so the
+// barrier counts warps. All 32 lanes must call it together. (Arrivals are atomics on one shared-memory word:
+// 128 per phase, one per thread, serialise into hundreds of cycles on a critical path.)
+ATTN_DEVICE_INLINE void mbar_arrive_warp(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 // Warp-uniform form of mbar_wait for roles in which the whole warp then issues warp-collective tcgen05.ld/st
 // (.sync.aligned): every lane waits, and the warp proceeds only if every lane succeeded, so a failure can
 // never leave part of a warp inside a collective. All 32 lanes must call it together.
