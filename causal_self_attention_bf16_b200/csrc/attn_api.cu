@@ -88,6 +88,8 @@ attn_status check_sizes(int B, int H, int T, int D, float scale) {
 }
 
 // Set the dynamic shared-memory opt-in of both big kernels once per device.
+int g_sm_count[64] = {};  // multiprocessors per device, set by prepare_device
+
 attn_status prepare_device(int* dev_out) {
   static std::mutex mu;
   static bool done[64] = {};
@@ -104,6 +106,10 @@ attn_status prepare_device(int* dev_out) {
   if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
       (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
     return cuda_fail(e, "cudaDeviceGetAttribute");
+  int sms = 0;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return cuda_fail(e, "cudaDeviceGetAttribute");
+  if (dev >= 0 && dev < 64) g_sm_count[dev] = sms;
   if (major != 10 || minor != 0) {
     std::snprintf(g_cuda_error, sizeof(g_cuda_error), "device %d is sm_%d%d; this library is built for sm_100a",
                   dev, major, minor);
@@ -212,8 +218,10 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   p.T = T;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_wait_limit_ns;
-  const unsigned n_qt = static_cast<unsigned>((T + attn::kTile - 1) / attn::kTile);
-  const dim3 grid(n_qt * static_cast<unsigned>(B * H));
+  // Persistent grid: one CTA per SM (fewer when there are fewer work items).
+  const long long n_items = static_cast<long long>((T + attn::kTile - 1) / attn::kTile) * B * H;
+  const int sms = (dev >= 0 && dev < 64 && g_sm_count[dev] > 0) ? g_sm_count[dev] : 148;
+  const dim3 grid(static_cast<unsigned>(n_items < sms ? n_items : sms));
   attn::attn_fwd_kernel<<<grid, attn::kFwdThreads, attn::kFwdSmemAlloc, static_cast<cudaStream_t>(stream)>>>(
       mq, mk, mv, mo, p);
   cudaError_t e = cudaGetLastError();

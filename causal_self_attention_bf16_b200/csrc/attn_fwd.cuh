@@ -5,8 +5,9 @@
 // own ChatGPT", section 5 "Flash Attention integration"; layout from section 1 "GPT model") and name the
 // Hopper Flash-Attention-3 kernel as the implementation. This kernel is a new design for Blackwell:
 //
-//   * one CTA per (128-query tile, batch, head), head-major so a head's K/V stay in L2 while its tiles run,
-//     heaviest (latest) query tile of each head first;
+//   * persistent: one CTA per SM walks work items (128-query tile, batch, head) in head-major order, so the
+//     K/V of the few heads in flight stay in L2; the rings run on across items, so the next item's loads
+//     and first S tiles overlap the current item's tail and epilogue;
 //   * warp 0 stages Q once and K tiles, warp 10 V tiles (three-deep rings) with TMA into 128-byte-swizzled
 //     shared memory;
 //   * warp 1 issues tcgen05.mma with the A operand in tensor memory: S = Q K^T (Q copied into tensor memory
@@ -18,7 +19,8 @@
 //     groups (through shared memory), so one tile's exponentials overlap the next tile's load and max. A
 //     thread owns a whole row of S, so row max and row sum need no shuffles; masking happens only on the
 //     diagonal tile (tiles above it are skipped); O is rescaled lazily, only when the running max grows by
-//     more than 2^8; the epilogue normalises O, stages it in shared memory and writes it with a TMA store.
+//     more than 2^8; the epilogue normalises O, stages it in the (by then free) Q buffer and writes it with a
+//     TMA store.
 //
 // Tensor memory (512 columns): S double buffer [0,256) (buffer j%2 belongs to the group of tile j), O
 // [256,384), Q (bf16 pairs) [384,448), P (bf16 pairs) [448,512). The MMA warp issues S(j+2) as soon as S(j)
@@ -32,8 +34,9 @@ namespace attn {
 
 constexpr int kTile = 128;        // query rows per CTA and keys per KV tile
 constexpr int kHeadDim = 128;     // D
-constexpr int kFwdThreads = 352;  // warp 0 TMA (Q, K), warp 1 MMA, warps 2..9 two softmax groups, warp 10 TMA (V)
-constexpr int kFwdWarpV = 10;
+constexpr int kFwdThreads = 384;  // warp 0 TMA (Q, K), warp 1 MMA, warps 2..9 two softmax groups, warp 10 TMA (V),
+                                  // warp 11 TMA store of O
+constexpr int kFwdWarpV = 10, kFwdWarpStore = 11;
 
 // Shared-memory layout of the forward kernel (offsets from a 1024-byte aligned base).
 constexpr uint32_t kFwdSmemQ = 0;                       // 32 KB: Q tile, two 64-column boxes of 16 KB
@@ -78,6 +81,8 @@ struct FwdParams {
 struct FwdBarriers {
   uint64_t q_full;
   uint64_t q_tmem;      // Q copied from shared into tensor memory by the softmax warps
+  uint64_t o_staged;    // both softmax groups have staged the item's output in the Q buffer
+  uint64_t q_free;      // the Q buffer's other use, staging an item's output for its TMA store, is over
   uint64_t k_full[kFwdStages], k_empty[kFwdStages];
   uint64_t v_full[kFwdStages], v_empty[kFwdStages];
   uint64_t s_full[2];   // S(j) landed in buffer j%2
@@ -98,10 +103,29 @@ static_assert(kFwdSmemAlloc <= 232448, "forward kernel exceeds the 227 KB shared
 // Error sites (recorded with a timeout in the device error word): 0x10 + barrier id, per role.
 enum : uint32_t {
   kSiteFwdLayout = 0x10, kSiteFwdProdKEmpty = 0x11, kSiteFwdProdVEmpty = 0x12, kSiteFwdMmaQ = 0x21, kSiteFwdMmaK = 0x22,
-  kSiteFwdMmaP = 0x23, kSiteFwdMmaV = 0x24, kSiteFwdMmaS = 0x25, kSiteFwdSmS = 0x31, kSiteFwdSmPV = 0x32, kSiteFwdEpi = 0x33, kSiteFwdSmX = 0x35, kSiteFwdSmQ = 0x36,
+  kSiteFwdMmaP = 0x23, kSiteFwdMmaV = 0x24, kSiteFwdMmaS = 0x25, kSiteFwdSmS = 0x31, kSiteFwdSmPV = 0x32, kSiteFwdEpi = 0x33, kSiteFwdSmX = 0x35, kSiteFwdSmQ = 0x36, kSiteFwdProdQ = 0x13, kSiteFwdStore = 0x14,
   kSiteFwdDrain = 0x34
 };
 
+// Work item k of this CTA. Items are (batch*head, query tile) pairs in head-major order, the heaviest query
+// tile of each head first. They are dealt to the G CTAs in rounds of G that alternate direction (item k*G + c
+// on even rounds, k*G + G-1-c on odd ones): that balances the causal work per CTA to within a few percent,
+// and the items in flight at any time cover only ~G/n_qt heads, whose K/V stay in L2.
+struct FwdItem {
+  int bh, qt;
+};
+__device__ __forceinline__ bool fwd_item(int k, int n_items, int n_qt, FwdItem& it) {
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  const long long idx = static_cast<long long>(k) * G + ((k & 1) ? G - 1 - c : c);
+  if (idx >= n_items) return false;
+  it.bh = static_cast<int>(idx / n_qt);
+  it.qt = n_qt - 1 - static_cast<int>(idx % n_qt);
+  return true;
+}
+
+// Persistent: one CTA per SM walks its work items. Every ring and buffer index is a running count over the
+// CTA's KV tiles (t) or items (k), so the producers stream the next item's Q, K and V while the current
+// item is computed, and the next item's first S tiles run while the current item's output is written.
 __global__ void __launch_bounds__(kFwdThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -119,18 +143,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int n_qt = (p.T + kTile - 1) / kTile;
-  // Head-major order, heaviest (latest) query tile first within a head: the CTAs in flight at any time
-  // cover only ~10 heads, so their K/V stay in L2 while every query tile of the head reads them.
-  const int bh = static_cast<int>(blockIdx.x / n_qt);
-  const int qt = n_qt - 1 - static_cast<int>(blockIdx.x % n_qt);
-  const int b = bh / p.H, h = bh % p.H;
-  const int q0 = qt * kTile;
-  const int n_kv = qt + 1;  // causal: KV tiles 0..qt
+  const int n_items = p.B * p.H * n_qt;
   volatile int* abort = &bars.abort;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
-    mbar_init(&bars.q_tmem, 8);  // counts warps (one arrival per softmax warp)
+    mbar_init(&bars.q_tmem, 8);  // counts warps (each softmax warp copies its rows of one head-dim half)
+    mbar_init(&bars.o_staged, 8);  // counts warps
+    mbar_init(&bars.q_free, 1);
     for (int s = 0; s < kFwdStages; ++s) {
       mbar_init(&bars.k_full[s], 1);
       mbar_init(&bars.k_empty[s], 1);
@@ -173,35 +193,78 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint8_t* ring = smem + (is_k ? kFwdSmemK : kFwdSmemV);
     if (leader) {
       tma_prefetch_desc(tm);
-      if (is_k) {
-        tma_prefetch_desc(&tm_q);
-        mbar_arrive_expect_tx(&bars.q_full, 2 * 16384);
-        for (int c = 0; c < 2; ++c) tma_load_4d(smem + kFwdSmemQ + c * 16384, &tm_q, &bars.q_full, c * 64, h, q0, b);
-      }
+      if (is_k) tma_prefetch_desc(&tm_q);
     }
     int issued[kFwdStages];
     for (int s = 0; s < kFwdStages; ++s) issued[s] = -1;
-    for (int j = 0; j < n_kv; ++j) {
-      const int s = j % kFwdStages;
-      if (j >= kFwdStages && !mbar_wait_warp(&empty[s], ((j - kFwdStages) / kFwdStages) & 1, abort, p.timeout_ns,
-                                             &g_device_error, is_k ? kSiteFwdProdKEmpty : kSiteFwdProdVEmpty))
-        break;
-      if (leader) {
-        mbar_arrive_expect_tx(&full[s], 2 * 16384);
-        for (int c = 0; c < 2; ++c) tma_load_4d(ring + s * 32768 + c * 16384, tm, &full[s], c * 64, h, j * kTile, b);
-        if (is_k) ATTN_TRACE_EVENT(1, j);
+    int q_issued = -1;
+    int t0 = 0;  // running KV tile count: ring slot t % kFwdStages, phase (t / kFwdStages) & 1
+    FwdItem it;
+    for (int k = 0; fwd_item(k, n_items, n_qt, it); ++k) {
+      const int b = it.bh / p.H, h = it.bh % p.H, n_kv = it.qt + 1;
+      if (is_k) {
+        // One Q buffer, which also stages each item's output for its TMA store. Q(1) may go in once Q(0) is in
+        // tensor memory; Q(k), k >= 2, once item k-2's output has been read out of the buffer by its store
+        // (which follows the copy of Q(k-1) into tensor memory in the same epilogue).
+        if (k == 1 && !mbar_wait_warp(&bars.q_tmem, 0, abort, p.timeout_ns, &g_device_error, kSiteFwdProdQ)) break;
+        if (k >= 2 &&
+            !mbar_wait_warp(&bars.q_free, (k - 2) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdProdQ))
+          break;
+        if (leader) {
+          mbar_arrive_expect_tx(&bars.q_full, 2 * 16384);
+          for (int c = 0; c < 2; ++c)
+            tma_load_4d(smem + kFwdSmemQ + c * 16384, &tm_q, &bars.q_full, c * 64, h, it.qt * kTile, b);
+        }
+        q_issued = k;
       }
-      issued[s] = j;
+      bool ok = true;
+      for (int j = 0; j < n_kv; ++j) {
+        const int t = t0 + j, s = t % kFwdStages;
+        if (t >= kFwdStages && !mbar_wait_warp(&empty[s], ((t - kFwdStages) / kFwdStages) & 1, abort, p.timeout_ns,
+                                               &g_device_error, is_k ? kSiteFwdProdKEmpty : kSiteFwdProdVEmpty)) {
+          ok = false;
+          break;
+        }
+        if (leader) {
+          mbar_arrive_expect_tx(&full[s], 2 * 16384);
+          for (int c = 0; c < 2; ++c) tma_load_4d(ring + s * 32768 + c * 16384, tm, &full[s], c * 64, h, j * kTile, b);
+          if (is_k) ATTN_TRACE_EVENT(1, t);
+        }
+        issued[s] = t;
+      }
+      if (!ok) break;
+      t0 += n_kv;
     }
     if (*abort) {
       // Let every copy this warp started land before the CTA's shared memory is released.
       volatile int no_abort = 0;
       const uint64_t lim = p.timeout_ns;
-      if (is_k) mbar_wait(&bars.q_full, 0, &no_abort, lim, &g_device_error, kSiteFwdDrain);
+      if (q_issued >= 0) mbar_wait(&bars.q_full, q_issued & 1, &no_abort, lim, &g_device_error, kSiteFwdDrain);
       for (int s = 0; s < kFwdStages; ++s)
         if (issued[s] >= 0)
           mbar_wait(&full[s], (issued[s] / kFwdStages) & 1, &no_abort, lim, &g_device_error, kSiteFwdDrain);
     }
+  } else if (warp == kFwdWarpStore) {
+    // ------------------------------------------------------------------ output store
+    // Once both softmax groups have staged an item's output in the Q buffer, one elected lane writes it with
+    // two TMA stores (rows past T are clipped) and frees the buffer for the next Q as soon as the stores
+    // have read it. Kept off the softmax warps, whose next tile would otherwise wait for the store.
+    const bool leader = elect_one();
+    if (leader) tma_prefetch_desc(&tm_o);
+    FwdItem it;
+    for (int k = 0; fwd_item(k, n_items, n_qt, it); ++k) {
+      if (!mbar_wait_warp(&bars.o_staged, k & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdStore)) break;
+      if (__any_sync(0xffffffffu, *abort != 0)) break;  // warp-uniform: the loop ends in a __syncwarp
+      if (leader) {
+        for (int c = 0; c < 2; ++c)
+          tma_store_4d(&tm_o, smem + kFwdSmemQ + c * 16384, c * 64, it.bh % p.H, it.qt * kTile, it.bh / p.H);
+        tma_store_commit();
+        tma_store_wait_read_all();
+        mbar_arrive(&bars.q_free);
+      }
+      __syncwarp();
+    }
+    if (leader) tma_store_wait_read_all();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     // The whole warp walks the schedule and computes the descriptors (warp-uniform, so they live in uniform
@@ -210,38 +273,38 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const bool leader = elect_one();
     const uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);  // Q (TMEM) x K (K-major)
     const uint32_t idesc_pv = idesc_bf16_f32(128, 128, false, true);  // P (TMEM) x V (MN-major)
-    // Descriptors are built once per operand and advanced by adding byte offsets in 16-byte units to the
+    // Descriptors are built per ring slot and advanced by adding byte offsets in 16-byte units to the
     // start-address field (one 64-bit add per K step; the tiles stay below 256 KB).
-    bool ok = mbar_wait_warp(&bars.q_tmem, 0, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaQ);
-    // PV(jp): O += P(jp) V(jp); P from tensor memory, V from ring slot jp % kFwdStages.
-    auto issue_pv = [&](int jp) -> bool {
-      const int pb = jp & 1, vs = jp % kFwdStages;
-      if (!mbar_wait_warp(&bars.p_full[pb], (jp >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaP))
+    // PV(t): O += P(t) V(t) (the first tile of an item overwrites O); P from tensor memory, V from ring slot
+    // t % kFwdStages.
+    auto issue_pv = [&](int t, bool first) -> bool {
+      const int pb = t & 1, vs = t % kFwdStages;
+      if (!mbar_wait_warp(&bars.p_full[pb], (t >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaP))
         return false;
-      if (!mbar_wait_warp(&bars.v_full[vs], (jp / kFwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaV))
+      if (!mbar_wait_warp(&bars.v_full[vs], (t / kFwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaV))
         return false;
-      if (leader) ATTN_TRACE_EVENT(15, jp);
+      if (leader) ATTN_TRACE_EVENT(15, t);
       tc_fence_after();
       const uint64_t dv = sdesc_sw128(smem_u32(smem + kFwdSmemV + vs * 32768), 16384, 1024);  // V, MN-major
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)  // K step kk: 16 keys = 2048 bytes further (128 in 16-byte units)
-        if (leader) mma_ts(tmem + kTmemO, tmem + kTmemP + kk * 8, dv + kk * 128, idesc_pv, (jp > 0 || kk > 0) ? 1u : 0u);
+        if (leader) mma_ts(tmem + kTmemO, tmem + kTmemP + kk * 8, dv + kk * 128, idesc_pv, (!first || kk > 0) ? 1u : 0u);
       if (leader) {
         mma_commit(&bars.pv_done[pb]);
-        ATTN_TRACE_EVENT(3, jp);
+        ATTN_TRACE_EVENT(3, t);
         mma_commit(&bars.v_empty[vs]);
       }
       return true;
     };
-    // S(j) = Q K(j)^T into S buffer j%2, once S(j-2) has been read out of it.
-    auto issue_s = [&](int j) -> bool {
-      const int ks = j % kFwdStages, sb = j & 1;
-      if (j >= 2 &&
-          !mbar_wait_warp(&bars.s_free[sb], ((j - 2) >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaS))
+    // S(t) = Q K(t)^T into S buffer t%2, once S(t-2) has been read out of it.
+    auto issue_s = [&](int t) -> bool {
+      const int ks = t % kFwdStages, sb = t & 1;
+      if (t >= 2 &&
+          !mbar_wait_warp(&bars.s_free[sb], ((t - 2) >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaS))
         return false;
-      if (!mbar_wait_warp(&bars.k_full[ks], (j / kFwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaK))
+      if (!mbar_wait_warp(&bars.k_full[ks], (t / kFwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaK))
         return false;
-      if (leader) ATTN_TRACE_EVENT(14, j);
+      if (leader) ATTN_TRACE_EVENT(14, t);
       tc_fence_after();
       const uint64_t dk = sdesc_sw128(smem_u32(smem + kFwdSmemK + ks * 32768), 16, 1024);  // K, K-major
 #pragma unroll
@@ -252,30 +315,39 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       if (leader) {
         mma_commit(&bars.s_full[sb]);
-        ATTN_TRACE_EVENT(2, j);
+        ATTN_TRACE_EVENT(2, t);
         mma_commit(&bars.k_empty[ks]);
       }
       return true;
     };
-    // Issue order S(0), S(1), S(2), PV(0), S(3), PV(1), ..., PV(n-2), PV(n-1): S(j+2) goes ahead of PV(j), so
-    // the group that owns tile j finds S(j+2) ready when it finishes tile j.
-    for (int j = 0; ok && j < n_kv + 2; ++j) {
-      if (j < n_kv && !issue_s(j)) ok = false;
-      else if (j >= 2 && !issue_pv(j - 2)) ok = false;
+    bool ok = true;
+    int t0 = 0;
+    FwdItem it;
+    for (int k = 0; ok && fwd_item(k, n_items, n_qt, it); ++k) {
+      const int n_kv = it.qt + 1;
+      // This item's Q is in tensor memory (copied once the previous item's MMAs had completed).
+      if (!mbar_wait_warp(&bars.q_tmem, k & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaQ)) break;
+      // Issue order S(0), S(1), S(2), PV(0), S(3), PV(1), ..., PV(n-2), PV(n-1) (tile indices within the
+      // item): S(j+2) goes ahead of PV(j), so the group that owns tile j finds S(j+2) ready when it is done.
+      for (int j = 0; ok && j < n_kv + 2; ++j) {
+        if (j < n_kv && !issue_s(t0 + j)) ok = false;
+        else if (j >= 2 && !issue_pv(t0 + j - 2, j == 2)) ok = false;
+      }
+      if (ok && leader) mma_commit(&bars.o_final);
+      t0 += n_kv;
     }
-    if (ok && leader) mma_commit(&bars.o_final);
     // Drain: wait until every MMA the leader issued has completed before tensor memory is released.
     if (leader) mma_commit(&bars.drain);
     volatile int no_abort = 0;
     mbar_wait(&bars.drain, 0, &no_abort, p.timeout_ns, &g_device_error, kSiteFwdDrain);
   } else {
     // ------------------------------------------------------------------ softmax / correction / epilogue
-    // Two warp groups take the KV tiles in turn: group g (warps 2..5 or 6..9) owns tiles j = g, g+2, ... and
-    // S buffer g. A thread holds one query row of its tile (128 keys) in registers. The online softmax is
-    // sequential only through the running max: the group publishes the max after its tile in shared memory
-    // and the other group, which has already loaded and reduced the next tile, takes it from there. So the
-    // exponentials of one tile overlap the load, max and exchange of the next, and two softmax warps per SM
-    // sub-partition keep the MUFU and FMA pipes busy.
+    // Two warp groups take the KV tiles in turn: group g (warps 2..5 or 6..9) owns the tiles whose running
+    // index t is g modulo 2, and S buffer g. A thread holds one query row of its tile (128 keys) in registers.
+    // The online softmax is sequential only through the running max: the group publishes the max after its
+    // tile in shared memory and the other group, which has already loaded and reduced the next tile, takes
+    // it from there. So the exponentials of one tile overlap the load, max and exchange of the next, and two
+    // softmax warps per SM sub-partition keep the MUFU and FMA pipes busy.
     const int g = (warp - 2) >> 2;
     const int quarter = warp & 3;           // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;    // query row within the tile
@@ -284,13 +356,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float* xm = reinterpret_cast<float*>(smem + kFwdSmemXchg);  // [2 slots, by tile parity][128 rows]: running max
     float* xl = xm + 2 * 128;                                    // [2 groups][128 rows]: partial sums, at the end
     const bool tracer = (threadIdx.x & 127) == 64;               // one thread per group records trace events
-    float m = -INFINITY;  // running max (scale*log2(e) units, stale by < 2^8) after this group's last tile
-    float l = 0.f;        // this group's partial row sum of exp2(c*S - m)
-    // Q goes to tensor memory once, so S = Q K^T reads only K from shared memory (an MMA with both operands
-    // in shared memory runs well below the tensor rate at N = 128). Group g copies head-dim box g of its
-    // row: word w of the row (head dims 2w, 2w+1) becomes TMEM column w, the A-operand layout of the MMA.
-    bool ok = mbar_wait_warp(&bars.q_full, 0, abort, p.timeout_ns, &g_device_error, kSiteFwdSmQ);
-    if (ok) {
+    // Q of item k goes to tensor memory, so S = Q K^T reads only K from shared memory (an MMA with both
+    // operands in shared memory runs well below the tensor rate at N = 128). Group g copies head-dim box g of
+    // its row: word w of the row (head dims 2w, 2w+1) becomes TMEM column w, the A-operand layout.
+    auto copy_q = [&](int k) -> bool {
+      if (!mbar_wait_warp(&bars.q_full, k & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdSmQ)) return false;
       uint32_t qw[32];
       const uint8_t* box = smem + kFwdSmemQ + g * 16384;
 #pragma unroll
@@ -305,162 +375,192 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(&bars.q_tmem);
-    }
-    for (int j = g; ok && j < n_kv; j += 2) {
-      const int sb = g;  // = j % 2
-      if (!mbar_wait_warp(&bars.s_full[sb], (j >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdSmS)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (tracer) ATTN_TRACE_EVENT(4, j);
-      float s[128];
-      {
-        uint32_t r[4][32];
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem + lane_base + kTmemS + sb * 128 + cc * 32, r[cc]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(r[cc][i]);
-      }
-      tc_fence_before();
-      mbar_arrive_warp(&bars.s_free[sb]);  // S(j+2) may now be written over this buffer
-      if (lane == 0 && j < 8) ATTN_TRACE_EVENT(12, j * 8 + warp - 2);
-      if (tracer) ATTN_TRACE_EVENT(8, j);
-      if (j == qt) {  // diagonal tile: key column > query row is masked
-#pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i > row) s[i] = -INFINITY;
-      }
-      // Row max of the tile as a tree over 16 independent partial maxima.
-      float pm[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) pm[i] = s[i];
-#pragma unroll
-      for (int i = 16; i < 128; ++i) pm[i & 15] = fmaxf(pm[i & 15], s[i]);
-#pragma unroll
-      for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-        for (int i = 0; i < w; ++i) pm[i] = fmaxf(pm[i], pm[i + w]);
-      const float m_tile = pm[0] * c;
-      // Running max after tile j-1, from the other group. A slot is rewritten two tiles later only after its
-      // reader has published the tile in between, so one phase of xchg per tile suffices.
-      float m_prev = -INFINITY;
-      if (j > 0) {
-        if (!mbar_wait_warp(&bars.xchg[sb ^ 1], ((j - 1) >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdSmX)) {
-          ok = false;
-          break;
-        }
-        m_prev = xm[(sb ^ 1) * 128 + row];
-      }
-      // Lazy rescaling: the running max moves only when the tile's max exceeds it by more than 2^8 (always on
-      // tile 0). Each row decides for itself, so a row's arithmetic never depends on another row's inputs
-      // (outputs before a position do not depend on inputs after it, bit for bit).
-      const bool need = m_tile > m_prev + kRescaleThreshold;
-      const float m_j = need ? m_tile : m_prev;
-      xm[sb * 128 + row] = m_j;
-      mbar_arrive_warp(&bars.xchg[sb]);
-      if (tracer) ATTN_TRACE_EVENT(11, j);
-      // P = exp2(c*S - m_j) for the 128 keys and the row sum, packed to bf16 pairs in registers. The last
-      // kFwdPolyPairs pairs of every 16 go through the FMA-pipe exp2 (exp2_poly), the rest through MUFU ex2.
-      const float neg_m = -m_j;
-      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial row sums
-      uint32_t pk[4][16];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float x0 = fmaf(s[cc * 32 + 2 * i], c, neg_m), x1 = fmaf(s[cc * 32 + 2 * i + 1], c, neg_m);
-          const bool poly = i >= 16 - kFwdPolyPairs;
-          const float p0 = poly ? exp2_poly(x0) : ex2(x0);
-          const float p1 = poly ? exp2_poly(x1) : ex2(x1);
-          ps[(2 * i) & 7] += p0;
-          ps[(2 * i + 1) & 7] += p1;
-          pk[cc][i] = pack_bf16x2(p0, p1);
-        }
-      }
-      const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      l = (m == m_j ? l : l * ex2(m - m_j)) + rs;  // this group's sum was relative to its previous max
-      m = m_j;
-      if (tracer) ATTN_TRACE_EVENT(9, j);
-      // The P buffer and O are free once PV(j-1) has landed. PV(j-3) landed before S(j) (issue order) and
-      // PV(j+1) waits for PV(j), which waits for this group, so pv_done[sb^1] is within one phase of j-1.
-      if (j > 0) {
-        if (!mbar_wait_warp(&bars.pv_done[sb ^ 1], ((j - 1) >> 1) & 1, abort, p.timeout_ns, &g_device_error,
-                            kSiteFwdSmPV)) {
+      return true;
+    };
+    FwdItem it;
+    bool have = fwd_item(0, n_items, n_qt, it);
+    bool ok = have ? copy_q(0) : true;
+    int t0 = 0;
+    for (int k = 0; have; ++k) {
+      const int qt = it.qt, n_kv = qt + 1;
+      FwdItem next;
+      const bool have_next = fwd_item(k + 1, n_items, n_qt, next);
+      float m = -INFINITY;  // running max (scale*log2(e) units, stale by < 2^8) after this group's last tile
+      float l = 0.f;        // this group's partial row sum of exp2(c*S - m)
+      for (int t = t0 + ((g - t0) & 1); ok && t < t0 + n_kv; t += 2) {
+        const int j = t - t0;  // tile index within the item
+        const int sb = g;      // = t % 2
+        if (!mbar_wait_warp(&bars.s_full[sb], (t >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdSmS)) {
           ok = false;
           break;
         }
         tc_fence_after();
-      }
+        if (tracer) ATTN_TRACE_EVENT(4, t);
+        float s[128];
+        {
+          uint32_t r[4][32];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_st16(tmem + lane_base + kTmemP + cc * 16, pk[cc]);
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // Some row of this warp moved its max: O (tiles 0..j-1, relative to m_prev) is scaled by
-        // 2^(m_prev - m_j) before PV(j) is issued. TMEM access is warp-collective, so the whole warp walks its
-        // rows; rows that kept their max get alpha = 1 exactly.
-        const float alpha = need ? ex2(m_prev - m_j) : 1.0f;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_base + kTmemO + cc * 32, o);
+          for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem + lane_base + kTmemS + sb * 128 + cc * 32, r[cc]);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(tmem + lane_base + kTmemO + cc * 32, o);
+          for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(r[cc][i]);
         }
+        tc_fence_before();
+        mbar_arrive_warp(&bars.s_free[sb]);  // S(t+2) may now be written over this buffer
+        if (lane == 0 && t < 8) ATTN_TRACE_EVENT(12, t * 8 + warp - 2);
+        if (tracer) ATTN_TRACE_EVENT(8, t);
+        if (j == qt) {  // diagonal tile: key column > query row is masked
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (i > row) s[i] = -INFINITY;
+        }
+        // Row max of the tile as a tree over 16 independent partial maxima.
+        float pm[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pm[i] = s[i];
+#pragma unroll
+        for (int i = 16; i < 128; ++i) pm[i & 15] = fmaxf(pm[i & 15], s[i]);
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+          for (int i = 0; i < w; ++i) pm[i] = fmaxf(pm[i], pm[i + w]);
+        const float m_tile = pm[0] * c;
+        // Running max after tile t-1, from the other group (none before an item's first tile). A slot is
+        // rewritten two tiles later only after its reader has published the tile in between (or, across
+        // items, after both groups have passed the epilogue), so one phase of xchg per tile suffices.
+        float m_prev = -INFINITY;
+        if (j > 0) {
+          if (!mbar_wait_warp(&bars.xchg[sb ^ 1], ((t - 1) >> 1) & 1, abort, p.timeout_ns, &g_device_error,
+                              kSiteFwdSmX)) {
+            ok = false;
+            break;
+          }
+          m_prev = xm[(sb ^ 1) * 128 + row];
+        }
+        // Lazy rescaling: the running max moves only when the tile's max exceeds it by more than 2^8 (always
+        // on an item's first tile). Each row decides for itself, so a row's arithmetic never depends on
+        // another row's inputs (outputs before a position do not depend on inputs after it, bit for bit).
+        const bool need = m_tile > m_prev + kRescaleThreshold;
+        const float m_j = need ? m_tile : m_prev;
+        xm[sb * 128 + row] = m_j;
+        mbar_arrive_warp(&bars.xchg[sb]);
+        if (tracer) ATTN_TRACE_EVENT(11, t);
+        // P = exp2(c*S - m_j) for the 128 keys and the row sum, packed to bf16 pairs in registers. The last
+        // kFwdPolyPairs pairs of every 16 go through the FMA-pipe exp2 (exp2_poly), the rest through MUFU ex2.
+        const float neg_m = -m_j;
+        float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial row sums
+        uint32_t pk[4][16];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float x0 = fmaf(s[cc * 32 + 2 * i], c, neg_m), x1 = fmaf(s[cc * 32 + 2 * i + 1], c, neg_m);
+            const bool poly = i >= 16 - kFwdPolyPairs;
+            const float p0 = poly ? exp2_poly(x0) : ex2(x0);
+            const float p1 = poly ? exp2_poly(x1) : ex2(x1);
+            ps[(2 * i) & 7] += p0;
+            ps[(2 * i + 1) & 7] += p1;
+            pk[cc][i] = pack_bf16x2(p0, p1);
+          }
+        }
+        const float rs = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        l = (m == m_j ? l : l * ex2(m - m_j)) + rs;  // this group's sum was relative to its previous max
+        m = m_j;
+        if (tracer) ATTN_TRACE_EVENT(9, t);
+        // P and O are free once PV(t-1) has landed (for an item's first tile, the previous item's last PV).
+        // PV(t-3) landed before S(t) (issue order) and PV(t+1) waits for PV(t), which waits for this group,
+        // so pv_done[sb^1] is within one phase of t-1.
+        if (t > 0) {
+          if (!mbar_wait_warp(&bars.pv_done[sb ^ 1], ((t - 1) >> 1) & 1, abort, p.timeout_ns, &g_device_error,
+                              kSiteFwdSmPV)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) tmem_st16(tmem + lane_base + kTmemP + cc * 16, pk[cc]);
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // Some row of this warp moved its max: O (tiles 0..j-1, relative to m_prev) is scaled by
+          // 2^(m_prev - m_j) before PV(t) is issued. TMEM access is warp-collective, so the whole warp walks
+          // its rows; rows that kept their max get alpha = 1 exactly.
+          const float alpha = need ? ex2(m_prev - m_j) : 1.0f;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_base + kTmemO + cc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tmem + lane_base + kTmemO + cc * 32, o);
+          }
+        }
+        tmem_wait_st();
+        if (tracer) ATTN_TRACE_EVENT(10, t);
+        tc_fence_before();
+        mbar_arrive_warp(&bars.p_full[sb]);
+        if (tracer) ATTN_TRACE_EVENT(5, t);
+        if (lane == 0 && t < 8) ATTN_TRACE_EVENT(13, t * 8 + warp - 2);
       }
-      tmem_wait_st();
-      if (tracer) ATTN_TRACE_EVENT(10, j);
+      // Epilogue of item k. The final running max is the one published for the item's last tile; each group
+      // brings its partial sum to it and the two are added. Every thread of both groups reaches the named
+      // barriers, failed or not, and both leave the item loop on the same decision (a barrier reduction).
+      if (tracer && k < 64) ATTN_TRACE_EVENT(6, k);
+      named_barrier(1, 256);
+      const float m_f = xm[((t0 + n_kv - 1) & 1) * 128 + row];
+      xl[g * 128 + row] = m == m_f ? l : l * ex2(m - m_f);  // a group without tiles has l = 0, m = -inf
+      named_barrier(1, 256);
+      const float l_row = xl[row] + xl[128 + row];
+      bool o_ready =
+          __all_sync(0xffffffffu, ok) && mbar_wait_warp(&bars.o_final, k & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdEpi);
+      if (!o_ready) ok = false;
+      // Every MMA of this item has completed: the next item's Q replaces this one in tensor memory now, so
+      // its first S tiles are computed while this item's output is written.
+      if (ok && have_next) ok = copy_q(k + 1);
+      // The Q buffer takes this item's output once the store of the previous item's output has read it (the
+      // next Q, loaded in between, implies that, but the last item has none). Each thread overwrites only the
+      // bytes of Q it has just copied (its row of box g).
+      if (o_ready && k > 0 &&
+          !mbar_wait_warp(&bars.q_free, (k - 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdEpi)) {
+        o_ready = false;
+        ok = false;
+      }
+      if (o_ready) {
+        if (tracer && k < 64) ATTN_TRACE_EVENT(7, k);
+        tc_fence_after();
+        const float inv_l = 1.0f / l_row;
+        // O / l -> bf16 -> this group's 64-column box of the Q buffer, in the 128-byte-swizzled layout of the
+        // TMA store. The thread writes exactly the bytes of Q it has just copied (its row of box g), so the
+        // copy and the staging need no barrier between them.
+        uint8_t* box = smem + kFwdSmemQ + g * 16384;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + kTmemO + 64 * g + cc * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[ch * 8 + 0]) * inv_l, __uint_as_float(o[ch * 8 + 1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(o[ch * 8 + 2]) * inv_l, __uint_as_float(o[ch * 8 + 3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(o[ch * 8 + 4]) * inv_l, __uint_as_float(o[ch * 8 + 5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(o[ch * 8 + 6]) * inv_l, __uint_as_float(o[ch * 8 + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(box + sw128_offset(row, cc * 4 + ch)) = v;
+          }
+        }
+        const int tq = qt * kTile + row;
+        if (g == 0 && tq < p.T) p.lse[static_cast<size_t>(it.bh) * p.T + tq] = (m_f + __log2f(l_row)) * 0.69314718055994531f;
+      }
+      // The staged rows go to the store warp; both groups have read O (the next item's first PV overwrites
+      // it) and agree on whether to go on.
+      fence_async_shared();
       tc_fence_before();
-      mbar_arrive_warp(&bars.p_full[sb]);
-      if (tracer) ATTN_TRACE_EVENT(5, j);
-      if (lane == 0 && j < 8) ATTN_TRACE_EVENT(13, j * 8 + warp - 2);
-    }
-    // Epilogue: O / l -> bf16 -> swizzled staging (reusing the Q buffer) -> TMA store; LSE in natural log.
-    // The final running max is the one published for the last tile; each group brings its partial sum to it
-    // and the two are added. Every thread of both groups reaches the named barriers, failed or not; the
-    // store is skipped on abort.
-    if (tracer) ATTN_TRACE_EVENT(6, g);
-    named_barrier(1, 256);
-    const float m_f = xm[((n_kv - 1) & 1) * 128 + row];
-    xl[g * 128 + row] = m == m_f ? l : l * ex2(m - m_f);  // a group without tiles has l = 0, m = -inf
-    named_barrier(1, 256);
-    const float l_row = xl[row] + xl[128 + row];
-    const bool epi_ok =
-        __all_sync(0xffffffffu, ok) && mbar_wait_warp(&bars.o_final, 0, abort, p.timeout_ns, &g_device_error, kSiteFwdEpi);
-    if (epi_ok) {
-      if (threadIdx.x == 64) ATTN_TRACE_EVENT(7, 0);
-      tc_fence_after();
-      const float inv_l = 1.0f / l_row;
-      uint8_t* box = smem + kFwdSmemQ + g * 16384;  // this group's 64 head-dim columns = one 64-column box
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tmem + lane_base + kTmemO + 64 * g + cc * 32, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(o[ch * 8 + 0]) * inv_l, __uint_as_float(o[ch * 8 + 1]) * inv_l);
-          v.y = pack_bf16x2(__uint_as_float(o[ch * 8 + 2]) * inv_l, __uint_as_float(o[ch * 8 + 3]) * inv_l);
-          v.z = pack_bf16x2(__uint_as_float(o[ch * 8 + 4]) * inv_l, __uint_as_float(o[ch * 8 + 5]) * inv_l);
-          v.w = pack_bf16x2(__uint_as_float(o[ch * 8 + 6]) * inv_l, __uint_as_float(o[ch * 8 + 7]) * inv_l);
-          *reinterpret_cast<uint4*>(box + sw128_offset(row, cc * 4 + ch)) = v;
-        }
-      }
-      const int t = q0 + row;
-      if (g == 0 && t < p.T) p.lse[static_cast<size_t>(bh) * p.T + t] = (m_f + __log2f(l_row)) * 0.69314718055994531f;
-    }
-    fence_async_shared();
-    named_barrier(1, 256);
-    if (warp == 2 && lane == 0 && !*abort) {
-      for (int cc = 0; cc < 2; ++cc) tma_store_4d(&tm_o, smem + kFwdSmemQ + cc * 16384, cc * 64, h, q0, b);
-      tma_store_commit();
-      tma_store_wait_read_all();
-      ATTN_TRACE_EVENT(6, 2);
+      mbar_arrive_warp(&bars.o_staged);
+      if (!named_barrier_and(1, 256, ok && have_next && !*abort)) break;
+      it = next;
+      t0 += n_kv;
     }
   }
 
