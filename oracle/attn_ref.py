@@ -85,42 +85,62 @@ def head_backward(q, k, v, do, scale: float, o=None):
     return dQ, dK, dV, delta
 
 
+def kv_group(H: int, Hkv: int) -> int:
+    """Query heads per key/value head. Grouped-query attention (apidog "Train your own ChatGPT", section 1 "GPT
+    model": fewer key/value heads than query heads, the value tensor viewed with n_kv_head heads) gives query
+    head h the key/value head h // (H // H_kv): consecutive query heads share one (the pages do not print the
+    mapping; this is the plainest reading, and H_kv = H is plain multi-head attention)."""
+    if Hkv < 1 or H % Hkv:
+        raise ValueError(f"H = {H} query heads cannot be grouped over H_kv = {Hkv} key/value heads")
+    return H // Hkv
+
+
 def attention_forward(q, k, v, scale: float) -> Tuple[np.ndarray, np.ndarray]:
-    """Full forward over [B, T, H, D] inputs. Returns O [B, T, H, D] and LSE [B, H, T], both float64."""
+    """Full forward over q [B, T, H, D] and k, v [B, T, H_kv, D] (H_kv divides H; H_kv = H is multi-head
+    attention). Returns O [B, T, H, D] and LSE [B, H, T], both float64."""
     q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
     B, T, H, D = q.shape
+    G = kv_group(H, k.shape[2])
     O = np.empty((B, T, H, D))
     LSE = np.empty((B, H, T))
     for b in range(B):
         for h in range(H):
-            o_bh, lse_bh, _ = head_forward(q[b, :, h], k[b, :, h], v[b, :, h], scale)
+            o_bh, lse_bh, _ = head_forward(q[b, :, h], k[b, :, h // G], v[b, :, h // G], scale)
             O[b, :, h] = o_bh
             LSE[b, h] = lse_bh
     return O, LSE
 
 
 def attention_backward(q, k, v, do, scale: float, o=None):
-    """Full backward over [B, T, H, D] inputs. Returns dQ, dK, dV [B, T, H, D] and Delta [B, H, T]."""
+    """Full backward over q, dO [B, T, H, D] and k, v [B, T, H_kv, D]. Returns dQ [B, T, H, D], dK, dV
+    [B, T, H_kv, D] and Delta [B, H, T]. A key/value head feeds every query head of its group, so its gradient
+    is the sum of the per-head gradients over the group (the chain rule over the shared input)."""
     q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
     o = None if o is None else _as_f64(o)
     B, T, H, D = q.shape
-    dQ, dK, dV = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    G = kv_group(H, k.shape[2])
+    dQ, dK, dV = np.empty_like(q), np.zeros_like(k), np.zeros_like(v)
     delta = np.empty((B, H, T))
     for b in range(B):
         for h in range(H):
             o_bh = None if o is None else o[b, :, h]
-            gq, gk, gv, dl = head_backward(q[b, :, h], k[b, :, h], v[b, :, h], do[b, :, h], scale, o_bh)
-            dQ[b, :, h], dK[b, :, h], dV[b, :, h] = gq, gk, gv
+            gq, gk, gv, dl = head_backward(q[b, :, h], k[b, :, h // G], v[b, :, h // G], do[b, :, h], scale, o_bh)
+            dQ[b, :, h] = gq
+            dK[b, :, h // G] += gk
+            dV[b, :, h // G] += gv
             delta[b, h] = dl
     return dQ, dK, dV, delta
 
 
 def slice_forward_backward(q, k, v, do, b: int, h: int, scale: float):
-    """Forward and backward of the single (b, h) slice of [B, T, H, D] inputs (slices are independent).
+    """Forward and backward of the single (b, h) query-head slice (slices are independent). q, dO are
+    [B, T, H, D], k, v [B, T, H_kv, D]; the slice reads key/value head h // (H // H_kv).
 
-    Returns a dict of float64 arrays: o [T, D], lse [T], dq, dk, dv [T, D], delta [T].
+    Returns a dict of float64 arrays: o [T, D], lse [T], dq, dk, dv [T, D], delta [T]; dk, dv are this query
+    head's contributions (a key/value head's gradient is their sum over its group).
     """
-    qs, ks, vs = _as_f64(q[b, :, h]), _as_f64(k[b, :, h]), _as_f64(v[b, :, h])
+    hk = h // kv_group(q.shape[2], k.shape[2])
+    qs, ks, vs = _as_f64(q[b, :, h]), _as_f64(k[b, :, hk]), _as_f64(v[b, :, hk])
     o, lse, _ = head_forward(qs, ks, vs, scale)
     out = {"o": o, "lse": lse}
     if do is not None:

@@ -222,6 +222,75 @@ def test_full_tensor_entry_points_match_torch():
 
 
 # ---------------------------------------------------------------------------------------------------------
+# Grouped-query attention: k, v with H_kv heads, query head h reads head h // (H // H_kv).
+
+def _torch_gqa(q, k, v, do, s):
+    """torch's float64 SDPA with its own grouped-query mode (enable_gqa) and autograd."""
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64).transpose(1, 2).requires_grad_() for x in (q, k, v))
+    to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True, scale=s, enable_gqa=True)
+    (to * torch.tensor(do).transpose(1, 2)).sum().backward()
+    return [x.transpose(1, 2).detach().numpy() for x in (to, tq.grad, tk.grad, tv.grad)]
+
+
+@pytest.mark.parametrize("H,Hkv", [(4, 2), (6, 2), (3, 1), (4, 4)])
+def test_gqa_matches_torch_enable_gqa(H, Hkv):
+    B, T, D = 2, 33, 16
+    rng = np.random.default_rng(7 + H + Hkv)
+    q, do = rng.standard_normal((B, T, H, D)), rng.standard_normal((B, T, H, D))
+    k, v = rng.standard_normal((B, T, Hkv, D)), rng.standard_normal((B, T, Hkv, D))
+    s = 1 / math.sqrt(D)
+    O, LSE = attn_ref.attention_forward(q, k, v, s)
+    dQ, dK, dV, _ = attn_ref.attention_backward(q, k, v, do, s)
+    to, gq, gk, gv = _torch_gqa(q, k, v, do, s)
+    np.testing.assert_allclose(O, to, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dQ, gq, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dK, gk, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dV, gv, rtol=1e-11, atol=1e-12)
+    # The slice entry point reads the group's key/value head; its dk is that head's contribution.
+    h = H - 1
+    sl = attn_ref.slice_forward_backward(q, k, v, do, 1, h, s)
+    np.testing.assert_allclose(sl["o"], O[1, :, h], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(sl["dq"], dQ[1, :, h], rtol=0, atol=1e-15)
+
+
+def test_gqa_key_gradient_by_finite_differences():
+    """dK of a shared key/value head is the sum over its query heads: checked by central differences of
+    L = sum(O * dO) with respect to single key and value entries."""
+    B, T, H, Hkv, D = 1, 6, 4, 2, 4
+    rng = np.random.default_rng(3)
+    q, do = rng.standard_normal((B, T, H, D)), rng.standard_normal((B, T, H, D))
+    k, v = rng.standard_normal((B, T, Hkv, D)), rng.standard_normal((B, T, Hkv, D))
+    s = 0.7
+    _, dK, dV, _ = attn_ref.attention_backward(q, k, v, do, s)
+    loss = lambda kk, vv: float((attn_ref.attention_forward(q, kk, vv, s)[0] * do).sum())
+    eps = 1e-6
+    for (t, hk, d) in [(0, 0, 1), (2, 1, 3), (5, 1, 0), (3, 0, 2)]:
+        kp, km = k.copy(), k.copy()
+        kp[0, t, hk, d] += eps
+        km[0, t, hk, d] -= eps
+        assert abs((loss(kp, v) - loss(km, v)) / (2 * eps) - dK[0, t, hk, d]) < 1e-7
+        vp, vm = v.copy(), v.copy()
+        vp[0, t, hk, d] += eps
+        vm[0, t, hk, d] -= eps
+        assert abs((loss(k, vp) - loss(k, vm)) / (2 * eps) - dV[0, t, hk, d]) < 1e-7
+
+
+def test_gqa_pin_catches_a_wrong_head_mapping():
+    """Interleaved sharing (h % H_kv) instead of consecutive sharing is caught by the torch pin."""
+    B, T, H, Hkv, D = 1, 20, 4, 2, 8
+    rng = np.random.default_rng(5)
+    q, do = rng.standard_normal((B, T, H, D)), rng.standard_normal((B, T, H, D))
+    k, v = rng.standard_normal((B, T, Hkv, D)), rng.standard_normal((B, T, Hkv, D))
+    s = 1 / math.sqrt(D)
+    wrong = np.stack([attn_ref.head_forward(q[0, :, h], k[0, :, h % Hkv], v[0, :, h % Hkv], s)[0] for h in range(H)],
+                     axis=1)[None]
+    to = _torch_gqa(q, k, v, do, s)[0]
+    assert np.abs(wrong - to).max() > 1e-3
+    with pytest.raises(ValueError):
+        attn_ref.attention_forward(q, k[:, :, :1].repeat(3, axis=2), v[:, :, :1].repeat(3, axis=2), s)
+
+
+# ---------------------------------------------------------------------------------------------------------
 # Mutation test: plant plausible mistakes in a copy of the oracle and require that some pin fails.
 
 def _mutant(kind):

@@ -12,6 +12,8 @@ is 32, halved to 16 for d24/d26 (ja.news.hada.io summary, "Bigger models"; apido
 
 Layout of every tensor: [B, T, H, D] contiguous, the layout the pages' model reshapes into before calling
 ``flash_attn_func`` (apidog, section 1 "GPT model", the value-embedding ``view(B, T, n_kv_head, head_dim)``).
+Grouped-query workloads (the same section lists grouped-query attention, fewer key/value heads than query
+heads) give k and v H_kv heads: [B, T, H_kv, D].
 """
 from __future__ import annotations
 
@@ -33,10 +35,15 @@ class Workload:
     H: int
     T: int
     D: int = HEAD_DIM
+    Hkv: int = 0                 # key/value heads (grouped-query attention); 0 means H
     seed: int = 0
     qk_prescale: float = 1.0     # multiply the fp32 draws of q and k by this before the bf16 cast
     key_bias: bool = False       # add one shared N(0,1) vector of length D to every key row
     recipe: str = ""
+
+    @property
+    def kv_heads(self) -> int:
+        return self.Hkv if self.Hkv else self.H
 
     @property
     def scale(self) -> float:
@@ -68,6 +75,14 @@ WORKLOADS: Dict[str, Workload] = {
                     recipe="q,k,v,dO ~ N(0,1); one shared bias b ~ N(0,1)^D added to every key row"),
     "d26": Workload("d26", B=16, H=13, T=2048,
                     recipe="q,k,v,dO ~ N(0,1) fp32 from seed 0, cast to bf16"),
+    # Grouped-query attention (the pages give no head counts for it; groups of 2 and 3 query heads per
+    # key/value head here).
+    "tiny_gqa": Workload("tiny_gqa", B=1, H=4, T=128, Hkv=2,
+                         recipe="q,dO [B,T,4,D], k,v [B,T,2,D] ~ N(0,1) fp32 from seed 0, cast to bf16"),
+    "d12_gqa": Workload("d12_gqa", B=32, H=6, T=2048, Hkv=2, qk_prescale=0.5,
+                        recipe="d12 with 2 key/value heads: q,dO [B,T,6,D], k,v [B,T,2,D]; q,k times 0.5"),
+    "d20_gqa": Workload("d20_gqa", B=32, H=10, T=2048, Hkv=5,
+                        recipe="d20 with 5 key/value heads: q,dO [B,T,10,D], k,v [B,T,5,D] ~ N(0,1)"),
 }
 # d26 sequence-length sweep at a fixed B*T = 32768 tokens per device.
 for _T in (512, 1024, 2048, 4096):
@@ -78,7 +93,7 @@ HEADLINE = "d20"
 
 
 def make_inputs(w: Workload, device: Optional[torch.device] = None, need_grad_input: bool = True):
-    """Draw (q, k, v, dO) for a workload as bf16 [B, T, H, D] tensors.
+    """Draw (q, k, v, dO) for a workload as bf16 tensors: q, dO [B, T, H, D]; k, v [B, T, H_kv, D].
 
     One CPU ``torch.Generator`` seeded with ``w.seed`` draws fp32 standard normals in the order q, k, v, dO and
     then (d24 only) the key bias. Pre-scaling and the bias are applied in fp32, then each tensor is rounded to
@@ -87,9 +102,10 @@ def make_inputs(w: Workload, device: Optional[torch.device] = None, need_grad_in
     g = torch.Generator(device="cpu")
     g.manual_seed(w.seed)
     shape = (w.B, w.T, w.H, w.D)
+    kv_shape = (w.B, w.T, w.kv_heads, w.D)
     q = torch.randn(shape, generator=g, dtype=torch.float32)
-    k = torch.randn(shape, generator=g, dtype=torch.float32)
-    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(kv_shape, generator=g, dtype=torch.float32)
+    v = torch.randn(kv_shape, generator=g, dtype=torch.float32)
     do = torch.randn(shape, generator=g, dtype=torch.float32) if need_grad_input else None
     if w.qk_prescale != 1.0:
         q.mul_(w.qk_prescale)
@@ -107,9 +123,9 @@ def key_bias_vector(w: Workload) -> torch.Tensor:
     """The shared key bias of a ``key_bias`` workload (fp32, length D), redrawn from the same stream."""
     g = torch.Generator(device="cpu")
     g.manual_seed(w.seed)
-    n = w.B * w.T * w.H * w.D
-    for _ in range(4):
-        torch.randn((n,), generator=g, dtype=torch.float32)
+    n, nkv = w.B * w.T * w.H * w.D, w.B * w.T * w.kv_heads * w.D
+    for size in (n, nkv, nkv, n):
+        torch.randn((size,), generator=g, dtype=torch.float32)
     return torch.randn((w.D,), generator=g, dtype=torch.float32)
 
 
