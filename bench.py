@@ -180,12 +180,12 @@ def oracle_sample(w: Workload, seconds: float, min_slices: int = 2, max_slices: 
 
     cores = len(os.sched_getaffinity(0))
     with threadpool_limits(limits=cores):
-        probe = make_inputs(w.with_shape(B=1, H=1, seed=w.seed + 1000))
+        probe = make_inputs(w.with_shape(B=1, H=1, Hkv=0, seed=w.seed + 1000))
         t0 = time.perf_counter()
         attn_ref.slice_forward_backward(*probe, 0, 0, w.scale)
         t1 = time.perf_counter() - t0
         k = int(max(min_slices, min(max_slices, round(seconds / max(t1, 1e-6)))))
-        q, kk, v, do = make_inputs(w.with_shape(B=1, H=k, seed=w.seed + 1001))
+        q, kk, v, do = make_inputs(w.with_shape(B=1, H=k, Hkv=1 if w.kv_heads != w.H else 0, seed=w.seed + 1001))
         t0 = time.perf_counter()
         for h in range(k):
             attn_ref.slice_forward_backward(q, kk, v, do, 0, h, w.scale)
@@ -209,7 +209,7 @@ def run_reference(args):
 
     cores = len(os.sched_getaffinity(0))
     slices = 2  # per step: a bounded sample of the workload
-    q, k, v, do = make_inputs(w.with_shape(B=1, H=slices, seed=w.seed + 2000))
+    q, k, v, do = make_inputs(w.with_shape(B=1, H=slices, Hkv=1 if w.kv_heads != w.H else 0, seed=w.seed + 2000))
     times = []
     with threadpool_limits(limits=cores):
         for it in range(args.warmup + args.steps):
@@ -235,7 +235,7 @@ def run_reference(args):
 
 
 def workload_config(w: Workload):
-    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "D": w.D, "causal": True,
+    return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.kv_heads, "T": w.T, "D": w.D, "causal": True,
             "scale": "1/sqrt(D)", "recipe": w.recipe,
             "flop_convention": "fwd 2*B*H*T^2*D, bwd 2.5x fwd",
             "l2": "no flush: q,k,v,dO together exceed the 126 MB L2" if 4 * w.B * w.T * w.H * w.D * 2 > 126e6
@@ -248,10 +248,10 @@ def make_device_inputs(w: Workload, device):
     import torch
     g = torch.Generator(device=device)
     g.manual_seed(w.seed)
-    shape = (w.B, w.T, w.H, w.D)
+    shape, kv_shape = (w.B, w.T, w.H, w.D), (w.B, w.T, w.kv_heads, w.D)
     q = torch.randn(shape, generator=g, device=device)
-    k = torch.randn(shape, generator=g, device=device)
-    v = torch.randn(shape, generator=g, device=device)
+    k = torch.randn(kv_shape, generator=g, device=device)
+    v = torch.randn(kv_shape, generator=g, device=device)
     do = torch.randn(shape, generator=g, device=device)
     if w.qk_prescale != 1.0:
         q.mul_(w.qk_prescale)
@@ -279,11 +279,13 @@ def run_ours(args):
     w = WORKLOADS[args.workload]
     lib = attn.load_library()
     B, H, T, D = w.B, w.H, w.T, w.D
+    Hkv = w.kv_heads
+    gqa = Hkv != H  # grouped-query attention: k, v, dk, dv have Hkv heads
     scale = w.scale
     q, k, v, do = make_device_inputs(w, device)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, T), dtype=torch.float32, device=device)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws_bytes = attn.attn_bwd_workspace_bytes(B, H, T, D)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
@@ -295,22 +297,29 @@ def run_ours(args):
         if st != 0:
             raise RuntimeError(f"{name}: {attn._STATUS.get(st, st)} {lib.attn_last_cuda_error().decode()}")
 
+    if not gqa:
+        # Four launches, each bracketed by events for the per-kernel roofline.
+        names = ["attn_fwd_kernel", "attn_bwd_prep_kernel", "attn_bwd_dkdv_kernel", "attn_bwd_dq_kernel"]
+        calls = [lambda: check(lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                            B, H, T, D, scale, sh), "attn_fwd"),
+                 lambda: check(lib.attn_bwd_preprocess(*bwd_args), "attn_bwd_preprocess"),
+                 lambda: check(lib.attn_bwd_dkdv(*bwd_args), "attn_bwd_dkdv"),
+                 lambda: check(lib.attn_bwd_dq_convert(*bwd_args), "attn_bwd_dq_convert")]
+    else:
+        # Grouped-query entry points: the forward kernel, then the whole backward (its three kernels).
+        gqa_bwd_args = bwd_args[:11] + (B, H, Hkv, T, D, scale, sh)
+        names = ["attn_fwd_kernel", "attn_bwd_gqa"]
+        calls = [lambda: check(lib.attn_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                                lse.data_ptr(), B, H, Hkv, T, D, scale, sh), "attn_fwd_gqa"),
+                 lambda: check(lib.attn_bwd_gqa(*gqa_bwd_args), "attn_bwd_gqa")]
+
     def step(ev=None):
+        for j, call in enumerate(calls):
+            if ev is not None:
+                ev[j].record(stream)
+            call()
         if ev is not None:
-            ev[0].record(stream)
-        check(lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, T, D,
-                           scale, sh), "attn_fwd")
-        if ev is not None:
-            ev[1].record(stream)
-        check(lib.attn_bwd_preprocess(*bwd_args), "attn_bwd_preprocess")
-        if ev is not None:
-            ev[2].record(stream)
-        check(lib.attn_bwd_dkdv(*bwd_args), "attn_bwd_dkdv")
-        if ev is not None:
-            ev[3].record(stream)
-        check(lib.attn_bwd_dq_convert(*bwd_args), "attn_bwd_dq_convert")
-        if ev is not None:
-            ev[4].record(stream)
+            ev[len(calls)].record(stream)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -318,7 +327,7 @@ def run_ours(args):
     if attn.get_device_error() != 0:
         raise RuntimeError("a kernel gave up on a bounded wait during warm-up")
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
     sampler = ClockSampler(gpu_id)
@@ -339,7 +348,6 @@ def run_ours(args):
     err = attn.get_device_error()
     if err != 0:
         raise RuntimeError(f"a kernel gave up on a bounded wait (error word {err:#x}); no number is reported")
-    names = ["attn_fwd_kernel", "attn_bwd_prep_kernel", "attn_bwd_dkdv_kernel", "attn_bwd_dq_kernel"]
     per = {n: [] for n in names}
     for ev in events:
         for j, n in enumerate(names):
@@ -355,15 +363,18 @@ def run_ours(args):
     peak_tf_sus = float(peaks.get("bf16_tflops_sustained", peak_tf))
     hbm = float(peaks["hbm_gbs"])
     n = B * T * H * D
+    nkv = B * T * Hkv * D
     kernels = {
         "attn_fwd_kernel": {"bound": "tensor", "unit": "TFLOP/s", "work": f_fwd, "per": 1e12,
-                            "alg_bytes": 4 * n * 2 + B * H * T * 4},
+                            "alg_bytes": (2 * n + 2 * nkv) * 2 + B * H * T * 4},
         "attn_bwd_prep_kernel": {"bound": "hbm", "unit": "GB/s", "work": 2 * n * 2 + B * H * T * 4 * 3 +
                                  B * H * ((T + 127) // 128 * 128) * 128 * 4, "per": 1e9},
         "attn_bwd_dkdv_kernel": {"bound": "tensor", "unit": "TFLOP/s", "work": f_bwd, "per": 1e12,
                                  "alg_bytes": 7 * n * 2 + B * H * T * 8},
         "attn_bwd_dq_kernel": {"bound": "hbm", "unit": "GB/s", "work": n * 4 + n * 2, "per": 1e9},
+        "attn_bwd_gqa": {"bound": "tensor", "unit": "TFLOP/s", "work": f_bwd, "per": 1e12},
     }
+    kernels = {name: kernels[name] for name in names}
     breakdown = {}
     for name, kinfo in kernels.items():
         t = avg[name] / 1e3
@@ -397,7 +408,8 @@ def run_ours(args):
     # forward, backward, D2H of o, lse, dq, dk, dv, every step.
     if not args.no_e2e:
         hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
-        ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=torch.bfloat16).pin_memory() for _ in range(4))
+        ho, hdq = (torch.empty(q.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2))
+        hdk, hdv = (torch.empty(k.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2))
         hlse = torch.empty((B, H, T), dtype=torch.float32).pin_memory()
 
         def e2e_step():
@@ -427,7 +439,8 @@ def run_ours(args):
         torch.cuda.synchronize(device)
         e_ms = reduce_max(s0.elapsed_time(s1), world, device)
         line["e2e"] = {"value": aggregate((f_fwd + f_bwd) * e_steps, world, e_ms / 1e3) / 1e12, "unit": UNIT,
-                       "h2d_bytes_per_step": 4 * n * 2, "d2h_bytes_per_step": 4 * n * 2 + B * H * T * 4,
+                       "h2d_bytes_per_step": (2 * n + 2 * nkv) * 2,
+                       "d2h_bytes_per_step": (2 * n + 2 * nkv) * 2 + B * H * T * 4,
                        "ms_per_step": e_ms / e_steps}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -38,6 +38,8 @@ SIGNATURES = {
     "attn_bwd_dkdv": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _F, _VP], _I),
     "attn_bwd_dq_convert": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _F, _VP], _I),
     "attn_bwd_noalloc": ([_VP] * 9 + [_I, _I, _I, _I, _F, _VP], _I),
+    "attn_fwd_gqa": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP], _I),
+    "attn_bwd_gqa": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _I, _F, _VP], _I),
     "attn_get_device_error": ([ctypes.POINTER(ctypes.c_uint32)], _I),
     "attn_clear_device_error": ([], _I),
     "attn_set_wait_limit_ns": ([_U64], _I),
@@ -104,15 +106,27 @@ def default_scale(D: int) -> float:
     return 1.0 / math.sqrt(D)
 
 
+def _kv_shape(q: torch.Tensor, k: torch.Tensor):
+    """[B, T, H_kv, D] of k and v: H_kv = H, or fewer key/value heads dividing H (grouped-query attention)."""
+    _check_qkv("k", k)
+    B, T, H, D = q.shape
+    Hkv = k.shape[2]
+    if (k.shape[0], k.shape[1], k.shape[3]) != (B, T, D) or Hkv < 1 or H % Hkv:
+        raise ValueError(f"k has shape {tuple(k.shape)}; expected [{B}, {T}, H_kv, {D}] with H_kv dividing {H}")
+    return (B, T, Hkv, D)
+
+
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,
              o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
              stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Causal attention forward. q, k, v: bf16 [B, T, H, D] on one CUDA device. Returns (o, lse [B, H, T])."""
+    """Causal attention forward. q: bf16 [B, T, H, D]; k, v: bf16 [B, T, H_kv, D] with H_kv = H, or H_kv
+    dividing H for grouped-query attention (query head h reads key/value head h // (H // H_kv)); all on one
+    CUDA device. Returns (o [B, T, H, D], lse [B, H, T])."""
     lib = load_library()
     _check_qkv("q", q)
     B, T, H, D = q.shape
-    _check_qkv("k", k, q.shape)
-    _check_qkv("v", v, q.shape)
+    kv = _kv_shape(q, k)
+    _check_qkv("v", v, kv)
     if o is None:
         o = torch.empty_like(q)
     _check_qkv("o", o, q.shape)
@@ -121,9 +135,14 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, T) or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous fp32 [B, H, T] tensor")
     scale = default_scale(D) if scale is None else float(scale)
-    st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, T, D, scale,
-                      _stream_handle(stream, q.device))
-    _check("attn_fwd", st)
+    if kv[2] == H:
+        st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, T, D, scale,
+                          _stream_handle(stream, q.device))
+        _check("attn_fwd", st)
+    else:
+        st = lib.attn_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, kv[2],
+                              T, D, scale, _stream_handle(stream, q.device))
+        _check("attn_fwd_gqa", st)
     return o, lse
 
 
@@ -135,28 +154,35 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
              dO: torch.Tensor, scale: Optional[float] = None, dq: Optional[torch.Tensor] = None,
              dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
              workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
-    """Causal attention backward. Returns (dq, dk, dv), bf16 [B, T, H, D]."""
+    """Causal attention backward. Returns (dq [B, T, H, D], dk, dv [B, T, H_kv, D]); with grouped-query
+    attention dk, dv are the gradients of the shared heads (summed over each group's query heads)."""
     lib = load_library()
     _check_qkv("q", q)
     B, T, H, D = q.shape
-    for name, t in (("k", k), ("v", v), ("o", o), ("dO", dO)):
+    kv = _kv_shape(q, k)
+    _check_qkv("v", v, kv)
+    for name, t in (("o", o), ("dO", dO)):
         _check_qkv(name, t, q.shape)
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, T) or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous fp32 [B, H, T] tensor")
     dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
-    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
-        _check_qkv(name, t, q.shape)
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_qkv("dq", dq, q.shape)
+    _check_qkv("dk", dk, kv)
+    _check_qkv("dv", dv, kv)
     need = attn_bwd_workspace_bytes(B, H, T, D)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     scale = default_scale(D) if scale is None else float(scale)
-    st = lib.attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dO.data_ptr(),
-                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
-                      workspace.numel() * workspace.element_size(), B, H, T, D, scale,
-                      _stream_handle(stream, q.device))
-    _check("attn_bwd", st)
+    ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dO.data_ptr(), dq.data_ptr(),
+            dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size())
+    if kv[2] == H:
+        st = lib.attn_bwd(*ptrs, B, H, T, D, scale, _stream_handle(stream, q.device))
+        _check("attn_bwd", st)
+    else:
+        st = lib.attn_bwd_gqa(*ptrs, B, H, kv[2], T, D, scale, _stream_handle(stream, q.device))
+        _check("attn_bwd_gqa", st)
     return dq, dk, dv
 
 
@@ -223,7 +249,8 @@ class CausalAttentionFunction(torch.autograd.Function):
 
 
 def causal_attention(q, k, v, scale: Optional[float] = None):
-    """Differentiable causal attention on bf16 [B, T, H, D] tensors (the flash_attn_func(causal=True) call)."""
+    """Differentiable causal attention on bf16 [B, T, H, D] tensors (the flash_attn_func(causal=True) call);
+    k, v may have fewer heads dividing H (grouped-query attention)."""
     return CausalAttentionFunction.apply(q, k, v, default_scale(q.shape[-1]) if scale is None else scale)
 
 

@@ -87,6 +87,12 @@ attn_status check_sizes(int B, int H, int T, int D, float scale) {
   return ATTN_OK;
 }
 
+// Grouped-query attention: H_kv key/value heads, dividing the H query heads.
+attn_status check_kv_heads(int H, int Hkv) {
+  if (Hkv < 1 || Hkv > H || H % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
 // Set the dynamic shared-memory opt-in of both big kernels once per device.
 int g_sm_count[64] = {};  // multiprocessors per device, set by prepare_device
 
@@ -188,16 +194,22 @@ attn_status attn_set_wait_limit_ns(uint64_t limit_ns) {
   return ATTN_OK;
 }
 
-attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T, int D,
-                     float scale, void* stream) {
+}  // extern "C"
+
+namespace {
+
+attn_status fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                       int T, int D, float scale, void* stream) {
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
   attn_status st = check_sizes(B, H, T, D, scale);
   if (st != ATTN_OK) return st;
+  if ((st = check_kv_heads(H, Hkv)) != ATTN_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return ATTN_ERR_MISALIGNED;
   const size_t nbytes = static_cast<size_t>(B) * T * H * D * 2;
+  const size_t kvbytes = static_cast<size_t>(B) * T * Hkv * D * 2;
   const size_t lbytes = static_cast<size_t>(B) * H * T * 4;
-  const Range rq = span(q, nbytes), rk = span(k, nbytes), rv = span(v, nbytes), ro = span(o, nbytes),
+  const Range rq = span(q, nbytes), rk = span(k, kvbytes), rv = span(v, kvbytes), ro = span(o, nbytes),
               rl = span(lse, lbytes);
   for (Range in : {rq, rk, rv})
     if (overlap(ro, in) || overlap(rl, in)) return ATTN_ERR_INVALID_ARG;
@@ -207,14 +219,15 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   if ((st = prepare_device(&dev)) != ATTN_OK) return st;
   CUtensorMap mq, mk, mv, mo;
   if ((st = make_map(&mq, q, B, H, T, attn::kTile)) != ATTN_OK) return st;
-  if ((st = make_map(&mk, k, B, H, T, attn::kTile)) != ATTN_OK) return st;
-  if ((st = make_map(&mv, v, B, H, T, attn::kTile)) != ATTN_OK) return st;
+  if ((st = make_map(&mk, k, B, Hkv, T, attn::kTile)) != ATTN_OK) return st;
+  if ((st = make_map(&mv, v, B, Hkv, T, attn::kTile)) != ATTN_OK) return st;
   if ((st = make_map(&mo, o, B, H, T, attn::kTile)) != ATTN_OK) return st;
 
   attn::FwdParams p;
   p.lse = lse;
   p.B = B;
   p.H = H;
+  p.Hkv = Hkv;
   p.T = T;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_wait_limit_ns;
@@ -227,6 +240,20 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_fwd_kernel launch");
   return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T, int D,
+                     float scale, void* stream) {
+  return fwd_launch(q, k, v, o, lse, B, H, H, T, D, scale, stream);
+}
+
+attn_status attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
+                         int T, int D, float scale, void* stream) {
+  return fwd_launch(q, k, v, o, lse, B, H, H_kv, T, D, scale, stream);
 }
 
 size_t attn_bwd_workspace_bytes(int B, int H, int T, int D) {
@@ -242,10 +269,11 @@ namespace {
 // bit 1: dK/dV with dQ accumulation, bit 2: dQ conversion) in that order on `stream`.
 attn_status bwd_launch(unsigned stages, const void* q, const void* k, const void* v, const void* o, const float* lse,
                        const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B,
-                       int H, int T, int D, float scale, void* stream) {
+                       int H, int Hkv, int T, int D, float scale, void* stream) {
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
   attn_status st = check_sizes(B, H, T, D, scale);
   if (st != ATTN_OK) return st;
+  if ((st = check_kv_heads(H, Hkv)) != ATTN_OK) return st;
   const WorkspaceLayout wl = workspace_layout(B, H, T);
   if (!workspace || workspace_bytes < wl.total) return ATTN_ERR_WORKSPACE;
   for (const void* ptr : {q, k, v, o, dO, static_cast<const void*>(lse), static_cast<const void*>(dq),
@@ -253,10 +281,11 @@ attn_status bwd_launch(unsigned stages, const void* q, const void* k, const void
     if (!aligned16(ptr)) return ATTN_ERR_MISALIGNED;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_MISALIGNED;
   const size_t nbytes = static_cast<size_t>(B) * T * H * D * 2;
+  const size_t kvbytes = static_cast<size_t>(B) * T * Hkv * D * 2;
   const size_t lbytes = static_cast<size_t>(B) * H * T * 4;
-  const Range ins[6] = {span(q, nbytes), span(k, nbytes), span(v, nbytes), span(o, nbytes), span(dO, nbytes),
+  const Range ins[6] = {span(q, nbytes), span(k, kvbytes), span(v, kvbytes), span(o, nbytes), span(dO, nbytes),
                         span(lse, lbytes)};
-  const Range outs[4] = {span(dq, nbytes), span(dk, nbytes), span(dv, nbytes), span(workspace, wl.total)};
+  const Range outs[4] = {span(dq, nbytes), span(dk, kvbytes), span(dv, kvbytes), span(workspace, wl.total)};
   for (int i = 0; i < 4; ++i) {
     for (int j = 0; j < 6; ++j)
       if (overlap(outs[i], ins[j])) return ATTN_ERR_INVALID_ARG;
@@ -269,10 +298,10 @@ attn_status bwd_launch(unsigned stages, const void* q, const void* k, const void
   CUtensorMap mq, mk, mv, mdo, mdk, mdv;
   if ((st = make_map(&mq, q, B, H, T, attn::kBwdQTile)) != ATTN_OK) return st;
   if ((st = make_map(&mdo, dO, B, H, T, attn::kBwdQTile)) != ATTN_OK) return st;
-  if ((st = make_map(&mk, k, B, H, T, attn::kBwdKTile)) != ATTN_OK) return st;
-  if ((st = make_map(&mv, v, B, H, T, attn::kBwdKTile)) != ATTN_OK) return st;
-  if ((st = make_map(&mdk, dk, B, H, T, attn::kBwdKTile)) != ATTN_OK) return st;
-  if ((st = make_map(&mdv, dv, B, H, T, attn::kBwdKTile)) != ATTN_OK) return st;
+  if ((st = make_map(&mk, k, B, Hkv, T, attn::kBwdKTile)) != ATTN_OK) return st;
+  if ((st = make_map(&mv, v, B, Hkv, T, attn::kBwdKTile)) != ATTN_OK) return st;
+  if ((st = make_map(&mdk, dk, B, Hkv, T, attn::kBwdKTile)) != ATTN_OK) return st;
+  if ((st = make_map(&mdv, dv, B, Hkv, T, attn::kBwdKTile)) != ATTN_OK) return st;
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   attn::BwdParams p;
@@ -285,6 +314,7 @@ attn_status bwd_launch(unsigned stages, const void* q, const void* k, const void
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.B = B;
   p.H = H;
+  p.Hkv = Hkv;
   p.T = T;
   p.Tp = attn::padded_T(T);
   p.scale = scale;
@@ -300,7 +330,7 @@ attn_status bwd_launch(unsigned stages, const void* q, const void* k, const void
   }
   if (stages & 2u) {
     const unsigned n_kt = static_cast<unsigned>((T + attn::kBwdKTile - 1) / attn::kBwdKTile);
-    attn::attn_bwd_dkdv_kernel<<<dim3(n_kt * static_cast<unsigned>(B * H)), attn::kBwdThreads,
+    attn::attn_bwd_dkdv_kernel<<<dim3(n_kt * static_cast<unsigned>(B * Hkv)), attn::kBwdThreads,
                                  attn::kBwdSmemAlloc, s>>>(mq, mk, mv, mdo, mdk, mdv, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_bwd_dkdv_kernel launch");
   }
@@ -320,12 +350,18 @@ extern "C" {
   const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dO, void *dq,     \
       void *dk, void *dv, void *workspace, size_t workspace_bytes, int B, int H, int T, int D, float scale,     \
       void *stream
-#define ATTN_BWD_PASS q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, H, T, D, scale, stream
+#define ATTN_BWD_PASS q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, H, H, T, D, scale, stream
 
 attn_status attn_bwd(ATTN_BWD_ARGS) { return bwd_launch(7u, ATTN_BWD_PASS); }
 attn_status attn_bwd_preprocess(ATTN_BWD_ARGS) { return bwd_launch(1u, ATTN_BWD_PASS); }
 attn_status attn_bwd_dkdv(ATTN_BWD_ARGS) { return bwd_launch(2u, ATTN_BWD_PASS); }
 attn_status attn_bwd_dq_convert(ATTN_BWD_ARGS) { return bwd_launch(4u, ATTN_BWD_PASS); }
+
+attn_status attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                         void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int H_kv,
+                         int T, int D, float scale, void* stream) {
+  return bwd_launch(7u, q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, H, H_kv, T, D, scale, stream);
+}
 
 attn_status attn_get_device_error(uint32_t* word) {
   if (!word) return ATTN_ERR_INVALID_ARG;
@@ -423,7 +459,7 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
   if ((st = noalloc_scratch_ptr(&scratch)) != ATTN_OK) return st;
   // Same three kernels as attn_bwd; the preprocess kernel rewrites every scratch byte the later kernels read
   // (including zeroing the dQ accumulator), so whatever an earlier call left there does not matter.
-  return bwd_launch(7u, q, k, v, o, lse, dO, dq, dk, dv, scratch, kNoAllocScratchBytes, B, H, T, D, scale, stream);
+  return bwd_launch(7u, q, k, v, o, lse, dO, dq, dk, dv, scratch, kNoAllocScratchBytes, B, H, H, T, D, scale, stream);
 }
 
 }  // extern "C"

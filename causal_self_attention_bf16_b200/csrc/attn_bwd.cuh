@@ -8,8 +8,9 @@
 // Three launches on the caller's stream:
 //   1. attn_bwd_prep_kernel: Delta (fp32, from the stored bf16 O), LSE * log2(e), and zeroing of the fp32 dQ
 //      accumulator. Rows past T are padded with LSE = +inf and Delta = 0 so they contribute nothing.
-//   2. attn_bwd_dkdv_kernel: one CTA per (128-key tile, batch, head) walks the 64-query tiles at or after
-//      its keys. Per query tile, five tcgen05 MMAs:
+//   2. attn_bwd_dkdv_kernel: one CTA per (128-key tile, batch, key/value head) walks the 64-query tiles at
+//      or after its keys, of every query head that reads this key/value head (one, or a group of them with
+//      grouped-query attention). Per query tile, five tcgen05 MMAs:
 //        S^T = K Q^T, dP^T = V dO^T            (K-major operands in shared memory)
 //        dV += P^T dO, dK += dS^T Q             (P^T, dS^T from tensor memory; dO, Q MN-major)
 //        dQ^T = K^T dS^T                        (both operands MN-major in shared memory)
@@ -59,6 +60,7 @@ struct BwdParams {
   float* dq_acc;             // [B*H, Tp/4, D, 4] fp32
   __nv_bfloat16* dq;         // [B, T, H, D]
   int B, H, T, Tp;
+  int Hkv;                   // key/value heads (divides H): the dK/dV kernel's CTA covers one of them
   float scale, scale_log2;
   uint64_t timeout_ns;
 };
@@ -183,14 +185,19 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   // Head-major order, heaviest key tile (the first, seen by every query tile) first within a head: the CTAs in
   // flight cover only ~10 heads, so their Q, dO and the head's fp32 dQ accumulator stay in L2.
+  // A CTA owns one key tile of one key/value head; with grouped-query attention (G query heads per key/value
+  // head) it walks the query tiles of every query head of the group in turn, so dK and dV sum over the group
+  // in tensor memory. Step i is query head hk*G + i/n, query tile i0 + i%n.
   const int n_kt = (p.T + kBwdKTile - 1) / kBwdKTile;
-  const int bh = static_cast<int>(blockIdx.x / n_kt);
+  const int G = p.H / p.Hkv;
+  const int bhk = static_cast<int>(blockIdx.x / n_kt);
   const int kt = static_cast<int>(blockIdx.x % n_kt);
-  const int b = bh / p.H, h = bh % p.H;
+  const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
   const int k0 = kt * kBwdKTile;
   const int n_q64 = (p.T + kBwdQTile - 1) / kBwdQTile;
   const int i0 = k0 / kBwdQTile;           // first query tile that sees these keys
-  const int n = n_q64 - i0;                // query tiles this CTA walks (>= 1)
+  const int n = n_q64 - i0;                // query tiles per query head (>= 1)
+  const int ns = G * n;                    // steps of this CTA
   volatile int* abort = &bars.abort;
 
   if (threadIdx.x == 0) {
@@ -232,18 +239,19 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       tma_prefetch_desc(&tm_do);
       mbar_arrive_expect_tx(&bars.kv_full, 4 * 16384);
       for (int c = 0; c < 2; ++c) {
-        tma_load_4d(smem + kBwdSmemK + c * 16384, &tm_k, &bars.kv_full, c * 64, h, k0, b);
-        tma_load_4d(smem + kBwdSmemV + c * 16384, &tm_v, &bars.kv_full, c * 64, h, k0, b);
+        tma_load_4d(smem + kBwdSmemK + c * 16384, &tm_k, &bars.kv_full, c * 64, hk, k0, b);
+        tma_load_4d(smem + kBwdSmemV + c * 16384, &tm_v, &bars.kv_full, c * 64, hk, k0, b);
       }
     }
     int last_issued[kBwdStages];
     for (int s = 0; s < kBwdStages; ++s) last_issued[s] = -1;
-    for (int i = 0; i < n; ++i) {
+    for (int i = 0; i < ns; ++i) {
       const int s = i % kBwdStages;
       if (i >= kBwdStages && !mbar_wait_warp(&bars.q_empty[s], ((i - kBwdStages) / kBwdStages) & 1, abort,
                                              p.timeout_ns, &g_device_error, kSiteBwdProdQEmpty))
         break;
-      const int q0 = (i0 + i) * kBwdQTile;
+      const int h = hk * G + i / n, bh = b * p.H + h;  // the step's query head
+      const int q0 = (i0 + i % n) * kBwdQTile;
       if (leader) {
         mbar_arrive_expect_tx(&bars.q_full[s], 2 * 16384 + 2 * 256);
         for (int c = 0; c < 2; ++c) {
@@ -344,9 +352,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     };
     // Pairs: A(i), A(i+1), B(i), B(i+1). The two softmax groups work on tiles i and i+1 at the same time,
     // and the dQ^T read-out of a pair overlaps the next pair's first MMAs.
-    for (int i = 0; ok && i < n; i += 2) {
-      ok = issue_a(i) && (i + 1 >= n || issue_a(i + 1));
-      ok = ok && issue_b(i) && (i + 1 >= n || issue_b(i + 1));
+    for (int i = 0; ok && i < ns; i += 2) {
+      ok = issue_a(i) && (i + 1 >= ns || issue_a(i + 1));
+      ok = ok && issue_b(i) && (i + 1 >= ns || issue_b(i + 1));
     }
     if (leader) {
       mma_commit(&bars.acc_done);
@@ -367,12 +375,12 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const int kg = k0 + krow;
     const float c = p.scale_log2;
     const bool group_leader = lane == 0 && quarter == 2;  // first warp of the group
-    float* acc_bh = p.dq_acc + static_cast<size_t>(bh) * p.Tp * 128;
     float* dq_stage = reinterpret_cast<float*>(smem + kBwdSmemDQ);
     bool ok = true;
-    for (int i = g; i < n; i += 2) {
+    for (int i = g; i < ns; i += 2) {
       const int s = i % kBwdStages, rb = g;
-      const int q0 = (i0 + i) * kBwdQTile;
+      const int q0 = (i0 + i % n) * kBwdQTile;
+      float* acc_bh = p.dq_acc + static_cast<size_t>(b * p.H + hk * G + i / n) * p.Tp * 128;  // step's query head
       if (!mbar_wait_warp(&bars.q_full[s], (i / kBwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdSmQ) ||
           !mbar_wait_warp(&bars.s_full[rb], (i >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdSmS)) {
         ok = false;
@@ -457,7 +465,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       fence_async_shared();
       named_barrier(2 + g, 128);
       if (group_leader) {
-        bulk_reduce_add_f32(acc_bh + static_cast<size_t>(((i0 + i) * kBwdQTile) >> 2) * 512, dq_stage, 32768);
+        bulk_reduce_add_f32(acc_bh + static_cast<size_t>(q0 >> 2) * 512, dq_stage, 32768);
         tma_store_commit();
         tma_store_wait_read_all();  // the staging buffer has been read: hand it to the next tile
         mbar_arrive(&bars.stage_free);
@@ -495,7 +503,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     named_barrier(1, 256);
     if ((warp == 2 || warp == 6) && lane == 0 && !*abort) {
       const CUtensorMap* tm = g == 0 ? &tm_dv : &tm_dk;
-      for (int cc = 0; cc < 2; ++cc) tma_store_4d(tm, stage + cc * 16384, cc * 64, h, k0, b);
+      for (int cc = 0; cc < 2; ++cc) tma_store_4d(tm, stage + cc * 16384, cc * 64, hk, k0, b);
       tma_store_commit();
       tma_store_wait_read_all();
     }

@@ -74,6 +74,7 @@ __device__ __forceinline__ float exp2_poly(float x) {
 struct FwdParams {
   float* lse;        // [B, H, T] fp32
   int B, H, T;
+  int Hkv;           // key/value heads (divides H); query head h reads key/value head h / (H / Hkv)
   float scale_log2;  // scale * log2(e)
   uint64_t timeout_ns;
 };
@@ -202,6 +203,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     FwdItem it;
     for (int k = 0; fwd_item(k, n_items, n_qt, it); ++k) {
       const int b = it.bh / p.H, h = it.bh % p.H, n_kv = it.qt + 1;
+      const int hk = h / (p.H / p.Hkv);  // grouped-query attention: the group's key/value head
       if (is_k) {
         // One Q buffer, which also stages each item's output for its TMA store. Q(1) may go in once Q(0) is in
         // tensor memory; Q(k), k >= 2, once item k-2's output has been read out of the buffer by its store
@@ -227,7 +229,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (leader) {
           mbar_arrive_expect_tx(&full[s], 2 * 16384);
-          for (int c = 0; c < 2; ++c) tma_load_4d(ring + s * 32768 + c * 16384, tm, &full[s], c * 64, h, j * kTile, b);
+          for (int c = 0; c < 2; ++c) tma_load_4d(ring + s * 32768 + c * 16384, tm, &full[s], c * 64, hk, j * kTile, b);
           if (is_k) ATTN_TRACE_EVENT(1, t);
         }
         issued[s] = t;

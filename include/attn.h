@@ -103,6 +103,21 @@ attn_status attn_bwd_dq_convert(const void* q, const void* k, const void* v, con
                                 size_t workspace_bytes, int B, int H, int T, int D, float scale, void* stream);
 
 /*
+ * Grouped-query attention (apidog "Train your own ChatGPT", section 1 "GPT model": fewer key/value heads than
+ * query heads). H_kv key/value heads, H_kv >= 1 dividing H; query head h reads key/value head h / (H / H_kv),
+ * so consecutive query heads share one (the pages do not print the mapping; this is the plainest reading).
+ * H_kv = H is exactly attn_fwd / attn_bwd. Otherwise the same contract, with these shapes:
+ *   q, o, dO, dq : bf16 [B, T, H, D];   k, v, dk, dv : bf16 [B, T, H_kv, D];   lse : fp32 [B, H, T]
+ * dk, dv are the gradients of the shared heads: the sum over each group's query heads. The workspace is
+ * attn_bwd_workspace_bytes(B, H, T, D) bytes (per query head). H_kv out of range: ATTN_ERR_INVALID_ARG.
+ */
+attn_status attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
+                         int T, int D, float scale, void* stream);
+attn_status attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                         int B, int H, int H_kv, int T, int D, float scale, void* stream);
+
+/*
  * Backward without caller-provided workspace, for callers that cannot allocate device memory (a custom-op or
  * plugin interface that passes tensors but no allocator or workspace; a fixed memory plan that forbids
  * cudaMalloc/cudaFree, and the synchronisation they can cause, during a step). The pages have no counterpart:

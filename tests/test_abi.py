@@ -110,6 +110,23 @@ def test_bwd_argument_errors(lib):
     assert bwd_call(lib, ptrs, ws, ws=ptrs[8]) == 1           # workspace aliases dv
 
 
+def test_gqa_argument_errors(lib):
+    """attn_fwd_gqa / attn_bwd_gqa reject key/value head counts that do not divide H, and check overlaps with
+    the k, v, dk, dv sizes of H_kv heads."""
+    qsize = 1 * 128 * 6 * 128 * 2
+    q, k, v, o, lse = fake_ptrs(5, qsize)
+    for hkv in (0, 4, 7, -2):
+        assert lib.attn_fwd_gqa(q, k, v, o, lse, 1, 6, hkv, 128, 128, 0.088, None) == 1
+    assert lib.attn_fwd_gqa(q, k, v, o, lse, 1, 6, 3, 128, 96, 0.088, None) == 2
+    assert lib.attn_fwd_gqa(q, k, v, k + 256, lse, 1, 6, 3, 128, 128, 0.088, None) == 1   # o overlaps k
+    ws = lib.attn_bwd_workspace_bytes(1, 6, 128, 128)
+    ptrs = fake_ptrs(10, max(qsize, ws))
+    args = lambda **over: [over.get(n, p) for n, p in zip(["q", "k", "v", "o", "lse", "dO", "dq", "dk", "dv", "ws"], ptrs)]
+    assert lib.attn_bwd_gqa(*args(), ws, 1, 6, 4, 128, 128, 0.088, None) == 1
+    assert lib.attn_bwd_gqa(*args(), ws - 1, 1, 6, 2, 128, 128, 0.088, None) == 6
+    assert lib.attn_bwd_gqa(*args(dk=ptrs[1]), ws, 1, 6, 2, 128, 128, 0.088, None) == 1    # dk aliases k
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
 def test_no_cpu_fallback_without_gpu(lib):
     """A well-formed call on a machine without an sm_100 GPU fails loudly instead of computing on the CPU."""
@@ -119,6 +136,7 @@ def test_no_cpu_fallback_without_gpu(lib):
     assert lib.attn_last_cuda_error().decode() != ""
     ws = lib.attn_bwd_workspace_bytes(1, 2, 128, 128)
     assert bwd_call(lib, fake_ptrs(10, max(size, ws)), ws) == 4
+    assert lib.attn_fwd_gqa(q, k, v, o, lse, 1, 2, 1, 128, 128, 0.088, None) == 4
 
 
 def test_binding_rejects_cpu_tensors(lib):

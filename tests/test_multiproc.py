@@ -2,7 +2,7 @@
 rank runs its own replica of the batch, no collective on the data path), so what runs across ranks is the
 timing reduction (max over ranks) and the whole-job aggregation (units of all ranks over the slowest time)."""
 import os
-import socket
+import tempfile
 
 import pytest
 import torch.distributed as dist
@@ -11,18 +11,11 @@ import torch.multiprocessing as mp
 import bench
 
 
-def _free_port():
-    s = socket.socket()
-    s.bind(("127.0.0.1", 0))
-    port = s.getsockname()[1]
-    s.close()
-    return port
-
-
-def _worker(rank, world, port, times, q):
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
-                      LOCAL_RANK=str(rank))
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+def _worker(rank, world, store_path, times, q):
+    # File rendezvous: no TCP port to pick, so nothing else on the machine can take it between the pick and
+    # the bind (bench.py itself uses torchrun's env:// rendezvous, covered by dist_env below).
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", init_method=f"file://{store_path}", rank=rank, world_size=world)
     try:
         r, w, local = bench.dist_env()
         assert (r, w, local) == (rank, world, rank)
@@ -36,9 +29,9 @@ def _worker(rank, world, port, times, q):
 def test_reduce_max_over_two_gloo_ranks():
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = _free_port()
     times = [1.25, 3.5]
-    mp.spawn(_worker, args=(2, port, times, q), nprocs=2, join=True)
+    with tempfile.TemporaryDirectory() as d:
+        mp.spawn(_worker, args=(2, os.path.join(d, "store"), times, q), nprocs=2, join=True)
     got = dict(q.get(timeout=30) for _ in range(2))
     assert got == {0: 3.5, 1: 3.5}
 

@@ -132,6 +132,43 @@ def test_full_size_sampled_slices(name):
         assert bool(torch.isfinite(t.float()).all())
 
 
+# Grouped-query attention: k, v with H_kv heads, query head h reads head h // (H // H_kv).
+GQA_SHAPES = [(1, 4, 2, 128), (2, 6, 2, 200), (1, 3, 1, 65), (1, 8, 4, 383), (2, 4, 1, 257), (1, 2, 2, 129)]
+
+
+@pytest.mark.parametrize("B,H,Hkv,T", GQA_SHAPES, ids=[f"B{b}H{h}Hkv{hk}T{t}" for b, h, hk, t in GQA_SHAPES])
+def test_gqa_full(B, H, Hkv, T):
+    full_compare(Workload("gqa", B=B, H=H, T=T, Hkv=Hkv, seed=T + H))
+
+
+def test_gqa_tiny_workload():
+    full_compare(WORKLOADS["tiny_gqa"])
+
+
+@pytest.mark.parametrize("name", ["d12_gqa", "d20_gqa"])
+def test_gqa_full_size_sampled_groups(name):
+    """Full-size grouped-query workloads: for sampled (b, key/value head) pairs, every query head of the group
+    is checked as an oracle slice, and the shared head's dK, dV against the sum of the group's slices."""
+    w = WORKLOADS[name]
+    q, k, v, do = make_inputs(w)
+    o, lse, dq, dk, dv = run_gpu(q, k, v, do, w.scale)
+    G = w.H // w.kv_heads
+    for (b, hk) in [(0, 0), (w.B - 1, w.kv_heads - 1)]:
+        dk_ref, dv_ref = 0.0, 0.0
+        for h in range(hk * G, (hk + 1) * G):
+            ref = attn_ref.slice_forward_backward(q, k, v, do, b, h, w.scale)
+            what = f"{name} slice (b={b}, h={h})"
+            check_o(to64(o[b, :, h]), ref["o"], what)
+            check_lse(to64(lse[b, h]), ref["lse"], what)
+            check_grad(to64(dq[b, :, h]), ref["dq"], "dQ", what)
+            dk_ref = dk_ref + ref["dk"]
+            dv_ref = dv_ref + ref["dv"]
+        check_grad(to64(dk[b, :, hk]), dk_ref, "dK", f"{name} kv head (b={b}, hk={hk})")
+        check_grad(to64(dv[b, :, hk]), dv_ref, "dV", f"{name} kv head (b={b}, hk={hk})")
+    for t in (o, dq, dk, dv):
+        assert bool(torch.isfinite(t.float()).all())
+
+
 def test_causality_on_gpu():
     """Perturbing q/k/v after position t leaves O and LSE at positions <= t bit-identical."""
     w = Workload("causal", B=2, H=2, T=300, seed=9)
