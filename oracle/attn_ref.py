@@ -36,7 +36,7 @@ identity; a hand-derived worked example under tests/golden/.
 """
 from __future__ import annotations
 
-from typing import Tuple
+from typing import Optional, Tuple
 
 import numpy as np
 
@@ -49,16 +49,25 @@ def _as_f64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
-def causal_mask(T: int) -> np.ndarray:
-    """Boolean [T, T] matrix, True where key j may be seen by query i (j <= i)."""
-    return np.tril(np.ones((T, T), dtype=bool))
+def causal_mask(T: int, window: Optional[int] = None) -> np.ndarray:
+    """Boolean [T, T] matrix, True where key j may be seen by query i: j <= i, and with a sliding window also
+    j >= i - window, so a query sees itself and the `window` keys before it. The pages pass
+    ``window_size=window_size`` to flash_attn_func and alternate short- and long-window layers ("SSSL") (apidog
+    "Train your own ChatGPT", section 1 "GPT model" and section 5 "Flash Attention integration"); reading:
+    flash_attn's left window, causal on the right; None is no window."""
+    m = np.tril(np.ones((T, T), dtype=bool))
+    if window is not None:
+        if window < 0:
+            raise ValueError("window must be >= 0 (or None for no window)")
+        m &= np.triu(np.ones((T, T), dtype=bool), -window)  # j - i >= -window
+    return m
 
 
-def head_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
+def head_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float, window: Optional[int] = None):
     """Forward of one (b, h) slice: q, k, v are [T, D] float64. Returns (O [T, D], LSE [T], P [T, T])."""
     T = q.shape[0]
     S = scale * (q @ k.T)
-    S = np.where(causal_mask(T), S, -np.inf)
+    S = np.where(causal_mask(T, window), S, -np.inf)
     m = S.max(axis=1, keepdims=True)           # finite: the diagonal is always visible
     E = np.exp(S - m)                          # exp(-inf) = 0 on masked entries
     l = E.sum(axis=1, keepdims=True)
@@ -68,12 +77,12 @@ def head_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
     return O, lse, P
 
 
-def head_backward(q, k, v, do, scale: float, o=None):
+def head_backward(q, k, v, do, scale: float, o=None, window: Optional[int] = None):
     """Backward of one (b, h) slice from the definition. Returns (dQ, dK, dV, Delta).
 
     ``o`` is the forward output used for Delta; by default the exact float64 output of ``head_forward``.
     """
-    O, _, P = head_forward(q, k, v, scale)
+    O, _, P = head_forward(q, k, v, scale, window)
     if o is None:
         o = O
     dV = P.T @ do
@@ -95,7 +104,7 @@ def kv_group(H: int, Hkv: int) -> int:
     return H // Hkv
 
 
-def attention_forward(q, k, v, scale: float) -> Tuple[np.ndarray, np.ndarray]:
+def attention_forward(q, k, v, scale: float, window: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
     """Full forward over q [B, T, H, D] and k, v [B, T, H_kv, D] (H_kv divides H; H_kv = H is multi-head
     attention). Returns O [B, T, H, D] and LSE [B, H, T], both float64."""
     q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
@@ -105,13 +114,13 @@ def attention_forward(q, k, v, scale: float) -> Tuple[np.ndarray, np.ndarray]:
     LSE = np.empty((B, H, T))
     for b in range(B):
         for h in range(H):
-            o_bh, lse_bh, _ = head_forward(q[b, :, h], k[b, :, h // G], v[b, :, h // G], scale)
+            o_bh, lse_bh, _ = head_forward(q[b, :, h], k[b, :, h // G], v[b, :, h // G], scale, window)
             O[b, :, h] = o_bh
             LSE[b, h] = lse_bh
     return O, LSE
 
 
-def attention_backward(q, k, v, do, scale: float, o=None):
+def attention_backward(q, k, v, do, scale: float, o=None, window: Optional[int] = None):
     """Full backward over q, dO [B, T, H, D] and k, v [B, T, H_kv, D]. Returns dQ [B, T, H, D], dK, dV
     [B, T, H_kv, D] and Delta [B, H, T]. A key/value head feeds every query head of its group, so its gradient
     is the sum of the per-head gradients over the group (the chain rule over the shared input)."""
@@ -124,7 +133,8 @@ def attention_backward(q, k, v, do, scale: float, o=None):
     for b in range(B):
         for h in range(H):
             o_bh = None if o is None else o[b, :, h]
-            gq, gk, gv, dl = head_backward(q[b, :, h], k[b, :, h // G], v[b, :, h // G], do[b, :, h], scale, o_bh)
+            gq, gk, gv, dl = head_backward(q[b, :, h], k[b, :, h // G], v[b, :, h // G], do[b, :, h], scale, o_bh,
+                                           window)
             dQ[b, :, h] = gq
             dK[b, :, h // G] += gk
             dV[b, :, h // G] += gv
@@ -132,7 +142,7 @@ def attention_backward(q, k, v, do, scale: float, o=None):
     return dQ, dK, dV, delta
 
 
-def slice_forward_backward(q, k, v, do, b: int, h: int, scale: float):
+def slice_forward_backward(q, k, v, do, b: int, h: int, scale: float, window: Optional[int] = None):
     """Forward and backward of the single (b, h) query-head slice (slices are independent). q, dO are
     [B, T, H, D], k, v [B, T, H_kv, D]; the slice reads key/value head h // (H // H_kv).
 
@@ -141,11 +151,11 @@ def slice_forward_backward(q, k, v, do, b: int, h: int, scale: float):
     """
     hk = h // kv_group(q.shape[2], k.shape[2])
     qs, ks, vs = _as_f64(q[b, :, h]), _as_f64(k[b, :, hk]), _as_f64(v[b, :, hk])
-    o, lse, _ = head_forward(qs, ks, vs, scale)
+    o, lse, _ = head_forward(qs, ks, vs, scale, window)
     out = {"o": o, "lse": lse}
     if do is not None:
         dos = _as_f64(do[b, :, h])
-        dq, dk, dv, delta = head_backward(qs, ks, vs, dos, scale)
+        dq, dk, dv, delta = head_backward(qs, ks, vs, dos, scale, window=window)
         out.update(dq=dq, dk=dk, dv=dv, delta=delta)
     return out
 

@@ -291,6 +291,75 @@ def test_gqa_pin_catches_a_wrong_head_mapping():
 
 
 # ---------------------------------------------------------------------------------------------------------
+# Sliding window: query i sees keys i - window .. i.
+
+def _band(T, window):
+    i = torch.arange(T)[:, None]
+    j = torch.arange(T)[None, :]
+    return (j <= i) & (j >= i - window)
+
+
+@pytest.mark.parametrize("T,window,H,Hkv", [(37, 5, 2, 2), (40, 0, 2, 2), (33, 16, 4, 2), (50, 1, 3, 1)])
+def test_window_matches_torch_with_band_mask(T, window, H, Hkv):
+    """torch's float64 SDPA given the band as an explicit boolean mask (and enable_gqa), with autograd."""
+    B, D = 2, 16
+    rng = np.random.default_rng(T + window)
+    q, do = rng.standard_normal((B, T, H, D)), rng.standard_normal((B, T, H, D))
+    k, v = rng.standard_normal((B, T, Hkv, D)), rng.standard_normal((B, T, Hkv, D))
+    s = 1 / math.sqrt(D)
+    O, LSE = attn_ref.attention_forward(q, k, v, s, window=window)
+    dQ, dK, dV, _ = attn_ref.attention_backward(q, k, v, do, s, window=window)
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64).transpose(1, 2).requires_grad_() for x in (q, k, v))
+    to = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=_band(T, window), scale=s,
+                                                          enable_gqa=True)
+    (to * torch.tensor(do).transpose(1, 2)).sum().backward()
+    np.testing.assert_allclose(O, to.transpose(1, 2).detach().numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dQ, tq.grad.transpose(1, 2).numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dK, tk.grad.transpose(1, 2).numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dV, tv.grad.transpose(1, 2).numpy(), rtol=1e-11, atol=1e-12)
+    # LSE against torch.logsumexp over the band.
+    kk = np.repeat(k, H // Hkv, axis=2)
+    S = s * np.einsum("bihd,bjhd->bhij", q, kk)
+    S = np.where(_band(T, window).numpy(), S, -np.inf)
+    np.testing.assert_allclose(LSE, torch.logsumexp(torch.tensor(S), dim=-1).numpy(), rtol=1e-13, atol=1e-13)
+
+
+def test_window_closed_forms():
+    """window >= T-1 is plain causal attention; window 0 leaves each query only itself: O = V exactly and
+    LSE = scale * q.k of the row's own key."""
+    T, D = 30, 8
+    q, k, v, do = rand_qkvdo(T, D, 4)
+    s = 0.4
+    O, LSE = attn_ref.attention_forward(q, k, v, s)
+    Ow, LSEw = attn_ref.attention_forward(q, k, v, s, window=T - 1)
+    np.testing.assert_array_equal(O, Ow)
+    np.testing.assert_array_equal(LSE, LSEw)
+    O0, LSE0 = attn_ref.attention_forward(q, k, v, s, window=0)
+    np.testing.assert_allclose(O0, v, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(LSE0[0, 0], s * (q[0, :, 0] * k[0, :, 0]).sum(axis=1), rtol=1e-14, atol=1e-14)
+    with pytest.raises(ValueError):
+        attn_ref.attention_forward(q, k, v, s, window=-2)
+
+
+def test_window_gradients_by_finite_differences():
+    T, D, window = 9, 4, 3
+    q, k, v, do = rand_qkvdo(T, D, 8)
+    s = 0.6
+    dQ, dK, dV, _ = attn_ref.attention_backward(q, k, v, do, s, window=window)
+    loss = lambda qq, kk, vv: float((attn_ref.attention_forward(qq, kk, vv, s, window=window)[0] * do).sum())
+    eps = 1e-6
+    for name, x, g in (("q", q, dQ), ("k", k, dK), ("v", v, dV)):
+        for (t, d) in [(0, 0), (4, 2), (8, 3), (6, 1)]:
+            xp, xm = x.copy(), x.copy()
+            xp[0, t, 0, d] += eps
+            xm[0, t, 0, d] -= eps
+            args_p = [xp if n == name else y for n, y in (("q", q), ("k", k), ("v", v))]
+            args_m = [xm if n == name else y for n, y in (("q", q), ("k", k), ("v", v))]
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - g[0, t, 0, d]) < 1e-7, (name, t, d)
+
+
+# ---------------------------------------------------------------------------------------------------------
 # Mutation test: plant plausible mistakes in a copy of the oracle and require that some pin fails.
 
 def _mutant(kind):

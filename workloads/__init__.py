@@ -36,6 +36,7 @@ class Workload:
     T: int
     D: int = HEAD_DIM
     Hkv: int = 0                 # key/value heads (grouped-query attention); 0 means H
+    window: int = -1             # sliding window: a query sees itself and this many keys before it; -1: none
     seed: int = 0
     qk_prescale: float = 1.0     # multiply the fp32 draws of q and k by this before the bf16 cast
     key_bias: bool = False       # add one shared N(0,1) vector of length D to every key row
@@ -52,8 +53,14 @@ class Workload:
 
     @property
     def fwd_flops(self) -> float:
-        """Causal forward FLOPs by the convention 2*B*H*T^2*D (half of the dense 4*B*H*T^2*D)."""
-        return 2.0 * self.B * self.H * self.T * self.T * self.D
+        """Causal forward FLOPs by the convention 2*B*H*T^2*D (half of the dense 4*B*H*T^2*D); with a sliding
+        window, scaled by the fraction of the causal (query, key) pairs that stay inside the window."""
+        f = 2.0 * self.B * self.H * self.T * self.T * self.D
+        if self.window >= 0:
+            T, W = self.T, self.window
+            kept = sum(min(i, W) + 1 for i in range(T)) if T <= 1 << 16 else T * (W + 1) - W * (W + 1) / 2
+            f *= kept / (T * (T + 1) / 2)
+        return f
 
     @property
     def bwd_flops(self) -> float:
@@ -83,6 +90,12 @@ WORKLOADS: Dict[str, Workload] = {
                         recipe="d12 with 2 key/value heads: q,dO [B,T,6,D], k,v [B,T,2,D]; q,k times 0.5"),
     "d20_gqa": Workload("d20_gqa", B=32, H=10, T=2048, Hkv=5,
                         recipe="d20 with 5 key/value heads: q,dO [B,T,10,D], k,v [B,T,5,D] ~ N(0,1)"),
+    # Sliding-window attention (the pages' "SSSL" layers: short-window layers between full-context ones; the
+    # window length is not on the pages: a quarter of the context here).
+    "tiny_sw": Workload("tiny_sw", B=1, H=2, T=300, window=100,
+                        recipe="q,k,v,dO ~ N(0,1) fp32 from seed 0, cast to bf16; window 100"),
+    "d20_sw": Workload("d20_sw", B=32, H=10, T=2048, window=512,
+                       recipe="d20 shape and recipe, sliding window of 512 keys"),
 }
 # d26 sequence-length sweep at a fixed B*T = 32768 tokens per device.
 for _T in (512, 1024, 2048, 4096):
