@@ -87,8 +87,9 @@ def recorded_traffic(kernel: str, workload: str):
 
 
 def flops(w: Workload):
-    f = 2.0 * w.B * w.H * w.T * w.T * w.D
-    return f, 2.5 * f
+    """Forward and backward FLOPs of the metric's convention (causal half; a sliding window scales it by the
+    fraction of causal pairs inside the window)."""
+    return w.fwd_flops, w.bwd_flops
 
 
 def dist_env():
@@ -182,15 +183,16 @@ def oracle_sample(w: Workload, seconds: float, min_slices: int = 2, max_slices: 
     with threadpool_limits(limits=cores):
         probe = make_inputs(w.with_shape(B=1, H=1, Hkv=0, seed=w.seed + 1000))
         t0 = time.perf_counter()
-        attn_ref.slice_forward_backward(*probe, 0, 0, w.scale)
+        win = w.window if w.window >= 0 else None
+        attn_ref.slice_forward_backward(*probe, 0, 0, w.scale, window=win)
         t1 = time.perf_counter() - t0
         k = int(max(min_slices, min(max_slices, round(seconds / max(t1, 1e-6)))))
         q, kk, v, do = make_inputs(w.with_shape(B=1, H=k, Hkv=1 if w.kv_heads != w.H else 0, seed=w.seed + 1001))
         t0 = time.perf_counter()
         for h in range(k):
-            attn_ref.slice_forward_backward(q, kk, v, do, 0, h, w.scale)
+            attn_ref.slice_forward_backward(q, kk, v, do, 0, h, w.scale, window=win)
         dt = time.perf_counter() - t0
-    f_slice = 3.5 * 2.0 * w.T * w.T * w.D
+    f_slice = 3.5 * w.with_shape(B=1, H=1).fwd_flops
     tflops = k * f_slice / dt / 1e12
     desc = (f"{k} (b,h) slices of {w.name} (T={w.T}, D={w.D}), fwd+bwd float64 numpy, "
             f"{dt:.1f} s; equal-cost independent slices, so the rate holds for the full batch of {w.B * w.H}")
@@ -215,11 +217,12 @@ def run_reference(args):
         for it in range(args.warmup + args.steps):
             t0 = time.perf_counter()
             for h in range(slices):
-                attn_ref.slice_forward_backward(q, k, v, do, 0, h, w.scale)
+                attn_ref.slice_forward_backward(q, k, v, do, 0, h, w.scale,
+                                                window=w.window if w.window >= 0 else None)
             if it >= args.warmup:
                 times.append(time.perf_counter() - t0)
     step = sum(times) / len(times)
-    f_step = slices * 3.5 * 2.0 * w.T * w.T * w.D
+    f_step = slices * 3.5 * w.with_shape(B=1, H=1).fwd_flops
     value = f_step / step / 1e12
     sample = f"{slices} (b,h) slices of {w.name} per step, float64 numpy oracle fwd+bwd"
     line = {
@@ -236,8 +239,10 @@ def run_reference(args):
 
 def workload_config(w: Workload):
     return {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.kv_heads, "T": w.T, "D": w.D, "causal": True,
+            "window": w.window,
             "scale": "1/sqrt(D)", "recipe": w.recipe,
-            "flop_convention": "fwd 2*B*H*T^2*D, bwd 2.5x fwd",
+            "flop_convention": "fwd 2*B*H*T^2*D (with a window: times the fraction of causal pairs inside it), "
+                               "bwd 2.5x fwd",
             "l2": "no flush: q,k,v,dO together exceed the 126 MB L2" if 4 * w.B * w.T * w.H * w.D * 2 > 126e6
             else "inputs smaller than L2"}
 
@@ -280,7 +285,8 @@ def run_ours(args):
     lib = attn.load_library()
     B, H, T, D = w.B, w.H, w.T, w.D
     Hkv = w.kv_heads
-    gqa = Hkv != H  # grouped-query attention: k, v, dk, dv have Hkv heads
+    window = w.window  # -1: no sliding window
+    gqa = Hkv != H or window >= 0  # grouped-query attention (k, v, dk, dv have Hkv heads) or a sliding window
     scale = w.scale
     q, k, v, do = make_device_inputs(w, device)
     o = torch.empty_like(q)
@@ -306,12 +312,13 @@ def run_ours(args):
                  lambda: check(lib.attn_bwd_dkdv(*bwd_args), "attn_bwd_dkdv"),
                  lambda: check(lib.attn_bwd_dq_convert(*bwd_args), "attn_bwd_dq_convert")]
     else:
-        # Grouped-query entry points: the forward kernel, then the whole backward (its three kernels).
-        gqa_bwd_args = bwd_args[:11] + (B, H, Hkv, T, D, scale, sh)
-        names = ["attn_fwd_kernel", "attn_bwd_gqa"]
-        calls = [lambda: check(lib.attn_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                                lse.data_ptr(), B, H, Hkv, T, D, scale, sh), "attn_fwd_gqa"),
-                 lambda: check(lib.attn_bwd_gqa(*gqa_bwd_args), "attn_bwd_gqa")]
+        # General entry points (key/value heads, window): the forward kernel, then the whole backward (its
+        # three kernels).
+        ex_bwd_args = bwd_args[:11] + (B, H, Hkv, T, D, scale, window, sh)
+        names = ["attn_fwd_kernel", "attn_bwd_ex"]
+        calls = [lambda: check(lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                               lse.data_ptr(), B, H, Hkv, T, D, scale, window, sh), "attn_fwd_ex"),
+                 lambda: check(lib.attn_bwd_ex(*ex_bwd_args), "attn_bwd_ex")]
 
     def step(ev=None):
         for j, call in enumerate(calls):
@@ -372,7 +379,7 @@ def run_ours(args):
         "attn_bwd_dkdv_kernel": {"bound": "tensor", "unit": "TFLOP/s", "work": f_bwd, "per": 1e12,
                                  "alg_bytes": 7 * n * 2 + B * H * T * 8},
         "attn_bwd_dq_kernel": {"bound": "hbm", "unit": "GB/s", "work": n * 4 + n * 2, "per": 1e9},
-        "attn_bwd_gqa": {"bound": "tensor", "unit": "TFLOP/s", "work": f_bwd, "per": 1e12},
+        "attn_bwd_ex": {"bound": "tensor", "unit": "TFLOP/s", "work": f_bwd, "per": 1e12},
     }
     kernels = {name: kernels[name] for name in names}
     breakdown = {}
@@ -417,8 +424,9 @@ def run_ours(args):
             k.copy_(hk, non_blocking=True)
             v.copy_(hv, non_blocking=True)
             do.copy_(hdo, non_blocking=True)
-            attn.attn_fwd(q, k, v, scale, o=o, lse=lse)
-            attn.attn_bwd(q, k, v, o, lse, do, scale, dq=dq, dk=dk, dv=dv, workspace=ws)
+            win = window if window >= 0 else None
+            attn.attn_fwd(q, k, v, scale, o=o, lse=lse, window=win)
+            attn.attn_bwd(q, k, v, o, lse, do, scale, dq=dq, dk=dk, dv=dv, workspace=ws, window=win)
             ho.copy_(o, non_blocking=True)
             hlse.copy_(lse, non_blocking=True)
             hdq.copy_(dq, non_blocking=True)

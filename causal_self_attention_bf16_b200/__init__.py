@@ -40,6 +40,8 @@ SIGNATURES = {
     "attn_bwd_noalloc": ([_VP] * 9 + [_I, _I, _I, _I, _F, _VP], _I),
     "attn_fwd_gqa": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _VP], _I),
     "attn_bwd_gqa": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _I, _F, _VP], _I),
+    "attn_fwd_ex": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP], _I),
+    "attn_bwd_ex": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _I, _F, _I, _VP], _I),
     "attn_get_device_error": ([ctypes.POINTER(ctypes.c_uint32)], _I),
     "attn_clear_device_error": ([], _I),
     "attn_set_wait_limit_ns": ([_U64], _I),
@@ -116,12 +118,21 @@ def _kv_shape(q: torch.Tensor, k: torch.Tensor):
     return (B, T, Hkv, D)
 
 
+def _window_arg(window: Optional[int]) -> int:
+    if window is None:
+        return -1
+    if int(window) < 0:
+        raise ValueError("window must be >= 0 (or None for no window)")
+    return int(window)
+
+
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,
              o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-             stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+             stream: Optional[torch.cuda.Stream] = None, window: Optional[int] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Causal attention forward. q: bf16 [B, T, H, D]; k, v: bf16 [B, T, H_kv, D] with H_kv = H, or H_kv
     dividing H for grouped-query attention (query head h reads key/value head h // (H // H_kv)); all on one
-    CUDA device. Returns (o [B, T, H, D], lse [B, H, T])."""
+    CUDA device. window: None, or a sliding window (query i sees keys i - window .. i). Returns
+    (o [B, T, H, D], lse [B, H, T])."""
     lib = load_library()
     _check_qkv("q", q)
     B, T, H, D = q.shape
@@ -135,7 +146,12 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, T) or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous fp32 [B, H, T] tensor")
     scale = default_scale(D) if scale is None else float(scale)
-    if kv[2] == H:
+    win = _window_arg(window)
+    if win >= 0:
+        st = lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, kv[2],
+                             T, D, scale, win, _stream_handle(stream, q.device))
+        _check("attn_fwd_ex", st)
+    elif kv[2] == H:
         st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, T, D, scale,
                           _stream_handle(stream, q.device))
         _check("attn_fwd", st)
@@ -153,8 +169,10 @@ def attn_bwd_workspace_bytes(B: int, H: int, T: int, D: int) -> int:
 def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
              dO: torch.Tensor, scale: Optional[float] = None, dq: Optional[torch.Tensor] = None,
              dk: Optional[torch.Tensor] = None, dv: Optional[torch.Tensor] = None,
-             workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
-    """Causal attention backward. Returns (dq [B, T, H, D], dk, dv [B, T, H_kv, D]); with grouped-query
+             workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+             window: Optional[int] = None):
+    """Causal attention backward (window as given to attn_fwd). Returns (dq [B, T, H, D], dk, dv [B, T, H_kv,
+    D]); with grouped-query
     attention dk, dv are the gradients of the shared heads (summed over each group's query heads)."""
     lib = load_library()
     _check_qkv("q", q)
@@ -177,7 +195,11 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     scale = default_scale(D) if scale is None else float(scale)
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dO.data_ptr(), dq.data_ptr(),
             dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size())
-    if kv[2] == H:
+    win = _window_arg(window)
+    if win >= 0:
+        st = lib.attn_bwd_ex(*ptrs, B, H, kv[2], T, D, scale, win, _stream_handle(stream, q.device))
+        _check("attn_bwd_ex", st)
+    elif kv[2] == H:
         st = lib.attn_bwd(*ptrs, B, H, T, D, scale, _stream_handle(stream, q.device))
         _check("attn_bwd", st)
     else:
@@ -235,23 +257,23 @@ class CausalAttentionFunction(torch.autograd.Function):
     """autograd wrapper: forward saves (q, k, v, o, lse); backward calls attn_bwd."""
 
     @staticmethod
-    def forward(ctx, q, k, v, scale):
-        o, lse = attn_fwd(q, k, v, scale)
+    def forward(ctx, q, k, v, scale, window=None):
+        o, lse = attn_fwd(q, k, v, scale, window=window)
         ctx.save_for_backward(q, k, v, o, lse)
-        ctx.scale = scale
+        ctx.scale, ctx.window = scale, window
         return o
 
     @staticmethod
     def backward(ctx, dO):
         q, k, v, o, lse = ctx.saved_tensors
-        dq, dk, dv = attn_bwd(q, k, v, o, lse, dO.contiguous(), ctx.scale)
-        return dq, dk, dv, None
+        dq, dk, dv = attn_bwd(q, k, v, o, lse, dO.contiguous(), ctx.scale, window=ctx.window)
+        return dq, dk, dv, None, None
 
 
-def causal_attention(q, k, v, scale: Optional[float] = None):
-    """Differentiable causal attention on bf16 [B, T, H, D] tensors (the flash_attn_func(causal=True) call);
-    k, v may have fewer heads dividing H (grouped-query attention)."""
-    return CausalAttentionFunction.apply(q, k, v, default_scale(q.shape[-1]) if scale is None else scale)
+def causal_attention(q, k, v, scale: Optional[float] = None, window: Optional[int] = None):
+    """Differentiable causal attention on bf16 [B, T, H, D] tensors (the flash_attn_func(causal=True,
+    window_size=(window, 0)) call); k, v may have fewer heads dividing H (grouped-query attention)."""
+    return CausalAttentionFunction.apply(q, k, v, default_scale(q.shape[-1]) if scale is None else scale, window)
 
 
 __all__ = ["attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "causal_attention", "CausalAttentionFunction",

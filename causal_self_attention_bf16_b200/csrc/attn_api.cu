@@ -199,11 +199,12 @@ attn_status attn_set_wait_limit_ns(uint64_t limit_ns) {
 namespace {
 
 attn_status fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
-                       int T, int D, float scale, void* stream) {
+                       int T, int D, float scale, int window, void* stream) {
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
   attn_status st = check_sizes(B, H, T, D, scale);
   if (st != ATTN_OK) return st;
   if ((st = check_kv_heads(H, Hkv)) != ATTN_OK) return st;
+  if (window < -1) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return ATTN_ERR_MISALIGNED;
   const size_t nbytes = static_cast<size_t>(B) * T * H * D * 2;
@@ -228,6 +229,7 @@ attn_status fwd_launch(const void* q, const void* k, const void* v, void* o, flo
   p.B = B;
   p.H = H;
   p.Hkv = Hkv;
+  p.window = window;
   p.T = T;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_wait_limit_ns;
@@ -248,12 +250,17 @@ extern "C" {
 
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T, int D,
                      float scale, void* stream) {
-  return fwd_launch(q, k, v, o, lse, B, H, H, T, D, scale, stream);
+  return fwd_launch(q, k, v, o, lse, B, H, H, T, D, scale, -1, stream);
 }
 
 attn_status attn_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
                          int T, int D, float scale, void* stream) {
-  return fwd_launch(q, k, v, o, lse, B, H, H_kv, T, D, scale, stream);
+  return fwd_launch(q, k, v, o, lse, B, H, H_kv, T, D, scale, -1, stream);
+}
+
+attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
+                        int T, int D, float scale, int window, void* stream) {
+  return fwd_launch(q, k, v, o, lse, B, H, H_kv, T, D, scale, window, stream);
 }
 
 size_t attn_bwd_workspace_bytes(int B, int H, int T, int D) {
@@ -269,11 +276,12 @@ namespace {
 // bit 1: dK/dV with dQ accumulation, bit 2: dQ conversion) in that order on `stream`.
 attn_status bwd_launch(unsigned stages, const void* q, const void* k, const void* v, const void* o, const float* lse,
                        const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B,
-                       int H, int Hkv, int T, int D, float scale, void* stream) {
+                       int H, int Hkv, int T, int D, float scale, int window, void* stream) {
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
   attn_status st = check_sizes(B, H, T, D, scale);
   if (st != ATTN_OK) return st;
   if ((st = check_kv_heads(H, Hkv)) != ATTN_OK) return st;
+  if (window < -1) return ATTN_ERR_INVALID_ARG;
   const WorkspaceLayout wl = workspace_layout(B, H, T);
   if (!workspace || workspace_bytes < wl.total) return ATTN_ERR_WORKSPACE;
   for (const void* ptr : {q, k, v, o, dO, static_cast<const void*>(lse), static_cast<const void*>(dq),
@@ -315,6 +323,7 @@ attn_status bwd_launch(unsigned stages, const void* q, const void* k, const void
   p.B = B;
   p.H = H;
   p.Hkv = Hkv;
+  p.window = window;
   p.T = T;
   p.Tp = attn::padded_T(T);
   p.scale = scale;
@@ -350,7 +359,7 @@ extern "C" {
   const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dO, void *dq,     \
       void *dk, void *dv, void *workspace, size_t workspace_bytes, int B, int H, int T, int D, float scale,     \
       void *stream
-#define ATTN_BWD_PASS q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, H, H, T, D, scale, stream
+#define ATTN_BWD_PASS q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, H, H, T, D, scale, -1, stream
 
 attn_status attn_bwd(ATTN_BWD_ARGS) { return bwd_launch(7u, ATTN_BWD_PASS); }
 attn_status attn_bwd_preprocess(ATTN_BWD_ARGS) { return bwd_launch(1u, ATTN_BWD_PASS); }
@@ -360,7 +369,15 @@ attn_status attn_bwd_dq_convert(ATTN_BWD_ARGS) { return bwd_launch(4u, ATTN_BWD_
 attn_status attn_bwd_gqa(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                          void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int H_kv,
                          int T, int D, float scale, void* stream) {
-  return bwd_launch(7u, q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, H, H_kv, T, D, scale, stream);
+  return bwd_launch(7u, q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, H, H_kv, T, D, scale, -1,
+                    stream);
+}
+
+attn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                        void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int H_kv,
+                        int T, int D, float scale, int window, void* stream) {
+  return bwd_launch(7u, q, k, v, o, lse, dO, dq, dk, dv, workspace, workspace_bytes, B, H, H_kv, T, D, scale, window,
+                    stream);
 }
 
 attn_status attn_get_device_error(uint32_t* word) {
@@ -459,7 +476,8 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
   if ((st = noalloc_scratch_ptr(&scratch)) != ATTN_OK) return st;
   // Same three kernels as attn_bwd; the preprocess kernel rewrites every scratch byte the later kernels read
   // (including zeroing the dQ accumulator), so whatever an earlier call left there does not matter.
-  return bwd_launch(7u, q, k, v, o, lse, dO, dq, dk, dv, scratch, kNoAllocScratchBytes, B, H, H, T, D, scale, stream);
+  return bwd_launch(7u, q, k, v, o, lse, dO, dq, dk, dv, scratch, kNoAllocScratchBytes, B, H, H, T, D, scale, -1,
+                    stream);
 }
 
 }  // extern "C"

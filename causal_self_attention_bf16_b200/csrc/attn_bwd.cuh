@@ -26,6 +26,8 @@
 // 64; after the softmax step, for each half h of the 64 queries, columns [32h, 32h+16) hold P^T and
 // [32h+16, 32h+32) hold dS^T (bf16 pairs) of those 32 queries, and the dQ^T MMA writes the last 64 columns.
 #pragma once
+#include <type_traits>
+
 #include "attn_common.cuh"
 #include "sm100.cuh"
 
@@ -61,6 +63,7 @@ struct BwdParams {
   __nv_bfloat16* dq;         // [B, T, H, D]
   int B, H, T, Tp;
   int Hkv;                   // key/value heads (divides H): the dK/dV kernel's CTA covers one of them
+  int window;                // sliding window: query i sees keys i - window .. i; -1: no window
   float scale, scale_log2;
   uint64_t timeout_ns;
 };
@@ -196,7 +199,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   const int k0 = kt * kBwdKTile;
   const int n_q64 = (p.T + kBwdQTile - 1) / kBwdQTile;
   const int i0 = k0 / kBwdQTile;           // first query tile that sees these keys
-  const int n = n_q64 - i0;                // query tiles per query head (>= 1)
+  // last query tile + 1: all of them, or with a sliding window those holding queries <= k0 + 127 + window
+  const int i_end = p.window < 0 ? n_q64 : min(n_q64, (k0 + kBwdKTile - 1 + p.window) / kBwdQTile + 1);
+  const int n = i_end - i0;                // query tiles per query head (>= 1)
   const int ns = G * n;                    // steps of this CTA
   volatile int* abort = &bars.abort;
 
@@ -389,45 +394,55 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       tc_fence_after();
       if (threadIdx.x == 64 || threadIdx.x == 192) ATTN_TRACE_EVENT(4, i);
       const bool diag = q0 < k0 + kBwdKTile;  // tile overlaps the key tile: queries before a key see nothing
+      // sliding window: queries after key + window see nothing (only tiles reaching past k0 + window have any)
+      const bool band = p.window >= 0 && q0 + kBwdQTile - 1 > k0 + p.window;
       uint8_t* dsrow = smem + kBwdSmemDS + rb * 16384;
+      // The half-tile body is instantiated twice: with the sliding-window mask (tiles that reach past a key's
+      // window) and without it, so unwindowed tiles carry no per-element window test.
+      auto halves = [&](auto band_flag) {
+        constexpr bool kBand = decltype(band_flag)::value;
 #pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {  // one half at a time keeps the live registers to one half's worth
-        const uint32_t r = tmem + lane_base + kTmemR + rb * 128 + 32 * hh;
-        const float4* lse4 = reinterpret_cast<const float4*>(smem + kBwdSmemLse + s * 256) + 8 * hh;
-        const float4* dlt4 = reinterpret_cast<const float4*>(smem + kBwdSmemDelta + s * 256) + 8 * hh;
-        uint32_t sv[32], dp[32];
-        tmem_ld32(r, sv);        // S^T of queries [32hh, 32hh+32)
-        tmem_ld32(r + 64, dp);   // dP^T of the same queries
-        tmem_wait_ld();
-        if (threadIdx.x == 64) ATTN_TRACE_EVENT(8, i * 2 + hh);
-        uint32_t ppk[16], dpk[16];
+        for (int hh = 0; hh < 2; ++hh) {  // one half at a time keeps the live registers to one half's worth
+          const uint32_t r = tmem + lane_base + kTmemR + rb * 128 + 32 * hh;
+          const float4* lse4 = reinterpret_cast<const float4*>(smem + kBwdSmemLse + s * 256) + 8 * hh;
+          const float4* dlt4 = reinterpret_cast<const float4*>(smem + kBwdSmemDelta + s * 256) + 8 * hh;
+          uint32_t sv[32], dp[32];
+          tmem_ld32(r, sv);        // S^T of queries [32hh, 32hh+32)
+          tmem_ld32(r + 64, dp);   // dP^T of the same queries
+          tmem_wait_ld();
+          if (threadIdx.x == 64) ATTN_TRACE_EVENT(8, i * 2 + hh);
+          uint32_t ppk[16], dpk[16];
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 l4 = lse4[q4], d4 = dlt4[q4];
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-          float pv[4], dsv[4];
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 l4 = lse4[q4], d4 = dlt4[q4];
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+            float pv[4], dsv[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int q = q4 * 4 + e;
-            float pe = ex2(fmaf(__uint_as_float(sv[q]), c, -lv[e]));
-            if (diag && q0 + 32 * hh + q < kg) pe = 0.f;
-            pv[e] = pe;
-            dsv[e] = pe * (__uint_as_float(dp[q]) - dv4[e]);
+            for (int e = 0; e < 4; ++e) {
+              const int q = q4 * 4 + e;
+              float pe = ex2(fmaf(__uint_as_float(sv[q]), c, -lv[e]));
+              if (diag && q0 + 32 * hh + q < kg) pe = 0.f;
+              if (kBand && q0 + 32 * hh + q > kg + p.window) pe = 0.f;
+              pv[e] = pe;
+              dsv[e] = pe * (__uint_as_float(dp[q]) - dv4[e]);
+            }
+            ppk[q4 * 2] = pack_bf16x2(pv[0], pv[1]);
+            ppk[q4 * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+            dpk[q4 * 2] = pack_bf16x2(dsv[0], dsv[1]);
+            dpk[q4 * 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
           }
-          ppk[q4 * 2] = pack_bf16x2(pv[0], pv[1]);
-          ppk[q4 * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-          dpk[q4 * 2] = pack_bf16x2(dsv[0], dsv[1]);
-          dpk[q4 * 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
-        }
-        if (threadIdx.x == 64) ATTN_TRACE_EVENT(9, i * 2 + hh);
-        tmem_st16(r, ppk);        // P^T  of these 32 queries: columns [32hh, 32hh+16)
-        tmem_st16(r + 16, dpk);   // dS^T of these 32 queries: columns [32hh+16, 32hh+32)
+          if (threadIdx.x == 64) ATTN_TRACE_EVENT(9, i * 2 + hh);
+          tmem_st16(r, ppk);        // P^T  of these 32 queries: columns [32hh, 32hh+16)
+          tmem_st16(r + 16, dpk);   // dS^T of these 32 queries: columns [32hh+16, 32hh+32)
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint4 v = make_uint4(dpk[ch * 4 + 0], dpk[ch * 4 + 1], dpk[ch * 4 + 2], dpk[ch * 4 + 3]);
-          *reinterpret_cast<uint4*>(dsrow + sw128_offset(krow, 4 * hh + ch)) = v;
+          for (int ch = 0; ch < 4; ++ch) {
+            uint4 v = make_uint4(dpk[ch * 4 + 0], dpk[ch * 4 + 1], dpk[ch * 4 + 2], dpk[ch * 4 + 3]);
+            *reinterpret_cast<uint4*>(dsrow + sw128_offset(krow, 4 * hh + ch)) = v;
+          }
         }
-      }
+      };
+      if (band) halves(std::true_type{});
+      else halves(std::false_type{});
       tmem_wait_st();
       if (threadIdx.x == 64) ATTN_TRACE_EVENT(10, i);
       fence_async_shared();

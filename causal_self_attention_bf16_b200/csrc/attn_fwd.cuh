@@ -75,6 +75,7 @@ struct FwdParams {
   float* lse;        // [B, H, T] fp32
   int B, H, T;
   int Hkv;           // key/value heads (divides H); query head h reads key/value head h / (H / Hkv)
+  int window;        // sliding window: query i sees keys i - window .. i; -1: no window
   float scale_log2;  // scale * log2(e)
   uint64_t timeout_ns;
 };
@@ -115,6 +116,11 @@ enum : uint32_t {
 struct FwdItem {
   int bh, qt;
 };
+// First KV tile a query tile needs: 0, or with a sliding window the tile holding key q0 - window.
+__device__ __forceinline__ int fwd_first_kv_tile(int qt, int window) {
+  return window < 0 ? 0 : max(0, qt * kTile - window) / kTile;
+}
+
 __device__ __forceinline__ bool fwd_item(int k, int n_items, int n_qt, FwdItem& it) {
   const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
   const long long idx = static_cast<long long>(k) * G + ((k & 1) ? G - 1 - c : c);
@@ -202,7 +208,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     int t0 = 0;  // running KV tile count: ring slot t % kFwdStages, phase (t / kFwdStages) & 1
     FwdItem it;
     for (int k = 0; fwd_item(k, n_items, n_qt, it); ++k) {
-      const int b = it.bh / p.H, h = it.bh % p.H, n_kv = it.qt + 1;
+      const int b = it.bh / p.H, h = it.bh % p.H, kt0 = fwd_first_kv_tile(it.qt, p.window), n_kv = it.qt + 1 - kt0;
       const int hk = h / (p.H / p.Hkv);  // grouped-query attention: the group's key/value head
       if (is_k) {
         // One Q buffer, which also stages each item's output for its TMA store. Q(1) may go in once Q(0) is in
@@ -229,7 +235,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         if (leader) {
           mbar_arrive_expect_tx(&full[s], 2 * 16384);
-          for (int c = 0; c < 2; ++c) tma_load_4d(ring + s * 32768 + c * 16384, tm, &full[s], c * 64, hk, j * kTile, b);
+          for (int c = 0; c < 2; ++c)
+            tma_load_4d(ring + s * 32768 + c * 16384, tm, &full[s], c * 64, hk, (kt0 + j) * kTile, b);
           if (is_k) ATTN_TRACE_EVENT(1, t);
         }
         issued[s] = t;
@@ -326,7 +333,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     int t0 = 0;
     FwdItem it;
     for (int k = 0; ok && fwd_item(k, n_items, n_qt, it); ++k) {
-      const int n_kv = it.qt + 1;
+      const int n_kv = it.qt + 1 - fwd_first_kv_tile(it.qt, p.window);
       // This item's Q is in tensor memory (copied once the previous item's MMAs had completed).
       if (!mbar_wait_warp(&bars.q_tmem, k & 1, abort, p.timeout_ns, &g_device_error, kSiteFwdMmaQ)) break;
       // Issue order S(0), S(1), S(2), PV(0), S(3), PV(1), ..., PV(n-2), PV(n-1) (tile indices within the
@@ -384,7 +391,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     bool ok = have ? copy_q(0) : true;
     int t0 = 0;
     for (int k = 0; have; ++k) {
-      const int qt = it.qt, n_kv = qt + 1;
+      const int qt = it.qt, kt0 = fwd_first_kv_tile(qt, p.window), n_kv = qt + 1 - kt0;
       FwdItem next;
       const bool have_next = fwd_item(k + 1, n_items, n_qt, next);
       float m = -INFINITY;  // running max (scale*log2(e) units, stale by < 2^8) after this group's last tile
@@ -413,10 +420,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_arrive_warp(&bars.s_free[sb]);  // S(t+2) may now be written over this buffer
         if (lane == 0 && t < 8) ATTN_TRACE_EVENT(12, t * 8 + warp - 2);
         if (tracer) ATTN_TRACE_EVENT(8, t);
-        if (j == qt) {  // diagonal tile: key column > query row is masked
+        if (kt0 + j == qt) {  // diagonal tile: key column > query row is masked
 #pragma unroll
           for (int i = 0; i < 128; ++i)
             if (i > row) s[i] = -INFINITY;
+        }
+        if (p.window >= 0) {  // sliding window: key (kt0+j)*128 + i < query - window is masked
+          const int lo = qt * kTile + row - p.window - (kt0 + j) * kTile;  // first visible column of this row
+          if (lo > 0) {
+#pragma unroll
+            for (int i = 0; i < 128; ++i)
+              if (i < lo) s[i] = -INFINITY;
+          }
         }
         // Row max of the tile as a tree over 16 independent partial maxima.
         float pm[16];
@@ -451,7 +466,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (tracer) ATTN_TRACE_EVENT(11, t);
         // P = exp2(c*S - m_j) for the 128 keys and the row sum, packed to bf16 pairs in registers. The last
         // kFwdPolyPairs pairs of every 16 go through the FMA-pipe exp2 (exp2_poly), the rest through MUFU ex2.
-        const float neg_m = -m_j;
+        // A row that has seen no key yet (only possible left of a sliding window) keeps m_j = -inf and all
+        // its scores are -inf: the reference 0 gives P = 0 there instead of NaN.
+        const float neg_m = m_j == -INFINITY ? 0.f : -m_j;
         float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial row sums
         uint32_t pk[4][16];
 #pragma unroll

@@ -118,6 +118,21 @@ attn_status attn_bwd_gqa(const void* q, const void* k, const void* v, const void
                          int B, int H, int H_kv, int T, int D, float scale, void* stream);
 
 /*
+ * General form: grouped-query attention (H_kv as for attn_fwd_gqa) and a sliding window. With window >= 0,
+ * query i sees keys i - window .. i only: itself and the `window` keys before it, flash_attn's
+ * window_size = (window, 0) next to causal (apidog "Train your own ChatGPT", section 5 "Flash Attention
+ * integration": flash_attn_func takes window_size; section 1 "GPT model": layers alternate short and long
+ * windows, "SSSL"; the pages give no length). window = -1: no window (plain causal). KV tiles wholly left
+ * of a query tile's window, and query tiles wholly past a key tile's window, are skipped. The forward's lse
+ * is the log-sum-exp over the window. window < -1: ATTN_ERR_INVALID_ARG. Same shapes and contract otherwise.
+ */
+attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int H_kv,
+                        int T, int D, float scale, int window, void* stream);
+attn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                        int B, int H, int H_kv, int T, int D, float scale, int window, void* stream);
+
+/*
  * Backward without caller-provided workspace, for callers that cannot allocate device memory (a custom-op or
  * plugin interface that passes tensors but no allocator or workspace; a fixed memory plan that forbids
  * cudaMalloc/cudaFree, and the synchronisation they can cause, during a step). The pages have no counterpart:

@@ -127,6 +127,19 @@ def test_gqa_argument_errors(lib):
     assert lib.attn_bwd_gqa(*args(dk=ptrs[1]), ws, 1, 6, 2, 128, 128, 0.088, None) == 1    # dk aliases k
 
 
+def test_window_argument_errors(lib):
+    """attn_fwd_ex / attn_bwd_ex take window >= 0, or -1 for none; anything below is an argument error."""
+    qsize = 1 * 128 * 2 * 128 * 2
+    q, k, v, o, lse = fake_ptrs(5, qsize)
+    for w in (-2, -100):
+        assert lib.attn_fwd_ex(q, k, v, o, lse, 1, 2, 2, 128, 128, 0.088, w, None) == 1
+    assert lib.attn_fwd_ex(q, k, v, o, lse, 1, 2, 3, 128, 128, 0.088, 5, None) == 1  # H_kv does not divide H
+    ws = lib.attn_bwd_workspace_bytes(1, 2, 128, 128)
+    ptrs = fake_ptrs(10, max(qsize, ws))
+    assert lib.attn_bwd_ex(*ptrs, ws, 1, 2, 2, 128, 128, 0.088, -2, None) == 1
+    assert lib.attn_bwd_ex(*ptrs, ws - 1, 1, 2, 2, 128, 128, 0.088, 4, None) == 6
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
 def test_no_cpu_fallback_without_gpu(lib):
     """A well-formed call on a machine without an sm_100 GPU fails loudly instead of computing on the CPU."""

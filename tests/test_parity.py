@@ -55,11 +55,11 @@ def to64(t):
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def run_gpu(q, k, v, do, scale):
+def run_gpu(q, k, v, do, scale, window=None):
     dev = torch.device("cuda")
     qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, do))
-    o, lse = attn.attn_fwd(qd, kd, vd, scale)
-    dq, dk, dv = attn.attn_bwd(qd, kd, vd, o, lse, dod, scale)
+    o, lse = attn.attn_fwd(qd, kd, vd, scale, window=window)
+    dq, dk, dv = attn.attn_bwd(qd, kd, vd, o, lse, dod, scale, window=window)
     torch.cuda.synchronize()
     assert attn.get_device_error() == 0
     return o, lse, dq, dk, dv
@@ -67,10 +67,11 @@ def run_gpu(q, k, v, do, scale):
 
 def full_compare(w: Workload):
     q, k, v, do = make_inputs(w)
-    o, lse, dq, dk, dv = run_gpu(q, k, v, do, w.scale)
-    O_ref, LSE_ref = attn_ref.attention_forward(q, k, v, w.scale)
-    dQ_ref, dK_ref, dV_ref, _ = attn_ref.attention_backward(q, k, v, do, w.scale)
-    what = f"{w.name} B={w.B} H={w.H} T={w.T}"
+    win = w.window if w.window >= 0 else None
+    o, lse, dq, dk, dv = run_gpu(q, k, v, do, w.scale, win)
+    O_ref, LSE_ref = attn_ref.attention_forward(q, k, v, w.scale, window=win)
+    dQ_ref, dK_ref, dV_ref, _ = attn_ref.attention_backward(q, k, v, do, w.scale, window=win)
+    what = f"{w.name} B={w.B} H={w.H} Hkv={w.kv_heads} T={w.T} window={w.window}"
     check_o(to64(o), O_ref, what)
     check_lse(to64(lse), LSE_ref, what)
     check_grad(to64(dq), dQ_ref, "dQ", what)
@@ -167,6 +168,46 @@ def test_gqa_full_size_sampled_groups(name):
         check_grad(to64(dv[b, :, hk]), dv_ref, "dV", f"{name} kv head (b={b}, hk={hk})")
     for t in (o, dq, dk, dv):
         assert bool(torch.isfinite(t.float()).all())
+
+
+# Sliding window: query i sees keys i - window .. i. Windows below, at and above a tile (64 or 128 rows), 0
+# (each query sees only itself) and 1, ragged T, and combined with grouped-query attention.
+WINDOW_SHAPES = [(1, 2, 2, 300, 100), (1, 1, 1, 257, 0), (1, 1, 1, 200, 1), (2, 2, 2, 513, 127), (1, 2, 2, 384, 128),
+                 (1, 2, 1, 401, 129), (1, 4, 2, 640, 63), (1, 2, 2, 700, 200), (1, 1, 1, 130, 500)]
+
+
+@pytest.mark.parametrize("B,H,Hkv,T,window", WINDOW_SHAPES,
+                         ids=[f"B{b}H{h}Hkv{hk}T{t}W{w}" for b, h, hk, t, w in WINDOW_SHAPES])
+def test_window_full(B, H, Hkv, T, window):
+    full_compare(Workload("sw", B=B, H=H, T=T, Hkv=Hkv, window=window, seed=T + window))
+
+
+def test_window_tiny_workload():
+    full_compare(WORKLOADS["tiny_sw"])
+
+
+def test_window_full_size_sampled_slices():
+    """d20 shape with a 512-key window, at full size through the benchmark's launch; sampled slices."""
+    w = WORKLOADS["d20_sw"]
+    q, k, v, do = make_inputs(w)
+    o, lse, dq, dk, dv = run_gpu(q, k, v, do, w.scale, w.window)
+    for (b, h) in sample_slices(w, k=2):
+        ref = attn_ref.slice_forward_backward(q, k, v, do, b, h, w.scale, window=w.window)
+        what = f"d20_sw slice (b={b}, h={h})"
+        check_o(to64(o[b, :, h]), ref["o"], what)
+        check_lse(to64(lse[b, h]), ref["lse"], what)
+        check_grad(to64(dq[b, :, h]), ref["dq"], "dQ", what)
+        check_grad(to64(dk[b, :, h]), ref["dk"], "dK", what)
+        check_grad(to64(dv[b, :, h]), ref["dv"], "dV", what)
+
+
+def test_window_zero_gives_v_exactly():
+    """window 0: every query sees only its own key, so O = V exactly and dV = dO exactly."""
+    w = Workload("w0", B=1, H=2, T=300, window=0, seed=9)
+    q, k, v, do = make_inputs(w)
+    o, lse, dq, dk, dv = run_gpu(q, k, v, do, w.scale, 0)
+    assert torch.equal(o.cpu(), v)
+    assert torch.equal(dv.cpu(), do)
 
 
 def test_causality_on_gpu():
