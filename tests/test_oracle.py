@@ -360,6 +360,65 @@ def test_window_gradients_by_finite_differences():
 
 
 # ---------------------------------------------------------------------------------------------------------
+# Decode against a key/value cache: query i of Tq sits at position L - Tq + i.
+
+def test_decode_equals_training_forward_when_the_cache_is_the_sequence():
+    """Tq = L: the new queries are the whole sequence, so decode is the causal training forward."""
+    B, T, H, Hkv, D = 2, 21, 4, 2, 8
+    rng = np.random.default_rng(11)
+    q = rng.standard_normal((B, T, H, D))
+    k, v = rng.standard_normal((B, T, Hkv, D)), rng.standard_normal((B, T, Hkv, D))
+    s = 0.3
+    O, LSE = attn_ref.decode_forward(q, k, v, [T, T], s)
+    O2, LSE2 = attn_ref.attention_forward(q, k, v, s)
+    np.testing.assert_allclose(O, O2, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(LSE, LSE2, rtol=1e-13, atol=1e-13)
+
+
+def test_decode_matches_torch_per_sequence():
+    """Ragged cache lengths, spare cache rows filled with garbage (never read), Tq = 3: each sequence equals
+    torch's float64 SDPA on its valid cache with the end-aligned causal mask (and enable_gqa)."""
+    B, Tq, H, Hkv, Tk, D = 3, 3, 6, 2, 40, 16
+    rng = np.random.default_rng(12)
+    q = rng.standard_normal((B, Tq, H, D))
+    kc, vc = rng.standard_normal((B, Tk, Hkv, D)), rng.standard_normal((B, Tk, Hkv, D))
+    lens = [40, 17, 3]
+    s = 1 / math.sqrt(D)
+    O, LSE = attn_ref.decode_forward(q, kc, vc, lens, s)
+    for b, L in enumerate(lens):
+        tq = torch.tensor(q[b:b + 1]).transpose(1, 2)
+        tk, tv = (torch.tensor(x[b:b + 1, :L]).transpose(1, 2) for x in (kc, vc))
+        pos = torch.arange(L - Tq, L)[:, None]
+        mask = torch.arange(L)[None, :] <= pos
+        ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=s, enable_gqa=True)
+        np.testing.assert_allclose(O[b:b + 1], ref.transpose(1, 2).numpy(), rtol=1e-12, atol=1e-12)
+    # garbage past the lengths does not matter
+    kc2, vc2 = kc.copy(), vc.copy()
+    kc2[1, 17:] = 1e6
+    vc2[2, 3:] = np.nan
+    O2, _ = attn_ref.decode_forward(q, kc2, vc2, lens, s)
+    np.testing.assert_array_equal(O, O2)
+
+
+def test_decode_single_query_and_empty_rows():
+    """Tq = 1 sees the whole valid cache (softmax over all L keys); a query before the first key (L < Tq)
+    returns 0 with LSE -inf; L = 1 returns the one value."""
+    B, Tk, H, D = 2, 9, 1, 4
+    rng = np.random.default_rng(13)
+    q = rng.standard_normal((B, 2, H, D))
+    kc, vc = rng.standard_normal((B, Tk, H, D)), rng.standard_normal((B, Tk, H, D))
+    s = 0.5
+    O, LSE = attn_ref.decode_forward(q[:, :1], kc, vc, [9, 1], s)
+    sc = s * kc[0, :, 0] @ q[0, 0, 0]
+    p = np.exp(sc - sc.max()) / np.exp(sc - sc.max()).sum()
+    np.testing.assert_allclose(O[0, 0, 0], p @ vc[0, :, 0], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(O[1, 0, 0], vc[1, 0, 0], rtol=0, atol=1e-15)
+    O2, LSE2 = attn_ref.decode_forward(q, kc, vc, [9, 1], s)   # Tq = 2, second sequence has one key
+    assert np.all(O2[1, 0, 0] == 0) and LSE2[1, 0, 0] == -np.inf
+    np.testing.assert_allclose(O2[1, 1, 0], vc[1, 0, 0], rtol=0, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------------------------------------
 # Mutation test: plant plausible mistakes in a copy of the oracle and require that some pin fails.
 
 def _mutant(kind):

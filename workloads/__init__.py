@@ -153,3 +153,51 @@ def sample_slices(w: Workload, k: int = 4, seed: int = 1234):
         if (b, h) not in picks:
             picks.append((b, h))
     return picks
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    """New queries against a key/value cache (the inference engine's cached decode): q [B, Tq, H, D], caches
+    [B, Tk, H_kv, D], cache_seqlens [B] drawn uniformly from [min_len, Tk] (a seeded mix of lengths)."""
+
+    name: str
+    B: int
+    H: int
+    Hkv: int
+    Tq: int
+    Tk: int
+    D: int = HEAD_DIM
+    min_len: int = 1
+    seed: int = 0
+    recipe: str = ""
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+
+DECODE_WORKLOADS: Dict[str, DecodeWorkload] = {
+    "decode_tiny": DecodeWorkload("decode_tiny", B=3, H=4, Hkv=2, Tq=2, Tk=300, seed=1,
+                                  recipe="q, caches ~ N(0,1) bf16; lengths uniform in [1, 300]"),
+    "decode_d20": DecodeWorkload("decode_d20", B=64, H=10, Hkv=10, Tq=1, Tk=2048, seed=2,
+                                 recipe="d20 heads, one new token per sequence, 64 sequences with cached lengths "
+                                        "uniform in [1, 2048]; q, caches ~ N(0,1) bf16"),
+    "decode_d20_gqa": DecodeWorkload("decode_d20_gqa", B=64, H=10, Hkv=5, Tq=1, Tk=2048, seed=3,
+                                     recipe="decode_d20 with 5 key/value heads"),
+}
+
+
+def make_decode_inputs(w: DecodeWorkload, device: Optional[torch.device] = None):
+    """(q, k_cache, v_cache, cache_seqlens): bf16 tensors and int32 lengths from one seeded CPU generator, in
+    the order lengths, q, k_cache, v_cache."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+    lens = torch.randint(w.min_len, w.Tk + 1, (w.B,), generator=g, dtype=torch.int64).to(torch.int32)
+    q = torch.randn((w.B, w.Tq, w.H, w.D), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    kc = torch.randn((w.B, w.Tk, w.Hkv, w.D), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    vc = torch.randn((w.B, w.Tk, w.Hkv, w.D), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    out = (q, kc, vc, lens)
+    if device is not None:
+        out = tuple(t.to(device) for t in out)
+    return out
+
