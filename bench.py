@@ -16,6 +16,7 @@ from __future__ import annotations
 
 import argparse
 import ctypes
+import dataclasses
 import hashlib
 import json
 import math
@@ -35,7 +36,7 @@ from workloads import WORKLOADS, Workload  # noqa: E402
 METRIC = "causal attention fwd+bwd TFLOP/s (bf16, d20 shape) and % of B200 tensor peak"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
-KERNEL_SOURCES = ["attn_api.cu", "attn_fwd.cuh", "attn_bwd.cuh", "attn_common.cuh", "sm100.cuh"]
+KERNEL_SOURCES = ["attn_api.cu", "attn_fwd.cuh", "attn_bwd.cuh", "attn_decode.cuh", "attn_common.cuh", "sm100.cuh"]
 
 
 def parse_args(argv=None):
@@ -43,7 +44,8 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="d20", choices=sorted(WORKLOADS))
+    from workloads import DECODE_WORKLOADS
+    ap.add_argument("--workload", default="d20", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
@@ -464,8 +466,105 @@ def run_ours(args):
     return 0
 
 
+DECODE_METRIC = "KV-cache decode attention HBM GB/s (bf16 cache)"
+
+
+def decode_bytes(w, lens):
+    """Algorithmic bytes of one decode call: the valid K and V rows, q, o and lse."""
+    kv = sum(int(x) for x in lens) * w.Hkv * w.D * 2 * 2
+    return kv + 2 * w.B * w.Tq * w.H * w.D * 2 + w.B * w.H * w.Tq * 4
+
+
+def run_decode(args):
+    """Cached decode (forward only): HBM-bound, measured in GB/s of algorithmic bytes against the measured
+    copy bandwidth. Inputs (q, caches over 1 GB in all for the d20 workloads) are resident; no L2 flush needed
+    when the cache exceeds L2, which the line states."""
+    from workloads import DECODE_WORKLOADS, make_decode_inputs
+    w = DECODE_WORKLOADS[args.workload]
+    rank, world, _ = dist_env()
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        from threadpoolctl import threadpool_limits
+
+        from oracle import attn_ref
+        q, kc, vc, lens = make_decode_inputs(w)
+        n = min(w.B, 4)
+        times = []
+        with threadpool_limits(limits=len(os.sched_getaffinity(0))):
+            for it in range(args.warmup + args.steps):
+                t0 = time.perf_counter()
+                attn_ref.decode_forward(q[:n], kc[:n], vc[:n], lens[:n].numpy(), w.scale)
+                if it >= args.warmup:
+                    times.append(time.perf_counter() - t0)
+        sw = dataclasses.replace(w, B=n)
+        value = decode_bytes(sw, lens[:n]) / (sum(times) / len(times)) / 1e9
+        print(json.dumps({"metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+                          "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "impl": "reference",
+                          "dtype": "f64", "data": "synthetic", "config": {"workload": w.name, "recipe": w.recipe},
+                          "cpu_baseline": {"value": value, "unit": "GB/s", "cores": len(os.sched_getaffinity(0)),
+                                           "kind": "oracle", "sample": f"{n} sequences of {w.name} per step"}}))
+        return 0
+    import torch
+
+    import causal_self_attention_bf16_b200 as attn
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    q, kc, vc, lens = (t.to(device) for t in make_decode_inputs(w))
+    o, lse = torch.empty_like(q), torch.empty((w.B, w.H, w.Tq), dtype=torch.float32, device=device)
+    lib = attn.load_library()
+    ws_bytes = int(lib.attn_decode_workspace_bytes(w.B, w.H, w.Hkv, w.Tq, w.Tk, w.D))
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
+    sh = torch.cuda.current_stream(device).cuda_stream
+
+    def call():
+        st = lib.attn_decode(q.data_ptr(), kc.data_ptr(), vc.data_ptr(), lens.data_ptr(), o.data_ptr(),
+                             lse.data_ptr(), ws.data_ptr(), ws_bytes, w.B, w.H, w.Hkv, w.Tq, w.Tk, w.D, w.scale, sh)
+        if st != 0:
+            raise RuntimeError(f"attn_decode: {attn._STATUS.get(st, st)}")
+
+    for _ in range(max(args.warmup, 3)):
+        call()
+    torch.cuda.synchronize(device)
+    # The cache of one call is smaller than L2 for some workloads: a 256 MB buffer is written between calls.
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.1)
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record()
+        call()
+        e1.record()
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    if attn.get_device_error() != 0:
+        raise RuntimeError("a decode kernel reported an error")
+    ms = sum(a.elapsed_time(b) for a, b in ev) / len(ev)
+    nbytes = decode_bytes(w, lens.cpu())
+    gbs = nbytes / (ms / 1e3) / 1e9
+    hbm = float(load_peaks()["hbm_gbs"])
+    print(json.dumps({
+        "metric": DECODE_METRIC, "value": gbs * world, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "ours",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.Hkv, "Tq": w.Tq, "Tk": w.Tk, "D": w.D,
+                   "recipe": w.recipe, "l2": "256 MB written between calls",
+                   "parallelism": f"replicas x{world} (no collective on the data path)"},
+        "roofline": {"kernel": "attn_decode (split + combine)", "bound": "hbm", "achieved": gbs, "peak": hbm,
+                     "unit": "GB/s", "frac": gbs / hbm, "traffic": None, "alg_bytes": nbytes},
+        "gpu_launches": 2 * args.steps, "clocks": clocks, "kernel_source_hash": kernel_source_hash(),
+    }))
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
+    from workloads import DECODE_WORKLOADS
+    if args.workload in DECODE_WORKLOADS:
+        return run_decode(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -42,6 +42,8 @@ SIGNATURES = {
     "attn_bwd_gqa": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _I, _F, _VP], _I),
     "attn_fwd_ex": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP], _I),
     "attn_bwd_ex": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _I, _F, _I, _VP], _I),
+    "attn_decode_workspace_bytes": ([_I] * 6, _SZ),
+    "attn_decode": ([_VP] * 7 + [_SZ] + [_I] * 6 + [_F, _VP], _I),
     "attn_get_device_error": ([ctypes.POINTER(ctypes.c_uint32)], _I),
     "attn_clear_device_error": ([], _I),
     "attn_set_wait_limit_ns": ([_U64], _I),
@@ -230,6 +232,40 @@ def attn_bwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch
     return dq, dk, dv
 
 
+def attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, cache_seqlens: torch.Tensor,
+                scale: Optional[float] = None, o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+    """Attention of Tq new queries against a key/value cache (the inference engine's cached decode).
+    q: bf16 [B, Tq, H, D]; k_cache, v_cache: bf16 [B, Tk, H_kv, D]; cache_seqlens: int32 [B] on the device, the
+    valid keys of each sequence (new tokens included). Query i sees keys 0 .. L - Tq + i. Returns
+    (o [B, Tq, H, D], lse [B, H, Tq])."""
+    lib = load_library()
+    _check_qkv("q", q)
+    _check_qkv("k_cache", k_cache)
+    B, Tq, H, D = q.shape
+    Tk, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape[0] != B or k_cache.shape[3] != D:
+        raise ValueError(f"k_cache has shape {tuple(k_cache.shape)}; expected [{B}, Tk, H_kv, {D}]")
+    _check_qkv("v_cache", v_cache, k_cache.shape)
+    if (cache_seqlens.dtype != torch.int32 or tuple(cache_seqlens.shape) != (B,) or
+            cache_seqlens.device != q.device or not cache_seqlens.is_contiguous()):
+        raise ValueError("cache_seqlens must be a contiguous int32 [B] tensor on q's device")
+    o = torch.empty_like(q) if o is None else o
+    _check_qkv("o", o, q.shape)
+    if lse is None:
+        lse = torch.empty((B, H, Tq), dtype=torch.float32, device=q.device)
+    need = int(lib.attn_decode_workspace_bytes(B, H, Hkv, Tq, Tk, D))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    scale = default_scale(D) if scale is None else float(scale)
+    st = lib.attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cache_seqlens.data_ptr(),
+                         o.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                         workspace.numel() * workspace.element_size(), B, H, Hkv, Tq, Tk, D, scale,
+                         _stream_handle(stream, q.device))
+    _check("attn_decode", st)
+    return o, lse
+
+
 def get_device_error() -> int:
     """The library's device-side error word (0 = no kernel gave up on a bounded wait). Synchronises."""
     word = ctypes.c_uint32(0)
@@ -276,6 +312,6 @@ def causal_attention(q, k, v, scale: Optional[float] = None, window: Optional[in
     return CausalAttentionFunction.apply(q, k, v, default_scale(q.shape[-1]) if scale is None else scale, window)
 
 
-__all__ = ["attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "causal_attention", "CausalAttentionFunction",
+__all__ = ["attn_fwd", "attn_bwd", "attn_decode", "attn_bwd_workspace_bytes", "causal_attention", "CausalAttentionFunction",
            "get_device_error", "clear_device_error", "set_wait_limit_ns", "selftest_wait_timeout", "AttnError",
            "load_library", "LIB_PATH", "SIGNATURES"]

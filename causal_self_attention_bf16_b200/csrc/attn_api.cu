@@ -10,6 +10,7 @@
 
 #include "attn.h"
 #include "attn_bwd.cuh"
+#include "attn_decode.cuh"
 #include "attn_fwd.cuh"
 
 namespace {
@@ -481,3 +482,118 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
 }
 
 }  // extern "C"
+
+namespace {
+
+// Splits of the cache per (sequence, key/value head): enough CTAs for ~8 per SM of a 148-SM part (each holds
+// ~64 KB of loads in flight), each split at least kDecChunkKeys keys (a multiple of the 128-key block).
+void decode_split(int B, int Hkv, int Tk, int* n_split, int* chunk) {
+  const long long pairs = static_cast<long long>(B) * Hkv;
+  long long want = (8 * 148 + pairs - 1) / pairs;
+  const long long max_split = (Tk + attn::kDecChunkKeys - 1) / attn::kDecChunkKeys;
+  if (want > max_split) want = max_split;
+  if (want < 1) want = 1;
+  long long c = (Tk + want - 1) / want;
+  c = (c + attn::kDecKeys - 1) / attn::kDecKeys * attn::kDecKeys;
+  *chunk = static_cast<int>(c);
+  *n_split = static_cast<int>((Tk + c - 1) / c);
+}
+
+attn_status check_decode(int B, int H, int Hkv, int Tq, int Tk, int D, float scale) {
+  if (B < 1 || H < 1 || Tq < 1 || Tk < 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  attn_status st = check_kv_heads(H, Hkv);
+  if (st != ATTN_OK) return st;
+  if (D != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((H / Hkv) * static_cast<long long>(Tq) > attn::kDecMaxRows) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * Hkv * ((Tk + attn::kDecChunkKeys - 1) / attn::kDecChunkKeys) > 0x7fffffffLL ||
+      static_cast<long long>(B) * H * Tq > 0x7fffffffLL / 8)
+    return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+size_t decode_workspace(int B, int H, int Hkv, int Tq, int Tk) {
+  int n_split = 1, chunk = 0;
+  decode_split(B, Hkv, Tk, &n_split, &chunk);
+  const size_t rows = static_cast<size_t>(B) * Hkv * n_split * ((H / Hkv) * Tq);
+  return rows * 128 * 4 + rows * 2 * 4;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t attn_decode_workspace_bytes(int B, int H, int H_kv, int Tq, int Tk, int D) {
+  if (check_decode(B, H, H_kv, Tq, Tk, D, 1.0f) != ATTN_OK) return 0;
+  return decode_workspace(B, H, H_kv, Tq, Tk);
+}
+
+attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* cache_seqlens, void* o,
+                        float* lse, void* workspace, size_t workspace_bytes, int B, int H, int H_kv, int Tq, int Tk,
+                        int D, float scale, void* stream) {
+  if (!q || !k_cache || !v_cache || !cache_seqlens || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  attn_status st = check_decode(B, H, H_kv, Tq, Tk, D, scale);
+  if (st != ATTN_OK) return st;
+  const size_t need = decode_workspace(B, H, H_kv, Tq, Tk);
+  if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  for (const void* ptr : {q, k_cache, v_cache, static_cast<const void*>(o), static_cast<const void*>(workspace)})
+    if (!aligned16(ptr)) return ATTN_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u))
+    return ATTN_ERR_MISALIGNED;
+  const size_t qbytes = static_cast<size_t>(B) * Tq * H * D * 2;
+  const size_t cbytes = static_cast<size_t>(B) * Tk * H_kv * D * 2;
+  const Range ins[4] = {span(q, qbytes), span(k_cache, cbytes), span(v_cache, cbytes),
+                        span(cache_seqlens, static_cast<size_t>(B) * 4)};
+  const Range outs[3] = {span(o, qbytes), span(lse, static_cast<size_t>(B) * H * Tq * 4), span(workspace, need)};
+  for (int i = 0; i < 3; ++i) {
+    for (int j = 0; j < 4; ++j)
+      if (overlap(outs[i], ins[j])) return ATTN_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 3; ++j)
+      if (overlap(outs[i], outs[j])) return ATTN_ERR_INVALID_ARG;
+  }
+  int dev = 0;
+  if ((st = prepare_device(&dev)) != ATTN_OK) return st;
+  attn::DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k_cache);
+  p.v = static_cast<const __nv_bfloat16*>(v_cache);
+  p.seqlens = cache_seqlens;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Hkv = H_kv;
+  p.Tq = Tq;
+  p.Tk = Tk;
+  p.R = (H / H_kv) * Tq;
+  decode_split(B, H_kv, Tk, &p.n_split, &p.chunk);
+  const size_t rows = static_cast<size_t>(B) * H_kv * p.n_split * p.R;
+  p.part_o = static_cast<float*>(workspace);
+  p.part_ml = static_cast<float*>(workspace) + rows * 128;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * H_kv * p.n_split);
+  cudaError_t e = cudaSuccess;
+  auto launch = [&](auto kernel, size_t smem_bytes) {
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes));
+    if (e == cudaSuccess) kernel<<<grid, attn::kDecThreads, smem_bytes, s>>>(p);
+  };
+  if (p.R <= 1) launch(attn::attn_decode_split_kernel<1>, attn::dec_smem_bytes<1>());
+  else if (p.R <= 2) launch(attn::attn_decode_split_kernel<2>, attn::dec_smem_bytes<2>());
+  else if (p.R <= 4) launch(attn::attn_decode_split_kernel<4>, attn::dec_smem_bytes<4>());
+  else if (p.R <= 8) launch(attn::attn_decode_split_kernel<8>, attn::dec_smem_bytes<8>());
+  else if (p.R <= 16) launch(attn::attn_decode_split_kernel<16>, attn::dec_smem_bytes<16>());
+  else launch(attn::attn_decode_split_kernel<32>, attn::dec_smem_bytes<32>());
+  if (e != cudaSuccess) return cuda_fail(e, "attn_decode_split_kernel attribute");
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "attn_decode_split_kernel launch");
+  const long long out_rows = static_cast<long long>(B) * H * Tq;
+  attn::attn_decode_combine_kernel<<<static_cast<unsigned>((out_rows + 7) / 8), 256, 0, s>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_decode_combine_kernel launch");
+  return ATTN_OK;
+}
+
+}  // extern "C"
+

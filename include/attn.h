@@ -133,6 +133,27 @@ attn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void*
                         int B, int H, int H_kv, int T, int D, float scale, int window, void* stream);
 
 /*
+ * Attention of Tq new queries against a key/value cache: the inference engine's cached decode
+ * (apidog "Train your own ChatGPT", section 6 "Inference engine": flash_attn_with_kvcache over a prefilled
+ * prompt cache). Forward only.
+ *   q            in : bf16 [B, Tq, H, D]
+ *   k_cache      in : bf16 [B, Tk, H_kv, D];  v_cache in : bf16 [B, Tk, H_kv, D]  (H_kv divides H, grouped as
+ *                     in attn_fwd_gqa)
+ *   cache_seqlens in: device int32 [B], valid keys of each sequence, the new tokens' keys included (the
+ *                     caller writes them into the cache first); values outside [0, Tk] are clamped
+ *   o           out : bf16 [B, Tq, H, D];  lse out : fp32 [B, H, Tq] (natural log)
+ *   workspace scratch: attn_decode_workspace_bytes(B, H, H_kv, Tq, Tk, D) bytes, 16-byte aligned
+ * Query i of sequence b sits at position L_b - Tq + i and sees keys 0 .. L_b - Tq + i; a query that sees no
+ * key gets o = 0, lse = -inf. (H / H_kv) * Tq must be <= 32 and D = 128 (else ATTN_ERR_UNSUPPORTED).
+ * Launches two kernels (per cache chunk, then the merge of the chunks). Calls sharing a workspace must not
+ * overlap in time on the GPU.
+ */
+size_t attn_decode_workspace_bytes(int B, int H, int H_kv, int Tq, int Tk, int D);
+attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* cache_seqlens, void* o,
+                        float* lse, void* workspace, size_t workspace_bytes, int B, int H, int H_kv, int Tq, int Tk,
+                        int D, float scale, void* stream);
+
+/*
  * Backward without caller-provided workspace, for callers that cannot allocate device memory (a custom-op or
  * plugin interface that passes tensors but no allocator or workspace; a fixed memory plan that forbids
  * cudaMalloc/cudaFree, and the synchronisation they can cause, during a step). The pages have no counterpart:

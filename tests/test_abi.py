@@ -140,6 +140,25 @@ def test_window_argument_errors(lib):
     assert lib.attn_bwd_ex(*ptrs, ws - 1, 1, 2, 2, 128, 128, 0.088, 4, None) == 6
 
 
+def test_decode_argument_errors(lib):
+    """attn_decode checks sizes, the row limit, the workspace and overlaps before any CUDA call."""
+    assert lib.attn_decode_workspace_bytes(2, 8, 2, 1, 1000, 128) > 0
+    assert lib.attn_decode_workspace_bytes(2, 8, 3, 1, 1000, 128) == 0     # H_kv does not divide H
+    assert lib.attn_decode_workspace_bytes(2, 64, 1, 1, 1000, 128) == 0    # 64 rows per CTA > 32
+    ws = lib.attn_decode_workspace_bytes(2, 8, 2, 1, 1000, 128)
+    q, kc, vc, lens, o, lse, w = fake_ptrs(7, max(2 * 1000 * 2 * 128 * 2, ws))
+    call = lambda **kw: lib.attn_decode(kw.get("q", q), kc, vc, kw.get("lens", lens), kw.get("o", o), lse,
+                                        kw.get("w", w), kw.get("wb", ws), 2, 8, kw.get("hkv", 2), 1, 1000,
+                                        kw.get("D", 128), 0.088, None)
+    assert call(q=None) == 1
+    assert call(hkv=3) == 1
+    assert call(D=64) == 2
+    assert call(wb=ws - 1) == 6
+    assert call(o=q) == 1                 # o aliases q
+    assert call(w=kc) == 1                # workspace aliases the cache
+    assert call(lens=lens + 2) == 3       # lengths must be 4-byte aligned
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
 def test_no_cpu_fallback_without_gpu(lib):
     """A well-formed call on a machine without an sm_100 GPU fails loudly instead of computing on the CPU."""

@@ -210,6 +210,45 @@ def test_window_zero_gives_v_exactly():
     assert torch.equal(dv.cpu(), do)
 
 
+# Decode against a key/value cache (forward only).
+DECODE_CASES = [("decode_tiny", None), ("small_mha", dict(B=2, H=2, Hkv=2, Tq=1, Tk=1000)),
+                ("gqa_tq3", dict(B=3, H=8, Hkv=2, Tq=3, Tk=700)), ("short", dict(B=4, H=1, Hkv=1, Tq=4, Tk=5)),
+                ("rows32", dict(B=1, H=16, Hkv=2, Tq=4, Tk=1300)), ("long", dict(B=1, H=2, Hkv=1, Tq=1, Tk=9000))]
+
+
+@pytest.mark.parametrize("name,shape", DECODE_CASES, ids=[c[0] for c in DECODE_CASES])
+def test_decode_full(name, shape):
+    from workloads import DECODE_WORKLOADS, DecodeWorkload, make_decode_inputs
+    w = DECODE_WORKLOADS[name] if shape is None else DecodeWorkload(name, seed=len(name), **shape)
+    q, kc, vc, lens = make_decode_inputs(w)
+    if name == "short":
+        lens = torch.tensor([0, 1, 3, 5], dtype=torch.int32)  # empty cache, fewer keys than new queries, full
+    dev = torch.device("cuda")
+    o, lse = attn.attn_decode(q.to(dev), kc.to(dev), vc.to(dev), lens.to(dev), w.scale)
+    torch.cuda.synchronize()
+    O_ref, LSE_ref = attn_ref.decode_forward(q, kc, vc, lens.numpy(), w.scale)
+    what = f"{name} lens={lens.tolist()[:6]}"
+    check_o(to64(o), O_ref, what)
+    finite = np.isfinite(LSE_ref)
+    assert np.array_equal(np.isfinite(to64(lse)), finite), f"{what}: -inf LSE pattern differs"
+    check_lse(to64(lse)[finite], LSE_ref[finite], what)
+    assert np.all(to64(o)[np.broadcast_to(~finite.transpose(0, 2, 1)[..., None], O_ref.shape)] == 0)
+
+
+def test_decode_full_size_sampled():
+    """The benchmark's decode workload (64 sequences, d20 heads, ragged lengths up to 2048), oracle on samples."""
+    from workloads import DECODE_WORKLOADS, make_decode_inputs
+    w = DECODE_WORKLOADS["decode_d20_gqa"]
+    q, kc, vc, lens = make_decode_inputs(w)
+    dev = torch.device("cuda")
+    o, lse = attn.attn_decode(q.to(dev), kc.to(dev), vc.to(dev), lens.to(dev), w.scale)
+    torch.cuda.synchronize()
+    for b in (0, 17, w.B - 1):
+        O_ref, LSE_ref = attn_ref.decode_forward(q[b:b + 1], kc[b:b + 1], vc[b:b + 1], lens[b:b + 1].numpy(), w.scale)
+        check_o(to64(o[b:b + 1]), O_ref, f"decode_d20_gqa b={b}")
+        check_lse(to64(lse[b:b + 1]), LSE_ref, f"decode_d20_gqa b={b}")
+
+
 def test_causality_on_gpu():
     """Perturbing q/k/v after position t leaves O and LSE at positions <= t bit-identical."""
     w = Workload("causal", B=2, H=2, T=300, seed=9)
