@@ -57,3 +57,50 @@ def test_sample_slices_include_corners_and_are_unique():
     assert s[0] == (0, 0) and s[1] == (w.B - 1, w.H - 1)
     assert len(set(s)) == len(s) == 5
     assert all(0 <= b < w.B and 0 <= h < w.H for b, h in s)
+
+
+def test_grouped_query_inputs_and_key_bias_stream():
+    """k, v carry H_kv heads; the draw order q, k, v, dO, bias is kept when the key/value heads differ."""
+    w = WORKLOADS["tiny_gqa"]
+    q, k, v, do = make_inputs(w)
+    assert tuple(q.shape) == tuple(do.shape) == (1, 128, 4, 128)
+    assert tuple(k.shape) == tuple(v.shape) == (1, 128, 2, 128) and w.kv_heads == 2
+    wb = Workload("gb", B=1, H=4, T=9, Hkv=2, seed=4, key_bias=True)
+    _, kb, _, _ = make_inputs(wb)
+    g = torch.Generator().manual_seed(4)
+    q_ = torch.randn((1, 9, 4, 128), generator=g)
+    k_ = torch.randn((1, 9, 2, 128), generator=g)
+    assert torch.equal(kb, (k_ + key_bias_vector(wb)).to(torch.bfloat16))
+
+
+def test_window_flops_scale_with_the_pairs_inside_the_band():
+    """A window keeps min(i, W) + 1 of query i's causal keys; W >= T - 1 is the plain causal count."""
+    full = WORKLOADS["d20"]
+    assert full.with_shape(window=full.T - 1).fwd_flops == full.fwd_flops
+    w = Workload("w", B=1, H=1, T=10, window=3)
+    kept = sum(min(i, 3) + 1 for i in range(10))          # 1 + 2 + 3 + 4 * 7 = 34 of 55 causal pairs
+    assert math.isclose(w.fwd_flops, 2 * 10 * 10 * 128 * kept / 55)
+    sw = WORKLOADS["d20_sw"]
+    assert 0.4 < sw.fwd_flops / full.fwd_flops < 0.45 and math.isclose(sw.bwd_flops, 2.5 * sw.fwd_flops)
+
+
+def test_decode_inputs_are_seeded_and_ragged():
+    from workloads import DECODE_WORKLOADS, make_decode_inputs
+    w = DECODE_WORKLOADS["decode_d20_gqa"]
+    q, kc, vc, lens = make_decode_inputs(w)
+    q2, kc2, vc2, lens2 = make_decode_inputs(w)
+    assert torch.equal(lens, lens2) and torch.equal(q, q2) and torch.equal(kc, kc2)
+    assert tuple(q.shape) == (64, 1, 10, 128) and tuple(kc.shape) == (64, 2048, 5, 128)
+    assert lens.dtype == torch.int32 and int(lens.min()) >= 1 and int(lens.max()) <= 2048
+    assert len(set(lens.tolist())) > 40  # a mix of lengths, not one
+
+
+def test_bench_decode_bytes_count_only_valid_cache_rows():
+    import bench
+    from workloads import DECODE_WORKLOADS
+    w = DECODE_WORKLOADS["decode_tiny"]
+    lens = torch.tensor([10, 0, 5], dtype=torch.int32)
+    kv = 15 * w.Hkv * w.D * 2 * 2
+    assert bench.decode_bytes(w, lens) == kv + 2 * w.B * w.Tq * w.H * w.D * 2 + w.B * w.H * w.Tq * 4
+    f, b = bench.flops(WORKLOADS["d20_sw"])
+    assert f == WORKLOADS["d20_sw"].fwd_flops and b == WORKLOADS["d20_sw"].bwd_flops
