@@ -508,8 +508,15 @@ def run_decode(args):
     import torch
 
     import causal_self_attention_bf16_b200 as attn
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
     q, kc, vc, lens = (t.to(device) for t in make_decode_inputs(w))
     o, lse = torch.empty_like(q), torch.empty((w.B, w.H, w.Tq), dtype=torch.float32, device=device)
     lib = attn.load_library()
@@ -531,6 +538,9 @@ def run_decode(args):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
     sampler = ClockSampler(gpu_id)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
     sampler.start()
     time.sleep(0.1)
     for e0, e1 in ev:
@@ -540,12 +550,18 @@ def run_decode(args):
         e1.record()
     torch.cuda.synchronize(device)
     clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
     if attn.get_device_error() != 0:
         raise RuntimeError("a decode kernel reported an error")
-    ms = sum(a.elapsed_time(b) for a, b in ev) / len(ev)
+    ms = reduce_max(sum(a.elapsed_time(b) for a, b in ev) / len(ev), world, device)  # slowest rank
     nbytes = decode_bytes(w, lens.cpu())
     gbs = nbytes / (ms / 1e3) / 1e9
     hbm = float(load_peaks()["hbm_gbs"])
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
     print(json.dumps({
         "metric": DECODE_METRIC, "value": gbs * world, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",

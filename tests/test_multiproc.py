@@ -60,3 +60,15 @@ def test_reference_arm_line(monkeypatch, capsys):
     assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["config"]["workload"] == "tiny"
+
+
+def test_decode_reference_arm_line(monkeypatch, capsys):
+    """The decode workloads have their own metric (GB/s of algorithmic bytes); the reference arm times the
+    oracle on a few sequences and prints one line."""
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    import json
+    assert bench.main(["--impl", "reference", "--workload", "decode_tiny", "--steps", "1", "--warmup", "0"]) == 0
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["metric"] == bench.DECODE_METRIC and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["impl"] == "reference" and line["cpu_baseline"]["kind"] == "oracle"
