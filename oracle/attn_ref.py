@@ -195,6 +195,76 @@ def decode_forward(q, k_cache, v_cache, cache_seqlens, scale: float) -> Tuple[np
     return O, LSE
 
 
+def _rope_angles(B: int, T: int, D: int, base: float, offsets) -> np.ndarray:
+    """Rotation angles [B, T, D/2]: position p = offsets[b] + t (offsets a scalar or a length-B array) times
+    the frequency base^(-2i/D) of pair i (RoFormer, Su et al. 2021, section 3.4.2)."""
+    off = np.broadcast_to(np.asarray(offsets, dtype=np.float64), (B,))
+    pos = off[:, None] + np.arange(T, dtype=np.float64)[None, :]          # [B, T]
+    inv_freq = float(base) ** (-2.0 * np.arange(D // 2) / D)               # [D/2]
+    return pos[:, :, None] * inv_freq[None, None, :]
+
+
+def _pairs(y: np.ndarray, pairing: str):
+    """The (first, second) members of each rotated pair: interleaved (2i, 2i+1), or half (i, i + D/2)."""
+    D = y.shape[-1]
+    if pairing == "interleaved":
+        return y[..., 0::2], y[..., 1::2]
+    if pairing == "half":
+        return y[..., : D // 2], y[..., D // 2:]
+    raise ValueError(f"pairing must be 'interleaved' or 'half', got {pairing!r}")
+
+
+def _unpairs(a: np.ndarray, b: np.ndarray, pairing: str) -> np.ndarray:
+    out = np.empty(a.shape[:-1] + (2 * a.shape[-1],))
+    if pairing == "interleaved":
+        out[..., 0::2], out[..., 1::2] = a, b
+    else:
+        out = np.concatenate([a, b], axis=-1)
+    return out
+
+
+def qk_norm_rope(x, base: float = 10000.0, eps: float = 1e-6, offsets=0, pairing: str = "interleaved") -> np.ndarray:
+    """The steps the model applies to q and k before attention (apidog "Train your own ChatGPT", section 1 "GPT
+    model", architecture features: rotary embeddings for relative positions without learned position
+    embeddings, and QK normalisation for stability; the pages give neither formula). Readings:
+      * QK normalisation: RMS normalisation of each head vector over D without a learnable weight,
+        y = x / sqrt(mean(x^2) + eps);
+      * rotary embedding (RoFormer, Su et al. 2021): each pair (first, second) of y at position p is turned by
+        the angle p * base^(-2i/D), first' = first cos - second sin, second' = first sin + second cos. Pair i
+        is (2i, 2i+1) ("interleaved", the paper's form) or (i, i + D/2) ("half");
+      * positions: row t of sequence b sits at offsets[b] + t (0 for a training batch; the cache length
+        before the new tokens for decode).
+    Rotation keeps the RMS, so the two steps commute.
+
+    x: [B, T, H, D] (q, or k with its own head count). Returns float64 [B, T, H, D].
+    """
+    x = _as_f64(x)
+    B, T, H, D = x.shape
+    y = x / np.sqrt((x * x).mean(axis=-1, keepdims=True) + eps)
+    ang = _rope_angles(B, T, D, base, offsets)[:, :, None, :]              # [B, T, 1, D/2]
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = _pairs(y, pairing)
+    return _unpairs(a * c - b * s, a * s + b * c, pairing)
+
+
+def qk_norm_rope_backward(x, dy, base: float = 10000.0, eps: float = 1e-6, offsets=0,
+                          pairing: str = "interleaved") -> np.ndarray:
+    """Gradient of sum(dy * qk_norm_rope(x)) with respect to x, by the chain rule through the two steps:
+      * rotation: the transpose turns each pair back by the same angle, g = R(-angle) dy;
+      * RMS normalisation y = x r, r = (mean(x^2) + eps)^(-1/2): dx = r (g - y mean(g y)).
+    Returns float64 [B, T, H, D].
+    """
+    x, dy = _as_f64(x), _as_f64(dy)
+    B, T, H, D = x.shape
+    r = 1.0 / np.sqrt((x * x).mean(axis=-1, keepdims=True) + eps)
+    y = x * r
+    ang = _rope_angles(B, T, D, base, offsets)[:, :, None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = _pairs(dy, pairing)
+    g = _unpairs(a * c + b * s, -a * s + b * c, pairing)
+    return r * (g - y * (g * y).mean(axis=-1, keepdims=True))
+
+
 def causal_flops(B: int, H: int, T: int, D: int) -> Tuple[float, float]:
     """FLOP convention of the measurement: forward 2*B*H*T^2*D, backward 2.5x that."""
     f = 2.0 * B * H * T * T * D

@@ -419,6 +419,167 @@ def test_decode_single_query_and_empty_rows():
 
 
 # ---------------------------------------------------------------------------------------------------------
+# QK normalisation + rotary embedding (the prologue before attention).
+
+def _complex_rotation(xn, pos, base, pairing):
+    """The rotary embedding as complex multiplication: the pair (a, b) is a + ib, turned by e^(i p theta_k)."""
+    D = xn.shape[-1]
+    a, b = (xn[..., 0::2], xn[..., 1::2]) if pairing == "interleaved" else (xn[..., :D // 2], xn[..., D // 2:])
+    theta = base ** (-2.0 * np.arange(D // 2) / D)
+    z = (a + 1j * b) * np.exp(1j * pos[..., None, None] * theta)
+    out = np.empty_like(xn)
+    if pairing == "interleaved":
+        out[..., 0::2], out[..., 1::2] = z.real, z.imag
+    else:
+        out[..., :D // 2], out[..., D // 2:] = z.real, z.imag
+    return out
+
+
+def rope_pin_rotation(f, pairing):
+    """RMS 1 per head vector (eps = 0); position 0 is the plain normalisation; the rotation equals the complex
+    product with e^(i p base^(-2i/D)) (numpy's complex exponential), also with per-sequence offsets."""
+    B, T, H, D = 2, 12, 2, 16
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((B, T, H, D)) * 3.0
+    y = f(x, base=100.0, eps=0.0, pairing=pairing)
+    np.testing.assert_allclose(np.sqrt((y * y).mean(axis=-1)), 1.0, rtol=1e-13)
+    xn = x / np.sqrt((x * x).mean(axis=-1, keepdims=True))
+    np.testing.assert_allclose(y[:, 0], xn[:, 0], rtol=0, atol=1e-14)
+    pos = np.broadcast_to(np.arange(T, dtype=np.float64), (B, T))
+    np.testing.assert_allclose(y, _complex_rotation(xn, pos, 100.0, pairing), rtol=0, atol=1e-12)
+    offs = np.array([5, 40])
+    np.testing.assert_allclose(f(x, base=100.0, eps=0.0, offsets=offs, pairing=pairing),
+                               _complex_rotation(xn, offs[:, None] + np.arange(T), 100.0, pairing), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(f(x[:, 5:], base=100.0, eps=0.0, offsets=5, pairing=pairing), y[:, 5:],
+                               rtol=0, atol=1e-12)
+
+
+def rope_pin_relative_and_eps(f, pairing):
+    """q.k after the embedding depends only on the position difference (what rotary embeddings are for); eps
+    enters under the square root: with x = 1 everywhere the output RMS is exactly 1 / sqrt(1 + eps)."""
+    rng = np.random.default_rng(22)
+    T, D = 12, 16
+    qv, kv = rng.standard_normal(D), rng.standard_normal(D)
+    yq = f(np.broadcast_to(qv, (1, T, 1, D)), base=100.0, pairing=pairing)
+    yk = f(np.broadcast_to(kv, (1, T, 1, D)), base=100.0, pairing=pairing)
+    dots = [(yq[0, t, 0] * yk[0, t - 3, 0]).sum() for t in range(3, T)]
+    np.testing.assert_allclose(dots, dots[0], rtol=1e-12)
+    y1 = f(np.ones((1, 4, 1, D)), base=100.0, eps=0.25, pairing=pairing)
+    np.testing.assert_allclose(np.sqrt((y1 * y1).mean(axis=-1)), 1.0 / np.sqrt(1.25), rtol=1e-13)
+
+
+def rope_pin_backward(f, fb, pairing):
+    """Central differences of sum(dy * f(x)) in float64, element by element, with per-sequence offsets; with
+    eps = 0 the gradient is orthogonal to x (the normalisation is scale-invariant)."""
+    rng = np.random.default_rng(8)
+    B, T, H, D = 2, 3, 2, 8
+    x = rng.standard_normal((B, T, H, D))
+    dy = rng.standard_normal((B, T, H, D))
+    kw = dict(base=30.0, eps=1e-3, offsets=np.array([0, 7]), pairing=pairing)
+    dx = fb(x, dy, **kw)
+    num = np.empty_like(x)
+    h = 1e-6
+    for idx in np.ndindex(x.shape):
+        xp, xm = x.copy(), x.copy()
+        xp[idx] += h
+        xm[idx] -= h
+        num[idx] = ((f(xp, **kw) - f(xm, **kw)) * dy).sum() / (2 * h)
+    np.testing.assert_allclose(dx, num, rtol=1e-6, atol=1e-8)
+    dx0 = fb(x, dy, base=30.0, eps=0.0, pairing=pairing)
+    np.testing.assert_allclose((dx0 * x).sum(axis=-1), 0.0, atol=1e-12)
+
+
+def run_rope_pins(f, fb):
+    for pairing in ("interleaved", "half"):
+        rope_pin_rotation(f, pairing)
+        rope_pin_relative_and_eps(f, pairing)
+        rope_pin_backward(f, fb, pairing)
+
+
+def test_qk_norm_rope_pins():
+    run_rope_pins(attn_ref.qk_norm_rope, attn_ref.qk_norm_rope_backward)
+
+
+def test_rope_pairings_differ_and_match_by_permutation():
+    """The two pairings are the same rotation after permuting the dimensions (i, i + D/2) -> (2i, 2i+1)."""
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((1, 9, 3, 16))
+    perm = np.empty(16, dtype=int)
+    perm[0::2], perm[1::2] = np.arange(8), np.arange(8, 16)     # interleaved slot j holds half-layout dim perm[j]
+    yi = attn_ref.qk_norm_rope(x[..., perm], base=50.0, pairing="interleaved")
+    yh = attn_ref.qk_norm_rope(x, base=50.0, pairing="half")
+    np.testing.assert_allclose(yi, yh[..., perm], rtol=0, atol=1e-13)
+    assert np.abs(attn_ref.qk_norm_rope(x, base=50.0, pairing="interleaved") - yh).max() > 0.1
+
+
+def _rope_mutant(kind):
+    """A copy of the prologue's forward and backward with one plausible mistake planted."""
+    def pairs(y, pairing):
+        D = y.shape[-1]
+        return (y[..., 0::2], y[..., 1::2]) if pairing == "interleaved" else (y[..., :D // 2], y[..., D // 2:])
+
+    def unpairs(a, b, pairing):
+        if pairing == "interleaved":
+            out = np.empty(a.shape[:-1] + (2 * a.shape[-1],))
+            out[..., 0::2], out[..., 1::2] = a, b
+            return out
+        return np.concatenate([a, b], axis=-1)
+
+    def angles(x, base, offsets):
+        B, T, _, D = x.shape
+        off = np.broadcast_to(np.asarray(offsets, dtype=np.float64), (B,))
+        pos = off[:, None] + np.arange(T)
+        if kind == "positions_ignore_offset":
+            pos = np.broadcast_to(np.arange(T, dtype=np.float64), (B, T))
+        expo = (-1.0 if kind == "freq_exponent_i_over_d" else -2.0) * np.arange(D // 2) / D
+        return (pos[:, :, None] * base ** expo)[:, :, None, :]
+
+    def rms(x, eps):
+        ms = (x * x).sum(axis=-1, keepdims=True) if kind == "sum_not_mean" else (x * x).mean(axis=-1, keepdims=True)
+        return 1.0 / (np.sqrt(ms) + eps) if kind == "eps_outside_sqrt" else 1.0 / np.sqrt(ms + eps)
+
+    def f(x, base=10000.0, eps=1e-6, offsets=0, pairing="interleaved"):
+        x = np.asarray(x, dtype=np.float64)
+        y = x * rms(x, eps)
+        ang = angles(x, base, offsets)
+        c, s = np.cos(ang), np.sin(ang)
+        if kind == "rotate_backwards":
+            s = -s
+        a, b = pairs(y, pairing)
+        return unpairs(a * c - b * s, a * s + b * c, pairing)
+
+    def fb(x, dy, base=10000.0, eps=1e-6, offsets=0, pairing="interleaved"):
+        x, dy = np.asarray(x, dtype=np.float64), np.asarray(dy, dtype=np.float64)
+        r = rms(x, eps)
+        y = x * r
+        ang = angles(x, base, offsets)
+        c, s = np.cos(ang), np.sin(ang)
+        if kind == "bwd_rotates_forward":
+            s = -s
+        a, b = pairs(dy, pairing)
+        g = unpairs(a * c + b * s, -a * s + b * c, pairing)
+        if kind == "bwd_drops_projection":
+            return r * g
+        return r * (g - y * (g * y).mean(axis=-1, keepdims=True))
+
+    return f, fb
+
+
+ROPE_MUTANTS = ["positions_ignore_offset", "freq_exponent_i_over_d", "sum_not_mean", "eps_outside_sqrt",
+                "rotate_backwards", "bwd_rotates_forward", "bwd_drops_projection"]
+
+
+def test_rope_mutant_control_passes():
+    run_rope_pins(*_rope_mutant("none"))
+
+
+@pytest.mark.parametrize("kind", ROPE_MUTANTS)
+def test_rope_pins_catch_planted_mistake(kind):
+    with pytest.raises(AssertionError):
+        run_rope_pins(*_rope_mutant(kind))
+
+
+# ---------------------------------------------------------------------------------------------------------
 # Mutation test: plant plausible mistakes in a copy of the oracle and require that some pin fails.
 
 def _mutant(kind):
