@@ -37,6 +37,7 @@ METRIC = "causal attention fwd+bwd TFLOP/s (bf16, d20 shape) and % of B200 tenso
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 KERNEL_SOURCES = ["attn_api.cu", "attn_fwd.cuh", "attn_bwd.cuh", "attn_decode.cuh", "attn_common.cuh", "sm100.cuh"]
+PROLOGUE_SOURCES = ["attn_rope.cu"]  # the prologue's kernels and launches are all in this file
 
 
 def parse_args(argv=None):
@@ -44,8 +45,9 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    from workloads import DECODE_WORKLOADS
-    ap.add_argument("--workload", default="d20", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS))
+    from workloads import DECODE_WORKLOADS, PROLOGUE_WORKLOADS
+    ap.add_argument("--workload", default="d20",
+                    choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(PROLOGUE_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
@@ -66,15 +68,15 @@ def load_peaks():
         return dict(FALLBACK_PEAKS)
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(sources=KERNEL_SOURCES) -> str:
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in sources:
         with open(os.path.join(ROOT, "causal_self_attention_bf16_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str, workload: str):
+def recorded_traffic(kernel: str, workload: str, sources=KERNEL_SOURCES):
     """DRAM bytes per launch from a committed ncu summary, if taken on the current kernel sources."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
@@ -83,7 +85,7 @@ def recorded_traffic(kernel: str, workload: str):
     except (OSError, ValueError):
         return None
     ent = d.get(kernel, {}).get(workload)
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(sources):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -576,11 +578,142 @@ def run_decode(args):
     return 0
 
 
+PROLOGUE_METRIC = "QK-norm + RoPE prologue HBM GB/s (fwd+bwd, bf16)"
+
+
+def prologue_bytes(w):
+    """Algorithmic bytes of one prologue step, per kernel: the forward reads q, k and writes them back
+    normalised and rotated (2 row passes); the backward reads q, k and the output gradients and writes the
+    input gradients (3 row passes). A row is D bf16 values."""
+    row_bytes = w.B * w.T * (w.H + w.Hkv) * w.D * 2
+    return 2 * row_bytes, 3 * row_bytes
+
+
+def run_prologue(args):
+    """QK normalisation + rotary embedding, forward and backward kernels: HBM-bound, measured in GB/s of
+    algorithmic bytes against the measured copy bandwidth. The d20 inputs (q, k and their gradients, over
+    600 MB) exceed L2, which the line states."""
+    from workloads import PROLOGUE_WORKLOADS, make_prologue_inputs
+    w = PROLOGUE_WORKLOADS[args.workload]
+    rank, world, _ = dist_env()
+    fwd_b, bwd_b = prologue_bytes(w)
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        from threadpoolctl import threadpool_limits
+
+        from oracle import attn_ref
+        q, k, gq, gk, offs = make_prologue_inputs(w)
+        n, t = min(w.B, 2), min(w.T, 256)
+        kw = dict(base=w.rope_base, eps=w.eps, pairing=w.pairing, offsets=0 if offs is None else offs[:n].numpy())
+        times = []
+        with threadpool_limits(limits=len(os.sched_getaffinity(0))):
+            for it in range(args.warmup + args.steps):
+                t0 = time.perf_counter()
+                for x, g in ((q, gq), (k, gk)):
+                    attn_ref.qk_norm_rope(x[:n, :t], **kw)
+                    attn_ref.qk_norm_rope_backward(x[:n, :t], g[:n, :t], **kw)
+                if it >= args.warmup:
+                    times.append(time.perf_counter() - t0)
+        frac = (n * t) / (w.B * w.T)
+        value = (fwd_b + bwd_b) * frac / (sum(times) / len(times)) / 1e9
+        print(json.dumps({"metric": PROLOGUE_METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+                          "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "impl": "reference",
+                          "dtype": "f64", "data": "synthetic", "config": {"workload": w.name, "recipe": w.recipe},
+                          "cpu_baseline": {"value": value, "unit": "GB/s", "cores": len(os.sched_getaffinity(0)),
+                                           "kind": "oracle",
+                                           "sample": f"{n} sequences x {t} positions of {w.name} per step"}}))
+        return 0
+    import torch
+
+    import causal_self_attention_bf16_b200 as attn
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    q, k, gq, gk, offs = make_prologue_inputs(w, device)
+    qo, ko, dq, dk = (torch.empty_like(t) for t in (q, k, q, k))
+    lib = attn.load_library()
+    sh = torch.cuda.current_stream(device).cuda_stream
+    pairing = attn.ROPE_PAIRINGS[w.pairing]
+    optr = None if offs is None else offs.data_ptr()
+
+    def fwd():
+        st = lib.attn_qk_norm_rope(q.data_ptr(), k.data_ptr(), qo.data_ptr(), ko.data_ptr(), optr, w.B, w.T, w.H,
+                                   w.Hkv, w.D, w.rope_base, w.eps, pairing, sh)
+        if st != 0:
+            raise RuntimeError(f"attn_qk_norm_rope: {attn._STATUS.get(st, st)}")
+
+    def bwd():
+        st = lib.attn_qk_norm_rope_bwd(q.data_ptr(), k.data_ptr(), gq.data_ptr(), gk.data_ptr(), dq.data_ptr(),
+                                       dk.data_ptr(), optr, w.B, w.T, w.H, w.Hkv, w.D, w.rope_base, w.eps, pairing, sh)
+        if st != 0:
+            raise RuntimeError(f"attn_qk_norm_rope_bwd: {attn._STATUS.get(st, st)}")
+
+    for _ in range(max(args.warmup, 3)):
+        fwd()
+        bwd()
+    torch.cuda.synchronize(device)
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    ev = [(mk(), mk(), mk()) for _ in range(args.steps)]
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    sampler = ClockSampler(gpu_id)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    sampler.start()
+    time.sleep(0.1)
+    for e0, e1, e2 in ev:
+        e0.record()
+        fwd()
+        e1.record()
+        bwd()
+        e2.record()
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_f = sum(a.elapsed_time(b) for a, b, _ in ev) / len(ev)
+    ms_b = sum(b.elapsed_time(c) for _, b, c in ev) / len(ev)
+    ms = reduce_max(ms_f + ms_b, world, device)
+    gbs = (fwd_b + bwd_b) / (ms / 1e3) / 1e9
+    bwd_gbs = bwd_b / (ms_b / 1e3) / 1e9
+    hbm = float(load_peaks()["hbm_gbs"])
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return 0
+    print(json.dumps({
+        "metric": PROLOGUE_METRIC, "value": gbs * world, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms, "ms_fwd": ms_f, "ms_bwd": ms_b, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "ours",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "H_kv": w.Hkv, "D": w.D,
+                   "pairing": w.pairing, "recipe": w.recipe, "l2": "inputs larger than L2, no flush",
+                   "parallelism": f"replicas x{world} (no collective on the data path)"},
+        "roofline": {"kernel": "qk_norm_rope_bwd_kernel", "bound": "hbm", "achieved": bwd_gbs, "peak": hbm,
+                     "unit": "GB/s", "frac": bwd_gbs / hbm, "alg_bytes": bwd_b,
+                     "traffic": recorded_traffic("qk_norm_rope_bwd_kernel", w.name, PROLOGUE_SOURCES)},
+        "fwd_roofline": {"kernel": "qk_norm_rope_kernel", "achieved": fwd_b / (ms_f / 1e3) / 1e9,
+                         "frac": fwd_b / (ms_f / 1e3) / 1e9 / hbm, "alg_bytes": fwd_b,
+                         "traffic": recorded_traffic("qk_norm_rope_kernel", w.name, PROLOGUE_SOURCES)},
+        "gpu_launches": 2 * args.steps, "clocks": clocks,
+        "kernel_source_hash": kernel_source_hash(PROLOGUE_SOURCES),
+    }))
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
-    from workloads import DECODE_WORKLOADS
+    from workloads import DECODE_WORKLOADS, PROLOGUE_WORKLOADS
     if args.workload in DECODE_WORKLOADS:
         return run_decode(args)
+    if args.workload in PROLOGUE_WORKLOADS:
+        return run_prologue(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -44,6 +44,9 @@ SIGNATURES = {
     "attn_bwd_ex": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _I, _F, _I, _VP], _I),
     "attn_decode_workspace_bytes": ([_I] * 6, _SZ),
     "attn_decode": ([_VP] * 7 + [_SZ] + [_I] * 6 + [_F, _VP], _I),
+    "attn_qk_norm_rope": ([_VP] * 5 + [_I] * 5 + [_F, _F, _I, _VP], _I),
+    "attn_qk_norm_rope_bwd": ([_VP] * 7 + [_I] * 5 + [_F, _F, _I, _VP], _I),
+    "attn_prologue_last_cuda_error": ([], ctypes.c_char_p),
     "attn_get_device_error": ([ctypes.POINTER(ctypes.c_uint32)], _I),
     "attn_clear_device_error": ([], _I),
     "attn_set_wait_limit_ns": ([_U64], _I),
@@ -86,7 +89,9 @@ def _check(fn: str, status: int):
     if status != ATTN_OK:
         detail = ""
         if status == 4:
-            detail = load_library().attn_last_cuda_error().decode(errors="replace")
+            lib = load_library()
+            text = lib.attn_prologue_last_cuda_error() if "qk_norm_rope" in fn else lib.attn_last_cuda_error()
+            detail = text.decode(errors="replace")
         raise AttnError(fn, status, detail)
 
 
@@ -266,6 +271,85 @@ def attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, c
     return o, lse
 
 
+ROPE_PAIRINGS = {"interleaved": 0, "half": 1}
+
+
+def _rope_args(q: torch.Tensor, k: torch.Tensor, pos_offsets: Optional[torch.Tensor], pairing: str):
+    _check_qkv("q", q)
+    _check_qkv("k", k)
+    B, T, H, D = q.shape
+    if (k.shape[0], k.shape[1], k.shape[3]) != (B, T, D) or k.device != q.device:
+        raise ValueError(f"k has shape {tuple(k.shape)}; expected [{B}, {T}, H_kv, {D}] on q's device")
+    if pairing not in ROPE_PAIRINGS:
+        raise ValueError(f"pairing must be one of {sorted(ROPE_PAIRINGS)}, got {pairing!r}")
+    ptr = None
+    if pos_offsets is not None:
+        if (pos_offsets.dtype != torch.int32 or tuple(pos_offsets.shape) != (B,) or
+                pos_offsets.device != q.device or not pos_offsets.is_contiguous()):
+            raise ValueError("pos_offsets must be a contiguous int32 [B] tensor on q's device")
+        ptr = pos_offsets.data_ptr()
+    return B, T, H, k.shape[2], D, ptr, ROPE_PAIRINGS[pairing]
+
+
+def qk_norm_rope(q: torch.Tensor, k: torch.Tensor, rope_base: float = 10000.0, eps: float = 1e-6,
+                 pos_offsets: Optional[torch.Tensor] = None, pairing: str = "interleaved", inplace: bool = False,
+                 stream: Optional[torch.cuda.Stream] = None):
+    """RMS-normalise each head vector of q [B, T, H, D] and k [B, T, H_kv, D], then rotate its pairs by
+    position (rotary embedding). Row t of sequence b sits at position pos_offsets[b] + t (int32 [B] on the
+    device; None = t). Returns (q_out, k_out), new tensors unless inplace."""
+    lib = load_library()
+    B, T, H, Hkv, D, offs, pr = _rope_args(q, k, pos_offsets, pairing)
+    q_out, k_out = (q, k) if inplace else (torch.empty_like(q), torch.empty_like(k))
+    st = lib.attn_qk_norm_rope(q.data_ptr(), k.data_ptr(), q_out.data_ptr(), k_out.data_ptr(), offs, B, T, H, Hkv,
+                               D, float(rope_base), float(eps), pr, _stream_handle(stream, q.device))
+    _check("attn_qk_norm_rope", st)
+    return q_out, k_out
+
+
+def qk_norm_rope_bwd(q: torch.Tensor, k: torch.Tensor, dq_out: torch.Tensor, dk_out: torch.Tensor,
+                     rope_base: float = 10000.0, eps: float = 1e-6, pos_offsets: Optional[torch.Tensor] = None,
+                     pairing: str = "interleaved", inplace: bool = False, stream: Optional[torch.cuda.Stream] = None):
+    """Gradients of q, k (the prologue's inputs) from the gradients dq_out, dk_out of its outputs. With
+    inplace the results overwrite dq_out, dk_out."""
+    lib = load_library()
+    B, T, H, Hkv, D, offs, pr = _rope_args(q, k, pos_offsets, pairing)
+    _check_qkv("dq_out", dq_out, q.shape)
+    _check_qkv("dk_out", dk_out, k.shape)
+    dq, dk = (dq_out, dk_out) if inplace else (torch.empty_like(q), torch.empty_like(k))
+    st = lib.attn_qk_norm_rope_bwd(q.data_ptr(), k.data_ptr(), dq_out.data_ptr(), dk_out.data_ptr(), dq.data_ptr(),
+                                   dk.data_ptr(), offs, B, T, H, Hkv, D, float(rope_base), float(eps), pr,
+                                   _stream_handle(stream, q.device))
+    _check("attn_qk_norm_rope_bwd", st)
+    return dq, dk
+
+
+class QKNormRopeFunction(torch.autograd.Function):
+    """autograd wrapper of the prologue: forward saves the raw q, k; backward calls qk_norm_rope_bwd."""
+
+    @staticmethod
+    def forward(ctx, q, k, rope_base, eps, pos_offsets, pairing):
+        q_out, k_out = qk_norm_rope(q, k, rope_base, eps, pos_offsets, pairing)
+        ctx.save_for_backward(q, k, pos_offsets)
+        ctx.args = (rope_base, eps, pairing)
+        return q_out, k_out
+
+    @staticmethod
+    def backward(ctx, dq_out, dk_out):
+        q, k, pos_offsets = ctx.saved_tensors
+        rope_base, eps, pairing = ctx.args
+        dq, dk = qk_norm_rope_bwd(q, k, dq_out.contiguous(), dk_out.contiguous(), rope_base, eps, pos_offsets,
+                                  pairing, inplace=True)
+        return dq, dk, None, None, None, None
+
+
+def qk_norm_rope_attention(q, k, v, scale: Optional[float] = None, window: Optional[int] = None,
+                           rope_base: float = 10000.0, eps: float = 1e-6, pairing: str = "interleaved"):
+    """Differentiable prologue + causal attention: QK normalisation and rotary embedding of q and k, then
+    causal_attention. Two launches forward (prologue, attention), the attention backward plus one launch back."""
+    qr, kr = QKNormRopeFunction.apply(q, k, rope_base, eps, None, pairing)
+    return causal_attention(qr, kr, v, scale, window)
+
+
 def get_device_error() -> int:
     """The library's device-side error word (0 = no kernel gave up on a bounded wait). Synchronises."""
     word = ctypes.c_uint32(0)
@@ -313,5 +397,6 @@ def causal_attention(q, k, v, scale: Optional[float] = None, window: Optional[in
 
 
 __all__ = ["attn_fwd", "attn_bwd", "attn_decode", "attn_bwd_workspace_bytes", "causal_attention", "CausalAttentionFunction",
+           "qk_norm_rope", "qk_norm_rope_bwd", "QKNormRopeFunction", "qk_norm_rope_attention",
            "get_device_error", "clear_device_error", "set_wait_limit_ns", "selftest_wait_timeout", "AttnError",
            "load_library", "LIB_PATH", "SIGNATURES"]

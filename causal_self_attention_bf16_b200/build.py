@@ -14,8 +14,8 @@ ROOT = os.path.dirname(PKG_DIR)
 CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libattn.so")
-SOURCES = ["attn_api.cu"]
-DEPENDS = ["attn_api.cu", "attn_fwd.cuh", "attn_bwd.cuh", "attn_decode.cuh", "attn_common.cuh", "sm100.cuh"]
+SOURCES = ["attn_api.cu", "attn_rope.cu"]
+DEPENDS = ["attn_api.cu", "attn_rope.cu", "attn_fwd.cuh", "attn_bwd.cuh", "attn_decode.cuh", "attn_common.cuh", "sm100.cuh"]
 
 
 def nvcc_path() -> str:

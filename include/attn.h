@@ -172,6 +172,42 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
                              float scale, void* stream);
 
 /*
+ * QK normalisation + rotary embedding: the prologue the model applies to q and k before attention
+ * (apidog "Train your own ChatGPT", section 1 "GPT model", architecture features: rotary embeddings for
+ * relative positions without learned position embeddings, QK normalisation for stability). The pages give no
+ * formula; this library's reading, per head vector x of D = 128 dims at time t of sequence b:
+ *   y = x / sqrt(mean(x^2) + eps)                       RMS normalisation, no learnable weight
+ *   (a, b) -> (a cos w - b sin w, a sin w + b cos w)    rotation of each pair (RoFormer, Su et al. 2021)
+ *   w = p * rope_base^(-2i/D),  p = pos_offsets[b] + t  (p = t when pos_offsets is NULL)
+ * Pair i is (2i, 2i+1) for ATTN_ROPE_INTERLEAVED (the paper's form) or (i, i + D/2) for ATTN_ROPE_HALF.
+ *   q      in : bf16 [B, T, H, D];     k     in : bf16 [B, T, H_kv, D]
+ *   q_out out : bf16 [B, T, H, D];     k_out out : bf16 [B, T, H_kv, D]
+ *               q_out may be q itself and k_out may be k itself (in place); no other overlap
+ *   pos_offsets in : device int32 [B] or NULL (decode: the cache length before the new tokens)
+ *   rope_base finite and > 0 (usually 10000); eps finite and >= 0; D = 128 (else ATTN_ERR_UNSUPPORTED)
+ * One kernel launch over the rows of both tensors. On ATTN_ERR_CUDA, attn_prologue_last_cuda_error()
+ * describes the failure.
+ */
+typedef enum { ATTN_ROPE_INTERLEAVED = 0, ATTN_ROPE_HALF = 1 } attn_rope_pairing;
+
+attn_status attn_qk_norm_rope(const void* q, const void* k, void* q_out, void* k_out, const int* pos_offsets, int B,
+                              int T, int H, int H_kv, int D, float rope_base, float eps, int pairing, void* stream);
+
+/*
+ * Backward of attn_qk_norm_rope: from q, k (its inputs) and dq_out, dk_out (the gradients of its outputs,
+ * e.g. attn_bwd's dq, dk), the gradients dq, dk of its inputs. Chain rule, per row, with r = (mean(x^2) +
+ * eps)^(-1/2) and y = x r: g = dy turned back by -w, dx = r (g - y mean(g y)).
+ *   dq may be dq_out itself and dk may be dk_out itself (in place); no other overlap of an output.
+ * Same arguments, layouts and errors as attn_qk_norm_rope otherwise. One kernel launch.
+ */
+attn_status attn_qk_norm_rope_bwd(const void* q, const void* k, const void* dq_out, const void* dk_out, void* dq,
+                                  void* dk, const int* pos_offsets, int B, int T, int H, int H_kv, int D,
+                                  float rope_base, float eps, int pairing, void* stream);
+
+/* Text of the last CUDA error seen by the two prologue calls above on the calling thread ("" if none). */
+const char* attn_prologue_last_cuda_error(void);
+
+/*
  * Device-side error word shared by the kernels of this library on the current device: 0 if no kernel has
  * given up on a bounded wait since the last clear; otherwise (site << 8) | 1. Synchronises the device.
  * Returns ATTN_ERR_TIMEOUT if the word is non-zero, ATTN_OK if it is zero, ATTN_ERR_CUDA on a CUDA error.

@@ -159,6 +159,36 @@ def test_decode_argument_errors(lib):
     assert call(lens=lens + 2) == 3       # lengths must be 4-byte aligned
 
 
+def test_qk_norm_rope_argument_errors(lib):
+    """The prologue checks sizes, base, eps, pairing, alignment and overlaps before any CUDA call; in place
+    (an output equal to its input) is allowed, a partial overlap is not."""
+    B, T, H, Hkv = 2, 100, 4, 2
+    qb, kb = B * T * H * 256, B * T * Hkv * 256
+    q, k, qo, ko, offs, gq, gk = fake_ptrs(7, qb)
+    fwd = lambda **kw: lib.attn_qk_norm_rope(kw.get("q", q), k, kw.get("qo", qo), kw.get("ko", ko),
+                                             kw.get("offs", offs), B, kw.get("T", T), H, kw.get("hkv", Hkv),
+                                             kw.get("D", 128), kw.get("base", 10000.0), kw.get("eps", 1e-6),
+                                             kw.get("pairing", 0), None)
+    assert fwd(q=None) == 1
+    assert fwd(T=0) == 1 and fwd(hkv=0) == 1
+    assert fwd(D=64) == 2
+    assert fwd(base=0.0) == 1 and fwd(base=float("inf")) == 1 and fwd(base=-2.0) == 1
+    assert fwd(eps=-1e-6) == 1 and fwd(eps=float("nan")) == 1
+    assert fwd(pairing=2) == 1 and fwd(pairing=-1) == 1
+    assert fwd(qo=qo + 8) == 3
+    assert fwd(offs=offs + 2) == 3
+    assert fwd(qo=q + 256) == 1           # output overlaps its input without being it
+    assert fwd(qo=k) == 1                 # q's output over k
+    assert fwd(ko=qo + qb - 256) == 1     # the two outputs overlap
+    assert fwd(offs=qo) == 1              # positions inside an output
+    bwd = lambda **kw: lib.attn_qk_norm_rope_bwd(q, k, kw.get("gq", gq), gk, kw.get("dq", qo), kw.get("dk", ko),
+                                                 None, B, T, H, Hkv, 128, 10000.0, 1e-6, kw.get("pairing", 1), None)
+    assert bwd(dq=q) == 1                 # dq over the input q
+    assert bwd(dq=gq + 256) == 1          # partial overlap with its own gradient
+    assert bwd(dq=gk) == 1                # dq over dk_out
+    assert bwd(pairing=5) == 1
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
 def test_no_cpu_fallback_without_gpu(lib):
     """A well-formed call on a machine without an sm_100 GPU fails loudly instead of computing on the CPU."""
@@ -169,6 +199,10 @@ def test_no_cpu_fallback_without_gpu(lib):
     ws = lib.attn_bwd_workspace_bytes(1, 2, 128, 128)
     assert bwd_call(lib, fake_ptrs(10, max(size, ws)), ws) == 4
     assert lib.attn_fwd_gqa(q, k, v, o, lse, 1, 2, 1, 128, 128, 0.088, None) == 4
+    # the prologue: in place is well formed, and still fails loudly
+    assert lib.attn_qk_norm_rope(q, k, q, k, None, 1, 128, 2, 2, 128, 10000.0, 1e-6, 0, None) == 4
+    assert lib.attn_prologue_last_cuda_error().decode() != ""
+    assert lib.attn_qk_norm_rope_bwd(q, k, o, lse, o, lse, None, 1, 128, 2, 2, 128, 10000.0, 1e-6, 1, None) == 4
 
 
 def test_binding_rejects_cpu_tensors(lib):

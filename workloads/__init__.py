@@ -201,3 +201,58 @@ def make_decode_inputs(w: DecodeWorkload, device: Optional[torch.device] = None)
         out = tuple(t.to(device) for t in out)
     return out
 
+
+
+@dataclasses.dataclass(frozen=True)
+class PrologueWorkload:
+    """Raw q [B, T, H, D] and k [B, T, H_kv, D] before QK normalisation and the rotary embedding, plus the
+    gradients of the prologue's outputs for its backward. Entries are N(0,1) times a per-row factor
+    exp(N(0, 0.5^2)), so row norms differ as projections of a residual stream do; with `offsets`, each
+    sequence starts at a position drawn uniformly from [0, max_offset] (decode's new tokens after a cache)."""
+
+    name: str
+    B: int
+    T: int
+    H: int
+    Hkv: int
+    D: int = HEAD_DIM
+    rope_base: float = 10000.0
+    eps: float = 1e-6
+    pairing: str = "interleaved"
+    max_offset: int = 0
+    seed: int = 0
+    recipe: str = ""
+
+
+PROLOGUE_WORKLOADS: Dict[str, PrologueWorkload] = {
+    "rope_tiny": PrologueWorkload("rope_tiny", B=2, T=37, H=5, Hkv=2, max_offset=100000, seed=11,
+                                  recipe="ragged positions (74 < 5 blocks of 16), 7 rows per position, offsets up "
+                                         "to 1e5"),
+    "rope_d20": PrologueWorkload("rope_d20", B=32, T=2048, H=10, Hkv=10, seed=12,
+                                 recipe="d20 training batch: 32 x 2048 tokens, 10 query and 10 key heads"),
+    "rope_d20_gqa": PrologueWorkload("rope_d20_gqa", B=32, T=2048, H=10, Hkv=5, pairing="half", seed=13,
+                                     recipe="rope_d20 with 5 key heads and the half pairing"),
+}
+
+
+def make_prologue_inputs(w: PrologueWorkload, device: Optional[torch.device] = None):
+    """(q, k, dq_out, dk_out, offsets): bf16 tensors and int32 [B] offsets (None when max_offset is 0) from
+    one seeded CPU generator, in the order q, q row factors, k, k row factors, dq_out, dk_out, offsets."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed)
+
+    def rows(heads):
+        x = torch.randn((w.B, w.T, heads, w.D), generator=g, dtype=torch.float32)
+        f = torch.exp(0.5 * torch.randn((w.B, w.T, heads, 1), generator=g, dtype=torch.float32))
+        return (x * f).to(torch.bfloat16)
+
+    q, k = rows(w.H), rows(w.Hkv)
+    dq = torch.randn((w.B, w.T, w.H, w.D), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    dk = torch.randn((w.B, w.T, w.Hkv, w.D), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    offs = None
+    if w.max_offset > 0:
+        offs = torch.randint(0, w.max_offset + 1, (w.B,), generator=g, dtype=torch.int64).to(torch.int32)
+    out = (q, k, dq, dk, offs)
+    if device is not None:
+        out = tuple(None if t is None else t.to(device) for t in out)
+    return out
