@@ -33,6 +33,13 @@ Pins (tests/test_oracle.py): softmax rows sum to one; causality under perturbati
 Q = 0 closed form (prefix mean, LSE = ln(t + 1)); equal keys; shift invariance of the keys; agreement with
 torch's float64 ``scaled_dot_product_attention`` and its autograd; central finite differences; the Delta
 identity; a hand-derived worked example under tests/golden/.
+
+Also here: grouped-query heads and the sliding window (``kv_group``, ``causal_mask``), cached decode
+(``decode_forward``), and the QK-normalisation + rotary-embedding prologue with its backward
+(``qk_norm_rope``, ``qk_norm_rope_backward``; RMS normalisation and the RoFormer rotation, readings stated in
+their docstrings). The prologue is pinned by the complex-exponential form of the rotation, relative-position
+invariance, a closed-form eps case, the agreement of the two pairings under a permutation, and central finite
+differences of the backward.
 """
 from __future__ import annotations
 
