@@ -505,7 +505,8 @@ def run_decode(args):
                           "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "impl": "reference",
                           "dtype": "f64", "data": "synthetic", "config": {"workload": w.name, "recipe": w.recipe},
                           "cpu_baseline": {"value": value, "unit": "GB/s", "cores": len(os.sched_getaffinity(0)),
-                                           "kind": "oracle", "sample": f"{n} sequences of {w.name} per step"}}))
+                                           "kind": "oracle", "sample": f"{n} sequences of {w.name} per step"},
+                          "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
         return 0
     import torch
 
@@ -622,7 +623,8 @@ def run_prologue(args):
                           "dtype": "f64", "data": "synthetic", "config": {"workload": w.name, "recipe": w.recipe},
                           "cpu_baseline": {"value": value, "unit": "GB/s", "cores": len(os.sched_getaffinity(0)),
                                            "kind": "oracle",
-                                           "sample": f"{n} sequences x {t} positions of {w.name} per step"}}))
+                                           "sample": f"{n} sequences x {t} positions of {w.name} per step"},
+                          "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
         return 0
     import torch
 

@@ -72,3 +72,25 @@ def test_decode_reference_arm_line(monkeypatch, capsys):
     line = json.loads(capsys.readouterr().out.strip())
     assert line["metric"] == bench.DECODE_METRIC and line["unit"] == "GB/s" and line["value"] > 0
     assert line["impl"] == "reference" and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_prologue_reference_arm_line(monkeypatch, capsys):
+    """The prologue workloads report GB/s of algorithmic bytes (forward + backward); the reference arm times the
+    oracle's prologue and its backward on a bounded sample and prints one line."""
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    import json
+    assert bench.main(["--impl", "reference", "--workload", "rope_tiny", "--steps", "1", "--warmup", "0"]) == 0
+    line = json.loads(capsys.readouterr().out.strip())
+    assert line["metric"] == bench.PROLOGUE_METRIC and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["impl"] == "reference" and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+
+
+@pytest.mark.parametrize("workload", ["decode_tiny", "rope_tiny"])
+def test_extra_reference_arms_run_on_rank0_only(monkeypatch, capsys, workload):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.main(["--impl", "reference", "--workload", workload, "--gpus", "2", "--steps", "1",
+                       "--warmup", "0"]) == 0
+    assert capsys.readouterr().out == ""

@@ -104,3 +104,23 @@ def test_bench_decode_bytes_count_only_valid_cache_rows():
     assert bench.decode_bytes(w, lens) == kv + 2 * w.B * w.Tq * w.H * w.D * 2 + w.B * w.H * w.Tq * 4
     f, b = bench.flops(WORKLOADS["d20_sw"])
     assert f == WORKLOADS["d20_sw"].fwd_flops and b == WORKLOADS["d20_sw"].bwd_flops
+
+
+def test_prologue_inputs_and_bytes():
+    """Seeded, shaped prologue inputs (offsets only when asked for), and the byte count of one step: the forward
+    reads and writes every row of q and k, the backward reads two and writes one."""
+    import bench
+    from workloads import PROLOGUE_WORKLOADS, make_prologue_inputs
+    w = PROLOGUE_WORKLOADS["rope_tiny"]
+    a, b = make_prologue_inputs(w), make_prologue_inputs(w)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    q, k, dq, dk, offs = a
+    assert tuple(q.shape) == tuple(dq.shape) == (2, 37, 5, 128) and tuple(k.shape) == tuple(dk.shape) == (2, 37, 2, 128)
+    assert q.dtype == k.dtype == torch.bfloat16 and offs.dtype == torch.int32 and tuple(offs.shape) == (2,)
+    assert int(offs.min()) >= 0 and int(offs.max()) <= w.max_offset
+    norms = q.float().pow(2).mean(-1).sqrt().flatten()
+    assert norms.max() / norms.min() > 2.0  # rows of different size, so the normalisation matters
+    assert make_prologue_inputs(PROLOGUE_WORKLOADS["rope_d20"].__class__("x", B=1, T=3, H=1, Hkv=1))[4] is None
+    row = 32 * 2048 * 20 * 128 * 2
+    assert bench.prologue_bytes(PROLOGUE_WORKLOADS["rope_d20"]) == (2 * row, 3 * row)
