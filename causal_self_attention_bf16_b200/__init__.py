@@ -337,8 +337,9 @@ class QKNormRopeFunction(torch.autograd.Function):
     def backward(ctx, dq_out, dk_out):
         q, k, pos_offsets = ctx.saved_tensors
         rope_base, eps, pairing = ctx.args
+        # out of place: autograd does not promise that the incoming gradient tensors are this function's to change
         dq, dk = qk_norm_rope_bwd(q, k, dq_out.contiguous(), dk_out.contiguous(), rope_base, eps, pos_offsets,
-                                  pairing, inplace=True)
+                                  pairing)
         return dq, dk, None, None, None, None
 
 
