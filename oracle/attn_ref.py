@@ -270,9 +270,3 @@ def qk_norm_rope_backward(x, dy, base: float = 10000.0, eps: float = 1e-6, offse
     a, b = _pairs(dy, pairing)
     g = _unpairs(a * c + b * s, -a * s + b * c, pairing)
     return r * (g - y * (g * y).mean(axis=-1, keepdims=True))
-
-
-def causal_flops(B: int, H: int, T: int, D: int) -> Tuple[float, float]:
-    """FLOP convention of the measurement: forward 2*B*H*T^2*D, backward 2.5x that."""
-    f = 2.0 * B * H * T * T * D
-    return f, 2.5 * f
