@@ -362,20 +362,20 @@ def test_window_gradients_by_finite_differences():
 # ---------------------------------------------------------------------------------------------------------
 # Decode against a key/value cache: query i of Tq sits at position L - Tq + i.
 
-def test_decode_equals_training_forward_when_the_cache_is_the_sequence():
+def decode_pin_whole_sequence(f):
     """Tq = L: the new queries are the whole sequence, so decode is the causal training forward."""
     B, T, H, Hkv, D = 2, 21, 4, 2, 8
     rng = np.random.default_rng(11)
     q = rng.standard_normal((B, T, H, D))
     k, v = rng.standard_normal((B, T, Hkv, D)), rng.standard_normal((B, T, Hkv, D))
     s = 0.3
-    O, LSE = attn_ref.decode_forward(q, k, v, [T, T], s)
+    O, LSE = f(q, k, v, [T, T], s)
     O2, LSE2 = attn_ref.attention_forward(q, k, v, s)
     np.testing.assert_allclose(O, O2, rtol=1e-13, atol=1e-13)
     np.testing.assert_allclose(LSE, LSE2, rtol=1e-13, atol=1e-13)
 
 
-def test_decode_matches_torch_per_sequence():
+def decode_pin_torch(f):
     """Ragged cache lengths, spare cache rows filled with garbage (never read), Tq = 3: each sequence equals
     torch's float64 SDPA on its valid cache with the end-aligned causal mask (and enable_gqa)."""
     B, Tq, H, Hkv, Tk, D = 3, 3, 6, 2, 40, 16
@@ -384,7 +384,7 @@ def test_decode_matches_torch_per_sequence():
     kc, vc = rng.standard_normal((B, Tk, Hkv, D)), rng.standard_normal((B, Tk, Hkv, D))
     lens = [40, 17, 3]
     s = 1 / math.sqrt(D)
-    O, LSE = attn_ref.decode_forward(q, kc, vc, lens, s)
+    O, LSE = f(q, kc, vc, lens, s)
     for b, L in enumerate(lens):
         tq = torch.tensor(q[b:b + 1]).transpose(1, 2)
         tk, tv = (torch.tensor(x[b:b + 1, :L]).transpose(1, 2) for x in (kc, vc))
@@ -396,26 +396,80 @@ def test_decode_matches_torch_per_sequence():
     kc2, vc2 = kc.copy(), vc.copy()
     kc2[1, 17:] = 1e6
     vc2[2, 3:] = np.nan
-    O2, _ = attn_ref.decode_forward(q, kc2, vc2, lens, s)
+    O2, _ = f(q, kc2, vc2, lens, s)
     np.testing.assert_array_equal(O, O2)
 
 
-def test_decode_single_query_and_empty_rows():
-    """Tq = 1 sees the whole valid cache (softmax over all L keys); a query before the first key (L < Tq)
-    returns 0 with LSE -inf; L = 1 returns the one value."""
+def decode_pin_closed_forms(f):
+    """Tq = 1 sees the whole valid cache (softmax over all L keys, LSE its log-sum-exp); a query before the
+    first key (L < Tq) returns 0 with LSE -inf; L = 1 returns the one value."""
     B, Tk, H, D = 2, 9, 1, 4
     rng = np.random.default_rng(13)
     q = rng.standard_normal((B, 2, H, D))
     kc, vc = rng.standard_normal((B, Tk, H, D)), rng.standard_normal((B, Tk, H, D))
     s = 0.5
-    O, LSE = attn_ref.decode_forward(q[:, :1], kc, vc, [9, 1], s)
+    O, LSE = f(q[:, :1], kc, vc, [9, 1], s)
     sc = s * kc[0, :, 0] @ q[0, 0, 0]
     p = np.exp(sc - sc.max()) / np.exp(sc - sc.max()).sum()
     np.testing.assert_allclose(O[0, 0, 0], p @ vc[0, :, 0], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(LSE[0, 0, 0], np.log(np.exp(sc).sum()), rtol=1e-13)
     np.testing.assert_allclose(O[1, 0, 0], vc[1, 0, 0], rtol=0, atol=1e-15)
-    O2, LSE2 = attn_ref.decode_forward(q, kc, vc, [9, 1], s)   # Tq = 2, second sequence has one key
+    O2, LSE2 = f(q, kc, vc, [9, 1], s)   # Tq = 2, second sequence has one key
     assert np.all(O2[1, 0, 0] == 0) and LSE2[1, 0, 0] == -np.inf
     np.testing.assert_allclose(O2[1, 1, 0], vc[1, 0, 0], rtol=0, atol=1e-15)
+
+
+DECODE_PINS = [decode_pin_whole_sequence, decode_pin_torch, decode_pin_closed_forms]
+
+
+@pytest.mark.parametrize("pin", DECODE_PINS)
+def test_decode_pins(pin):
+    pin(attn_ref.decode_forward)
+
+
+def _decode_mutant(kind):
+    """A copy of the decode oracle with one plausible mistake planted."""
+    def f(q, k_cache, v_cache, cache_seqlens, scale):
+        q, kc, vc = (np.asarray(x, dtype=np.float64) for x in (q, k_cache, v_cache))
+        B, Tq, H, D = q.shape
+        Hkv = kc.shape[2]
+        G = H // Hkv
+        O, LSE = np.zeros((B, Tq, H, D)), np.full((B, H, Tq), -np.inf)
+        for b in range(B):
+            L = kc.shape[1] if kind == "lengths_ignored" else int(cache_seqlens[b])
+            for h in range(H):
+                hk = h % Hkv if kind == "kv_head_modulo" else h // G
+                k, v = kc[b, :L, hk], vc[b, :L, hk]
+                for i in range(Tq):
+                    last = {"top_left_mask": i, "last_key_off_by_one": L - Tq + i - 1}.get(kind, L - Tq + i)
+                    if last < 0:
+                        continue
+                    sc = scale * (k[: last + 1] @ q[b, i, h])
+                    m = sc.max()
+                    e = np.exp(sc - m)
+                    O[b, i, h] = (e @ v[: last + 1]) / e.sum()
+                    LSE[b, h, i] = m + (np.log2(e.sum()) if kind == "lse_log2" else np.log(e.sum()))
+        return O, LSE
+    return f
+
+
+DECODE_MUTANTS = ["lengths_ignored", "kv_head_modulo", "top_left_mask", "last_key_off_by_one", "lse_log2"]
+
+
+def test_decode_mutant_control_passes():
+    for pin in DECODE_PINS:
+        pin(_decode_mutant("none"))
+
+
+@pytest.mark.parametrize("kind", DECODE_MUTANTS)
+def test_decode_pins_catch_planted_mistake(kind):
+    caught = []
+    for pin in DECODE_PINS:
+        try:
+            pin(_decode_mutant(kind))
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no decode pin caught the planted mistake {kind!r}"
 
 
 # ---------------------------------------------------------------------------------------------------------
