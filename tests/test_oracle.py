@@ -341,6 +341,20 @@ def test_window_closed_forms():
         attn_ref.attention_forward(q, k, v, s, window=-2)
 
 
+@pytest.mark.parametrize("kind", ["left_edge_excluded", "one_key_wider", "window_ignored"])
+def test_window_pin_catches_a_wrong_band(monkeypatch, kind):
+    """Planted mistakes in the band the oracle builds: the torch band-mask pin must fail on each."""
+    def mutated(T, window=None):
+        i, j = np.arange(T)[:, None], np.arange(T)[None, :]
+        if window is None or kind == "window_ignored":
+            return j <= i
+        lo = {"left_edge_excluded": i - window + 1, "one_key_wider": i - window - 1}[kind]
+        return (j <= i) & (j >= lo)
+    monkeypatch.setattr(attn_ref, "causal_mask", mutated)
+    with pytest.raises(AssertionError):
+        test_window_matches_torch_with_band_mask(37, 5, 2, 2)
+
+
 def test_window_gradients_by_finite_differences():
     T, D, window = 9, 4, 3
     q, k, v, do = rand_qkvdo(T, D, 8)
