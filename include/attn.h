@@ -184,7 +184,8 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
  *   q_out out : bf16 [B, T, H, D];     k_out out : bf16 [B, T, H_kv, D]
  *               q_out may be q itself and k_out may be k itself (in place); no other overlap
  *   pos_offsets in : device int32 [B] or NULL (decode: the cache length before the new tokens)
- *   rope_base finite and > 0 (usually 10000); eps finite and >= 0; D = 128 (else ATTN_ERR_UNSUPPORTED)
+ *   rope_base finite and > 0 (usually 10000); eps finite and >= 0; D = 128 (else ATTN_ERR_UNSUPPORTED).
+ *   With eps = 0 an all-zero row has no direction and its output is NaN (the formula's 0/0); eps > 0 maps it to 0.
  * One kernel launch over the rows of both tensors. On ATTN_ERR_CUDA, attn_prologue_last_cuda_error()
  * describes the failure.
  */
