@@ -20,7 +20,8 @@
  *   - The caller owns and allocates every buffer, including the backward workspace. The library never
  *     allocates, frees or synchronises; all work is enqueued asynchronously on `stream` (a cudaStream_t;
  *     NULL = legacy default stream) on the current CUDA device.
- *   - Outputs must not overlap inputs or each other.
+ *   - Outputs must not overlap inputs or each other (the QK-norm + RoPE prologue calls alone also accept an
+ *     output that is exactly its own input, for in-place use).
  *   - Argument errors are detected on the host before anything is launched and leave outputs untouched.
  *   - There is no CPU fallback: on a machine without an sm_100 device the calls return ATTN_ERR_CUDA.
  */
