@@ -16,7 +16,9 @@
  *
  * Conventions for every entry point
  *   - Tensors are device pointers. q, k, v, o, dO, dq, dk, dv: bf16, [B, T, H, D] contiguous (D fastest).
- *     lse: fp32 [B, H, T] contiguous. Every pointer must be 16-byte aligned (TMA requirement).
+ *     lse: fp32 [B, H, T] contiguous. Every pointer must be 16-byte aligned (TMA requirement), except the
+ *     int32 / fp32 vectors of attn_decode (lse, cache_seqlens) and attn_qk_norm_rope[_bwd] (pos_offsets),
+ *     which need 4 bytes.
  *   - The caller owns and allocates every buffer, including the backward workspace. The library never
  *     allocates, frees or synchronises; all work is enqueued asynchronously on `stream` (a cudaStream_t;
  *     NULL = legacy default stream) on the current CUDA device.
