@@ -150,23 +150,32 @@ class ClockSampler:
             self.proc.kill()
         self.file.flush()
         self.file.seek(0)
-        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.count(",") >= 8]
+        text = self.file.read()
         self.file.close()
         os.unlink(self.file.name)
-        sm, smax, power, reasons = [], [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            try:
-                sm.append(float(r[1]))
-                smax.append(float(r[2]))
-                power.append(float(r[3]))
-            except ValueError:
-                continue
-            for name, val in zip(names, r[5:9]):
-                if val.strip().lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "power_w_max": max(power) if power else None, "reasons": sorted(reasons), "samples": len(sm)}
+        return summarize_clocks(text)
+
+
+def summarize_clocks(text: str):
+    """Median SM clock, the maximum clock and power, and every throttle reason seen Active, from nvidia-smi's
+    `--query-gpu=ClockSampler.FIELDS --format=csv,noheader,nounits` lines. Rows that do not parse (a line cut
+    off when the sampler is stopped, "[N/A]" values) are skipped."""
+    rows = [r.split(",") for r in text.strip().splitlines() if r.count(",") >= 8]
+    sm, smax, power, reasons = [], [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for r in rows:
+        try:
+            vals = float(r[1]), float(r[2]), float(r[3])
+        except ValueError:
+            continue
+        sm.append(vals[0])
+        smax.append(vals[1])
+        power.append(vals[2])
+        for name, val in zip(names, r[5:9]):
+            if val.strip().lower() == "active":
+                reasons.add(name)
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+            "power_w_max": max(power) if power else None, "reasons": sorted(reasons), "samples": len(sm)}
 
 
 # ------------------------------------------------------------------------------------------------ CPU oracle

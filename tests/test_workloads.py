@@ -124,3 +124,21 @@ def test_prologue_inputs_and_bytes():
     assert make_prologue_inputs(PROLOGUE_WORKLOADS["rope_d20"].__class__("x", B=1, T=3, H=1, Hkv=1))[4] is None
     row = 32 * 2048 * 20 * 128 * 2
     assert bench.prologue_bytes(PROLOGUE_WORKLOADS["rope_d20"]) == (2 * row, 3 * row)
+
+
+def test_clock_summary_parses_nvidia_smi_rows():
+    """The clocks object of the bench line: median SM clock under load, max clock and power, and throttle
+    reasons seen Active in any sample; unparsable rows are skipped."""
+    import bench
+    text = "\n".join([
+        "0, 1965, 1965, 700.5, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1897, 1965, 998.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1830, 1965, 1001.2, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, [N/A], 1965, 10.0, 0x0, Not Active, Active, Not Active, Not Active",   # skipped entirely
+        "0, 1965, 19",                                                               # cut off
+    ])
+    c = bench.summarize_clocks(text)
+    assert c["samples"] == 3 and c["sm_mhz"] == 1897.0 and c["sm_max_mhz"] == 1965.0
+    assert c["power_w_max"] == 1001.2 and c["reasons"] == ["sw_power_cap"]
+    empty = bench.summarize_clocks("")
+    assert empty["samples"] == 0 and empty["sm_mhz"] is None and empty["reasons"] == []
