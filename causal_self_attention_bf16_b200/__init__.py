@@ -100,15 +100,32 @@ def _stream_handle(stream: Optional[torch.cuda.Stream], device: torch.device) ->
     return s.cuda_stream
 
 
-def _check_qkv(name: str, t: torch.Tensor, shape=None):
+def _require_cuda(name: str, t) -> None:
     if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
         raise ValueError(f"{name} must be a CUDA tensor")
+
+
+def _check_qkv(name: str, t: torch.Tensor, shape=None, device: Optional[torch.device] = None):
+    """A bf16, contiguous, 4-D tensor (of `shape`, on `device`, where given)."""
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a tensor")
     if t.dtype != torch.bfloat16:
         raise ValueError(f"{name} must be bfloat16, got {t.dtype}")
     if t.dim() != 4 or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous [B, T, H, D] tensor")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}; every tensor of one call must be on {device}")
+
+
+def _check_f32(name: str, t: torch.Tensor, shape, device: torch.device):
+    """A contiguous fp32 tensor of `shape` on `device` (lse)."""
+    if (not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or tuple(t.shape) != tuple(shape)
+            or not t.is_contiguous()):
+        raise ValueError(f"{name} must be a contiguous fp32 {list(shape)} tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}; every tensor of one call must be on {device}")
 
 
 def default_scale(D: int) -> float:
@@ -117,12 +134,53 @@ def default_scale(D: int) -> float:
 
 def _kv_shape(q: torch.Tensor, k: torch.Tensor):
     """[B, T, H_kv, D] of k and v: H_kv = H, or fewer key/value heads dividing H (grouped-query attention)."""
-    _check_qkv("k", k)
+    _check_qkv("k", k, device=q.device)
     B, T, H, D = q.shape
     Hkv = k.shape[2]
     if (k.shape[0], k.shape[1], k.shape[3]) != (B, T, D) or Hkv < 1 or H % Hkv:
         raise ValueError(f"k has shape {tuple(k.shape)}; expected [{B}, {T}, H_kv, {D}] with H_kv dividing {H}")
     return (B, T, Hkv, D)
+
+
+def _fwd_tensors(q, k, v, o, lse):
+    """Check the forward's tensors (all on q's device) and allocate the outputs not given. Returns
+    (o, lse, H_kv)."""
+    _check_qkv("q", q)
+    B, T, H, D = q.shape
+    kv = _kv_shape(q, k)
+    _check_qkv("v", v, kv, q.device)
+    o = torch.empty_like(q) if o is None else o
+    _check_qkv("o", o, q.shape, q.device)
+    if lse is None:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    _check_f32("lse", lse, (B, H, T), q.device)
+    return o, lse, kv[2]
+
+
+def _bwd_tensors(q, k, v, o, lse, dO, dq, dk, dv, same_heads: bool = False):
+    """Check the backward's tensors (all on q's device; with same_heads, k and v must have q's shape) and
+    allocate the gradients not given. The kernels read and write whole tensors of these shapes, so every
+    caller-supplied buffer is checked here: a smaller one would be written past its end. Returns
+    (dq, dk, dv, H_kv)."""
+    _check_qkv("q", q)
+    B, T, H, D = q.shape
+    dev = q.device
+    if same_heads:
+        _check_qkv("k", k, q.shape, dev)
+        kv = tuple(q.shape)
+    else:
+        kv = _kv_shape(q, k)
+    _check_qkv("v", v, kv, dev)
+    for name, t in (("o", o), ("dO", dO)):
+        _check_qkv(name, t, q.shape, dev)
+    _check_f32("lse", lse, (B, H, T), dev)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_qkv("dq", dq, q.shape, dev)
+    _check_qkv("dk", dk, kv, dev)
+    _check_qkv("dv", dv, kv, dev)
+    return dq, dk, dv, kv[2]
 
 
 def _window_arg(window: Optional[int]) -> int:
@@ -141,31 +199,25 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[
     CUDA device. window: None, or a sliding window (query i sees keys i - window .. i). Returns
     (o [B, T, H, D], lse [B, H, T])."""
     lib = load_library()
-    _check_qkv("q", q)
+    _require_cuda("q", q)
+    o, lse, Hkv = _fwd_tensors(q, k, v, o, lse)
     B, T, H, D = q.shape
-    kv = _kv_shape(q, k)
-    _check_qkv("v", v, kv)
-    if o is None:
-        o = torch.empty_like(q)
-    _check_qkv("o", o, q.shape)
-    if lse is None:
-        lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, T) or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous fp32 [B, H, T] tensor")
     scale = default_scale(D) if scale is None else float(scale)
     win = _window_arg(window)
-    if win >= 0:
-        st = lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, kv[2],
-                             T, D, scale, win, _stream_handle(stream, q.device))
-        _check("attn_fwd_ex", st)
-    elif kv[2] == H:
-        st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, T, D, scale,
-                          _stream_handle(stream, q.device))
-        _check("attn_fwd", st)
-    else:
-        st = lib.attn_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, kv[2],
-                              T, D, scale, _stream_handle(stream, q.device))
-        _check("attn_fwd_gqa", st)
+    with torch.cuda.device(q.device):
+        sh = _stream_handle(stream, q.device)
+        if win >= 0:
+            st = lib.attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, Hkv,
+                                 T, D, scale, win, sh)
+            _check("attn_fwd_ex", st)
+        elif Hkv == H:
+            st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, T, D,
+                              scale, sh)
+            _check("attn_fwd", st)
+        else:
+            st = lib.attn_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, Hkv,
+                                  T, D, scale, sh)
+            _check("attn_fwd_gqa", st)
     return o, lse
 
 
@@ -182,36 +234,29 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     D]); with grouped-query
     attention dk, dv are the gradients of the shared heads (summed over each group's query heads)."""
     lib = load_library()
-    _check_qkv("q", q)
+    _require_cuda("q", q)
+    dq, dk, dv, Hkv = _bwd_tensors(q, k, v, o, lse, dO, dq, dk, dv)
     B, T, H, D = q.shape
-    kv = _kv_shape(q, k)
-    _check_qkv("v", v, kv)
-    for name, t in (("o", o), ("dO", dO)):
-        _check_qkv(name, t, q.shape)
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, T) or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous fp32 [B, H, T] tensor")
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
-    _check_qkv("dq", dq, q.shape)
-    _check_qkv("dk", dk, kv)
-    _check_qkv("dv", dv, kv)
     need = attn_bwd_workspace_bytes(B, H, T, D)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    elif workspace.device != q.device:
+        raise ValueError(f"workspace is on {workspace.device}; every tensor of one call must be on {q.device}")
     scale = default_scale(D) if scale is None else float(scale)
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dO.data_ptr(), dq.data_ptr(),
             dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size())
     win = _window_arg(window)
-    if win >= 0:
-        st = lib.attn_bwd_ex(*ptrs, B, H, kv[2], T, D, scale, win, _stream_handle(stream, q.device))
-        _check("attn_bwd_ex", st)
-    elif kv[2] == H:
-        st = lib.attn_bwd(*ptrs, B, H, T, D, scale, _stream_handle(stream, q.device))
-        _check("attn_bwd", st)
-    else:
-        st = lib.attn_bwd_gqa(*ptrs, B, H, kv[2], T, D, scale, _stream_handle(stream, q.device))
-        _check("attn_bwd_gqa", st)
+    with torch.cuda.device(q.device):
+        sh = _stream_handle(stream, q.device)
+        if win >= 0:
+            st = lib.attn_bwd_ex(*ptrs, B, H, Hkv, T, D, scale, win, sh)
+            _check("attn_bwd_ex", st)
+        elif Hkv == H:
+            st = lib.attn_bwd(*ptrs, B, H, T, D, scale, sh)
+            _check("attn_bwd", st)
+        else:
+            st = lib.attn_bwd_gqa(*ptrs, B, H, Hkv, T, D, scale, sh)
+            _check("attn_bwd_gqa", st)
     return dq, dk, dv
 
 
@@ -222,17 +267,14 @@ def attn_bwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch
     """Backward using the library's built-in scratch array instead of a caller workspace (for callers that
     cannot allocate device memory; sizes up to B*H*roundup(T,128) <= 64512). Returns (dq, dk, dv)."""
     lib = load_library()
-    _check_qkv("q", q)
+    _require_cuda("q", q)
+    dq, dk, dv, _ = _bwd_tensors(q, k, v, o, lse, dO, dq, dk, dv, same_heads=True)
     B, T, H, D = q.shape
-    for name, t in (("k", k), ("v", v), ("o", o), ("dO", dO)):
-        _check_qkv(name, t, q.shape)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
     scale = default_scale(D) if scale is None else float(scale)
-    st = lib.attn_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                              dO.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, T, D, scale,
-                              _stream_handle(stream, q.device))
+    with torch.cuda.device(q.device):
+        st = lib.attn_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                  dO.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, T, D, scale,
+                                  _stream_handle(stream, q.device))
     _check("attn_bwd_noalloc", st)
     return dq, dk, dv
 
@@ -245,28 +287,34 @@ def attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, c
     valid keys of each sequence (new tokens included). Query i sees keys 0 .. L - Tq + i. Returns
     (o [B, Tq, H, D], lse [B, H, Tq])."""
     lib = load_library()
+    _require_cuda("q", q)
     _check_qkv("q", q)
-    _check_qkv("k_cache", k_cache)
+    dev = q.device
+    _check_qkv("k_cache", k_cache, device=dev)
     B, Tq, H, D = q.shape
     Tk, Hkv = k_cache.shape[1], k_cache.shape[2]
     if k_cache.shape[0] != B or k_cache.shape[3] != D:
         raise ValueError(f"k_cache has shape {tuple(k_cache.shape)}; expected [{B}, Tk, H_kv, {D}]")
-    _check_qkv("v_cache", v_cache, k_cache.shape)
-    if (cache_seqlens.dtype != torch.int32 or tuple(cache_seqlens.shape) != (B,) or
-            cache_seqlens.device != q.device or not cache_seqlens.is_contiguous()):
+    _check_qkv("v_cache", v_cache, k_cache.shape, dev)
+    if (not isinstance(cache_seqlens, torch.Tensor) or cache_seqlens.dtype != torch.int32 or
+            tuple(cache_seqlens.shape) != (B,) or cache_seqlens.device != dev or not cache_seqlens.is_contiguous()):
         raise ValueError("cache_seqlens must be a contiguous int32 [B] tensor on q's device")
     o = torch.empty_like(q) if o is None else o
-    _check_qkv("o", o, q.shape)
+    _check_qkv("o", o, q.shape, dev)
     if lse is None:
-        lse = torch.empty((B, H, Tq), dtype=torch.float32, device=q.device)
+        lse = torch.empty((B, H, Tq), dtype=torch.float32, device=dev)
+    _check_f32("lse", lse, (B, H, Tq), dev)
     need = int(lib.attn_decode_workspace_bytes(B, H, Hkv, Tq, Tk, D))
     if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    elif workspace.device != dev:
+        raise ValueError(f"workspace is on {workspace.device}; every tensor of one call must be on {dev}")
     scale = default_scale(D) if scale is None else float(scale)
-    st = lib.attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cache_seqlens.data_ptr(),
-                         o.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
-                         workspace.numel() * workspace.element_size(), B, H, Hkv, Tq, Tk, D, scale,
-                         _stream_handle(stream, q.device))
+    with torch.cuda.device(dev):
+        st = lib.attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cache_seqlens.data_ptr(),
+                             o.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), B, H, Hkv, Tq, Tk, D, scale,
+                             _stream_handle(stream, dev))
     _check("attn_decode", st)
     return o, lse
 
@@ -275,6 +323,7 @@ ROPE_PAIRINGS = {"interleaved": 0, "half": 1}
 
 
 def _rope_args(q: torch.Tensor, k: torch.Tensor, pos_offsets: Optional[torch.Tensor], pairing: str):
+    _require_cuda("q", q)
     _check_qkv("q", q)
     _check_qkv("k", k)
     B, T, H, D = q.shape
@@ -300,8 +349,9 @@ def qk_norm_rope(q: torch.Tensor, k: torch.Tensor, rope_base: float = 10000.0, e
     lib = load_library()
     B, T, H, Hkv, D, offs, pr = _rope_args(q, k, pos_offsets, pairing)
     q_out, k_out = (q, k) if inplace else (torch.empty_like(q), torch.empty_like(k))
-    st = lib.attn_qk_norm_rope(q.data_ptr(), k.data_ptr(), q_out.data_ptr(), k_out.data_ptr(), offs, B, T, H, Hkv,
-                               D, float(rope_base), float(eps), pr, _stream_handle(stream, q.device))
+    with torch.cuda.device(q.device):
+        st = lib.attn_qk_norm_rope(q.data_ptr(), k.data_ptr(), q_out.data_ptr(), k_out.data_ptr(), offs, B, T, H,
+                                   Hkv, D, float(rope_base), float(eps), pr, _stream_handle(stream, q.device))
     _check("attn_qk_norm_rope", st)
     return q_out, k_out
 
@@ -313,12 +363,13 @@ def qk_norm_rope_bwd(q: torch.Tensor, k: torch.Tensor, dq_out: torch.Tensor, dk_
     inplace the results overwrite dq_out, dk_out."""
     lib = load_library()
     B, T, H, Hkv, D, offs, pr = _rope_args(q, k, pos_offsets, pairing)
-    _check_qkv("dq_out", dq_out, q.shape)
-    _check_qkv("dk_out", dk_out, k.shape)
+    _check_qkv("dq_out", dq_out, q.shape, q.device)
+    _check_qkv("dk_out", dk_out, k.shape, q.device)
     dq, dk = (dq_out, dk_out) if inplace else (torch.empty_like(q), torch.empty_like(k))
-    st = lib.attn_qk_norm_rope_bwd(q.data_ptr(), k.data_ptr(), dq_out.data_ptr(), dk_out.data_ptr(), dq.data_ptr(),
-                                   dk.data_ptr(), offs, B, T, H, Hkv, D, float(rope_base), float(eps), pr,
-                                   _stream_handle(stream, q.device))
+    with torch.cuda.device(q.device):
+        st = lib.attn_qk_norm_rope_bwd(q.data_ptr(), k.data_ptr(), dq_out.data_ptr(), dk_out.data_ptr(),
+                                       dq.data_ptr(), dk.data_ptr(), offs, B, T, H, Hkv, D, float(rope_base),
+                                       float(eps), pr, _stream_handle(stream, q.device))
     _check("attn_qk_norm_rope_bwd", st)
     return dq, dk
 

@@ -165,7 +165,9 @@ attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
  *     enough for B * H * roundup(T, 128) <= 64512; larger sizes return ATTN_ERR_WORKSPACE and launch nothing.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  *   - The first call on each device looks the array's device address up (cudaGetSymbolAddress, with that
- *     device current); make that first call before any stream capture.
+ *     device current); make that first call before any stream capture. The address is kept for the life of
+ *     the process: after cudaDeviceReset on that device it is stale, so do not call this entry point there
+ *     again in the same process.
  *   - All calls share the one array, which keeps the last call's contents; each call rewrites everything it
  *     reads from it (the dQ accumulator is zeroed first). Calls that overlap in time on the GPU (different
  *     streams, or different host threads on one device) race on the array and give wrong results.

@@ -218,3 +218,44 @@ def test_binding_signatures_match_header_argument_counts():
         assert m, name
         params = [p for p in m.group(1).split(",") if p.strip() and p.strip() != "void"]
         assert len(params) == len(argtypes), f"{name}: header has {len(params)} params, binding {len(argtypes)}"
+
+
+def test_binding_checks_every_backward_buffer():
+    """The backward wrappers (attn_bwd and attn_bwd_noalloc share one check) reject an lse of the wrong dtype,
+    shape or layout and a gradient buffer of the wrong shape: the kernels read and write whole tensors, so a
+    smaller buffer would be written past its end."""
+    B, T, H, D = 1, 16, 2, 128
+    q = torch.zeros(B, T, H, D, dtype=torch.bfloat16)
+    lse = torch.zeros(B, H, T, dtype=torch.float32)
+    dq, dk, dv, hkv = attn._bwd_tensors(q, q, q, q, lse, q, None, None, None, same_heads=True)
+    assert dq.shape == q.shape and hkv == H
+    bad_lse = [lse.to(torch.bfloat16), torch.zeros(B, H, T - 1), torch.zeros(B, T, H).transpose(1, 2)]
+    for bad in bad_lse:
+        with pytest.raises(ValueError):
+            attn._bwd_tensors(q, q, q, q, bad, q, None, None, None, same_heads=True)
+        with pytest.raises(ValueError):
+            attn._fwd_tensors(q, q, q, None, bad)
+    small = torch.zeros(B, T - 1, H, D, dtype=torch.bfloat16)
+    for pos in range(3):
+        grads = [None, None, None]
+        grads[pos] = small
+        with pytest.raises(ValueError):
+            attn._bwd_tensors(q, q, q, q, lse, q, *grads, same_heads=True)
+    # same_heads (the allocation-free form has no key/value head count): fewer key/value heads are rejected
+    kv = torch.zeros(B, T, 1, D, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        attn._bwd_tensors(q, kv, kv, q, lse, q, None, None, None, same_heads=True)
+    assert attn._bwd_tensors(q, kv, kv, q, lse, q, None, None, None)[3] == 1
+
+
+def test_binding_rejects_tensors_on_different_devices():
+    B, T, H, D = 1, 16, 2, 128
+    q = torch.zeros(B, T, H, D, dtype=torch.bfloat16)
+    other = torch.zeros(B, T, H, D, dtype=torch.bfloat16, device="meta")
+    lse = torch.zeros(B, H, T, dtype=torch.float32)
+    with pytest.raises(ValueError, match="one call"):
+        attn._bwd_tensors(q, other, q, q, lse, q, None, None, None)
+    with pytest.raises(ValueError, match="one call"):
+        attn._bwd_tensors(q, q, q, q, lse.to("meta"), q, None, None, None)
+    with pytest.raises(ValueError, match="one call"):
+        attn._fwd_tensors(q, q, other, None, None)
