@@ -293,16 +293,16 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint64_t dk_mnmaj = sdesc_sw128(smem_u32(smem + kBwdSmemK), 16384, 1024);  // K^T as MN-major A
     bool ok = mbar_wait_warp(&bars.kv_full, 0, abort, p.timeout_ns, &g_device_error, kSiteBwdMmaKV);
     tc_fence_after();
-    // A(i): S^T and dP^T of query tile i into buffer i%2, once its Q/dO tile has landed and the buffer is free
-    // (dQ^T of tile i-2 read out, and its dV/dK MMAs, which read P^T/dS^T from the buffer, complete).
+    // A(i): dP^T and S^T of query tile i into buffer i%2, once its Q/dO tile has landed. dP^T goes first: it
+    // overwrites the buffer's last 64 columns, free once the softmax group has read dQ^T of tile i-2 out of
+    // them; S^T overwrites the first 64, where P^T and dS^T of tile i-2 stay until the dV and dK MMAs of
+    // B(i-2) have read them, so that wait comes second and overlaps dP^T's execution.
     auto issue_a = [&](int i) -> bool {
       const int s = i % kBwdStages, rb = i & 1;
       if (!mbar_wait_warp(&bars.q_full[s], (i / kBwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdMmaQ))
         return false;
-      if (i >= 2 && (!mbar_wait_warp(&bars.dq_empty[rb], ((i - 2) >> 1) & 1, abort, p.timeout_ns, &g_device_error,
-                                     kSiteBwdMmaDqEmpty) ||
-                     !mbar_wait_warp(&bars.b_done[rb], ((i - 2) >> 1) & 1, abort, p.timeout_ns, &g_device_error,
-                                     kSiteBwdMmaDqEmpty)))
+      if (i >= 2 && !mbar_wait_warp(&bars.dq_empty[rb], ((i - 2) >> 1) & 1, abort, p.timeout_ns, &g_device_error,
+                                    kSiteBwdMmaDqEmpty))
         return false;
       if (leader) ATTN_TRACE_EVENT(12, i);
       tc_fence_after();
@@ -313,13 +313,17 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t ka = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;  // 128-row boxes, in 16-byte units
         const uint32_t kb = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;   // 64-row boxes
-        if (leader) mma_ss(r, dk_kmaj + ka, dq0 + kb, id_s, kk > 0);
+        if (leader) mma_ss(r + 64, dv_kmaj + ka, ddo0 + kb, id_s, kk > 0);
       }
+      if (i >= 2 && !mbar_wait_warp(&bars.b_done[rb], ((i - 2) >> 1) & 1, abort, p.timeout_ns, &g_device_error,
+                                    kSiteBwdMmaDqEmpty))
+        return false;
+      tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t ka = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
         const uint32_t kb = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
-        if (leader) mma_ss(r + 64, dv_kmaj + ka, ddo0 + kb, id_s, kk > 0);
+        if (leader) mma_ss(r, dk_kmaj + ka, dq0 + kb, id_s, kk > 0);
       }
       if (leader) {
         mma_commit(&bars.s_full[rb]);
@@ -355,12 +359,12 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       }
       return true;
     };
-    // Pairs: A(i), A(i+1), B(i), B(i+1). The two softmax groups work on tiles i and i+1 at the same time,
-    // and the dQ^T read-out of a pair overlaps the next pair's first MMAs.
-    for (int i = 0; ok && i < ns; i += 2) {
-      ok = issue_a(i) && (i + 1 >= ns || issue_a(i + 1));
-      ok = ok && issue_b(i) && (i + 1 >= ns || issue_b(i + 1));
-    }
+    // Order A(0), A(1), B(0), A(2), B(1), ..., A(n-1), B(n-2), B(n-1): while the softmax group of tile i works
+    // (from the end of A(i) until B(i) can start), the tensor core has B(i-1) and A(i+1) to do, a whole step
+    // of MMAs; the groups' tiles alternate, so their softmax phases hardly overlap.
+    ok = ok && issue_a(0);
+    for (int i = 1; ok && i < ns; ++i) ok = issue_a(i) && issue_b(i - 1);
+    ok = ok && issue_b(ns - 1);
     if (leader) {
       mma_commit(&bars.acc_done);
       mma_commit(&bars.drain);

@@ -337,6 +337,126 @@ ATTN_DEVICE_INLINE void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
 }
 
 // ---------------------------------------------------------------------------------------------------------
+// CTA pairs (a cluster of two CTAs on the two SMs of a TPC): tcgen05 with cta_group::2 lets one thread of the
+// even CTA issue MMAs of M = 256 whose A operand and accumulator are split by rows between the two CTAs'
+// tensor memories and whose B operand is split by columns between the two CTAs' shared memories, so each SM
+// stages and reads only half of B.
+
+ATTN_DEVICE_INLINE uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Every thread of both CTAs; orders earlier shared-memory writes and barrier inits cluster-wide.
+ATTN_DEVICE_INLINE void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Shared::cluster address of the variable at the same offset in the shared memory of CTA `rank` of the cluster.
+ATTN_DEVICE_INLINE uint32_t mapa_shared(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+
+// Arrive on an mbarrier of either CTA of the cluster (release at cluster scope, so the arriving thread's earlier
+// writes, and after a tcgen05.fence::before_thread_sync its tensor-memory accesses, are ordered before it).
+ATTN_DEVICE_INLINE void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// One arrival for the whole warp on a barrier of CTA `rank` (see mbar_arrive_warp).
+ATTN_DEVICE_INLINE void mbar_arrive_warp_cluster(uint64_t* bar, uint32_t rank) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(mapa_shared(bar, rank));
+}
+
+ATTN_DEVICE_INLINE bool mbar_try_wait_cluster(uint32_t bar_addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait for a barrier that threads of the other CTA arrive on (acquire at cluster scope). On a timeout it
+// also raises the other CTA's abort flag (`peer_abort`, a shared::cluster address), so the pair stops together.
+ATTN_DEVICE_INLINE bool mbar_wait_pair(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t peer_abort,
+                                       uint64_t limit_ns, uint32_t* err_word, uint32_t site) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait_cluster(a, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_cluster(a, parity)) return true;
+    if ((i & 63u) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > limit_ns) {
+        *abort = 1;
+        asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(peer_abort), "r"(1) : "memory");
+        atomicOr(err_word, DEV_ERR_TIMEOUT | (site << 8));
+        return false;
+      }
+    }
+  }
+}
+
+ATTN_DEVICE_INLINE bool mbar_wait_pair_warp(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t peer_abort,
+                                            uint64_t limit_ns, uint32_t* err_word, uint32_t site) {
+  const bool ok = mbar_wait_pair(bar, parity, abort, peer_abort, limit_ns, err_word, site);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// TMA tile load into this CTA's shared memory whose completion (complete_tx) is counted on an mbarrier of
+// either CTA of the pair (`bar_cluster`, a shared::cluster address). No multicast.
+ATTN_DEVICE_INLINE void tma_load_4d_pair(void* dst, const void* tmap, uint32_t bar_cluster, int c0, int c1, int c2,
+                                         int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+// Tensor memory of a pair: executed by the same warp of both CTAs; both get the same column base.
+ATTN_DEVICE_INLINE void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+ATTN_DEVICE_INLINE void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+ATTN_DEVICE_INLINE void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem], M = 256 over the pair (issued by one thread of the even CTA).
+ATTN_DEVICE_INLINE void mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                    uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+// Arrive once on the barrier at `bar`'s offset in each CTA of `cta_mask` when every tcgen05 operation issued so
+// far by this thread has completed.
+ATTN_DEVICE_INLINE void mma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(cta_mask)
+      : "memory");
+}
+
+// ---------------------------------------------------------------------------------------------------------
 // Small numeric helpers
 
 ATTN_DEVICE_INLINE float ex2(float x) {

@@ -1,8 +1,8 @@
 """A discrete-event model of the dK/dV backward kernel's barrier protocol, checked on the CPU.
 
 attn_bwd_dkdv_kernel's roles talk only through mbarriers: the TMA producer (K and V once, then query tiles of
-Q, dO, LSE and Delta through a 3-slot ring), the MMA warp (per pair of query tiles A(i), A(i+1), B(i), B(i+1):
-A writes S^T and dP^T into tensor-memory buffer i % 2, B computes dQ^T, then dV and dK), and two softmax groups
+Q, dO, LSE and Delta through a 3-slot ring), the MMA warp (in the order A(0), A(1), B(0), A(2), B(1), ...,
+B(n-1): A writes dP^T, then S^T into tensor-memory buffer i % 2, B computes dQ^T, then dV and dK), and two softmax groups
 that take the tiles in turn (group g owns the tiles i = g mod 2 and buffer g). Each group hands the 32 KB dQ
 staging buffer to the other in tile order through one barrier. Barrier counts follow the kernel: the
 softmax-side barriers count warps, so a group of four warps is one actor arriving 4. MMAs, commits and copies
@@ -76,8 +76,8 @@ def mma(m):
         s, rb = i % STAGES, i & 1
         yield m.wait(f"q_full{s}", i // STAGES)
         if i >= 2:
-            yield m.wait(f"dq_empty{rb}", (i - 2) >> 1)
-            yield m.wait(f"b_done{rb}", (i - 2) >> 1)
+            yield m.wait(f"dq_empty{rb}", (i - 2) >> 1)  # dP^T overwrites the dQ^T columns
+            yield m.wait(f"b_done{rb}", (i - 2) >> 1)    # S^T overwrites P^T, dS^T
         m.b[f"s_full{rb}"].arrive()
 
     def issue_b(i):
@@ -87,13 +87,11 @@ def mma(m):
         m.b[f"b_done{rb}"].arrive()
         m.b[f"q_empty{s}"].arrive()
 
-    for i in range(0, m.ns, 2):
+    yield from issue_a(0)
+    for i in range(1, m.ns):
         yield from issue_a(i)
-        if i + 1 < m.ns:
-            yield from issue_a(i + 1)
-        yield from issue_b(i)
-        if i + 1 < m.ns:
-            yield from issue_b(i + 1)
+        yield from issue_b(i - 1)
+    yield from issue_b(m.ns - 1)
     m.b["acc_done"].arrive()
     m.b["drain"].arrive()
     yield m.wait("drain", 0)
