@@ -95,7 +95,8 @@ attn_status check_kv_heads(int H, int Hkv) {
 }
 
 // Set the dynamic shared-memory opt-in of both big kernels once per device.
-int g_sm_count[64] = {};  // multiprocessors per device, set by prepare_device
+int g_sm_count[64] = {};       // multiprocessors per device, set by prepare_device
+int g_fwd_clusters[64] = {};   // CTA pairs of the forward kernel that fit on the device at once
 
 attn_status prepare_device(int* dev_out) {
   static std::mutex mu;
@@ -128,6 +129,20 @@ attn_status prepare_device(int* dev_out) {
   if ((e = cudaFuncSetAttribute(attn::attn_bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 attn::kBwdSmemAlloc)) != cudaSuccess)
     return cuda_fail(e, "cudaFuncSetAttribute(attn_bwd_dkdv_kernel)");
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * 74);
+    cfg.blockDim = dim3(attn::kFwdThreads);
+    cfg.dynamicSmemBytes = attn::kFwdSmemAlloc;
+    int n = 0;
+    if ((e = cudaOccupancyMaxActiveClusters(&n, attn::attn_fwd_kernel, &cfg)) != cudaSuccess)
+      return cuda_fail(e, "cudaOccupancyMaxActiveClusters(attn_fwd_kernel)");
+    if (n < 1) {
+      std::snprintf(g_cuda_error, sizeof(g_cuda_error), "device %d cannot co-schedule a pair of forward CTAs", dev);
+      return ATTN_ERR_CUDA;
+    }
+    if (dev >= 0 && dev < 64) g_fwd_clusters[dev] = n;
+  }
   if (dev >= 0 && dev < 64) done[dev] = true;
   return ATTN_OK;
 }
@@ -221,7 +236,7 @@ attn_status fwd_launch(const void* q, const void* k, const void* v, void* o, flo
   if ((st = prepare_device(&dev)) != ATTN_OK) return st;
   CUtensorMap mq, mk, mv, mo;
   if ((st = make_map(&mq, q, B, H, T, attn::kTile)) != ATTN_OK) return st;
-  if ((st = make_map(&mk, k, B, Hkv, T, attn::kTile)) != ATTN_OK) return st;
+  if ((st = make_map(&mk, k, B, Hkv, T, attn::kFwdKRows)) != ATTN_OK) return st;
   if ((st = make_map(&mv, v, B, Hkv, T, attn::kTile)) != ATTN_OK) return st;
   if ((st = make_map(&mo, o, B, H, T, attn::kTile)) != ATTN_OK) return st;
 
@@ -234,10 +249,11 @@ attn_status fwd_launch(const void* q, const void* k, const void* v, void* o, flo
   p.T = T;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = g_wait_limit_ns;
-  // Persistent grid: one CTA per SM (fewer when there are fewer work items).
-  const long long n_items = static_cast<long long>((T + attn::kTile - 1) / attn::kTile) * B * H;
-  const int sms = (dev >= 0 && dev < 64 && g_sm_count[dev] > 0) ? g_sm_count[dev] : 148;
-  const dim3 grid(static_cast<unsigned>(n_items < sms ? n_items : sms));
+  // Persistent grid of CTA pairs: as many pairs as fit at once (one per TPC), fewer when there are fewer work
+  // items (pairs of query tiles).
+  const long long n_items = static_cast<long long>((T + 2 * attn::kTile - 1) / (2 * attn::kTile)) * B * H;
+  const int pairs = (dev >= 0 && dev < 64 && g_fwd_clusters[dev] > 0) ? g_fwd_clusters[dev] : 74;
+  const dim3 grid(2u * static_cast<unsigned>(n_items < pairs ? n_items : pairs));
   attn::attn_fwd_kernel<<<grid, attn::kFwdThreads, attn::kFwdSmemAlloc, static_cast<cudaStream_t>(stream)>>>(
       mq, mk, mv, mo, p);
   cudaError_t e = cudaGetLastError();

@@ -360,10 +360,12 @@ ATTN_DEVICE_INLINE uint32_t mapa_shared(const void* p, uint32_t rank) {
   return r;
 }
 
-// Arrive on an mbarrier of either CTA of the cluster (release at cluster scope, so the arriving thread's earlier
-// writes, and after a tcgen05.fence::before_thread_sync its tensor-memory accesses, are ordered before it).
+// Arrive on an mbarrier of either CTA of the cluster. The default (CTA-scope release) semantics, as for a local
+// arrival: what the pair hands over this way is tensor memory, ordered by tcgen05.wait and the tcgen05 fences
+// around the barrier, and shared memory that only the tensor cores read. (A cluster-scope release waits for
+// all of the thread's earlier writes to become visible cluster-wide: ~1-2k cycles on a hot path.)
 ATTN_DEVICE_INLINE void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // One arrival for the whole warp on a barrier of CTA `rank` (see mbar_arrive_warp).
@@ -372,27 +374,15 @@ ATTN_DEVICE_INLINE void mbar_arrive_warp_cluster(uint64_t* bar, uint32_t rank) {
   if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(mapa_shared(bar, rank));
 }
 
-ATTN_DEVICE_INLINE bool mbar_try_wait_cluster(uint32_t bar_addr, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred P;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 P, [%1], %2;\n\t"
-      "selp.b32 %0, 1, 0, P;\n\t}"
-      : "=r"(ok)
-      : "r"(bar_addr), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// mbar_wait for a barrier that threads of the other CTA arrive on (acquire at cluster scope). On a timeout it
-// also raises the other CTA's abort flag (`peer_abort`, a shared::cluster address), so the pair stops together.
+// mbar_wait for a barrier of a CTA pair. On a timeout it also raises the other CTA's abort flag (`peer_abort`,
+// a shared::cluster address), so the pair stops together.
 ATTN_DEVICE_INLINE bool mbar_wait_pair(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t peer_abort,
                                        uint64_t limit_ns, uint32_t* err_word, uint32_t site) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait_cluster(a, parity)) return true;
+  if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait_cluster(a, parity)) return true;
+    if (mbar_try_wait(a, parity)) return true;
     if ((i & 63u) == 0) {
       if (*abort) return false;
       if (global_timer_ns() - t0 > limit_ns) {

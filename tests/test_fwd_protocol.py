@@ -1,10 +1,11 @@
 """A discrete-event model of the persistent forward kernel's barrier protocol, checked on the CPU.
 
-attn_fwd_kernel's roles talk only through mbarriers (and, between its two softmax groups, three named barriers
-per work item). This model replays each role's waits and arrivals in the kernel's order -- the K and V
-producers with the one Q buffer, the MMA warp, the two softmax groups with their epilogue, the output-store
-warp -- with barrier counts as in the kernel (softmax-side barriers count warps: a group of four warps is one
-actor arriving 4). Loads and MMAs complete at once (timing does not matter for these properties). Over random
+attn_fwd_kernel runs as CTA pairs whose roles talk only through mbarriers (and, between the two softmax groups
+of a CTA, three named barriers per work item). This model replays each role's waits and arrivals in the
+kernel's order -- in each CTA the K and V producers with the one Q buffer, the two softmax groups with their
+epilogue and the output-store warp; in the even CTA the MMA warp -- with barrier counts as in the kernel
+(softmax-side barriers count warps: a group of four warps is one actor arriving 4; the pair barriers of the even
+CTA count the arrivals of both CTAs; a multicast commit arrives once in each CTA). Loads and MMAs complete at once (timing does not matter for these properties). Over random
 work-item mixes and random interleavings it checks that
 
   * every role runs to the end (no deadlock: a role only waits for something another role will still do), and
@@ -18,7 +19,7 @@ import random
 
 import pytest
 
-STAGES = 3  # K and V ring depth
+STAGES = 4  # K and V ring depth
 
 
 class Barrier:
@@ -33,18 +34,29 @@ class Barrier:
 
 
 class Model:
+    """Barriers of both CTAs of a pair. Local and multicast-completed barriers exist once per CTA (suffix r);
+    the pair barriers live in the even CTA. A K or V ring slot's pair barrier completes after the even CTA's
+    arming arrival and the two halves' copy completions (modelled as three arrivals, in any order)."""
+
     def __init__(self, items):
         self.items = items
-        self.b = {}
-        for name, count in [("q_full", 1), ("q_tmem", 8), ("q_free", 1), ("o_staged", 8), ("o_final", 1)]:
-            self.b[name] = Barrier(count)
+        self.b = {"q_ready": Barrier(16)}
+        for r in range(2):
+            for name, count in [("q_full", 1), ("q_tmem", 8), ("q_free", 1), ("o_staged", 8), ("o_final", 1)]:
+                self.b[f"{name}{r}"] = Barrier(count)
+            for s in range(STAGES):
+                for name in ("k_empty", "v_empty"):
+                    self.b[f"{name}{s}_{r}"] = Barrier(1)
+            for s in range(2):
+                for name, count in (("s_full", 1), ("xchg", 4), ("pv_done", 1)):
+                    self.b[f"{name}{s}_{r}"] = Barrier(count)
         for s in range(STAGES):
-            for name in ("k_full", "k_empty", "v_full", "v_empty"):
-                self.b[f"{name}{s}"] = Barrier(1)
+            for name in ("k_full", "v_full"):
+                self.b[f"{name}{s}"] = Barrier(3)
         for s in range(2):
-            for name, count in (("s_full", 1), ("s_free", 4), ("p_full", 4), ("xchg", 4), ("pv_done", 1)):
-                self.b[f"{name}{s}"] = Barrier(count)
-        self.named = {"A": [0, 0], "B": [0, 0], "C": [0, 0]}  # passes of each named barrier, per group
+            for name in ("s_free", "p_full"):
+                self.b[f"{name}{s}"] = Barrier(8)
+        self.named = {(w, r): [0, 0] for w in "ABC" for r in range(2)}  # passes of each named barrier, per group
         self.violations = []
 
     def wait(self, name, n):
@@ -57,53 +69,72 @@ class Model:
             return bar.done > n
         return ready
 
-    def named_barrier(self, which, g, k):
-        self.named[which][g] += 1
-        return lambda: min(self.named[which]) > k
+    def both(self, name):
+        """A multicast commit: one arrival on the barrier at the same offset in each CTA."""
+        for r in range(2):
+            self.b[f"{name}_{r}" if name[-1].isdigit() else f"{name}{r}"].arrive()
+
+    def named_barrier(self, which, r, g, k):
+        self.named[(which, r)][g] += 1
+        return lambda: min(self.named[(which, r)]) > k
 
 
-def producer(m, is_k):
+def producer(m, r, is_k):
     t0 = 0
     for k, n in enumerate(m.items):
-        if is_k:  # one Q buffer, shared with the output staging of item k-2
+        if is_k:  # one Q buffer per CTA, shared with the output staging of item k-2
             if k == 1:
-                yield m.wait("q_tmem", 0)
+                yield m.wait(f"q_tmem{r}", 0)
             if k >= 2:
-                yield m.wait("q_free", k - 2)
-            m.b["q_full"].arrive()
+                yield m.wait(f"q_free{r}", k - 2)
+            m.b[f"q_full{r}"].arrive()
         for j in range(n):
             t = t0 + j
             s = t % STAGES
             if t >= STAGES:
-                yield m.wait(("k_empty" if is_k else "v_empty") + str(s), (t - STAGES) // STAGES)
-            m.b[("k_full" if is_k else "v_full") + str(s)].arrive()
+                yield m.wait(("k_empty" if is_k else "v_empty") + f"{s}_{r}", (t - STAGES) // STAGES)
+            full = m.b[("k_full" if is_k else "v_full") + str(s)]
+            if r == 0:
+                full.arrive()  # arm the pair barrier with both halves' bytes
+            full.arrive()      # this CTA's half landed
         t0 += n
 
 
-def mma(m, order="per_item"):
+def mma(m, order="dynamic"):
+    def ready(name, n):
+        bar = m.b[name]
+        if bar.done > n + 1:
+            m.violations.append((name, n, bar.done))
+        return bar.done > n
+
+    def s_ready(t):
+        return (t < 2 or ready(f"s_free{t & 1}", (t - 2) // 2)) and ready(f"k_full{t % STAGES}", t // STAGES)
+
+    def pv_ready(t):
+        return ready(f"p_full{t & 1}", t // 2) and ready(f"v_full{t % STAGES}", t // STAGES)
+
     def issue_s(t):
-        if t >= 2:
-            yield m.wait(f"s_free{t & 1}", (t - 2) // 2)
-        yield m.wait(f"k_full{t % STAGES}", t // STAGES)
-        m.b[f"s_full{t & 1}"].arrive()
-        m.b[f"k_empty{t % STAGES}"].arrive()
+        m.both(f"s_full{t & 1}")
+        m.both(f"k_empty{t % STAGES}")
 
     def issue_pv(t):
-        yield m.wait(f"p_full{t & 1}", t // 2)
-        yield m.wait(f"v_full{t % STAGES}", t // STAGES)
-        m.b[f"pv_done{t & 1}"].arrive()
-        m.b[f"v_empty{t % STAGES}"].arrive()
+        m.both(f"pv_done{t & 1}")
+        m.both(f"v_empty{t % STAGES}")
 
-    if order == "per_item":  # the kernel: per item S(0), S(1), S(2), PV(0), ..., PV(n-1), then o_final
+    if order == "dynamic":  # the kernel: per item, whichever of S(js), PV(jp) is ready (S first), then o_final
         t0 = 0
         for k, n in enumerate(m.items):
-            yield m.wait("q_tmem", k)
-            for j in range(n + 2):
-                if j < n:
-                    yield from issue_s(t0 + j)
-                if j >= 2:
-                    yield from issue_pv(t0 + j - 2)
-            m.b["o_final"].arrive()
+            yield m.wait("q_ready", k)
+            js = jp = 0
+            while jp < n:
+                yield lambda: (js < n and s_ready(t0 + js)) or (jp < js and pv_ready(t0 + jp))
+                if js < n and s_ready(t0 + js):
+                    issue_s(t0 + js)
+                    js += 1
+                else:
+                    issue_pv(t0 + jp)
+                    jp += 1
+            m.both("o_final")
             t0 += n
     else:  # negative control: one stream over all items, PVs two tiles behind, no flush at item starts
         starts = [sum(m.items[:k]) for k in range(len(m.items))]
@@ -112,65 +143,71 @@ def mma(m, order="per_item"):
         tp = 0
         for ts in range(total):
             if ts in starts:
-                yield m.wait("q_tmem", starts.index(ts))
-            yield from issue_s(ts)
+                yield m.wait("q_ready", starts.index(ts))
+            yield lambda: s_ready(ts)
+            issue_s(ts)
             if ts + 1 - tp >= 3:
-                yield from issue_pv(tp)
+                yield lambda: pv_ready(tp)
+                issue_pv(tp)
                 if tp in ends:
-                    m.b["o_final"].arrive()
+                    m.both("o_final")
                 tp += 1
         while tp < total:
-            yield from issue_pv(tp)
+            yield lambda: pv_ready(tp)
+            issue_pv(tp)
             if tp in ends:
-                m.b["o_final"].arrive()
+                m.both("o_final")
             tp += 1
 
 
-def softmax_group(m, g):
+def softmax_group(m, r, g):
     def copy_q(k):
-        yield m.wait("q_full", k)
-        m.b["q_tmem"].arrive(4)
+        yield m.wait(f"q_full{r}", k)
+        m.b[f"q_tmem{r}"].arrive(4)
+        m.b["q_ready"].arrive(4)
 
     yield from copy_q(0)
     t0 = 0
     for k, n in enumerate(m.items):
         have_next = k + 1 < len(m.items)
         t = t0 + ((g - t0) & 1)
-        while t < t0 + n:  # the group's tiles of the item
+        while t < t0 + n:  # the group's tiles of the item (a tile above the diagonal takes the same steps)
             j = t - t0
-            yield m.wait(f"s_full{g}", t // 2)
+            yield m.wait(f"s_full{g}_{r}", t // 2)
             m.b[f"s_free{g}"].arrive(4)
             if j > 0:
-                yield m.wait(f"xchg{g ^ 1}", (t - 1) // 2)
-            m.b[f"xchg{g}"].arrive(4)
+                yield m.wait(f"xchg{g ^ 1}_{r}", (t - 1) // 2)
+            m.b[f"xchg{g}_{r}"].arrive(4)
             if t > 0:
-                yield m.wait(f"pv_done{(t - 1) & 1}", (t - 1) // 2)
+                yield m.wait(f"pv_done{(t - 1) & 1}_{r}", (t - 1) // 2)
             m.b[f"p_full{g}"].arrive(4)
             t += 2
-        yield m.named_barrier("A", g, k)
-        yield m.named_barrier("B", g, k)
-        yield m.wait("o_final", k)
+        yield m.named_barrier("A", r, g, k)
+        yield m.named_barrier("B", r, g, k)
+        yield m.wait(f"o_final{r}", k)
         if have_next:
             yield from copy_q(k + 1)
         if k > 0:
-            yield m.wait("q_free", k - 1)
-        m.b["o_staged"].arrive(4)
-        yield m.named_barrier("C", g, k)
+            yield m.wait(f"q_free{r}", k - 1)
+        m.b[f"o_staged{r}"].arrive(4)
+        yield m.named_barrier("C", r, g, k)
         t0 += n
 
 
-def store_warp(m):
+def store_warp(m, r):
     for k in range(len(m.items)):
-        yield m.wait("o_staged", k)
-        m.b["q_free"].arrive()
+        yield m.wait(f"o_staged{r}", k)
+        m.b[f"q_free{r}"].arrive()
 
 
-def run(items, seed, order="per_item"):
-    """Random interleaving of the roles; returns (finished, violations)."""
+def run(items, seed, order="dynamic"):
+    """Random interleaving of the roles of both CTAs; returns (finished, violations)."""
     m = Model(items)
     rng = random.Random(seed)
-    roles = {"k": producer(m, True), "v": producer(m, False), "mma": mma(m, order),
-             "g0": softmax_group(m, 0), "g1": softmax_group(m, 1), "store": store_warp(m)}
+    roles = {"mma": mma(m, order)}
+    for r in range(2):
+        roles.update({f"k{r}": producer(m, r, True), f"v{r}": producer(m, r, False), f"g0_{r}": softmax_group(m, r, 0),
+                      f"g1_{r}": softmax_group(m, r, 1), f"store{r}": store_warp(m, r)})
     waiting = {name: None for name in roles}
     alive = set(roles)
     while alive:
