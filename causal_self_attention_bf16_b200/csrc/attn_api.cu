@@ -355,8 +355,10 @@ attn_status bwd_launch(unsigned stages, const void* q, const void* k, const void
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_bwd_prep_kernel launch");
   }
   if (stages & 2u) {
-    const unsigned n_kt = static_cast<unsigned>((T + attn::kBwdKTile - 1) / attn::kBwdKTile);
-    attn::attn_bwd_dkdv_kernel<<<dim3(n_kt * static_cast<unsigned>(B * Hkv)), attn::kBwdThreads,
+    // Persistent grid: one CTA per SM (fewer when there are fewer work items, key tiles x key/value heads).
+    const long long n_items = static_cast<long long>((T + attn::kBwdKTile - 1) / attn::kBwdKTile) * B * Hkv;
+    const int sms = (dev >= 0 && dev < 64 && g_sm_count[dev] > 0) ? g_sm_count[dev] : 148;
+    attn::attn_bwd_dkdv_kernel<<<dim3(static_cast<unsigned>(n_items < sms ? n_items : sms)), attn::kBwdThreads,
                                  attn::kBwdSmemAlloc, s>>>(mq, mk, mv, mdo, mdk, mdv, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_bwd_dkdv_kernel launch");
   }

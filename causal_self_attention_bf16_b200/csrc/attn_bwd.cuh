@@ -36,7 +36,9 @@ namespace attn {
 constexpr int kBwdQTile = 64;       // queries per inner tile
 constexpr int kBwdKTile = 128;      // keys per CTA
 constexpr int kBwdStages = 3;       // Q/dO/LSE/Delta ring depth
-constexpr int kBwdThreads = 320;    // warp 0 TMA, warp 1 MMA, warps 2..9 two softmax/dQ groups
+constexpr int kBwdThreads = 352;    // warp 0 TMA (query tiles), warp 1 MMA, warps 2..9 two softmax/dQ
+                                    // groups, warp 10 TMA (K, V)
+constexpr int kBwdWarpKV = 10;
 
 constexpr uint32_t kBwdSmemK = 0;                                 // 32 KB
 constexpr uint32_t kBwdSmemV = 32768;                             // 32 KB
@@ -144,15 +146,18 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const BwdParams p) {
 // ------------------------------------------------------------------------------------------------ dK/dV
 
 struct BwdBarriers {
-  uint64_t kv_full;
+  uint64_t k_full, v_full;  // K / V of the current work item landed (one phase per item)
+  uint64_t k_free, v_free;  // the MMAs that read an item's K / V are done: the next item's may load
   uint64_t q_full[kBwdStages], q_empty[kBwdStages];
   uint64_t s_full[2];    // S^T, dP^T of buffer b ready
   uint64_t p_full[2];    // P^T, dS^T written (TMEM + smem)
-  uint64_t dq_full[2];   // dQ^T of buffer b ready (also: dV, dK MMAs of that tile done)
-  uint64_t dq_empty[2];  // dQ^T read out: buffer b free
-  uint64_t b_done[2];    // dV, dK MMAs of the tile in buffer b done (buffer's P^T, dS^T consumed)
-  uint64_t stage_free;   // dQ staging buffer read by the previous tile's bulk reduction (one phase per tile)
-  uint64_t acc_done;     // all MMAs done (epilogue)
+  uint64_t dq_full[2];   // dQ^T of buffer b ready
+  uint64_t dq_empty[2];  // dQ^T read out: buffer b's last 64 columns free
+  uint64_t b_done[2];    // dV, dK MMAs of the step in buffer b done (buffer's P^T, dS^T consumed)
+  uint64_t stage_free[2];  // the dQ staging buffer has been read by the bulk reduction of a step: [gs % 2],
+                          // arrived by that step's group leader (one phase per step of that group)
+  uint64_t acc_done;     // every MMA of an item done: its dV, dK are final (one phase per item)
+  uint64_t acc_free;     // dV, dK read out of tensor memory by the epilogue (8 warps, one phase per item)
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -163,12 +168,42 @@ constexpr uint32_t kBwdSmemAlloc = kBwdSmemBytes + sizeof(BwdBarriers);
 static_assert(kBwdSmemAlloc <= 232448, "dK/dV kernel exceeds the 227 KB shared-memory opt-in");
 
 enum : uint32_t {
-  kSiteBwdLayout = 0x40, kSiteBwdProdQEmpty = 0x41, kSiteBwdMmaKV = 0x51, kSiteBwdMmaQ = 0x52, kSiteBwdMmaDqEmpty = 0x53,
-  kSiteBwdMmaP = 0x54, kSiteBwdSmS = 0x61, kSiteBwdSmQ = 0x62, kSiteBwdSmEpi = 0x63, kSiteBwdDq = 0x71,
-  kSiteBwdDrain = 0x72
+  kSiteBwdLayout = 0x40, kSiteBwdProdQEmpty = 0x41, kSiteBwdProdKV = 0x42, kSiteBwdMmaKV = 0x51, kSiteBwdMmaQ = 0x52,
+  kSiteBwdMmaDqEmpty = 0x53, kSiteBwdMmaP = 0x54, kSiteBwdMmaAcc = 0x55, kSiteBwdSmS = 0x61, kSiteBwdSmQ = 0x62,
+  kSiteBwdSmEpi = 0x63, kSiteBwdDq = 0x71, kSiteBwdDrain = 0x72
 };
 
+// Work item k of this CTA: one 128-key tile of one key/value head. Items are ordered head-major with the
+// heaviest key tile (the first, seen by every query tile) first within a head, and dealt to the CTAs in rounds
+// that alternate direction, as the forward does: the CTAs in flight cover only ~10 heads, so their Q, dO and
+// the heads' fp32 dQ accumulators stay in L2, and the causal work per CTA evens out.
+struct BwdItem {
+  int b, hk, kt;
+  int i0, n;  // query tiles i0 .. i0+n-1 of every query head of the group see these keys
+};
+__device__ __forceinline__ bool bwd_item(int k, const BwdParams& p, BwdItem& it) {
+  const int n_kt = (p.T + kBwdKTile - 1) / kBwdKTile;
+  const long long n_items = static_cast<long long>(p.B) * p.Hkv * n_kt;
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  const long long idx = static_cast<long long>(k) * G + ((k & 1) ? G - 1 - c : c);
+  if (idx >= n_items) return false;
+  const int bhk = static_cast<int>(idx / n_kt);
+  it.kt = static_cast<int>(idx % n_kt);
+  it.b = bhk / p.Hkv;
+  it.hk = bhk % p.Hkv;
+  const int n_q64 = (p.T + kBwdQTile - 1) / kBwdQTile;
+  const int k0 = it.kt * kBwdKTile;
+  it.i0 = k0 / kBwdQTile;  // first query tile that sees these keys
+  // last query tile + 1: all of them, or with a sliding window those holding queries <= k0 + 127 + window
+  const int i_end = p.window < 0 ? n_q64 : min(n_q64, (k0 + kBwdKTile - 1 + p.window) / kBwdQTile + 1);
+  it.n = i_end - it.i0;
+  return true;
+}
 
+// Persistent: one CTA per SM walks its work items. Every ring slot, tensor-memory buffer and per-step barrier
+// phase follows a running step count over all of the CTA's items (gs), every per-item barrier phase the item
+// count (k), so the query tiles of the next item stream in during the current one, and the next item's V and K
+// load as soon as the last MMA that reads this item's has completed.
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -186,27 +221,15 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   BwdBarriers& bars = *reinterpret_cast<BwdBarriers*>(smem + kBwdSmemBytes);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  // Head-major order, heaviest key tile (the first, seen by every query tile) first within a head: the CTAs in
-  // flight cover only ~10 heads, so their Q, dO and the head's fp32 dQ accumulator stay in L2.
-  // A CTA owns one key tile of one key/value head; with grouped-query attention (G query heads per key/value
-  // head) it walks the query tiles of every query head of the group in turn, so dK and dV sum over the group
-  // in tensor memory. Step i is query head hk*G + i/n, query tile i0 + i%n.
-  const int n_kt = (p.T + kBwdKTile - 1) / kBwdKTile;
-  const int G = p.H / p.Hkv;
-  const int bhk = static_cast<int>(blockIdx.x / n_kt);
-  const int kt = static_cast<int>(blockIdx.x % n_kt);
-  const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
-  const int k0 = kt * kBwdKTile;
-  const int n_q64 = (p.T + kBwdQTile - 1) / kBwdQTile;
-  const int i0 = k0 / kBwdQTile;           // first query tile that sees these keys
-  // last query tile + 1: all of them, or with a sliding window those holding queries <= k0 + 127 + window
-  const int i_end = p.window < 0 ? n_q64 : min(n_q64, (k0 + kBwdKTile - 1 + p.window) / kBwdQTile + 1);
-  const int n = i_end - i0;                // query tiles per query head (>= 1)
-  const int ns = G * n;                    // steps of this CTA
+  const int G = p.H / p.Hkv;  // query heads per key/value head: a step is (query head, 64-query tile)
   volatile int* abort = &bars.abort;
+  const uint64_t lim = p.timeout_ns;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars.kv_full, 1);
+    mbar_init(&bars.k_full, 1);
+    mbar_init(&bars.v_full, 1);
+    mbar_init(&bars.k_free, 1);
+    mbar_init(&bars.v_free, 1);
     for (int s = 0; s < kBwdStages; ++s) {
       mbar_init(&bars.q_full[s], 1);
       mbar_init(&bars.q_empty[s], 1);
@@ -218,8 +241,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       mbar_init(&bars.dq_empty[s], 4);  // likewise
       mbar_init(&bars.b_done[s], 1);
     }
-    mbar_init(&bars.stage_free, 1);
+    mbar_init(&bars.stage_free[0], 1);
+    mbar_init(&bars.stage_free[1], 1);
     mbar_init(&bars.acc_done, 1);
+    mbar_init(&bars.acc_free, 8);  // the warps of both groups
     mbar_init(&bars.drain, 1);
     bars.abort = 0;
     fence_barrier_init();
@@ -235,47 +260,78 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   if (threadIdx.x == 0) ATTN_TRACE_EVENT(0, 0);
 
   if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    // The whole warp walks the loop (warp-uniform control flow, so addresses and coordinates stay in uniform
-    // registers); one lane, elected once, issues every copy.
+    // ------------------------------------------------------------------ TMA producer: query tiles
+    // Q, dO, LSE*log2(e) and Delta of every step through the ring. The whole warp walks the loop (warp-uniform
+    // control flow, so addresses and coordinates stay in uniform registers); one lane, elected once, issues.
     const bool leader = elect_one();
     if (leader) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(&bars.kv_full, 4 * 16384);
-      for (int c = 0; c < 2; ++c) {
-        tma_load_4d(smem + kBwdSmemK + c * 16384, &tm_k, &bars.kv_full, c * 64, hk, k0, b);
-        tma_load_4d(smem + kBwdSmemV + c * 16384, &tm_v, &bars.kv_full, c * 64, hk, k0, b);
-      }
     }
     int last_issued[kBwdStages];
     for (int s = 0; s < kBwdStages; ++s) last_issued[s] = -1;
-    for (int i = 0; i < ns; ++i) {
-      const int s = i % kBwdStages;
-      if (i >= kBwdStages && !mbar_wait_warp(&bars.q_empty[s], ((i - kBwdStages) / kBwdStages) & 1, abort,
-                                             p.timeout_ns, &g_device_error, kSiteBwdProdQEmpty))
-        break;
-      const int h = hk * G + i / n, bh = b * p.H + h;  // the step's query head
-      const int q0 = (i0 + i % n) * kBwdQTile;
-      if (leader) {
-        mbar_arrive_expect_tx(&bars.q_full[s], 2 * 16384 + 2 * 256);
-        for (int c = 0; c < 2; ++c) {
-          tma_load_4d(smem + kBwdSmemQ + s * 16384 + c * 8192, &tm_q, &bars.q_full[s], c * 64, h, q0, b);
-          tma_load_4d(smem + kBwdSmemDO + s * 16384 + c * 8192, &tm_do, &bars.q_full[s], c * 64, h, q0, b);
+    int gs = 0;
+    bool ok = true;
+    BwdItem it;
+    for (int k = 0; ok && bwd_item(k, p, it); ++k) {
+      for (int i = 0; i < G * it.n; ++i, ++gs) {
+        const int s = gs % kBwdStages;
+        if (gs >= kBwdStages && !mbar_wait_warp(&bars.q_empty[s], ((gs - kBwdStages) / kBwdStages) & 1, abort, lim,
+                                                &g_device_error, kSiteBwdProdQEmpty)) {
+          ok = false;
+          break;
         }
-        bulk_load(smem + kBwdSmemLse + s * 256, p.lse2 + static_cast<size_t>(bh) * p.Tp + q0, 256, &bars.q_full[s]);
-        bulk_load(smem + kBwdSmemDelta + s * 256, p.delta + static_cast<size_t>(bh) * p.Tp + q0, 256, &bars.q_full[s]);
-        ATTN_TRACE_EVENT(1, i);
+        const int h = it.hk * G + i / it.n, bh = it.b * p.H + h;  // the step's query head
+        const int q0 = (it.i0 + i % it.n) * kBwdQTile;
+        if (leader) {
+          mbar_arrive_expect_tx(&bars.q_full[s], 2 * 16384 + 2 * 256);
+          for (int c = 0; c < 2; ++c) {
+            tma_load_4d(smem + kBwdSmemQ + s * 16384 + c * 8192, &tm_q, &bars.q_full[s], c * 64, h, q0, it.b);
+            tma_load_4d(smem + kBwdSmemDO + s * 16384 + c * 8192, &tm_do, &bars.q_full[s], c * 64, h, q0, it.b);
+          }
+          bulk_load(smem + kBwdSmemLse + s * 256, p.lse2 + static_cast<size_t>(bh) * p.Tp + q0, 256, &bars.q_full[s]);
+          bulk_load(smem + kBwdSmemDelta + s * 256, p.delta + static_cast<size_t>(bh) * p.Tp + q0, 256,
+                    &bars.q_full[s]);
+          ATTN_TRACE_EVENT(1, gs);
+        }
+        last_issued[s] = gs;
       }
-      last_issued[s] = i;
     }
     if (*abort) {
       volatile int no_abort = 0;
-      mbar_wait(&bars.kv_full, 0, &no_abort, p.timeout_ns, &g_device_error, kSiteBwdDrain);
       for (int s = 0; s < kBwdStages; ++s)
         if (last_issued[s] >= 0)
-          mbar_wait(&bars.q_full[s], (last_issued[s] / kBwdStages) & 1, &no_abort, p.timeout_ns, &g_device_error,
+          mbar_wait(&bars.q_full[s], (last_issued[s] / kBwdStages) & 1, &no_abort, lim, &g_device_error,
                     kSiteBwdDrain);
+    }
+  } else if (warp == kBwdWarpKV) {
+    // ------------------------------------------------------------------ TMA producer: K and V of each item
+    // V is read only by the dP^T MMAs, K also by the dQ^T MMAs of the last step: each loads for the next item
+    // as soon as the MMAs that read the current one have completed.
+    const bool leader = elect_one();
+    int k_issued = -1, v_issued = -1;
+    BwdItem it;
+    for (int k = 0; bwd_item(k, p, it); ++k) {
+      const int k0 = it.kt * kBwdKTile;
+      if (k >= 1 && !mbar_wait_warp(&bars.v_free, (k - 1) & 1, abort, lim, &g_device_error, kSiteBwdProdKV)) break;
+      if (leader) {
+        mbar_arrive_expect_tx(&bars.v_full, 2 * 16384);
+        for (int c = 0; c < 2; ++c)
+          tma_load_4d(smem + kBwdSmemV + c * 16384, &tm_v, &bars.v_full, c * 64, it.hk, k0, it.b);
+      }
+      v_issued = k;
+      if (k >= 1 && !mbar_wait_warp(&bars.k_free, (k - 1) & 1, abort, lim, &g_device_error, kSiteBwdProdKV)) break;
+      if (leader) {
+        mbar_arrive_expect_tx(&bars.k_full, 2 * 16384);
+        for (int c = 0; c < 2; ++c)
+          tma_load_4d(smem + kBwdSmemK + c * 16384, &tm_k, &bars.k_full, c * 64, it.hk, k0, it.b);
+      }
+      k_issued = k;
+    }
+    if (*abort) {
+      volatile int no_abort = 0;
+      if (v_issued >= 0) mbar_wait(&bars.v_full, v_issued & 1, &no_abort, lim, &g_device_error, kSiteBwdDrain);
+      if (k_issued >= 0) mbar_wait(&bars.k_full, k_issued & 1, &no_abort, lim, &g_device_error, kSiteBwdDrain);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -291,20 +347,20 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint64_t dk_kmaj = sdesc_sw128(smem_u32(smem + kBwdSmemK), 16, 1024);      // K as K-major A
     const uint64_t dv_kmaj = sdesc_sw128(smem_u32(smem + kBwdSmemV), 16, 1024);      // V as K-major A
     const uint64_t dk_mnmaj = sdesc_sw128(smem_u32(smem + kBwdSmemK), 16384, 1024);  // K^T as MN-major A
-    bool ok = mbar_wait_warp(&bars.kv_full, 0, abort, p.timeout_ns, &g_device_error, kSiteBwdMmaKV);
-    tc_fence_after();
-    // A(i): dP^T and S^T of query tile i into buffer i%2, once its Q/dO tile has landed. dP^T goes first: it
-    // overwrites the buffer's last 64 columns, free once the softmax group has read dQ^T of tile i-2 out of
-    // them; S^T overwrites the first 64, where P^T and dS^T of tile i-2 stay until the dV and dK MMAs of
-    // B(i-2) have read them, so that wait comes second and overlaps dP^T's execution.
-    auto issue_a = [&](int i) -> bool {
-      const int s = i % kBwdStages, rb = i & 1;
-      if (!mbar_wait_warp(&bars.q_full[s], (i / kBwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdMmaQ))
+    // A(gs): dP^T and S^T of step gs into buffer gs%2, once its Q/dO tile has landed. dP^T goes first: it
+    // overwrites the buffer's last 64 columns, free once the softmax group has read dQ^T of step gs-2 out of
+    // them; S^T overwrites the first 64, where P^T and dS^T of step gs-2 stay until the dV and dK MMAs of
+    // B(gs-2) have read them, so that wait comes second and overlaps dP^T's execution. An item's first step
+    // also waits for the item's V (before dP^T) and K (before S^T).
+    auto issue_a = [&](int gs, bool first, int k) -> bool {
+      const int s = gs % kBwdStages, rb = gs & 1;
+      if (!mbar_wait_warp(&bars.q_full[s], (gs / kBwdStages) & 1, abort, lim, &g_device_error, kSiteBwdMmaQ))
         return false;
-      if (i >= 2 && !mbar_wait_warp(&bars.dq_empty[rb], ((i - 2) >> 1) & 1, abort, p.timeout_ns, &g_device_error,
-                                    kSiteBwdMmaDqEmpty))
+      if (gs >= 2 && !mbar_wait_warp(&bars.dq_empty[rb], ((gs - 2) >> 1) & 1, abort, lim, &g_device_error,
+                                     kSiteBwdMmaDqEmpty))
         return false;
-      if (leader) ATTN_TRACE_EVENT(12, i);
+      if (first && !mbar_wait_warp(&bars.v_full, k & 1, abort, lim, &g_device_error, kSiteBwdMmaKV)) return false;
+      if (leader) ATTN_TRACE_EVENT(12, gs);
       tc_fence_after();
       const uint64_t dq0 = sdesc_sw128(smem_u32(smem + kBwdSmemQ + s * 16384), 16, 1024);
       const uint64_t ddo0 = sdesc_sw128(smem_u32(smem + kBwdSmemDO + s * 16384), 16, 1024);
@@ -315,9 +371,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const uint32_t kb = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;   // 64-row boxes
         if (leader) mma_ss(r + 64, dv_kmaj + ka, ddo0 + kb, id_s, kk > 0);
       }
-      if (i >= 2 && !mbar_wait_warp(&bars.b_done[rb], ((i - 2) >> 1) & 1, abort, p.timeout_ns, &g_device_error,
-                                    kSiteBwdMmaDqEmpty))
+      if (gs >= 2 && !mbar_wait_warp(&bars.b_done[rb], ((gs - 2) >> 1) & 1, abort, lim, &g_device_error,
+                                     kSiteBwdMmaDqEmpty))
         return false;
+      if (first && !mbar_wait_warp(&bars.k_full, k & 1, abort, lim, &g_device_error, kSiteBwdMmaKV)) return false;
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
@@ -327,15 +384,17 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       }
       if (leader) {
         mma_commit(&bars.s_full[rb]);
-        ATTN_TRACE_EVENT(2, i);
+        ATTN_TRACE_EVENT(2, gs);
       }
       return true;
     };
-    // B(i): dQ^T = K^T dS^T first (its own commit, so the read-out of dQ^T overlaps the rest), then
-    // dV += P^T dO and dK += dS^T Q (commit: the tile's buffer and its Q/dO ring slot are free).
-    auto issue_b = [&](int i) -> bool {
-      const int s = i % kBwdStages, rb = i & 1;
-      if (!mbar_wait_warp(&bars.p_full[rb], (i >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdMmaP))
+    // B(gs): dQ^T = K^T dS^T first (its own commit, so the read-out of dQ^T overlaps the rest), then
+    // dV += P^T dO and dK += dS^T Q (commit: the step's buffer and its Q/dO ring slot are free). An item's
+    // last dQ^T is the last MMA to read its K; its first dV, dK MMAs overwrite the accumulators, which the
+    // previous item's epilogue must have read out.
+    auto issue_b = [&](int gs, bool first, bool last, int k) -> bool {
+      const int s = gs % kBwdStages, rb = gs & 1;
+      if (!mbar_wait_warp(&bars.p_full[rb], (gs >> 1) & 1, abort, lim, &g_device_error, kSiteBwdMmaP))
         return false;
       tc_fence_after();
       const uint64_t dq_mn = sdesc_sw128(smem_u32(smem + kBwdSmemQ + s * 16384), 8192, 1024);
@@ -345,187 +404,227 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
         if (leader) mma_ss(r + 64, dk_mnmaj + kk * 128, dds_mn + kk * 128, id_dq, kk > 0);
-      if (leader) mma_commit(&bars.dq_full[rb]);
+      if (leader) {
+        mma_commit(&bars.dq_full[rb]);
+        if (last) mma_commit(&bars.k_free);
+      }
+      if (first && k >= 1 &&
+          !mbar_wait_warp(&bars.acc_free, (k - 1) & 1, abort, lim, &g_device_error, kSiteBwdMmaAcc))
+        return false;
+      tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        if (leader) mma_ts(tmem + kTmemDV, r + (kk >> 1) * 32 + (kk & 1) * 8, ddo_mn + kk * 128, id_acc, (i > 0 || kk > 0));
+        if (leader)
+          mma_ts(tmem + kTmemDV, r + (kk >> 1) * 32 + (kk & 1) * 8, ddo_mn + kk * 128, id_acc, (!first || kk > 0));
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        if (leader) mma_ts(tmem + kTmemDK, r + (kk >> 1) * 32 + 16 + (kk & 1) * 8, dq_mn + kk * 128, id_acc, (i > 0 || kk > 0));
+        if (leader)
+          mma_ts(tmem + kTmemDK, r + (kk >> 1) * 32 + 16 + (kk & 1) * 8, dq_mn + kk * 128, id_acc, (!first || kk > 0));
       if (leader) {
         mma_commit(&bars.b_done[rb]);
         mma_commit(&bars.q_empty[s]);
-        ATTN_TRACE_EVENT(3, i);
+        ATTN_TRACE_EVENT(3, gs);
       }
       return true;
     };
-    // Order A(0), A(1), B(0), A(2), B(1), ..., A(n-1), B(n-2), B(n-1): while the softmax group of tile i works
-    // (from the end of A(i) until B(i) can start), the tensor core has B(i-1) and A(i+1) to do, a whole step
-    // of MMAs; the groups' tiles alternate, so their softmax phases hardly overlap.
-    ok = ok && issue_a(0);
-    for (int i = 1; ok && i < ns; ++i) ok = issue_a(i) && issue_b(i - 1);
-    ok = ok && issue_b(ns - 1);
-    if (leader) {
-      mma_commit(&bars.acc_done);
-      mma_commit(&bars.drain);
+    // Per item: A(0), A(1), B(0), A(2), B(1), ..., A(n-1), B(n-2), B(n-1). While the softmax group of step i
+    // works (from the end of A(i) until B(i) can start), the tensor core has B(i-1) and A(i+1) to do, a whole
+    // step of MMAs; the groups' steps alternate, so their softmax phases hardly overlap.
+    bool ok = true;
+    int gs = 0;
+    BwdItem it;
+    for (int k = 0; ok && bwd_item(k, p, it); ++k) {
+      const int ns = G * it.n;
+      ok = issue_a(gs, true, k);
+      for (int i = 1; ok && i < ns; ++i) ok = issue_a(gs + i, false, k) && issue_b(gs + i - 1, i == 1, false, k);
+      if (ok && leader) mma_commit(&bars.v_free);  // every dP^T of the item (the last in A(n-1)) issued
+      ok = ok && issue_b(gs + ns - 1, ns == 1, true, k);
+      if (ok && leader) mma_commit(&bars.acc_done);
+      gs += ns;
     }
+    if (leader) mma_commit(&bars.drain);
     volatile int no_abort = 0;
-    mbar_wait(&bars.drain, 0, &no_abort, p.timeout_ns, &g_device_error, kSiteBwdDrain);
-  } else if (warp < 10) {
+    mbar_wait(&bars.drain, 0, &no_abort, lim, &g_device_error, kSiteBwdDrain);
+  } else {
     // ------------------------------------------------------------------ softmax: one thread per (key row, half)
-    // Two warp groups alternate tiles (ping-pong): group g (warps 2..5 or 6..9) handles the query tiles with
-    // i % 2 == g, which are exactly the tiles of tensor-memory buffer g, so each group has two tiles of
+    // Two warp groups alternate steps (ping-pong): group g (warps 2..5 or 6..9) handles the steps with
+    // gs % 2 == g, which are exactly the steps of tensor-memory buffer g, so each group has a whole step of
     // tensor-core work to hide its softmax behind. A thread handles one key row, in two halves of 32 query
     // columns; each half's packed P^T and dS^T (16 + 16 columns) go over that half's own 32 columns of S^T.
+    // After an item's steps both groups write its dV (group 0) and dK (group 1).
     const int g = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int krow = quarter * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const int kg = k0 + krow;
     const float c = p.scale_log2;
     const bool group_leader = lane == 0 && quarter == 2;  // first warp of the group
     float* dq_stage = reinterpret_cast<float*>(smem + kBwdSmemDQ);
+    // The staging buffer passes between the groups in step order. Step gs's reduction reports on
+    // stage_free[gs % 2], so a group waits only on the other group's barrier, whose phase can be neither behind
+    // nor ahead of the wait by more than one: the other group's next arrival needs this group's next staging.
+    // (With one barrier for both groups a warp could wait two phases ahead of it -- its own leader's arrival
+    // for the previous step still pending -- and a parity wait would then pass at once.)
+    auto wait_staged = [&](int step) -> bool {  // the reduction of `step` has read the staging buffer
+      return mbar_wait_warp(&bars.stage_free[step & 1], (step >> 1) & 1, abort, lim, &g_device_error, kSiteBwdDq);
+    };
     bool ok = true;
-    for (int i = g; i < ns; i += 2) {
-      const int s = i % kBwdStages, rb = g;
-      const int q0 = (i0 + i % n) * kBwdQTile;
-      float* acc_bh = p.dq_acc + static_cast<size_t>(b * p.H + hk * G + i / n) * p.Tp * 128;  // step's query head
-      if (!mbar_wait_warp(&bars.q_full[s], (i / kBwdStages) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdSmQ) ||
-          !mbar_wait_warp(&bars.s_full[rb], (i >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdSmS)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (threadIdx.x == 64 || threadIdx.x == 192) ATTN_TRACE_EVENT(4, i);
-      const bool diag = q0 < k0 + kBwdKTile;  // tile overlaps the key tile: queries before a key see nothing
-      // sliding window: queries after key + window see nothing (only tiles reaching past k0 + window have any)
-      const bool band = p.window >= 0 && q0 + kBwdQTile - 1 > k0 + p.window;
-      uint8_t* dsrow = smem + kBwdSmemDS + rb * 16384;
-      // The half-tile body is instantiated twice: with the sliding-window mask (tiles that reach past a key's
-      // window) and without it, so unwindowed tiles carry no per-element window test.
-      auto halves = [&](auto band_flag) {
-        constexpr bool kBand = decltype(band_flag)::value;
+    int gs0 = 0;  // running step count at the start of the item
+    BwdItem it;
+    for (int k = 0; bwd_item(k, p, it); ++k) {
+      const int ns = G * it.n;
+      const int k0 = it.kt * kBwdKTile;
+      const int kg = k0 + krow;
+      for (int gs = gs0 + ((g - gs0) & 1); ok && gs < gs0 + ns; gs += 2) {
+        const int i = gs - gs0;
+        const int s = gs % kBwdStages, rb = g;
+        const int q0 = (it.i0 + i % it.n) * kBwdQTile;
+        float* acc_bh = p.dq_acc + static_cast<size_t>(it.b * p.H + it.hk * G + i / it.n) * p.Tp * 128;  // step's query head
+        if (!mbar_wait_warp(&bars.q_full[s], (gs / kBwdStages) & 1, abort, lim, &g_device_error, kSiteBwdSmQ) ||
+            !mbar_wait_warp(&bars.s_full[rb], (gs >> 1) & 1, abort, lim, &g_device_error, kSiteBwdSmS)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (threadIdx.x == 64 || threadIdx.x == 192) ATTN_TRACE_EVENT(4, gs);
+        const bool diag = q0 < k0 + kBwdKTile;  // tile overlaps the key tile: queries before a key see nothing
+        // sliding window: queries after key + window see nothing (only tiles reaching past k0 + window have any)
+        const bool band = p.window >= 0 && q0 + kBwdQTile - 1 > k0 + p.window;
+        uint8_t* dsrow = smem + kBwdSmemDS + rb * 16384;
+        // The half-tile body is instantiated twice: with the sliding-window mask (tiles that reach past a key's
+        // window) and without it, so unwindowed tiles carry no per-element window test.
+        auto halves = [&](auto band_flag) {
+          constexpr bool kBand = decltype(band_flag)::value;
 #pragma unroll 1
-        for (int hh = 0; hh < 2; ++hh) {  // one half at a time keeps the live registers to one half's worth
-          const uint32_t r = tmem + lane_base + kTmemR + rb * 128 + 32 * hh;
-          const float4* lse4 = reinterpret_cast<const float4*>(smem + kBwdSmemLse + s * 256) + 8 * hh;
-          const float4* dlt4 = reinterpret_cast<const float4*>(smem + kBwdSmemDelta + s * 256) + 8 * hh;
-          uint32_t sv[32], dp[32];
-          tmem_ld32(r, sv);        // S^T of queries [32hh, 32hh+32)
-          tmem_ld32(r + 64, dp);   // dP^T of the same queries
-          tmem_wait_ld();
-          if (threadIdx.x == 64) ATTN_TRACE_EVENT(8, i * 2 + hh);
-          uint32_t ppk[16], dpk[16];
+          for (int hh = 0; hh < 2; ++hh) {  // one half at a time keeps the live registers to one half's worth
+            const uint32_t r = tmem + lane_base + kTmemR + rb * 128 + 32 * hh;
+            const float4* lse4 = reinterpret_cast<const float4*>(smem + kBwdSmemLse + s * 256) + 8 * hh;
+            const float4* dlt4 = reinterpret_cast<const float4*>(smem + kBwdSmemDelta + s * 256) + 8 * hh;
+            uint32_t sv[32], dp[32];
+            tmem_ld32(r, sv);        // S^T of queries [32hh, 32hh+32)
+            tmem_ld32(r + 64, dp);   // dP^T of the same queries
+            tmem_wait_ld();
+            uint32_t ppk[16], dpk[16];
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            const float4 l4 = lse4[q4], d4 = dlt4[q4];
-            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-            float pv[4], dsv[4];
+            for (int q4 = 0; q4 < 8; ++q4) {
+              const float4 l4 = lse4[q4], d4 = dlt4[q4];
+              const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+              float pv[4], dsv[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int q = q4 * 4 + e;
-              float pe = ex2(fmaf(__uint_as_float(sv[q]), c, -lv[e]));
-              if (diag && q0 + 32 * hh + q < kg) pe = 0.f;
-              if (kBand && q0 + 32 * hh + q > kg + p.window) pe = 0.f;
-              pv[e] = pe;
-              dsv[e] = pe * (__uint_as_float(dp[q]) - dv4[e]);
+              for (int e = 0; e < 4; ++e) {
+                const int q = q4 * 4 + e;
+                float pe = ex2(fmaf(__uint_as_float(sv[q]), c, -lv[e]));
+                if (diag && q0 + 32 * hh + q < kg) pe = 0.f;
+                if (kBand && q0 + 32 * hh + q > kg + p.window) pe = 0.f;
+                pv[e] = pe;
+                dsv[e] = pe * (__uint_as_float(dp[q]) - dv4[e]);
+              }
+              ppk[q4 * 2] = pack_bf16x2(pv[0], pv[1]);
+              ppk[q4 * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+              dpk[q4 * 2] = pack_bf16x2(dsv[0], dsv[1]);
+              dpk[q4 * 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
             }
-            ppk[q4 * 2] = pack_bf16x2(pv[0], pv[1]);
-            ppk[q4 * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-            dpk[q4 * 2] = pack_bf16x2(dsv[0], dsv[1]);
-            dpk[q4 * 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
+            tmem_st16(r, ppk);        // P^T  of these 32 queries: columns [32hh, 32hh+16)
+            tmem_st16(r + 16, dpk);   // dS^T of these 32 queries: columns [32hh+16, 32hh+32)
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+              uint4 v = make_uint4(dpk[ch * 4 + 0], dpk[ch * 4 + 1], dpk[ch * 4 + 2], dpk[ch * 4 + 3]);
+              *reinterpret_cast<uint4*>(dsrow + sw128_offset(krow, 4 * hh + ch)) = v;
+            }
           }
-          if (threadIdx.x == 64) ATTN_TRACE_EVENT(9, i * 2 + hh);
-          tmem_st16(r, ppk);        // P^T  of these 32 queries: columns [32hh, 32hh+16)
-          tmem_st16(r + 16, dpk);   // dS^T of these 32 queries: columns [32hh+16, 32hh+32)
+        };
+        if (band) halves(std::true_type{});
+        else halves(std::false_type{});
+        tmem_wait_st();
+        fence_async_shared();
+        tc_fence_before();
+        mbar_arrive_warp(&bars.p_full[rb]);
+        if (threadIdx.x == 64 || threadIdx.x == 192) ATTN_TRACE_EVENT(5, gs);
+
+        // dQ^T of this step (thread = d, 64 query columns) -> staging buffer in the accumulator's [q/4][d][4]
+        // layout, where the tile is one contiguous 32 KB block -> one bulk reduce-add on the async engine. The
+        // staging buffer passes between the two groups in step order through stage_free.
+        if (!mbar_wait_warp(&bars.dq_full[rb], (gs >> 1) & 1, abort, lim, &g_device_error, kSiteBwdDq)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (threadIdx.x == 64) ATTN_TRACE_EVENT(6, gs);
+        uint32_t a[2][32];
+        tmem_ld32(tmem + lane_base + kTmemR + rb * 128 + 64, a[0]);
+        tmem_ld32(tmem + lane_base + kTmemR + rb * 128 + 96, a[1]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive_warp(&bars.dq_empty[rb]);  // dQ^T is in registers: the tensor-memory columns are free
+        if (gs > 0 && !wait_staged(gs - 1)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            *reinterpret_cast<float4*>(dq_stage + ((8 * hh + q4) * 128 + krow) * 4) =
+                make_float4(__uint_as_float(a[hh][4 * q4]), __uint_as_float(a[hh][4 * q4 + 1]),
+                            __uint_as_float(a[hh][4 * q4 + 2]), __uint_as_float(a[hh][4 * q4 + 3]));
+        fence_async_shared();
+        named_barrier(2 + g, 128);
+        if (group_leader) {
+          bulk_reduce_add_f32(acc_bh + static_cast<size_t>(q0 >> 2) * 512, dq_stage, 32768);
+          tma_store_commit();
+          tma_store_wait_read_all();  // the staging buffer has been read: hand it to the next step
+          mbar_arrive(&bars.stage_free[g]);
+          ATTN_TRACE_EVENT(7, gs);
+        }
+      }
+      // Epilogue of the item: group 0 writes dV, group 1 writes scale*dK: TMEM -> bf16 -> swizzled staging ->
+      // TMA store (rows past T are clipped). Group 0 stages in the dQ staging buffer once the item's last
+      // bulk reduction has read it, group 1 in the two dS^T buffers, free once the item's MMAs are done.
+      // Both groups reach every named barrier, failed or not; nothing is stored after a failure.
+      const int gs_last = gs0 + ns - 1;
+      bool epi_ok = __all_sync(0xffffffffu, ok) &&
+                    mbar_wait_warp(&bars.acc_done, k & 1, abort, lim, &g_device_error, kSiteBwdSmEpi);
+      // group 0: the last reductions of both groups (steps gs_last and gs_last - 1) have read the staging buffer
+      if (epi_ok && g == 0) epi_ok = wait_staged(gs_last) && (gs_last == 0 || wait_staged(gs_last - 1));
+      uint8_t* stage = smem + (g == 0 ? kBwdSmemDQ : kBwdSmemDS);  // 32 KB each: two 16 KB boxes
+      if (epi_ok) {
+        tc_fence_after();
+        const float mul = g == 0 ? 1.0f : p.scale;
+        const uint32_t col = g == 0 ? kTmemDV : kTmemDK;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_base + col + cc * 32, o);
+          tmem_wait_ld();
+          if (cc == 3) {  // the accumulator has been read: the next item's first dV, dK MMAs may overwrite it
+            tc_fence_before();
+            mbar_arrive_warp(&bars.acc_free);
+          }
+          uint8_t* box = stage + (cc >> 1) * 16384;
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
-            uint4 v = make_uint4(dpk[ch * 4 + 0], dpk[ch * 4 + 1], dpk[ch * 4 + 2], dpk[ch * 4 + 3]);
-            *reinterpret_cast<uint4*>(dsrow + sw128_offset(krow, 4 * hh + ch)) = v;
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[ch * 8 + 0]) * mul, __uint_as_float(o[ch * 8 + 1]) * mul);
+            v.y = pack_bf16x2(__uint_as_float(o[ch * 8 + 2]) * mul, __uint_as_float(o[ch * 8 + 3]) * mul);
+            v.z = pack_bf16x2(__uint_as_float(o[ch * 8 + 4]) * mul, __uint_as_float(o[ch * 8 + 5]) * mul);
+            v.w = pack_bf16x2(__uint_as_float(o[ch * 8 + 6]) * mul, __uint_as_float(o[ch * 8 + 7]) * mul);
+            *reinterpret_cast<uint4*>(box + sw128_offset(krow, (cc & 1) * 4 + ch)) = v;
           }
         }
-      };
-      if (band) halves(std::true_type{});
-      else halves(std::false_type{});
-      tmem_wait_st();
-      if (threadIdx.x == 64) ATTN_TRACE_EVENT(10, i);
-      fence_async_shared();
-      if (threadIdx.x == 64) ATTN_TRACE_EVENT(11, i);
-      tc_fence_before();
-      mbar_arrive_warp(&bars.p_full[rb]);
-      if (threadIdx.x == 64 || threadIdx.x == 192) ATTN_TRACE_EVENT(5, i);
-
-      // dQ^T of this tile (thread = d, 64 query columns) -> staging buffer in the accumulator's [q/4][d][4]
-      // layout, where the tile is one contiguous 32 KB block -> one bulk reduce-add on the async engine. The
-      // staging buffer passes between the two groups in tile order through stage_free.
-      if (!mbar_wait_warp(&bars.dq_full[rb], (i >> 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdDq)) {
-        ok = false;
-        break;
       }
-      tc_fence_after();
-      if (threadIdx.x == 64) ATTN_TRACE_EVENT(6, i);
-      uint32_t a[2][32];
-      tmem_ld32(tmem + lane_base + kTmemR + rb * 128 + 64, a[0]);
-      tmem_ld32(tmem + lane_base + kTmemR + rb * 128 + 96, a[1]);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive_warp(&bars.dq_empty[rb]);  // dQ^T is in registers: the tensor-memory buffer is free
-      if (i > 0 && !mbar_wait_warp(&bars.stage_free, (i - 1) & 1, abort, p.timeout_ns, &g_device_error, kSiteBwdDq)) {
-        ok = false;
-        break;
-      }
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4)
-          *reinterpret_cast<float4*>(dq_stage + ((8 * hh + q4) * 128 + krow) * 4) =
-              make_float4(__uint_as_float(a[hh][4 * q4]), __uint_as_float(a[hh][4 * q4 + 1]),
-                          __uint_as_float(a[hh][4 * q4 + 2]), __uint_as_float(a[hh][4 * q4 + 3]));
       fence_async_shared();
       named_barrier(2 + g, 128);
-      if (group_leader) {
-        bulk_reduce_add_f32(acc_bh + static_cast<size_t>(q0 >> 2) * 512, dq_stage, 32768);
+      if (group_leader && epi_ok && !*abort) {
+        const CUtensorMap* tm = g == 0 ? &tm_dv : &tm_dk;
+        for (int cc = 0; cc < 2; ++cc) tma_store_4d(tm, stage + cc * 16384, cc * 64, it.hk, k0, it.b);
         tma_store_commit();
-        tma_store_wait_read_all();  // the staging buffer has been read: hand it to the next tile
-        mbar_arrive(&bars.stage_free);
-        ATTN_TRACE_EVENT(7, i);
+        tma_store_wait_read_all();  // the staging area is free again
       }
+      // Both groups continue only once both stores have read their staging: the next item's first dS^T and dQ
+      // staging writes go there. Leave together on the same decision.
+      if (!named_barrier_and(1, 256, epi_ok && !*abort)) break;
+      gs0 += ns;
     }
-    if (group_leader) tma_store_wait_all();  // this group's reductions are complete before the CTA retires
-    // Epilogue: group 0 writes dV, group 1 writes scale*dK: TMEM -> bf16 -> swizzled staging -> TMA store
-    // (rows past T are clipped). Both groups reach the named barrier, failed or not; no store on abort.
-    const bool epi_ok = __all_sync(0xffffffffu, ok) &&
-                        mbar_wait_warp(&bars.acc_done, 0, abort, p.timeout_ns, &g_device_error, kSiteBwdSmEpi);
-    uint8_t* stage = smem + (g == 0 ? kBwdSmemQ : kBwdSmemDO);  // 32 KB each (first two ring slots)
-    if (epi_ok) {
-      tc_fence_after();
-      const float mul = g == 0 ? 1.0f : p.scale;
-      const uint32_t col = g == 0 ? kTmemDV : kTmemDK;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tmem + lane_base + col + cc * 32, o);
-        tmem_wait_ld();
-        uint8_t* box = stage + (cc >> 1) * 16384;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(o[ch * 8 + 0]) * mul, __uint_as_float(o[ch * 8 + 1]) * mul);
-          v.y = pack_bf16x2(__uint_as_float(o[ch * 8 + 2]) * mul, __uint_as_float(o[ch * 8 + 3]) * mul);
-          v.z = pack_bf16x2(__uint_as_float(o[ch * 8 + 4]) * mul, __uint_as_float(o[ch * 8 + 5]) * mul);
-          v.w = pack_bf16x2(__uint_as_float(o[ch * 8 + 6]) * mul, __uint_as_float(o[ch * 8 + 7]) * mul);
-          *reinterpret_cast<uint4*>(box + sw128_offset(krow, (cc & 1) * 4 + ch)) = v;
-        }
-      }
-    }
-    fence_async_shared();
-    named_barrier(1, 256);
-    if ((warp == 2 || warp == 6) && lane == 0 && !*abort) {
-      const CUtensorMap* tm = g == 0 ? &tm_dv : &tm_dk;
-      for (int cc = 0; cc < 2; ++cc) tma_store_4d(tm, stage + cc * 16384, cc * 64, hk, k0, b);
-      tma_store_commit();
-      tma_store_wait_read_all();
-    }
+    if (group_leader) tma_store_wait_all();  // this group's reductions and stores are complete before exit
   }
 
   tc_fence_before();

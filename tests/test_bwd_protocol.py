@@ -1,22 +1,28 @@
 """A discrete-event model of the dK/dV backward kernel's barrier protocol, checked on the CPU.
 
-attn_bwd_dkdv_kernel's roles talk only through mbarriers: the TMA producer (K and V once, then query tiles of
-Q, dO, LSE and Delta through a 3-slot ring), the MMA warp (in the order A(0), A(1), B(0), A(2), B(1), ...,
-B(n-1): A writes dP^T, then S^T into tensor-memory buffer i % 2, B computes dQ^T, then dV and dK), and two softmax groups
-that take the tiles in turn (group g owns the tiles i = g mod 2 and buffer g). Each group hands the 32 KB dQ
-staging buffer to the other in tile order through one barrier. Barrier counts follow the kernel: the
-softmax-side barriers count warps, so a group of four warps is one actor arriving 4. MMAs, commits and copies
-complete at once (timing does not matter for these properties). Over random step counts and interleavings the
-model checks that
+attn_bwd_dkdv_kernel is persistent: a CTA walks several work items (key tiles), and its roles talk only through
+mbarriers: the TMA producer of query tiles (Q, dO, LSE and Delta of every step through a 3-slot ring, running on
+across items), the K/V producer (each item's V once the last dP^T of the previous item is done, its K once the
+last dQ^T is), the MMA warp (per item in the order A(0), A(1), B(0), A(2), B(1), ..., B(n-1): A writes dP^T, then
+S^T into tensor-memory buffer gs % 2 of the running step gs, B computes dQ^T, then dV and dK), and two softmax
+groups that take the steps in turn (group g owns the steps gs = g mod 2 and buffer g) and after each item write
+its dV and dK (the item's first dV, dK MMAs wait until they have been read out). The groups hand the 32 KB dQ
+staging buffer to each other in step order: step gs's bulk reduction reports on stage_free[gs % 2]. Barrier
+counts follow the kernel: the softmax-side barriers count warps, and each group is two actors -- the leader's
+warp, which also issues the reductions and reports their reads, and the other three warps, which can run ahead
+of it. MMAs, commits and copies complete at once (timing does not matter for these properties). Over random item
+mixes and interleavings the model checks that
 
-  * every role runs to the end (no deadlock: a role only waits for something another role will still do), and
+  * every role runs to the end (no deadlock: a role only waits for something another role will still do),
   * no parity wait can be fooled: when a wait for phase n of a barrier succeeds, phase n + 1 has not completed
     yet (a parity wait only sees the current phase's parity, so a waiter two phases behind would hang or pass
-    on the wrong phase).
+    on the wrong phase), and
+  * the staging buffer is never written (dQ of a step, or an item's dV) while a reduction is still reading it.
 
-Two negative controls must fail: the dQ staging hand-off waiting for the tile's own release (an off-by-one)
-deadlocks, and a producer that refills ring slots without waiting for their release runs the softmax groups'
-waits two phases behind.
+Negative controls must fail: a producer that refills ring slots without waiting for their release runs the
+softmax groups' waits two phases behind; one stage barrier shared by both groups lets a warp wait two phases
+ahead of it and stage over a tile being read; an epilogue that stages dV without waiting for the item's last
+reductions does the same.
 """
 import random
 
@@ -37,17 +43,26 @@ class Barrier:
 
 
 class Model:
-    def __init__(self, ns, bug=None):
-        self.ns, self.bug = ns, bug
-        self.b = {"kv_full": Barrier(1), "stage_free": Barrier(1), "acc_done": Barrier(1), "drain": Barrier(1)}
+    def __init__(self, items, bug=None):
+        self.items, self.bug = items, bug  # items: steps of each work item of the CTA
+        self.b = {name: Barrier(1) for name in ("k_full", "v_full", "k_free", "v_free", "stage_free0",
+                                                 "stage_free1", "acc_done", "drain")}
+        self.b["acc_free"] = Barrier(8)
         for s in range(STAGES):
             self.b[f"q_full{s}"] = Barrier(1)
             self.b[f"q_empty{s}"] = Barrier(1)
         for r in range(2):
             for name, count in (("s_full", 1), ("p_full", 4), ("dq_full", 1), ("dq_empty", 4), ("b_done", 1)):
                 self.b[f"{name}{r}"] = Barrier(count)
-        self.epilogue_named = 0  # groups that reached the epilogue's named barrier
+        self.named = {}  # named barrier instance -> actors that reached it
+        self.single_done = 0  # completions of a single stage barrier for both groups (negative control)
+        self.staged_reads_pending = set()  # steps whose dQ staging has been written but not yet read
         self.violations = []
+
+    def wait_single(self, n):
+        """The parity wait of one stage barrier shared by both groups: it passes when the barrier's current
+        phase has the other parity, also when it is two phases behind completion n."""
+        return lambda: (self.single_done & 1) != (n & 1) or self.single_done > n
 
     def wait(self, name, n):
         """Wait for completion n (0-based) of a barrier: the kernel's parity wait on phase n."""
@@ -61,65 +76,128 @@ class Model:
 
 
 def producer(m):
-    m.b["kv_full"].arrive()
-    for i in range(m.ns):
-        s = i % STAGES
-        if i >= STAGES and m.bug != "no_ring_release_wait":
-            yield m.wait(f"q_empty{s}", (i - STAGES) // STAGES)
-        m.b[f"q_full{s}"].arrive()
+    gs = 0
+    for ns in m.items:
+        for _ in range(ns):
+            s = gs % STAGES
+            if gs >= STAGES and m.bug != "no_ring_release_wait":
+                yield m.wait(f"q_empty{s}", (gs - STAGES) // STAGES)
+            m.b[f"q_full{s}"].arrive()
+            gs += 1
+
+
+def kv_producer(m):
+    for k, _ in enumerate(m.items):
+        if k >= 1:
+            yield m.wait("v_free", k - 1)
+        m.b["v_full"].arrive()
+        if k >= 1:
+            yield m.wait("k_free", k - 1)
+        m.b["k_full"].arrive()
 
 
 def mma(m):
-    yield m.wait("kv_full", 0)
-
-    def issue_a(i):
-        s, rb = i % STAGES, i & 1
-        yield m.wait(f"q_full{s}", i // STAGES)
-        if i >= 2:
-            yield m.wait(f"dq_empty{rb}", (i - 2) >> 1)  # dP^T overwrites the dQ^T columns
-            yield m.wait(f"b_done{rb}", (i - 2) >> 1)    # S^T overwrites P^T, dS^T
+    def issue_a(gs, first, k):
+        s, rb = gs % STAGES, gs & 1
+        yield m.wait(f"q_full{s}", gs // STAGES)
+        if gs >= 2:
+            yield m.wait(f"dq_empty{rb}", (gs - 2) >> 1)  # dP^T overwrites the dQ^T columns
+        if first:
+            yield m.wait("v_full", k)
+        if gs >= 2:
+            yield m.wait(f"b_done{rb}", (gs - 2) >> 1)    # S^T overwrites P^T, dS^T
+        if first:
+            yield m.wait("k_full", k)
         m.b[f"s_full{rb}"].arrive()
 
-    def issue_b(i):
-        s, rb = i % STAGES, i & 1
-        yield m.wait(f"p_full{rb}", i >> 1)
+    def issue_b(gs, first, last, k):
+        s, rb = gs % STAGES, gs & 1
+        yield m.wait(f"p_full{rb}", gs >> 1)
         m.b[f"dq_full{rb}"].arrive()
+        if last:
+            m.b["k_free"].arrive()
+        if first and k >= 1:
+            yield m.wait("acc_free", k - 1)
         m.b[f"b_done{rb}"].arrive()
         m.b[f"q_empty{s}"].arrive()
 
-    yield from issue_a(0)
-    for i in range(1, m.ns):
-        yield from issue_a(i)
-        yield from issue_b(i - 1)
-    yield from issue_b(m.ns - 1)
-    m.b["acc_done"].arrive()
+    gs = 0
+    for k, ns in enumerate(m.items):
+        yield from issue_a(gs, True, k)
+        for i in range(1, ns):
+            yield from issue_a(gs + i, False, k)
+            yield from issue_b(gs + i - 1, i == 1, False, k)
+        m.b["v_free"].arrive()
+        yield from issue_b(gs + ns - 1, ns == 1, True, k)
+        m.b["acc_done"].arrive()
+        gs += ns
     m.b["drain"].arrive()
     yield m.wait("drain", 0)
 
 
-def softmax_group(m, g):
-    for i in range(g, m.ns, 2):
-        s, rb = i % STAGES, g
-        yield m.wait(f"q_full{s}", i // STAGES)
-        yield m.wait(f"s_full{rb}", i >> 1)
-        m.b[f"p_full{rb}"].arrive(4)
-        yield m.wait(f"dq_full{rb}", i >> 1)
-        m.b[f"dq_empty{rb}"].arrive(4)
-        if m.bug == "stage_wait_own_release":
-            yield m.wait("stage_free", i)
-        elif i > 0:
-            yield m.wait("stage_free", i - 1)
-        m.b["stage_free"].arrive()  # the group leader, once the bulk reduction has read the staging buffer
-    yield m.wait("acc_done", 0)
-    m.epilogue_named += 1
-    yield lambda: m.epilogue_named == 2  # named barrier of both groups before the dK / dV stores
+def named_barrier(m, key, actor, n_actors):
+    m.named.setdefault(key, set()).add(actor)
+    return lambda: len(m.named[key]) == n_actors
 
 
-def run(ns, seed, bug=None):
+def softmax_warps(m, g, lead):
+    """The warps of softmax group g: the group leader's warp (lead) or the other three. They run the same waits;
+    the leader also issues each step's bulk reduction of the dQ staging buffer and reports its read on
+    stage_free[g], after the group's staging barrier, so the other warps can run ahead of it."""
+    n = 1 if lead else 3
+    actor = (g, lead)
+
+    def wait_staged(step):
+        return m.wait(f"stage_free{step & 1}", step >> 1)
+
+    gs0 = 0
+    for k, ns in enumerate(m.items):
+        for gs in range(gs0 + ((g - gs0) & 1), gs0 + ns, 2):
+            s, rb = gs % STAGES, g
+            yield m.wait(f"q_full{s}", gs // STAGES)
+            yield m.wait(f"s_full{rb}", gs >> 1)
+            m.b[f"p_full{rb}"].arrive(n)
+            yield m.wait(f"dq_full{rb}", gs >> 1)
+            m.b[f"dq_empty{rb}"].arrive(n)
+            if gs > 0:
+                if m.bug == "single_stage_barrier":  # one barrier for both groups, waited at its own parity
+                    yield m.wait_single(gs - 1)
+                else:
+                    yield wait_staged(gs - 1)
+            if m.staged_reads_pending:
+                m.violations.append(("dQ staged over an unread tile", gs))
+            yield named_barrier(m, ("stage", gs), actor, 2)
+            if lead:
+                m.staged_reads_pending.add(gs)   # the bulk reduction is issued ...
+                yield lambda: True
+                m.staged_reads_pending.discard(gs)  # ... and has read the buffer
+                m.b[f"stage_free{g}"].arrive()
+                m.single_done += 1
+        # epilogue: both groups, after the item's last MMA; group 0 stages dV where the last dQ tile was staged
+        yield m.wait("acc_done", k)
+        gs_last = gs0 + ns - 1
+        if g == 0 and m.bug != "epilogue_skips_stage_wait":
+            if m.bug == "single_stage_barrier":
+                yield m.wait_single(gs_last)
+            else:
+                yield wait_staged(gs_last)
+                if gs_last > 0:
+                    yield wait_staged(gs_last - 1)
+        if g == 0 and m.staged_reads_pending:
+            m.violations.append(("dV staged over a dQ tile not yet read", k))
+        m.b["acc_free"].arrive(n)
+        yield named_barrier(m, ("epilogue", k), actor, 4)  # both groups, after the stores
+        gs0 += ns
+
+
+def run(items, seed, bug=None):
     """Random interleaving of the roles; returns (finished, violations)."""
-    m = Model(ns, bug)
+    m = Model(items, bug)
     rng = random.Random(seed)
-    roles = {"tma": producer(m), "mma": mma(m), "g0": softmax_group(m, 0), "g1": softmax_group(m, 1)}
+    roles = {"tma": producer(m), "kv": kv_producer(m), "mma": mma(m)}
+    for g in range(2):
+        for lead in (True, False):
+            roles[f"g{g}{'lead' if lead else 'rest'}"] = softmax_warps(m, g, lead)
     waiting = {name: None for name in roles}
     alive = set(roles)
     while alive:
@@ -134,33 +212,48 @@ def run(ns, seed, bug=None):
     return True, m.violations
 
 
+def random_items(rng):
+    """A CTA's work items: steps per item, long and short ones mixed (one-step items stress the boundaries)."""
+    return [rng.randint(1, 32) if rng.random() < 0.6 else rng.randint(1, 3) for _ in range(rng.randint(1, 6))]
+
+
 def test_protocol_has_no_deadlock_and_no_ambiguous_parity_wait():
-    """Step counts of every shape the kernel meets: one tile, odd counts (a lone last A/B), the G * n steps of
-    grouped-query heads, and long walks."""
+    """Item mixes of every shape the kernel meets: one-step items, odd step counts (a lone last A/B), the G * n
+    steps of grouped-query heads, and long walks, several items per CTA."""
     rng = random.Random(99)
     for trial in range(1500):
-        ns = rng.choice([1, 2, 3, 4, 5]) if rng.random() < 0.4 else rng.randint(1, 64)
-        finished, violations = run(ns, trial)
-        assert finished, f"deadlock with {ns} steps (schedule seed {trial})"
-        assert not violations, f"parity wait two phases behind with {ns} steps: {violations[:3]}"
+        items = random_items(rng)
+        finished, violations = run(items, trial)
+        assert finished, f"deadlock with items {items} (schedule seed {trial})"
+        assert not violations, f"parity wait two phases behind with items {items}: {violations[:3]}"
 
 
-@pytest.mark.parametrize("ns", [1, 2, 3, 6, 7, 32, 33])
-def test_protocol_corner_step_counts(ns):
+@pytest.mark.parametrize("items", [[1], [2], [3], [1, 1, 1], [32, 1, 2], [6, 7], [33, 32, 31]])
+def test_protocol_corner_item_mixes(items):
     for seed in range(100):
-        finished, violations = run(ns, seed)
+        finished, violations = run(items, seed)
         assert finished and not violations
 
 
-def test_model_catches_a_deadlocking_hand_off():
-    """Negative control: tile i waiting for its own release of the staging buffer never proceeds."""
-    assert not run(1, 0, bug="stage_wait_own_release")[0]
-    assert not any(run(ns, seed, bug="stage_wait_own_release")[0] for ns in (2, 5) for seed in range(20))
+def test_model_catches_a_single_stage_barrier_race():
+    """Negative control: with one stage barrier for both groups a warp can wait two phases ahead of it (its own
+    leader's arrival still pending), pass at once and stage over a tile that is still being read."""
+    rng = random.Random(11)
+    caught = sum(bool(run(random_items(rng), seed, bug="single_stage_barrier")[1]) for seed in range(300))
+    assert caught > 0
 
 
 def test_model_catches_a_ring_overrun():
     """Negative control: without the wait for a slot's release the producer can complete a slot's phases two
     ahead of a softmax group's wait."""
     rng = random.Random(3)
-    caught = sum(bool(run(rng.randint(7, 40), seed, bug="no_ring_release_wait")[1]) for seed in range(200))
+    caught = sum(bool(run(random_items(rng), seed, bug="no_ring_release_wait")[1]) for seed in range(200))
+    assert caught > 0
+
+
+def test_model_catches_an_epilogue_overwriting_the_last_dq_tile():
+    """Negative control: group 0's dV staging without the wait for the item's last bulk reduction can overwrite
+    a dQ tile that the other group's reduction has not read yet."""
+    rng = random.Random(5)
+    caught = sum(bool(run(random_items(rng), seed, bug="epilogue_skips_stage_wait")[1]) for seed in range(200))
     assert caught > 0
