@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const BwdParams p) {
 struct BwdBarriers {
   uint64_t k_full, v_full;  // K / V of the current work item landed (one phase per item)
   uint64_t k_free, v_free;  // the MMAs that read an item's K / V are done: the next item's may load
+  uint64_t kv_issued;       // an item's K and V loads are issued: its query tiles may queue behind them
   uint64_t q_full[kBwdStages], q_empty[kBwdStages];
   uint64_t s_full[2];    // S^T, dP^T of buffer b ready
   uint64_t p_full[2];    // P^T, dS^T written (TMEM + smem)
@@ -230,6 +231,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     mbar_init(&bars.v_full, 1);
     mbar_init(&bars.k_free, 1);
     mbar_init(&bars.v_free, 1);
+    mbar_init(&bars.kv_issued, 1);
     for (int s = 0; s < kBwdStages; ++s) {
       mbar_init(&bars.q_full[s], 1);
       mbar_init(&bars.q_empty[s], 1);
@@ -274,6 +276,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     bool ok = true;
     BwdItem it;
     for (int k = 0; ok && bwd_item(k, p, it); ++k) {
+      // The item's first query tiles are needed together with its K and V, which load only once the previous
+      // item's last MMAs have read theirs: queueing the tiles behind them on the copy engine gets all three
+      // in sooner than loading the tiles early and the K/V behind them.
+      if (!mbar_wait_warp(&bars.kv_issued, k & 1, abort, lim, &g_device_error, kSiteBwdProdQEmpty)) break;
       for (int i = 0; i < G * it.n; ++i, ++gs) {
         const int s = gs % kBwdStages;
         if (gs >= kBwdStages && !mbar_wait_warp(&bars.q_empty[s], ((gs - kBwdStages) / kBwdStages) & 1, abort, lim,
@@ -307,12 +313,18 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   } else if (warp == kBwdWarpKV) {
     // ------------------------------------------------------------------ TMA producer: K and V of each item
     // V is read only by the dP^T MMAs, K also by the dQ^T MMAs of the last step: each loads for the next item
-    // as soon as the MMAs that read the current one have completed.
+    // as soon as the MMAs that read the current one have completed. Both come from DRAM (a key tile is read by
+    // one CTA only), so the next item's are first prefetched into L2 while the current item is computed.
     const bool leader = elect_one();
     int k_issued = -1, v_issued = -1;
-    BwdItem it;
+    BwdItem it, nx;
     for (int k = 0; bwd_item(k, p, it); ++k) {
       const int k0 = it.kt * kBwdKTile;
+      if (leader && bwd_item(k + 1, p, nx))
+        for (int c = 0; c < 2; ++c) {
+          tma_prefetch_l2_4d(&tm_k, c * 64, nx.hk, nx.kt * kBwdKTile, nx.b);
+          tma_prefetch_l2_4d(&tm_v, c * 64, nx.hk, nx.kt * kBwdKTile, nx.b);
+        }
       if (k >= 1 && !mbar_wait_warp(&bars.v_free, (k - 1) & 1, abort, lim, &g_device_error, kSiteBwdProdKV)) break;
       if (leader) {
         mbar_arrive_expect_tx(&bars.v_full, 2 * 16384);
@@ -327,6 +339,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           tma_load_4d(smem + kBwdSmemK + c * 16384, &tm_k, &bars.k_full, c * 64, it.hk, k0, it.b);
       }
       k_issued = k;
+      mbar_arrive_warp(&bars.kv_issued);
     }
     if (*abort) {
       volatile int no_abort = 0;

@@ -169,6 +169,14 @@ ATTN_DEVICE_INLINE void tma_load_4d(void* dst, const void* tmap, uint64_t* bar, 
       : "memory");
 }
 
+// Prefetch a TMA tile into L2 (no shared memory, no completion to wait for).
+ATTN_DEVICE_INLINE void tma_prefetch_l2_4d(const void* tmap, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+
 ATTN_DEVICE_INLINE void tma_store_4d(const void* tmap, const void* src, int c0, int c1, int c2, int c3) {
   asm volatile(
       "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(

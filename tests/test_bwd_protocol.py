@@ -2,7 +2,7 @@
 
 attn_bwd_dkdv_kernel is persistent: a CTA walks several work items (key tiles), and its roles talk only through
 mbarriers: the TMA producer of query tiles (Q, dO, LSE and Delta of every step through a 3-slot ring, running on
-across items), the K/V producer (each item's V once the last dP^T of the previous item is done, its K once the
+across items; an item's tiles are queued once its K and V loads are), the K/V producer (each item's V once the last dP^T of the previous item is done, its K once the
 last dQ^T is), the MMA warp (per item in the order A(0), A(1), B(0), A(2), B(1), ..., B(n-1): A writes dP^T, then
 S^T into tensor-memory buffer gs % 2 of the running step gs, B computes dQ^T, then dV and dK), and two softmax
 groups that take the steps in turn (group g owns the steps gs = g mod 2 and buffer g) and after each item write
@@ -45,7 +45,7 @@ class Barrier:
 class Model:
     def __init__(self, items, bug=None):
         self.items, self.bug = items, bug  # items: steps of each work item of the CTA
-        self.b = {name: Barrier(1) for name in ("k_full", "v_full", "k_free", "v_free", "stage_free0",
+        self.b = {name: Barrier(1) for name in ("k_full", "v_full", "k_free", "v_free", "kv_issued", "stage_free0",
                                                  "stage_free1", "acc_done", "drain")}
         self.b["acc_free"] = Barrier(8)
         for s in range(STAGES):
@@ -77,7 +77,8 @@ class Model:
 
 def producer(m):
     gs = 0
-    for ns in m.items:
+    for k, ns in enumerate(m.items):
+        yield m.wait("kv_issued", k)  # the item's query tiles queue behind its K and V
         for _ in range(ns):
             s = gs % STAGES
             if gs >= STAGES and m.bug != "no_ring_release_wait":
@@ -94,6 +95,7 @@ def kv_producer(m):
         if k >= 1:
             yield m.wait("k_free", k - 1)
         m.b["k_full"].arrive()
+        m.b["kv_issued"].arrive()
 
 
 def mma(m):
