@@ -36,7 +36,8 @@ from workloads import WORKLOADS, Workload  # noqa: E402
 METRIC = "causal attention fwd+bwd TFLOP/s (bf16, d20 shape) and % of B200 tensor peak"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
-KERNEL_SOURCES = ["attn_api.cu", "attn_fwd.cuh", "attn_bwd.cuh", "attn_decode.cuh", "attn_common.cuh", "sm100.cuh"]
+KERNEL_SOURCES = ["attn_api.cu", "attn_fwd.cuh", "attn_bwd.cuh", "attn_decode.cuh", "attn_common.cuh", "attn_errors.h",
+                  "sm100.cuh"]
 PROLOGUE_SOURCES = ["attn_rope.cu"]  # the prologue's kernels and launches are all in this file
 
 
@@ -52,6 +53,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed oracle sample")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--sustained-seconds", type=float, default=2.5,
+                    help="length of the sustained leg (the same step looped, with its own clock record); 0 skips it")
     return ap.parse_args(argv)
 
 
@@ -242,7 +245,7 @@ def run_reference(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": workload_config(w),
+        "config": dict(workload_config(w), parallelism=f"replicas x{args.gpus} (no collective on the data path)"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -263,20 +266,10 @@ def workload_config(w: Workload):
 # ------------------------------------------------------------------------------------------------ GPU arm
 
 def make_device_inputs(w: Workload, device):
-    import torch
-    g = torch.Generator(device=device)
-    g.manual_seed(w.seed)
-    shape, kv_shape = (w.B, w.T, w.H, w.D), (w.B, w.T, w.kv_heads, w.D)
-    q = torch.randn(shape, generator=g, device=device)
-    k = torch.randn(kv_shape, generator=g, device=device)
-    v = torch.randn(kv_shape, generator=g, device=device)
-    do = torch.randn(shape, generator=g, device=device)
-    if w.qk_prescale != 1.0:
-        q.mul_(w.qk_prescale)
-        k.mul_(w.qk_prescale)
-    if w.key_bias:
-        k.add_(torch.randn((w.D,), generator=g, device=device))
-    return [t.to(torch.bfloat16) for t in (q, k, v, do)]
+    """The workload's seeded inputs (workloads.make_inputs: the same CPU generator and bytes the parity tests
+    check), copied to the device."""
+    from workloads import make_inputs
+    return [t.to(device) for t in make_inputs(w)]
 
 
 def run_ours(args):
@@ -423,6 +416,30 @@ def run_ours(args):
         "roofline": roofline, "kernels": breakdown, "gpu_launches": 4 * args.steps, "clocks": clocks,
         "kernel_source_hash": kernel_source_hash(),
     }
+
+    # Sustained leg: the same step back to back for a few seconds, its own clock record, against the sustained
+    # (power-capped) GEMM peak. The headline value stays the timed steps above (a burst of args.steps steps).
+    if args.sustained_seconds > 0:
+        n_sus = max(1, int(math.ceil(args.sustained_seconds * 1e3 / ms_step)))
+        sampler = ClockSampler(gpu_id)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(device)
+        sampler.start()
+        time.sleep(0.1)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(n_sus):
+            step()
+        s1.record(stream)
+        torch.cuda.synchronize(device)
+        sus_clocks = sampler.stop()
+        sus_ms = reduce_max(s0.elapsed_time(s1), world, device)
+        sus_value = aggregate((f_fwd + f_bwd) * n_sus, world, sus_ms / 1e3) / 1e12
+        line["sustained"] = {"value": sus_value, "unit": UNIT, "steps": n_sus, "seconds": sus_ms / 1e3,
+                             "ms_per_step": sus_ms / n_sus, "pct_of_sustained_peak": 100.0 * (sus_value / world) /
+                             peak_tf_sus, "peak": peak_tf_sus, "clocks": sus_clocks}
+        line["gpu_launches_sustained"] = 4 * n_sus  # forward + the backward's three kernels, per step
 
     # End to end through the public Python API with host buffers: H2D of q, k, v, dO from pinned memory,
     # forward, backward, D2H of o, lse, dq, dk, dv, every step.

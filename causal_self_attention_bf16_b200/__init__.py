@@ -46,7 +46,6 @@ SIGNATURES = {
     "attn_decode": ([_VP] * 7 + [_SZ] + [_I] * 6 + [_F, _VP], _I),
     "attn_qk_norm_rope": ([_VP] * 5 + [_I] * 5 + [_F, _F, _I, _VP], _I),
     "attn_qk_norm_rope_bwd": ([_VP] * 7 + [_I] * 5 + [_F, _F, _I, _VP], _I),
-    "attn_prologue_last_cuda_error": ([], ctypes.c_char_p),
     "attn_get_device_error": ([ctypes.POINTER(ctypes.c_uint32)], _I),
     "attn_clear_device_error": ([], _I),
     "attn_set_wait_limit_ns": ([_U64], _I),
@@ -90,8 +89,7 @@ def _check(fn: str, status: int):
         detail = ""
         if status == 4:
             lib = load_library()
-            text = lib.attn_prologue_last_cuda_error() if "qk_norm_rope" in fn else lib.attn_last_cuda_error()
-            detail = text.decode(errors="replace")
+            detail = lib.attn_last_cuda_error().decode(errors="replace")
         raise AttnError(fn, status, detail)
 
 

@@ -15,7 +15,7 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libattn.so")
 SOURCES = ["attn_api.cu", "attn_rope.cu"]
-DEPENDS = ["attn_api.cu", "attn_rope.cu", "attn_fwd.cuh", "attn_bwd.cuh", "attn_decode.cuh", "attn_common.cuh", "sm100.cuh"]
+DEPENDS = ["attn_api.cu", "attn_rope.cu", "attn_fwd.cuh", "attn_bwd.cuh", "attn_decode.cuh", "attn_common.cuh", "attn_errors.h", "sm100.cuh"]
 
 
 def nvcc_path() -> str:

@@ -10,12 +10,17 @@
 
 #include "attn.h"
 #include "attn_bwd.cuh"
+#include "attn_errors.h"
 #include "attn_decode.cuh"
 #include "attn_fwd.cuh"
 
+namespace attn {
+thread_local char g_cuda_error[kErrorTextBytes] = "";
+}  // namespace attn
+
 namespace {
 
-thread_local char g_cuda_error[256] = "";
+using attn::g_cuda_error;
 uint64_t g_wait_limit_ns = 1000ull * 1000 * 1000;  // 1 s
 
 attn_status cuda_fail(cudaError_t e, const char* what) {
@@ -187,7 +192,7 @@ __global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
 
 extern "C" {
 
-int attn_abi_version(void) { return 1; }
+int attn_abi_version(void) { return 2; }
 
 const char* attn_status_string(attn_status s) {
   switch (s) {

@@ -23,6 +23,7 @@
 #include <cstdio>
 
 #include "attn.h"
+#include "attn_errors.h"
 
 namespace {
 
@@ -30,8 +31,6 @@ constexpr int kRopeThreads = 256;
 constexpr int kRopeChunks = 16;                            // 16-byte chunks in a 128-dim bf16 row
 constexpr int kRopePositions = kRopeThreads / kRopeChunks;  // positions per block iteration
 constexpr int kRopeUnroll = 4;                             // rows in flight per thread
-
-thread_local char g_rope_error[256] = "";
 
 struct RopeParams {
   const __nv_bfloat16* x[2];  // q, k as given (the input of the prologue)
@@ -254,7 +253,7 @@ attn_status launch(bool backward, const RopeParams& p, int pairing, void* stream
   }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
-    std::snprintf(g_rope_error, sizeof(g_rope_error), "%s launch: %s",
+    std::snprintf(attn::g_cuda_error, attn::kErrorTextBytes, "%s launch: %s",
                   backward ? "qk_norm_rope_bwd_kernel" : "qk_norm_rope_kernel", cudaGetErrorString(e));
     return ATTN_ERR_CUDA;
   }
@@ -264,8 +263,6 @@ attn_status launch(bool backward, const RopeParams& p, int pairing, void* stream
 }  // namespace
 
 extern "C" {
-
-const char* attn_prologue_last_cuda_error(void) { return g_rope_error; }
 
 attn_status attn_qk_norm_rope(const void* q, const void* k, void* q_out, void* k_out, const int* pos_offsets, int B,
                               int T, int H, int H_kv, int D, float rope_base, float eps, int pairing, void* stream) {

@@ -47,7 +47,8 @@ typedef enum {
   ATTN_ERR_WORKSPACE = 6     /* backward workspace missing or smaller than attn_bwd_workspace_bytes() */
 } attn_status;
 
-/* Version of this ABI; bumped on any incompatible change of a signature or of a buffer layout. */
+/* Version of this ABI; bumped on any incompatible change of a signature or of a buffer layout
+ * (2: the prologue calls report CUDA errors through attn_last_cuda_error like every other call). */
 int attn_abi_version(void);
 
 /* Human-readable name of a status code (static storage; never NULL). */
@@ -191,8 +192,8 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
  *   pos_offsets in : device int32 [B] or NULL (decode: the cache length before the new tokens)
  *   rope_base finite and > 0 (usually 10000); eps finite and >= 0; D = 128 (else ATTN_ERR_UNSUPPORTED).
  *   With eps = 0 an all-zero row has no direction and its output is NaN (the formula's 0/0); eps > 0 maps it to 0.
- * One kernel launch over the rows of both tensors. On ATTN_ERR_CUDA, attn_prologue_last_cuda_error()
- * describes the failure.
+ * One kernel launch over the rows of both tensors. On ATTN_ERR_CUDA, attn_last_cuda_error() describes the
+ * failure.
  */
 typedef enum { ATTN_ROPE_INTERLEAVED = 0, ATTN_ROPE_HALF = 1 } attn_rope_pairing;
 
@@ -209,9 +210,6 @@ attn_status attn_qk_norm_rope(const void* q, const void* k, void* q_out, void* k
 attn_status attn_qk_norm_rope_bwd(const void* q, const void* k, const void* dq_out, const void* dk_out, void* dq,
                                   void* dk, const int* pos_offsets, int B, int T, int H, int H_kv, int D,
                                   float rope_base, float eps, int pairing, void* stream);
-
-/* Text of the last CUDA error seen by the two prologue calls above on the calling thread ("" if none). */
-const char* attn_prologue_last_cuda_error(void);
 
 /*
  * Device-side error word shared by the kernels of this library on the current device: 0 if no kernel has

@@ -44,7 +44,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_abi_version_and_status_strings(lib):
-    assert lib.attn_abi_version() == 1
+    assert lib.attn_abi_version() == 2
     for code, name in attn._STATUS.items():
         assert lib.attn_status_string(code).decode() == name
 
@@ -201,7 +201,7 @@ def test_no_cpu_fallback_without_gpu(lib):
     assert lib.attn_fwd_gqa(q, k, v, o, lse, 1, 2, 1, 128, 128, 0.088, None) == 4
     # the prologue: in place is well formed, and still fails loudly
     assert lib.attn_qk_norm_rope(q, k, q, k, None, 1, 128, 2, 2, 128, 10000.0, 1e-6, 0, None) == 4
-    assert lib.attn_prologue_last_cuda_error().decode() != ""
+    assert lib.attn_last_cuda_error().decode() != ""
     assert lib.attn_qk_norm_rope_bwd(q, k, o, lse, o, lse, None, 1, 128, 2, 2, 128, 10000.0, 1e-6, 1, None) == 4
 
 
