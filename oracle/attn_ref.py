@@ -167,7 +167,8 @@ def slice_forward_backward(q, k, v, do, b: int, h: int, scale: float, window: Op
     return out
 
 
-def decode_forward(q, k_cache, v_cache, cache_seqlens, scale: float) -> Tuple[np.ndarray, np.ndarray]:
+def decode_forward(q, k_cache, v_cache, cache_seqlens, scale: float,
+                   window: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
     """Attention of a few new queries against a key/value cache (the inference engine's
     flash_attn_with_kvcache over a prefilled cache: apidog "Train your own ChatGPT", section 6 "Inference
     engine").
@@ -175,8 +176,10 @@ def decode_forward(q, k_cache, v_cache, cache_seqlens, scale: float) -> Tuple[np
     q: [B, Tq, H, D]; k_cache, v_cache: [B, Tk, H_kv, D] (H_kv divides H, grouped as in ``attention_forward``);
     cache_seqlens: [B] integers, the number of valid cached keys of each sequence, the Tq new tokens' keys
     included (the caller has written them). Reading (the pages give no more): query i of sequence b sits at
-    position L_b - Tq + i and sees keys 0 .. L_b - Tq + i (causal, aligned to the end of the cache). A query that
-    sees no key (L_b - Tq + i < 0) returns O = 0 and LSE = -inf. Returns O [B, Tq, H, D], LSE [B, H, Tq].
+    position p = L_b - Tq + i and sees keys 0 .. p (causal, aligned to the end of the cache); with a sliding
+    window (the model's short-window layers, section 1 "GPT model", decoded through the same call) only keys
+    p - window .. p, the band of ``causal_mask``. A query that sees no key (p < 0) returns O = 0 and
+    LSE = -inf. Returns O [B, Tq, H, D], LSE [B, H, Tq].
     """
     q, kc, vc = _as_f64(q), _as_f64(k_cache), _as_f64(v_cache)
     B, Tq, H, D = q.shape
@@ -184,6 +187,8 @@ def decode_forward(q, k_cache, v_cache, cache_seqlens, scale: float) -> Tuple[np
     lens = np.asarray(cache_seqlens, dtype=np.int64).reshape(-1)
     if lens.shape[0] != B or (lens < 0).any() or (lens > kc.shape[1]).any():
         raise ValueError("cache_seqlens must hold B lengths in [0, Tk]")
+    if window is not None and window < 0:
+        raise ValueError("window must be >= 0 or None")
     O = np.zeros((B, Tq, H, D))
     LSE = np.full((B, H, Tq), -np.inf)
     for b in range(B):
@@ -191,13 +196,14 @@ def decode_forward(q, k_cache, v_cache, cache_seqlens, scale: float) -> Tuple[np
         for h in range(H):
             k, v = kc[b, :L, h // G], vc[b, :L, h // G]
             for i in range(Tq):
-                last = L - Tq + i                      # last visible key
+                last = L - Tq + i                      # last visible key: the query's own position
                 if last < 0:
                     continue
-                s = scale * (k[: last + 1] @ q[b, i, h])
+                first = 0 if window is None else max(0, last - window)
+                s = scale * (k[first: last + 1] @ q[b, i, h])
                 m = s.max()
                 e = np.exp(s - m)
-                O[b, i, h] = (e @ v[: last + 1]) / e.sum()
+                O[b, i, h] = (e @ v[first: last + 1]) / e.sum()
                 LSE[b, h, i] = m + np.log(e.sum())
     return O, LSE
 

@@ -433,7 +433,64 @@ def decode_pin_closed_forms(f):
     np.testing.assert_allclose(O2[1, 1, 0], vc[1, 0, 0], rtol=0, atol=1e-15)
 
 
-DECODE_PINS = [decode_pin_whole_sequence, decode_pin_torch, decode_pin_closed_forms]
+def decode_pin_window_torch(f):
+    """Sliding window in decode: ragged lengths, Tq = 3, grouped heads, windows below, at and above the
+    lengths: each sequence equals torch's float64 SDPA with the band p - W <= j <= p aligned to the end of
+    the cache, given as an explicit mask."""
+    B, Tq, H, Hkv, Tk, D = 3, 3, 4, 2, 40, 8
+    rng = np.random.default_rng(14)
+    q = rng.standard_normal((B, Tq, H, D))
+    kc, vc = rng.standard_normal((B, Tk, Hkv, D)), rng.standard_normal((B, Tk, Hkv, D))
+    lens = [40, 17, 4]
+    s = 0.4
+    for W in (0, 1, 5, 16, 100):
+        O, LSE = f(q, kc, vc, lens, s, window=W)
+        for b, L in enumerate(lens):
+            tq = torch.tensor(q[b:b + 1]).transpose(1, 2)
+            tk, tv = (torch.tensor(x[b:b + 1, :L]).transpose(1, 2) for x in (kc, vc))
+            pos = torch.arange(L - Tq, L)[:, None]
+            j = torch.arange(L)[None, :]
+            mask = (j <= pos) & (j >= pos - W)
+            ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=mask, scale=s,
+                                                                   enable_gqa=True)
+            got = O[b:b + 1]
+            valid = (pos[:, 0] >= 0).numpy()                # rows before the first key: O = 0 (SDPA gives NaN)
+            np.testing.assert_allclose(got[:, valid], ref.transpose(1, 2).numpy()[:, valid], rtol=1e-12,
+                                       atol=1e-12)
+            logits = s * (tq @ tk.repeat_interleave(H // Hkv, dim=1).transpose(-1, -2))   # [1, H, Tq, L]
+            lse_ref = torch.logsumexp(logits.masked_fill(~mask, -np.inf), dim=-1)[0].numpy()
+            np.testing.assert_allclose(LSE[b][:, valid], lse_ref[:, valid], rtol=1e-12, atol=1e-12)
+
+
+def decode_pin_window_limits(f):
+    """A window of L - 1 or more is no window; window 0 sees only the query's own key (O = V[p], LSE =
+    s q.k_p); Tq = L with a window is the windowed training forward."""
+    B, Tq, H, Tk, D = 2, 2, 2, 12, 4
+    rng = np.random.default_rng(15)
+    q = rng.standard_normal((B, Tq, H, D))
+    kc, vc = rng.standard_normal((B, Tk, H, D)), rng.standard_normal((B, Tk, H, D))
+    lens = [12, 7]
+    s = 0.7
+    O0, L0 = f(q, kc, vc, lens, s)
+    O1, L1 = f(q, kc, vc, lens, s, window=11)
+    np.testing.assert_array_equal(O0, O1)
+    np.testing.assert_array_equal(L0, L1)
+    Ow, Lw = f(q, kc, vc, lens, s, window=0)
+    for b, L in enumerate(lens):
+        for i in range(Tq):
+            p = L - Tq + i
+            np.testing.assert_allclose(Ow[b, i], vc[b, p], rtol=0, atol=1e-15)
+            np.testing.assert_allclose(Lw[b, :, i], s * np.einsum("hd,hd->h", q[b, i], kc[b, p]), rtol=1e-13)
+    T = 9
+    qq, kk, vv = (rng.standard_normal((1, T, H, D)) for _ in range(3))
+    Od, Ld = f(qq, kk, vv, [T], s, window=3)
+    Of, Lf = attn_ref.attention_forward(qq, kk, vv, s, window=3)
+    np.testing.assert_allclose(Od, Of, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(Ld, Lf, rtol=1e-13, atol=1e-13)
+
+
+DECODE_PINS = [decode_pin_whole_sequence, decode_pin_torch, decode_pin_closed_forms, decode_pin_window_torch,
+               decode_pin_window_limits]
 
 
 @pytest.mark.parametrize("pin", DECODE_PINS)
@@ -443,8 +500,10 @@ def test_decode_pins(pin):
 
 def _decode_mutant(kind):
     """A copy of the decode oracle with one plausible mistake planted."""
-    def f(q, k_cache, v_cache, cache_seqlens, scale):
+    def f(q, k_cache, v_cache, cache_seqlens, scale, window=None):
         q, kc, vc = (np.asarray(x, dtype=np.float64) for x in (q, k_cache, v_cache))
+        if kind == "window_ignored":
+            window = None
         B, Tq, H, D = q.shape
         Hkv = kc.shape[2]
         G = H // Hkv
@@ -458,16 +517,24 @@ def _decode_mutant(kind):
                     last = {"top_left_mask": i, "last_key_off_by_one": L - Tq + i - 1}.get(kind, L - Tq + i)
                     if last < 0:
                         continue
-                    sc = scale * (k[: last + 1] @ q[b, i, h])
+                    first = 0
+                    if window is not None:
+                        first = {"window_one_short": last - window + 1,
+                                 "window_from_query_index": i - window}.get(kind, last - window)
+                        first = max(0, first)
+                    if first > last:
+                        continue
+                    sc = scale * (k[first: last + 1] @ q[b, i, h])
                     m = sc.max()
                     e = np.exp(sc - m)
-                    O[b, i, h] = (e @ v[: last + 1]) / e.sum()
+                    O[b, i, h] = (e @ v[first: last + 1]) / e.sum()
                     LSE[b, h, i] = m + (np.log2(e.sum()) if kind == "lse_log2" else np.log(e.sum()))
         return O, LSE
     return f
 
 
-DECODE_MUTANTS = ["lengths_ignored", "kv_head_modulo", "top_left_mask", "last_key_off_by_one", "lse_log2"]
+DECODE_MUTANTS = ["lengths_ignored", "kv_head_modulo", "top_left_mask", "last_key_off_by_one", "lse_log2",
+                  "window_ignored", "window_one_short", "window_from_query_index"]
 
 
 def test_decode_mutant_control_passes():
