@@ -498,8 +498,10 @@ DECODE_METRIC = "KV-cache decode attention HBM GB/s (bf16 cache)"
 
 
 def decode_bytes(w, lens):
-    """Algorithmic bytes of one decode call: the valid K and V rows, q, o and lse."""
-    kv = sum(int(x) for x in lens) * w.Hkv * w.D * 2 * 2
+    """Algorithmic bytes of one decode call: the K and V rows some query sees (all valid rows, or with a sliding
+    window the last Tq + window of them), q, o and lse."""
+    seen = [int(x) if w.window < 0 else min(int(x), w.Tq + w.window) for x in lens]
+    kv = sum(seen) * w.Hkv * w.D * 2 * 2
     return kv + 2 * w.B * w.Tq * w.H * w.D * 2 + w.B * w.H * w.Tq * 4
 
 
@@ -522,7 +524,8 @@ def run_decode(args):
         with threadpool_limits(limits=len(os.sched_getaffinity(0))):
             for it in range(args.warmup + args.steps):
                 t0 = time.perf_counter()
-                attn_ref.decode_forward(q[:n], kc[:n], vc[:n], lens[:n].numpy(), w.scale)
+                attn_ref.decode_forward(q[:n], kc[:n], vc[:n], lens[:n].numpy(), w.scale,
+                                        window=w.window if w.window >= 0 else None)
                 if it >= args.warmup:
                     times.append(time.perf_counter() - t0)
         sw = dataclasses.replace(w, B=n)
@@ -554,8 +557,9 @@ def run_decode(args):
     sh = torch.cuda.current_stream(device).cuda_stream
 
     def call():
-        st = lib.attn_decode(q.data_ptr(), kc.data_ptr(), vc.data_ptr(), lens.data_ptr(), o.data_ptr(),
-                             lse.data_ptr(), ws.data_ptr(), ws_bytes, w.B, w.H, w.Hkv, w.Tq, w.Tk, w.D, w.scale, sh)
+        st = lib.attn_decode_ex(q.data_ptr(), kc.data_ptr(), vc.data_ptr(), lens.data_ptr(), o.data_ptr(),
+                                lse.data_ptr(), ws.data_ptr(), ws_bytes, w.B, w.H, w.Hkv, w.Tq, w.Tk, w.D, w.scale,
+                                w.window, sh)
         if st != 0:
             raise RuntimeError(f"attn_decode: {attn._STATUS.get(st, st)}")
 
@@ -596,7 +600,7 @@ def run_decode(args):
         "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "ours",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.Hkv, "Tq": w.Tq, "Tk": w.Tk, "D": w.D,
-                   "recipe": w.recipe, "l2": "256 MB written between calls",
+                   "window": w.window, "recipe": w.recipe, "l2": "256 MB written between calls",
                    "parallelism": f"replicas x{world} (no collective on the data path)"},
         "roofline": {"kernel": "attn_decode (split + combine)", "bound": "hbm", "achieved": gbs, "peak": hbm,
                      "unit": "GB/s", "frac": gbs / hbm, "traffic": None, "alg_bytes": nbytes},

@@ -44,6 +44,7 @@ SIGNATURES = {
     "attn_bwd_ex": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _I, _F, _I, _VP], _I),
     "attn_decode_workspace_bytes": ([_I] * 6, _SZ),
     "attn_decode": ([_VP] * 7 + [_SZ] + [_I] * 6 + [_F, _VP], _I),
+    "attn_decode_ex": ([_VP] * 7 + [_SZ] + [_I] * 6 + [_F, _I, _VP], _I),
     "attn_qk_norm_rope": ([_VP] * 5 + [_I] * 5 + [_F, _F, _I, _VP], _I),
     "attn_qk_norm_rope_bwd": ([_VP] * 7 + [_I] * 5 + [_F, _F, _I, _VP], _I),
     "attn_get_device_error": ([ctypes.POINTER(ctypes.c_uint32)], _I),
@@ -279,11 +280,12 @@ def attn_bwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch
 
 def attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, cache_seqlens: torch.Tensor,
                 scale: Optional[float] = None, o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+                workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+                window: Optional[int] = None):
     """Attention of Tq new queries against a key/value cache (the inference engine's cached decode).
     q: bf16 [B, Tq, H, D]; k_cache, v_cache: bf16 [B, Tk, H_kv, D]; cache_seqlens: int32 [B] on the device, the
-    valid keys of each sequence (new tokens included). Query i sees keys 0 .. L - Tq + i. Returns
-    (o [B, Tq, H, D], lse [B, H, Tq])."""
+    valid keys of each sequence (new tokens included). Query i, at position p = L - Tq + i, sees keys 0 .. p, or
+    with a sliding window keys p - window .. p. Returns (o [B, Tq, H, D], lse [B, H, Tq])."""
     lib = load_library()
     _require_cuda("q", q)
     _check_qkv("q", q)
@@ -308,12 +310,13 @@ def attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, c
     elif workspace.device != dev:
         raise ValueError(f"workspace is on {workspace.device}; every tensor of one call must be on {dev}")
     scale = default_scale(D) if scale is None else float(scale)
+    win = _window_arg(window)
     with torch.cuda.device(dev):
-        st = lib.attn_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cache_seqlens.data_ptr(),
-                             o.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
-                             workspace.numel() * workspace.element_size(), B, H, Hkv, Tq, Tk, D, scale,
-                             _stream_handle(stream, dev))
-    _check("attn_decode", st)
+        st = lib.attn_decode_ex(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), cache_seqlens.data_ptr(),
+                                o.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size(), B, H, Hkv, Tq, Tk, D, scale, win,
+                                _stream_handle(stream, dev))
+    _check("attn_decode_ex", st)
     return o, lse
 
 

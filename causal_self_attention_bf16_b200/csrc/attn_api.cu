@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -535,9 +536,14 @@ attn_status check_decode(int B, int H, int Hkv, int Tq, int Tk, int D, float sca
   return ATTN_OK;
 }
 
+// Keys a sequence's rows can see: the whole cache, or with a sliding window the Tq + window before its end.
+int decode_span(int Tq, int Tk, int window) {
+  return window < 0 ? Tk : static_cast<int>(std::min<long long>(Tk, static_cast<long long>(Tq) + window));
+}
+
 size_t decode_workspace(int B, int H, int Hkv, int Tq, int Tk) {
   int n_split = 1, chunk = 0;
-  decode_split(B, Hkv, Tk, &n_split, &chunk);
+  decode_split(B, Hkv, Tk, &n_split, &chunk);  // no window: the most chunks, enough for any window
   const size_t rows = static_cast<size_t>(B) * Hkv * n_split * ((H / Hkv) * Tq);
   return rows * 128 * 4 + rows * 2 * 4;
 }
@@ -551,12 +557,13 @@ size_t attn_decode_workspace_bytes(int B, int H, int H_kv, int Tq, int Tk, int D
   return decode_workspace(B, H, H_kv, Tq, Tk);
 }
 
-attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* cache_seqlens, void* o,
-                        float* lse, void* workspace, size_t workspace_bytes, int B, int H, int H_kv, int Tq, int Tk,
-                        int D, float scale, void* stream) {
+attn_status attn_decode_ex(const void* q, const void* k_cache, const void* v_cache, const int* cache_seqlens,
+                           void* o, float* lse, void* workspace, size_t workspace_bytes, int B, int H, int H_kv,
+                           int Tq, int Tk, int D, float scale, int window, void* stream) {
   if (!q || !k_cache || !v_cache || !cache_seqlens || !o || !lse) return ATTN_ERR_INVALID_ARG;
   attn_status st = check_decode(B, H, H_kv, Tq, Tk, D, scale);
   if (st != ATTN_OK) return st;
+  if (window < -1) return ATTN_ERR_INVALID_ARG;
   const size_t need = decode_workspace(B, H, H_kv, Tq, Tk);
   if (!workspace || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
   for (const void* ptr : {q, k_cache, v_cache, static_cast<const void*>(o), static_cast<const void*>(workspace)})
@@ -589,7 +596,8 @@ attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
   p.Tq = Tq;
   p.Tk = Tk;
   p.R = (H / H_kv) * Tq;
-  decode_split(B, H_kv, Tk, &p.n_split, &p.chunk);
+  p.window = window;
+  decode_split(B, H_kv, decode_span(Tq, Tk, window), &p.n_split, &p.chunk);
   const size_t rows = static_cast<size_t>(B) * H_kv * p.n_split * p.R;
   p.part_o = static_cast<float*>(workspace);
   p.part_ml = static_cast<float*>(workspace) + rows * 128;
@@ -616,6 +624,13 @@ attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
   attn::attn_decode_combine_kernel<<<static_cast<unsigned>((out_rows + 7) / 8), 256, 0, s>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_decode_combine_kernel launch");
   return ATTN_OK;
+}
+
+attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* cache_seqlens, void* o,
+                        float* lse, void* workspace, size_t workspace_bytes, int B, int H, int H_kv, int Tq, int Tk,
+                        int D, float scale, void* stream) {
+  return attn_decode_ex(q, k_cache, v_cache, cache_seqlens, o, lse, workspace, workspace_bytes, B, H, H_kv, Tq, Tk, D,
+                        scale, -1, stream);
 }
 
 }  // extern "C"

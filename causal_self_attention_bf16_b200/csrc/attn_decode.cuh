@@ -3,9 +3,9 @@
 // prompt cache).
 //
 //   q [B, Tq, H, D] bf16; k_cache, v_cache [B, Tk, H_kv, D] bf16; cache_seqlens [B] int32 (valid keys per
-//   sequence, the new tokens' keys included). Query i of sequence b sits at position L_b - Tq + i and sees keys
-//   0 .. L_b - Tq + i. Out: o [B, Tq, H, D] bf16, lse [B, H, Tq] fp32 (natural log; -inf and o = 0 for a query
-//   that sees no key).
+//   sequence, the new tokens' keys included). Query i of sequence b sits at position p = L_b - Tq + i and sees
+//   keys 0 .. p, or with a sliding window keys p - window .. p. Out: o [B, Tq, H, D] bf16, lse [B, H, Tq] fp32
+//   (natural log; -inf and o = 0 for a query that sees no key).
 //
 // The work is a stream over the cache, HBM-bound (a few FLOPs per byte of K/V), so it runs on CUDA cores:
 //   1. attn_decode_split_kernel: one CTA per (sequence, key/value head, chunk of the cache). The G = H / H_kv
@@ -39,6 +39,7 @@ struct DecodeParams {
   float* part_o;               // [B * H_kv, n_split, R, D] fp32, unnormalised
   float* part_ml;              // [B * H_kv, n_split, R, 2]: running max (log2 units) and sum
   int B, H, Hkv, Tq, Tk, R, n_split, chunk;
+  int window;                  // sliding window: query at position p sees keys p - window .. p; -1: none
   float scale_log2;            // scale * log2(e)
 };
 
@@ -62,7 +63,10 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const De
   const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
   const int G = p.H / p.Hkv, R = p.R;
   const int L = min(max(p.seqlens[b], 0), p.Tk);   // lengths outside [0, Tk] are clamped
-  const int key_lo = sp * p.chunk, key_hi = min(L, key_lo + p.chunk);
+  // The chunks split the keys any row of this sequence sees: from the first row's window start (0 without a
+  // window) to the end of the cache.
+  const int start = p.window < 0 ? 0 : max(0, L - p.Tq - p.window);
+  const int key_lo = start + sp * p.chunk, key_hi = min(L, key_lo + p.chunk);
   const size_t row_stride = static_cast<size_t>(p.Hkv) * 128;   // elements between consecutive keys
 
   // Row r = g * Tq + i: query head hk * G + g, new token i, which sees keys up to L - Tq + i.
@@ -112,8 +116,9 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const De
         s0 = fmaf(qb.z, __uint_as_float(w[3] << 16), s0);
         s1 = fmaf(qb.w, __uint_as_float(w[3] & 0xffff0000u), s1);
       }
-      const int last = L - p.Tq + r % p.Tq;  // last key this row sees
-      sc[r][t] = (t < nk && kb + t <= last) ? s0 + s1 : -INFINITY;
+      const int last = L - p.Tq + r % p.Tq;  // last key this row sees (its own position)
+      const bool seen = t < nk && kb + t <= last && (p.window < 0 || kb + t >= last - p.window);
+      sc[r][t] = seen ? s0 + s1 : -INFINITY;
     }
     // The V block to shared memory (rows past the block are zeros, so P = 0 times them stays 0).
 #pragma unroll

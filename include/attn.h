@@ -158,6 +158,19 @@ attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache,
                         int D, float scale, void* stream);
 
 /*
+ * attn_decode with a sliding window, for the model's short-window layers (apidog "Train your own ChatGPT",
+ * section 1 "GPT model": layers alternate short and long windows, "SSSL"; section 6 "Inference engine": the
+ * engine decodes every layer through the same cached call). With window >= 0 the query at position
+ * p = L_b - Tq + i sees keys p - window .. p only, the band of attn_fwd_ex aligned to the end of the cache;
+ * window = -1 is attn_decode. Chunks of the cache wholly outside every row's band are not read. The
+ * workspace is attn_decode_workspace_bytes(B, H, H_kv, Tq, Tk, D) bytes, enough for any window.
+ * window < -1: ATTN_ERR_INVALID_ARG. Otherwise the contract of attn_decode.
+ */
+attn_status attn_decode_ex(const void* q, const void* k_cache, const void* v_cache, const int* cache_seqlens,
+                           void* o, float* lse, void* workspace, size_t workspace_bytes, int B, int H, int H_kv,
+                           int Tq, int Tk, int D, float scale, int window, void* stream);
+
+/*
  * Backward without caller-provided workspace, for callers that cannot allocate device memory (a custom-op or
  * plugin interface that passes tensors but no allocator or workspace; a fixed memory plan that forbids
  * cudaMalloc/cudaFree, and the synchronisation they can cause, during a step). The pages have no counterpart:

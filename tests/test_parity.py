@@ -235,6 +235,45 @@ def test_decode_full(name, shape):
     assert np.all(to64(o)[np.broadcast_to(~finite.transpose(0, 2, 1)[..., None], O_ref.shape)] == 0)
 
 
+DECODE_WINDOWS = [0, 1, 100, 127, 128, 129, 300, 5000]
+
+
+@pytest.mark.parametrize("window", DECODE_WINDOWS)
+def test_decode_window_full(window):
+    """Sliding window in cached decode: ragged lengths, grouped heads, Tq = 3, windows below, at and above a
+    128-key block and beyond the cache; every output against the oracle's end-aligned band."""
+    from workloads import DecodeWorkload, make_decode_inputs
+    w = DecodeWorkload("decode_sw", B=3, H=8, Hkv=2, Tq=3, Tk=1300, seed=41 + window)
+    q, kc, vc, lens = make_decode_inputs(w)
+    dev = torch.device("cuda")
+    o, lse = attn.attn_decode(q.to(dev), kc.to(dev), vc.to(dev), lens.to(dev), w.scale, window=window)
+    torch.cuda.synchronize()
+    O_ref, LSE_ref = attn_ref.decode_forward(q, kc, vc, lens.numpy(), w.scale, window=window)
+    what = f"decode window={window} lens={lens.tolist()}"
+    check_o(to64(o), O_ref, what)
+    finite = np.isfinite(LSE_ref)
+    assert np.array_equal(np.isfinite(to64(lse)), finite), f"{what}: -inf LSE pattern differs"
+    check_lse(to64(lse)[finite], LSE_ref[finite], what)
+
+
+def test_decode_window_long_cache_single_token():
+    """One new token per sequence against 9000 cached keys with a 1000-key window: the chunks cover only the
+    band, and window >= the cache length equals no window bit for bit."""
+    from workloads import DecodeWorkload, make_decode_inputs
+    w = DecodeWorkload("decode_sw_long", B=2, H=4, Hkv=1, Tq=1, Tk=9000, seed=77)
+    q, kc, vc, lens = make_decode_inputs(w)
+    dev = torch.device("cuda")
+    args = (q.to(dev), kc.to(dev), vc.to(dev), lens.to(dev), w.scale)
+    o, lse = attn.attn_decode(*args, window=1000)
+    torch.cuda.synchronize()
+    O_ref, LSE_ref = attn_ref.decode_forward(q, kc, vc, lens.numpy(), w.scale, window=1000)
+    check_o(to64(o), O_ref, "decode window=1000 Tk=9000")
+    check_lse(to64(lse), LSE_ref, "decode window=1000 Tk=9000")
+    o_all, lse_all = attn.attn_decode(*args)
+    o_big, lse_big = attn.attn_decode(*args, window=9000)
+    assert torch.equal(o_all, o_big) and torch.equal(lse_all, lse_big)
+
+
 def test_decode_full_size_sampled():
     """The benchmark's decode workload (64 sequences, d20 heads, ragged lengths up to 2048), oracle on samples."""
     from workloads import DECODE_WORKLOADS, make_decode_inputs

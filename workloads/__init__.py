@@ -169,6 +169,7 @@ class DecodeWorkload:
     D: int = HEAD_DIM
     min_len: int = 1
     seed: int = 0
+    window: int = -1             # sliding window (the model's short-window layers); -1: none
     recipe: str = ""
 
     @property
@@ -184,6 +185,8 @@ DECODE_WORKLOADS: Dict[str, DecodeWorkload] = {
                                         "uniform in [1, 2048]; q, caches ~ N(0,1) bf16"),
     "decode_d20_gqa": DecodeWorkload("decode_d20_gqa", B=64, H=10, Hkv=5, Tq=1, Tk=2048, seed=3,
                                      recipe="decode_d20 with 5 key/value heads"),
+    "decode_d20_sw": DecodeWorkload("decode_d20_sw", B=64, H=10, Hkv=10, Tq=1, Tk=2048, seed=2, window=512,
+                                    recipe="decode_d20 through a short-window layer: window 512"),
 }
 
 
