@@ -492,95 +492,99 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const int s = gs % kBwdStages, rb = g;
         const int q0 = (it.i0 + i % it.n) * kBwdQTile;
         float* acc_bh = p.dq_acc + static_cast<size_t>(it.b * p.H + it.hk * G + i / it.n) * p.Tp * 128;  // step's query head
-        if (!mbar_wait_warp(&bars.q_full[s], (gs / kBwdStages) & 1, abort, lim, &g_device_error, kSiteBwdSmQ) ||
-            !mbar_wait_warp(&bars.s_full[rb], (gs >> 1) & 1, abort, lim, &g_device_error, kSiteBwdSmS)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (threadIdx.x == 64 || threadIdx.x == 192) ATTN_TRACE_EVENT(4, gs);
-        const bool diag = q0 < k0 + kBwdKTile;  // tile overlaps the key tile: queries before a key see nothing
-        // sliding window: queries after key + window see nothing (only tiles reaching past k0 + window have any)
-        const bool band = p.window >= 0 && q0 + kBwdQTile - 1 > k0 + p.window;
-        uint8_t* dsrow = smem + kBwdSmemDS + rb * 16384;
-        // The half-tile body is instantiated twice: with the sliding-window mask (tiles that reach past a key's
-        // window) and without it, so unwindowed tiles carry no per-element window test.
-        auto halves = [&](auto band_flag) {
-          constexpr bool kBand = decltype(band_flag)::value;
+        bool step_ok =
+            mbar_wait_warp(&bars.q_full[s], (gs / kBwdStages) & 1, abort, lim, &g_device_error, kSiteBwdSmQ) &&
+            mbar_wait_warp(&bars.s_full[rb], (gs >> 1) & 1, abort, lim, &g_device_error, kSiteBwdSmS);
+        if (step_ok) {
+          tc_fence_after();
+          if (threadIdx.x == 64 || threadIdx.x == 192) ATTN_TRACE_EVENT(4, gs);
+          const bool diag = q0 < k0 + kBwdKTile;  // tile overlaps the key tile: queries before a key see nothing
+          // sliding window: queries after key + window see nothing (only tiles reaching past k0 + window have any)
+          const bool band = p.window >= 0 && q0 + kBwdQTile - 1 > k0 + p.window;
+          uint8_t* dsrow = smem + kBwdSmemDS + rb * 16384;
+          // The half-tile body is instantiated twice: with the sliding-window mask (tiles that reach past a key's
+          // window) and without it, so unwindowed tiles carry no per-element window test.
+          auto halves = [&](auto band_flag) {
+            constexpr bool kBand = decltype(band_flag)::value;
 #pragma unroll 1
-          for (int hh = 0; hh < 2; ++hh) {  // one half at a time keeps the live registers to one half's worth
-            const uint32_t r = tmem + lane_base + kTmemR + rb * 128 + 32 * hh;
-            const float4* lse4 = reinterpret_cast<const float4*>(smem + kBwdSmemLse + s * 256) + 8 * hh;
-            const float4* dlt4 = reinterpret_cast<const float4*>(smem + kBwdSmemDelta + s * 256) + 8 * hh;
-            uint32_t sv[32], dp[32];
-            tmem_ld32(r, sv);        // S^T of queries [32hh, 32hh+32)
-            tmem_ld32(r + 64, dp);   // dP^T of the same queries
-            tmem_wait_ld();
-            uint32_t ppk[16], dpk[16];
+            for (int hh = 0; hh < 2; ++hh) {  // one half at a time keeps the live registers to one half's worth
+              const uint32_t r = tmem + lane_base + kTmemR + rb * 128 + 32 * hh;
+              const float4* lse4 = reinterpret_cast<const float4*>(smem + kBwdSmemLse + s * 256) + 8 * hh;
+              const float4* dlt4 = reinterpret_cast<const float4*>(smem + kBwdSmemDelta + s * 256) + 8 * hh;
+              uint32_t sv[32], dp[32];
+              tmem_ld32(r, sv);        // S^T of queries [32hh, 32hh+32)
+              tmem_ld32(r + 64, dp);   // dP^T of the same queries
+              tmem_wait_ld();
+              uint32_t ppk[16], dpk[16];
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4) {
-              const float4 l4 = lse4[q4], d4 = dlt4[q4];
-              const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-              float pv[4], dsv[4];
+              for (int q4 = 0; q4 < 8; ++q4) {
+                const float4 l4 = lse4[q4], d4 = dlt4[q4];
+                const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+                float pv[4], dsv[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int q = q4 * 4 + e;
-                float pe = ex2(fmaf(__uint_as_float(sv[q]), c, -lv[e]));
-                if (diag && q0 + 32 * hh + q < kg) pe = 0.f;
-                if (kBand && q0 + 32 * hh + q > kg + p.window) pe = 0.f;
-                pv[e] = pe;
-                dsv[e] = pe * (__uint_as_float(dp[q]) - dv4[e]);
+                for (int e = 0; e < 4; ++e) {
+                  const int q = q4 * 4 + e;
+                  float pe = ex2(fmaf(__uint_as_float(sv[q]), c, -lv[e]));
+                  if (diag && q0 + 32 * hh + q < kg) pe = 0.f;
+                  if (kBand && q0 + 32 * hh + q > kg + p.window) pe = 0.f;
+                  pv[e] = pe;
+                  dsv[e] = pe * (__uint_as_float(dp[q]) - dv4[e]);
+                }
+                ppk[q4 * 2] = pack_bf16x2(pv[0], pv[1]);
+                ppk[q4 * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+                dpk[q4 * 2] = pack_bf16x2(dsv[0], dsv[1]);
+                dpk[q4 * 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
               }
-              ppk[q4 * 2] = pack_bf16x2(pv[0], pv[1]);
-              ppk[q4 * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-              dpk[q4 * 2] = pack_bf16x2(dsv[0], dsv[1]);
-              dpk[q4 * 2 + 1] = pack_bf16x2(dsv[2], dsv[3]);
-            }
-            tmem_st16(r, ppk);        // P^T  of these 32 queries: columns [32hh, 32hh+16)
-            tmem_st16(r + 16, dpk);   // dS^T of these 32 queries: columns [32hh+16, 32hh+32)
+              tmem_st16(r, ppk);        // P^T  of these 32 queries: columns [32hh, 32hh+16)
+              tmem_st16(r + 16, dpk);   // dS^T of these 32 queries: columns [32hh+16, 32hh+32)
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-              uint4 v = make_uint4(dpk[ch * 4 + 0], dpk[ch * 4 + 1], dpk[ch * 4 + 2], dpk[ch * 4 + 3]);
-              *reinterpret_cast<uint4*>(dsrow + sw128_offset(krow, 4 * hh + ch)) = v;
+              for (int ch = 0; ch < 4; ++ch) {
+                uint4 v = make_uint4(dpk[ch * 4 + 0], dpk[ch * 4 + 1], dpk[ch * 4 + 2], dpk[ch * 4 + 3]);
+                *reinterpret_cast<uint4*>(dsrow + sw128_offset(krow, 4 * hh + ch)) = v;
+              }
             }
-          }
-        };
-        if (band) halves(std::true_type{});
-        else halves(std::false_type{});
-        tmem_wait_st();
-        fence_async_shared();
-        tc_fence_before();
-        mbar_arrive_warp(&bars.p_full[rb]);
-        if (threadIdx.x == 64 || threadIdx.x == 192) ATTN_TRACE_EVENT(5, gs);
+          };
+          if (band) halves(std::true_type{});
+          else halves(std::false_type{});
+          tmem_wait_st();
+          fence_async_shared();
+          tc_fence_before();
+          mbar_arrive_warp(&bars.p_full[rb]);
+          if (threadIdx.x == 64 || threadIdx.x == 192) ATTN_TRACE_EVENT(5, gs);
+        }
 
         // dQ^T of this step (thread = d, 64 query columns) -> staging buffer in the accumulator's [q/4][d][4]
         // layout, where the tile is one contiguous 32 KB block -> one bulk reduce-add on the async engine. The
         // staging buffer passes between the two groups in step order through stage_free.
-        if (!mbar_wait_warp(&bars.dq_full[rb], (gs >> 1) & 1, abort, lim, &g_device_error, kSiteBwdDq)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (threadIdx.x == 64) ATTN_TRACE_EVENT(6, gs);
+        step_ok = step_ok && mbar_wait_warp(&bars.dq_full[rb], (gs >> 1) & 1, abort, lim, &g_device_error, kSiteBwdDq);
         uint32_t a[2][32];
-        tmem_ld32(tmem + lane_base + kTmemR + rb * 128 + 64, a[0]);
-        tmem_ld32(tmem + lane_base + kTmemR + rb * 128 + 96, a[1]);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive_warp(&bars.dq_empty[rb]);  // dQ^T is in registers: the tensor-memory columns are free
-        if (gs > 0 && !wait_staged(gs - 1)) {
+        if (step_ok) {
+          tc_fence_after();
+          if (threadIdx.x == 64) ATTN_TRACE_EVENT(6, gs);
+          tmem_ld32(tmem + lane_base + kTmemR + rb * 128 + 64, a[0]);
+          tmem_ld32(tmem + lane_base + kTmemR + rb * 128 + 96, a[1]);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive_warp(&bars.dq_empty[rb]);  // dQ^T is in registers: the tensor-memory columns are free
+        }
+        step_ok = step_ok && (gs == 0 || wait_staged(gs - 1));
+        if (step_ok) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+              *reinterpret_cast<float4*>(dq_stage + ((8 * hh + q4) * 128 + krow) * 4) =
+                  make_float4(__uint_as_float(a[hh][4 * q4]), __uint_as_float(a[hh][4 * q4 + 1]),
+                              __uint_as_float(a[hh][4 * q4 + 2]), __uint_as_float(a[hh][4 * q4 + 3]));
+          fence_async_shared();
+        }
+        // Every warp of the group reaches this barrier, failed or not, and the group leaves the walk together
+        // on the AND of the warps' states (a warp leaving alone would meet its siblings at a later barrier of
+        // the same id and desynchronise the group).
+        if (!named_barrier_and(2 + g, 128, step_ok)) {
           ok = false;
           break;
         }
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4)
-            *reinterpret_cast<float4*>(dq_stage + ((8 * hh + q4) * 128 + krow) * 4) =
-                make_float4(__uint_as_float(a[hh][4 * q4]), __uint_as_float(a[hh][4 * q4 + 1]),
-                            __uint_as_float(a[hh][4 * q4 + 2]), __uint_as_float(a[hh][4 * q4 + 3]));
-        fence_async_shared();
-        named_barrier(2 + g, 128);
         if (group_leader) {
           bulk_reduce_add_f32(acc_bh + static_cast<size_t>(q0 >> 2) * 512, dq_stage, 32768);
           tma_store_commit();
