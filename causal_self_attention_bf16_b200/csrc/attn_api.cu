@@ -356,8 +356,8 @@ attn_status bwd_launch(unsigned stages, const void* q, const void* k, const void
 
   cudaError_t e;
   if (stages & 1u) {
-    const size_t rows = static_cast<size_t>(B) * H * p.Tp;
-    attn::attn_bwd_prep_kernel<<<grid_for(rows * 16, 256), 256, 0, s>>>(p);
+    const size_t quads = static_cast<size_t>(B) * H * p.Tp / 4;  // a 16-thread group per four padded rows
+    attn::attn_bwd_prep_kernel<<<grid_for(quads * 16, 256), 256, 0, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_bwd_prep_kernel launch");
   }
   if (stages & 2u) {

@@ -72,72 +72,108 @@ struct BwdParams {
 
 // ------------------------------------------------------------------------------------------------ prep
 
-// One 16-thread group per (b, t, h) row: Delta = sum_d dO * O in fp32; LSE * log2(e); zero the accumulator.
+// One 16-thread group per (bh, four consecutive padded rows): Delta = sum_d dO * O in fp32 and LSE * log2(e)
+// for the four rows, and zeroing of the accumulator block that holds them (2 KB, contiguous in the [t/4][d][4]
+// layout). Each thread has its eight 16-byte loads (four rows of o and dO) in flight at once, and every group
+// writes as many bytes as it reads, so the read and write streams interleave over the whole grid.
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const BwdParams p) {
-  const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.Tp;  // padded rows, ordered (bh, t)
+  const int64_t quads = static_cast<int64_t>(p.B) * p.H * (p.Tp / 4);  // ordered (bh, t/4)
   const int sub = threadIdx.x & 15;
   const int64_t group = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
   const int64_t ngroups = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
-  for (int64_t r = group; r < rows; r += ngroups) {
-    const int bh = static_cast<int>(r / p.Tp), t = static_cast<int>(r % p.Tp);
+  for (int64_t qd = group; qd < quads; qd += ngroups) {
+    const int bh = static_cast<int>(qd / (p.Tp / 4)), t0 = static_cast<int>(qd % (p.Tp / 4)) * 4;
     const int b = bh / p.H, h = bh % p.H;
-    float acc = 0.f;
-    if (t < p.T) {
-      const size_t off = ((static_cast<size_t>(b) * p.T + t) * p.H + h) * 128 + sub * 8;
-      const uint4 ov = *reinterpret_cast<const uint4*>(p.o + off);
-      const uint4 gv = *reinterpret_cast<const uint4*>(p.dO + off);
-      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
-      const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv);
+    uint4 ov[4], gv[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      ov[j] = make_uint4(0u, 0u, 0u, 0u);
+      gv[j] = make_uint4(0u, 0u, 0u, 0u);
+      if (t0 + j < p.T) {
+        const size_t off = ((static_cast<size_t>(b) * p.T + t0 + j) * p.H + h) * 128 + sub * 8;
+        ov[j] = *reinterpret_cast<const uint4*>(p.o + off);
+        gv[j] = *reinterpret_cast<const uint4*>(p.dO + off);
+      }
+    }
+    // zero the block of these four rows: 512 floats, 8 float4 per thread
+    float4* blk = reinterpret_cast<float4*>(p.dq_acc + static_cast<size_t>(bh) * p.Tp * 128 +
+                                            static_cast<size_t>(t0) * 128);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) blk[j * 16 + sub] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float acc[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov[j]);
+      const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv[j]);
+      acc[j] = 0.f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2 of = __bfloat1622float2(o2[i]);
         const float2 gf = __bfloat1622float2(g2[i]);
-        acc = fmaf(of.x, gf.x, acc);
-        acc = fmaf(of.y, gf.y, acc);
+        acc[j] = fmaf(of.x, gf.x, acc[j]);
+        acc[j] = fmaf(of.y, gf.y, acc[j]);
       }
     }
 #pragma unroll
-    for (int w = 8; w >= 1; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w, 16);
-    if (sub == 0) {
-      p.delta[r] = acc;
+    for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], w, 16);
+    if (sub < 4) {  // thread j of the group writes row t0 + j
+      const int t = t0 + sub;
+      const float a = sub == 0 ? acc[0] : sub == 1 ? acc[1] : sub == 2 ? acc[2] : acc[3];
+      const int64_t r = static_cast<int64_t>(bh) * p.Tp + t;
+      p.delta[r] = a;
       p.lse2[r] = t < p.T ? p.lse[static_cast<size_t>(bh) * p.T + t] * 1.4426950408889634f : INFINITY;
     }
   }
-  // Zero the dQ accumulator with 16-byte stores.
-  const int64_t n4 = static_cast<int64_t>(p.B) * p.H * p.Tp * 128 / 4;
-  float4* acc4 = reinterpret_cast<float4*>(p.dq_acc);
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // ------------------------------------------------------------------------------------------------ dQ out
 
-// dq[b, t, h, d] = bf16(scale * acc[bh, t/4, d, t%4]). One thread per (bh, t/4, 4 consecutive d).
+// dq[b, t, h, d] = bf16(scale * acc[bh, t/4, d, t%4]). One thread per (bh, t/4, 4 consecutive d): 64
+// contiguous accumulator bytes in, 8 bytes of four rows out (a warp writes whole 256-byte rows). Each thread
+// takes two items per pass of the grid-stride loop and issues both items' loads before either's stores.
 __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const BwdParams p) {
   const int64_t t4n = (p.T + 3) / 4;
   const int64_t items = static_cast<int64_t>(p.B) * p.H * t4n * 32;
-  for (int64_t it = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it < items;
-       it += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int dc = static_cast<int>(it & 31);         // d chunk: d = 4*dc .. 4*dc+3
-    const int64_t rest = it >> 5;
-    const int t4 = static_cast<int>(rest % t4n);
-    const int bh = static_cast<int>(rest / t4n);
-    const int b = bh / p.H, h = bh % p.H;
-    const float4* src = reinterpret_cast<const float4*>(p.dq_acc + static_cast<size_t>(bh) * p.Tp * 128 +
-                                                        static_cast<size_t>(t4) * 512 + dc * 16);
-    const float4 a0 = src[0], a1 = src[1], a2 = src[2], a3 = src[3];  // d = 4dc+0..3, each holding t%4 = 0..3
-    const float s = p.scale;
-    const float v[4][4] = {{a0.x, a1.x, a2.x, a3.x}, {a0.y, a1.y, a2.y, a3.y}, {a0.z, a1.z, a2.z, a3.z},
-                           {a0.w, a1.w, a2.w, a3.w}};
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t it0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it0 < items; it0 += 2 * stride) {
+    float4 a[2][4];
 #pragma unroll
-    for (int tt = 0; tt < 4; ++tt) {
-      const int t = t4 * 4 + tt;
-      if (t < p.T) {
-        uint2 w;
-        w.x = sm100::pack_bf16x2(v[tt][0] * s, v[tt][1] * s);
-        w.y = sm100::pack_bf16x2(v[tt][2] * s, v[tt][3] * s);
-        *reinterpret_cast<uint2*>(p.dq + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * 128 + dc * 4) = w;
+    for (int u = 0; u < 2; ++u) {
+      const int64_t it = it0 + u * stride;
+      if (it < items) {
+        const int dc = static_cast<int>(it & 31);  // d chunk: d = 4*dc .. 4*dc+3
+        const int64_t rest = it >> 5;
+        const int t4 = static_cast<int>(rest % t4n);
+        const int bh = static_cast<int>(rest / t4n);
+        const float4* src = reinterpret_cast<const float4*>(p.dq_acc + static_cast<size_t>(bh) * p.Tp * 128 +
+                                                            static_cast<size_t>(t4) * 512 + dc * 16);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) a[u][c] = src[c];  // d = 4dc + c, holding t%4 = 0..3
+      }
+    }
+    const float s = p.scale;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int64_t it = it0 + u * stride;
+      if (it >= items) break;
+      const int dc = static_cast<int>(it & 31);
+      const int64_t rest = it >> 5;
+      const int t4 = static_cast<int>(rest % t4n);
+      const int bh = static_cast<int>(rest / t4n);
+      const int b = bh / p.H, h = bh % p.H;
+      const float v[4][4] = {{a[u][0].x, a[u][1].x, a[u][2].x, a[u][3].x}, {a[u][0].y, a[u][1].y, a[u][2].y, a[u][3].y},
+                             {a[u][0].z, a[u][1].z, a[u][2].z, a[u][3].z}, {a[u][0].w, a[u][1].w, a[u][2].w, a[u][3].w}};
+#pragma unroll
+      for (int tt = 0; tt < 4; ++tt) {
+        const int t = t4 * 4 + tt;
+        if (t < p.T) {
+          uint2 w;
+          w.x = sm100::pack_bf16x2(v[tt][0] * s, v[tt][1] * s);
+          w.y = sm100::pack_bf16x2(v[tt][2] * s, v[tt][3] * s);
+          *reinterpret_cast<uint2*>(p.dq + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * 128 + dc * 4) = w;
+        }
       }
     }
   }
