@@ -18,7 +18,8 @@
 //      (exp2 against the stored LSE), then read their tile's dQ^T out of tensor memory, stage it in shared
 //      memory in the accumulator's layout and add it into the fp32 accumulator with one bulk reduction
 //      (cp.reduce.async.bulk .add.f32, 32 contiguous KB) on the async engine. dK, dV stay in tensor memory
-//      for the whole walk and leave through a TMA store.
+//      for the whole walk; the groups stage them in shared memory and the K/V warp stores them by TMA while
+//      the groups go on with the next key tile.
 //   3. attn_bwd_dq_kernel: dQ = bf16(scale * accumulator) back in [B, T, H, D].
 //
 // Tensor memory of the dK/dV kernel (512 columns): dV [0,128), dK [128,256), and two 128-column tile
@@ -37,7 +38,7 @@ constexpr int kBwdQTile = 64;       // queries per inner tile
 constexpr int kBwdKTile = 128;      // keys per CTA
 constexpr int kBwdStages = 3;       // Q/dO/LSE/Delta ring depth
 constexpr int kBwdThreads = 352;    // warp 0 TMA (query tiles), warp 1 MMA, warps 2..9 two softmax/dQ
-                                    // groups, warp 10 TMA (K, V)
+                                    // groups, warp 10 TMA (K, V in; dV, dK out)
 constexpr int kBwdWarpKV = 10;
 
 constexpr uint32_t kBwdSmemK = 0;                                 // 32 KB
@@ -163,8 +164,9 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const BwdParams p) {
       const int t4 = static_cast<int>(rest % t4n);
       const int bh = static_cast<int>(rest / t4n);
       const int b = bh / p.H, h = bh % p.H;
-      const float v[4][4] = {{a[u][0].x, a[u][1].x, a[u][2].x, a[u][3].x}, {a[u][0].y, a[u][1].y, a[u][2].y, a[u][3].y},
-                             {a[u][0].z, a[u][1].z, a[u][2].z, a[u][3].z}, {a[u][0].w, a[u][1].w, a[u][2].w, a[u][3].w}};
+      const float4* x = a[u];
+      const float v[4][4] = {{x[0].x, x[1].x, x[2].x, x[3].x}, {x[0].y, x[1].y, x[2].y, x[3].y},
+                             {x[0].z, x[1].z, x[2].z, x[3].z}, {x[0].w, x[1].w, x[2].w, x[3].w}};
 #pragma unroll
       for (int tt = 0; tt < 4; ++tt) {
         const int t = t4 * 4 + tt;
@@ -195,6 +197,9 @@ struct BwdBarriers {
                           // arrived by that step's group leader (one phase per step of that group)
   uint64_t acc_done;     // every MMA of an item done: its dV, dK are final (one phase per item)
   uint64_t acc_free;     // dV, dK read out of tensor memory by the epilogue (8 warps, one phase per item)
+  uint64_t epi_staged;   // an item's dV and dK staged in shared memory for their stores (8 warps, one phase per item)
+  uint64_t ds_read;      // an item's dK stores have read the dS^T buffers (one phase per item)
+  uint64_t dq_read;      // an item's dV stores have read the dQ staging buffer (one phase per item)
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -207,7 +212,7 @@ static_assert(kBwdSmemAlloc <= 232448, "dK/dV kernel exceeds the 227 KB shared-m
 enum : uint32_t {
   kSiteBwdLayout = 0x40, kSiteBwdProdQEmpty = 0x41, kSiteBwdProdKV = 0x42, kSiteBwdMmaKV = 0x51, kSiteBwdMmaQ = 0x52,
   kSiteBwdMmaDqEmpty = 0x53, kSiteBwdMmaP = 0x54, kSiteBwdMmaAcc = 0x55, kSiteBwdSmS = 0x61, kSiteBwdSmQ = 0x62,
-  kSiteBwdSmEpi = 0x63, kSiteBwdDq = 0x71, kSiteBwdDrain = 0x72
+  kSiteBwdSmEpi = 0x63, kSiteBwdSmEpiRead = 0x64, kSiteBwdKvEpi = 0x43, kSiteBwdDq = 0x71, kSiteBwdDrain = 0x72
 };
 
 // Work item k of this CTA: one 128-key tile of one key/value head. Items are ordered head-major with the
@@ -283,6 +288,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     mbar_init(&bars.stage_free[1], 1);
     mbar_init(&bars.acc_done, 1);
     mbar_init(&bars.acc_free, 8);  // the warps of both groups
+    mbar_init(&bars.epi_staged, 8);
+    mbar_init(&bars.ds_read, 1);
+    mbar_init(&bars.dq_read, 1);
     mbar_init(&bars.drain, 1);
     bars.abort = 0;
     fence_barrier_init();
@@ -347,28 +355,58 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     kSiteBwdDrain);
     }
   } else if (warp == kBwdWarpKV) {
-    // ------------------------------------------------------------------ TMA producer: K and V of each item
+    // ------------------------------------------------------------------ TMA: K and V in, dV and dK out
     // V is read only by the dP^T MMAs, K also by the dQ^T MMAs of the last step: each loads for the next item
     // as soon as the MMAs that read the current one have completed. Both come from DRAM (a key tile is read by
     // one CTA only), so the next item's are first prefetched into L2 while the current item is computed.
+    // This warp also stores each item's dV and dK once both softmax groups have staged them (group 0 stages dV
+    // in the dQ staging buffer, group 1 dK in the two dS^T buffers) and reports when the stores have read the
+    // staging, dK's first (ds_read: the next item's first step writes a dS^T buffer early) and dV's second
+    // (dq_read: the dQ staging comes at the step's end): the groups go on with the next item meanwhile and wait
+    // for a report only before they write to that buffer again. In time, item k-1's stores come after item k's
+    // K load.
     const bool leader = elect_one();
     int k_issued = -1, v_issued = -1;
-    BwdItem it, nx;
-    for (int k = 0; bwd_item(k, p, it); ++k) {
+    BwdItem it, nx, prev;
+    auto store_epilogue = [&](int k, const BwdItem& e) -> bool {  // item k = e: dV and dK to global
+      if (!mbar_wait_warp(&bars.epi_staged, k & 1, abort, lim, &g_device_error, kSiteBwdKvEpi)) return false;
+      if (leader && !*abort) {
+        const int r0 = e.kt * kBwdKTile;
+        for (int c = 0; c < 2; ++c) tma_store_4d(&tm_dk, smem + kBwdSmemDS + c * 16384, c * 64, e.hk, r0, e.b);
+        tma_store_commit();
+        for (int c = 0; c < 2; ++c) tma_store_4d(&tm_dv, smem + kBwdSmemDQ + c * 16384, c * 64, e.hk, r0, e.b);
+        tma_store_commit();
+        tma_store_wait_read<1>();  // dK's group (the older one) has read the dS^T buffers
+        mbar_arrive(&bars.ds_read);
+        tma_store_wait_read<0>();
+        mbar_arrive(&bars.dq_read);
+      }
+      __syncwarp();
+      return true;
+    };
+    int k = 0;
+    bool ok = true;
+    for (; bwd_item(k, p, it); ++k) {
       const int k0 = it.kt * kBwdKTile;
       if (leader && bwd_item(k + 1, p, nx))
         for (int c = 0; c < 2; ++c) {
           tma_prefetch_l2_4d(&tm_k, c * 64, nx.hk, nx.kt * kBwdKTile, nx.b);
           tma_prefetch_l2_4d(&tm_v, c * 64, nx.hk, nx.kt * kBwdKTile, nx.b);
         }
-      if (k >= 1 && !mbar_wait_warp(&bars.v_free, (k - 1) & 1, abort, lim, &g_device_error, kSiteBwdProdKV)) break;
+      if (k >= 1 && !mbar_wait_warp(&bars.v_free, (k - 1) & 1, abort, lim, &g_device_error, kSiteBwdProdKV)) {
+        ok = false;
+        break;
+      }
       if (leader) {
         mbar_arrive_expect_tx(&bars.v_full, 2 * 16384);
         for (int c = 0; c < 2; ++c)
           tma_load_4d(smem + kBwdSmemV + c * 16384, &tm_v, &bars.v_full, c * 64, it.hk, k0, it.b);
       }
       v_issued = k;
-      if (k >= 1 && !mbar_wait_warp(&bars.k_free, (k - 1) & 1, abort, lim, &g_device_error, kSiteBwdProdKV)) break;
+      if (k >= 1 && !mbar_wait_warp(&bars.k_free, (k - 1) & 1, abort, lim, &g_device_error, kSiteBwdProdKV)) {
+        ok = false;
+        break;
+      }
       if (leader) {
         mbar_arrive_expect_tx(&bars.k_full, 2 * 16384);
         for (int c = 0; c < 2; ++c)
@@ -376,7 +414,14 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       }
       k_issued = k;
       mbar_arrive_warp(&bars.kv_issued);
+      if (k >= 1 && !store_epilogue(k - 1, prev)) {
+        ok = false;
+        break;
+      }
+      prev = it;
     }
+    if (ok && k >= 1) store_epilogue(k - 1, prev);  // the last item's
+    if (leader) tma_store_wait_all();  // the stores are complete before the CTA exits
     if (*abort) {
       volatile int no_abort = 0;
       if (v_issued >= 0) mbar_wait(&bars.v_full, v_issued & 1, &no_abort, lim, &g_device_error, kSiteBwdDrain);
@@ -527,7 +572,11 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const int i = gs - gs0;
         const int s = gs % kBwdStages, rb = g;
         const int q0 = (it.i0 + i % it.n) * kBwdQTile;
-        float* acc_bh = p.dq_acc + static_cast<size_t>(it.b * p.H + it.hk * G + i / it.n) * p.Tp * 128;  // step's query head
+        // the step's query head's accumulator
+        float* acc_bh = p.dq_acc + static_cast<size_t>(it.b * p.H + it.hk * G + i / it.n) * p.Tp * 128;
+        // The group's first step of an item writes its dS^T buffer and then the dQ staging buffer, which the
+        // previous item's dK and dV stores read from: it waits for each report just before the first write.
+        const bool first_of_item = k > 0 && gs < gs0 + 2;
         bool step_ok =
             mbar_wait_warp(&bars.q_full[s], (gs / kBwdStages) & 1, abort, lim, &g_device_error, kSiteBwdSmQ) &&
             mbar_wait_warp(&bars.s_full[rb], (gs >> 1) & 1, abort, lim, &g_device_error, kSiteBwdSmS);
@@ -540,6 +589,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           uint8_t* dsrow = smem + kBwdSmemDS + rb * 16384;
           // The half-tile body is instantiated twice: with the sliding-window mask (tiles that reach past a key's
           // window) and without it, so unwindowed tiles carry no per-element window test.
+          bool ds_ok = true;  // the dS^T buffer may be written (the previous item's dK stores have read it)
           auto halves = [&](auto band_flag) {
             constexpr bool kBand = decltype(band_flag)::value;
 #pragma unroll 1
@@ -573,19 +623,26 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
               }
               tmem_st16(r, ppk);        // P^T  of these 32 queries: columns [32hh, 32hh+16)
               tmem_st16(r + 16, dpk);   // dS^T of these 32 queries: columns [32hh+16, 32hh+32)
+              if (hh == 0 && first_of_item)
+                ds_ok = mbar_wait_warp(&bars.ds_read, (k - 1) & 1, abort, lim, &g_device_error, kSiteBwdSmEpiRead);
+              if (ds_ok) {
 #pragma unroll
-              for (int ch = 0; ch < 4; ++ch) {
-                uint4 v = make_uint4(dpk[ch * 4 + 0], dpk[ch * 4 + 1], dpk[ch * 4 + 2], dpk[ch * 4 + 3]);
-                *reinterpret_cast<uint4*>(dsrow + sw128_offset(krow, 4 * hh + ch)) = v;
+                for (int ch = 0; ch < 4; ++ch) {
+                  uint4 v = make_uint4(dpk[ch * 4 + 0], dpk[ch * 4 + 1], dpk[ch * 4 + 2], dpk[ch * 4 + 3]);
+                  *reinterpret_cast<uint4*>(dsrow + sw128_offset(krow, 4 * hh + ch)) = v;
+                }
               }
             }
           };
           if (band) halves(std::true_type{});
           else halves(std::false_type{});
           tmem_wait_st();
-          fence_async_shared();
-          tc_fence_before();
-          mbar_arrive_warp(&bars.p_full[rb]);
+          step_ok = ds_ok;
+          if (step_ok) {
+            fence_async_shared();
+            tc_fence_before();
+            mbar_arrive_warp(&bars.p_full[rb]);
+          }
           if (threadIdx.x == 64 || threadIdx.x == 192) ATTN_TRACE_EVENT(5, gs);
         }
 
@@ -603,7 +660,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           tc_fence_before();
           mbar_arrive_warp(&bars.dq_empty[rb]);  // dQ^T is in registers: the tensor-memory columns are free
         }
-        step_ok = step_ok && (gs == 0 || wait_staged(gs - 1));
+        step_ok = step_ok && (gs == 0 || wait_staged(gs - 1)) &&
+                  (!first_of_item ||  // the previous item's dV stores have read the staging buffer
+                   mbar_wait_warp(&bars.dq_read, (k - 1) & 1, abort, lim, &g_device_error, kSiteBwdSmEpiRead));
         if (step_ok) {
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh)
@@ -629,13 +688,16 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           ATTN_TRACE_EVENT(7, gs);
         }
       }
-      // Epilogue of the item: group 0 writes dV, group 1 writes scale*dK: TMEM -> bf16 -> swizzled staging ->
-      // TMA store (rows past T are clipped). Group 0 stages in the dQ staging buffer once the item's last
-      // bulk reduction has read it, group 1 in the two dS^T buffers, free once the item's MMAs are done.
-      // Both groups reach every named barrier, failed or not; nothing is stored after a failure.
+      // Epilogue of the item: group 0 stages dV, group 1 scale*dK: TMEM -> bf16 -> swizzled shared memory, and
+      // the K/V warp stores both (rows past T are clipped). Group 0 stages in the dQ staging buffer once the
+      // item's last bulk reductions have read it, group 1 in the two dS^T buffers, free once the item's MMAs are
+      // done; each waits until the previous item's stores have read its buffer (a group without a step in this
+      // item has not waited for that yet). The group leaves the item together, failed or not.
       const int gs_last = gs0 + ns - 1;
       bool epi_ok = __all_sync(0xffffffffu, ok) &&
-                    mbar_wait_warp(&bars.acc_done, k & 1, abort, lim, &g_device_error, kSiteBwdSmEpi);
+                    mbar_wait_warp(&bars.acc_done, k & 1, abort, lim, &g_device_error, kSiteBwdSmEpi) &&
+                    (k == 0 || mbar_wait_warp(g == 0 ? &bars.dq_read : &bars.ds_read, (k - 1) & 1, abort, lim,
+                                              &g_device_error, kSiteBwdSmEpiRead));
       // group 0: the last reductions of both groups (steps gs_last and gs_last - 1) have read the staging buffer
       if (epi_ok && g == 0) epi_ok = wait_staged(gs_last) && (gs_last == 0 || wait_staged(gs_last - 1));
       uint8_t* stage = smem + (g == 0 ? kBwdSmemDQ : kBwdSmemDS);  // 32 KB each: two 16 KB boxes
@@ -663,18 +725,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             *reinterpret_cast<uint4*>(box + sw128_offset(krow, (cc & 1) * 4 + ch)) = v;
           }
         }
+        fence_async_shared();
+        mbar_arrive_warp(&bars.epi_staged);  // the K/V warp stores once all eight warps have staged
       }
-      fence_async_shared();
-      named_barrier(2 + g, 128);
-      if (group_leader && epi_ok && !*abort) {
-        const CUtensorMap* tm = g == 0 ? &tm_dv : &tm_dk;
-        for (int cc = 0; cc < 2; ++cc) tma_store_4d(tm, stage + cc * 16384, cc * 64, it.hk, k0, it.b);
-        tma_store_commit();
-        tma_store_wait_read_all();  // the staging area is free again
-      }
-      // Both groups continue only once both stores have read their staging: the next item's first dS^T and dQ
-      // staging writes go there. Leave together on the same decision.
-      if (!named_barrier_and(1, 256, epi_ok && !*abort)) break;
+      if (!named_barrier_and(2 + g, 128, epi_ok && !*abort)) break;
       gs0 += ns;
     }
     if (group_leader) tma_store_wait_all();  // this group's reductions and stores are complete before exit

@@ -193,6 +193,12 @@ ATTN_DEVICE_INLINE void tma_store_wait_read_all() {
 
 ATTN_DEVICE_INLINE void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Wait until at most N of this thread's most recent bulk groups still read their shared-memory source.
+template <int N>
+ATTN_DEVICE_INLINE void tma_store_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
 // Untiled bulk copy global -> shared; both addresses 16-byte aligned, bytes a multiple of 16.
 ATTN_DEVICE_INLINE void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(

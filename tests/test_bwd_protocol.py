@@ -5,8 +5,11 @@ mbarriers: the TMA producer of query tiles (Q, dO, LSE and Delta of every step t
 across items; an item's tiles are queued once its K and V loads are), the K/V producer (each item's V once the last dP^T of the previous item is done, its K once the
 last dQ^T is), the MMA warp (per item in the order A(0), A(1), B(0), A(2), B(1), ..., B(n-1): A writes dP^T, then
 S^T into tensor-memory buffer gs % 2 of the running step gs, B computes dQ^T, then dV and dK), and two softmax
-groups that take the steps in turn (group g owns the steps gs = g mod 2 and buffer g) and after each item write
-its dV and dK (the item's first dV, dK MMAs wait until they have been read out). The groups hand the 32 KB dQ
+groups that take the steps in turn (group g owns the steps gs = g mod 2 and buffer g) and after each item stage
+its dV and dK in shared memory (the next item's first dV, dK MMAs wait until they have been read out of tensor
+memory); the K/V producer issues the stores once both groups have staged them (epi_staged) and reports when
+dK's have read the dS^T buffers (ds_read) and when dV's have read the dQ staging buffer (dq_read); each group
+waits for those reports before its first write to the same buffers in the next item. The groups hand the 32 KB dQ
 staging buffer to each other in step order: step gs's bulk reduction reports on stage_free[gs % 2]. Barrier
 counts follow the kernel: the softmax-side barriers count warps, and each group is two actors -- the leader's
 warp, which also issues the reductions and reports their reads, and the other three warps, which can run ahead
@@ -17,12 +20,13 @@ mixes and interleavings the model checks that
   * no parity wait can be fooled: when a wait for phase n of a barrier succeeds, phase n + 1 has not completed
     yet (a parity wait only sees the current phase's parity, so a waiter two phases behind would hang or pass
     on the wrong phase), and
-  * the staging buffer is never written (dQ of a step, or an item's dV) while a reduction is still reading it.
+  * the staging buffer is never written (dQ of a step, or an item's dV) while a reduction is still reading it,
+    and neither it nor a dS^T buffer is written while the previous item's dV, dK stores are reading them.
 
 Negative controls must fail: a producer that refills ring slots without waiting for their release runs the
 softmax groups' waits two phases behind; one stage barrier shared by both groups lets a warp wait two phases
 ahead of it and stage over a tile being read; an epilogue that stages dV without waiting for the item's last
-reductions does the same.
+reductions does the same; a first step that does not wait for the previous item's stores writes over them.
 """
 import random
 
@@ -46,8 +50,10 @@ class Model:
     def __init__(self, items, bug=None):
         self.items, self.bug = items, bug  # items: steps of each work item of the CTA
         self.b = {name: Barrier(1) for name in ("k_full", "v_full", "k_free", "v_free", "kv_issued", "stage_free0",
-                                                 "stage_free1", "acc_done", "drain")}
+                                                 "stage_free1", "acc_done", "drain", "ds_read",
+                                                 "dq_read")}
         self.b["acc_free"] = Barrier(8)
+        self.b["epi_staged"] = Barrier(8)
         for s in range(STAGES):
             self.b[f"q_full{s}"] = Barrier(1)
             self.b[f"q_empty{s}"] = Barrier(1)
@@ -57,6 +63,8 @@ class Model:
         self.named = {}  # named barrier instance -> actors that reached it
         self.single_done = 0  # completions of a single stage barrier for both groups (negative control)
         self.staged_reads_pending = set()  # steps whose dQ staging has been written but not yet read
+        self.ds_reads_pending = set()      # items whose dK staging (the dS^T buffers) the stores have not read
+        self.dq_reads_pending = set()      # items whose dV staging (the dQ staging buffer) they have not read
         self.violations = []
 
     def wait_single(self, n):
@@ -88,6 +96,17 @@ def producer(m):
 
 
 def kv_producer(m):
+    def store_epilogue(k):  # item k's dK, then dV stores, once both groups have staged them
+        yield m.wait("epi_staged", k)
+        m.ds_reads_pending.add(k)
+        m.dq_reads_pending.add(k)
+        yield lambda: True
+        m.ds_reads_pending.discard(k)  # the dK stores have read the dS^T buffers
+        m.b["ds_read"].arrive()
+        yield lambda: True
+        m.dq_reads_pending.discard(k)  # the dV stores have read the dQ staging buffer
+        m.b["dq_read"].arrive()
+
     for k, _ in enumerate(m.items):
         if k >= 1:
             yield m.wait("v_free", k - 1)
@@ -96,6 +115,9 @@ def kv_producer(m):
             yield m.wait("k_free", k - 1)
         m.b["k_full"].arrive()
         m.b["kv_issued"].arrive()
+        if k >= 1:
+            yield from store_epilogue(k - 1)
+    yield from store_epilogue(len(m.items) - 1)
 
 
 def mma(m):
@@ -152,12 +174,21 @@ def softmax_warps(m, g, lead):
     def wait_staged(step):
         return m.wait(f"stage_free{step & 1}", step >> 1)
 
+    def wait_read(name, k):  # the previous item's dK (ds_read) or dV (dq_read) stores have read their staging
+        if k >= 1 and m.bug != "no_epilogue_read_wait":
+            yield m.wait(name, k - 1)
+
     gs0 = 0
     for k, ns in enumerate(m.items):
+        first = True
         for gs in range(gs0 + ((g - gs0) & 1), gs0 + ns, 2):
             s, rb = gs % STAGES, g
             yield m.wait(f"q_full{s}", gs // STAGES)
             yield m.wait(f"s_full{rb}", gs >> 1)
+            if first:
+                yield from wait_read("ds_read", k)
+            if m.ds_reads_pending:
+                m.violations.append(("dS^T written over an unread dK staging", gs))
             m.b[f"p_full{rb}"].arrive(n)
             yield m.wait(f"dq_full{rb}", gs >> 1)
             m.b[f"dq_empty{rb}"].arrive(n)
@@ -166,7 +197,10 @@ def softmax_warps(m, g, lead):
                     yield m.wait_single(gs - 1)
                 else:
                     yield wait_staged(gs - 1)
-            if m.staged_reads_pending:
+            if first:
+                yield from wait_read("dq_read", k)
+                first = False
+            if m.staged_reads_pending or m.dq_reads_pending:
                 m.violations.append(("dQ staged over an unread tile", gs))
             yield named_barrier(m, ("stage", gs), actor, 2)
             if lead:
@@ -185,10 +219,14 @@ def softmax_warps(m, g, lead):
                 yield wait_staged(gs_last)
                 if gs_last > 0:
                     yield wait_staged(gs_last - 1)
+        yield from wait_read("dq_read" if g == 0 else "ds_read", k)  # a group without a step here has not waited
         if g == 0 and m.staged_reads_pending:
             m.violations.append(("dV staged over a dQ tile not yet read", k))
+        if (g == 0 and m.dq_reads_pending) or (g == 1 and m.ds_reads_pending):
+            m.violations.append(("dV or dK staged over the previous item's unread staging", k))
         m.b["acc_free"].arrive(n)
-        yield named_barrier(m, ("epilogue", k), actor, 4)  # both groups, after the stores
+        m.b["epi_staged"].arrive(n)  # the K/V producer issues the stores
+        yield named_barrier(m, ("epilogue", k, g), actor, 2)  # the group leaves the item together
         gs0 += ns
 
 
@@ -258,4 +296,12 @@ def test_model_catches_an_epilogue_overwriting_the_last_dq_tile():
     a dQ tile that the other group's reduction has not read yet."""
     rng = random.Random(5)
     caught = sum(bool(run(random_items(rng), seed, bug="epilogue_skips_stage_wait")[1]) for seed in range(200))
+    assert caught > 0
+
+
+def test_model_catches_a_step_writing_over_the_previous_items_stores():
+    """Negative control: a group whose first step of an item does not wait for the previous item's dV, dK stores
+    to have read their staging writes dS^T (or stages dQ) over it."""
+    rng = random.Random(7)
+    caught = sum(bool(run(random_items(rng), seed, bug="no_epilogue_read_wait")[1]) for seed in range(300))
     assert caught > 0
