@@ -320,12 +320,19 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     bool ok = true;
     BwdItem it;
     for (int k = 0; ok && bwd_item(k, p, it); ++k) {
-      // The item's first query tiles are needed together with its K and V, which load only once the previous
-      // item's last MMAs have read theirs: queueing the tiles behind them on the copy engine gets all three
-      // in sooner than loading the tiles early and the K/V behind them.
-      if (!mbar_wait_warp(&bars.kv_issued, k & 1, abort, lim, &g_device_error, kSiteBwdProdQEmpty)) break;
-      for (int i = 0; i < G * it.n; ++i, ++gs) {
+      // An item's K loads only once the previous item's last MMAs have read that item's K, and its first S^T
+      // MMA waits for it; its first dP^T MMA needs only V, loaded earlier, and the first dO tile. So the item's
+      // first two query tiles go out as soon as their ring slots are free, ahead of K, and the later ones
+      // queue behind K on the copy engine (with nothing else in flight, the CTA's first item loads K and V
+      // first). The wait on kv_issued comes exactly once per item, so its parity never skips a phase.
+      const int ns = G * it.n;
+      const int kv_gate = k == 0 ? 0 : min(2, ns - 1);
+      for (int i = 0; i < ns; ++i, ++gs) {
         const int s = gs % kBwdStages;
+        if (i == kv_gate && !mbar_wait_warp(&bars.kv_issued, k & 1, abort, lim, &g_device_error, kSiteBwdProdQEmpty)) {
+          ok = false;
+          break;
+        }
         if (gs >= kBwdStages && !mbar_wait_warp(&bars.q_empty[s], ((gs - kBwdStages) / kBwdStages) & 1, abort, lim,
                                                 &g_device_error, kSiteBwdProdQEmpty)) {
           ok = false;

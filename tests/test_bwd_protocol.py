@@ -3,7 +3,7 @@
 attn_bwd_dkdv_kernel is persistent: a CTA walks several work items (key tiles), and its roles talk only through
 mbarriers: the TMA producer of query tiles (Q, dO, LSE and Delta of every step through a 3-slot ring, running on
 across items; an item's tiles are queued once its K and V loads are), the K/V producer (each item's V once the last dP^T of the previous item is done, its K once the
-last dQ^T is), the MMA warp (per item in the order A(0), A(1), B(0), A(2), B(1), ..., B(n-1): A writes dP^T, then
+last dQ^T is; an item's first two query tiles may go ahead of them, the rest queue behind), the MMA warp (per item in the order A(0), A(1), B(0), A(2), B(1), ..., B(n-1): A writes dP^T, then
 S^T into tensor-memory buffer gs % 2 of the running step gs, B computes dQ^T, then dV and dK), and two softmax
 groups that take the steps in turn (group g owns the steps gs = g mod 2 and buffer g) and after each item stage
 its dV and dK in shared memory (the next item's first dV, dK MMAs wait until they have been read out of tensor
@@ -86,8 +86,9 @@ class Model:
 def producer(m):
     gs = 0
     for k, ns in enumerate(m.items):
-        yield m.wait("kv_issued", k)  # the item's query tiles queue behind its K and V
-        for _ in range(ns):
+        for i in range(ns):
+            if i == (0 if k == 0 else min(2, ns - 1)):  # once per item: its later tiles queue behind its K and V
+                yield m.wait("kv_issued", k)
             s = gs % STAGES
             if gs >= STAGES and m.bug != "no_ring_release_wait":
                 yield m.wait(f"q_empty{s}", (gs - STAGES) // STAGES)
