@@ -223,11 +223,13 @@ struct BwdItem {
   int b, hk, kt;
   int i0, n;  // query tiles i0 .. i0+n-1 of every query head of the group see these keys
 };
+// The host caps B * H * ceil(T / 128) at 2^30, so item indices (fewer than that plus one round of CTAs) fit in
+// 32 bits and decode with 32-bit divisions.
 __device__ __forceinline__ bool bwd_item(int k, const BwdParams& p, BwdItem& it) {
-  const int n_kt = (p.T + kBwdKTile - 1) / kBwdKTile;
-  const long long n_items = static_cast<long long>(p.B) * p.Hkv * n_kt;
-  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
-  const long long idx = static_cast<long long>(k) * G + ((k & 1) ? G - 1 - c : c);
+  const unsigned n_kt = static_cast<unsigned>(p.T + kBwdKTile - 1) / kBwdKTile;
+  const unsigned n_items = static_cast<unsigned>(p.B) * static_cast<unsigned>(p.Hkv) * n_kt;
+  const unsigned G = gridDim.x, c = blockIdx.x;
+  const unsigned idx = static_cast<unsigned>(k) * G + ((k & 1) ? G - 1 - c : c);
   if (idx >= n_items) return false;
   const int bhk = static_cast<int>(idx / n_kt);
   it.kt = static_cast<int>(idx % n_kt);
@@ -570,17 +572,21 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     };
     bool ok = true;
     int gs0 = 0;  // running step count at the start of the item
-    BwdItem it;
-    for (int k = 0; bwd_item(k, p, it); ++k) {
+    BwdItem it, nxt;
+    bool have = bwd_item(0, p, it);
+    for (int k = 0; have; ++k) {
       const int ns = G * it.n;
       const int k0 = it.kt * kBwdKTile;
       const int kg = k0 + krow;
+      // Step i of the item is query tile qi = i mod n of query head hq = i / n of the group; the group takes
+      // every second step, so both advance by counting (no division per step).
+      int qi = (g - gs0) & 1, hq = 0;
+      while (qi >= it.n) qi -= it.n, ++hq;
       for (int gs = gs0 + ((g - gs0) & 1); ok && gs < gs0 + ns; gs += 2) {
-        const int i = gs - gs0;
         const int s = gs % kBwdStages, rb = g;
-        const int q0 = (it.i0 + i % it.n) * kBwdQTile;
+        const int q0 = (it.i0 + qi) * kBwdQTile;
         // the step's query head's accumulator
-        float* acc_bh = p.dq_acc + static_cast<size_t>(it.b * p.H + it.hk * G + i / it.n) * p.Tp * 128;
+        float* acc_bh = p.dq_acc + static_cast<size_t>(it.b * p.H + it.hk * G + hq) * p.Tp * 128;
         // The group's first step of an item writes its dS^T buffer and then the dQ staging buffer, which the
         // previous item's dK and dV stores read from: it waits for each report just before the first write.
         const bool first_of_item = k > 0 && gs < gs0 + 2;
@@ -694,6 +700,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           mbar_arrive(&bars.stage_free[g]);
           ATTN_TRACE_EVENT(7, gs);
         }
+        qi += 2;
+        while (qi >= it.n) qi -= it.n, ++hq;
       }
       // Epilogue of the item: group 0 stages dV, group 1 scale*dK: TMEM -> bf16 -> swizzled shared memory, and
       // the K/V warp stores both (rows past T are clipped). Group 0 stages in the dQ staging buffer once the
@@ -701,6 +709,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       // done; each waits until the previous item's stores have read its buffer (a group without a step in this
       // item has not waited for that yet). The group leaves the item together, failed or not.
       const int gs_last = gs0 + ns - 1;
+      const bool have_next = bwd_item(k + 1, p, nxt);  // decoded while the item's last MMAs finish
       bool epi_ok = __all_sync(0xffffffffu, ok) &&
                     mbar_wait_warp(&bars.acc_done, k & 1, abort, lim, &g_device_error, kSiteBwdSmEpi) &&
                     (k == 0 || mbar_wait_warp(g == 0 ? &bars.dq_read : &bars.ds_read, (k - 1) & 1, abort, lim,
@@ -737,6 +746,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       }
       if (!named_barrier_and(2 + g, 128, epi_ok && !*abort)) break;
       gs0 += ns;
+      it = nxt;
+      have = have_next;
     }
     if (group_leader) tma_store_wait_all();  // this group's reductions and stores are complete before exit
   }
