@@ -197,7 +197,8 @@ struct BwdBarriers {
                           // arrived by that step's group leader (one phase per step of that group)
   uint64_t acc_done;     // every MMA of an item done: its dV, dK are final (one phase per item)
   uint64_t acc_free;     // dV, dK read out of tensor memory by the epilogue (8 warps, one phase per item)
-  uint64_t epi_staged;   // an item's dV and dK staged in shared memory for their stores (8 warps, one phase per item)
+  uint64_t dk_staged;    // an item's dK staged in the dS^T buffers for its store (4 warps, one phase per item)
+  uint64_t dv_staged;    // an item's dV staged in the dQ staging buffer for its store (4 warps, one phase per item)
   uint64_t ds_read;      // an item's dK stores have read the dS^T buffers (one phase per item)
   uint64_t dq_read;      // an item's dV stores have read the dQ staging buffer (one phase per item)
   uint64_t drain;
@@ -290,7 +291,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     mbar_init(&bars.stage_free[1], 1);
     mbar_init(&bars.acc_done, 1);
     mbar_init(&bars.acc_free, 8);  // the warps of both groups
-    mbar_init(&bars.epi_staged, 8);
+    mbar_init(&bars.dk_staged, 4);
+    mbar_init(&bars.dv_staged, 4);
     mbar_init(&bars.ds_read, 1);
     mbar_init(&bars.dq_read, 1);
     mbar_init(&bars.drain, 1);
@@ -368,25 +370,28 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // V is read only by the dP^T MMAs, K also by the dQ^T MMAs of the last step: each loads for the next item
     // as soon as the MMAs that read the current one have completed. Both come from DRAM (a key tile is read by
     // one CTA only), so the next item's are first prefetched into L2 while the current item is computed.
-    // This warp also stores each item's dV and dK once both softmax groups have staged them (group 0 stages dV
-    // in the dQ staging buffer, group 1 dK in the two dS^T buffers) and reports when the stores have read the
-    // staging, dK's first (ds_read: the next item's first step writes a dS^T buffer early) and dV's second
-    // (dq_read: the dQ staging comes at the step's end): the groups go on with the next item meanwhile and wait
-    // for a report only before they write to that buffer again. In time, item k-1's stores come after item k's
-    // K load.
+    // This warp also stores each item's dK as soon as it is staged in the two dS^T buffers and reports when the
+    // store has read them (ds_read: the next item's first step writes a dS^T buffer early), then dV, staged in
+    // the dQ staging buffer (dq_read: the dQ staging comes at a step's end). The softmax groups go on with the
+    // next item meanwhile and wait for a report only before they write to that buffer again. In time, item
+    // k-1's stores come after item k's K load.
     const bool leader = elect_one();
     int k_issued = -1, v_issued = -1;
     BwdItem it, nx, prev;
-    auto store_epilogue = [&](int k, const BwdItem& e) -> bool {  // item k = e: dV and dK to global
-      if (!mbar_wait_warp(&bars.epi_staged, k & 1, abort, lim, &g_device_error, kSiteBwdKvEpi)) return false;
+    auto store_epilogue = [&](int k, const BwdItem& e) -> bool {  // item k = e: dK, then dV, to global
+      const int r0 = e.kt * kBwdKTile;
+      if (!mbar_wait_warp(&bars.dk_staged, k & 1, abort, lim, &g_device_error, kSiteBwdKvEpi)) return false;
       if (leader && !*abort) {
-        const int r0 = e.kt * kBwdKTile;
         for (int c = 0; c < 2; ++c) tma_store_4d(&tm_dk, smem + kBwdSmemDS + c * 16384, c * 64, e.hk, r0, e.b);
         tma_store_commit();
+        tma_store_wait_read<0>();
+        mbar_arrive(&bars.ds_read);
+      }
+      __syncwarp();
+      if (!mbar_wait_warp(&bars.dv_staged, k & 1, abort, lim, &g_device_error, kSiteBwdKvEpi)) return false;
+      if (leader && !*abort) {
         for (int c = 0; c < 2; ++c) tma_store_4d(&tm_dv, smem + kBwdSmemDQ + c * 16384, c * 64, e.hk, r0, e.b);
         tma_store_commit();
-        tma_store_wait_read<1>();  // dK's group (the older one) has read the dS^T buffers
-        mbar_arrive(&bars.ds_read);
         tma_store_wait_read<0>();
         mbar_arrive(&bars.dq_read);
       }
@@ -703,24 +708,27 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         qi += 2;
         while (qi >= it.n) qi -= it.n, ++hq;
       }
-      // Epilogue of the item: group 0 stages dV, group 1 scale*dK: TMEM -> bf16 -> swizzled shared memory, and
-      // the K/V warp stores both (rows past T are clipped). Group 0 stages in the dQ staging buffer once the
-      // item's last bulk reductions have read it, group 1 in the two dS^T buffers, free once the item's MMAs are
-      // done; each waits until the previous item's stores have read its buffer (a group without a step in this
-      // item has not waited for that yet). The group leaves the item together, failed or not.
+      // Epilogue of the item: TMEM -> bf16 -> swizzled shared memory, and the K/V warp stores (rows past T are
+      // clipped). The group of the item's last step is the late one: its last bulk reduction still reads the dQ
+      // staging buffer, so it stages dV there once that (and the other group's last reduction) has read it. The
+      // other group stages scale*dK in the two dS^T buffers, free once the item's MMAs are done, and its store
+      // goes out at once; that group also runs the next item's first step. Each group first waits until the
+      // previous item's store has read its buffer (a group without a step in this item has not waited for that
+      // yet). The group leaves the item together, failed or not.
       const int gs_last = gs0 + ns - 1;
+      const bool dv_group = (gs_last & 1) == g;
       const bool have_next = bwd_item(k + 1, p, nxt);  // decoded while the item's last MMAs finish
       bool epi_ok = __all_sync(0xffffffffu, ok) &&
                     mbar_wait_warp(&bars.acc_done, k & 1, abort, lim, &g_device_error, kSiteBwdSmEpi) &&
-                    (k == 0 || mbar_wait_warp(g == 0 ? &bars.dq_read : &bars.ds_read, (k - 1) & 1, abort, lim,
+                    (k == 0 || mbar_wait_warp(dv_group ? &bars.dq_read : &bars.ds_read, (k - 1) & 1, abort, lim,
                                               &g_device_error, kSiteBwdSmEpiRead));
-      // group 0: the last reductions of both groups (steps gs_last and gs_last - 1) have read the staging buffer
-      if (epi_ok && g == 0) epi_ok = wait_staged(gs_last) && (gs_last == 0 || wait_staged(gs_last - 1));
-      uint8_t* stage = smem + (g == 0 ? kBwdSmemDQ : kBwdSmemDS);  // 32 KB each: two 16 KB boxes
+      // the dV group: the last reductions of both groups (steps gs_last and gs_last - 1) have read the buffer
+      if (epi_ok && dv_group) epi_ok = wait_staged(gs_last) && (gs_last == 0 || wait_staged(gs_last - 1));
+      uint8_t* stage = smem + (dv_group ? kBwdSmemDQ : kBwdSmemDS);  // 32 KB each: two 16 KB boxes
       if (epi_ok) {
         tc_fence_after();
-        const float mul = g == 0 ? 1.0f : p.scale;
-        const uint32_t col = g == 0 ? kTmemDV : kTmemDK;
+        const float mul = dv_group ? 1.0f : p.scale;
+        const uint32_t col = dv_group ? kTmemDV : kTmemDK;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t o[32];
@@ -742,7 +750,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           }
         }
         fence_async_shared();
-        mbar_arrive_warp(&bars.epi_staged);  // the K/V warp stores once all eight warps have staged
+        mbar_arrive_warp(dv_group ? &bars.dv_staged : &bars.dk_staged);  // the K/V warp stores it
       }
       if (!named_barrier_and(2 + g, 128, epi_ok && !*abort)) break;
       gs0 += ns;

@@ -2,16 +2,19 @@
 
 attn_bwd_dkdv_kernel is persistent: a CTA walks several work items (key tiles), and its roles talk only through
 mbarriers: the TMA producer of query tiles (Q, dO, LSE and Delta of every step through a 3-slot ring, running on
-across items; an item's tiles are queued once its K and V loads are), the K/V producer (each item's V once the last dP^T of the previous item is done, its K once the
-last dQ^T is; an item's first two query tiles may go ahead of them, the rest queue behind), the MMA warp (per item in the order A(0), A(1), B(0), A(2), B(1), ..., B(n-1): A writes dP^T, then
-S^T into tensor-memory buffer gs % 2 of the running step gs, B computes dQ^T, then dV and dK), and two softmax
+across items; an item's first two tiles go out as soon as their slots free, the later ones queue behind the
+item's K and V loads), the K/V producer (each item's V once the last dP^T of the previous item is done, its K
+once the last dQ^T is; then the previous item's dK and dV stores), the MMA warp (per item in the order A(0),
+A(1), B(0), A(2), B(1), ..., B(n-1): A writes dP^T, then S^T into tensor-memory buffer gs % 2 of the running
+step gs, B computes dQ^T, then dV and dK), and two softmax
 groups that take the steps in turn (group g owns the steps gs = g mod 2 and buffer g) and after each item stage
 its dV and dK in shared memory (the next item's first dV, dK MMAs wait until they have been read out of tensor
-memory); the K/V producer issues the stores once both groups have staged them (epi_staged) and reports when
-dK's have read the dS^T buffers (ds_read) and when dV's have read the dQ staging buffer (dq_read); each group
-waits for those reports before its first write to the same buffers in the next item. The groups hand the 32 KB dQ
-staging buffer to each other in step order: step gs's bulk reduction reports on stage_free[gs % 2]. Barrier
-counts follow the kernel: the softmax-side barriers count warps, and each group is two actors -- the leader's
+memory): the group of the item's last step stages dV in the dQ staging buffer (after its own last reduction
+has read it), the other group dK in the two dS^T buffers. The K/V producer stores dK once it is staged
+(dk_staged) and reports when the store has read the dS^T buffers (ds_read), then does the same for dV
+(dv_staged, dq_read); each group waits for those reports before its first write to the same buffers in the next
+item. The groups hand the 32 KB dQ staging buffer to each other in step order: step gs's bulk reduction
+reports on stage_free[gs % 2]. Barrier counts follow the kernel: the softmax-side barriers count warps, and each group is two actors -- the leader's
 warp, which also issues the reductions and reports their reads, and the other three warps, which can run ahead
 of it. MMAs, commits and copies complete at once (timing does not matter for these properties). Over random item
 mixes and interleavings the model checks that
@@ -24,9 +27,10 @@ mixes and interleavings the model checks that
     and neither it nor a dS^T buffer is written while the previous item's dV, dK stores are reading them.
 
 Negative controls must fail: a producer that refills ring slots without waiting for their release runs the
-softmax groups' waits two phases behind; one stage barrier shared by both groups lets a warp wait two phases
-ahead of it and stage over a tile being read; an epilogue that stages dV without waiting for the item's last
-reductions does the same; a first step that does not wait for the previous item's stores writes over them.
+softmax groups' waits two phases behind; one stage barrier shared by both groups, with dV always staged by
+group 0, lets a warp wait two phases ahead of it and stage over a tile being read; an epilogue that stages dV
+without waiting for the item's last reductions does the same; a first step that does not wait for the previous
+item's stores writes over them.
 """
 import random
 
@@ -53,7 +57,8 @@ class Model:
                                                  "stage_free1", "acc_done", "drain", "ds_read",
                                                  "dq_read")}
         self.b["acc_free"] = Barrier(8)
-        self.b["epi_staged"] = Barrier(8)
+        self.b["dk_staged"] = Barrier(4)  # the four warps of the group that stages dK
+        self.b["dv_staged"] = Barrier(4)
         for s in range(STAGES):
             self.b[f"q_full{s}"] = Barrier(1)
             self.b[f"q_empty{s}"] = Barrier(1)
@@ -97,13 +102,14 @@ def producer(m):
 
 
 def kv_producer(m):
-    def store_epilogue(k):  # item k's dK, then dV stores, once both groups have staged them
-        yield m.wait("epi_staged", k)
+    def store_epilogue(k):  # item k's dK store once dK is staged, then its dV store once dV is
+        yield m.wait("dk_staged", k)
         m.ds_reads_pending.add(k)
-        m.dq_reads_pending.add(k)
         yield lambda: True
         m.ds_reads_pending.discard(k)  # the dK stores have read the dS^T buffers
         m.b["ds_read"].arrive()
+        yield m.wait("dv_staged", k)
+        m.dq_reads_pending.add(k)
         yield lambda: True
         m.dq_reads_pending.discard(k)  # the dV stores have read the dQ staging buffer
         m.b["dq_read"].arrive()
@@ -210,23 +216,27 @@ def softmax_warps(m, g, lead):
                 m.staged_reads_pending.discard(gs)  # ... and has read the buffer
                 m.b[f"stage_free{g}"].arrive()
                 m.single_done += 1
-        # epilogue: both groups, after the item's last MMA; group 0 stages dV where the last dQ tile was staged
+        # epilogue, after the item's last MMA: the group of the item's last step (late: its last reduction still
+        # reads the dQ staging buffer) stages dV there, the other group stages dK in the two dS^T buffers
         yield m.wait("acc_done", k)
         gs_last = gs0 + ns - 1
-        if g == 0 and m.bug != "epilogue_skips_stage_wait":
+        # (the negative control "single_stage_barrier" keeps the dV staging on group 0, where one stage barrier
+        # for both groups is unsafe)
+        dv_group = (g == 0) if m.bug == "single_stage_barrier" else (gs_last & 1) == g
+        if dv_group and m.bug != "epilogue_skips_stage_wait":
             if m.bug == "single_stage_barrier":
                 yield m.wait_single(gs_last)
             else:
                 yield wait_staged(gs_last)
                 if gs_last > 0:
                     yield wait_staged(gs_last - 1)
-        yield from wait_read("dq_read" if g == 0 else "ds_read", k)  # a group without a step here has not waited
-        if g == 0 and m.staged_reads_pending:
+        yield from wait_read("dq_read" if dv_group else "ds_read", k)  # a group without a step here has not waited
+        if dv_group and m.staged_reads_pending:
             m.violations.append(("dV staged over a dQ tile not yet read", k))
-        if (g == 0 and m.dq_reads_pending) or (g == 1 and m.ds_reads_pending):
+        if (dv_group and m.dq_reads_pending) or (not dv_group and m.ds_reads_pending):
             m.violations.append(("dV or dK staged over the previous item's unread staging", k))
         m.b["acc_free"].arrive(n)
-        m.b["epi_staged"].arrive(n)  # the K/V producer issues the stores
+        m.b["dv_staged" if dv_group else "dk_staged"].arrive(n)  # the K/V producer issues that store
         yield named_barrier(m, ("epilogue", k, g), actor, 2)  # the group leaves the item together
         gs0 += ns
 
@@ -277,8 +287,9 @@ def test_protocol_corner_item_mixes(items):
 
 
 def test_model_catches_a_single_stage_barrier_race():
-    """Negative control: with one stage barrier for both groups a warp can wait two phases ahead of it (its own
-    leader's arrival still pending), pass at once and stage over a tile that is still being read."""
+    """Negative control: with one stage barrier for both groups and dV always staged by group 0, a warp of group
+    0 whose group did not run the item's last step can wait two phases ahead of it (its own leader's arrival
+    still pending), pass at once and stage over a tile that is still being read."""
     rng = random.Random(11)
     caught = sum(bool(run(random_items(rng), seed, bug="single_stage_barrier")[1]) for seed in range(300))
     assert caught > 0
