@@ -55,27 +55,6 @@ constexpr uint32_t kTmemS = 0, kTmemO = 256, kTmemQ = 384, kTmemP = 448;
 // Lazy rescaling threshold on the running max, in log2 units (values of P stay below 2^8).
 constexpr float kRescaleThreshold = 8.0f;
 
-// Pairs of columns, out of every 16, whose exp2 runs on the FMA pipe (exp2_poly) instead of MUFU: with the
-// tensor cores of a pair, MUFU's 16 exponentials per clock per SM take as long as the MMAs of a tile.
-#ifndef ATTN_FWD_POLY_PAIRS
-#define ATTN_FWD_POLY_PAIRS 0
-#endif
-constexpr int kFwdPolyPairs = ATTN_FWD_POLY_PAIRS;
-
-// 2^x on the FMA pipe, for x <= 8 (softmax arguments). Cody-Waite style reduction: n = round(x) by the
-// 1.5 * 2^23 magic addition (t's low mantissa bits then hold n), f = x - n in [-1/2, 1/2]; 2^f by a cubic
-// fitted for least maximum relative error (7.5e-5; fit_exp2_poly.py prints the coefficients and the bound);
-// 2^n by adding n to the exponent field (n << 23 equals t's bits << 23 modulo 2^32 because the magic
-// constant's bits vanish under that shift). Below -126 the exponent field would underflow, so those
-// arguments (true values under 1.2e-38, masked keys at -inf among them) return exactly 0.
-__device__ __forceinline__ float exp2_poly(float x) {
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(0.0551716668f, f, 0.242611135f), f, 0.693260987f), f, 0.999928073f);
-  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-  return x < -126.0f ? 0.0f : r;  // masked keys (-inf) give exactly 0
-}
-
 struct FwdParams {
   float* lse;        // [B, H, T] fp32
   int B, H, T;
@@ -576,10 +555,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         xm[sb * 128 + row] = m_j;
         mbar_arrive_warp(&bars.xchg[sb]);
         if (tracer) ATTN_TRACE_EVENT(11, t);
-        // P = exp2(c*S - m_j) for the 128 keys and the row sum, packed to bf16 pairs in registers; the last
-        // kFwdPolyPairs pairs of every 16 go through exp2_poly, the rest through MUFU ex2. A row that
-        // has seen no key yet (only possible left of a sliding window) keeps m_j = -inf and all its scores are
-        // -inf: the reference 0 gives P = 0 there instead of NaN.
+        // P = exp2(c*S - m_j) for the 128 keys (MUFU ex2) and the row sum, packed to bf16 pairs in registers.
+        // A row that has seen no key yet (only possible left of a sliding window) keeps m_j = -inf and all its
+        // scores are -inf: the reference 0 gives P = 0 there instead of NaN.
         const float neg_m = m_j == -INFINITY ? 0.f : -m_j;
         float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent partial row sums
         uint32_t pk[4][16];
@@ -588,9 +566,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float x0 = fmaf(s[cc * 32 + 2 * i], c, neg_m), x1 = fmaf(s[cc * 32 + 2 * i + 1], c, neg_m);
-            const bool poly = i >= 16 - kFwdPolyPairs;
-            const float p0 = poly ? exp2_poly(x0) : ex2(x0);
-            const float p1 = poly ? exp2_poly(x1) : ex2(x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
             ps[(2 * i) & 7] += p0;
             ps[(2 * i + 1) & 7] += p1;
             pk[cc][i] = pack_bf16x2(p0, p1);
