@@ -20,10 +20,11 @@ import torch
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG_DIR, "libattn.so")
+DEBUG_LIB_PATH = os.path.join(_PKG_DIR, "libattn_debug.so")  # the same sources with address checks
 
 ATTN_OK = 0
 _STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_MISALIGNED",
-           4: "ATTN_ERR_CUDA", 5: "ATTN_ERR_TIMEOUT", 6: "ATTN_ERR_WORKSPACE"}
+           4: "ATTN_ERR_CUDA", 5: "ATTN_ERR_TIMEOUT", 6: "ATTN_ERR_WORKSPACE", 7: "ATTN_ERR_BOUNDS"}
 
 # Exported symbols of the C ABI (include/attn.h), with their ctypes signatures.
 _VP, _I, _F, _SZ, _U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint64
@@ -51,6 +52,8 @@ SIGNATURES = {
     "attn_clear_device_error": ([], _I),
     "attn_set_wait_limit_ns": ([_U64], _I),
     "attn_selftest_wait_timeout": ([_U64, _VP], _I),
+    "attn_is_debug_build": ([], _I),
+    "attn_selftest_bounds_check": ([_VP], _I),
 }
 
 
@@ -68,21 +71,30 @@ class AttnError(RuntimeError):
 _lib = None
 
 
-def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Load libattn.so (once) and attach the C signatures. Raises if it has not been built."""
-    global _lib
-    if _lib is not None:
-        return _lib
+def open_library(path: str) -> ctypes.CDLL:
+    """Open a build of the library (libattn.so or libattn_debug.so) with the C signatures attached."""
     if not os.path.exists(path):
         raise ImportError(f"{path} is missing: build it with `python -m causal_self_attention_bf16_b200.build` "
-                          "(or __graft_entry__.build()); there is no fallback implementation")
+                          "(--debug for libattn_debug.so, or __graft_entry__.build()); there is no fallback "
+                          "implementation")
     lib = ctypes.CDLL(path)
     for name, (argtypes, restype) in SIGNATURES.items():
         fn = getattr(lib, name)
         fn.argtypes = argtypes
         fn.restype = restype
-    _lib = lib
     return lib
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """The library every function of this package calls, loaded once: libattn.so, or libattn_debug.so (the
+    address-checking build) when the environment sets ATTN_LIBRARY=debug. Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if path is None:
+        path = DEBUG_LIB_PATH if os.environ.get("ATTN_LIBRARY") == "debug" else LIB_PATH
+    _lib = open_library(path)
+    return _lib
 
 
 def _check(fn: str, status: int):
@@ -404,10 +416,11 @@ def qk_norm_rope_attention(q, k, v, scale: Optional[float] = None, window: Optio
 
 
 def get_device_error() -> int:
-    """The library's device-side error word (0 = no kernel gave up on a bounded wait). Synchronises."""
+    """The library's device-side error word (0 = no kernel gave up on a bounded wait and, in the debug build, no
+    address check failed). Synchronises."""
     word = ctypes.c_uint32(0)
     st = load_library().attn_get_device_error(ctypes.byref(word))
-    if st not in (0, 5):
+    if st not in (0, 5, 7):
         _check("attn_get_device_error", st)
     return int(word.value)
 

@@ -189,6 +189,16 @@ __global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
   if (threadIdx.x == 0) sm100::mbar_wait(&bar, 0, &abort_flag, limit_ns, &attn::g_device_error, 0x7f);
 }
 
+#ifdef ATTN_DEBUG
+// Self-test of the debug build's address checks (see attn_selftest_bounds_check): one checked store whose
+// index (1) lies past the declared one-element extent of its array. The check records the site and skips the
+// store, so nothing is written; the array has a second element all the same, so the index is inside the memory.
+__device__ int g_bounds_selftest_cell[2];
+__global__ void bounds_selftest_kernel(int index) {
+  if (ATTN_IN_RANGE(index, 1, 1, attn::kSiteChkSelftest, &attn::g_device_error)) g_bounds_selftest_cell[index] = 1;
+}
+#endif
+
 }  // namespace
 
 extern "C" {
@@ -204,6 +214,7 @@ const char* attn_status_string(attn_status s) {
     case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
     case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
     case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE";
+    case ATTN_ERR_BOUNDS: return "ATTN_ERR_BOUNDS";
   }
   return "ATTN_ERR_UNKNOWN";
 }
@@ -411,13 +422,20 @@ attn_status attn_get_device_error(uint32_t* word) {
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
   e = cudaMemcpyFromSymbol(word, attn::g_device_error, sizeof(uint32_t));
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol(g_device_error)");
-  return *word ? ATTN_ERR_TIMEOUT : ATTN_OK;
+  uint32_t rope_word = 0;
+  e = static_cast<cudaError_t>(attn::rope_error_word(&rope_word));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol(g_rope_error)");
+  *word |= rope_word;
+  if (*word & sm100::DEV_ERR_TIMEOUT) return ATTN_ERR_TIMEOUT;
+  return *word ? ATTN_ERR_BOUNDS : ATTN_OK;
 }
 
 attn_status attn_clear_device_error(void) {
   const uint32_t zero = 0;
   cudaError_t e = cudaMemcpyToSymbol(attn::g_device_error, &zero, sizeof(uint32_t));
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol(g_device_error)");
+  e = static_cast<cudaError_t>(attn::rope_error_clear());
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol(g_rope_error)");
   e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
   return ATTN_OK;
@@ -436,6 +454,26 @@ int attn_trace_dump(void* dst, size_t bytes) {
   return e == cudaSuccess ? 0 : -1;
 }
 #endif
+
+int attn_is_debug_build(void) {
+#ifdef ATTN_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+attn_status attn_selftest_bounds_check(void* stream) {
+#ifdef ATTN_DEBUG
+  bounds_selftest_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(1);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "bounds_selftest_kernel launch");
+  return ATTN_OK;
+#else
+  (void)stream;
+  return ATTN_ERR_UNSUPPORTED;  // the release build has no address checks to test
+#endif
+}
 
 attn_status attn_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
   if (limit_ns < 1000 || limit_ns > 10ull * 1000 * 1000 * 1000) return ATTN_ERR_INVALID_ARG;

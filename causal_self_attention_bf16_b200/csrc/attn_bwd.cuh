@@ -79,6 +79,8 @@ struct BwdParams {
 // writes as many bytes as it reads, so the read and write streams interleave over the whole grid.
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const BwdParams p) {
   const int64_t quads = static_cast<int64_t>(p.B) * p.H * (p.Tp / 4);  // ordered (bh, t/4)
+  const size_t n_lse = static_cast<size_t>(p.B) * p.H * p.T, n_in = n_lse * 128;  // lse; o and dO
+  const size_t n_rows = static_cast<size_t>(p.B) * p.H * p.Tp;                       // padded rows
   const int sub = threadIdx.x & 15;
   const int64_t group = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
   const int64_t ngroups = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 4;
@@ -90,17 +92,19 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const BwdParams p) {
     for (int j = 0; j < 4; ++j) {
       ov[j] = make_uint4(0u, 0u, 0u, 0u);
       gv[j] = make_uint4(0u, 0u, 0u, 0u);
-      if (t0 + j < p.T) {
-        const size_t off = ((static_cast<size_t>(b) * p.T + t0 + j) * p.H + h) * 128 + sub * 8;
+      const size_t off = ((static_cast<size_t>(b) * p.T + t0 + j) * p.H + h) * 128 + sub * 8;
+      if (t0 + j < p.T && ATTN_IN_RANGE(off, 8, n_in, kSiteChkPrepIn, &g_device_error)) {
         ov[j] = *reinterpret_cast<const uint4*>(p.o + off);
         gv[j] = *reinterpret_cast<const uint4*>(p.dO + off);
       }
     }
     // zero the block of these four rows: 512 floats, 8 float4 per thread
-    float4* blk = reinterpret_cast<float4*>(p.dq_acc + static_cast<size_t>(bh) * p.Tp * 128 +
-                                            static_cast<size_t>(t0) * 128);
+    const size_t blk_off = static_cast<size_t>(bh) * p.Tp * 128 + static_cast<size_t>(t0) * 128;
+    float4* blk = reinterpret_cast<float4*>(p.dq_acc + blk_off);
+    if (ATTN_IN_RANGE(blk_off, 512, n_rows * 128, kSiteChkPrepAcc, &g_device_error)) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) blk[j * 16 + sub] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < 8; ++j) blk[j * 16 + sub] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     float acc[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -123,8 +127,12 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const BwdParams p) {
       const int t = t0 + sub;
       const float a = sub == 0 ? acc[0] : sub == 1 ? acc[1] : sub == 2 ? acc[2] : acc[3];
       const int64_t r = static_cast<int64_t>(bh) * p.Tp + t;
-      p.delta[r] = a;
-      p.lse2[r] = t < p.T ? p.lse[static_cast<size_t>(bh) * p.T + t] * 1.4426950408889634f : INFINITY;
+      const size_t li = static_cast<size_t>(bh) * p.T + t;
+      const bool lse_ok = t < p.T && ATTN_IN_RANGE(li, 1, n_lse, kSiteChkPrepLse, &g_device_error);
+      if (ATTN_IN_RANGE(r, 1, n_rows, kSiteChkPrepRow, &g_device_error)) {
+        p.delta[r] = a;
+        p.lse2[r] = lse_ok ? p.lse[li] * 1.4426950408889634f : INFINITY;
+      }
     }
   }
 }
@@ -138,8 +146,9 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const BwdParams p) {
   const int64_t t4n = (p.T + 3) / 4;
   const int64_t items = static_cast<int64_t>(p.B) * p.H * t4n * 32;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const size_t n_acc = static_cast<size_t>(p.B) * p.H * p.Tp * 128, n_dq = static_cast<size_t>(p.B) * p.T * p.H * 128;
   for (int64_t it0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; it0 < items; it0 += 2 * stride) {
-    float4 a[2][4];
+    float4 a[2][4] = {};
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int64_t it = it0 + u * stride;
@@ -148,10 +157,12 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const BwdParams p) {
         const int64_t rest = it >> 5;
         const int t4 = static_cast<int>(rest % t4n);
         const int bh = static_cast<int>(rest / t4n);
-        const float4* src = reinterpret_cast<const float4*>(p.dq_acc + static_cast<size_t>(bh) * p.Tp * 128 +
-                                                            static_cast<size_t>(t4) * 512 + dc * 16);
+        const size_t off = static_cast<size_t>(bh) * p.Tp * 128 + static_cast<size_t>(t4) * 512 + dc * 16;
+        const float4* src = reinterpret_cast<const float4*>(p.dq_acc + off);
+        if (ATTN_IN_RANGE(off, 16, n_acc, kSiteChkDqIn, &g_device_error)) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) a[u][c] = src[c];  // d = 4dc + c, holding t%4 = 0..3
+          for (int c = 0; c < 4; ++c) a[u][c] = src[c];  // d = 4dc + c, holding t%4 = 0..3
+        }
       }
     }
     const float s = p.scale;
@@ -170,11 +181,12 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const BwdParams p) {
 #pragma unroll
       for (int tt = 0; tt < 4; ++tt) {
         const int t = t4 * 4 + tt;
-        if (t < p.T) {
+        const size_t off = ((static_cast<size_t>(b) * p.T + t) * p.H + h) * 128 + dc * 4;
+        if (t < p.T && ATTN_IN_RANGE(off, 4, n_dq, kSiteChkDqOut, &g_device_error)) {
           uint2 w;
           w.x = sm100::pack_bf16x2(v[tt][0] * s, v[tt][1] * s);
           w.y = sm100::pack_bf16x2(v[tt][2] * s, v[tt][3] * s);
-          *reinterpret_cast<uint2*>(p.dq + ((static_cast<size_t>(b) * p.T + t) * p.H + h) * 128 + dc * 4) = w;
+          *reinterpret_cast<uint2*>(p.dq + off) = w;
         }
       }
     }
@@ -345,14 +357,20 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         const int h = it.hk * G + i / it.n, bh = it.b * p.H + h;  // the step's query head
         const int q0 = (it.i0 + i % it.n) * kBwdQTile;
         if (leader) {
-          mbar_arrive_expect_tx(&bars.q_full[s], 2 * 16384 + 2 * 256);
+          // the step's 64 rows of LSE*log2(e) and Delta (plain addresses: checked in the debug build, where a
+          // failed check skips the two loads and the barrier expects only the tiles)
+          const size_t roff = static_cast<size_t>(bh) * p.Tp + q0;
+          const bool rows_ok =
+              ATTN_IN_RANGE(roff, 64, static_cast<size_t>(p.B) * p.H * p.Tp, kSiteChkBwdRows, &g_device_error);
+          mbar_arrive_expect_tx(&bars.q_full[s], 2 * 16384 + (rows_ok ? 2 * 256 : 0));
           for (int c = 0; c < 2; ++c) {
             tma_load_4d(smem + kBwdSmemQ + s * 16384 + c * 8192, &tm_q, &bars.q_full[s], c * 64, h, q0, it.b);
             tma_load_4d(smem + kBwdSmemDO + s * 16384 + c * 8192, &tm_do, &bars.q_full[s], c * 64, h, q0, it.b);
           }
-          bulk_load(smem + kBwdSmemLse + s * 256, p.lse2 + static_cast<size_t>(bh) * p.Tp + q0, 256, &bars.q_full[s]);
-          bulk_load(smem + kBwdSmemDelta + s * 256, p.delta + static_cast<size_t>(bh) * p.Tp + q0, 256,
-                    &bars.q_full[s]);
+          if (rows_ok) {
+            bulk_load(smem + kBwdSmemLse + s * 256, p.lse2 + roff, 256, &bars.q_full[s]);
+            bulk_load(smem + kBwdSmemDelta + s * 256, p.delta + roff, 256, &bars.q_full[s]);
+          }
           ATTN_TRACE_EVENT(1, gs);
         }
         last_issued[s] = gs;
@@ -699,7 +717,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           break;
         }
         if (group_leader) {
-          bulk_reduce_add_f32(acc_bh + static_cast<size_t>(q0 >> 2) * 512, dq_stage, 32768);
+          // the tile's 8192 accumulator floats (checked in the debug build; a failed check skips the reduction)
+          if (ATTN_IN_RANGE(static_cast<size_t>(acc_bh - p.dq_acc) + static_cast<size_t>(q0 >> 2) * 512, 8192,
+                            static_cast<size_t>(p.B) * p.H * p.Tp * 128, kSiteChkBwdReduce, &g_device_error))
+            bulk_reduce_add_f32(acc_bh + static_cast<size_t>(q0 >> 2) * 512, dq_stage, 32768);
           tma_store_commit();
           tma_store_wait_read_all();  // the staging buffer has been read: hand it to the next step
           mbar_arrive(&bars.stage_free[g]);

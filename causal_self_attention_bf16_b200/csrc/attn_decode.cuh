@@ -68,12 +68,14 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const De
   const int start = p.window < 0 ? 0 : max(0, L - p.Tq - p.window);
   const int key_lo = start + sp * p.chunk, key_hi = min(L, key_lo + p.chunk);
   const size_t row_stride = static_cast<size_t>(p.Hkv) * 128;   // elements between consecutive keys
+  const size_t n_q = static_cast<size_t>(p.B) * p.Tq * p.H * 128, n_kv = static_cast<size_t>(p.B) * p.Tk * row_stride;
 
   // Row r = g * Tq + i: query head hk * G + g, new token i, which sees keys up to L - Tq + i.
   for (int r = 0; r < R; ++r) {
     const int g = r / p.Tq, i = r % p.Tq;
     const size_t qi = ((static_cast<size_t>(b) * p.Tq + i) * p.H + hk * G + g) * 128 + t;
-    qs[r][t] = __bfloat162float(p.q[qi]) * p.scale_log2;
+    qs[r][t] = ATTN_IN_RANGE(qi, 1, n_q, kSiteChkDecQ, &g_device_error) ? __bfloat162float(p.q[qi]) * p.scale_log2
+                                                                         : 0.f;
   }
   if (t < R) {
     row_m[t] = -INFINITY;
@@ -86,18 +88,23 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const De
 
   for (int kb = key_lo; kb < key_hi; kb += kDecKeys) {
     const int nk = min(kDecKeys, key_hi - kb);
-    const __nv_bfloat16* kbase = p.k + ((static_cast<size_t>(b) * p.Tk + kb) * p.Hkv + hk) * 128;
-    const __nv_bfloat16* vbase = p.v + ((static_cast<size_t>(b) * p.Tk + kb) * p.Hkv + hk) * 128;
+    const size_t kv_off = ((static_cast<size_t>(b) * p.Tk + kb) * p.Hkv + hk) * 128;  // key kb's row
+    const __nv_bfloat16* kbase = p.k + kv_off;
+    const __nv_bfloat16* vbase = p.v + kv_off;
     // Issue this block's loads first: the thread's K row (16 x 16 bytes) and 16 of the V block's 16-byte
     // chunks (coalesced: consecutive threads, consecutive chunks of a row), so ~64 KB per CTA are in flight.
     uint4 kw[16], vw[16];
 #pragma unroll
     for (int c = 0; c < 16; ++c)
-      kw[c] = t < nk ? reinterpret_cast<const uint4*>(kbase + t * row_stride)[c] : make_uint4(0, 0, 0, 0);
+      kw[c] = t < nk && ATTN_IN_RANGE(kv_off + t * row_stride + c * 8, 8, n_kv, kSiteChkDecK, &g_device_error)
+                  ? reinterpret_cast<const uint4*>(kbase + t * row_stride)[c]
+                  : make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
       const int idx = u * kDecThreads + t, row = idx / 16, c = idx % 16;
-      vw[u] = row < nk ? reinterpret_cast<const uint4*>(vbase + row * row_stride)[c] : make_uint4(0, 0, 0, 0);
+      vw[u] = row < nk && ATTN_IN_RANGE(kv_off + row * row_stride + c * 8, 8, n_kv, kSiteChkDecV, &g_device_error)
+                  ? reinterpret_cast<const uint4*>(vbase + row * row_stride)[c]
+                  : make_uint4(0, 0, 0, 0);
     }
     // Scores of key kb + t against every row (keys past the block, or past a row's last key, are -inf).
     for (int r = 0; r < R; ++r) {
@@ -177,14 +184,18 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const De
   }
 
   // The chunk's partial result (an empty chunk leaves max -inf, sum 0, O 0).
-  float* po = p.part_o + (static_cast<size_t>(bhk) * p.n_split + sp) * R * 128;
+  const size_t n_part = static_cast<size_t>(p.B) * p.Hkv * p.n_split * R;  // partial rows
+  const size_t part = (static_cast<size_t>(bhk) * p.n_split + sp) * R;      // this chunk's first one
+  float* po = p.part_o + part * 128;
+  if (ATTN_IN_RANGE(part, R, n_part, kSiteChkDecPart, &g_device_error)) {
 #pragma unroll
-  for (int r = 0; r < kRows; ++r)
-    if (r < R) po[r * 128 + t] = acc[r];
-  if (t < R) {
-    float* pml = p.part_ml + ((static_cast<size_t>(bhk) * p.n_split + sp) * R + t) * 2;
-    pml[0] = row_m[t];
-    pml[1] = row_l[t];
+    for (int r = 0; r < kRows; ++r)
+      if (r < R) po[r * 128 + t] = acc[r];
+    if (t < R) {
+      float* pml = p.part_ml + (part + t) * 2;
+      pml[0] = row_m[t];
+      pml[1] = row_l[t];
+    }
   }
 }
 
@@ -195,6 +206,10 @@ __global__ void __launch_bounds__(256) attn_decode_combine_kernel(const DecodePa
   const int i = row % p.Tq, h = (row / p.Tq) % p.H, b = row / (p.Tq * p.H);
   const int G = p.H / p.Hkv, hk = h / G, r = (h % G) * p.Tq + i;
   const size_t base = static_cast<size_t>(b) * p.Hkv + hk;
+  const size_t n_part = static_cast<size_t>(p.B) * p.Hkv * p.n_split * p.R;  // partial rows
+  if (!ATTN_IN_RANGE((base * p.n_split) * p.R + r, static_cast<size_t>(p.n_split - 1) * p.R + 1, n_part,
+                     kSiteChkDecComb, &g_device_error))
+    return;  // every partial row of this output (s = 0 .. n_split - 1) must lie in the workspace
   float m = -INFINITY;
   for (int s = 0; s < p.n_split; ++s) m = fmaxf(m, p.part_ml[((base * p.n_split + s) * p.R + r) * 2]);
   float l = 0.f;
@@ -217,9 +232,12 @@ __global__ void __launch_bounds__(256) attn_decode_combine_kernel(const DecodePa
   uint2 out;
   out.x = sm100::pack_bf16x2(o4.x * inv, o4.y * inv);
   out.y = sm100::pack_bf16x2(o4.z * inv, o4.w * inv);
-  reinterpret_cast<uint2*>(p.o + ((static_cast<size_t>(b) * p.Tq + i) * p.H + h) * 128)[lane] = out;
-  if (lane == 0)
-    p.lse[(static_cast<size_t>(b) * p.H + h) * p.Tq + i] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+  const size_t o_off = ((static_cast<size_t>(b) * p.Tq + i) * p.H + h) * 128;
+  if (ATTN_IN_RANGE(o_off + lane * 4, 4, static_cast<size_t>(p.B) * p.Tq * p.H * 128, kSiteChkDecO, &g_device_error))
+    reinterpret_cast<uint2*>(p.o + o_off)[lane] = out;
+  const size_t lse_i = (static_cast<size_t>(b) * p.H + h) * p.Tq + i;
+  if (lane == 0 && ATTN_IN_RANGE(lse_i, 1, static_cast<size_t>(p.B) * p.H * p.Tq, kSiteChkDecLse, &g_device_error))
+    p.lse[lse_i] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
 }
 
 }  // namespace attn

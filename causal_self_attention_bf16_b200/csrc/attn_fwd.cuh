@@ -656,8 +656,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             *reinterpret_cast<uint4*>(box + sw128_offset(row, cc * 4 + ch)) = v;
           }
         }
-        if (g == 0 && qrow < p.T)
-          p.lse[static_cast<size_t>(it.bh) * p.T + qrow] = (m_f + __log2f(l_row)) * 0.69314718055994531f;
+        const size_t lse_i = static_cast<size_t>(it.bh) * p.T + qrow;
+        if (g == 0 && qrow < p.T &&
+            ATTN_IN_RANGE(lse_i, 1, static_cast<size_t>(p.B) * p.H * p.T, kSiteChkFwdLse, &g_device_error))
+          p.lse[lse_i] = (m_f + __log2f(l_row)) * 0.69314718055994531f;
       }
       // The staged rows go to the store warp; both groups have read O (the next item's first PV overwrites
       // it) and agree on whether to go on.

@@ -25,6 +25,12 @@
 #include "attn.h"
 #include "attn_errors.h"
 
+namespace attn {
+// This unit's device error word (kind 2 = an address check of the debug build failed, site in the higher bits).
+__device__ uint32_t g_rope_error;
+}  // namespace attn
+using attn::g_rope_error;
+
 namespace {
 
 constexpr int kRopeThreads = 256;
@@ -123,6 +129,25 @@ __device__ __forceinline__ void partner(const uint4& raw, const float (&v)[8], f
   }
 }
 
+// Debug builds (-DATTN_DEBUG) check each row chunk's address against the rows the host passed before the access;
+// a failed check records kind 2 (out of range) with its site in this unit's own device error word (the
+// attention kernels' word lives in another translation unit; attn_get_device_error ORs the two) and the access
+// is skipped. In the release build the check is the constant true.
+constexpr uint32_t kRopeSiteLoad = 0x91, kRopeSiteStore = 0x92;
+__device__ __forceinline__ bool row_ok(const RopeParams& p, int h, long long P, int c, uint32_t site) {
+#ifdef ATTN_DEBUG
+  const bool is_q = h < p.heads[0];
+  const long long nh = is_q ? p.heads[0] : p.heads[1];
+  const long long off = (P * nh + (is_q ? h : h - p.heads[0])) * 128 + 8 * c;
+  if (P >= 0 && h >= 0 && off >= 0 && off + 8 <= p.n_pos * nh * 128) return true;
+  atomicOr(&g_rope_error, 2u | (site << 8));
+  return false;
+#else
+  (void)p, (void)h, (void)P, (void)c, (void)site;
+  return true;
+#endif
+}
+
 __device__ __forceinline__ double position(const RopeParams& p, long long P) {
   const int b = static_cast<int>(P / p.T);
   const long long t = P - static_cast<long long>(b) * p.T;
@@ -151,7 +176,9 @@ __global__ void __launch_bounds__(kRopeThreads, 4) qk_norm_rope_kernel(RopeParam
 #pragma unroll
       for (int u = 0; u < kRopeUnroll; ++u) {
         const bool live = valid && h0 + u < rows;
-        raw[u] = live ? *reinterpret_cast<const uint4*>(row_ptr(p, p.x[0], p.x[1], h0 + u, P, c)) : kZero4;
+        raw[u] = live && row_ok(p, h0 + u, P, c, kRopeSiteLoad)
+                     ? *reinterpret_cast<const uint4*>(row_ptr(p, p.x[0], p.x[1], h0 + u, P, c))
+                     : kZero4;
       }
 #pragma unroll
       for (int u = 0; u < kRopeUnroll; ++u) {
@@ -164,7 +191,8 @@ __global__ void __launch_bounds__(kRopeThreads, 4) qk_norm_rope_kernel(RopeParam
         partner<kHalf>(raw[u], x, px);
 #pragma unroll
         for (int j = 0; j < 8; ++j) y[j] = (x[j] * r) * cs[j] + sign_of<kHalf>(c, j) * (px[j] * r) * sn[j];
-        if (valid && h0 + u < rows) *reinterpret_cast<uint4*>(row_ptr(p, p.out[0], p.out[1], h0 + u, P, c)) = pack8(y);
+        if (valid && h0 + u < rows && row_ok(p, h0 + u, P, c, kRopeSiteStore))
+          *reinterpret_cast<uint4*>(row_ptr(p, p.out[0], p.out[1], h0 + u, P, c)) = pack8(y);
       }
     }
   }
@@ -188,8 +216,9 @@ __global__ void __launch_bounds__(kRopeThreads) qk_norm_rope_bwd_kernel(RopePara
 #pragma unroll
       for (int u = 0; u < kRopeUnroll; ++u) {
         const bool live = valid && h0 + u < rows;
-        xr[u] = live ? *reinterpret_cast<const uint4*>(row_ptr(p, p.x[0], p.x[1], h0 + u, P, c)) : kZero4;
-        gr[u] = live ? *reinterpret_cast<const uint4*>(row_ptr(p, p.g[0], p.g[1], h0 + u, P, c)) : kZero4;
+        const bool in = live && row_ok(p, h0 + u, P, c, kRopeSiteLoad);
+        xr[u] = in ? *reinterpret_cast<const uint4*>(row_ptr(p, p.x[0], p.x[1], h0 + u, P, c)) : kZero4;
+        gr[u] = in ? *reinterpret_cast<const uint4*>(row_ptr(p, p.g[0], p.g[1], h0 + u, P, c)) : kZero4;
       }
 #pragma unroll
       for (int u = 0; u < kRopeUnroll; ++u) {
@@ -210,7 +239,8 @@ __global__ void __launch_bounds__(kRopeThreads) qk_norm_rope_bwd_kernel(RopePara
         dot = sum16(dot) * (1.f / 128.f);
 #pragma unroll
         for (int j = 0; j < 8; ++j) g[j] = r * (g[j] - (x[j] * r) * dot);
-        if (valid && h0 + u < rows) *reinterpret_cast<uint4*>(row_ptr(p, p.out[0], p.out[1], h0 + u, P, c)) = pack8(g);
+        if (valid && h0 + u < rows && row_ok(p, h0 + u, P, c, kRopeSiteStore))
+          *reinterpret_cast<uint4*>(row_ptr(p, p.out[0], p.out[1], h0 + u, P, c)) = pack8(g);
       }
     }
   }
@@ -338,3 +368,14 @@ attn_status attn_qk_norm_rope_bwd(const void* q, const void* k, const void* dq_o
 }
 
 }  // extern "C"
+
+namespace attn {
+// Read and clear this unit's device error word (synchronous; the caller has synchronised the device).
+int rope_error_word(uint32_t* word) {
+  return static_cast<int>(cudaMemcpyFromSymbol(word, g_rope_error, sizeof(uint32_t)));
+}
+int rope_error_clear() {
+  const uint32_t zero = 0;
+  return static_cast<int>(cudaMemcpyToSymbol(g_rope_error, &zero, sizeof(uint32_t)));
+}
+}  // namespace attn

@@ -17,7 +17,23 @@ namespace sm100 {
 // ---------------------------------------------------------------------------------------------------------
 // Error reporting shared with the host (see attn_get_device_error in include/attn.h).
 // Bits: low 8 bits = error kind, next bits = where (kernel-specific site id).
-enum : uint32_t { DEV_ERR_TIMEOUT = 1u };
+enum : uint32_t { DEV_ERR_TIMEOUT = 1u, DEV_ERR_BOUNDS = 2u };
+
+// Debug builds (-DATTN_DEBUG, libattn_debug.so) check every plain-address access -- the ones no tensor map
+// bounds -- before it is made: `off` .. `off + len` (in elements) must lie inside the `n` elements the host
+// passed for that array. A failed check records DEV_ERR_BOUNDS | (site << 8) in *err and the caller skips the
+// access. In the release build the check is the constant true and costs nothing.
+ATTN_DEVICE_INLINE bool range_ok(uint64_t off, uint64_t len, uint64_t n, uint32_t site, uint32_t* err) {
+  if (off <= n && len <= n - off) return true;
+  atomicOr(err, DEV_ERR_BOUNDS | (site << 8));
+  return false;
+}
+#ifdef ATTN_DEBUG
+#define ATTN_IN_RANGE(off, len, n, site, err) \
+  (::sm100::range_ok(static_cast<uint64_t>(off), static_cast<uint64_t>(len), static_cast<uint64_t>(n), (site), (err)))
+#else
+#define ATTN_IN_RANGE(off, len, n, site, err) (true)
+#endif
 
 ATTN_DEVICE_INLINE uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

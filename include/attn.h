@@ -44,7 +44,8 @@ typedef enum {
   ATTN_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned */
   ATTN_ERR_CUDA = 4,         /* a CUDA runtime/driver call or a launch failed; see attn_last_cuda_error() */
   ATTN_ERR_TIMEOUT = 5,      /* a kernel gave up on a bounded wait (reported by attn_get_device_error) */
-  ATTN_ERR_WORKSPACE = 6     /* backward workspace missing or smaller than attn_bwd_workspace_bytes() */
+  ATTN_ERR_WORKSPACE = 6,    /* backward workspace missing or smaller than attn_bwd_workspace_bytes() */
+  ATTN_ERR_BOUNDS = 7        /* debug build: a kernel's address check failed (reported by attn_get_device_error) */
 } attn_status;
 
 /* Version of this ABI; bumped on any incompatible change of a signature or of a buffer layout
@@ -225,9 +226,11 @@ attn_status attn_qk_norm_rope_bwd(const void* q, const void* k, const void* dq_o
                                   float rope_base, float eps, int pairing, void* stream);
 
 /*
- * Device-side error word shared by the kernels of this library on the current device: 0 if no kernel has
- * given up on a bounded wait since the last clear; otherwise (site << 8) | 1. Synchronises the device.
- * Returns ATTN_ERR_TIMEOUT if the word is non-zero, ATTN_OK if it is zero, ATTN_ERR_CUDA on a CUDA error.
+ * Device-side error word of the kernels of this library on the current device since the last clear: 0, or the
+ * OR of (site << 8) | kind over what went wrong, kind 1 = a kernel gave up on a bounded wait, kind 2 = (debug
+ * build only) a kernel's address check failed and the access was skipped; the site bits name the wait or the
+ * check (diagnostic only). Synchronises the device. Returns ATTN_ERR_TIMEOUT if kind 1 is set, else
+ * ATTN_ERR_BOUNDS if the word is non-zero, ATTN_OK if it is zero, ATTN_ERR_CUDA on a CUDA error.
  */
 attn_status attn_get_device_error(uint32_t* word);
 
@@ -247,6 +250,18 @@ attn_status attn_set_wait_limit_ns(uint64_t limit_ns);
  * Used by the failure-detection test; never part of the attention path.
  */
 attn_status attn_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
+/*
+ * Debug build. libattn_debug.so is this library compiled with -DATTN_DEBUG: every kernel access through a plain
+ * address (the ones no TMA tensor map bounds: LSE/Delta rows, dQ accumulator reductions and conversion, the
+ * forward's LSE, the decode kernels' cache, partial and output rows, the prologue's rows) is first checked
+ * against the extent of its array; a failed check sets kind 2 in the device error word and skips the access.
+ * Same symbols, same results, slower. attn_is_debug_build() returns 1 in it, 0 in libattn.so.
+ * attn_selftest_bounds_check() launches one checked store past its array's declared extent (debug build: the
+ * check records site 0x7e and skips the store); in the release build it returns ATTN_ERR_UNSUPPORTED.
+ */
+int attn_is_debug_build(void);
+attn_status attn_selftest_bounds_check(void* stream);
 
 #ifdef __cplusplus
 }
