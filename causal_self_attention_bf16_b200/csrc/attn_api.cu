@@ -547,8 +547,9 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
 
 namespace {
 
-// Splits of the cache per (sequence, key/value head): enough CTAs for ~8 per SM of a 148-SM part (each holds
-// ~64 KB of loads in flight), each split at least kDecChunkKeys keys (a multiple of the 128-key block).
+// Splits of the cache per (sequence, key/value head): about 8 CTAs per SM of a 148-SM part in all (one is resident
+// per SM at a time, with its 224 KB ring; several waves even out the sequences' different lengths), each split
+// at least kDecChunkKeys keys (a multiple of the 128-key block).
 void decode_split(int B, int Hkv, int Tk, int* n_split, int* chunk) {
   const long long pairs = static_cast<long long>(B) * Hkv;
   long long want = (8 * 148 + pairs - 1) / pairs;
@@ -640,21 +641,28 @@ attn_status attn_decode_ex(const void* q, const void* k_cache, const void* v_cac
   p.part_o = static_cast<float*>(workspace);
   p.part_ml = static_cast<float*>(workspace) + rows * 128;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = g_wait_limit_ns;
+  CUtensorMap mk, mv;  // the caches as [B, Tk, H_kv, 128]: 128-key x 64-dim boxes
+  if ((st = make_map(&mk, k_cache, B, H_kv, Tk, attn::kDecKeys)) != ATTN_OK) return st;
+  if ((st = make_map(&mv, v_cache, B, H_kv, Tk, attn::kDecKeys)) != ATTN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * H_kv * p.n_split);
   cudaError_t e = cudaSuccess;
-  auto launch = [&](auto kernel, size_t smem_bytes) {
+  auto launch = [&](auto kernel, size_t smem_bytes, int threads) {
     static std::mutex mu;
     std::lock_guard<std::mutex> lock(mu);
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_bytes));
-    if (e == cudaSuccess) kernel<<<grid, attn::kDecThreads, smem_bytes, s>>>(p);
+    if (e == cudaSuccess) kernel<<<grid, threads, smem_bytes, s>>>(mk, mv, p);
   };
-  if (p.R <= 1) launch(attn::attn_decode_split_kernel<1>, attn::dec_smem_bytes<1>());
-  else if (p.R <= 2) launch(attn::attn_decode_split_kernel<2>, attn::dec_smem_bytes<2>());
-  else if (p.R <= 4) launch(attn::attn_decode_split_kernel<4>, attn::dec_smem_bytes<4>());
-  else if (p.R <= 8) launch(attn::attn_decode_split_kernel<8>, attn::dec_smem_bytes<8>());
-  else if (p.R <= 16) launch(attn::attn_decode_split_kernel<16>, attn::dec_smem_bytes<16>());
-  else launch(attn::attn_decode_split_kernel<32>, attn::dec_smem_bytes<32>());
+#define ATTN_DEC_LAUNCH(R) \
+  launch(attn::attn_decode_split_kernel<R>, attn::dec_smem_bytes<R>(), attn::dec_threads<R>())
+  if (p.R <= 1) ATTN_DEC_LAUNCH(1);
+  else if (p.R <= 2) ATTN_DEC_LAUNCH(2);
+  else if (p.R <= 4) ATTN_DEC_LAUNCH(4);
+  else if (p.R <= 8) ATTN_DEC_LAUNCH(8);
+  else if (p.R <= 16) ATTN_DEC_LAUNCH(16);
+  else ATTN_DEC_LAUNCH(32);
+#undef ATTN_DEC_LAUNCH
   if (e != cudaSuccess) return cuda_fail(e, "attn_decode_split_kernel attribute");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_decode_split_kernel launch");

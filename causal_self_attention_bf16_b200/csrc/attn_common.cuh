@@ -14,7 +14,7 @@ __device__ uint32_t g_device_error;
 enum : uint32_t {
   kSiteChkPrepIn = 0x81, kSiteChkPrepAcc = 0x82, kSiteChkPrepRow = 0x83, kSiteChkPrepLse = 0x84,
   kSiteChkDqIn = 0x85, kSiteChkDqOut = 0x86, kSiteChkBwdRows = 0x87, kSiteChkBwdReduce = 0x88,
-  kSiteChkFwdLse = 0x89, kSiteChkDecQ = 0x8a, kSiteChkDecK = 0x8b, kSiteChkDecV = 0x8c, kSiteChkDecPart = 0x8d,
+  kSiteChkFwdLse = 0x89, kSiteChkDecQ = 0x8a, kSiteChkDecPart = 0x8d,
   kSiteChkDecComb = 0x8e, kSiteChkDecO = 0x8f, kSiteChkDecLse = 0x90, kSiteChkSelftest = 0x7e
 };
 

@@ -10,12 +10,15 @@
 // The work is a stream over the cache, HBM-bound (a few FLOPs per byte of K/V), so it runs on CUDA cores:
 //   1. attn_decode_split_kernel: one CTA per (sequence, key/value head, chunk of the cache). The G = H / H_kv
 //      query heads of the group and their Tq new tokens (R = G * Tq rows) share every K and V row the CTA
-//      reads, so the cache is read once. Per block of 128 keys: each thread scores one key against all rows
-//      (its K row in registers, the rows in shared memory) while the V block streams into shared memory with
-//      16-byte coalesced loads, a warp per row updates the running max and sum (online softmax in base 2), and
-//      each thread accumulates one of the 128 output dimensions of every row from the V block. The chunk's
-//      unnormalised O, running max and sum go to a workspace. The kernel is instantiated for 1, 2, 4, 8, 16 and
-//      32 rows so that the row accumulators of small groups take few registers.
+//      reads, so the cache is read once. The cache streams through a three-stage shared-memory ring of
+//      128-key K and V blocks loaded by TMA (one thread issues four 16 KB boxes per block onto the stage's
+//      mbarrier), two blocks in flight while one is used; rows past a sequence's length are masked, never
+//      used. Per block: two or four threads score each key against all rows (a part of the dims each,
+//      shuffles to add), a warp per row updates the running max and sum (online softmax in base 2), and a
+//      thread per pair of output dimensions and slice of the block's keys accumulates O; the slices are added
+//      once per chunk.
+//      The chunk's unnormalised O, running max and sum go to a workspace. The kernel is instantiated for 1, 2,
+//      4, 8, 16 and 32 rows.
 //   2. attn_decode_combine_kernel: one warp per (sequence, query head, new token) merges the chunks by their
 //      log-sum-exp and writes o and lse.
 #pragma once
@@ -24,10 +27,17 @@
 
 namespace attn {
 
-constexpr int kDecThreads = 128;   // one thread per key of a block and per output dimension
-constexpr int kDecKeys = 128;      // keys per block
-constexpr int kDecMaxRows = 32;    // R = (H / H_kv) * Tq query rows per CTA, at most
-constexpr int kDecChunkKeys = 256; // keys per split of the cache, at least
+// Threads of the split kernel. Scoring takes kThreads / 128 threads per key, each over 128 / that dims; P V takes
+// a thread per pair of output dimensions and kThreads / 64-th of the block's keys. 256 for every group size:
+// 512 (four threads per key, eight key slices) measured 34 % slower on decode_d20 -- a row's softmax is one
+// warp's work, and more warps only wait longer at the block's barriers.
+template <int kRows>
+__host__ __device__ constexpr int dec_threads() { return 256; }
+constexpr int kDecKeys = 128;       // keys per block
+constexpr int kDecStages = 3;       // K/V blocks in the shared-memory ring (two in flight while one is used)
+constexpr int kDecMaxRows = 32;     // R = (H / H_kv) * Tq query rows per CTA, at most
+constexpr int kDecChunkKeys = 256;  // keys per split of the cache, at least
+constexpr uint32_t kDecBlockBytes = kDecKeys * 256;  // one K or V block: 128 keys x 128 dims, bf16
 
 struct DecodeParams {
   const __nv_bfloat16* q;      // [B, Tq, H, D]
@@ -41,22 +51,51 @@ struct DecodeParams {
   int B, H, Hkv, Tq, Tk, R, n_split, chunk;
   int window;                  // sliding window: query at position p sees keys p - window .. p; -1: none
   float scale_log2;            // scale * log2(e)
+  uint64_t timeout_ns;         // limit of any single wait
 };
 
-// Dynamic shared memory of the split kernel for up to kRows query rows: the rows (fp32, pre-scaled), the
-// block's scores, and the block's V rows (bf16).
+// Dynamic shared memory of the split kernel for up to kRows query rows (no static shared memory, so the block
+// starts 1024-byte aligned, as the 128-byte-swizzled TMA boxes need): the ring of (K block, V block) pairs, the
+// rows (fp32, pre-scaled), the block's scores, then P, the rows' running max, sum and rescale factor, and one
+// mbarrier per ring stage. 224 KB at kRows = 32.
 template <int kRows>
-constexpr size_t dec_smem_bytes() {
-  return kRows * 128 * 4 + kRows * kDecKeys * 4 + kDecKeys * 128 * 2;
+__host__ __device__ constexpr size_t dec_bar_offset() {  // the stage barriers, 8-byte aligned
+  return (kDecStages * 2 * kDecBlockBytes + 2 * kRows * 128 * 4 + 3 * kRows * 4 + 7) / 8 * 8;
 }
+template <int kRows>
+__host__ __device__ constexpr size_t dec_smem_bytes() {
+  return dec_bar_offset<kRows>() + kDecStages * 8 + 8;  // + the abort flag
+}
+static_assert(dec_smem_bytes<kDecMaxRows>() <= 232448, "decode split kernel exceeds the 227 KB shared-memory opt-in");
+
+// A K or V block is two TMA boxes of 64 dims x 128 keys (16 KB each, dims 0-63 then 64-127) in the 128-byte
+// swizzle: 16-byte chunk c of key j's 128-byte row of a box sits at chunk c ^ (j & 7). The scoring reads (a lane
+// pair per key, eight chunks each) and the P V reads (a warp over one 128-byte row) hit every bank evenly.
+__device__ __forceinline__ uint32_t dec_box_off(int j, int c) { return j * 128 + ((c ^ (j & 7)) << 4); }
+
+enum : uint32_t { kSiteDecFull = 0x31, kSiteDecDrain = 0x32 };
 
 template <int kRows>
-__global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const DecodeParams p) {
-  extern __shared__ float4 dec_smem[];
-  float (*qs)[128] = reinterpret_cast<float (*)[128]>(dec_smem);                  // query rows * scale*log2(e)
-  float (*sc)[kDecKeys] = reinterpret_cast<float (*)[kDecKeys]>(qs + kRows);      // scores, then P
-  __nv_bfloat16 (*vs)[128] = reinterpret_cast<__nv_bfloat16 (*)[128]>(sc + kRows); // the block's V rows
-  __shared__ float row_m[kRows], row_l[kRows], row_a[kRows];
+__global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel(
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
+  using namespace sm100;
+  constexpr int kThreads = dec_threads<kRows>();
+  constexpr int kPart = kThreads / kDecKeys;   // scoring threads per key (2 or 4), kDims = 128 / kPart dims each
+  constexpr int kDims = 128 / kPart;
+  constexpr int kSlices = kThreads / 64;       // P V: key slices of kSliceKeys keys (4 x 32 or 8 x 16)
+  constexpr int kSliceKeys = kDecKeys / kSlices;
+  extern __shared__ __align__(1024) uint8_t dec_smem[];
+  if (smem_u32(dec_smem) & 1023u) {  // the swizzled boxes need a 1024-byte aligned block
+    if (threadIdx.x == 0) atomicOr(&g_device_error, DEV_ERR_TIMEOUT | (kSiteDecFull << 8));
+    return;
+  }
+  float (*qs)[128] = reinterpret_cast<float (*)[128]>(dec_smem + kDecStages * 2 * kDecBlockBytes);
+  float (*sc)[kDecKeys] = reinterpret_cast<float (*)[kDecKeys]>(qs + kRows);  // scores, then P
+  float* row_m = reinterpret_cast<float*>(sc + kRows);
+  float* row_l = row_m + kRows;
+  float* row_a = row_l + kRows;
+  uint64_t* full = reinterpret_cast<uint64_t*>(dec_smem + dec_bar_offset<kRows>());
+  volatile int* abort = reinterpret_cast<volatile int*>(full + kDecStages);
 
   const int t = threadIdx.x, warp = t / 32, lane = t % 32;
   const int bhk = blockIdx.x / p.n_split, sp = blockIdx.x % p.n_split;
@@ -67,75 +106,111 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const De
   // window) to the end of the cache.
   const int start = p.window < 0 ? 0 : max(0, L - p.Tq - p.window);
   const int key_lo = start + sp * p.chunk, key_hi = min(L, key_lo + p.chunk);
-  const size_t row_stride = static_cast<size_t>(p.Hkv) * 128;   // elements between consecutive keys
-  const size_t n_q = static_cast<size_t>(p.B) * p.Tq * p.H * 128, n_kv = static_cast<size_t>(p.B) * p.Tk * row_stride;
+  const int nblk = key_hi > key_lo ? (key_hi - key_lo + kDecKeys - 1) / kDecKeys : 0;
+  const size_t n_q = static_cast<size_t>(p.B) * p.Tq * p.H * 128;
+  const uint64_t lim = p.timeout_ns;
+
+  if (t == 0) {
+    for (int st = 0; st < kDecStages; ++st) mbar_init(&full[st], 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // Block n's K and V into ring stage n % kDecStages: four TMA boxes, 64 KB on the stage's barrier. The tensor
+  // maps bound the copies (rows past the cache come as zeros); rows past a sequence's length are masked below.
+  const bool issuer = t == 0;
+  auto issue = [&](int n) {
+    if (issuer && n < nblk) {
+      const int kb = key_lo + n * kDecKeys;
+      uint8_t* ks = dec_smem + (n % kDecStages) * 2 * kDecBlockBytes;
+      uint64_t* bar = &full[n % kDecStages];
+      mbar_arrive_expect_tx(bar, 2 * kDecBlockBytes);
+      for (int c = 0; c < 2; ++c) {
+        tma_load_4d(ks + c * 16384, &tm_k, bar, c * 64, hk, kb, b);
+        tma_load_4d(ks + kDecBlockBytes + c * 16384, &tm_v, bar, c * 64, hk, kb, b);
+      }
+    }
+  };
+  if (issuer) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+#pragma unroll
+  for (int n = 0; n < kDecStages - 1; ++n) issue(n);
 
   // Row r = g * Tq + i: query head hk * G + g, new token i, which sees keys up to L - Tq + i.
-  for (int r = 0; r < R; ++r) {
-    const int g = r / p.Tq, i = r % p.Tq;
-    const size_t qi = ((static_cast<size_t>(b) * p.Tq + i) * p.H + hk * G + g) * 128 + t;
-    qs[r][t] = ATTN_IN_RANGE(qi, 1, n_q, kSiteChkDecQ, &g_device_error) ? __bfloat162float(p.q[qi]) * p.scale_log2
-                                                                         : 0.f;
+  for (int e = t; e < R * 128; e += kThreads) {
+    const int r = e / 128, d = e % 128, g = r / p.Tq, i = r % p.Tq;
+    const size_t qi = ((static_cast<size_t>(b) * p.Tq + i) * p.H + hk * G + g) * 128 + d;
+    qs[r][d] = ATTN_IN_RANGE(qi, 1, n_q, kSiteChkDecQ, &g_device_error) ? __bfloat162float(p.q[qi]) * p.scale_log2
+                                                                        : 0.f;
   }
   if (t < R) {
     row_m[t] = -INFINITY;
     row_l[t] = 0.f;
   }
-  float acc[kRows];
+  // P V: output dimensions 2 dp, 2 dp + 1 over keys [kSliceKeys kq, kSliceKeys (kq + 1)) of each block
+  const int dp = t & 63, kq = t >> 6;
+  float acc[kRows][2];
 #pragma unroll
-  for (int r = 0; r < kRows; ++r) acc[r] = 0.f;
-  __syncthreads();
+  for (int r = 0; r < kRows; ++r) acc[r][0] = acc[r][1] = 0.f;
 
-  for (int kb = key_lo; kb < key_hi; kb += kDecKeys) {
-    const int nk = min(kDecKeys, key_hi - kb);
-    const size_t kv_off = ((static_cast<size_t>(b) * p.Tk + kb) * p.Hkv + hk) * 128;  // key kb's row
-    const __nv_bfloat16* kbase = p.k + kv_off;
-    const __nv_bfloat16* vbase = p.v + kv_off;
-    // Issue this block's loads first: the thread's K row (16 x 16 bytes) and 16 of the V block's 16-byte
-    // chunks (coalesced: consecutive threads, consecutive chunks of a row), so ~64 KB per CTA are in flight.
-    uint4 kw[16], vw[16];
-#pragma unroll
-    for (int c = 0; c < 16; ++c)
-      kw[c] = t < nk && ATTN_IN_RANGE(kv_off + t * row_stride + c * 8, 8, n_kv, kSiteChkDecK, &g_device_error)
-                  ? reinterpret_cast<const uint4*>(kbase + t * row_stride)[c]
-                  : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const int idx = u * kDecThreads + t, row = idx / 16, c = idx % 16;
-      vw[u] = row < nk && ATTN_IN_RANGE(kv_off + row * row_stride + c * 8, 8, n_kv, kSiteChkDecV, &g_device_error)
-                  ? reinterpret_cast<const uint4*>(vbase + row * row_stride)[c]
-                  : make_uint4(0, 0, 0, 0);
+  int consumed = 0;  // blocks whose barrier phase this CTA has waited for
+  bool ok = true;
+  for (int n = 0; n < nblk; ++n) {
+    __syncthreads();  // block n-1's stage and the scores are no longer read: the stage takes block n + 2
+    issue(n + kDecStages - 1);
+    if (!mbar_wait_warp(&full[n % kDecStages], (n / kDecStages) & 1, abort, lim, &g_device_error, kSiteDecFull)) {
+      ok = false;
     }
-    // Scores of key kb + t against every row (keys past the block, or past a row's last key, are -inf).
-    for (int r = 0; r < R; ++r) {
-      const float4* q4 = reinterpret_cast<const float4*>(qs[r]);
-      float s0 = 0.f, s1 = 0.f;
+    if (!__syncthreads_and(ok)) {
+      ok = false;
+      break;
+    }
+    consumed = n + 1;
+    const int kb = key_lo + n * kDecKeys, nk = min(kDecKeys, key_hi - kb);
+    const uint8_t* ks = dec_smem + (n % kDecStages) * 2 * kDecBlockBytes;
+    const uint8_t* vs = ks + kDecBlockBytes;
+    {
+      // Scores of key j = t / kPart against every row: this thread takes dims [kDims h, kDims (h + 1)),
+      // h = t % kPart, and the key's threads (adjacent lanes) add their parts. Keys past the block, past the
+      // sequence or past a row's last key are -inf (selected, so whatever those rows of the cache hold never
+      // enters a score).
+      const int j = t / kPart, h = t % kPart;
+      const int box = (h * kDims) / 64, c0 = ((h * kDims) % 64) / 8;  // the part's first 16-byte chunk
+      uint4 kw[kDims / 8];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float4 qa = q4[2 * c], qb = q4[2 * c + 1];
-        const uint32_t w[4] = {kw[c].x, kw[c].y, kw[c].z, kw[c].w};
-        s0 = fmaf(qa.x, __uint_as_float(w[0] << 16), s0);
-        s1 = fmaf(qa.y, __uint_as_float(w[0] & 0xffff0000u), s1);
-        s0 = fmaf(qa.z, __uint_as_float(w[1] << 16), s0);
-        s1 = fmaf(qa.w, __uint_as_float(w[1] & 0xffff0000u), s1);
-        s0 = fmaf(qb.x, __uint_as_float(w[2] << 16), s0);
-        s1 = fmaf(qb.y, __uint_as_float(w[2] & 0xffff0000u), s1);
-        s0 = fmaf(qb.z, __uint_as_float(w[3] << 16), s0);
-        s1 = fmaf(qb.w, __uint_as_float(w[3] & 0xffff0000u), s1);
+      for (int c = 0; c < kDims / 8; ++c)
+        kw[c] = *reinterpret_cast<const uint4*>(ks + box * 16384 + dec_box_off(j, c0 + c));
+      for (int r = 0; r < R; ++r) {
+        const float4* q4 = reinterpret_cast<const float4*>(qs[r] + kDims * h);
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < kDims / 8; ++c) {
+          const float4 qa = q4[2 * c], qb = q4[2 * c + 1];
+          const uint32_t w[4] = {kw[c].x, kw[c].y, kw[c].z, kw[c].w};
+          s0 = fmaf(qa.x, __uint_as_float(w[0] << 16), s0);
+          s1 = fmaf(qa.y, __uint_as_float(w[0] & 0xffff0000u), s1);
+          s0 = fmaf(qa.z, __uint_as_float(w[1] << 16), s0);
+          s1 = fmaf(qa.w, __uint_as_float(w[1] & 0xffff0000u), s1);
+          s0 = fmaf(qb.x, __uint_as_float(w[2] << 16), s0);
+          s1 = fmaf(qb.y, __uint_as_float(w[2] & 0xffff0000u), s1);
+          s0 = fmaf(qb.z, __uint_as_float(w[3] << 16), s0);
+          s1 = fmaf(qb.w, __uint_as_float(w[3] & 0xffff0000u), s1);
+        }
+        float sj = s0 + s1;
+#pragma unroll
+        for (int o = 1; o < kPart; o <<= 1) sj += __shfl_xor_sync(0xffffffffu, sj, o);
+        if (h == 0) {
+          const int last = L - p.Tq + r % p.Tq;  // last key this row sees (its own position)
+          const bool seen = j < nk && kb + j <= last && (p.window < 0 || kb + j >= last - p.window);
+          sc[r][j] = seen ? sj : -INFINITY;
+        }
       }
-      const int last = L - p.Tq + r % p.Tq;  // last key this row sees (its own position)
-      const bool seen = t < nk && kb + t <= last && (p.window < 0 || kb + t >= last - p.window);
-      sc[r][t] = seen ? s0 + s1 : -INFINITY;
-    }
-    // The V block to shared memory (rows past the block are zeros, so P = 0 times them stays 0).
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const int idx = u * kDecThreads + t;
-      reinterpret_cast<uint4*>(vs)[idx] = vw[u];
     }
     __syncthreads();
     // Online softmax, a warp per row: block max, running max, exp2 in place, running sum, O's rescale factor.
-    for (int r = warp; r < R; r += kDecThreads / 32) {
+    for (int r = warp; r < R; r += kThreads / 32) {
       float x[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) x[e] = sc[r][lane * 4 + e];
@@ -162,35 +237,67 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(const De
       }
     }
     __syncthreads();
-    // O[r][t] = O[r][t] * a_r + sum_j P[r][j] V[j][t]: thread t is output dimension t.
+    // O[r][d] = O[r][d] * a_r + sum_j P[r][j] V[j][d] for this thread's two dims over its slice of the keys:
+    // one 4-byte load per key for V (a warp reads one 128-byte box row), P four keys at a time. V rows past
+    // the sequence's keys are taken as 0 (selected, not multiplied, so the cache's contents there do not
+    // matter), and their P is 0.
 #pragma unroll
     for (int r = 0; r < kRows; ++r)
-      if (r < R) acc[r] *= row_a[r];
-    for (int j0 = 0; j0 < nk; j0 += 8) {
-      float vv[8];
+      if (r < R) acc[r][0] *= row_a[r], acc[r][1] *= row_a[r];
+    const uint8_t* vbox = vs + (dp >> 5) * 16384;
+#pragma unroll 2
+    for (int j0 = kSliceKeys * kq; j0 < kSliceKeys * (kq + 1); j0 += 4) {
+      float v0[4], v1[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) vv[e] = __bfloat162float(vs[j0 + e][t]);
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(
+            *reinterpret_cast<const __nv_bfloat162*>(vbox + dec_box_off(j0 + e, (dp & 31) >> 2) + (dp & 3) * 4));
+        const bool in = j0 + e < nk;
+        v0[e] = in ? f.x : 0.f;
+        v1[e] = in ? f.y : 0.f;
+      }
 #pragma unroll
       for (int r = 0; r < kRows; ++r) {
         if (r < R) {
-          float a = acc[r];
+          const float4 pr = *reinterpret_cast<const float4*>(&sc[r][j0]);
+          const float pe[4] = {pr.x, pr.y, pr.z, pr.w};
+          float a0 = acc[r][0], a1 = acc[r][1];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) a = fmaf(sc[r][j0 + e], vv[e], a);  // P and V are 0 past the block
-          acc[r] = a;
+          for (int e = 0; e < 4; ++e) a0 = fmaf(pe[e], v0[e], a0), a1 = fmaf(pe[e], v1[e], a1);
+          acc[r][0] = a0;
+          acc[r][1] = a1;
         }
       }
     }
-    __syncthreads();  // the next block overwrites sc and vs
   }
+  // Blocks issued but not consumed (only after a failure: at most the failed block and the two after it) land
+  // before the CTA leaves.
+  if (t == 0) {
+    volatile int no_abort = 0;
+    for (int n = consumed; n < min(nblk, consumed + kDecStages); ++n)
+      mbar_wait(&full[n % kDecStages], (n / kDecStages) & 1, &no_abort, lim, &g_device_error, kSiteDecDrain);
+  }
+  __syncthreads();  // the ring is no longer read: it takes the key slices' accumulators
+  if (!ok) return;
 
-  // The chunk's partial result (an empty chunk leaves max -inf, sum 0, O 0).
+  // The chunk's partial result (an empty chunk leaves max -inf, sum 0, O 0): the key slices' accumulators of
+  // each dimension are added, then O, the running max and the sum go to the workspace.
+  float* red = reinterpret_cast<float*>(dec_smem);  // [kq][r][128]: 2 KB x kSlices x R, at most 64 KB of 192
+#pragma unroll
+  for (int r = 0; r < kRows; ++r)
+    if (r < R) *reinterpret_cast<float2*>(red + (kq * R + r) * 128 + 2 * dp) = make_float2(acc[r][0], acc[r][1]);
+  __syncthreads();
   const size_t n_part = static_cast<size_t>(p.B) * p.Hkv * p.n_split * R;  // partial rows
   const size_t part = (static_cast<size_t>(bhk) * p.n_split + sp) * R;      // this chunk's first one
   float* po = p.part_o + part * 128;
   if (ATTN_IN_RANGE(part, R, n_part, kSiteChkDecPart, &g_device_error)) {
+    for (int e = t; e < R * 128; e += kThreads) {
+      const int r = e / 128, dd = e % 128;
+      float sum = 0.f;
 #pragma unroll
-    for (int r = 0; r < kRows; ++r)
-      if (r < R) po[r * 128 + t] = acc[r];
+      for (int q = 0; q < kSlices; ++q) sum += red[(q * R + r) * 128 + dd];
+      po[r * 128 + dd] = sum;
+    }
     if (t < R) {
       float* pml = p.part_ml + (part + t) * 2;
       pml[0] = row_m[t];

@@ -31,8 +31,8 @@ ATTN_DEVICE_INLINE bool range_ok(uint64_t off, uint64_t len, uint64_t n, uint32_
 #ifdef ATTN_DEBUG
 #define ATTN_IN_RANGE(off, len, n, site, err) \
   (::sm100::range_ok(static_cast<uint64_t>(off), static_cast<uint64_t>(len), static_cast<uint64_t>(n), (site), (err)))
-#else
-#define ATTN_IN_RANGE(off, len, n, site, err) (true)
+#else  // the arguments are referenced (not evaluated), so extents computed only for the checks stay "used"
+#define ATTN_IN_RANGE(off, len, n, site, err) (static_cast<void>(sizeof((off) + (len) + (n))), true)
 #endif
 
 ATTN_DEVICE_INLINE uint32_t smem_u32(const void* p) {
@@ -213,6 +213,20 @@ ATTN_DEVICE_INLINE void tma_store_wait_all() { asm volatile("cp.async.bulk.wait_
 template <int N>
 ATTN_DEVICE_INLINE void tma_store_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// 16-byte asynchronous copy global -> shared through L2 only (cp.async.cg), tracked by this thread's cp.async
+// groups; with fill = false nothing is read and the 16 bytes are zeroed. Both addresses 16-byte aligned.
+ATTN_DEVICE_INLINE void cp_async_16(void* smem_dst, const void* gmem_src, bool fill) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src),
+               "r"(fill ? 16 : 0)
+               : "memory");
+}
+ATTN_DEVICE_INLINE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's most recent cp.async groups are still in flight.
+template <int N>
+ATTN_DEVICE_INLINE void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // Untiled bulk copy global -> shared; both addresses 16-byte aligned, bytes a multiple of 16.
