@@ -68,8 +68,8 @@ struct FwdParams {
 // both; "mc" barriers exist in both CTAs and are completed by the even CTA's multicast tcgen05.commit.
 struct FwdBarriers {
   uint64_t q_full;      // local: this CTA's Q tile landed
-  uint64_t q_tmem;      // local: this CTA's Q copied into its tensor memory (8 warps)
-  uint64_t q_ready;     // pair: both CTAs' Q in tensor memory (16 warps)
+  uint64_t q_tmem;      // local: this CTA's Q copied into its tensor memory (the 4 warps of one group)
+  uint64_t q_ready;     // pair: both CTAs' Q in tensor memory (8 warps)
   uint64_t o_staged;    // local: both softmax groups have staged the item's output in the Q buffer (8 warps)
   uint64_t q_free;      // local: the Q buffer's other use, staging an item's output for its TMA store, is over
   uint64_t k_full[kFwdStages], v_full[kFwdStages];    // pair: both halves of a K / V tile landed
@@ -80,6 +80,7 @@ struct FwdBarriers {
   uint64_t xchg[2];     // local: running max after tile j published in slot j%2 (4 warps)
   uint64_t pv_done[2];  // mc: PV(j) completed (barrier j%2): P is free, O holds tiles 0..j
   uint64_t o_final;     // mc: committed once after an item's last PV: the epilogue's wait
+  uint64_t s_done;      // mc: committed once after an item's last S: its Q in tensor memory is no longer read
   uint64_t drain;       // local (even CTA): every MMA done
   uint32_t tmem_base;
   int abort;
@@ -109,12 +110,14 @@ __device__ __forceinline__ int fwd_first_kv_tile(int qt, int window) {
   return window < 0 ? 0 : max(0, qt * kTile - window) / kTile;
 }
 
+// The host caps B * H * (query tiles) well below 2^31, so item indices (fewer than n_items plus one round of
+// pairs) fit in 32 bits and decode with 32-bit divisions.
 __device__ __forceinline__ bool fwd_item(int k, int n_items, int n_qp, FwdItem& it) {
-  const int G = static_cast<int>(gridDim.x) / 2, c = static_cast<int>(blockIdx.x) / 2;
-  const long long idx = static_cast<long long>(k) * G + ((k & 1) ? G - 1 - c : c);
-  if (idx >= n_items) return false;
-  it.bh = static_cast<int>(idx / n_qp);
-  it.qp = n_qp - 1 - static_cast<int>(idx % n_qp);
+  const unsigned G = gridDim.x / 2, c = blockIdx.x / 2;
+  const unsigned idx = static_cast<unsigned>(k) * G + ((k & 1) ? G - 1 - c : c);
+  if (idx >= static_cast<unsigned>(n_items)) return false;
+  it.bh = static_cast<int>(idx / static_cast<unsigned>(n_qp));
+  it.qp = n_qp - 1 - static_cast<int>(idx % static_cast<unsigned>(n_qp));
   return true;
 }
 
@@ -149,8 +152,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
-    mbar_init(&bars.q_tmem, 8);    // counts warps (each softmax warp copies its rows of one head-dim half)
-    mbar_init(&bars.q_ready, 16);  // the same arrivals from both CTAs
+    mbar_init(&bars.q_tmem, 4);    // counts warps (one softmax group copies both head-dim halves of its rows)
+    mbar_init(&bars.q_ready, 8);   // the same arrivals from both CTAs
     mbar_init(&bars.o_staged, 8);  // counts warps
     mbar_init(&bars.q_free, 1);
     for (int s = 0; s < kFwdStages; ++s) {
@@ -167,6 +170,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_init(&bars.pv_done[s], 1);
     }
     mbar_init(&bars.o_final, 1);
+    mbar_init(&bars.s_done, 1);
     mbar_init(&bars.drain, 1);
     bars.abort = misaligned ? 1 : 0;
     fence_barrier_init();
@@ -373,6 +377,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         while (jp < n_kv) {
           if (js < n_kv && s_ready(t0 + js)) {
             issue_s(t0 + js++);
+            if (js == n_kv && leader) mma_commit_pair(&bars.s_done, 3);  // the item's Q may be replaced
             t_idle = 0;
           } else if (jp < js && pv_ready(t0 + jp)) {
             issue_pv(t0 + jp, jp == 0);
@@ -418,22 +423,25 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float* xm = reinterpret_cast<float*>(smem + kFwdSmemXchg);  // [2 slots, by tile parity][128 rows]: running max
     float* xl = xm + 2 * 128;                                    // [2 groups][128 rows]: partial sums, at the end
     const bool tracer = (threadIdx.x & 127) == 64;               // one thread per group records trace events
-    // Q of item k goes to tensor memory, so S = Q K^T reads only K from shared memory. Group g copies
-    // head-dim box g of its row: word w of the row (head dims 2w, 2w+1) becomes TMEM column w, the A-operand
-    // layout. Each warp then arrives on this CTA's q_tmem and on the pair's q_ready.
+    // Q of item k goes to tensor memory, so S = Q K^T reads only K from shared memory. One group copies both
+    // head-dim boxes of its rows: word w of a row (head dims 2w, 2w+1) becomes TMEM column w, the A-operand
+    // layout. Each of its warps then arrives on this CTA's q_tmem and on the pair's q_ready.
     auto copy_q = [&](int k) -> bool {
       if (!mbar_wait_pair_warp(&bars.q_full, k & 1, abort, peer_abort, lim, &g_device_error, kSiteFwdSmQ)) return false;
-      uint32_t qw[32];
-      const uint8_t* box = smem + kFwdSmemQ + g * 16384;
+#pragma unroll 1
+      for (int box = 0; box < 2; ++box) {
+        uint32_t qw[32];
+        const uint8_t* src = smem + kFwdSmemQ + box * 16384;
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const uint4 v = *reinterpret_cast<const uint4*>(box + sw128_offset(row, ch));
-        qw[ch * 4 + 0] = v.x;
-        qw[ch * 4 + 1] = v.y;
-        qw[ch * 4 + 2] = v.z;
-        qw[ch * 4 + 3] = v.w;
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src + sw128_offset(row, ch));
+          qw[ch * 4 + 0] = v.x;
+          qw[ch * 4 + 1] = v.y;
+          qw[ch * 4 + 2] = v.z;
+          qw[ch * 4 + 3] = v.w;
+        }
+        tmem_st32(tmem + lane_base + kTmemQ + 32 * box, qw);
       }
-      tmem_st32(tmem + lane_base + kTmemQ + 32 * g, qw);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive_warp(&bars.q_tmem);
@@ -442,15 +450,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     };
     FwdItem it;
     bool have = fwd_item(0, n_items, n_qp, it);
-    bool ok = have ? copy_q(0) : true;
+    bool ok = have && g == 0 ? copy_q(0) : true;  // group 0 copies the first item's Q
     int t0 = 0;
     for (int k = 0; have; ++k) {
       int kt0, n_kv;
       fwd_item_tiles(it.qp, n_qt, p.window, kt0, n_kv);
       const int qt = 2 * it.qp + static_cast<int>(rank);  // this CTA's query tile
       const int qrow = qt * kTile + row;                   // this thread's query position
-      FwdItem next;
-      const bool have_next = fwd_item(k + 1, n_items, n_qp, next);
       float m = -INFINITY;  // running max (scale*log2(e) units, stale by < 2^8) after this group's last tile
       float l = 0.f;        // this group's partial row sum of exp2(c*S - m)
       for (int t = t0 + ((g - t0) & 1); ok && t < t0 + n_kv; t += 2) {
@@ -610,6 +616,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_arrive_warp_cluster(&bars.p_full[sb], 0);
         if (tracer) ATTN_TRACE_EVENT(5, t);
       }
+      // The next item, decoded here, where the wait for this item's last PV hides the arithmetic.
+      FwdItem next;
+      const bool have_next = fwd_item(k + 1, n_items, n_qp, next);
+      // The group without the item's last tile (it has finished its own tiles) copies the next item's Q into
+      // tensor memory once the item's last S MMA has completed, so the next item's first S tiles queue right
+      // behind this item's last PV instead of waiting for this epilogue. The copy reads the Q buffer before the
+      // epilogue's first barrier, after which both groups stage the output there.
+      if (ok && have_next && g == (((t0 + n_kv - 1) & 1) ^ 1))
+        ok = mbar_wait_pair_warp(&bars.s_done, k & 1, abort, peer_abort, lim, &g_device_error, kSiteFwdSmQ) &&
+             copy_q(k + 1);
       // Epilogue of item k. The final running max is the one published for the item's last tile; each group
       // brings its partial sum to it and the two are added. Every thread of both groups reaches the named
       // barriers, failed or not, and both leave the item loop on the same decision (a barrier reduction).
@@ -622,12 +638,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       bool o_ready = __all_sync(0xffffffffu, ok) &&
                      mbar_wait_pair_warp(&bars.o_final, k & 1, abort, peer_abort, lim, &g_device_error, kSiteFwdEpi);
       if (!o_ready) ok = false;
-      // Every MMA of this item has completed: the next item's Q replaces this one in tensor memory now, so
-      // its first S tiles are computed while this item's output is written.
-      if (ok && have_next) ok = copy_q(k + 1);
       // The Q buffer takes this item's output once the store of the previous item's output has read it (the
-      // next Q, loaded in between, implies that, but the last item has none). Each thread overwrites only the
-      // bytes of Q it has just copied (its row of box g).
+      // next Q, loaded in between, implies that, but the last item has none); the next Q was copied out of it
+      // before the barriers above.
       if (o_ready && k > 0 &&
           !mbar_wait_pair_warp(&bars.q_free, (k - 1) & 1, abort, peer_abort, lim, &g_device_error, kSiteFwdEpi)) {
         o_ready = false;
@@ -638,21 +651,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
         const float inv_l = 1.0f / l_row;
         // O / l -> bf16 -> this group's 64-column box of the Q buffer, in the 128-byte-swizzled layout of the
-        // TMA store. The thread writes exactly the bytes of Q it has just copied (its row of box g), so the
-        // copy and the staging need no barrier between them.
+        // TMA store.
         uint8_t* box = smem + kFwdSmemQ + g * 16384;
+        uint32_t o[2][32];  // both 32-column chunks of this group's half of O, loaded before one wait
+        tmem_ld32(tmem + lane_base + kTmemO + 64 * g, o[0]);
+        tmem_ld32(tmem + lane_base + kTmemO + 64 * g + 32, o[1]);
+        tmem_wait_ld();
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tmem + lane_base + kTmemO + 64 * g + cc * 32, o);
-          tmem_wait_ld();
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
+            const uint32_t* w = o[cc] + ch * 8;
             uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(o[ch * 8 + 0]) * inv_l, __uint_as_float(o[ch * 8 + 1]) * inv_l);
-            v.y = pack_bf16x2(__uint_as_float(o[ch * 8 + 2]) * inv_l, __uint_as_float(o[ch * 8 + 3]) * inv_l);
-            v.z = pack_bf16x2(__uint_as_float(o[ch * 8 + 4]) * inv_l, __uint_as_float(o[ch * 8 + 5]) * inv_l);
-            v.w = pack_bf16x2(__uint_as_float(o[ch * 8 + 6]) * inv_l, __uint_as_float(o[ch * 8 + 7]) * inv_l);
+            v.x = pack_bf16x2(__uint_as_float(w[0]) * inv_l, __uint_as_float(w[1]) * inv_l);
+            v.y = pack_bf16x2(__uint_as_float(w[2]) * inv_l, __uint_as_float(w[3]) * inv_l);
+            v.z = pack_bf16x2(__uint_as_float(w[4]) * inv_l, __uint_as_float(w[5]) * inv_l);
+            v.w = pack_bf16x2(__uint_as_float(w[6]) * inv_l, __uint_as_float(w[7]) * inv_l);
             *reinterpret_cast<uint4*>(box + sw128_offset(row, cc * 4 + ch)) = v;
           }
         }

@@ -12,8 +12,11 @@ work-item mixes and random interleavings it checks that
   * no parity wait can be fooled: when a wait for phase n of a barrier succeeds, phase n + 1 has not completed
     yet (a parity wait only sees the current phase's parity, so a waiter two phases behind would hang).
 
-A negative control (an MMA issue order, tried during development, that ran the S tiles of item k+2 before the
-last PVs of item k) must deadlock in the model.
+The group without an item's last tile copies the next item's Q into tensor memory as soon as the item's last S
+MMA has completed (s_done), so the next item's first S tiles queue right behind the item's last PV; the model
+also checks that the epilogue never stages the output over a Q that has not been copied yet. Negative controls:
+an MMA issue order tried during development (the S tiles of item k+2 before the last PVs of item k) must
+deadlock, and a Q copy that does not wait for s_done must be caught.
 """
 import random
 
@@ -40,9 +43,10 @@ class Model:
 
     def __init__(self, items):
         self.items = items
-        self.b = {"q_ready": Barrier(16)}
+        self.b = {"q_ready": Barrier(8)}
         for r in range(2):
-            for name, count in [("q_full", 1), ("q_tmem", 8), ("q_free", 1), ("o_staged", 8), ("o_final", 1)]:
+            for name, count in [("q_full", 1), ("q_tmem", 4), ("q_free", 1), ("o_staged", 8), ("o_final", 1),
+                                ("s_done", 1)]:
                 self.b[f"{name}{r}"] = Barrier(count)
             for s in range(STAGES):
                 for name in ("k_empty", "v_empty"):
@@ -57,6 +61,7 @@ class Model:
             for name in ("s_free", "p_full"):
                 self.b[f"{name}{s}"] = Barrier(8)
         self.named = {(w, r): [0, 0] for w in "ABC" for r in range(2)}  # passes of each named barrier, per group
+        self.q_copied = [-1, -1]  # per CTA: the last item whose Q is in tensor memory
         self.violations = []
 
     def wait(self, name, n):
@@ -131,6 +136,8 @@ def mma(m, order="dynamic"):
                 if js < n and s_ready(t0 + js):
                     issue_s(t0 + js)
                     js += 1
+                    if js == n:
+                        m.both("s_done")  # the item's Q in tensor memory is no longer read
                 else:
                     issue_pv(t0 + jp)
                     jp += 1
@@ -160,13 +167,15 @@ def mma(m, order="dynamic"):
             tp += 1
 
 
-def softmax_group(m, r, g):
-    def copy_q(k):
+def softmax_group(m, r, g, bug=None):
+    def copy_q(k):  # one group copies both head-dim halves of the item's Q into this CTA's tensor memory
         yield m.wait(f"q_full{r}", k)
+        m.q_copied[r] = k
         m.b[f"q_tmem{r}"].arrive(4)
         m.b["q_ready"].arrive(4)
 
-    yield from copy_q(0)
+    if g == 0:
+        yield from copy_q(0)
     t0 = 0
     for k, n in enumerate(m.items):
         have_next = k + 1 < len(m.items)
@@ -182,13 +191,20 @@ def softmax_group(m, r, g):
                 yield m.wait(f"pv_done{(t - 1) & 1}_{r}", (t - 1) // 2)
             m.b[f"p_full{g}"].arrive(4)
             t += 2
+        # the group without the item's last tile copies the next item's Q once the item's last S has completed
+        if have_next and g == ((t0 + n - 1) & 1) ^ 1:
+            if bug != "copy_before_last_s":
+                yield m.wait(f"s_done{r}", k)
+            elif m.b[f"s_done{r}"].done <= k:
+                m.violations.append(("next Q copied over a Q still read by this item's S", k))
+            yield from copy_q(k + 1)
         yield m.named_barrier("A", r, g, k)
         yield m.named_barrier("B", r, g, k)
         yield m.wait(f"o_final{r}", k)
-        if have_next:
-            yield from copy_q(k + 1)
         if k > 0:
             yield m.wait(f"q_free{r}", k - 1)
+        if have_next and m.q_copied[r] < k + 1:  # the staging below overwrites the Q buffer
+            m.violations.append(("output staged over a Q not yet copied", k))
         m.b[f"o_staged{r}"].arrive(4)
         yield m.named_barrier("C", r, g, k)
         t0 += n
@@ -200,14 +216,15 @@ def store_warp(m, r):
         m.b[f"q_free{r}"].arrive()
 
 
-def run(items, seed, order="dynamic"):
+def run(items, seed, order="dynamic", bug=None):
     """Random interleaving of the roles of both CTAs; returns (finished, violations)."""
     m = Model(items)
     rng = random.Random(seed)
     roles = {"mma": mma(m, order)}
     for r in range(2):
-        roles.update({f"k{r}": producer(m, r, True), f"v{r}": producer(m, r, False), f"g0_{r}": softmax_group(m, r, 0),
-                      f"g1_{r}": softmax_group(m, r, 1), f"store{r}": store_warp(m, r)})
+        roles.update({f"k{r}": producer(m, r, True), f"v{r}": producer(m, r, False),
+                      f"g0_{r}": softmax_group(m, r, 0, bug), f"g1_{r}": softmax_group(m, r, 1, bug),
+                      f"store{r}": store_warp(m, r)})
     waiting = {name: None for name in roles}
     alive = set(roles)
     while alive:
@@ -249,3 +266,11 @@ def test_model_catches_a_deadlocking_issue_order():
     deadlocks = sum(not run(random_items(rng), trial, order="stream")[0] for trial in range(300))
     assert deadlocks > 0
     assert not run([2, 1, 2], 0, order="stream")[0]
+
+
+def test_model_catches_a_q_copy_that_does_not_wait_for_the_last_s():
+    """Negative control: copying the next item's Q without waiting for the item's last S MMA can overwrite a Q
+    that an S MMA still reads."""
+    rng = random.Random(9)
+    caught = sum(bool(run(random_items(rng), trial, bug="copy_before_last_s")[1]) for trial in range(300))
+    assert caught > 0
