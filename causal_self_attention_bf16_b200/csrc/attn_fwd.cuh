@@ -15,12 +15,15 @@
 //     per-CTA TMA copies (no multicast) whose completion is counted on the even CTA's barriers.
 //   * persistent: the pairs walk work items (pair of query tiles, batch, head) in head-major order, so the
 //     K/V of the few heads in flight stay in L2; the rings run on across items.
-//   * in each CTA: warp 0 stages Q once per item and the K ring, warp 10 the V ring (four-deep), warp 1 (of
-//     the even CTA) issues the MMAs, warps 2..9, two groups of four, run the online softmax straight out of
+//   * in each CTA: warp 0 stages Q once per item and the K ring, warp 2 the V ring (four-deep), warp 1 (of
+//     the even CTA) issues the MMAs, warps 4..11, two groups of four, run the online softmax straight out of
 //     tensor memory, one thread per query row: group g takes KV tiles j = g, g+2, ..., and only the running
 //     row max passes between the groups (through shared memory), so one tile's exponentials overlap the next
 //     tile's load and max. A thread owns a whole row of S, so row max and row sum need no shuffles; O is
-//     rescaled lazily, only when the running max grows by more than 2^8; warp 11 writes the normalised O.
+//     rescaled lazily, only when the running max grows by more than 2^8; warp 3 writes the normalised O.
+//     The first warpgroup (warps 0..3) hands most of its registers to the two softmax warpgroups, whose
+//     threads hold a row of scores and its packed probabilities at once (setmaxnreg: 40 and 232 registers
+//     per thread against 168 at launch; 4 x 32 x 40 + 8 x 32 x 232 = 384 x 168, the launch's whole file).
 //   * the pair's last KV tile is the odd CTA's diagonal tile and lies wholly above the even CTA's diagonal:
 //     the even CTA masks all of it (P = 0) without computing exponentials.
 //
@@ -36,9 +39,16 @@ namespace attn {
 
 constexpr int kTile = 128;        // query rows per CTA and keys per KV tile
 constexpr int kHeadDim = 128;     // D
-constexpr int kFwdThreads = 384;  // warp 0 TMA (Q, K), warp 1 MMA, warps 2..9 two softmax groups, warp 10 TMA (V),
-                                  // warp 11 TMA store of O
-constexpr int kFwdWarpV = 10, kFwdWarpStore = 11;
+constexpr int kFwdThreads = 384;  // warp 0 TMA (Q, K), warp 1 MMA, warp 2 TMA (V), warp 3 TMA store of O,
+                                  // warps 4..11 two softmax groups
+constexpr int kFwdWarpV = 2, kFwdWarpStore = 3;
+// Registers per thread after the split (setmaxnreg): the launch gives each of the 384 threads 168 (the
+// launch bounds' limit); the producer warpgroup keeps 40 and the two softmax warpgroups take the rest.
+constexpr int kFwdRegsLaunch = 168, kFwdRegsProducer = 40, kFwdRegsSoftmax = 232;
+static_assert(4 * 32 * kFwdRegsProducer + 8 * 32 * kFwdRegsSoftmax == kFwdThreads * kFwdRegsLaunch,
+              "the register split must hand over exactly the launch's registers");
+static_assert(kFwdRegsLaunch * kFwdThreads <= 65536 && kFwdRegsLaunch % 8 == 0 && kFwdRegsLaunch <= 65536 / kFwdThreads,
+              "launch register count");
 constexpr int kFwdKRows = kTile / 2;  // keys of a KV tile staged by each CTA of the pair
 
 // Shared-memory layout of the forward kernel (offsets from a 1024-byte aligned base; the same in both CTAs).
@@ -197,232 +207,238 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   if (*abort) {
     // nothing was issued
-  } else if (warp == 0 || warp == kFwdWarpV) {
-    // ------------------------------------------------------------------ TMA producers (both CTAs)
-    // Warp 0 stages Q and this CTA's half of every K tile, warp 10 its half of every V tile. Each walks its
-    // loop warp-uniformly (addresses and coordinates stay in uniform registers); one elected lane issues. The
-    // even CTA's lane also arms the pair's full barrier with the bytes of both halves.
-    const bool is_k = warp == 0;
-    const bool leader = elect_one();
-    const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
-    uint64_t* full = is_k ? bars.k_full : bars.v_full;
-    uint64_t* empty = is_k ? bars.k_empty : bars.v_empty;
-    uint8_t* ring = smem + (is_k ? kFwdSmemK : kFwdSmemV);
-    if (leader) {
-      tma_prefetch_desc(tm);
-      if (is_k) tma_prefetch_desc(&tm_q);
-    }
-    int issued[kFwdStages];
-    for (int s = 0; s < kFwdStages; ++s) issued[s] = -1;
-    int q_issued = -1;
-    int t0 = 0;  // running KV tile count: ring slot t % kFwdStages, phase (t / kFwdStages) & 1
-    FwdItem it;
-    for (int k = 0; fwd_item(k, n_items, n_qp, it); ++k) {
-      const int b = it.bh / p.H, h = it.bh % p.H;
-      int kt0, n_kv;
-      fwd_item_tiles(it.qp, n_qt, p.window, kt0, n_kv);
-      const int hk = h / (p.H / p.Hkv);  // grouped-query attention: the group's key/value head
-      if (is_k) {
-        // One Q buffer, which also stages each item's output for its TMA store. Q(1) may go in once Q(0) is in
-        // tensor memory; Q(k), k >= 2, once item k-2's output has been read out of the buffer by its store
-        // (which follows the copy of Q(k-1) into tensor memory in the same epilogue).
-        if (k == 1 && !mbar_wait_pair_warp(&bars.q_tmem, 0, abort, peer_abort, lim, &g_device_error, kSiteFwdProdQ))
-          break;
-        if (k >= 2 &&
-            !mbar_wait_pair_warp(&bars.q_free, (k - 2) & 1, abort, peer_abort, lim, &g_device_error, kSiteFwdProdQ))
-          break;
-        if (leader) {
-          mbar_arrive_expect_tx(&bars.q_full, 2 * 16384);
-          for (int c = 0; c < 2; ++c)
-            tma_load_4d(smem + kFwdSmemQ + c * 16384, &tm_q, &bars.q_full, c * 64, h,
-                        (2 * it.qp + static_cast<int>(rank)) * kTile, b);
-        }
-        q_issued = k;
-      }
-      bool ok = true;
-      for (int j = 0; j < n_kv; ++j) {
-        const int t = t0 + j, s = t % kFwdStages;
-        if (t >= kFwdStages &&
-            !mbar_wait_pair_warp(&empty[s], ((t - kFwdStages) / kFwdStages) & 1, abort, peer_abort, lim,
-                                 &g_device_error, is_k ? kSiteFwdProdKEmpty : kSiteFwdProdVEmpty)) {
-          ok = false;
-          break;
-        }
-        if (leader) {
-          if (is_lead) mbar_arrive_expect_tx(&full[s], 2 * kFwdSlot);
-          const uint32_t bar = mapa_shared(&full[s], 0);
-          const int kt = kt0 + j;
-          if (is_k) {  // keys [kt*128 + 64r, +64), both head-dim boxes
-            for (int c = 0; c < 2; ++c)
-              tma_load_4d_pair(ring + s * kFwdSlot + c * 8192, tm, bar, c * 64, hk,
-                               kt * kTile + kFwdKRows * static_cast<int>(rank), b);
-            ATTN_TRACE_EVENT(1, t);
-          } else {     // all 128 keys, head dimensions [64r, 64r+64)
-            tma_load_4d_pair(ring + s * kFwdSlot, tm, bar, 64 * static_cast<int>(rank), hk, kt * kTile, b);
-          }
-        }
-        issued[s] = t;
-      }
-      if (!ok) break;
-      t0 += n_kv;
-    }
-    if (*abort) {
-      // Let every copy this CTA started land before its shared memory is released. The K/V halves count on
-      // the even CTA's barriers, which the even CTA drains; this CTA's own Q copy counts here.
-      volatile int no_abort = 0;
-      if (q_issued >= 0) mbar_wait(&bars.q_full, q_issued & 1, &no_abort, lim, &g_device_error, kSiteFwdDrain);
-      if (is_lead) {
-        for (int s = 0; s < kFwdStages; ++s)
-          if (issued[s] >= 0)
-            mbar_wait(&full[s], (issued[s] / kFwdStages) & 1, &no_abort, lim, &g_device_error, kSiteFwdDrain);
-      } else {
-        const uint64_t t_end = global_timer_ns() + 50000;  // the odd CTA cannot see its halves land: 50 us
-        while (global_timer_ns() < t_end) {
-        }
-      }
-    }
-  } else if (warp == kFwdWarpStore) {
-    // ------------------------------------------------------------------ output store (both CTAs)
-    // Once both softmax groups have staged an item's output in the Q buffer, one elected lane writes it with
-    // two TMA stores (rows past T are clipped; a tile wholly past T is not stored) and frees the buffer for
-    // the next Q as soon as the stores have read it.
-    const bool leader = elect_one();
-    if (leader) tma_prefetch_desc(&tm_o);
-    FwdItem it;
-    for (int k = 0; fwd_item(k, n_items, n_qp, it); ++k) {
-      if (!mbar_wait_pair_warp(&bars.o_staged, k & 1, abort, peer_abort, lim, &g_device_error, kSiteFwdStore)) break;
-      if (__any_sync(0xffffffffu, *abort != 0)) break;  // warp-uniform: the loop ends in a __syncwarp
-      const int qt = 2 * it.qp + static_cast<int>(rank);
-      if (leader) {
-        if (qt < n_qt) {
-          for (int c = 0; c < 2; ++c)
-            tma_store_4d(&tm_o, smem + kFwdSmemQ + c * 16384, c * 64, it.bh % p.H, qt * kTile, it.bh / p.H);
-          tma_store_commit();
-          tma_store_wait_read_all();
-        }
-        mbar_arrive(&bars.q_free);
-      }
-      __syncwarp();
-    }
-    if (leader) tma_store_wait_all();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer (even CTA only)
-    // The whole warp walks the schedule and computes the descriptors (warp-uniform, so they live in uniform
-    // registers); the lane elected once issues every tcgen05.mma and tcgen05.commit (a commit tracks the
-    // MMAs of the thread that issues it, so it must be the same lane throughout).
-    if (is_lead) {
+  } else if (warp < 4) {
+    // The producer warpgroup gives registers back before the softmax warpgroups claim them (every warp of a
+    // warpgroup executes the same setmaxnreg).
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kFwdRegsProducer) : "memory");
+    if (warp == 0 || warp == kFwdWarpV) {
+      // ------------------------------------------------------------------ TMA producers (both CTAs)
+      // Warp 0 stages Q and this CTA's half of every K tile, warp 2 its half of every V tile. Each walks its
+      // loop warp-uniformly (addresses and coordinates stay in uniform registers); one elected lane issues. The
+      // even CTA's lane also arms the pair's full barrier with the bytes of both halves.
+      const bool is_k = warp == 0;
       const bool leader = elect_one();
-      const uint32_t idesc_s = idesc_bf16_f32(256, 128, false, false);  // Q (TMEM) x K (K-major), M = 256
-      const uint32_t idesc_pv = idesc_bf16_f32(256, 128, false, true);  // P (TMEM) x V (MN-major), M = 256
-      // PV(t): O += P(t) V(t) (the first tile of an item overwrites O); P from tensor memory, V from ring slot
-      // t % kFwdStages: each CTA holds all 128 keys of its 64 output dimensions, one 16 KB box.
-      auto issue_pv = [&](int t, bool first) {
-        const int pb = t & 1, vs = t % kFwdStages;
-        if (leader) ATTN_TRACE_EVENT(15, t);
-        tc_fence_after();
-        const uint64_t dv = sdesc_sw128(smem_u32(smem + kFwdSmemV + vs * kFwdSlot), kFwdSlot, 1024);  // MN-major
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // K step kk: 16 keys = 2048 bytes further (128 in 16-byte units)
-          if (leader)
-            mma_ts_pair(tmem + kTmemO, tmem + kTmemP + kk * 8, dv + kk * 128, idesc_pv, (!first || kk > 0) ? 1u : 0u);
-        if (leader) {
-          mma_commit_pair(&bars.pv_done[pb], 3);
-          ATTN_TRACE_EVENT(3, t);
-          mma_commit_pair(&bars.v_empty[vs], 3);
-        }
-      };
-      // S(t) = Q K(t)^T into S buffer t%2. Each CTA holds 64 keys of the tile as two 8 KB boxes of 64 head
-      // dimensions.
-      auto issue_s = [&](int t) {
-        const int ks = t % kFwdStages, sb = t & 1;
-        if (leader) ATTN_TRACE_EVENT(14, t);
-        tc_fence_after();
-        const uint64_t dk = sdesc_sw128(smem_u32(smem + kFwdSmemK + ks * kFwdSlot), 16, 1024);  // K, K-major
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // K step kk: 16 head-dim columns = 8 TMEM columns of Q; for K the
-          // second 64-column box from kk = 4, 32 bytes per step within a box
-          const uint32_t koff = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
-          if (leader)
-            mma_ts_pair(tmem + kTmemS + sb * 128, tmem + kTmemQ + kk * 8, dk + koff, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        if (leader) {
-          mma_commit_pair(&bars.s_full[sb], 3);
-          ATTN_TRACE_EVENT(2, t);
-          mma_commit_pair(&bars.k_empty[ks], 3);
-        }
-      };
-      // Readiness tests (warp-uniform, non-blocking). S(t) needs its K tile and S buffer t%2 read out of S(t-2)
-      // in both CTAs; PV(t) needs P(t) from both CTAs and its V tile.
-      auto s_ready = [&](int t) {
-        const bool ok_s = t < 2 || mbar_test(&bars.s_free[t & 1], ((t - 2) >> 1) & 1);
-        return __all_sync(0xffffffffu, ok_s && mbar_test(&bars.k_full[t % kFwdStages], (t / kFwdStages) & 1));
-      };
-      auto pv_ready = [&](int t) {
-        return __all_sync(0xffffffffu, mbar_test(&bars.p_full[t & 1], (t >> 1) & 1) &&
-                                           mbar_test(&bars.v_full[t % kFwdStages], (t / kFwdStages) & 1));
-      };
-      bool ok = true;
-      int t0 = 0;
+      const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+      uint64_t* full = is_k ? bars.k_full : bars.v_full;
+      uint64_t* empty = is_k ? bars.k_empty : bars.v_empty;
+      uint8_t* ring = smem + (is_k ? kFwdSmemK : kFwdSmemV);
+      if (leader) {
+        tma_prefetch_desc(tm);
+        if (is_k) tma_prefetch_desc(&tm_q);
+      }
+      int issued[kFwdStages];
+      for (int s = 0; s < kFwdStages; ++s) issued[s] = -1;
+      int q_issued = -1;
+      int t0 = 0;  // running KV tile count: ring slot t % kFwdStages, phase (t / kFwdStages) & 1
       FwdItem it;
-      for (int k = 0; ok && fwd_item(k, n_items, n_qp, it); ++k) {
+      for (int k = 0; fwd_item(k, n_items, n_qp, it); ++k) {
+        const int b = it.bh / p.H, h = it.bh % p.H;
         int kt0, n_kv;
         fwd_item_tiles(it.qp, n_qt, p.window, kt0, n_kv);
-        // This item's Q is in both CTAs' tensor memory (copied once the previous item's MMAs had completed).
-        if (!mbar_wait_pair_warp(&bars.q_ready, k & 1, abort, peer_abort, lim, &g_device_error, kSiteFwdMmaQ)) break;
-        // Issue whichever MMA is ready, S first: the S tiles run ahead as far as the two S buffers allow, so
-        // a softmax group never waits for its scores behind a PV whose P is still being computed; the PVs go
-        // in tile order as their P arrives. The tensor cores execute in issue order.
-        int js = 0, jp = 0;  // next S and next PV of the item
-        uint64_t t_idle = 0;
-        while (jp < n_kv) {
-          if (js < n_kv && s_ready(t0 + js)) {
-            issue_s(t0 + js++);
-            if (js == n_kv && leader) mma_commit_pair(&bars.s_done, 3);  // the item's Q may be replaced
-            t_idle = 0;
-          } else if (jp < js && pv_ready(t0 + jp)) {
-            issue_pv(t0 + jp, jp == 0);
-            ++jp;
-            t_idle = 0;
-          } else {
-            // Nothing ready: bounded like every wait of the kernel.
-            const uint64_t now = global_timer_ns();
-            if (t_idle == 0) t_idle = now;
-            const bool give_up = __any_sync(0xffffffffu, *abort != 0 || now - t_idle > lim);
-            if (give_up) {
-              if (lane == 0 && !*abort) {
-                *abort = 1;
-                asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(peer_abort), "r"(1) : "memory");
-                atomicOr(&g_device_error, DEV_ERR_TIMEOUT | (kSiteFwdMmaS << 8));
-              }
-              ok = false;
-              break;
+        const int hk = h / (p.H / p.Hkv);  // grouped-query attention: the group's key/value head
+        if (is_k) {
+          // One Q buffer, which also stages each item's output for its TMA store. Q(1) may go in once Q(0) is in
+          // tensor memory; Q(k), k >= 2, once item k-2's output has been read out of the buffer by its store
+          // (which follows the copy of Q(k-1) into tensor memory in the same epilogue).
+          if (k == 1 && !mbar_wait_pair_warp(&bars.q_tmem, 0, abort, peer_abort, lim, &g_device_error, kSiteFwdProdQ))
+            break;
+          if (k >= 2 &&
+              !mbar_wait_pair_warp(&bars.q_free, (k - 2) & 1, abort, peer_abort, lim, &g_device_error, kSiteFwdProdQ))
+            break;
+          if (leader) {
+            mbar_arrive_expect_tx(&bars.q_full, 2 * 16384);
+            for (int c = 0; c < 2; ++c)
+              tma_load_4d(smem + kFwdSmemQ + c * 16384, &tm_q, &bars.q_full, c * 64, h,
+                          (2 * it.qp + static_cast<int>(rank)) * kTile, b);
+          }
+          q_issued = k;
+        }
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
+          const int t = t0 + j, s = t % kFwdStages;
+          if (t >= kFwdStages &&
+              !mbar_wait_pair_warp(&empty[s], ((t - kFwdStages) / kFwdStages) & 1, abort, peer_abort, lim,
+                                   &g_device_error, is_k ? kSiteFwdProdKEmpty : kSiteFwdProdVEmpty)) {
+            ok = false;
+            break;
+          }
+          if (leader) {
+            if (is_lead) mbar_arrive_expect_tx(&full[s], 2 * kFwdSlot);
+            const uint32_t bar = mapa_shared(&full[s], 0);
+            const int kt = kt0 + j;
+            if (is_k) {  // keys [kt*128 + 64r, +64), both head-dim boxes
+              for (int c = 0; c < 2; ++c)
+                tma_load_4d_pair(ring + s * kFwdSlot + c * 8192, tm, bar, c * 64, hk,
+                                 kt * kTile + kFwdKRows * static_cast<int>(rank), b);
+              ATTN_TRACE_EVENT(1, t);
+            } else {     // all 128 keys, head dimensions [64r, 64r+64)
+              tma_load_4d_pair(ring + s * kFwdSlot, tm, bar, 64 * static_cast<int>(rank), hk, kt * kTile, b);
             }
           }
+          issued[s] = t;
         }
-        if (ok && leader) mma_commit_pair(&bars.o_final, 3);
+        if (!ok) break;
         t0 += n_kv;
       }
-      // Drain: wait until every MMA the leader issued has completed before tensor memory is released.
-      if (leader) mma_commit_pair(&bars.drain, 1);
-      volatile int no_abort = 0;
-      mbar_wait(&bars.drain, 0, &no_abort, lim, &g_device_error, kSiteFwdDrain);
+      if (*abort) {
+        // Let every copy this CTA started land before its shared memory is released. The K/V halves count on
+        // the even CTA's barriers, which the even CTA drains; this CTA's own Q copy counts here.
+        volatile int no_abort = 0;
+        if (q_issued >= 0) mbar_wait(&bars.q_full, q_issued & 1, &no_abort, lim, &g_device_error, kSiteFwdDrain);
+        if (is_lead) {
+          for (int s = 0; s < kFwdStages; ++s)
+            if (issued[s] >= 0)
+              mbar_wait(&full[s], (issued[s] / kFwdStages) & 1, &no_abort, lim, &g_device_error, kSiteFwdDrain);
+        } else {
+          const uint64_t t_end = global_timer_ns() + 50000;  // the odd CTA cannot see its halves land: 50 us
+          while (global_timer_ns() < t_end) {
+          }
+        }
+      }
+    } else if (warp == kFwdWarpStore) {
+      // ------------------------------------------------------------------ output store (both CTAs)
+      // Once both softmax groups have staged an item's output in the Q buffer, one elected lane writes it with
+      // two TMA stores (rows past T are clipped; a tile wholly past T is not stored) and frees the buffer for
+      // the next Q as soon as the stores have read it.
+      const bool leader = elect_one();
+      if (leader) tma_prefetch_desc(&tm_o);
+      FwdItem it;
+      for (int k = 0; fwd_item(k, n_items, n_qp, it); ++k) {
+        if (!mbar_wait_pair_warp(&bars.o_staged, k & 1, abort, peer_abort, lim, &g_device_error, kSiteFwdStore)) break;
+        if (__any_sync(0xffffffffu, *abort != 0)) break;  // warp-uniform: the loop ends in a __syncwarp
+        const int qt = 2 * it.qp + static_cast<int>(rank);
+        if (leader) {
+          if (qt < n_qt) {
+            for (int c = 0; c < 2; ++c)
+              tma_store_4d(&tm_o, smem + kFwdSmemQ + c * 16384, c * 64, it.bh % p.H, qt * kTile, it.bh / p.H);
+            tma_store_commit();
+            tma_store_wait_read_all();
+          }
+          mbar_arrive(&bars.q_free);
+        }
+        __syncwarp();
+      }
+      if (leader) tma_store_wait_all();
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer (even CTA only)
+      // The whole warp walks the schedule and computes the descriptors (warp-uniform, so they live in uniform
+      // registers); the lane elected once issues every tcgen05.mma and tcgen05.commit (a commit tracks the
+      // MMAs of the thread that issues it, so it must be the same lane throughout).
+      if (is_lead) {
+        const bool leader = elect_one();
+        const uint32_t idesc_s = idesc_bf16_f32(256, 128, false, false);  // Q (TMEM) x K (K-major), M = 256
+        const uint32_t idesc_pv = idesc_bf16_f32(256, 128, false, true);  // P (TMEM) x V (MN-major), M = 256
+        // PV(t): O += P(t) V(t) (the first tile of an item overwrites O); P from tensor memory, V from ring slot
+        // t % kFwdStages: each CTA holds all 128 keys of its 64 output dimensions, one 16 KB box.
+        auto issue_pv = [&](int t, bool first) {
+          const int pb = t & 1, vs = t % kFwdStages;
+          if (leader) ATTN_TRACE_EVENT(15, t);
+          tc_fence_after();
+          const uint64_t dv = sdesc_sw128(smem_u32(smem + kFwdSmemV + vs * kFwdSlot), kFwdSlot, 1024);  // MN-major
+  #pragma unroll
+          for (int kk = 0; kk < 8; ++kk)  // K step kk: 16 keys = 2048 bytes further (128 in 16-byte units)
+            if (leader)
+              mma_ts_pair(tmem + kTmemO, tmem + kTmemP + kk * 8, dv + kk * 128, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+          if (leader) {
+            mma_commit_pair(&bars.pv_done[pb], 3);
+            ATTN_TRACE_EVENT(3, t);
+            mma_commit_pair(&bars.v_empty[vs], 3);
+          }
+        };
+        // S(t) = Q K(t)^T into S buffer t%2. Each CTA holds 64 keys of the tile as two 8 KB boxes of 64 head
+        // dimensions.
+        auto issue_s = [&](int t) {
+          const int ks = t % kFwdStages, sb = t & 1;
+          if (leader) ATTN_TRACE_EVENT(14, t);
+          tc_fence_after();
+          const uint64_t dk = sdesc_sw128(smem_u32(smem + kFwdSmemK + ks * kFwdSlot), 16, 1024);  // K, K-major
+  #pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {  // K step kk: 16 head-dim columns = 8 TMEM columns of Q; for K the
+            // second 64-column box from kk = 4, 32 bytes per step within a box
+            const uint32_t koff = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+            if (leader)
+              mma_ts_pair(tmem + kTmemS + sb * 128, tmem + kTmemQ + kk * 8, dk + koff, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          if (leader) {
+            mma_commit_pair(&bars.s_full[sb], 3);
+            ATTN_TRACE_EVENT(2, t);
+            mma_commit_pair(&bars.k_empty[ks], 3);
+          }
+        };
+        // Readiness tests (warp-uniform, non-blocking). S(t) needs its K tile and S buffer t%2 read out of S(t-2)
+        // in both CTAs; PV(t) needs P(t) from both CTAs and its V tile.
+        auto s_ready = [&](int t) {
+          const bool ok_s = t < 2 || mbar_test(&bars.s_free[t & 1], ((t - 2) >> 1) & 1);
+          return __all_sync(0xffffffffu, ok_s && mbar_test(&bars.k_full[t % kFwdStages], (t / kFwdStages) & 1));
+        };
+        auto pv_ready = [&](int t) {
+          return __all_sync(0xffffffffu, mbar_test(&bars.p_full[t & 1], (t >> 1) & 1) &&
+                                             mbar_test(&bars.v_full[t % kFwdStages], (t / kFwdStages) & 1));
+        };
+        bool ok = true;
+        int t0 = 0;
+        FwdItem it;
+        for (int k = 0; ok && fwd_item(k, n_items, n_qp, it); ++k) {
+          int kt0, n_kv;
+          fwd_item_tiles(it.qp, n_qt, p.window, kt0, n_kv);
+          // This item's Q is in both CTAs' tensor memory (copied once the previous item's MMAs had completed).
+          if (!mbar_wait_pair_warp(&bars.q_ready, k & 1, abort, peer_abort, lim, &g_device_error, kSiteFwdMmaQ)) break;
+          // Issue whichever MMA is ready, S first: the S tiles run ahead as far as the two S buffers allow, so
+          // a softmax group never waits for its scores behind a PV whose P is still being computed; the PVs go
+          // in tile order as their P arrives. The tensor cores execute in issue order.
+          int js = 0, jp = 0;  // next S and next PV of the item
+          uint64_t t_idle = 0;
+          while (jp < n_kv) {
+            if (js < n_kv && s_ready(t0 + js)) {
+              issue_s(t0 + js++);
+              if (js == n_kv && leader) mma_commit_pair(&bars.s_done, 3);  // the item's Q may be replaced
+              t_idle = 0;
+            } else if (jp < js && pv_ready(t0 + jp)) {
+              issue_pv(t0 + jp, jp == 0);
+              ++jp;
+              t_idle = 0;
+            } else {
+              // Nothing ready: bounded like every wait of the kernel.
+              const uint64_t now = global_timer_ns();
+              if (t_idle == 0) t_idle = now;
+              const bool give_up = __any_sync(0xffffffffu, *abort != 0 || now - t_idle > lim);
+              if (give_up) {
+                if (lane == 0 && !*abort) {
+                  *abort = 1;
+                  asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(peer_abort), "r"(1) : "memory");
+                  atomicOr(&g_device_error, DEV_ERR_TIMEOUT | (kSiteFwdMmaS << 8));
+                }
+                ok = false;
+                break;
+              }
+            }
+          }
+          if (ok && leader) mma_commit_pair(&bars.o_final, 3);
+          t0 += n_kv;
+        }
+        // Drain: wait until every MMA the leader issued has completed before tensor memory is released.
+        if (leader) mma_commit_pair(&bars.drain, 1);
+        volatile int no_abort = 0;
+        mbar_wait(&bars.drain, 0, &no_abort, lim, &g_device_error, kSiteFwdDrain);
+      }
     }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kFwdRegsSoftmax) : "memory");
     // ------------------------------------------------------------------ softmax / correction / epilogue
-    // Two warp groups take the KV tiles in turn: group g (warps 2..5 or 6..9) owns the tiles whose running
+    // Two warp groups take the KV tiles in turn: group g (warps 4..7 or 8..11) owns the tiles whose running
     // index t is g modulo 2, and S buffer g. A thread holds one query row of its tile (128 keys) in registers.
     // The online softmax is sequential only through the running max: the group publishes the max after its
     // tile in shared memory and the other group, which has already loaded and reduced the next tile, takes
     // it from there. So the exponentials of one tile overlap the load, max and exchange of the next, and two
     // softmax warps per SM sub-partition keep the MUFU and FMA pipes busy.
-    const int g = (warp - 2) >> 2;
+    const int g = (warp - 4) >> 2;
     const int quarter = warp & 3;           // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;    // query row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const float c = p.scale_log2;
     float* xm = reinterpret_cast<float*>(smem + kFwdSmemXchg);  // [2 slots, by tile parity][128 rows]: running max
     float* xl = xm + 2 * 128;                                    // [2 groups][128 rows]: partial sums, at the end
-    const bool tracer = (threadIdx.x & 127) == 64;               // one thread per group records trace events
+    const bool tracer = (threadIdx.x & 127) == 0;                // one thread per group records trace events
     // Q of item k goes to tensor memory, so S = Q K^T reads only K from shared memory. One group copies both
     // head-dim boxes of its rows: word w of a row (head dims 2w, 2w+1) becomes TMEM column w, the A-operand
     // layout. Each of its warps then arrives on this CTA's q_tmem and on the pair's q_ready.
