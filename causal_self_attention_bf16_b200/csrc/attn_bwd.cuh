@@ -15,9 +15,9 @@
 //        dV += P^T dO, dK += dS^T Q             (P^T, dS^T from tensor memory; dO, Q MN-major)
 //        dQ^T = K^T dS^T                        (both operands MN-major in shared memory)
 //      Two warp groups taking alternate query tiles (one thread per key row) turn S^T, dP^T into P^T, dS^T
-//      (exp2 against the stored LSE), then read their tile's dQ^T out of tensor memory, stage it in shared
-//      memory in the accumulator's layout and add it into the fp32 accumulator with one bulk reduction
-//      (cp.reduce.async.bulk .add.f32, 32 contiguous KB) on the async engine. dK, dV stay in tensor memory
+//      (exp2 against the stored LSE), then read their tile's dQ^T out of tensor memory and stage it in shared
+//      memory in the accumulator's layout; a reduction warp adds it into the fp32 accumulator with one bulk
+//      reduction (cp.reduce.async.bulk .add.f32, 32 contiguous KB) on the async engine. dK, dV stay in tensor memory
 //      for the whole walk; the groups stage them in shared memory and the K/V warp stores them by TMA while
 //      the groups go on with the next key tile.
 //   3. attn_bwd_dq_kernel: dQ = bf16(scale * accumulator) back in [B, T, H, D].
@@ -37,9 +37,9 @@ namespace attn {
 constexpr int kBwdQTile = 64;       // queries per inner tile
 constexpr int kBwdKTile = 128;      // keys per CTA
 constexpr int kBwdStages = 3;       // Q/dO/LSE/Delta ring depth
-constexpr int kBwdThreads = 352;    // warp 0 TMA (query tiles), warp 1 MMA, warps 2..9 two softmax/dQ
-                                    // groups, warp 10 TMA (K, V in; dV, dK out)
-constexpr int kBwdWarpKV = 10;
+constexpr int kBwdThreads = 384;    // warp 0 TMA (query tiles), warp 1 MMA, warps 2..9 two softmax/dQ
+                                    // groups, warp 10 TMA (K, V in; dV, dK out), warp 11 dQ reductions
+constexpr int kBwdWarpKV = 10, kBwdWarpReduce = 11;
 
 constexpr uint32_t kBwdSmemK = 0;                                 // 32 KB
 constexpr uint32_t kBwdSmemV = 32768;                             // 32 KB
@@ -205,8 +205,10 @@ struct BwdBarriers {
   uint64_t dq_full[2];   // dQ^T of buffer b ready
   uint64_t dq_empty[2];  // dQ^T read out: buffer b's last 64 columns free
   uint64_t b_done[2];    // dV, dK MMAs of the step in buffer b done (buffer's P^T, dS^T consumed)
+  uint64_t dq_staged[2];   // a step's dQ^T tile is staged for its reduction: [gs % 2], arrived by that step's
+                          // group leader after the group's staging barrier (one phase per step of that group)
   uint64_t stage_free[2];  // the dQ staging buffer has been read by the bulk reduction of a step: [gs % 2],
-                          // arrived by that step's group leader (one phase per step of that group)
+                          // arrived by the reduction warp (one phase per step of that group)
   uint64_t acc_done;     // every MMA of an item done: its dV, dK are final (one phase per item)
   uint64_t acc_free;     // dV, dK read out of tensor memory by the epilogue (8 warps, one phase per item)
   uint64_t dk_staged;    // an item's dK staged in the dS^T buffers for its store (4 warps, one phase per item)
@@ -214,6 +216,7 @@ struct BwdBarriers {
   uint64_t ds_read;      // an item's dK stores have read the dS^T buffers (one phase per item)
   uint64_t dq_read;      // an item's dV stores have read the dQ staging buffer (one phase per item)
   uint64_t drain;
+  float* red_dst[2];     // accumulator address of the tile staged for dq_staged[g], written before that arrival
   uint32_t tmem_base;
   int abort;
 };
@@ -225,7 +228,8 @@ static_assert(kBwdSmemAlloc <= 232448, "dK/dV kernel exceeds the 227 KB shared-m
 enum : uint32_t {
   kSiteBwdLayout = 0x40, kSiteBwdProdQEmpty = 0x41, kSiteBwdProdKV = 0x42, kSiteBwdMmaKV = 0x51, kSiteBwdMmaQ = 0x52,
   kSiteBwdMmaDqEmpty = 0x53, kSiteBwdMmaP = 0x54, kSiteBwdMmaAcc = 0x55, kSiteBwdSmS = 0x61, kSiteBwdSmQ = 0x62,
-  kSiteBwdSmEpi = 0x63, kSiteBwdSmEpiRead = 0x64, kSiteBwdKvEpi = 0x43, kSiteBwdDq = 0x71, kSiteBwdDrain = 0x72
+  kSiteBwdSmEpi = 0x63, kSiteBwdSmEpiRead = 0x64, kSiteBwdKvEpi = 0x43, kSiteBwdDq = 0x71, kSiteBwdDrain = 0x72,
+  kSiteBwdReduce = 0x73
 };
 
 // Work item k of this CTA: one 128-key tile of one key/value head. Items are ordered head-major with the
@@ -299,6 +303,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       mbar_init(&bars.dq_empty[s], 4);  // likewise
       mbar_init(&bars.b_done[s], 1);
     }
+    mbar_init(&bars.dq_staged[0], 1);
+    mbar_init(&bars.dq_staged[1], 1);
     mbar_init(&bars.stage_free[0], 1);
     mbar_init(&bars.stage_free[1], 1);
     mbar_init(&bars.acc_done, 1);
@@ -459,6 +465,39 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (v_issued >= 0) mbar_wait(&bars.v_full, v_issued & 1, &no_abort, lim, &g_device_error, kSiteBwdDrain);
       if (k_issued >= 0) mbar_wait(&bars.k_full, k_issued & 1, &no_abort, lim, &g_device_error, kSiteBwdDrain);
     }
+  } else if (warp == kBwdWarpReduce) {
+    // ------------------------------------------------------------------ dQ reductions
+    // Each step's dQ^T tile, staged by its softmax group in the accumulator's layout, is one contiguous 32 KB
+    // block of the fp32 accumulator: one bulk reduce-add on the async engine adds it in. This warp issues them
+    // in step order and waits for each to have read the staging buffer before handing the buffer on
+    // (stage_free), so no softmax warp ever stalls on that read.
+    const bool leader = elect_one();
+    const size_t acc_floats = static_cast<size_t>(p.B) * p.H * p.Tp * 128;
+    int gs = 0;
+    bool ok = true;
+    BwdItem it;
+    for (int k = 0; ok && bwd_item(k, p, it); ++k) {
+      const int ns = G * it.n;
+      for (int i = 0; i < ns; ++i, ++gs) {
+        const int g = gs & 1;
+        if (!mbar_wait_warp(&bars.dq_staged[g], (gs >> 1) & 1, abort, lim, &g_device_error, kSiteBwdReduce)) {
+          ok = false;
+          break;
+        }
+        if (leader) {
+          // the tile's 8192 accumulator floats (checked in the debug build; a failed check skips the reduction)
+          float* dst = bars.red_dst[g];
+          if (ATTN_IN_RANGE(static_cast<size_t>(dst - p.dq_acc), 8192, acc_floats, kSiteChkBwdReduce, &g_device_error))
+            bulk_reduce_add_f32(dst, smem + kBwdSmemDQ, 32768);
+          tma_store_commit();
+          tma_store_wait_read_all();  // the staging buffer has been read: hand it to the next step
+          mbar_arrive(&bars.stage_free[g]);
+          ATTN_TRACE_EVENT(7, gs);
+        }
+        __syncwarp();
+      }
+    }
+    if (leader) tma_store_wait_all();  // the reductions are complete before the CTA exits
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     // The whole warp walks the schedule and computes the descriptors (warp-uniform, so they live in uniform
@@ -716,15 +755,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           ok = false;
           break;
         }
-        if (group_leader) {
-          // the tile's 8192 accumulator floats (checked in the debug build; a failed check skips the reduction)
-          if (ATTN_IN_RANGE(static_cast<size_t>(acc_bh - p.dq_acc) + static_cast<size_t>(q0 >> 2) * 512, 8192,
-                            static_cast<size_t>(p.B) * p.H * p.Tp * 128, kSiteChkBwdReduce, &g_device_error))
-            bulk_reduce_add_f32(acc_bh + static_cast<size_t>(q0 >> 2) * 512, dq_stage, 32768);
-          tma_store_commit();
-          tma_store_wait_read_all();  // the staging buffer has been read: hand it to the next step
-          mbar_arrive(&bars.stage_free[g]);
-          ATTN_TRACE_EVENT(7, gs);
+        if (group_leader) {  // the reduction warp adds the staged tile into the accumulator
+          bars.red_dst[g] = acc_bh + static_cast<size_t>(q0 >> 2) * 512;
+          mbar_arrive(&bars.dq_staged[g]);
         }
         qi += 2;
         while (qi >= it.n) qi -= it.n, ++hq;
@@ -778,7 +811,6 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       it = nxt;
       have = have_next;
     }
-    if (group_leader) tma_store_wait_all();  // this group's reductions and stores are complete before exit
   }
 
   tc_fence_before();

@@ -29,8 +29,8 @@
 //
 // Tensor memory (512 columns per CTA, allocated for the pair): S double buffer [0,256) (buffer j%2 belongs to
 // the group of tile j), O [256,384), Q (bf16 pairs) [384,448), P (bf16 pairs) [448,512). The MMA thread issues
-// whichever MMA is ready, S first: S(j+2) as soon as S(j) has been read out in both CTAs and K(j+2) has landed,
-// PV(j) in tile order once P(j) is stored; the group of tile j stores P(j) once PV(j-1) has landed.
+// whichever MMA is ready, PV first: PV(j) in tile order once P(j) is stored, S(j+2) as soon as S(j) has been
+// read out in both CTAs and K(j+2) has landed; the group of tile j stores P(j) once PV(j-1) has landed.
 #pragma once
 #include "attn_common.cuh"
 #include "sm100.cuh"
@@ -383,19 +383,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           fwd_item_tiles(it.qp, n_qt, p.window, kt0, n_kv);
           // This item's Q is in both CTAs' tensor memory (copied once the previous item's MMAs had completed).
           if (!mbar_wait_pair_warp(&bars.q_ready, k & 1, abort, peer_abort, lim, &g_device_error, kSiteFwdMmaQ)) break;
-          // Issue whichever MMA is ready, S first: the S tiles run ahead as far as the two S buffers allow, so
-          // a softmax group never waits for its scores behind a PV whose P is still being computed; the PVs go
-          // in tile order as their P arrives. The tensor cores execute in issue order.
+          // Issue whichever MMA is ready, PV first. The PVs go in tile order as their P arrives, and P(j+1) can
+          // only be stored once PV(j) has read P(j), so a PV that queued behind an S would hold up the next
+          // tile's P; the S tiles run ahead as far as the two S buffers allow and have time to spare. The
+          // tensor cores execute in issue order.
           int js = 0, jp = 0;  // next S and next PV of the item
           uint64_t t_idle = 0;
           while (jp < n_kv) {
-            if (js < n_kv && s_ready(t0 + js)) {
-              issue_s(t0 + js++);
-              if (js == n_kv && leader) mma_commit_pair(&bars.s_done, 3);  // the item's Q may be replaced
-              t_idle = 0;
-            } else if (jp < js && pv_ready(t0 + jp)) {
+            if (jp < js && pv_ready(t0 + jp)) {
               issue_pv(t0 + jp, jp == 0);
               ++jp;
+              t_idle = 0;
+            } else if (js < n_kv && s_ready(t0 + js)) {
+              issue_s(t0 + js++);
+              if (js == n_kv && leader) mma_commit_pair(&bars.s_done, 3);  // the item's Q may be replaced
               t_idle = 0;
             } else {
               // Nothing ready: bounded like every wait of the kernel.

@@ -13,10 +13,11 @@ memory): the group of the item's last step stages dV in the dQ staging buffer (a
 has read it), the other group dK in the two dS^T buffers. The K/V producer stores dK once it is staged
 (dk_staged) and reports when the store has read the dS^T buffers (ds_read), then does the same for dV
 (dv_staged, dq_read); each group waits for those reports before its first write to the same buffers in the next
-item. The groups hand the 32 KB dQ staging buffer to each other in step order: step gs's bulk reduction
-reports on stage_free[gs % 2]. Barrier counts follow the kernel: the softmax-side barriers count warps, and each group is two actors -- the leader's
-warp, which also issues the reductions and reports their reads, and the other three warps, which can run ahead
-of it. MMAs, commits and copies complete at once (timing does not matter for these properties). Over random item
+item. The groups hand the 32 KB dQ staging buffer to each other in step order: a group's leader reports a
+staged tile on dq_staged[gs % 2], the reduction warp issues the step's bulk reduction and reports its read on
+stage_free[gs % 2]. Barrier counts follow the kernel: the softmax-side barriers count warps, and each group is
+two actors -- the leader's warp, which also reports the staged tiles, and the other three warps, which can run
+ahead of it. MMAs, commits and copies complete at once (timing does not matter for these properties). Over random item
 mixes and interleavings the model checks that
 
   * every role runs to the end (no deadlock: a role only waits for something another role will still do),
@@ -54,8 +55,8 @@ class Model:
     def __init__(self, items, bug=None):
         self.items, self.bug = items, bug  # items: steps of each work item of the CTA
         self.b = {name: Barrier(1) for name in ("k_full", "v_full", "k_free", "v_free", "kv_issued", "stage_free0",
-                                                 "stage_free1", "acc_done", "drain", "ds_read",
-                                                 "dq_read")}
+                                                 "stage_free1", "dq_staged0", "dq_staged1", "acc_done", "drain",
+                                                 "ds_read", "dq_read")}
         self.b["acc_free"] = Barrier(8)
         self.b["dk_staged"] = Barrier(4)  # the four warps of the group that stages dK
         self.b["dv_staged"] = Barrier(4)
@@ -173,8 +174,8 @@ def named_barrier(m, key, actor, n_actors):
 
 def softmax_warps(m, g, lead):
     """The warps of softmax group g: the group leader's warp (lead) or the other three. They run the same waits;
-    the leader also issues each step's bulk reduction of the dQ staging buffer and reports its read on
-    stage_free[g], after the group's staging barrier, so the other warps can run ahead of it."""
+    the leader also reports each staged dQ tile to the reduction warp (dq_staged[g]) after the group's staging
+    barrier, so the other warps can run ahead of it."""
     n = 1 if lead else 3
     actor = (g, lead)
 
@@ -211,11 +212,8 @@ def softmax_warps(m, g, lead):
                 m.violations.append(("dQ staged over an unread tile", gs))
             yield named_barrier(m, ("stage", gs), actor, 2)
             if lead:
-                m.staged_reads_pending.add(gs)   # the bulk reduction is issued ...
-                yield lambda: True
-                m.staged_reads_pending.discard(gs)  # ... and has read the buffer
-                m.b[f"stage_free{g}"].arrive()
-                m.single_done += 1
+                m.staged_reads_pending.add(gs)  # staged; the reduction warp reads it
+                m.b[f"dq_staged{g}"].arrive()
         # epilogue, after the item's last MMA: the group of the item's last step (late: its last reduction still
         # reads the dQ staging buffer) stages dV there, the other group stages dK in the two dS^T buffers
         yield m.wait("acc_done", k)
@@ -241,11 +239,25 @@ def softmax_warps(m, g, lead):
         gs0 += ns
 
 
+def reducer(m):
+    """The reduction warp: in step order, once a step's dQ tile is staged, one bulk reduction reads the staging
+    buffer; then stage_free[gs % 2] hands the buffer on."""
+    gs = 0
+    for ns in m.items:
+        for _ in range(ns):
+            yield m.wait(f"dq_staged{gs & 1}", gs >> 1)
+            yield lambda: True
+            m.staged_reads_pending.discard(gs)  # the reduction has read the buffer
+            m.b[f"stage_free{gs & 1}"].arrive()
+            m.single_done += 1
+            gs += 1
+
+
 def run(items, seed, bug=None):
     """Random interleaving of the roles; returns (finished, violations)."""
     m = Model(items, bug)
     rng = random.Random(seed)
-    roles = {"tma": producer(m), "kv": kv_producer(m), "mma": mma(m)}
+    roles = {"tma": producer(m), "kv": kv_producer(m), "mma": mma(m), "reduce": reducer(m)}
     for g in range(2):
         for lead in (True, False):
             roles[f"g{g}{'lead' if lead else 'rest'}"] = softmax_warps(m, g, lead)

@@ -126,21 +126,21 @@ def mma(m, order="dynamic"):
         m.both(f"pv_done{t & 1}")
         m.both(f"v_empty{t % STAGES}")
 
-    if order == "dynamic":  # the kernel: per item, whichever of S(js), PV(jp) is ready (S first), then o_final
+    if order == "dynamic":  # the kernel: per item, whichever of PV(jp), S(js) is ready (PV first), then o_final
         t0 = 0
         for k, n in enumerate(m.items):
             yield m.wait("q_ready", k)
             js = jp = 0
             while jp < n:
                 yield lambda: (js < n and s_ready(t0 + js)) or (jp < js and pv_ready(t0 + jp))
-                if js < n and s_ready(t0 + js):
+                if jp < js and pv_ready(t0 + jp):
+                    issue_pv(t0 + jp)
+                    jp += 1
+                else:
                     issue_s(t0 + js)
                     js += 1
                     if js == n:
                         m.both("s_done")  # the item's Q in tensor memory is no longer read
-                else:
-                    issue_pv(t0 + jp)
-                    jp += 1
             m.both("o_final")
             t0 += n
     else:  # negative control: one stream over all items, PVs two tiles behind, no flush at item starts
