@@ -547,12 +547,14 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
 
 namespace {
 
-// Splits of the cache per (sequence, key/value head): about 8 CTAs per SM of a 148-SM part in all (one is resident
-// per SM at a time, with its 224 KB ring; several waves even out the sequences' different lengths), each split
-// at least kDecChunkKeys keys (a multiple of the 128-key block).
+// Splits of the cache per (sequence, key/value head): about 4 CTAs per SM of a 148-SM part in all (one is resident
+// per SM at a time, with its 224 KB ring; a few waves even out the sequences' different lengths, and each CTA's
+// ramp-up, its first blocks' loads, is paid fewer times than with 8 or 16: on the decode workloads 4 per SM ran
+// 1-6 % faster than 8 and 10-25 % faster than 16, and 2 or 1 lost 10 % with grouped heads), each split at least
+// kDecChunkKeys keys (a multiple of the 128-key block).
 void decode_split(int B, int Hkv, int Tk, int* n_split, int* chunk) {
   const long long pairs = static_cast<long long>(B) * Hkv;
-  long long want = (8 * 148 + pairs - 1) / pairs;
+  long long want = (4 * 148 + pairs - 1) / pairs;
   const long long max_split = (Tk + attn::kDecChunkKeys - 1) / attn::kDecChunkKeys;
   if (want > max_split) want = max_split;
   if (want < 1) want = 1;
