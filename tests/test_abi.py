@@ -140,6 +140,16 @@ def test_window_argument_errors(lib):
     assert lib.attn_bwd_ex(*ptrs, ws - 1, 1, 2, 2, 128, 128, 0.088, 4, None) == 6
 
 
+def test_decode_split_rule(lib):
+    """The cache is split into about 4 CTAs per SM of a 148-SM part, in chunks of at least 256 keys that are whole
+    128-key blocks; the workspace holds each chunk's unnormalised O (128 floats) and its max and sum per row."""
+    row = (128 + 2) * 4
+    assert lib.attn_decode_workspace_bytes(64, 10, 10, 1, 2048, 128) == 640 * 1 * 1 * row  # 640 pairs: no split
+    assert lib.attn_decode_workspace_bytes(64, 10, 5, 1, 2048, 128) == 320 * 2 * 2 * row   # 320 pairs: 2 chunks
+    assert lib.attn_decode_workspace_bytes(2, 8, 2, 1, 1000, 128) == 4 * 4 * 4 * row      # 4 chunks of 256 keys
+    assert lib.attn_decode_workspace_bytes(1, 1, 1, 1, 100, 128) == 1 * row               # shorter than a chunk
+
+
 def test_decode_argument_errors(lib):
     """attn_decode checks sizes, the row limit, the workspace and overlaps before any CUDA call."""
     assert lib.attn_decode_workspace_bytes(2, 8, 2, 1, 1000, 128) > 0
