@@ -553,6 +553,7 @@ def run_decode(args):
     o, lse = torch.empty_like(q), torch.empty((w.B, w.H, w.Tq), dtype=torch.float32, device=device)
     lib = attn.load_library()
     ws_bytes = int(lib.attn_decode_workspace_bytes(w.B, w.H, w.Hkv, w.Tq, w.Tk, w.D))
+    per_call = int(lib.attn_decode_kernels(w.B, w.H, w.Hkv, w.Tq, w.Tk, w.D, w.window))  # kernels per call
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
     sh = torch.cuda.current_stream(device).cuda_stream
 
@@ -602,9 +603,10 @@ def run_decode(args):
         "config": {"workload": w.name, "B": w.B, "H": w.H, "H_kv": w.Hkv, "Tq": w.Tq, "Tk": w.Tk, "D": w.D,
                    "window": w.window, "recipe": w.recipe, "l2": "256 MB written between calls",
                    "parallelism": f"replicas x{world} (no collective on the data path)"},
-        "roofline": {"kernel": "attn_decode (split + combine)", "bound": "hbm", "achieved": gbs, "peak": hbm,
+        "roofline": {"kernel": "attn_decode (split" + (" + combine)" if per_call > 1 else ")"), "bound": "hbm",
+                     "achieved": gbs, "peak": hbm,
                      "unit": "GB/s", "frac": gbs / hbm, "traffic": None, "alg_bytes": nbytes},
-        "gpu_launches": 2 * args.steps, "clocks": clocks, "kernel_source_hash": kernel_source_hash(),
+        "gpu_launches": per_call * args.steps, "clocks": clocks, "kernel_source_hash": kernel_source_hash(),
     }))
     return 0
 

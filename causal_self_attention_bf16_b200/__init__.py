@@ -44,6 +44,7 @@ SIGNATURES = {
     "attn_fwd_ex": ([_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _VP], _I),
     "attn_bwd_ex": ([_VP] * 10 + [_SZ, _I, _I, _I, _I, _I, _F, _I, _VP], _I),
     "attn_decode_workspace_bytes": ([_I] * 6, _SZ),
+    "attn_decode_kernels": ([_I] * 7, _I),
     "attn_decode": ([_VP] * 7 + [_SZ] + [_I] * 6 + [_F, _VP], _I),
     "attn_decode_ex": ([_VP] * 7 + [_SZ] + [_I] * 6 + [_F, _I, _VP], _I),
     "attn_qk_norm_rope": ([_VP] * 5 + [_I] * 5 + [_F, _F, _I, _VP], _I),

@@ -598,6 +598,13 @@ size_t attn_decode_workspace_bytes(int B, int H, int H_kv, int Tq, int Tk, int D
   return decode_workspace(B, H, H_kv, Tq, Tk);
 }
 
+int attn_decode_kernels(int B, int H, int H_kv, int Tq, int Tk, int D, int window) {
+  if (check_decode(B, H, H_kv, Tq, Tk, D, 1.0f) != ATTN_OK || window < -1) return 0;
+  int n_split = 1, chunk = 0;
+  decode_split(B, H_kv, decode_span(Tq, Tk, window), &n_split, &chunk);
+  return n_split > 1 ? 2 : 1;
+}
+
 attn_status attn_decode_ex(const void* q, const void* k_cache, const void* v_cache, const int* cache_seqlens,
                            void* o, float* lse, void* workspace, size_t workspace_bytes, int B, int H, int H_kv,
                            int Tq, int Tk, int D, float scale, int window, void* stream) {
@@ -668,9 +675,11 @@ attn_status attn_decode_ex(const void* q, const void* k_cache, const void* v_cac
   if (e != cudaSuccess) return cuda_fail(e, "attn_decode_split_kernel attribute");
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "attn_decode_split_kernel launch");
-  const long long out_rows = static_cast<long long>(B) * H * Tq;
-  attn::attn_decode_combine_kernel<<<static_cast<unsigned>((out_rows + 7) / 8), 256, 0, s>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_decode_combine_kernel launch");
+  if (p.n_split > 1) {  // (with one chunk per (sequence, head) the split kernel wrote o and lse itself)
+    const long long out_rows = static_cast<long long>(B) * H * Tq;
+    attn::attn_decode_combine_kernel<<<static_cast<unsigned>((out_rows + 7) / 8), 256, 0, s>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "attn_decode_combine_kernel launch");
+  }
   return ATTN_OK;
 }
 

@@ -17,10 +17,11 @@
 //      shuffles to add), a warp per row updates the running max and sum (online softmax in base 2), and a
 //      thread per pair of output dimensions and slice of the block's keys accumulates O; the slices are added
 //      once per chunk.
-//      The chunk's unnormalised O, running max and sum go to a workspace. The kernel is instantiated for 1, 2,
-//      4, 8, 16 and 32 rows.
-//   2. attn_decode_combine_kernel: one warp per (sequence, query head, new token) merges the chunks by their
-//      log-sum-exp and writes o and lse.
+//      The chunk's unnormalised O, running max and sum go to a workspace; when the cache is not split (one
+//      chunk per (sequence, head)) the kernel normalises and writes o and lse itself. The kernel is
+//      instantiated for 1, 2, 4, 8, 16 and 32 rows.
+//   2. attn_decode_combine_kernel (only when the cache is split): one warp per (sequence, query head, new
+//      token) merges the chunks by their log-sum-exp and writes o and lse.
 #pragma once
 #include "attn_common.cuh"
 #include "sm100.cuh"
@@ -287,6 +288,29 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
   for (int r = 0; r < kRows; ++r)
     if (r < R) *reinterpret_cast<float2*>(red + (kq * R + r) * 128 + 2 * dp) = make_float2(acc[r][0], acc[r][1]);
   __syncthreads();
+  if (p.n_split == 1) {
+    // The only chunk of its (sequence, head): the result is final, so it is normalised and written here as the
+    // combine kernel would (that kernel is not launched): o = O / l, lse = m + log2(l) in natural-log units.
+    for (int e = t; e < R * 128; e += kThreads) {
+      const int r = e / 128, dd = e % 128, i = r % p.Tq, h = hk * G + r / p.Tq;
+      float sum = 0.f;
+#pragma unroll
+      for (int q = 0; q < kSlices; ++q) sum += red[(q * R + r) * 128 + dd];
+      const float l = row_l[r];
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const size_t o_off = ((static_cast<size_t>(b) * p.Tq + i) * p.H + h) * 128 + dd;
+      if (ATTN_IN_RANGE(o_off, 1, static_cast<size_t>(p.B) * p.Tq * p.H * 128, kSiteChkDecO, &g_device_error))
+        p.o[o_off] = __float2bfloat16_rn(sum * inv);
+    }
+    if (t < R) {
+      const int i = t % p.Tq, h = hk * G + t / p.Tq;
+      const float l = row_l[t];
+      const size_t lse_i = (static_cast<size_t>(b) * p.H + h) * p.Tq + i;
+      if (ATTN_IN_RANGE(lse_i, 1, static_cast<size_t>(p.B) * p.H * p.Tq, kSiteChkDecLse, &g_device_error))
+        p.lse[lse_i] = l > 0.f ? (row_m[t] + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    }
+    return;
+  }
   const size_t n_part = static_cast<size_t>(p.B) * p.Hkv * p.n_split * R;  // partial rows
   const size_t part = (static_cast<size_t>(bhk) * p.n_split + sp) * R;      // this chunk's first one
   float* po = p.part_o + part * 128;

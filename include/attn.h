@@ -150,10 +150,17 @@ attn_status attn_bwd_ex(const void* q, const void* k, const void* v, const void*
  *   workspace scratch: attn_decode_workspace_bytes(B, H, H_kv, Tq, Tk, D) bytes, 16-byte aligned
  * Query i of sequence b sits at position L_b - Tq + i and sees keys 0 .. L_b - Tq + i; a query that sees no
  * key gets o = 0, lse = -inf. (H / H_kv) * Tq must be <= 32 and D = 128 (else ATTN_ERR_UNSUPPORTED).
- * Launches two kernels (per cache chunk, then the merge of the chunks). Calls sharing a workspace must not
- * overlap in time on the GPU.
+ * Launches one or two kernels (per cache chunk, then, when the cache is split into several chunks per (sequence,
+ * head), the merge of the chunks; attn_decode_kernels tells which). Calls sharing a workspace must not overlap
+ * in time on the GPU.
  */
 size_t attn_decode_workspace_bytes(int B, int H, int H_kv, int Tq, int Tk, int D);
+/*
+ * Kernels one attn_decode_ex call with these sizes and window launches: 1 when each (sequence, key/value head)
+ * is one chunk of the cache, 2 when the chunks are merged by a second kernel. 0 for arguments attn_decode_ex
+ * rejects (sizes, D, the row limit, window < -1). Host-only; no CUDA call.
+ */
+int attn_decode_kernels(int B, int H, int H_kv, int Tq, int Tk, int D, int window);
 attn_status attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* cache_seqlens, void* o,
                         float* lse, void* workspace, size_t workspace_bytes, int B, int H, int H_kv, int Tq, int Tk,
                         int D, float scale, void* stream);

@@ -150,6 +150,17 @@ def test_decode_split_rule(lib):
     assert lib.attn_decode_workspace_bytes(1, 1, 1, 1, 100, 128) == 1 * row               # shorter than a chunk
 
 
+def test_decode_kernel_count(lib):
+    """One kernel when each (sequence, head) is one chunk of the cache (it writes o and lse itself), two when the
+    chunks are merged by a second kernel; 0 for arguments attn_decode_ex rejects."""
+    assert lib.attn_decode_kernels(64, 10, 10, 1, 2048, 128, -1) == 1   # 640 pairs: no split
+    assert lib.attn_decode_kernels(64, 10, 5, 1, 2048, 128, -1) == 2    # 320 pairs: 2 chunks
+    assert lib.attn_decode_kernels(64, 10, 10, 1, 2048, 128, 512) == 1  # the window's band is one chunk
+    assert lib.attn_decode_kernels(4, 1, 1, 4, 5, 128, -1) == 1         # shorter than a chunk
+    assert lib.attn_decode_kernels(2, 8, 3, 1, 1000, 128, -1) == 0      # H_kv does not divide H
+    assert lib.attn_decode_kernels(2, 8, 2, 1, 1000, 128, -2) == 0      # window < -1
+
+
 def test_decode_argument_errors(lib):
     """attn_decode checks sizes, the row limit, the workspace and overlaps before any CUDA call."""
     assert lib.attn_decode_workspace_bytes(2, 8, 2, 1, 1000, 128) > 0

@@ -274,18 +274,23 @@ def test_decode_window_long_cache_single_token():
     assert torch.equal(o_all, o_big) and torch.equal(lse_all, lse_big)
 
 
-def test_decode_full_size_sampled():
-    """The benchmark's decode workload (64 sequences, d20 heads, ragged lengths up to 2048), oracle on samples."""
+@pytest.mark.parametrize("name", ["decode_d20", "decode_d20_gqa", "decode_d20_sw"])
+def test_decode_full_size_sampled(name):
+    """The benchmark's decode workloads (64 sequences, d20 heads, ragged lengths up to 2048), oracle on samples.
+    decode_d20 and decode_d20_sw take one cache chunk per (sequence, head), whose kernel writes o and lse itself;
+    decode_d20_gqa splits the cache and merges the chunks in a second kernel."""
     from workloads import DECODE_WORKLOADS, make_decode_inputs
-    w = DECODE_WORKLOADS["decode_d20_gqa"]
+    w = DECODE_WORKLOADS[name]
+    win = w.window if w.window >= 0 else None
     q, kc, vc, lens = make_decode_inputs(w)
     dev = torch.device("cuda")
-    o, lse = attn.attn_decode(q.to(dev), kc.to(dev), vc.to(dev), lens.to(dev), w.scale)
+    o, lse = attn.attn_decode(q.to(dev), kc.to(dev), vc.to(dev), lens.to(dev), w.scale, window=win)
     torch.cuda.synchronize()
     for b in (0, 17, w.B - 1):
-        O_ref, LSE_ref = attn_ref.decode_forward(q[b:b + 1], kc[b:b + 1], vc[b:b + 1], lens[b:b + 1].numpy(), w.scale)
-        check_o(to64(o[b:b + 1]), O_ref, f"decode_d20_gqa b={b}")
-        check_lse(to64(lse[b:b + 1]), LSE_ref, f"decode_d20_gqa b={b}")
+        O_ref, LSE_ref = attn_ref.decode_forward(q[b:b + 1], kc[b:b + 1], vc[b:b + 1], lens[b:b + 1].numpy(), w.scale,
+                                                 window=win)
+        check_o(to64(o[b:b + 1]), O_ref, f"{name} b={b}")
+        check_lse(to64(lse[b:b + 1]), LSE_ref, f"{name} b={b}")
 
 
 def test_causality_on_gpu():
