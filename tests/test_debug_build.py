@@ -131,15 +131,18 @@ def test_debug_build_matches_release_on_attention(libs, B, H, Hkv, T, window):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("window", [-1, 100])
-def test_debug_build_matches_release_on_decode(libs, window):
+@pytest.mark.parametrize("window,Tk,kernels", [(-1, 700, 2), (100, 700, 1), (-1, 200, 1)])
+def test_debug_build_matches_release_on_decode(libs, window, Tk, kernels):
+    """A split cache (chunks merged by the second kernel), and a window band or a cache short enough to be one
+    chunk per (sequence, head), whose split kernel writes o and lse itself."""
     release, debug = libs
     dev = torch.device("cuda:0")
     g = torch.Generator().manual_seed(77)
-    B, H, Hkv, Tq, Tk = 3, 8, 2, 2, 700
+    B, H, Hkv, Tq = 3, 8, 2, 2
+    assert release.attn_decode_kernels(B, H, Hkv, Tq, Tk, 128, window) == kernels
     q = _randn((B, Tq, H, 128), g, dev)
     kc, vc = _randn((B, Tk, Hkv, 128), g, dev), _randn((B, Tk, Hkv, 128), g, dev)
-    lens = torch.tensor([700, 1, 333], dtype=torch.int32, device=dev)
+    lens = torch.tensor([Tk, 1, Tk // 2], dtype=torch.int32, device=dev)
     assert debug.attn_clear_device_error() == 0
     ref = _decode(release, q, kc, vc, lens, H, Hkv, window, 128 ** -0.5)
     got = _decode(debug, q, kc, vc, lens, H, Hkv, window, 128 ** -0.5)
