@@ -646,6 +646,13 @@ attn_status attn_decode_ex(const void* q, const void* k_cache, const void* v_cac
   p.R = (H / H_kv) * Tq;
   p.window = window;
   decode_split(B, H_kv, decode_span(Tq, Tk, window), &p.n_split, &p.chunk);
+  // Longest chunks first when a chunk can hold 8 or more blocks and the sort's scratch (a count per block count,
+  // 16 bits per (sequence, chunk) pair) fits the ring's first stage (up to about 32k pairs). Measured on the
+  // decode workloads: 8.3 % less time with 16-block chunks, 4.6 % with 8, 0.9 % more with 5 (the window's band),
+  // where the chunks differ little and the sort's latency at each CTA's start is not won back.
+  const long long order_nb = p.chunk / attn::kDecKeys;
+  const long long order_bytes = (order_nb + 1) * 4 + static_cast<long long>(B) * p.n_split * 2;
+  p.order_nb = order_nb >= 8 && order_bytes <= attn::kDecOrderScratch ? static_cast<int>(order_nb) : 0;
   const size_t rows = static_cast<size_t>(B) * H_kv * p.n_split * p.R;
   p.part_o = static_cast<float*>(workspace);
   p.part_ml = static_cast<float*>(workspace) + rows * 128;

@@ -8,9 +8,9 @@
 //   (natural log; -inf and o = 0 for a query that sees no key).
 //
 // The work is a stream over the cache, HBM-bound (a few FLOPs per byte of K/V), so it runs on CUDA cores:
-//   1. attn_decode_split_kernel: one CTA per (sequence, key/value head, chunk of the cache). The G = H / H_kv
-//      query heads of the group and their Tq new tokens (R = G * Tq rows) share every K and V row the CTA
-//      reads, so the cache is read once. The cache streams through a three-stage shared-memory ring of
+//   1. attn_decode_split_kernel: one CTA per (sequence, key/value head, chunk of the cache), the chunks with the
+//      most blocks first (each CTA counting-sorts the lengths). The G = H / H_kv query heads of the group and
+//      their Tq new tokens (R = G * Tq rows) share every K and V row the CTA reads, so the cache is read once. The cache streams through a three-stage shared-memory ring of
 //      128-key K and V blocks loaded by TMA (one thread issues four 16 KB boxes per block onto the stage's
 //      mbarrier), two blocks in flight while one is used; rows past a sequence's length are masked, never
 //      used. Per block: two or four threads score each key against all rows (a part of the dims each,
@@ -51,21 +51,23 @@ struct DecodeParams {
   float* part_ml;              // [B * H_kv, n_split, R, 2]: running max (log2 units) and sum
   int B, H, Hkv, Tq, Tk, R, n_split, chunk;
   int window;                  // sliding window: query at position p sees keys p - window .. p; -1: none
+  int order_nb;                // > 0: the CTAs take the (sequence, chunk) pairs longest first, and no chunk
+                               // holds more than order_nb 128-key blocks; 0: in index order
   float scale_log2;            // scale * log2(e)
   uint64_t timeout_ns;         // limit of any single wait
 };
 
 // Dynamic shared memory of the split kernel for up to kRows query rows (no static shared memory, so the block
 // starts 1024-byte aligned, as the 128-byte-swizzled TMA boxes need): the ring of (K block, V block) pairs, the
-// rows (fp32, pre-scaled), the block's scores, then P, the rows' running max, sum and rescale factor, and one
-// mbarrier per ring stage. 224 KB at kRows = 32.
+// rows (fp32, pre-scaled), the block's scores, then P, the rows' running max, sum and rescale factor, one
+// mbarrier per ring stage, then two ints (the abort flag, the longest-first order's pick). 224 KB at kRows = 32.
 template <int kRows>
 __host__ __device__ constexpr size_t dec_bar_offset() {  // the stage barriers, 8-byte aligned
   return (kDecStages * 2 * kDecBlockBytes + 2 * kRows * 128 * 4 + 3 * kRows * 4 + 7) / 8 * 8;
 }
 template <int kRows>
 __host__ __device__ constexpr size_t dec_smem_bytes() {
-  return dec_bar_offset<kRows>() + kDecStages * 8 + 8;  // + the abort flag
+  return dec_bar_offset<kRows>() + kDecStages * 8 + 8;  // + the abort flag and the longest-first order's pick
 }
 static_assert(dec_smem_bytes<kDecMaxRows>() <= 232448, "decode split kernel exceeds the 227 KB shared-memory opt-in");
 
@@ -75,6 +77,85 @@ static_assert(dec_smem_bytes<kDecMaxRows>() <= 232448, "decode split kernel exce
 __device__ __forceinline__ uint32_t dec_box_off(int j, int c) { return j * 128 + ((c ^ (j & 7)) << 4); }
 
 enum : uint32_t { kSiteDecFull = 0x31, kSiteDecDrain = 0x32 };
+
+// The keys [key_lo, key_hi) that chunk sp of sequence b covers, in nblk 128-key blocks: from the first row's
+// window start (0 without a window) on, chunk keys per split, up to the sequence's length L.
+struct DecChunk {
+  int L, key_lo, key_hi, nblk;
+};
+__device__ __forceinline__ DecChunk dec_chunk(const DecodeParams& p, int b, int sp) {
+  DecChunk c;
+  c.L = min(max(p.seqlens[b], 0), p.Tk);  // lengths outside [0, Tk] are clamped
+  const int start = p.window < 0 ? 0 : max(0, c.L - p.Tq - p.window);
+  c.key_lo = start + sp * p.chunk;
+  c.key_hi = min(c.L, c.key_lo + p.chunk);
+  c.nblk = c.key_hi > c.key_lo ? (c.key_hi - c.key_lo + kDecKeys - 1) / kDecKeys : 0;
+  return c;
+}
+
+// Bytes of the ring's first stage that the longest-first order may use as scratch: a histogram of order_nb + 1
+// ints and a block count (16 bits) per (sequence, chunk) pair.
+constexpr int kDecOrderScratch = 2 * kDecBlockBytes;
+
+// The (sequence, chunk) pair b * n_split + sp that position q takes in the longest-first order: a counting sort of
+// the B * n_split pairs by block count, most blocks first, equal counts in index order. The block scheduler
+// starts CTAs roughly in index order, so with the chunks in index order the last wave holds long and short chunks
+// alike and SMs idle while the long ones finish; longest first, the short chunks fill in at the end (the list-
+// scheduling rule). Every CTA sorts the same lengths the same way, so the positions map onto the pairs one to
+// one. Called by all threads; the ring's first stage is the scratch (the TMA copies into it come after the proxy
+// fence and barrier at the end) and *picked the result's slot.
+template <int kThreads>
+__device__ int dec_longest_first(const DecodeParams& p, int q, uint8_t* scratch, volatile int* picked) {
+  int* hist = reinterpret_cast<int*>(scratch);                        // [order_nb + 1]
+  uint16_t* nb = reinterpret_cast<uint16_t*>(hist + p.order_nb + 1);  // [B * n_split]
+  const int t = threadIdx.x, lane = t & 31, n_pairs = p.B * p.n_split;
+  for (int i = t; i <= p.order_nb; i += kThreads) hist[i] = 0;
+  if (t == 0) *picked = -1;
+  __syncthreads();
+  for (int i = t; i < n_pairs; i += kThreads) {
+    const int n = min(dec_chunk(p, i / p.n_split, i % p.n_split).nblk, p.order_nb);
+    nb[i] = static_cast<uint16_t>(n);
+    atomicAdd(&hist[n], 1);
+  }
+  __syncthreads();
+  if (t < 32) {
+    // The count x whose pairs hold position q, walking the counts from order_nb down 32 at a time (lane l takes
+    // count top - l), and q's rank r among them.
+    int x = -1, r = 0, above = 0;  // above: pairs with more blocks than this window's counts
+    for (int top = p.order_nb; top >= 0 && x < 0; top -= 32) {
+      const int c = top - lane >= 0 ? hist[top - lane] : 0;
+      int s = c;  // pairs in this window's counts top .. top - lane
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, s, d);
+        if (lane >= d) s += y;
+      }
+      const int first = above + s - c;  // position of this count's first pair
+      const unsigned hit = __ballot_sync(0xffffffffu, c > 0 && q >= first && q < first + c);
+      if (hit) {
+        const int l = __ffs(hit) - 1;
+        x = top - l;
+        r = q - __shfl_sync(0xffffffffu, first, l);
+      }
+      above += __shfl_sync(0xffffffffu, s, 31);
+    }
+    // The r-th pair with x blocks, in index order, 32 pairs at a time.
+    for (int base = 0; x >= 0 && base < n_pairs; base += 32) {
+      unsigned m = __ballot_sync(0xffffffffu, base + lane < n_pairs && nb[base + lane] == x);
+      const int c = __popc(m);
+      if (r < c) {
+        for (int k = 0; k < r; ++k) m &= m - 1;
+        if (lane == 0) *picked = base + __ffs(m) - 1;
+        break;
+      }
+      r -= c;
+    }
+  }
+  sm100::fence_async_shared();  // the generic accesses above come before the TMA copies into the ring
+  __syncthreads();
+  const int pair = *picked;
+  return pair >= 0 ? pair : q;  // (always found: the counts' position ranges partition 0 .. n_pairs - 1)
+}
 
 template <int kRows>
 __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel(
@@ -99,15 +180,18 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
   volatile int* abort = reinterpret_cast<volatile int*>(full + kDecStages);
 
   const int t = threadIdx.x, warp = t / 32, lane = t % 32;
-  const int bhk = blockIdx.x / p.n_split, sp = blockIdx.x % p.n_split;
-  const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
+  // CTA i takes key/value head i % H_kv of the (sequence, chunk) pair at position i / H_kv: in index order, or
+  // longest first.
+  const int hk = blockIdx.x % p.Hkv;
+  int pair = blockIdx.x / p.Hkv;
+  if (p.order_nb > 0)
+    pair = dec_longest_first<kThreads>(p, pair, dec_smem, abort + 1);
+  const int b = pair / p.n_split, sp = pair % p.n_split, bhk = b * p.Hkv + hk;
   const int G = p.H / p.Hkv, R = p.R;
-  const int L = min(max(p.seqlens[b], 0), p.Tk);   // lengths outside [0, Tk] are clamped
   // The chunks split the keys any row of this sequence sees: from the first row's window start (0 without a
   // window) to the end of the cache.
-  const int start = p.window < 0 ? 0 : max(0, L - p.Tq - p.window);
-  const int key_lo = start + sp * p.chunk, key_hi = min(L, key_lo + p.chunk);
-  const int nblk = key_hi > key_lo ? (key_hi - key_lo + kDecKeys - 1) / kDecKeys : 0;
+  const DecChunk ch = dec_chunk(p, b, sp);
+  const int L = ch.L, key_lo = ch.key_lo, key_hi = ch.key_hi, nblk = ch.nblk;
   const size_t n_q = static_cast<size_t>(p.B) * p.Tq * p.H * 128;
   const uint64_t lim = p.timeout_ns;
 

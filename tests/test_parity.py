@@ -274,6 +274,55 @@ def test_decode_window_long_cache_single_token():
     assert torch.equal(o_all, o_big) and torch.equal(lse_all, lse_big)
 
 
+@pytest.mark.parametrize("window", [None, 1000])
+def test_decode_many_sequences_every_chunk_once(window):
+    """600 one-head sequences against a 4352-key cache (34 blocks of 128): one chunk per sequence, so the CTAs'
+    longest-first order sorts 600 (sequence, chunk) pairs over 35 block counts, several 32-wide windows of
+    each. Six seeded sequences hold random keys and values and go to the oracle; every other cache is zero, so
+    its output is exactly 0 and its LSE ln(keys seen) (-inf for an empty cache). o and lse start as NaN: every
+    (sequence, chunk) must be computed, and computed once."""
+    B, Tk, D = 600, 4352, 128
+    g = torch.Generator(device="cpu")
+    g.manual_seed(4352)
+    lens = torch.randint(1, Tk + 1, (B,), generator=g, dtype=torch.int64).to(torch.int32)
+    lens[3], lens[4], lens[5] = 0, Tk, 1
+    q = torch.randn((B, 1, 1, D), generator=g).to(torch.bfloat16)
+    picks = [0, 3, 4, 5, 311, B - 1]
+    dev = torch.device("cuda")
+    kc = torch.zeros((B, Tk, 1, D), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    cpu_k, cpu_v = {}, {}
+    for b in picks:
+        cpu_k[b] = torch.zeros((1, Tk, 1, D), dtype=torch.bfloat16)
+        cpu_v[b] = torch.zeros((1, Tk, 1, D), dtype=torch.bfloat16)
+        L = int(lens[b])
+        cpu_k[b][0, :L] = torch.randn((L, 1, D), generator=g).to(torch.bfloat16)
+        cpu_v[b][0, :L] = torch.randn((L, 1, D), generator=g).to(torch.bfloat16)
+        kc[b].copy_(cpu_k[b][0])
+        vc[b].copy_(cpu_v[b][0])
+    o = torch.full((B, 1, 1, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    lse = torch.full((B, 1, 1), float("nan"), dtype=torch.float32, device=dev)
+    scale = D ** -0.5
+    attn.attn_decode(q.to(dev), kc, vc, lens.to(dev), scale, o=o, lse=lse, window=window)
+    torch.cuda.synchronize()
+    assert attn.load_library().attn_decode_kernels(B, 1, 1, 1, Tk, D, -1 if window is None else window) == 1
+    o64, lse64 = to64(o), to64(lse)
+    for b in picks:
+        O_ref, LSE_ref = attn_ref.decode_forward(q[b:b + 1], cpu_k[b], cpu_v[b], lens[b:b + 1].numpy(), scale,
+                                                 window=window)
+        what = f"decode B=600 b={b} L={int(lens[b])}"
+        check_o(o64[b:b + 1], O_ref, what)
+        finite = np.isfinite(LSE_ref)
+        assert np.array_equal(np.isfinite(lse64[b:b + 1]), finite), f"{what}: -inf LSE pattern differs"
+        check_lse(lse64[b:b + 1][finite], LSE_ref[finite], what)
+    rest = np.array([b for b in range(B) if b not in picks])
+    seen = lens.numpy()[rest].astype(np.float64)
+    if window is not None:
+        seen = np.minimum(seen, window + 1)
+    assert np.all(o64[rest] == 0), "a zero cache must give o = 0 exactly (NaN: a chunk was never computed)"
+    check_lse(lse64[rest, 0, 0], np.log(seen), "decode B=600 zero caches")
+
+
 @pytest.mark.parametrize("name", ["decode_d20", "decode_d20_gqa", "decode_d20_sw"])
 def test_decode_full_size_sampled(name):
     """The benchmark's decode workloads (64 sequences, d20 heads, ragged lengths up to 2048), oracle on samples.
