@@ -646,13 +646,11 @@ attn_status attn_decode_ex(const void* q, const void* k_cache, const void* v_cac
   p.R = (H / H_kv) * Tq;
   p.window = window;
   decode_split(B, H_kv, decode_span(Tq, Tk, window), &p.n_split, &p.chunk);
-  // Longest chunks first when a chunk can hold 8 or more blocks and the sort's scratch (a count per block count,
-  // 16 bits per (sequence, chunk) pair) fits the ring's first stage (up to about 32k pairs). Measured on the
-  // decode workloads: 8.3 % less time with 16-block chunks, 4.6 % with 8, 0.9 % more with 5 (the window's band),
-  // where the chunks differ little and the sort's latency at each CTA's start is not won back.
+  // Longest chunks first whenever the sort's scratch (a count per block count, 16 bits per (sequence, chunk)
+  // pair) fits the ring's first stage: up to about 32k pairs.
   const long long order_nb = p.chunk / attn::kDecKeys;
   const long long order_bytes = (order_nb + 1) * 4 + static_cast<long long>(B) * p.n_split * 2;
-  p.order_nb = order_nb >= 8 && order_bytes <= attn::kDecOrderScratch ? static_cast<int>(order_nb) : 0;
+  p.order_nb = order_bytes <= attn::kDecOrderScratch ? static_cast<int>(order_nb) : 0;
   const size_t rows = static_cast<size_t>(B) * H_kv * p.n_split * p.R;
   p.part_o = static_cast<float*>(workspace);
   p.part_ml = static_cast<float*>(workspace) + rows * 128;
@@ -662,7 +660,11 @@ attn_status attn_decode_ex(const void* q, const void* k_cache, const void* v_cac
   if ((st = make_map(&mk, k_cache, B, H_kv, Tk, attn::kDecKeys)) != ATTN_OK) return st;
   if ((st = make_map(&mv, v_cache, B, H_kv, Tk, attn::kDecKeys)) != ATTN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * H_kv * p.n_split);
+  // One CTA per SM (a CTA's ring takes most of an SM's shared memory) walks its share of the units, its ring
+  // running on from one unit into the next, while each share fits a CTA's unit list; else one CTA per unit.
+  const long long n_units = static_cast<long long>(B) * H_kv * p.n_split;
+  const long long sms = (dev >= 0 && dev < 64 && g_sm_count[dev] > 0) ? g_sm_count[dev] : 148;
+  const unsigned grid = static_cast<unsigned>(n_units <= attn::kDecMaxUnits * sms ? std::min(n_units, sms) : n_units);
   cudaError_t e = cudaSuccess;
   auto launch = [&](auto kernel, size_t smem_bytes, int threads) {
     static std::mutex mu;

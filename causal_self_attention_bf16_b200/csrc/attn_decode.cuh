@@ -8,15 +8,16 @@
 //   (natural log; -inf and o = 0 for a query that sees no key).
 //
 // The work is a stream over the cache, HBM-bound (a few FLOPs per byte of K/V), so it runs on CUDA cores:
-//   1. attn_decode_split_kernel: one CTA per (sequence, key/value head, chunk of the cache), the chunks with the
-//      most blocks first (each CTA counting-sorts the lengths). The G = H / H_kv query heads of the group and
-//      their Tq new tokens (R = G * Tq rows) share every K and V row the CTA reads, so the cache is read once. The cache streams through a three-stage shared-memory ring of
-//      128-key K and V blocks loaded by TMA (one thread issues four 16 KB boxes per block onto the stage's
-//      mbarrier), two blocks in flight while one is used; rows past a sequence's length are masked, never
-//      used. Per block: two or four threads score each key against all rows (a part of the dims each,
-//      shuffles to add), a warp per row updates the running max and sum (online softmax in base 2), and a
-//      thread per pair of output dimensions and slice of the block's keys accumulates O; the slices are added
-//      once per chunk.
+//   1. attn_decode_split_kernel: the units are (sequence, key/value head, chunk of the cache), the chunks with
+//      the most blocks first (each CTA counting-sorts the lengths). A persistent grid, one CTA per SM, deals
+//      them out in rounds, back and forth; the G = H / H_kv query heads of a unit's group and their Tq new
+//      tokens (R = G * Tq rows) share every K and V row the CTA reads, so the cache is read once. The CTA's
+//      units stream through a three-stage shared-memory ring of 128-key K and V blocks loaded by TMA (one
+//      thread issues four 16 KB boxes per block onto the stage's mbarrier), two blocks in flight while one is
+//      used, on from one unit into the next; rows past a sequence's length are masked, never used. Per block:
+//      two or four threads score each key against all rows (a part of the dims each, shuffles to add), a warp
+//      per row updates the running max and sum (online softmax in base 2), and a thread per pair of output
+//      dimensions and slice of the block's keys accumulates O; the slices are added once per unit.
 //      The chunk's unnormalised O, running max and sum go to a workspace; when the cache is not split (one
 //      chunk per (sequence, head)) the kernel normalises and writes o and lse itself. The kernel is
 //      instantiated for 1, 2, 4, 8, 16 and 32 rows.
@@ -38,6 +39,7 @@ constexpr int kDecKeys = 128;       // keys per block
 constexpr int kDecStages = 3;       // K/V blocks in the shared-memory ring (two in flight while one is used)
 constexpr int kDecMaxRows = 32;     // R = (H / H_kv) * Tq query rows per CTA, at most
 constexpr int kDecChunkKeys = 256;  // keys per split of the cache, at least
+constexpr int kDecMaxUnits = 64;    // (sequence, key/value head, chunk) units one CTA walks, at most
 constexpr uint32_t kDecBlockBytes = kDecKeys * 256;  // one K or V block: 128 keys x 128 dims, bf16
 
 struct DecodeParams {
@@ -57,17 +59,23 @@ struct DecodeParams {
   uint64_t timeout_ns;         // limit of any single wait
 };
 
+// A unit of the split kernel's walk: chunk sp of sequence b for key/value head hk, and the chunk's keys
+// [key_lo, key_hi) of the sequence's L, in nblk 128-key blocks.
+struct DecUnit {
+  int b, sp, hk, L, key_lo, key_hi, nblk;
+};
+
 // Dynamic shared memory of the split kernel for up to kRows query rows (no static shared memory, so the block
 // starts 1024-byte aligned, as the 128-byte-swizzled TMA boxes need): the ring of (K block, V block) pairs, the
 // rows (fp32, pre-scaled), the block's scores, then P, the rows' running max, sum and rescale factor, one
-// mbarrier per ring stage, then two ints (the abort flag, the longest-first order's pick). 224 KB at kRows = 32.
+// mbarrier per ring stage, the abort flag (8 bytes) and the CTA's units (DecUnit each). 224 KB at kRows = 32.
 template <int kRows>
 __host__ __device__ constexpr size_t dec_bar_offset() {  // the stage barriers, 8-byte aligned
   return (kDecStages * 2 * kDecBlockBytes + 2 * kRows * 128 * 4 + 3 * kRows * 4 + 7) / 8 * 8;
 }
 template <int kRows>
 __host__ __device__ constexpr size_t dec_smem_bytes() {
-  return dec_bar_offset<kRows>() + kDecStages * 8 + 8;  // + the abort flag and the longest-first order's pick
+  return dec_bar_offset<kRows>() + kDecStages * 8 + 8 + kDecMaxUnits * sizeof(DecUnit);
 }
 static_assert(dec_smem_bytes<kDecMaxRows>() <= 232448, "decode split kernel exceeds the 227 KB shared-memory opt-in");
 
@@ -97,20 +105,18 @@ __device__ __forceinline__ DecChunk dec_chunk(const DecodeParams& p, int b, int 
 // ints and a block count (16 bits) per (sequence, chunk) pair.
 constexpr int kDecOrderScratch = 2 * kDecBlockBytes;
 
-// The (sequence, chunk) pair b * n_split + sp that position q takes in the longest-first order: a counting sort of
-// the B * n_split pairs by block count, most blocks first, equal counts in index order. The block scheduler
-// starts CTAs roughly in index order, so with the chunks in index order the last wave holds long and short chunks
-// alike and SMs idle while the long ones finish; longest first, the short chunks fill in at the end (the list-
-// scheduling rule). Every CTA sorts the same lengths the same way, so the positions map onto the pairs one to
-// one. Called by all threads; the ring's first stage is the scratch (the TMA copies into it come after the proxy
-// fence and barrier at the end) and *picked the result's slot.
+// The longest-first order of the (sequence, chunk) pairs b * n_split + sp: a counting sort by block count, most
+// blocks first, equal counts in index order. The CTAs deal the units out in this order, so that the short chunks
+// fill in at the end (the list-scheduling rule); in index order each SM's last units hold long and short chunks
+// alike and SMs idle while the long ones finish. Every CTA sorts the same lengths the same way, so the order is
+// one permutation. dec_order_build (all threads) counts the pairs per block count into scratch: a histogram of
+// order_nb + 1 ints, then each pair's count in 16 bits.
 template <int kThreads>
-__device__ int dec_longest_first(const DecodeParams& p, int q, uint8_t* scratch, volatile int* picked) {
+__device__ void dec_order_build(const DecodeParams& p, uint8_t* scratch) {
   int* hist = reinterpret_cast<int*>(scratch);                        // [order_nb + 1]
   uint16_t* nb = reinterpret_cast<uint16_t*>(hist + p.order_nb + 1);  // [B * n_split]
-  const int t = threadIdx.x, lane = t & 31, n_pairs = p.B * p.n_split;
+  const int t = threadIdx.x, n_pairs = p.B * p.n_split;
   for (int i = t; i <= p.order_nb; i += kThreads) hist[i] = 0;
-  if (t == 0) *picked = -1;
   __syncthreads();
   for (int i = t; i < n_pairs; i += kThreads) {
     const int n = min(dec_chunk(p, i / p.n_split, i % p.n_split).nblk, p.order_nb);
@@ -118,43 +124,51 @@ __device__ int dec_longest_first(const DecodeParams& p, int q, uint8_t* scratch,
     atomicAdd(&hist[n], 1);
   }
   __syncthreads();
-  if (t < 32) {
-    // The count x whose pairs hold position q, walking the counts from order_nb down 32 at a time (lane l takes
-    // count top - l), and q's rank r among them.
-    int x = -1, r = 0, above = 0;  // above: pairs with more blocks than this window's counts
-    for (int top = p.order_nb; top >= 0 && x < 0; top -= 32) {
-      const int c = top - lane >= 0 ? hist[top - lane] : 0;
-      int s = c;  // pairs in this window's counts top .. top - lane
+}
+
+// The pair at position q of the order (called by a whole warp; the same value in every lane), or -1 if q is not a
+// position (it always is for q in 0 .. B * n_split - 1: the counts' position ranges partition them).
+__device__ __forceinline__ int dec_order_find(const DecodeParams& p, int q, const uint8_t* scratch) {
+  const int* hist = reinterpret_cast<const int*>(scratch);
+  const uint16_t* nb = reinterpret_cast<const uint16_t*>(hist + p.order_nb + 1);
+  const int lane = threadIdx.x & 31, n_pairs = p.B * p.n_split;
+  // The count x whose pairs hold position q, walking the counts from order_nb down 32 at a time (lane l takes
+  // count top - l), and q's rank r among them.
+  int x = -1, r = 0, above = 0;  // above: pairs with more blocks than this window's counts
+  for (int top = p.order_nb; top >= 0 && x < 0; top -= 32) {
+    const int c = top - lane >= 0 ? hist[top - lane] : 0;
+    int s = c;  // pairs in this window's counts top .. top - lane
 #pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, s, d);
-        if (lane >= d) s += y;
-      }
-      const int first = above + s - c;  // position of this count's first pair
-      const unsigned hit = __ballot_sync(0xffffffffu, c > 0 && q >= first && q < first + c);
-      if (hit) {
-        const int l = __ffs(hit) - 1;
-        x = top - l;
-        r = q - __shfl_sync(0xffffffffu, first, l);
-      }
-      above += __shfl_sync(0xffffffffu, s, 31);
+    for (int d = 1; d < 32; d <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, d);
+      if (lane >= d) s += y;
     }
-    // The r-th pair with x blocks, in index order, 32 pairs at a time.
-    for (int base = 0; x >= 0 && base < n_pairs; base += 32) {
-      unsigned m = __ballot_sync(0xffffffffu, base + lane < n_pairs && nb[base + lane] == x);
-      const int c = __popc(m);
-      if (r < c) {
-        for (int k = 0; k < r; ++k) m &= m - 1;
-        if (lane == 0) *picked = base + __ffs(m) - 1;
-        break;
-      }
-      r -= c;
+    const int first = above + s - c;  // position of this count's first pair
+    const unsigned hit = __ballot_sync(0xffffffffu, c > 0 && q >= first && q < first + c);
+    if (hit) {
+      const int l = __ffs(hit) - 1;
+      x = top - l;
+      r = q - __shfl_sync(0xffffffffu, first, l);
     }
+    above += __shfl_sync(0xffffffffu, s, 31);
   }
-  sm100::fence_async_shared();  // the generic accesses above come before the TMA copies into the ring
-  __syncthreads();
-  const int pair = *picked;
-  return pair >= 0 ? pair : q;  // (always found: the counts' position ranges partition 0 .. n_pairs - 1)
+  // The r-th pair with x blocks, in index order, 32 pairs at a time.
+  for (int base = 0; x >= 0 && base < n_pairs; base += 32) {
+    unsigned m = __ballot_sync(0xffffffffu, base + lane < n_pairs && nb[base + lane] == x);
+    const int c = __popc(m);
+    if (r < c) {
+      for (int k = 0; k < r; ++k) m &= m - 1;
+      return base + __ffs(m) - 1;
+    }
+    r -= c;
+  }
+  return -1;
+}
+
+// Position of a CTA's k-th unit: the units are dealt to the G CTAs in rounds, back and forth (CTA c takes
+// positions c, 2G - 1 - c, 2G + c, ...), so that with the units longest first every CTA's total is about even.
+__device__ __forceinline__ long long dec_unit_pos(int c, int k, int G) {
+  return static_cast<long long>(k) * G + ((k & 1) ? G - 1 - c : c);
 }
 
 template <int kRows>
@@ -178,239 +192,302 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
   float* row_a = row_l + kRows;
   uint64_t* full = reinterpret_cast<uint64_t*>(dec_smem + dec_bar_offset<kRows>());
   volatile int* abort = reinterpret_cast<volatile int*>(full + kDecStages);
+  DecUnit* units = reinterpret_cast<DecUnit*>(full + kDecStages + 1);  // this CTA's units, in walk order
 
   const int t = threadIdx.x, warp = t / 32, lane = t % 32;
-  // CTA i takes key/value head i % H_kv of the (sequence, chunk) pair at position i / H_kv: in index order, or
-  // longest first.
-  const int hk = blockIdx.x % p.Hkv;
-  int pair = blockIdx.x / p.Hkv;
-  if (p.order_nb > 0)
-    pair = dec_longest_first<kThreads>(p, pair, dec_smem, abort + 1);
-  const int b = pair / p.n_split, sp = pair % p.n_split, bhk = b * p.Hkv + hk;
   const int G = p.H / p.Hkv, R = p.R;
-  // The chunks split the keys any row of this sequence sees: from the first row's window start (0 without a
-  // window) to the end of the cache.
-  const DecChunk ch = dec_chunk(p, b, sp);
-  const int L = ch.L, key_lo = ch.key_lo, key_hi = ch.key_hi, nblk = ch.nblk;
   const size_t n_q = static_cast<size_t>(p.B) * p.Tq * p.H * 128;
   const uint64_t lim = p.timeout_ns;
-
+  // The units (sequence, key/value head, chunk) in order: position i is head i % H_kv of the (sequence, chunk)
+  // pair at position i / H_kv of the pairs, longest first or in index order. This CTA takes positions
+  // dec_unit_pos(blockIdx.x, k, gridDim.x), k = 0, 1, ...: one unit per CTA when the grid has one CTA per unit,
+  // else a persistent walk whose K/V ring runs on from one unit into the next.
+  const long long n_units = static_cast<long long>(p.B) * p.Hkv * p.n_split;
+  int n_mine = 0;
+  while (n_mine < kDecMaxUnits && dec_unit_pos(blockIdx.x, n_mine, gridDim.x) < n_units) ++n_mine;
+  if (p.order_nb > 0) dec_order_build<kThreads>(p, dec_smem);
+  for (int k = warp; k < n_mine; k += kThreads / 32) {
+    const long long pos = dec_unit_pos(blockIdx.x, k, gridDim.x);
+    const int pp = static_cast<int>(pos / p.Hkv), hk = static_cast<int>(pos % p.Hkv);
+    int pair = p.order_nb > 0 ? dec_order_find(p, pp, dec_smem) : pp;
+    if (pair < 0) pair = pp;
+    if (lane == 0) {
+      const DecChunk c = dec_chunk(p, pair / p.n_split, pair % p.n_split);
+      units[k] = DecUnit{pair / p.n_split, pair % p.n_split, hk, c.L, c.key_lo, c.key_hi, c.nblk};
+    }
+  }
   if (t == 0) {
     for (int st = 0; st < kDecStages; ++st) mbar_init(&full[st], 1);
     *abort = 0;
     fence_barrier_init();
   }
+  fence_async_shared();  // the order's generic accesses to the ring come before the TMA copies into it
   __syncthreads();
-  // Block n's K and V into ring stage n % kDecStages: four TMA boxes, 64 KB on the stage's barrier. The tensor
-  // maps bound the copies (rows past the cache come as zeros); rows past a sequence's length are masked below.
+
+  // The issue cursor (thread 0 only): block ib of unit ik's inb blocks, keys from ikey, sequence ibq, head ihk.
+  // Blocks go out in one stream over the CTA's units: the n-th into ring stage n % kDecStages.
   const bool issuer = t == 0;
-  auto issue = [&](int n) {
-    if (issuer && n < nblk) {
-      const int kb = key_lo + n * kDecKeys;
-      uint8_t* ks = dec_smem + (n % kDecStages) * 2 * kDecBlockBytes;
-      uint64_t* bar = &full[n % kDecStages];
-      mbar_arrive_expect_tx(bar, 2 * kDecBlockBytes);
-      for (int c = 0; c < 2; ++c) {
-        tma_load_4d(ks + c * 16384, &tm_k, bar, c * 64, hk, kb, b);
-        tma_load_4d(ks + kDecBlockBytes + c * 16384, &tm_v, bar, c * 64, hk, kb, b);
+  int issued = 0, ik = 0, ib = 0, inb = -1, ikey = 0, ibq = 0, ihk = 0;
+  auto issue_next = [&]() {
+    if (!issuer) return;
+    while (ik < n_mine) {
+      if (inb < 0) {
+        const DecUnit& un = units[ik];
+        inb = un.nblk, ikey = un.key_lo, ibq = un.b, ihk = un.hk, ib = 0;
       }
+      if (ib < inb) break;
+      ++ik, inb = -1;
     }
+    if (ik >= n_mine) return;
+    // Four TMA boxes, 64 KB on the stage's barrier. The tensor maps bound the copies (rows past the cache come
+    // as zeros); rows past a sequence's length are masked below.
+    const int kb = ikey + ib * kDecKeys, st = issued % kDecStages;
+    uint8_t* ks = dec_smem + st * 2 * kDecBlockBytes;
+    mbar_arrive_expect_tx(&full[st], 2 * kDecBlockBytes);
+    for (int c = 0; c < 2; ++c) {
+      tma_load_4d(ks + c * 16384, &tm_k, &full[st], c * 64, ihk, kb, ibq);
+      tma_load_4d(ks + kDecBlockBytes + c * 16384, &tm_v, &full[st], c * 64, ihk, kb, ibq);
+    }
+    ++ib, ++issued;
   };
   if (issuer) {
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
 #pragma unroll
-  for (int n = 0; n < kDecStages - 1; ++n) issue(n);
+  for (int n = 0; n < kDecStages - 1; ++n) issue_next();
 
-  // Row r = g * Tq + i: query head hk * G + g, new token i, which sees keys up to L - Tq + i.
-  for (int e = t; e < R * 128; e += kThreads) {
-    const int r = e / 128, d = e % 128, g = r / p.Tq, i = r % p.Tq;
-    const size_t qi = ((static_cast<size_t>(b) * p.Tq + i) * p.H + hk * G + g) * 128 + d;
-    qs[r][d] = ATTN_IN_RANGE(qi, 1, n_q, kSiteChkDecQ, &g_device_error) ? __bfloat162float(p.q[qi]) * p.scale_log2
-                                                                        : 0.f;
-  }
-  if (t < R) {
-    row_m[t] = -INFINITY;
-    row_l[t] = 0.f;
-  }
+  // Unit k's rows, R x 128 bf16 of q, in registers (elements t, t + kThreads, ...): read a unit ahead, so that
+  // the loads' latency hides behind the previous unit's blocks. Row r = g * Tq + i is query head hk * G + g,
+  // new token i, which sees keys up to L - Tq + i.
+  constexpr int kQPer = (kRows * 128 + kThreads - 1) / kThreads;
+  __nv_bfloat16 qv[kQPer];
+  auto fetch_q = [&](int k) {
+    const int qb = units[k].b, qh = units[k].hk;
+#pragma unroll
+    for (int x = 0; x < kQPer; ++x) {
+      const int e = t + x * kThreads;
+      qv[x] = __float2bfloat16_rn(0.f);
+      if (e < R * 128) {
+        const int r = e / 128, d = e % 128, g = r / p.Tq, i = r % p.Tq;
+        const size_t qi = ((static_cast<size_t>(qb) * p.Tq + i) * p.H + qh * G + g) * 128 + d;
+        if (ATTN_IN_RANGE(qi, 1, n_q, kSiteChkDecQ, &g_device_error)) qv[x] = p.q[qi];
+      }
+    }
+  };
+  fetch_q(0);  // (every CTA has a unit: position blockIdx.x < the grid <= the units)
+
   // P V: output dimensions 2 dp, 2 dp + 1 over keys [kSliceKeys kq, kSliceKeys (kq + 1)) of each block
   const int dp = t & 63, kq = t >> 6;
-  float acc[kRows][2];
-#pragma unroll
-  for (int r = 0; r < kRows; ++r) acc[r][0] = acc[r][1] = 0.f;
-
-  int consumed = 0;  // blocks whose barrier phase this CTA has waited for
+  int consumed = 0;  // blocks of the stream whose barrier phase this CTA has waited for
   bool ok = true;
-  for (int n = 0; n < nblk; ++n) {
-    __syncthreads();  // block n-1's stage and the scores are no longer read: the stage takes block n + 2
-    issue(n + kDecStages - 1);
-    if (!mbar_wait_warp(&full[n % kDecStages], (n / kDecStages) & 1, abort, lim, &g_device_error, kSiteDecFull)) {
-      ok = false;
-    }
-    if (!__syncthreads_and(ok)) {
-      ok = false;
-      break;
-    }
-    consumed = n + 1;
-    const int kb = key_lo + n * kDecKeys, nk = min(kDecKeys, key_hi - kb);
-    const uint8_t* ks = dec_smem + (n % kDecStages) * 2 * kDecBlockBytes;
-    const uint8_t* vs = ks + kDecBlockBytes;
-    {
-      // Scores of key j = t / kPart against every row: this thread takes dims [kDims h, kDims (h + 1)),
-      // h = t % kPart, and the key's threads (adjacent lanes) add their parts. Keys past the block, past the
-      // sequence or past a row's last key are -inf (selected, so whatever those rows of the cache hold never
-      // enters a score).
-      const int j = t / kPart, h = t % kPart;
-      const int box = (h * kDims) / 64, c0 = ((h * kDims) % 64) / 8;  // the part's first 16-byte chunk
-      uint4 kw[kDims / 8];
+  for (int k = 0; k < n_mine && ok; ++k) {
+    const DecUnit un = units[k];
+    const int b = un.b, sp = un.sp, hk = un.hk, bhk = b * p.Hkv + hk;
+    const int L = un.L, key_lo = un.key_lo, key_hi = un.key_hi, nblk = un.nblk;
 #pragma unroll
-      for (int c = 0; c < kDims / 8; ++c)
-        kw[c] = *reinterpret_cast<const uint4*>(ks + box * 16384 + dec_box_off(j, c0 + c));
-      for (int r = 0; r < R; ++r) {
-        const float4* q4 = reinterpret_cast<const float4*>(qs[r] + kDims * h);
-        float s0 = 0.f, s1 = 0.f;
+    for (int x = 0; x < kQPer; ++x) {
+      const int e = t + x * kThreads;
+      if (e < R * 128) qs[e / 128][e % 128] = __bfloat162float(qv[x]) * p.scale_log2;
+    }
+    if (k + 1 < n_mine) fetch_q(k + 1);
+    if (t < R) {
+      row_m[t] = -INFINITY;
+      row_l[t] = 0.f;
+    }
+    float acc[kRows][2];
 #pragma unroll
-        for (int c = 0; c < kDims / 8; ++c) {
-          const float4 qa = q4[2 * c], qb = q4[2 * c + 1];
-          const uint32_t w[4] = {kw[c].x, kw[c].y, kw[c].z, kw[c].w};
-          s0 = fmaf(qa.x, __uint_as_float(w[0] << 16), s0);
-          s1 = fmaf(qa.y, __uint_as_float(w[0] & 0xffff0000u), s1);
-          s0 = fmaf(qa.z, __uint_as_float(w[1] << 16), s0);
-          s1 = fmaf(qa.w, __uint_as_float(w[1] & 0xffff0000u), s1);
-          s0 = fmaf(qb.x, __uint_as_float(w[2] << 16), s0);
-          s1 = fmaf(qb.y, __uint_as_float(w[2] & 0xffff0000u), s1);
-          s0 = fmaf(qb.z, __uint_as_float(w[3] << 16), s0);
-          s1 = fmaf(qb.w, __uint_as_float(w[3] & 0xffff0000u), s1);
+    for (int r = 0; r < kRows; ++r) acc[r][0] = acc[r][1] = 0.f;
+
+    for (int n = 0; n < nblk; ++n) {
+      __syncthreads();  // the previous block's stage and the scores are no longer read: the stage takes the next
+      issue_next();     // block but one of the stream
+      const int g = consumed;
+      if (!mbar_wait_warp(&full[g % kDecStages], (g / kDecStages) & 1, abort, lim, &g_device_error, kSiteDecFull))
+        ok = false;
+      if (!__syncthreads_and(ok)) {
+        ok = false;
+        break;
+      }
+      consumed = g + 1;
+      const uint8_t* ks = dec_smem + (g % kDecStages) * 2 * kDecBlockBytes;
+      const uint8_t* vs = ks + kDecBlockBytes;
+      const int kb = key_lo + n * kDecKeys, nk = min(kDecKeys, key_hi - kb);
+      {
+        // Scores of key j = t / kPart against every row: this thread takes dims [kDims h, kDims (h + 1)),
+        // h = t % kPart, and the key's threads (adjacent lanes) add their parts. Keys past the block, past the
+        // sequence or past a row's last key are -inf (selected, so whatever those rows of the cache hold never
+        // enters a score).
+        const int j = t / kPart, h = t % kPart;
+        const int box = (h * kDims) / 64, c0 = ((h * kDims) % 64) / 8;  // the part's first 16-byte chunk
+        uint4 kw[kDims / 8];
+#pragma unroll
+        for (int c = 0; c < kDims / 8; ++c)
+          kw[c] = *reinterpret_cast<const uint4*>(ks + box * 16384 + dec_box_off(j, c0 + c));
+        for (int r = 0; r < R; ++r) {
+          const float4* q4 = reinterpret_cast<const float4*>(qs[r] + kDims * h);
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int c = 0; c < kDims / 8; ++c) {
+            const float4 qa = q4[2 * c], qb = q4[2 * c + 1];
+            const uint32_t w[4] = {kw[c].x, kw[c].y, kw[c].z, kw[c].w};
+            s0 = fmaf(qa.x, __uint_as_float(w[0] << 16), s0);
+            s1 = fmaf(qa.y, __uint_as_float(w[0] & 0xffff0000u), s1);
+            s0 = fmaf(qa.z, __uint_as_float(w[1] << 16), s0);
+            s1 = fmaf(qa.w, __uint_as_float(w[1] & 0xffff0000u), s1);
+            s0 = fmaf(qb.x, __uint_as_float(w[2] << 16), s0);
+            s1 = fmaf(qb.y, __uint_as_float(w[2] & 0xffff0000u), s1);
+            s0 = fmaf(qb.z, __uint_as_float(w[3] << 16), s0);
+            s1 = fmaf(qb.w, __uint_as_float(w[3] & 0xffff0000u), s1);
+          }
+          float sj = s0 + s1;
+#pragma unroll
+          for (int o = 1; o < kPart; o <<= 1) sj += __shfl_xor_sync(0xffffffffu, sj, o);
+          if (h == 0) {
+            const int last = L - p.Tq + r % p.Tq;  // last key this row sees (its own position)
+            const bool seen = j < nk && kb + j <= last && (p.window < 0 || kb + j >= last - p.window);
+            sc[r][j] = seen ? sj : -INFINITY;
+          }
         }
-        float sj = s0 + s1;
+      }
+      __syncthreads();
+      // Online softmax, a warp per row: block max, running max, exp2 in place, running sum, O's rescale factor.
+      for (int r = warp; r < R; r += kThreads / 32) {
+        float x[4];
 #pragma unroll
-        for (int o = 1; o < kPart; o <<= 1) sj += __shfl_xor_sync(0xffffffffu, sj, o);
-        if (h == 0) {
-          const int last = L - p.Tq + r % p.Tq;  // last key this row sees (its own position)
-          const bool seen = j < nk && kb + j <= last && (p.window < 0 || kb + j >= last - p.window);
-          sc[r][j] = seen ? sj : -INFINITY;
+        for (int e = 0; e < 4; ++e) x[e] = sc[r][lane * 4 + e];
+        float mb = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+        const float m_old = row_m[r];
+        const float m_new = fmaxf(m_old, mb);
+        float sum = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float pe = m_new == -INFINITY ? 0.f : exp2f(x[e] - m_new);
+          sc[r][lane * 4 + e] = pe;
+          sum += pe;
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        __syncwarp();
+        if (lane == 0) {
+          const float a = m_old == m_new ? 1.f : exp2f(m_old - m_new);  // 0 when nothing was seen before
+          row_a[r] = a;
+          row_l[r] = row_l[r] * a + sum;
+          row_m[r] = m_new;
         }
       }
-    }
-    __syncthreads();
-    // Online softmax, a warp per row: block max, running max, exp2 in place, running sum, O's rescale factor.
-    for (int r = warp; r < R; r += kThreads / 32) {
-      float x[4];
+      __syncthreads();
+      // O[r][d] = O[r][d] * a_r + sum_j P[r][j] V[j][d] for this thread's two dims over its slice of the keys:
+      // one 4-byte load per key for V (a warp reads one 128-byte box row), P four keys at a time. V rows past
+      // the sequence's keys are taken as 0 (selected, not multiplied, so the cache's contents there do not
+      // matter), and their P is 0.
 #pragma unroll
-      for (int e = 0; e < 4; ++e) x[e] = sc[r][lane * 4 + e];
-      float mb = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
-      const float m_old = row_m[r];
-      const float m_new = fmaxf(m_old, mb);
-      float sum = 0.f;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float pe = m_new == -INFINITY ? 0.f : exp2f(x[e] - m_new);
-        sc[r][lane * 4 + e] = pe;
-        sum += pe;
-      }
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      __syncwarp();
-      if (lane == 0) {
-        const float a = m_old == m_new ? 1.f : exp2f(m_old - m_new);  // 0 when nothing was seen before
-        row_a[r] = a;
-        row_l[r] = row_l[r] * a + sum;
-        row_m[r] = m_new;
-      }
-    }
-    __syncthreads();
-    // O[r][d] = O[r][d] * a_r + sum_j P[r][j] V[j][d] for this thread's two dims over its slice of the keys:
-    // one 4-byte load per key for V (a warp reads one 128-byte box row), P four keys at a time. V rows past
-    // the sequence's keys are taken as 0 (selected, not multiplied, so the cache's contents there do not
-    // matter), and their P is 0.
-#pragma unroll
-    for (int r = 0; r < kRows; ++r)
-      if (r < R) acc[r][0] *= row_a[r], acc[r][1] *= row_a[r];
-    const uint8_t* vbox = vs + (dp >> 5) * 16384;
+      for (int r = 0; r < kRows; ++r)
+        if (r < R) acc[r][0] *= row_a[r], acc[r][1] *= row_a[r];
+      const uint8_t* vbox = vs + (dp >> 5) * 16384;
 #pragma unroll 2
-    for (int j0 = kSliceKeys * kq; j0 < kSliceKeys * (kq + 1); j0 += 4) {
-      float v0[4], v1[4];
+      for (int j0 = kSliceKeys * kq; j0 < kSliceKeys * (kq + 1); j0 += 4) {
+        float v0[4], v1[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(
-            *reinterpret_cast<const __nv_bfloat162*>(vbox + dec_box_off(j0 + e, (dp & 31) >> 2) + (dp & 3) * 4));
-        const bool in = j0 + e < nk;
-        v0[e] = in ? f.x : 0.f;
-        v1[e] = in ? f.y : 0.f;
-      }
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(
+              *reinterpret_cast<const __nv_bfloat162*>(vbox + dec_box_off(j0 + e, (dp & 31) >> 2) + (dp & 3) * 4));
+          const bool in = j0 + e < nk;
+          v0[e] = in ? f.x : 0.f;
+          v1[e] = in ? f.y : 0.f;
+        }
 #pragma unroll
-      for (int r = 0; r < kRows; ++r) {
-        if (r < R) {
-          const float4 pr = *reinterpret_cast<const float4*>(&sc[r][j0]);
-          const float pe[4] = {pr.x, pr.y, pr.z, pr.w};
-          float a0 = acc[r][0], a1 = acc[r][1];
+        for (int r = 0; r < kRows; ++r) {
+          if (r < R) {
+            const float4 pr = *reinterpret_cast<const float4*>(&sc[r][j0]);
+            const float pe[4] = {pr.x, pr.y, pr.z, pr.w};
+            float a0 = acc[r][0], a1 = acc[r][1];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) a0 = fmaf(pe[e], v0[e], a0), a1 = fmaf(pe[e], v1[e], a1);
-          acc[r][0] = a0;
-          acc[r][1] = a1;
+            for (int e = 0; e < 4; ++e) a0 = fmaf(pe[e], v0[e], a0), a1 = fmaf(pe[e], v1[e], a1);
+            acc[r][0] = a0;
+            acc[r][1] = a1;
+          }
         }
       }
     }
+    if (!ok) break;
+    __syncthreads();  // P and the rows' state are final; the q rows and scores become the reduction's buffers
+    // The chunk's result (an empty chunk leaves max -inf, sum 0, O 0): the key slices' accumulators of each pair
+    // of dims are added in slice order by slice 0's threads, handed over through two buffers in turn (the q
+    // rows and the scores, R x 128 floats each).
+    float* xb[2] = {&qs[0][0], &sc[0][0]};
+    float sum[kRows][2];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) sum[r][0] = 0.f + acc[r][0], sum[r][1] = 0.f + acc[r][1];
+#pragma unroll
+    for (int j = 1; j <= kSlices; ++j) {
+      if (j < kSlices && kq == j) {
+#pragma unroll
+        for (int r = 0; r < kRows; ++r)
+          if (r < R)
+            *reinterpret_cast<float2*>(xb[(j - 1) & 1] + r * 128 + 2 * dp) = make_float2(acc[r][0], acc[r][1]);
+      }
+      if (j >= 2 && kq == 0) {
+#pragma unroll
+        for (int r = 0; r < kRows; ++r)
+          if (r < R) {
+            const float2 x = *reinterpret_cast<const float2*>(xb[j & 1] + r * 128 + 2 * dp);
+            sum[r][0] += x.x, sum[r][1] += x.y;
+          }
+      }
+      if (j < kSlices) __syncthreads();
+    }
+    if (p.n_split == 1) {
+      // The only chunk of its (sequence, head): the result is final, so it is normalised and written here as the
+      // combine kernel would (that kernel is not launched): o = O / l, lse = m + log2(l) in natural-log units.
+      if (kq == 0) {
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+          if (r < R) {
+            const int i = r % p.Tq, h = hk * G + r / p.Tq;
+            const float l = row_l[r];
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const size_t o_off = ((static_cast<size_t>(b) * p.Tq + i) * p.H + h) * 128 + 2 * dp;
+            if (ATTN_IN_RANGE(o_off, 2, static_cast<size_t>(p.B) * p.Tq * p.H * 128, kSiteChkDecO, &g_device_error))
+              *reinterpret_cast<__nv_bfloat162*>(p.o + o_off) =
+                  __halves2bfloat162(__float2bfloat16_rn(sum[r][0] * inv), __float2bfloat16_rn(sum[r][1] * inv));
+          }
+        }
+      }
+      if (t < R) {
+        const int i = t % p.Tq, h = hk * G + t / p.Tq;
+        const float l = row_l[t];
+        const size_t lse_i = (static_cast<size_t>(b) * p.H + h) * p.Tq + i;
+        if (ATTN_IN_RANGE(lse_i, 1, static_cast<size_t>(p.B) * p.H * p.Tq, kSiteChkDecLse, &g_device_error))
+          p.lse[lse_i] = l > 0.f ? (row_m[t] + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      }
+    } else {
+      const size_t n_part = static_cast<size_t>(p.B) * p.Hkv * p.n_split * R;  // partial rows
+      const size_t part = (static_cast<size_t>(bhk) * p.n_split + sp) * R;      // this chunk's first one
+      if (ATTN_IN_RANGE(part, R, n_part, kSiteChkDecPart, &g_device_error)) {
+        if (kq == 0) {
+#pragma unroll
+          for (int r = 0; r < kRows; ++r)
+            if (r < R)
+              *reinterpret_cast<float2*>(p.part_o + (part + r) * 128 + 2 * dp) = make_float2(sum[r][0], sum[r][1]);
+        }
+        if (t < R) {
+          float* pml = p.part_ml + (part + t) * 2;
+          pml[0] = row_m[t];
+          pml[1] = row_l[t];
+        }
+      }
+    }
+    __syncthreads();  // the q rows, scores and rows' state are free for the next unit
   }
   // Blocks issued but not consumed (only after a failure: at most the failed block and the two after it) land
   // before the CTA leaves.
   if (t == 0) {
     volatile int no_abort = 0;
-    for (int n = consumed; n < min(nblk, consumed + kDecStages); ++n)
-      mbar_wait(&full[n % kDecStages], (n / kDecStages) & 1, &no_abort, lim, &g_device_error, kSiteDecDrain);
-  }
-  __syncthreads();  // the ring is no longer read: it takes the key slices' accumulators
-  if (!ok) return;
-
-  // The chunk's partial result (an empty chunk leaves max -inf, sum 0, O 0): the key slices' accumulators of
-  // each dimension are added, then O, the running max and the sum go to the workspace.
-  float* red = reinterpret_cast<float*>(dec_smem);  // [kq][r][128]: 2 KB x kSlices x R, at most 64 KB of 192
-#pragma unroll
-  for (int r = 0; r < kRows; ++r)
-    if (r < R) *reinterpret_cast<float2*>(red + (kq * R + r) * 128 + 2 * dp) = make_float2(acc[r][0], acc[r][1]);
-  __syncthreads();
-  if (p.n_split == 1) {
-    // The only chunk of its (sequence, head): the result is final, so it is normalised and written here as the
-    // combine kernel would (that kernel is not launched): o = O / l, lse = m + log2(l) in natural-log units.
-    for (int e = t; e < R * 128; e += kThreads) {
-      const int r = e / 128, dd = e % 128, i = r % p.Tq, h = hk * G + r / p.Tq;
-      float sum = 0.f;
-#pragma unroll
-      for (int q = 0; q < kSlices; ++q) sum += red[(q * R + r) * 128 + dd];
-      const float l = row_l[r];
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const size_t o_off = ((static_cast<size_t>(b) * p.Tq + i) * p.H + h) * 128 + dd;
-      if (ATTN_IN_RANGE(o_off, 1, static_cast<size_t>(p.B) * p.Tq * p.H * 128, kSiteChkDecO, &g_device_error))
-        p.o[o_off] = __float2bfloat16_rn(sum * inv);
-    }
-    if (t < R) {
-      const int i = t % p.Tq, h = hk * G + t / p.Tq;
-      const float l = row_l[t];
-      const size_t lse_i = (static_cast<size_t>(b) * p.H + h) * p.Tq + i;
-      if (ATTN_IN_RANGE(lse_i, 1, static_cast<size_t>(p.B) * p.H * p.Tq, kSiteChkDecLse, &g_device_error))
-        p.lse[lse_i] = l > 0.f ? (row_m[t] + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-    }
-    return;
-  }
-  const size_t n_part = static_cast<size_t>(p.B) * p.Hkv * p.n_split * R;  // partial rows
-  const size_t part = (static_cast<size_t>(bhk) * p.n_split + sp) * R;      // this chunk's first one
-  float* po = p.part_o + part * 128;
-  if (ATTN_IN_RANGE(part, R, n_part, kSiteChkDecPart, &g_device_error)) {
-    for (int e = t; e < R * 128; e += kThreads) {
-      const int r = e / 128, dd = e % 128;
-      float sum = 0.f;
-#pragma unroll
-      for (int q = 0; q < kSlices; ++q) sum += red[(q * R + r) * 128 + dd];
-      po[r * 128 + dd] = sum;
-    }
-    if (t < R) {
-      float* pml = p.part_ml + (part + t) * 2;
-      pml[0] = row_m[t];
-      pml[1] = row_l[t];
-    }
+    for (int g = consumed; g < issued; ++g)
+      mbar_wait(&full[g % kDecStages], (g / kDecStages) & 1, &no_abort, lim, &g_device_error, kSiteDecDrain);
   }
 }
 
