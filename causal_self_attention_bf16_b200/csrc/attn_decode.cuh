@@ -12,12 +12,14 @@
 //      the most blocks first (each CTA counting-sorts the lengths). A persistent grid, one CTA per SM, deals
 //      them out in rounds, back and forth; the G = H / H_kv query heads of a unit's group and their Tq new
 //      tokens (R = G * Tq rows) share every K and V row the CTA reads, so the cache is read once. The CTA's
-//      units stream through a three-stage shared-memory ring of 128-key K and V blocks loaded by TMA (one
-//      thread issues four 16 KB boxes per block onto the stage's mbarrier), two blocks in flight while one is
-//      used, on from one unit into the next; rows past a sequence's length are masked, never used. Per block:
-//      two or four threads score each key against all rows (a part of the dims each, shuffles to add), a warp
-//      per row updates the running max and sum (online softmax in base 2), and a thread per pair of output
-//      dimensions and slice of the block's keys accumulates O; the slices are added once per unit.
+//      units stream through a shared-memory ring of 128-key K and V blocks loaded by TMA (three stages, two
+//      for 32 rows; one thread issues four 16 KB boxes per block onto the stage's mbarrier), all but one block
+//      in flight while one is used, on from one unit into the next; rows past a sequence's length are masked,
+//      never used. Per block, in four independent groups of two warps that each take 32 of the block's keys
+//      (one CTA barrier per block, for the ring): two threads score each key against all rows (half the dims
+//      each, a shuffle to add), the group updates its own running max and its warps' running sums (online
+//      softmax in base 2), and a thread per pair of output dimensions accumulates O over the group's keys. The
+//      groups' results are merged once per unit by their maxima.
 //      The chunk's unnormalised O, running max and sum go to a workspace; when the cache is not split (one
 //      chunk per (sequence, head)) the kernel normalises and writes o and lse itself. The kernel is
 //      instantiated for 1, 2, 4, 8, 16 and 32 rows.
@@ -36,7 +38,6 @@ namespace attn {
 template <int kRows>
 __host__ __device__ constexpr int dec_threads() { return 256; }
 constexpr int kDecKeys = 128;       // keys per block
-constexpr int kDecStages = 3;       // K/V blocks in the shared-memory ring (two in flight while one is used)
 constexpr int kDecMaxRows = 32;     // R = (H / H_kv) * Tq query rows per CTA, at most
 constexpr int kDecChunkKeys = 256;  // keys per split of the cache, at least
 constexpr int kDecMaxUnits = 64;    // (sequence, key/value head, chunk) units one CTA walks, at most
@@ -59,6 +60,11 @@ struct DecodeParams {
   uint64_t timeout_ns;         // limit of any single wait
 };
 
+// K/V blocks in the shared-memory ring: three (two in flight while one is used), two for 32 rows, whose q rows
+// and scores (32 KB) leave no room for a third beside the groups' softmax state.
+template <int kRows>
+__host__ __device__ constexpr int dec_stages() { return kRows >= 32 ? 2 : 3; }
+
 // A unit of the split kernel's walk: chunk sp of sequence b for key/value head hk, and the chunk's keys
 // [key_lo, key_hi) of the sequence's L, in nblk 128-key blocks.
 struct DecUnit {
@@ -67,15 +73,16 @@ struct DecUnit {
 
 // Dynamic shared memory of the split kernel for up to kRows query rows (no static shared memory, so the block
 // starts 1024-byte aligned, as the 128-byte-swizzled TMA boxes need): the ring of (K block, V block) pairs, the
-// rows (fp32, pre-scaled), the block's scores, then P, the rows' running max, sum and rescale factor, one
-// mbarrier per ring stage, the abort flag (8 bytes) and the CTA's units (DecUnit each). 224 KB at kRows = 32.
+// rows (fp32, pre-scaled), the block's scores, then P, each warp's block max and running sum per row, each
+// group's running max per row (two slots), one mbarrier per ring stage, the abort flag (8 bytes) and the CTA's
+// units (DecUnit each): 195 KB for one row, 211 KB for 16, 165 KB for 32 (two ring stages).
 template <int kRows>
 __host__ __device__ constexpr size_t dec_bar_offset() {  // the stage barriers, 8-byte aligned
-  return (kDecStages * 2 * kDecBlockBytes + 2 * kRows * 128 * 4 + 3 * kRows * 4 + 7) / 8 * 8;
+  return (dec_stages<kRows>() * 2 * kDecBlockBytes + 2 * kRows * 128 * 4 + 24 * kRows * 4 + 7) / 8 * 8;
 }
 template <int kRows>
 __host__ __device__ constexpr size_t dec_smem_bytes() {
-  return dec_bar_offset<kRows>() + kDecStages * 8 + 8 + kDecMaxUnits * sizeof(DecUnit);
+  return dec_bar_offset<kRows>() + dec_stages<kRows>() * 8 + 8 + kDecMaxUnits * sizeof(DecUnit);
 }
 static_assert(dec_smem_bytes<kDecMaxRows>() <= 232448, "decode split kernel exceeds the 227 KB shared-memory opt-in");
 
@@ -176,6 +183,7 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   using namespace sm100;
   constexpr int kThreads = dec_threads<kRows>();
+  constexpr int kStages = dec_stages<kRows>();
   constexpr int kPart = kThreads / kDecKeys;   // scoring threads per key (2 or 4), kDims = 128 / kPart dims each
   constexpr int kDims = 128 / kPart;
   constexpr int kSlices = kThreads / 64;       // P V: key slices of kSliceKeys keys (4 x 32 or 8 x 16)
@@ -185,14 +193,14 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
     if (threadIdx.x == 0) atomicOr(&g_device_error, DEV_ERR_TIMEOUT | (kSiteDecFull << 8));
     return;
   }
-  float (*qs)[128] = reinterpret_cast<float (*)[128]>(dec_smem + kDecStages * 2 * kDecBlockBytes);
+  float (*qs)[128] = reinterpret_cast<float (*)[128]>(dec_smem + kStages * 2 * kDecBlockBytes);
   float (*sc)[kDecKeys] = reinterpret_cast<float (*)[kDecKeys]>(qs + kRows);  // scores, then P
-  float* row_m = reinterpret_cast<float*>(sc + kRows);
-  float* row_l = row_m + kRows;
-  float* row_a = row_l + kRows;
+  float* wmax = reinterpret_cast<float*>(sc + kRows);  // [8][kRows]: each warp's block max per row
+  float* gl = wmax + 8 * kRows;                        // [8][kRows]: each warp's running sum per row
+  float* gm = gl + 8 * kRows;                          // [2][4][kRows]: each group's running max, by block parity
   uint64_t* full = reinterpret_cast<uint64_t*>(dec_smem + dec_bar_offset<kRows>());
-  volatile int* abort = reinterpret_cast<volatile int*>(full + kDecStages);
-  DecUnit* units = reinterpret_cast<DecUnit*>(full + kDecStages + 1);  // this CTA's units, in walk order
+  volatile int* abort = reinterpret_cast<volatile int*>(full + kStages);
+  DecUnit* units = reinterpret_cast<DecUnit*>(full + kStages + 1);  // this CTA's units, in walk order
 
   const int t = threadIdx.x, warp = t / 32, lane = t % 32;
   const int G = p.H / p.Hkv, R = p.R;
@@ -217,7 +225,7 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
     }
   }
   if (t == 0) {
-    for (int st = 0; st < kDecStages; ++st) mbar_init(&full[st], 1);
+    for (int st = 0; st < kStages; ++st) mbar_init(&full[st], 1);
     *abort = 0;
     fence_barrier_init();
   }
@@ -225,7 +233,7 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
   __syncthreads();
 
   // The issue cursor (thread 0 only): block ib of unit ik's inb blocks, keys from ikey, sequence ibq, head ihk.
-  // Blocks go out in one stream over the CTA's units: the n-th into ring stage n % kDecStages.
+  // Blocks go out in one stream over the CTA's units: the n-th into ring stage n % kStages.
   const bool issuer = t == 0;
   int issued = 0, ik = 0, ib = 0, inb = -1, ikey = 0, ibq = 0, ihk = 0;
   auto issue_next = [&]() {
@@ -241,7 +249,7 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
     if (ik >= n_mine) return;
     // Four TMA boxes, 64 KB on the stage's barrier. The tensor maps bound the copies (rows past the cache come
     // as zeros); rows past a sequence's length are masked below.
-    const int kb = ikey + ib * kDecKeys, st = issued % kDecStages;
+    const int kb = ikey + ib * kDecKeys, st = issued % kStages;
     uint8_t* ks = dec_smem + st * 2 * kDecBlockBytes;
     mbar_arrive_expect_tx(&full[st], 2 * kDecBlockBytes);
     for (int c = 0; c < 2; ++c) {
@@ -255,7 +263,7 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
     tma_prefetch_desc(&tm_v);
   }
 #pragma unroll
-  for (int n = 0; n < kDecStages - 1; ++n) issue_next();
+  for (int n = 0; n < kStages - 1; ++n) issue_next();
 
   // Unit k's rows, R x 128 bf16 of q, in registers (elements t, t + kThreads, ...): read a unit ahead, so that
   // the loads' latency hides behind the previous unit's blocks. Row r = g * Tq + i is query head hk * G + g,
@@ -291,26 +299,27 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
       if (e < R * 128) qs[e / 128][e % 128] = __bfloat162float(qv[x]) * p.scale_log2;
     }
     if (k + 1 < n_mine) fetch_q(k + 1);
-    if (t < R) {
-      row_m[t] = -INFINITY;
-      row_l[t] = 0.f;
-    }
+    if (t < 8 * kRows) gl[t] = 0.f;
+    if (t < 4 * kRows) gm[t] = -INFINITY;  // parity 0, which the first block reads
     float acc[kRows][2];
 #pragma unroll
     for (int r = 0; r < kRows; ++r) acc[r][0] = acc[r][1] = 0.f;
 
     for (int n = 0; n < nblk; ++n) {
-      __syncthreads();  // the previous block's stage and the scores are no longer read: the stage takes the next
-      issue_next();     // block but one of the stream
-      const int g = consumed;
-      if (!mbar_wait_warp(&full[g % kDecStages], (g / kDecStages) & 1, abort, lim, &g_device_error, kSiteDecFull))
-        ok = false;
+      // The previous block's stage and P are no longer read (the stage takes the stream's block after next), and
+      // every warp's waits so far succeeded. A warp whose wait for this block runs out computes on regardless;
+      // the CTA leaves at the next block's barrier (or the unit's) without writing the unit.
       if (!__syncthreads_and(ok)) {
         ok = false;
         break;
       }
-      consumed = g + 1;
-      const uint8_t* ks = dec_smem + (g % kDecStages) * 2 * kDecBlockBytes;
+      issue_next();
+      const int g = consumed;
+      if (mbar_wait_warp(&full[g % kStages], (g / kStages) & 1, abort, lim, &g_device_error, kSiteDecFull))
+        consumed = g + 1;
+      else
+        ok = false;
+      const uint8_t* ks = dec_smem + (g % kStages) * 2 * kDecBlockBytes;
       const uint8_t* vs = ks + kDecBlockBytes;
       const int kb = key_lo + n * kDecKeys, nk = min(kDecKeys, key_hi - kb);
       {
@@ -343,49 +352,49 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
           float sj = s0 + s1;
 #pragma unroll
           for (int o = 1; o < kPart; o <<= 1) sj += __shfl_xor_sync(0xffffffffu, sj, o);
-          if (h == 0) {
-            const int last = L - p.Tq + r % p.Tq;  // last key this row sees (its own position)
-            const bool seen = j < nk && kb + j <= last && (p.window < 0 || kb + j >= last - p.window);
-            sc[r][j] = seen ? sj : -INFINITY;
+          const int last = L - p.Tq + r % p.Tq;  // last key this row sees (its own position)
+          const bool seen = j < nk && kb + j <= last && (p.window < 0 || kb + j >= last - p.window);
+          const float v = seen ? sj : -INFINITY;
+          if (h == 0) sc[r][j] = v;
+          float mx = v;  // the warp's block max (its 32 / kPart keys)
+#pragma unroll
+          for (int o = kPart; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          if (lane == 0) wmax[warp * kRows + r] = mx;
+        }
+      }
+      // The group's online softmax (its two warps; keys [32 kq, 32 kq + 32) of the block): the running max of
+      // each row takes the two warps' block maxima, P = exp2(s - max) replaces the scores in place, each warp
+      // adds its P to its own running sum, and O is rescaled. The running max alternates between two slots by
+      // block parity, so this block's reads never meet the write for the next.
+      named_barrier(1 + kq, 64);
+      {
+        const int j = t / kPart, h = t % kPart;
+        const float* gm_old = gm + ((n & 1) * 4 + kq) * kRows;
+        float* gm_new = gm + (((n + 1) & 1) * 4 + kq) * kRows;
+#pragma unroll
+        for (int r = 0; r < kRows; ++r) {
+          if (r < R) {
+            const float m_old = gm_old[r];
+            const float m_new = fmaxf(m_old, fmaxf(wmax[2 * kq * kRows + r], wmax[(2 * kq + 1) * kRows + r]));
+            const float a = m_old == m_new ? 1.f : exp2f(m_old - m_new);  // 0 when nothing was seen before
+            float pe = 0.f;
+            if (h == 0) {
+              pe = m_new == -INFINITY ? 0.f : exp2f(sc[r][j] - m_new);
+              sc[r][j] = pe;
+            }
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) pe += __shfl_xor_sync(0xffffffffu, pe, o);
+            if (lane == 0) gl[warp * kRows + r] = gl[warp * kRows + r] * a + pe;
+            if ((t & 63) == 0) gm_new[r] = m_new;
+            acc[r][0] *= a, acc[r][1] *= a;
           }
         }
       }
-      __syncthreads();
-      // Online softmax, a warp per row: block max, running max, exp2 in place, running sum, O's rescale factor.
-      for (int r = warp; r < R; r += kThreads / 32) {
-        float x[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = sc[r][lane * 4 + e];
-        float mb = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
-        const float m_old = row_m[r];
-        const float m_new = fmaxf(m_old, mb);
-        float sum = 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float pe = m_new == -INFINITY ? 0.f : exp2f(x[e] - m_new);
-          sc[r][lane * 4 + e] = pe;
-          sum += pe;
-        }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        __syncwarp();
-        if (lane == 0) {
-          const float a = m_old == m_new ? 1.f : exp2f(m_old - m_new);  // 0 when nothing was seen before
-          row_a[r] = a;
-          row_l[r] = row_l[r] * a + sum;
-          row_m[r] = m_new;
-        }
-      }
-      __syncthreads();
+      named_barrier(1 + kq, 64);  // the group's P is written
       // O[r][d] = O[r][d] * a_r + sum_j P[r][j] V[j][d] for this thread's two dims over its slice of the keys:
       // one 4-byte load per key for V (a warp reads one 128-byte box row), P four keys at a time. V rows past
       // the sequence's keys are taken as 0 (selected, not multiplied, so the cache's contents there do not
       // matter), and their P is 0.
-#pragma unroll
-      for (int r = 0; r < kRows; ++r)
-        if (r < R) acc[r][0] *= row_a[r], acc[r][1] *= row_a[r];
       const uint8_t* vbox = vs + (dp >> 5) * 16384;
 #pragma unroll 2
       for (int j0 = kSliceKeys * kq; j0 < kSliceKeys * (kq + 1); j0 += 4) {
@@ -413,14 +422,34 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
       }
     }
     if (!ok) break;
-    __syncthreads();  // P and the rows' state are final; the q rows and scores become the reduction's buffers
-    // The chunk's result (an empty chunk leaves max -inf, sum 0, O 0): the key slices' accumulators of each pair
-    // of dims are added in slice order by slice 0's threads, handed over through two buffers in turn (the q
-    // rows and the scores, R x 128 floats each).
+    __syncthreads();  // the groups' states are final; the q rows and scores become the reduction's buffers
+    // The unit's result (an empty chunk leaves max -inf, sum 0, O 0). Per row the largest group max M; group g's
+    // O and sums count with the factor 2^(m_g - M) (0 for a group that saw no key). The key slices' scaled O of
+    // each pair of dims are added in slice order by slice 0's threads, handed over through two buffers in turn
+    // (the q rows and the scores, R x 128 floats each); thread r < R puts row r's M and sum in wmax.
+    const float* gm_fin = gm + (nblk & 1) * 4 * kRows;  // the parity the unit's last block wrote
     float* xb[2] = {&qs[0][0], &sc[0][0]};
     float sum[kRows][2];
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) sum[r][0] = 0.f + acc[r][0], sum[r][1] = 0.f + acc[r][1];
+    for (int r = 0; r < kRows; ++r) {
+      if (r < R) {
+        const float m0 = gm_fin[r], m1 = gm_fin[kRows + r], m2 = gm_fin[2 * kRows + r], m3 = gm_fin[3 * kRows + r];
+        const float M = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+        const float mg = gm_fin[kq * kRows + r];
+        const float f = mg == -INFINITY ? 0.f : exp2f(mg - M);
+        acc[r][0] *= f, acc[r][1] *= f;
+        sum[r][0] = 0.f + acc[r][0], sum[r][1] = 0.f + acc[r][1];
+        if (t == r) {
+          const float fs[4] = {m0 == -INFINITY ? 0.f : exp2f(m0 - M), m1 == -INFINITY ? 0.f : exp2f(m1 - M),
+                               m2 == -INFINITY ? 0.f : exp2f(m2 - M), m3 == -INFINITY ? 0.f : exp2f(m3 - M)};
+          float l = 0.f;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) l += fs[q] * (gl[2 * q * kRows + r] + gl[(2 * q + 1) * kRows + r]);
+          wmax[r] = M;
+          wmax[kRows + r] = l;
+        }
+      }
+    }
 #pragma unroll
     for (int j = 1; j <= kSlices; ++j) {
       if (j < kSlices && kq == j) {
@@ -441,13 +470,13 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
     }
     if (p.n_split == 1) {
       // The only chunk of its (sequence, head): the result is final, so it is normalised and written here as the
-      // combine kernel would (that kernel is not launched): o = O / l, lse = m + log2(l) in natural-log units.
+      // combine kernel would (that kernel is not launched): o = O / l, lse = M + log2(l) in natural-log units.
       if (kq == 0) {
 #pragma unroll
         for (int r = 0; r < kRows; ++r) {
           if (r < R) {
             const int i = r % p.Tq, h = hk * G + r / p.Tq;
-            const float l = row_l[r];
+            const float l = wmax[kRows + r];
             const float inv = l > 0.f ? 1.f / l : 0.f;
             const size_t o_off = ((static_cast<size_t>(b) * p.Tq + i) * p.H + h) * 128 + 2 * dp;
             if (ATTN_IN_RANGE(o_off, 2, static_cast<size_t>(p.B) * p.Tq * p.H * 128, kSiteChkDecO, &g_device_error))
@@ -458,10 +487,10 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
       }
       if (t < R) {
         const int i = t % p.Tq, h = hk * G + t / p.Tq;
-        const float l = row_l[t];
+        const float l = wmax[kRows + t];
         const size_t lse_i = (static_cast<size_t>(b) * p.H + h) * p.Tq + i;
         if (ATTN_IN_RANGE(lse_i, 1, static_cast<size_t>(p.B) * p.H * p.Tq, kSiteChkDecLse, &g_device_error))
-          p.lse[lse_i] = l > 0.f ? (row_m[t] + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+          p.lse[lse_i] = l > 0.f ? (wmax[t] + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       }
     } else {
       const size_t n_part = static_cast<size_t>(p.B) * p.Hkv * p.n_split * R;  // partial rows
@@ -475,19 +504,19 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
         }
         if (t < R) {
           float* pml = p.part_ml + (part + t) * 2;
-          pml[0] = row_m[t];
-          pml[1] = row_l[t];
+          pml[0] = wmax[t];
+          pml[1] = wmax[kRows + t];
         }
       }
     }
-    __syncthreads();  // the q rows, scores and rows' state are free for the next unit
+    __syncthreads();  // the q rows, scores and the groups' states are free for the next unit
   }
   // Blocks issued but not consumed (only after a failure: at most the failed block and the two after it) land
   // before the CTA leaves.
   if (t == 0) {
     volatile int no_abort = 0;
     for (int g = consumed; g < issued; ++g)
-      mbar_wait(&full[g % kDecStages], (g / kDecStages) & 1, &no_abort, lim, &g_device_error, kSiteDecDrain);
+      mbar_wait(&full[g % kStages], (g / kStages) & 1, &no_abort, lim, &g_device_error, kSiteDecDrain);
   }
 }
 
