@@ -31,10 +31,11 @@
 
 namespace attn {
 
-// Threads of the split kernel. Scoring takes kThreads / 128 threads per key, each over 128 / that dims; P V takes
-// a thread per pair of output dimensions and kThreads / 64-th of the block's keys. 256 for every group size:
-// 512 (four threads per key, eight key slices) measured 34 % slower on decode_d20 -- a row's softmax is one
-// warp's work, and more warps only wait longer at the block's barriers.
+// Threads of the split kernel. Scoring takes kThreads / 128 threads per key, each over 128 / that dims; the
+// threads form kThreads / 64 groups of two warps, each taking kThreads / 64-th of a block's keys (scoring,
+// softmax and P V) with a thread per pair of output dimensions. 256 for every group size: 512 (four threads per
+// key, eight groups) measured 29-36 % slower on the decode workloads, the extra warps only lengthening each
+// block's chains of shared-memory loads and shuffles.
 template <int kRows>
 __host__ __device__ constexpr int dec_threads() { return 256; }
 constexpr int kDecKeys = 128;       // keys per block
@@ -78,7 +79,9 @@ struct DecUnit {
 // units (DecUnit each): 195 KB for one row, 211 KB for 16, 165 KB for 32 (two ring stages).
 template <int kRows>
 __host__ __device__ constexpr size_t dec_bar_offset() {  // the stage barriers, 8-byte aligned
-  return (dec_stages<kRows>() * 2 * kDecBlockBytes + 2 * kRows * 128 * 4 + 24 * kRows * 4 + 7) / 8 * 8;
+  constexpr int kWarps = dec_threads<kRows>() / 32, kGroups = kWarps / 2;
+  return (dec_stages<kRows>() * 2 * kDecBlockBytes + 2 * kRows * 128 * 4 + (2 * kWarps + 2 * kGroups) * kRows * 4 + 7) /
+         8 * 8;
 }
 template <int kRows>
 __host__ __device__ constexpr size_t dec_smem_bytes() {
@@ -184,6 +187,7 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
   using namespace sm100;
   constexpr int kThreads = dec_threads<kRows>();
   constexpr int kStages = dec_stages<kRows>();
+  constexpr int kWarps = kThreads / 32, kGroups = kWarps / 2;  // a group: two warps, one key slice
   constexpr int kPart = kThreads / kDecKeys;   // scoring threads per key (2 or 4), kDims = 128 / kPart dims each
   constexpr int kDims = 128 / kPart;
   constexpr int kSlices = kThreads / 64;       // P V: key slices of kSliceKeys keys (4 x 32 or 8 x 16)
@@ -195,9 +199,9 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
   }
   float (*qs)[128] = reinterpret_cast<float (*)[128]>(dec_smem + kStages * 2 * kDecBlockBytes);
   float (*sc)[kDecKeys] = reinterpret_cast<float (*)[kDecKeys]>(qs + kRows);  // scores, then P
-  float* wmax = reinterpret_cast<float*>(sc + kRows);  // [8][kRows]: each warp's block max per row
-  float* gl = wmax + 8 * kRows;                        // [8][kRows]: each warp's running sum per row
-  float* gm = gl + 8 * kRows;                          // [2][4][kRows]: each group's running max, by block parity
+  float* wmax = reinterpret_cast<float*>(sc + kRows);  // [kWarps][kRows]: each warp's block max per row
+  float* gl = wmax + kWarps * kRows;                   // [kWarps][kRows]: each warp's running sum per row
+  float* gm = gl + kWarps * kRows;                     // [2][kGroups][kRows]: each group's running max, by parity
   uint64_t* full = reinterpret_cast<uint64_t*>(dec_smem + dec_bar_offset<kRows>());
   volatile int* abort = reinterpret_cast<volatile int*>(full + kStages);
   DecUnit* units = reinterpret_cast<DecUnit*>(full + kStages + 1);  // this CTA's units, in walk order
@@ -299,8 +303,8 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
       if (e < R * 128) qs[e / 128][e % 128] = __bfloat162float(qv[x]) * p.scale_log2;
     }
     if (k + 1 < n_mine) fetch_q(k + 1);
-    if (t < 8 * kRows) gl[t] = 0.f;
-    if (t < 4 * kRows) gm[t] = -INFINITY;  // parity 0, which the first block reads
+    for (int i = t; i < kWarps * kRows; i += kThreads) gl[i] = 0.f;
+    for (int i = t; i < kGroups * kRows; i += kThreads) gm[i] = -INFINITY;  // parity 0, which the first block reads
     float acc[kRows][2];
 #pragma unroll
     for (int r = 0; r < kRows; ++r) acc[r][0] = acc[r][1] = 0.f;
@@ -369,8 +373,8 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
       named_barrier(1 + kq, 64);
       {
         const int j = t / kPart, h = t % kPart;
-        const float* gm_old = gm + ((n & 1) * 4 + kq) * kRows;
-        float* gm_new = gm + (((n + 1) & 1) * 4 + kq) * kRows;
+        const float* gm_old = gm + ((n & 1) * kGroups + kq) * kRows;
+        float* gm_new = gm + (((n + 1) & 1) * kGroups + kq) * kRows;
 #pragma unroll
         for (int r = 0; r < kRows; ++r) {
           if (r < R) {
@@ -427,24 +431,26 @@ __global__ void __launch_bounds__(dec_threads<kRows>()) attn_decode_split_kernel
     // O and sums count with the factor 2^(m_g - M) (0 for a group that saw no key). The key slices' scaled O of
     // each pair of dims are added in slice order by slice 0's threads, handed over through two buffers in turn
     // (the q rows and the scores, R x 128 floats each); thread r < R puts row r's M and sum in wmax.
-    const float* gm_fin = gm + (nblk & 1) * 4 * kRows;  // the parity the unit's last block wrote
+    const float* gm_fin = gm + (nblk & 1) * kGroups * kRows;  // the parity the unit's last block wrote
     float* xb[2] = {&qs[0][0], &sc[0][0]};
     float sum[kRows][2];
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
       if (r < R) {
-        const float m0 = gm_fin[r], m1 = gm_fin[kRows + r], m2 = gm_fin[2 * kRows + r], m3 = gm_fin[3 * kRows + r];
-        const float M = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+        float M = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < kGroups; ++q) M = fmaxf(M, gm_fin[q * kRows + r]);
         const float mg = gm_fin[kq * kRows + r];
         const float f = mg == -INFINITY ? 0.f : exp2f(mg - M);
         acc[r][0] *= f, acc[r][1] *= f;
         sum[r][0] = 0.f + acc[r][0], sum[r][1] = 0.f + acc[r][1];
         if (t == r) {
-          const float fs[4] = {m0 == -INFINITY ? 0.f : exp2f(m0 - M), m1 == -INFINITY ? 0.f : exp2f(m1 - M),
-                               m2 == -INFINITY ? 0.f : exp2f(m2 - M), m3 == -INFINITY ? 0.f : exp2f(m3 - M)};
           float l = 0.f;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) l += fs[q] * (gl[2 * q * kRows + r] + gl[(2 * q + 1) * kRows + r]);
+          for (int q = 0; q < kGroups; ++q) {
+            const float mq = gm_fin[q * kRows + r];
+            l += (mq == -INFINITY ? 0.f : exp2f(mq - M)) * (gl[2 * q * kRows + r] + gl[(2 * q + 1) * kRows + r]);
+          }
           wmax[r] = M;
           wmax[kRows + r] = l;
         }
