@@ -323,6 +323,41 @@ def test_decode_many_sequences_every_chunk_once(window):
     check_lse(lse64[rest, 0, 0], np.log(seen), "decode B=600 zero caches")
 
 
+def test_decode_one_cta_per_unit_beyond_the_walk_limit():
+    """1000 sequences of 10 heads against a 128-key cache: 10,000 (sequence, head) units, more than a persistent
+    CTA per SM lists (64 each), so the grid takes one CTA per unit. Three seeded sequences go to the oracle;
+    every other cache is zero (o = 0 exactly, LSE = ln(keys seen)); o and lse start as NaN."""
+    B, H, Tk, D = 1000, 10, 128, 128
+    g = torch.Generator(device="cpu")
+    g.manual_seed(10000)
+    lens = torch.randint(1, Tk + 1, (B,), generator=g, dtype=torch.int64).to(torch.int32)
+    q = torch.randn((B, 1, H, D), generator=g).to(torch.bfloat16)
+    picks = [0, 517, B - 1]
+    dev = torch.device("cuda")
+    kc = torch.zeros((B, Tk, H, D), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    cpu_k, cpu_v = {}, {}
+    for b in picks:
+        cpu_k[b] = torch.randn((1, Tk, H, D), generator=g).to(torch.bfloat16)
+        cpu_v[b] = torch.randn((1, Tk, H, D), generator=g).to(torch.bfloat16)
+        kc[b].copy_(cpu_k[b][0])
+        vc[b].copy_(cpu_v[b][0])
+    o = torch.full((B, 1, H, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    lse = torch.full((B, H, 1), float("nan"), dtype=torch.float32, device=dev)
+    scale = D ** -0.5
+    attn.attn_decode(q.to(dev), kc, vc, lens.to(dev), scale, o=o, lse=lse)
+    torch.cuda.synchronize()
+    o64, lse64 = to64(o), to64(lse)
+    for b in picks:
+        O_ref, LSE_ref = attn_ref.decode_forward(q[b:b + 1], cpu_k[b], cpu_v[b], lens[b:b + 1].numpy(), scale)
+        check_o(o64[b:b + 1], O_ref, f"decode B=1000 b={b}")
+        check_lse(lse64[b:b + 1], LSE_ref, f"decode B=1000 b={b}")
+    rest = np.array([b for b in range(B) if b not in picks])
+    assert np.all(o64[rest] == 0), "a zero cache must give o = 0 exactly (NaN: a unit was never computed)"
+    seen = np.broadcast_to(lens.numpy()[rest].astype(np.float64)[:, None, None], lse64[rest].shape)
+    check_lse(lse64[rest], np.log(seen), "decode B=1000 zero caches")
+
+
 @pytest.mark.parametrize("name", ["decode_d20", "decode_d20_gqa", "decode_d20_sw"])
 def test_decode_full_size_sampled(name):
     """The benchmark's decode workloads (64 sequences, d20 heads, ragged lengths up to 2048), oracle on samples.
