@@ -547,11 +547,11 @@ attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const 
 
 namespace {
 
-// Splits of the cache per (sequence, key/value head): about 4 CTAs per SM of a 148-SM part in all (one is resident
-// per SM at a time, with its 224 KB ring; a few waves even out the sequences' different lengths, and each CTA's
-// ramp-up, its first blocks' loads, is paid fewer times than with 8 or 16: on the decode workloads 4 per SM ran
-// 1-6 % faster than 8 and 10-25 % faster than 16, and 2 or 1 lost 10 % with grouped heads), each split at least
-// kDecChunkKeys keys (a multiple of the 128-key block).
+// Splits of the cache per (sequence, key/value head): about 4 units per SM of a 148-SM part in all, each split at
+// least kDecChunkKeys keys (a multiple of the 128-key block). The persistent split kernel deals the units out
+// longest first; a few units per SM let the short ones even out the SMs' totals, while more would add merge work
+// (with one CTA per unit, 4 per SM ran 1-6 % faster than 8 and 10-25 % faster than 16, and 2 or 1 lost 10 % with
+// grouped heads).
 void decode_split(int B, int Hkv, int Tk, int* n_split, int* chunk) {
   const long long pairs = static_cast<long long>(B) * Hkv;
   long long want = (4 * 148 + pairs - 1) / pairs;
